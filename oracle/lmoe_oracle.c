@@ -1,0 +1,309 @@
+/*
+ * lmoe_oracle.c -- plain fp64 CPU oracle of the LatentMoE layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is what the CUDA library is checked
+ * against; it is never part of the product path.  Only tests/, the smoke
+ * check in __graft_entry__.py and the CPU-baseline leg of bench.py may load
+ * it.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [Explained]  "LatentMoE: NVIDIA's Latent Mixture of Experts Explained
+ *                Through Equations, Architecture, Code and..." (Towards AI):
+ *                Figure 3 (router), Figure 8 (the latent layer with shapes),
+ *                Figure 9 (the latent expert), the MoE and LatentMoE code
+ *                modules, and the paragraph after Figure 1 (SwiGLU has a
+ *                third matrix beside W1).
+ *   [README]     "Latent-MoE" GitHub README, sections Usage and the two
+ *                variants (eff / acc).
+ *   [Shaping]    "Shaping Latent Mixture-of-Experts" summary page, Table 9
+ *                (expert matrices W_g, W_u, W_o).
+ *
+ * What it computes, per token x (width d), in the order the LatentMoE code
+ * module of [Explained] takes the steps:
+ *   1. s_e = sum_i x_i W_r[e][i] (+ b_e)                  router on x, not z
+ *   2. p   = softmax(s) over all N' experts
+ *   3. the K' experts with the largest s, ordered by (s desc, e asc)
+ *   4. g_k = p_{id_k} / sum_k' p_{id_k'}                   gates sum to 1
+ *   5. z   = W_down x                                      d -> l, no bias
+ *   6. u   = sum_{k=0..K'-1} g_k E_{id_k}(z),  E(v) = W_o (silu(W_g v) * (W_u v))
+ *   7. y   = W_up u + sum_{j=0..n_s-1} S_j(x)              S_j: SwiGLU at width d
+ * Readings where the pages are silent (each listed in the design doc):
+ *   - experts are SwiGLU with three matrices (the pages' code shows squared
+ *     ReLU with two; the article says SwiGLU carries over with a third
+ *     matrix, and [Shaping] Table 9 names W_g, W_u, W_o); silu(a)=a/(1+e^-a);
+ *   - top-K' ties go to the lower expert index; selection is made on s
+ *     (the same set as on p, and immune to exp rounding in fp64);
+ *   - the optional router bias is added to the logits before the softmax;
+ *   - slot order k = 0..K'-1 is the summation order of the combine, then
+ *     W_up, then the shared experts in index order.
+ * Arithmetic is fp64 throughout; inputs are widened exactly from f32 or
+ * bf16 (a bf16 value is the top 16 bits of an IEEE f32).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ODT_F32 = 0, ODT_BF16 = 1, ODT_F64 = 2 };
+
+typedef struct {
+  int32_t d, l, m, n_routed, k_active, n_shared, m_shared;
+  int32_t dtype;             /* element type of x and every weight below */
+  const void *w_router;      /* [N'][d] */
+  const double *b_router;    /* [N'] or NULL */
+  const void *w_down;        /* [l][d] */
+  const void *w_up;          /* [d][l] */
+  const void *w_gate;        /* [N'][m][l] */
+  const void *w_upx;         /* [N'][m][l] */
+  const void *w_out;         /* [N'][l][m] */
+  const void *s_gate;        /* [n_s][m_s][d] */
+  const void *s_up;          /* [n_s][m_s][d] */
+  const void *s_out;         /* [n_s][d][m_s] */
+} oracle_layer;
+
+/* Exact widening of one stored element to double. */
+static double elem(const void *base, int dt, size_t i) {
+  if (dt == ODT_F32) return (double)((const float *)base)[i];
+  if (dt == ODT_BF16) {
+    uint32_t u = (uint32_t)((const uint16_t *)base)[i] << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+  }
+  return ((const double *)base)[i];
+}
+
+/* out[r] = sum_c W[off + r*cols + c] * v[c], for r < rows. */
+static void matvec(const void *W, int dt, size_t off, int rows, int cols,
+                   const double *v, double *out) {
+  for (int r = 0; r < rows; ++r) {
+    double acc = 0.0;
+    size_t base = off + (size_t)r * (size_t)cols;
+    for (int c = 0; c < cols; ++c) acc += elem(W, dt, base + (size_t)c) * v[c];
+    out[r] = acc;
+  }
+}
+
+static double silu(double a) { return a / (1.0 + exp(-a)); }
+
+/* One SwiGLU feed-forward: out = W_o (silu(W_g v) * (W_u v)).
+ * W_g, W_u: [hid][in_w] at element offset off_in; W_o: [out_w][hid] at off_out.
+ * [Explained], paragraph after Figure 1 (gated activation with a third matrix)
+ * and Figure 9 (the hidden width is m on both sides). */
+static void swiglu_ffn(const oracle_layer *L, const void *Wg, const void *Wu,
+                       const void *Wo, size_t off_in, size_t off_out, int in_w,
+                       int hid, int out_w, const double *v, double *out,
+                       double *scratch /* 2*hid */) {
+  double *a = scratch, *b = scratch + hid;
+  matvec(Wg, L->dtype, off_in, hid, in_w, v, a);
+  matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
+  for (int j = 0; j < hid; ++j) a[j] = silu(a[j]) * b[j];
+  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);
+}
+
+/* ---- step 1: router logits, [Explained] Figure 3 and "routes in FULL d" */
+static void router_row(const oracle_layer *L, const void *x, int xdt,
+                       int64_t t, double *s) {
+  const int d = L->d, N = L->n_routed;
+  for (int e = 0; e < N; ++e) {
+    double acc = 0.0;
+    for (int i = 0; i < d; ++i)
+      acc += elem(x, xdt, (size_t)t * d + i) *
+             elem(L->w_router, L->dtype, (size_t)e * d + i);
+    s[e] = acc + (L->b_router ? L->b_router[e] : 0.0);
+  }
+}
+
+void oracle_router_logits(const oracle_layer *L, const void *x, int64_t T,
+                          double *s /* [T][N'] */) {
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t t = 0; t < T; ++t) router_row(L, x, L->dtype, t, s + t * L->n_routed);
+}
+
+/* ---- steps 2-4 for one token: softmax, top-K', renormalised gates.
+ * [Explained] LatentMoE code: topk(softmax(scores)), then w / w.sum(). */
+static void select_row(const double *s, int N, int K, int32_t *ids,
+                       double *gates, unsigned char *taken) {
+  double smax = s[0];
+  for (int e = 1; e < N; ++e) if (s[e] > smax) smax = s[e];
+  double denom = 0.0;
+  for (int e = 0; e < N; ++e) denom += exp(s[e] - smax);
+  memset(taken, 0, (size_t)N);
+  for (int k = 0; k < K; ++k) {
+    int best = -1;
+    for (int e = 0; e < N; ++e) {
+      if (taken[e]) continue;
+      if (best < 0 || s[e] > s[best]) best = e; /* strict: ties keep lower e */
+    }
+    taken[best] = 1;
+    ids[k] = best;
+  }
+  double psum = 0.0;
+  for (int k = 0; k < K; ++k) {
+    gates[k] = exp(s[ids[k]] - smax) / denom; /* p_{id_k} */
+    psum += gates[k];
+  }
+  for (int k = 0; k < K; ++k) gates[k] /= psum;
+}
+
+int oracle_select(const double *s, int64_t T, int N, int K, int32_t *ids,
+                  double *gates) {
+  if (K < 1 || K > N) return -1;
+#pragma omp parallel
+  {
+    unsigned char *taken = (unsigned char *)malloc((size_t)N);
+#pragma omp for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+      select_row(s + t * N, N, K, ids + t * K, gates + t * K, taken);
+    free(taken);
+  }
+  return 0;
+}
+
+/* Gates for caller-given ids: p_{id_k} / sum p over the given set. */
+static void gates_for_ids(const double *s, int N, int K, const int32_t *ids,
+                          double *gates) {
+  double smax = s[0];
+  for (int e = 1; e < N; ++e) if (s[e] > smax) smax = s[e];
+  double denom = 0.0;
+  for (int e = 0; e < N; ++e) denom += exp(s[e] - smax);
+  double psum = 0.0;
+  for (int k = 0; k < K; ++k) {
+    gates[k] = exp(s[ids[k]] - smax) / denom;
+    psum += gates[k];
+  }
+  for (int k = 0; k < K; ++k) gates[k] /= psum;
+}
+
+/* ---- components, exposed so tests can recompose the layer another way */
+
+/* z = W_down x_t   ([Explained] Figure 6 upper half, "the only d-wide op") */
+void oracle_down(const oracle_layer *L, const void *x, int64_t t, double *z) {
+  double *xv = (double *)malloc(sizeof(double) * (size_t)L->d);
+  for (int i = 0; i < L->d; ++i) xv[i] = elem(x, L->dtype, (size_t)t * L->d + i);
+  matvec(L->w_down, L->dtype, 0, L->l, L->d, xv, z);
+  free(xv);
+}
+
+/* out = E_e(z), one routed latent expert l -> m -> l ([Explained] Figure 9) */
+void oracle_expert(const oracle_layer *L, int e, const double *z, double *out) {
+  double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)L->m);
+  swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * L->m * L->l,
+             (size_t)e * L->l * L->m, L->l, L->m, L->l, z, out, scratch);
+  free(scratch);
+}
+
+/* out = W_up u   ([Explained] Figure 6 lower half) */
+void oracle_up(const oracle_layer *L, const double *u, double *out) {
+  matvec(L->w_up, L->dtype, 0, L->d, L->l, u, out);
+}
+
+/* out = sum_j S_j(x_t), the shared experts at width d, in index order */
+void oracle_shared(const oracle_layer *L, const void *x, int64_t t, double *out) {
+  const int d = L->d, ms = L->m_shared;
+  double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+  double *tmp = (double *)malloc(sizeof(double) * (size_t)d);
+  double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)(ms > 0 ? ms : 1));
+  for (int i = 0; i < d; ++i) { xv[i] = elem(x, L->dtype, (size_t)t * d + i); out[i] = 0.0; }
+  for (int j = 0; j < L->n_shared; ++j) {
+    swiglu_ffn(L, L->s_gate, L->s_up, L->s_out, (size_t)j * ms * d,
+               (size_t)j * d * ms, d, ms, d, xv, tmp, scratch);
+    for (int i = 0; i < d; ++i) out[i] += tmp[i];
+  }
+  free(xv); free(tmp); free(scratch);
+}
+
+/* ---- the whole layer for a list of tokens.
+ * ids_in == NULL: route each token (steps 1-4).  Otherwise use ids_in[t][k]
+ * as the selection (gates renormalised over that set) -- used when a token's
+ * K'-th and (K'+1)-th logits are too close for the selection to be unique.
+ * y[n][d] for n < n_tok is the output of token tokens[n]. */
+int oracle_forward(const oracle_layer *L, const void *x, int64_t T,
+                   const int64_t *tokens, int64_t n_tok, const int32_t *ids_in,
+                   double *y, int32_t *ids_out, double *gates_out) {
+  const int d = L->d, l = L->l, m = L->m, N = L->n_routed, K = L->k_active;
+  if (K < 1 || K > N || l < 1 || d < 1 || m < 1) return -1;
+  int err = 0;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+    double *z = (double *)malloc(sizeof(double) * (size_t)l);
+    double *u = (double *)malloc(sizeof(double) * (size_t)l);
+    double *eo = (double *)malloc(sizeof(double) * (size_t)l);
+    double *sh = (double *)malloc(sizeof(double) * (size_t)d);
+    int32_t *ids = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
+    double *g = (double *)malloc(sizeof(double) * (size_t)K);
+    unsigned char *taken = (unsigned char *)malloc((size_t)N);
+    int ms = L->m_shared > 0 ? L->m_shared : 1;
+    double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)(m > ms ? m : ms));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t n = 0; n < n_tok; ++n) {
+      const int64_t t = tokens ? tokens[n] : n;
+      if (t < 0 || t >= T) { err = -2; continue; }
+      router_row(L, x, L->dtype, t, s);
+      if (ids_in) {
+        memcpy(ids, ids_in + t * K, sizeof(int32_t) * (size_t)K);
+        gates_for_ids(s, N, K, ids, g);
+      } else {
+        select_row(s, N, K, ids, g, taken);
+      }
+      for (int i = 0; i < d; ++i) xv[i] = elem(x, L->dtype, (size_t)t * d + i);
+      matvec(L->w_down, L->dtype, 0, l, d, xv, z);
+      for (int i = 0; i < l; ++i) u[i] = 0.0;
+      for (int k = 0; k < K; ++k) { /* slot loop, in slot order */
+        const int e = ids[k];
+        swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * m * l,
+                   (size_t)e * l * m, l, m, l, z, eo, scratch);
+        for (int i = 0; i < l; ++i) u[i] += g[k] * eo[i];
+      }
+      double *yr = y + n * d;
+      matvec(L->w_up, L->dtype, 0, d, l, u, yr);
+      for (int j = 0; j < L->n_shared; ++j) {
+        swiglu_ffn(L, L->s_gate, L->s_up, L->s_out, (size_t)j * L->m_shared * d,
+                   (size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch);
+        for (int i = 0; i < d; ++i) yr[i] += sh[i];
+      }
+      if (ids_out) memcpy(ids_out + n * K, ids, sizeof(int32_t) * (size_t)K);
+      if (gates_out) memcpy(gates_out + n * K, g, sizeof(double) * (size_t)K);
+    }
+    free(s); free(xv); free(z); free(u); free(eo); free(sh); free(ids); free(g);
+    free(taken); free(scratch);
+  }
+  return err;
+}
+
+/* ---- dispatch: group the (token, slot) pairs by expert.
+ * [Explained] code: "for e in e_ids.unique(): sel = e_ids == e" visits, per
+ * expert, the tokens that chose it in token order.  Written out plainly:
+ * offsets[e] = number of pairs with expert < e (exclusive prefix count);
+ * perm lists, expert by expert, the flat pair index t*K+k with t ascending;
+ * pos is the inverse of perm. */
+int oracle_dispatch(const int32_t *ids, int64_t T, int K, int N,
+                    int32_t *offsets, int32_t *perm, int32_t *pos) {
+  int64_t cursor = 0;
+  for (int e = 0; e < N; ++e) {
+    offsets[e] = (int32_t)cursor;
+    for (int64_t t = 0; t < T; ++t)
+      for (int k = 0; k < K; ++k)
+        if (ids[t * K + k] == e) {
+          perm[cursor] = (int32_t)(t * K + k);
+          pos[t * K + k] = (int32_t)cursor;
+          ++cursor;
+        }
+  }
+  offsets[N] = (int32_t)cursor;
+  return cursor == T * (int64_t)K ? 0 : -1; /* -1: an id outside [0, N) */
+}
+
+int oracle_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -1,0 +1,167 @@
+/*
+ * lmoe.h -- C ABI of the B200 (sm_100a) LatentMoE layer forward.
+ *
+ * The layer (sources: "LatentMoE: NVIDIA's Latent Mixture of Experts
+ * Explained Through Equations, Architecture, Code and..." -- Figures 3, 6, 8
+ * and 9 and the LatentMoE code module; the Latent-MoE GitHub README --
+ * "Usage" and the eff / acc variants):
+ *
+ *   s   = x W_r^T (+ b_r)                 router on the full-width token x
+ *   ids = top-K'(s), ties -> lower index   slot order = logit descending
+ *   g   = softmax(s) at ids, renormalised to sum to 1 over the K' slots
+ *   z   = x W_down^T                       d -> l = d / alpha, no bias
+ *   u   = sum_k g_k E_{ids_k}(z),          E(v) = W_o (silu(W_g v) * (W_u v))
+ *   y   = u W_up^T + sum_j S_j(x),         S_j: shared SwiGLU experts at width d
+ *
+ * Sizes: N' = alpha * n_experts, K' = alpha * top_k ("acc") or top_k ("eff"),
+ * unless overridden.  y excludes the residual connection.
+ *
+ * Conventions for every call below:
+ *   - Return value: LMOE_OK (0) or a negative LMOE_ERR_* code; no exceptions
+ *     cross this boundary.  lmoe_strerror() names a code.
+ *   - Pointers named *_dev / device pointers are CUDA device memory on the
+ *     handle's device; *_host pointers are host memory (pinned or pageable).
+ *     The caller owns every buffer it passes; the handle owns its weight
+ *     copies and workspace (sized once at lmoe_create from max_tokens;
+ *     lmoe_forward allocates nothing).
+ *   - Matrices are row-major in nn.Linear [out][in] layout.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on it unless stated; one stream at a
+ *     time per handle (the workspace is shared by all calls of a handle).
+ *   - Errors found on the host are returned before anything is enqueued.
+ *     Errors found on the device (a bounded wait that ran out) are recorded
+ *     in a sticky status word that lmoe_device_status() reads.
+ */
+#ifndef LMOE_H
+#define LMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Variants of the Latent-MoE README: "eff" keeps K' = K, "acc" scales K' = alpha K. */
+typedef enum { LMOE_EFF = 0, LMOE_ACC = 1 } lmoe_variant;
+
+/* Element type of x, y and every weight.  LMOE_F32 runs fp32 CUDA-core
+ * kernels end to end; LMOE_BF16 runs bf16 tensor-core (tcgen05) GEMMs with
+ * fp32 accumulation and bf16 intermediates (z, expert hidden, expert out,
+ * combined u, shared hidden). */
+typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
+
+enum {
+  LMOE_OK = 0,
+  LMOE_ERR_INVALID_CONFIG = -1,  /* d % alpha != 0, K' outside [1, N'], sizes <= 0 */
+  LMOE_ERR_NULL_ARG = -2,        /* a required pointer is NULL */
+  LMOE_ERR_NOT_LOADED = -3,      /* route/forward before lmoe_load_weights */
+  LMOE_ERR_TOO_MANY_TOKENS = -4, /* T > max_tokens or T < 0 */
+  LMOE_ERR_CUDA = -5,            /* a CUDA runtime / driver call failed */
+  LMOE_ERR_DEVICE_TIMEOUT = -6,  /* a kernel's bounded wait ran out (status word) */
+  LMOE_ERR_UNSUPPORTED = -7,     /* valid layer, but a shape this build does not tile */
+  LMOE_ERR_OUT_OF_MEMORY = -8    /* workspace or weight allocation failed */
+};
+
+/* Layer hyper-parameters.  Field names follow LatentMoEConfig of the
+ * Latent-MoE README ("Usage"): d, m, n_experts (N), top_k (K), alpha,
+ * n_shared, variant.  Additions: m_shared (shared-expert width), dtype,
+ * n_routed_override / top_k_override (0 = derive N' and K' from the variant),
+ * has_router_bias, max_tokens (workspace size; forward never allocates).
+ * LMOE_BF16 additionally needs d, l, m_shared*n_shared to be multiples of 64,
+ * m and m_shared multiples of 128, and N' <= 512 (else LMOE_ERR_UNSUPPORTED). */
+typedef struct {
+  int32_t d, m, n_experts, top_k, alpha, n_shared, m_shared;
+  int32_t variant;           /* lmoe_variant */
+  int32_t dtype;             /* lmoe_dtype */
+  int32_t n_routed_override; /* N' if > 0 */
+  int32_t top_k_override;    /* K' if > 0 */
+  int32_t has_router_bias;   /* 1: a float32 bias [N'] is added to the logits */
+  int32_t max_tokens;        /* largest T any later call may pass */
+} lmoe_config;
+
+typedef struct lmoe_layer *lmoe_handle;
+
+/* Device pointers to the caller's weights, element type = cfg.dtype (the
+ * router bias is always float32), nn.Linear [out][in] row-major:
+ *   w_router [N'][d], b_router [N'] or NULL, w_down [l][d], w_up [d][l],
+ *   w_gate [N'][m][l], w_upx [N'][m][l], w_out [N'][l][m],
+ *   s_gate [n_s][m_s][d], s_up [n_s][m_s][d], s_out [n_s][d][m_s]
+ * (s_* may be NULL when n_shared == 0). */
+typedef struct {
+  const void *w_router;
+  const float *b_router;
+  const void *w_down, *w_up;
+  const void *w_gate, *w_upx, *w_out;
+  const void *s_gate, *s_up, *s_out;
+} lmoe_weights;
+
+/* Validates *cfg, derives l, N', K', allocates the handle's workspace for
+ * cfg->max_tokens tokens on the current CUDA device, and returns the handle
+ * in *out.  Synchronous.  Errors: NULL_ARG, INVALID_CONFIG, UNSUPPORTED,
+ * OUT_OF_MEMORY, CUDA. */
+int lmoe_create(const lmoe_config *cfg, lmoe_handle *out);
+
+/* Copies the weights into handle-owned device memory, repacked for the
+ * kernels (bf16: router, W_down and the shared gate/up rows stacked into one
+ * matrix over x; expert gate/up rows interleaved in blocks of 128; W_up and
+ * the shared down-projections concatenated along their input dimension).
+ * The caller's buffers may be freed once `stream` has passed this call.
+ * Errors: NULL_ARG, CUDA. */
+int lmoe_load_weights(lmoe_handle h, const lmoe_weights *w, void *stream);
+
+/* Routing only (router GEMM, softmax / top-K' / renormalise, dispatch).
+ * x_dev [T][d]; outputs (device, any may be NULL):
+ *   ids [T][K'] int32, slot order = logit descending, ties -> lower index;
+ *   gates [T][K'] float32, summing to 1 per token;
+ *   offsets [N'+1] int32, offsets[e] = number of (token, slot) pairs routed
+ *     to experts < e (exclusive scan of the per-expert histogram);
+ *   perm [T*K'] int32: perm[offsets[e] + r] = t*K' + k for the r-th token
+ *     (ascending t) that chose expert e, in slot k.
+ * T == 0 is allowed (offsets all 0).  Errors: NULL_ARG, NOT_LOADED,
+ * TOO_MANY_TOKENS, CUDA. */
+int lmoe_route(lmoe_handle h, const void *x_dev, int32_t T, int32_t *ids,
+               float *gates, int32_t *offsets, int32_t *perm, void *stream);
+
+/* The layer forward: y_dev [T][d] = layer(x_dev [T][d]), element type
+ * cfg.dtype.  x and y must not overlap.  Graph-capturable: no host sync, no
+ * allocation.  T == 0 is a no-op.  Errors: NULL_ARG, NOT_LOADED,
+ * TOO_MANY_TOKENS, CUDA. */
+int lmoe_forward(lmoe_handle h, const void *x_dev, void *y_dev, int32_t T, void *stream);
+
+/* End-to-end variant with HOST buffers: copies x_host to a handle-owned
+ * device staging buffer, runs lmoe_forward, copies y back to y_host, and
+ * synchronises `stream` before returning.  Pinned host memory gives full
+ * copy bandwidth.  Errors: as lmoe_forward. */
+int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T,
+                      void *stream);
+
+/* Derived sizes: l = d / alpha, N', K'.  Any output pointer may be NULL. */
+int lmoe_get_dims(lmoe_handle h, int32_t *l, int32_t *n_routed, int32_t *k_active);
+
+/* Synchronises `stream`, then returns and clears the handle's sticky
+ * device-side status (LMOE_OK or LMOE_ERR_DEVICE_TIMEOUT), or LMOE_ERR_CUDA
+ * if the stream reports an error. */
+int lmoe_device_status(lmoe_handle h, void *stream);
+
+/* Test and profiling hook: the device address and element count of one of
+ * the handle's intermediate buffers after the last call on the stream
+ * (which: 0 logits f32 [T][N'], 1 z [T][l], 2 permuted z [T*K'][l],
+ * 3 expert hidden [T*K'][m], 4 expert out [T*K'][l], 5 [u | shared hidden]
+ * [T][l + n_s m_s], 6 ids, 7 gates, 8 offsets, 9 perm, 10 pos [T*K'] (inverse
+ * of perm), 11 number of 128-row expert tiles).  Errors: NULL_ARG,
+ * INVALID_CONFIG (unknown `which`). */
+int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel);
+
+/* Human-readable name of a status code (static string). */
+const char *lmoe_strerror(int code);
+
+/* Frees the handle and everything it owns (synchronises the device first).
+ * NULL is a no-op. */
+int lmoe_destroy(lmoe_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMOE_H */

@@ -1,0 +1,89 @@
+// kernels.h -- host-side launchers of the LatentMoE kernels (internal).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lmoe {
+
+// Rows of one grouped-GEMM M-tile: expert `expert`, permuted rows
+// [row0, min(row0 + tile_m, row_end)).
+struct TileEntry {
+  int32_t row0, row_end, expert, pad;
+};
+
+// ---- routing (route_kernels.cu)
+// ids/gates from fp32 logits [T][ld] (+ bias [N]); one warp per token.
+cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, int N, int K,
+                        int32_t *ids, float *gates, cudaStream_t s);
+
+// Tokens per dispatch chunk and the per-chunk count matrix size.
+constexpr int kDispatchChunk = 256;
+inline int dispatch_chunks(int T) { return (T + kDispatchChunk - 1) / kDispatchChunk; }
+
+// Histogram -> exclusive scan -> stable scatter.  Writes offsets [N+1],
+// perm / pos / row_expert [T*K], and the M-tile table (tile_m rows per tile;
+// capacity max_tiles entries) plus its length in *n_tiles.
+cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,
+                            int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *row_expert,
+                            TileEntry *tiles, int32_t *n_tiles, int tile_m, int max_tiles,
+                            cudaStream_t s);
+
+// dst[p][:] = src[perm[p] / K][:], rows of `row_bytes` (multiple of 16).
+cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
+                                int row_bytes, void *dst, cudaStream_t s);
+
+// u[t][0:l] (row stride ldu) = sum_k gates[t][k] * O[pos[t*K+k]][0:l] in slot
+// order, fp32 accumulation; element type bf16 (is_bf16) or f32.
+cudaError_t launch_combine(const void *O, const int32_t *pos, const float *gates, int T, int K,
+                           int l, void *u, int ldu, bool is_bf16, cudaStream_t s);
+
+// ---- fp32 CUDA-core path (simt_kernels.cu)
+cudaError_t simt_linear(const float *A, int lda, const float *B, int ldb, float *C, int ldc,
+                        int M, int N, int Kdim, cudaStream_t s);
+// H[r][c] = silu(A_r . Wg[e][c%mw]) * (A_r . Wu[e][c%mw]) for c < Ncols, where
+// e = row_expert[r] if row_expert else c / mw; Wg/Wu are [*][mw][Kdim].
+cudaError_t simt_swiglu(const float *A, int lda, const float *Wg, const float *Wu, int mw,
+                        const int32_t *row_expert, float *H, int ldh, int M, int Ncols, int Kdim,
+                        cudaStream_t s);
+// O[r][c] = H_r . Wo[row_expert[r]][c]   (Wo [*][Ncols][Kdim])
+cudaError_t simt_expert_down(const float *H, int ldh, const float *Wo,
+                             const int32_t *row_expert, float *O, int ldo, int M, int Ncols,
+                             int Kdim, cudaStream_t s);
+
+// ---- bf16 tcgen05 GEMMs (tc_gemm.cu)
+enum TcMode : int {
+  TC_X_FUSED = 0,   // x [T][d] x W_x: router logits | z | shared SwiGLU hidden
+  TC_EXPERT_GU = 1, // grouped: permuted z x W_gu[e] -> SwiGLU -> H
+  TC_EXPERT_DOWN = 2,  // grouped: H x W_o[e] -> O (bf16)
+  TC_OUT = 3,       // [u | shared hidden] x W_y -> y (bf16)
+};
+
+struct TcParams {
+  int mode;
+  int M;               // dense: rows (T); grouped: unused (tile table)
+  int Kdim;            // reduction length, multiple of 64
+  int n_tiles_n;       // N-tiles of 256 columns
+  const TileEntry *tiles;   // grouped modes
+  const int32_t *n_mtiles;  // grouped modes: device count of M-tiles
+  int b_rows_per_expert;    // grouped modes: B rows per expert (2m or l)
+  // TC_X_FUSED column regions (multiples of 256): [0, r_end) router logits,
+  // [r_end, z_end) z, [z_end, ...) shared gate/up interleaved in blocks of 128.
+  int r_end, z_end, n_routed, l;
+  float *logits; int ld_logits;
+  __nv_bfloat16 *z; int ld_z;
+  __nv_bfloat16 *out; int ld_out;   // H, O, y, or Ucat (+ column offset for shared)
+  int out_col0;
+  int32_t *status;
+};
+
+// Encodes a 2-D bf16 K-major tensor map (rows x cols, row stride in
+// elements) with a {64, box_rows} box and 128-byte swizzle.  Host only.
+int make_tmap_bf16(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
+                   int64_t cols, int64_t row_stride_elems, int box_rows);
+
+cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p,
+                           int num_sms, int max_ctas, cudaStream_t s);
+
+}  // namespace lmoe

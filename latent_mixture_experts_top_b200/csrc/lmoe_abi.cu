@@ -1,0 +1,535 @@
+// lmoe_abi.cu -- the C ABI declared in include/lmoe.h.
+//
+// One handle = one LatentMoE layer on one device: validated hyper-parameters
+// (Latent-MoE README, "Usage": d, m, n_experts, top_k, alpha, n_shared,
+// variant), repacked weight copies, a workspace sized for max_tokens, and the
+// TMA tensor maps of every operand whose address is fixed.  lmoe_forward
+// enqueues the whole layer on the caller's stream without allocating or
+// synchronising.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/lmoe.h"
+#include "kernels.h"
+
+using namespace lmoe;
+
+namespace {
+
+constexpr int kTileM = 128;   // grouped-GEMM M-tile (tcgen05 M)
+constexpr int kTileN = 256;   // tcgen05 N per tile
+
+struct alignas(64) TensorMap64 {
+  unsigned char bytes[128];   // CUtensorMap is 128 bytes, 64-byte aligned
+};
+
+struct Workspace {
+  float *logits = nullptr;
+  int32_t *ids = nullptr;
+  float *gates = nullptr;
+  int32_t *chunk_counts = nullptr;
+  int32_t *offsets = nullptr;
+  int32_t *perm = nullptr, *pos = nullptr, *row_expert = nullptr;
+  TileEntry *tiles = nullptr;
+  int32_t *n_tiles = nullptr;
+  void *z = nullptr, *zp = nullptr, *H = nullptr, *O = nullptr, *ucat = nullptr;
+  void *x_stage = nullptr, *y_stage = nullptr;
+  int32_t *status = nullptr;
+};
+
+}  // namespace
+
+struct lmoe_layer {
+  lmoe_config cfg;
+  int d = 0, l = 0, m = 0, N = 0, K = 0, ns = 0, ms = 0, Tmax = 0;
+  int bf16 = 0;
+  size_t esize = 4;
+  int device = 0, num_sms = 0;
+  bool loaded = false;
+  int max_tiles = 0;
+  // bf16 layout of the stacked x-matrix: [W_r | pad][W_down | pad][shared gate/up]
+  int n_pad = 0, l_pad = 0, nx_rows = 0;
+  int ky = 0;  // l + n_s * m_s, the reduction length of the last GEMM
+  // weights (handle-owned)
+  void *w_router = nullptr;  // f32 path: [N][d]
+  float *b_router = nullptr;
+  void *w_x = nullptr;       // bf16 path: [nx_rows][d]
+  void *w_down = nullptr;    // f32 path: [l][d]
+  void *w_gu = nullptr;      // bf16: [N][2m][l] interleaved by 128; f32: unused
+  void *w_gate = nullptr, *w_upx = nullptr;  // f32 path: [N][m][l]
+  void *w_out = nullptr;     // [N][l][m]
+  void *s_gate = nullptr, *s_up = nullptr;   // f32 path: [ns][ms][d]
+  void *w_y = nullptr;       // [d][l + ns ms] = [W_up | S_o(0) | S_o(1) ...]
+  Workspace ws;
+  TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
+};
+
+namespace {
+
+int cuda_err(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA; }
+
+// Keeps the caller's current device and switches to the handle's.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+template <typename T>
+bool dalloc(T **p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  return cudaMalloc(reinterpret_cast<void **>(p), bytes) == cudaSuccess;
+}
+
+void free_all(lmoe_layer *h) {
+  void *ptrs[] = {h->w_router, h->b_router, h->w_x, h->w_down, h->w_gu, h->w_gate, h->w_upx,
+                  h->w_out, h->s_gate, h->s_up, h->w_y, h->ws.logits, h->ws.ids, h->ws.gates,
+                  h->ws.chunk_counts, h->ws.offsets, h->ws.perm, h->ws.pos, h->ws.row_expert,
+                  h->ws.tiles, h->ws.n_tiles, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
+                  h->ws.x_stage, h->ws.y_stage, h->ws.status};
+  for (void *p : ptrs)
+    if (p) cudaFree(p);
+}
+
+int validate(const lmoe_config *c, lmoe_layer *h) {
+  if (c->d <= 0 || c->m <= 0 || c->alpha <= 0 || c->max_tokens <= 0 || c->n_shared < 0)
+    return LMOE_ERR_INVALID_CONFIG;
+  if (c->variant != LMOE_EFF && c->variant != LMOE_ACC) return LMOE_ERR_INVALID_CONFIG;
+  if (c->dtype != LMOE_F32 && c->dtype != LMOE_BF16) return LMOE_ERR_INVALID_CONFIG;
+  if (c->d % c->alpha) return LMOE_ERR_INVALID_CONFIG;
+  if (c->n_shared > 0 && c->m_shared <= 0) return LMOE_ERR_INVALID_CONFIG;
+  const int64_t N = c->n_routed_override > 0 ? c->n_routed_override
+                                             : static_cast<int64_t>(c->alpha) * c->n_experts;
+  const int64_t K = c->top_k_override > 0
+                        ? c->top_k_override
+                        : (c->variant == LMOE_ACC ? static_cast<int64_t>(c->alpha) * c->top_k
+                                                  : c->top_k);
+  if (N < 1 || K < 1 || K > N) return LMOE_ERR_INVALID_CONFIG;
+  if (N > 1024) return LMOE_ERR_UNSUPPORTED;
+  h->d = c->d;
+  h->l = c->d / c->alpha;
+  h->m = c->m;
+  h->N = static_cast<int>(N);
+  h->K = static_cast<int>(K);
+  h->ns = c->n_shared;
+  h->ms = c->n_shared > 0 ? c->m_shared : 0;
+  h->Tmax = c->max_tokens;
+  h->bf16 = c->dtype == LMOE_BF16;
+  h->esize = h->bf16 ? 2 : 4;
+  h->ky = h->l + h->ns * h->ms;
+  if (static_cast<int64_t>(h->Tmax) * h->K > INT32_MAX / 2) return LMOE_ERR_UNSUPPORTED;
+  if (h->bf16) {
+    if (h->d % 64 || h->l % 64 || h->m % 128 || (h->ns > 0 && h->ms % 128) || h->N % 32)
+      return LMOE_ERR_UNSUPPORTED;
+  } else {
+    if (h->l % 4 || h->ky % 4) return LMOE_ERR_UNSUPPORTED;
+  }
+  return LMOE_OK;
+}
+
+int make_map(TensorMap64 *dst, const void *base, int64_t rows, int64_t cols, int64_t stride,
+             int box_rows) {
+  return make_tmap_bf16(dst->bytes, base, rows, cols, stride, box_rows) == 0 ? LMOE_OK
+                                                                             : LMOE_ERR_CUDA;
+}
+
+// Device-to-device 2-D copy in elements of size es.
+cudaError_t copy2d(void *dst, size_t dpitch_el, const void *src, size_t spitch_el,
+                   size_t width_el, size_t height, size_t es, cudaStream_t s) {
+  if (width_el == 0 || height == 0) return cudaSuccess;
+  return cudaMemcpy2DAsync(dst, dpitch_el * es, src, spitch_el * es, width_el * es, height,
+                           cudaMemcpyDeviceToDevice, s);
+}
+
+char *off(void *base, size_t elems, size_t es) { return static_cast<char *>(base) + elems * es; }
+
+}  // namespace
+
+extern "C" {
+
+const char *lmoe_strerror(int code) {
+  switch (code) {
+    case LMOE_OK: return "ok";
+    case LMOE_ERR_INVALID_CONFIG: return "invalid configuration or argument";
+    case LMOE_ERR_NULL_ARG: return "required pointer is NULL";
+    case LMOE_ERR_NOT_LOADED: return "weights not loaded";
+    case LMOE_ERR_TOO_MANY_TOKENS: return "token count outside [0, max_tokens]";
+    case LMOE_ERR_CUDA: return "CUDA call failed";
+    case LMOE_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait ran out";
+    case LMOE_ERR_UNSUPPORTED: return "shape not supported by this build";
+    case LMOE_ERR_OUT_OF_MEMORY: return "device allocation failed";
+    default: return "unknown status";
+  }
+}
+
+int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
+  if (!cfg || !out) return LMOE_ERR_NULL_ARG;
+  *out = nullptr;
+  lmoe_layer *h = new (std::nothrow) lmoe_layer();
+  if (!h) return LMOE_ERR_OUT_OF_MEMORY;
+  h->cfg = *cfg;
+  int rc = validate(cfg, h);
+  if (rc != LMOE_OK) { delete h; return rc; }
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) !=
+          cudaSuccess) {
+    delete h;
+    return LMOE_ERR_CUDA;
+  }
+  const size_t T = h->Tmax, TK = static_cast<size_t>(h->Tmax) * h->K, es = h->esize;
+  const size_t N = h->N, d = h->d, l = h->l, m = h->m;
+  h->max_tiles = static_cast<int>(TK / kTileM + N + 1);
+  h->n_pad = (h->N + kTileN - 1) / kTileN * kTileN;
+  h->l_pad = (h->l + kTileN - 1) / kTileN * kTileN;
+  h->nx_rows = h->n_pad + h->l_pad + 2 * h->ns * h->ms;
+  Workspace &w = h->ws;
+  bool ok = dalloc(&w.logits, T * N * 4) && dalloc(&w.ids, TK * 4) && dalloc(&w.gates, TK * 4) &&
+            dalloc(&w.chunk_counts, static_cast<size_t>(dispatch_chunks(h->Tmax)) * N * 4) &&
+            dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TK * 4) && dalloc(&w.pos, TK * 4) &&
+            dalloc(&w.row_expert, TK * 4) &&
+            dalloc(&w.tiles, static_cast<size_t>(h->max_tiles) * sizeof(TileEntry)) &&
+            dalloc(&w.n_tiles, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
+            dalloc(&w.H, TK * m * es) && dalloc(&w.O, TK * l * es) &&
+            dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
+            dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16);
+  if (ok) {  // weights
+    if (h->bf16) {
+      ok = dalloc(&h->w_x, static_cast<size_t>(h->nx_rows) * d * es) &&
+           dalloc(&h->w_gu, N * 2 * m * l * es) && dalloc(&h->w_out, N * l * m * es) &&
+           dalloc(&h->w_y, d * h->ky * es);
+    } else {
+      ok = dalloc(&h->w_router, N * d * es) && dalloc(&h->w_down, l * d * es) &&
+           dalloc(&h->w_gate, N * m * l * es) && dalloc(&h->w_upx, N * m * l * es) &&
+           dalloc(&h->w_out, N * l * m * es) &&
+           dalloc(&h->s_gate, static_cast<size_t>(h->ns) * h->ms * d * es) &&
+           dalloc(&h->s_up, static_cast<size_t>(h->ns) * h->ms * d * es) &&
+           dalloc(&h->w_y, d * h->ky * es);
+    }
+    if (ok && cfg->has_router_bias) ok = dalloc(&h->b_router, N * 4);
+  }
+  if (!ok) {
+    cudaGetLastError();
+    free_all(h);
+    delete h;
+    return LMOE_ERR_OUT_OF_MEMORY;
+  }
+  if (cudaMemset(w.status, 0, 16) != cudaSuccess || cudaMemset(w.n_tiles, 0, 16) != cudaSuccess ||
+      cudaMemset(w.ucat, 0, T * h->ky * es) != cudaSuccess) {
+    free_all(h);
+    delete h;
+    return LMOE_ERR_CUDA;
+  }
+  if (h->bf16) {
+    rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TK), h->l, h->l, kTileM);
+    if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, static_cast<int64_t>(TK), h->m, h->m, kTileM);
+    if (rc == LMOE_OK) rc = make_map(&h->tm_ucat, w.ucat, h->Tmax, h->ky, h->ky, kTileM);
+    if (rc == LMOE_OK)
+      rc = make_map(&h->tm_wx, h->w_x, h->nx_rows, h->d, h->d, kTileN);
+    if (rc == LMOE_OK)
+      rc = make_map(&h->tm_wgu, h->w_gu, static_cast<int64_t>(N) * 2 * h->m, h->l, h->l, kTileN);
+    if (rc == LMOE_OK)
+      rc = make_map(&h->tm_wo, h->w_out, static_cast<int64_t>(N) * h->l, h->m, h->m, kTileN);
+    if (rc == LMOE_OK) rc = make_map(&h->tm_wy, h->w_y, h->d, h->ky, h->ky, kTileN);
+    if (rc != LMOE_OK) {
+      free_all(h);
+      delete h;
+      return rc;
+    }
+  }
+  *out = h;
+  return LMOE_OK;
+}
+
+int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
+  if (!h || !wt) return LMOE_ERR_NULL_ARG;
+  if (!wt->w_router || !wt->w_down || !wt->w_up || !wt->w_gate || !wt->w_upx || !wt->w_out)
+    return LMOE_ERR_NULL_ARG;
+  if (h->ns > 0 && (!wt->s_gate || !wt->s_up || !wt->s_out)) return LMOE_ERR_NULL_ARG;
+  if (h->cfg.has_router_bias && !wt->b_router) return LMOE_ERR_NULL_ARG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t es = h->esize, N = h->N, d = h->d, l = h->l, m = h->m, ns = h->ns, ms = h->ms;
+  const size_t ky = h->ky;
+  cudaError_t e = cudaSuccess;
+  auto cp = [&](void *dst, const void *src, size_t bytes) {
+    if (e == cudaSuccess && bytes) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s);
+  };
+  if (h->cfg.has_router_bias) cp(h->b_router, wt->b_router, N * 4);
+  // W_y = [W_up | S_o(0) | ... ]  ([d][l + ns ms])
+  if (e == cudaSuccess) e = copy2d(h->w_y, ky, wt->w_up, l, l, d, es, s);
+  for (size_t j = 0; j < ns && e == cudaSuccess; ++j)
+    e = copy2d(off(h->w_y, l + j * ms, es), ky, off(const_cast<void *>(wt->s_out), j * d * ms, es),
+               ms, ms, d, es, s);
+  cp(h->w_out, wt->w_out, N * l * m * es);
+  if (h->bf16) {
+    // Stacked x-matrix: rows [0,N) W_r, [n_pad, n_pad+l) W_down, then for each
+    // block b of 128 shared hidden units: 128 gate rows followed by the 128
+    // matching up rows.  Padding rows are zero.
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->w_x, 0, static_cast<size_t>(h->nx_rows) * d * es, s);
+    cp(h->w_x, wt->w_router, N * d * es);
+    cp(off(h->w_x, static_cast<size_t>(h->n_pad) * d, es), wt->w_down, l * d * es);
+    const size_t sh0 = static_cast<size_t>(h->n_pad + h->l_pad);
+    for (size_t b = 0; b < ns * ms / 128; ++b) {
+      cp(off(h->w_x, (sh0 + 256 * b) * d, es), off(const_cast<void *>(wt->s_gate), 128 * b * d, es),
+         128 * d * es);
+      cp(off(h->w_x, (sh0 + 256 * b + 128) * d, es),
+         off(const_cast<void *>(wt->s_up), 128 * b * d, es), 128 * d * es);
+    }
+    // Expert gate/up: per expert, blocks of 128 gate rows then 128 up rows.
+    for (size_t b = 0; b < m / 128 && e == cudaSuccess; ++b) {
+      e = copy2d(off(h->w_gu, 256 * b * l, es), 2 * m * l,
+                 off(const_cast<void *>(wt->w_gate), 128 * b * l, es), m * l, 128 * l, N, es, s);
+      if (e == cudaSuccess)
+        e = copy2d(off(h->w_gu, (256 * b + 128) * l, es), 2 * m * l,
+                   off(const_cast<void *>(wt->w_upx), 128 * b * l, es), m * l, 128 * l, N, es, s);
+    }
+  } else {
+    cp(h->w_router, wt->w_router, N * d * es);
+    cp(h->w_down, wt->w_down, l * d * es);
+    cp(h->w_gate, wt->w_gate, N * m * l * es);
+    cp(h->w_upx, wt->w_upx, N * m * l * es);
+    cp(h->s_gate, wt->s_gate, ns * ms * d * es);
+    cp(h->s_up, wt->s_up, ns * ms * d * es);
+  }
+  if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  h->loaded = true;
+  return LMOE_OK;
+}
+
+static int check_call(lmoe_handle h, int32_t T) {
+  if (!h) return LMOE_ERR_NULL_ARG;
+  if (!h->loaded) return LMOE_ERR_NOT_LOADED;
+  if (T < 0 || T > h->Tmax) return LMOE_ERR_TOO_MANY_TOKENS;
+  return LMOE_OK;
+}
+
+// Router logits (+ z and shared hidden when full) and the routing steps.
+static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cudaStream_t s) {
+  Workspace &w = h->ws;
+  cudaError_t e = cudaSuccess;
+  if (h->bf16) {
+    TensorMap64 tm_x;
+    if (make_map(&tm_x, x, T, h->d, h->d, kTileM) != LMOE_OK) return cudaErrorInvalidValue;
+    TcParams p = {};
+    p.mode = TC_X_FUSED;
+    p.M = T;
+    p.Kdim = h->d;
+    p.n_tiles_n = (full ? h->nx_rows : h->n_pad) / kTileN;
+    p.r_end = h->n_pad;
+    p.z_end = h->n_pad + h->l_pad;
+    p.n_routed = h->N;
+    p.l = h->l;
+    p.logits = w.logits;
+    p.ld_logits = h->N;
+    p.z = static_cast<__nv_bfloat16 *>(w.z);
+    p.ld_z = h->l;
+    p.out = static_cast<__nv_bfloat16 *>(w.ucat);
+    p.ld_out = h->ky;
+    p.out_col0 = h->l;
+    p.status = w.status;
+    const int tiles = (T + kTileM - 1) / kTileM * p.n_tiles_n;
+    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, tiles, s);
+  } else {
+    e = simt_linear(static_cast<const float *>(x), h->d, static_cast<const float *>(h->w_router),
+                    h->d, w.logits, h->N, T, h->N, h->d, s);
+  }
+  if (e != cudaSuccess) return e;
+  e = launch_topk(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates, s);
+  if (e != cudaSuccess) return e;
+  return launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, w.offsets, w.perm, w.pos,
+                         w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s);
+}
+
+int lmoe_route(lmoe_handle h, const void *x, int32_t T, int32_t *ids, float *gates,
+               int32_t *offsets, int32_t *perm, void *stream) {
+  int rc = check_call(h, T);
+  if (rc != LMOE_OK) return rc;
+  if (T > 0 && !x) return LMOE_ERR_NULL_ARG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace &w = h->ws;
+  cudaError_t e = cudaSuccess;
+  if (T > 0) {
+    e = run_route(h, x, T, false, s);
+  } else {
+    e = cudaMemsetAsync(w.offsets, 0, (h->N + 1) * sizeof(int32_t), s);
+  }
+  const size_t TK = static_cast<size_t>(T) * h->K;
+  if (e == cudaSuccess && ids && TK)
+    e = cudaMemcpyAsync(ids, w.ids, TK * 4, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && gates && TK)
+    e = cudaMemcpyAsync(gates, w.gates, TK * 4, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && offsets)
+    e = cudaMemcpyAsync(offsets, w.offsets, (h->N + 1) * 4, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && perm && TK)
+    e = cudaMemcpyAsync(perm, w.perm, TK * 4, cudaMemcpyDeviceToDevice, s);
+  return cuda_err(e);
+}
+
+static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream_t s) {
+  Workspace &w = h->ws;
+  const int TK = T * h->K;
+  cudaError_t e = run_route(h, x, T, true, s);
+  if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  if (h->bf16) {
+    e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * 2, w.zp, s);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    TcParams p = {};
+    p.mode = TC_EXPERT_GU;
+    p.Kdim = h->l;
+    p.n_tiles_n = 2 * h->m / kTileN;
+    p.tiles = w.tiles;
+    p.n_mtiles = w.n_tiles;
+    p.b_rows_per_expert = 2 * h->m;
+    p.out = static_cast<__nv_bfloat16 *>(w.H);
+    p.ld_out = h->m;
+    p.status = w.status;
+    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    p.mode = TC_EXPERT_DOWN;
+    p.Kdim = h->m;
+    p.n_tiles_n = (h->l + kTileN - 1) / kTileN;
+    p.b_rows_per_expert = h->l;
+    p.out = static_cast<__nv_bfloat16 *>(w.O);
+    p.ld_out = h->l;
+    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, p, h->num_sms, h->num_sms, s);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    e = launch_combine(w.O, w.pos, w.gates, T, h->K, h->l, w.ucat, h->ky, true, s);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    TcParams q = {};
+    q.mode = TC_OUT;
+    q.M = T;
+    q.Kdim = h->ky;
+    q.n_tiles_n = (h->d + kTileN - 1) / kTileN;
+    q.out = static_cast<__nv_bfloat16 *>(y);
+    q.ld_out = h->d;
+    q.status = w.status;
+    const int tiles = (T + kTileM - 1) / kTileM * q.n_tiles_n;
+    e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, q, h->num_sms, tiles, s);
+  } else {
+    const float *xf = static_cast<const float *>(x);
+    float *zf = static_cast<float *>(w.z), *zpf = static_cast<float *>(w.zp);
+    float *Hf = static_cast<float *>(w.H), *Of = static_cast<float *>(w.O);
+    float *uf = static_cast<float *>(w.ucat);
+    e = simt_linear(xf, h->d, static_cast<const float *>(h->w_down), h->d, zf, h->l, T, h->l,
+                    h->d, s);
+    if (e == cudaSuccess) e = launch_permute_rows(zf, w.perm, h->K, TK, h->l * 4, zpf, s);
+    if (e == cudaSuccess)
+      e = simt_swiglu(zpf, h->l, static_cast<const float *>(h->w_gate),
+                      static_cast<const float *>(h->w_upx), h->m, w.row_expert, Hf, h->m, TK,
+                      h->m, h->l, s);
+    if (e == cudaSuccess)
+      e = simt_expert_down(Hf, h->m, static_cast<const float *>(h->w_out), w.row_expert, Of, h->l,
+                           TK, h->l, h->m, s);
+    if (e == cudaSuccess) e = launch_combine(Of, w.pos, w.gates, T, h->K, h->l, uf, h->ky, false, s);
+    if (e == cudaSuccess && h->ns > 0)
+      e = simt_swiglu(xf, h->d, static_cast<const float *>(h->s_gate),
+                      static_cast<const float *>(h->s_up), h->ms, nullptr, uf + h->l, h->ky, T,
+                      h->ns * h->ms, h->d, s);
+    if (e == cudaSuccess)
+      e = simt_linear(uf, h->ky, static_cast<const float *>(h->w_y), h->ky,
+                      static_cast<float *>(y), h->d, T, h->d, h->ky, s);
+  }
+  return cuda_err(e);
+}
+
+int lmoe_forward(lmoe_handle h, const void *x, void *y, int32_t T, void *stream) {
+  int rc = check_call(h, T);
+  if (rc != LMOE_OK) return rc;
+  if (T == 0) return LMOE_OK;
+  if (!x || !y) return LMOE_ERR_NULL_ARG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  return forward_impl(h, x, y, T, static_cast<cudaStream_t>(stream));
+}
+
+int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T, void *stream) {
+  int rc = check_call(h, T);
+  if (rc != LMOE_OK) return rc;
+  if (T == 0) return LMOE_OK;
+  if (!x_host || !y_host) return LMOE_ERR_NULL_ARG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * h->d * h->esize;
+  if (cudaMemcpyAsync(h->ws.x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  rc = forward_impl(h, h->ws.x_stage, h->ws.y_stage, T, s);
+  if (rc != LMOE_OK) return rc;
+  if (cudaMemcpyAsync(y_host, h->ws.y_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  return cuda_err(cudaStreamSynchronize(s));
+}
+
+int lmoe_get_dims(lmoe_handle h, int32_t *l, int32_t *n_routed, int32_t *k_active) {
+  if (!h) return LMOE_ERR_NULL_ARG;
+  if (l) *l = h->l;
+  if (n_routed) *n_routed = h->N;
+  if (k_active) *k_active = h->K;
+  return LMOE_OK;
+}
+
+int lmoe_device_status(lmoe_handle h, void *stream) {
+  if (!h) return LMOE_ERR_NULL_ARG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LMOE_ERR_CUDA;
+  int32_t st = 0;
+  if (cudaMemcpy(&st, h->ws.status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  if (st != 0) {
+    cudaMemset(h->ws.status, 0, sizeof(st));
+    return LMOE_ERR_DEVICE_TIMEOUT;
+  }
+  return LMOE_OK;
+}
+
+int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel) {
+  if (!h || !dev_ptr || !numel) return LMOE_ERR_NULL_ARG;
+  const int64_t T = h->Tmax, TK = static_cast<int64_t>(h->Tmax) * h->K;
+  const Workspace &w = h->ws;
+  switch (which) {
+    case 0: *dev_ptr = w.logits; *numel = T * h->N; break;
+    case 1: *dev_ptr = w.z; *numel = T * h->l; break;
+    case 2: *dev_ptr = w.zp; *numel = TK * h->l; break;
+    case 3: *dev_ptr = w.H; *numel = TK * h->m; break;
+    case 4: *dev_ptr = w.O; *numel = TK * h->l; break;
+    case 5: *dev_ptr = w.ucat; *numel = T * h->ky; break;
+    case 6: *dev_ptr = w.ids; *numel = TK; break;
+    case 7: *dev_ptr = w.gates; *numel = TK; break;
+    case 8: *dev_ptr = w.offsets; *numel = h->N + 1; break;
+    case 9: *dev_ptr = w.perm; *numel = TK; break;
+    case 10: *dev_ptr = w.pos; *numel = TK; break;
+    case 11: *dev_ptr = w.n_tiles; *numel = 1; break;
+    default: return LMOE_ERR_INVALID_CONFIG;
+  }
+  return LMOE_OK;
+}
+
+int lmoe_destroy(lmoe_handle h) {
+  if (!h) return LMOE_OK;
+  {
+    DeviceGuard g(h->device);
+    cudaDeviceSynchronize();
+    free_all(h);
+  }
+  delete h;
+  return LMOE_OK;
+}
+
+}  // extern "C"

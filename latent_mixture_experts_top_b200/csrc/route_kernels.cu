@@ -1,0 +1,384 @@
+// route_kernels.cu -- routing, dispatch, permutation and combine kernels.
+//
+// Sources: "LatentMoE Explained" (Towards AI), Figure 3 (router: one score
+// per expert, softmax, top-K), the LatentMoE code module (top-k of the
+// softmax, w / w.sum(), the slot loop "for e in e_ids.unique(): sel = e_ids
+// == e; out[sel] += gate[sel] * expert(z[sel])").  The pages' masked loop is
+// replaced by a histogram -> exclusive scan -> stable scatter that yields the
+// same grouping (experts in index order, tokens ascending within an expert)
+// in three launches and no host synchronisation.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lmoe {
+namespace {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// Order-preserving map of a float to an unsigned key (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// ---------------------------------------------------------------- top-K'
+// One warp per token.  Lane j holds experts e = 32 i + j (i < VPL).  A 64-bit
+// key (float key << 32 | ~e) makes one max-reduction pick the largest logit
+// and, among equal logits, the lower expert index.  K' rounds of a warp
+// butterfly max select the slots in order.  Gates: g_k = e^{s_k - s_0} /
+// sum_j e^{s_j - s_0}, which equals softmax(s) at the selected experts
+// renormalised to sum to one (the softmax denominator cancels).
+template <int VPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int ld,
+                                                   const float *__restrict__ bias, int T, int N,
+                                                   int K, int32_t *__restrict__ ids,
+                                                   float *__restrict__ gates) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const float *row = logits + static_cast<size_t>(t) * ld;
+  unsigned long long key[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    if (e < N) {
+      const float v = row[e] + (bias ? bias[e] : 0.0f);
+      key[i] = (static_cast<unsigned long long>(float_key(v)) << 32) |
+               static_cast<uint32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
+    } else {
+      key[i] = 0ull;
+    }
+  }
+  int32_t *ids_row = ids + static_cast<size_t>(t) * K;
+  float *g_row = gates + static_cast<size_t>(t) * K;
+  float s0 = 0.0f;
+  for (int k = 0; k < K; ++k) {
+    unsigned long long best = key[0];
+#pragma unroll
+    for (int i = 1; i < VPL; ++i) best = key[i] > best ? key[i] : best;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(kFull, best, off);
+      best = o > best ? o : best;
+    }
+    const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best & 0xFFFFFFFFull));
+    const float v = key_float(static_cast<uint32_t>(best >> 32));
+    if (k == 0) s0 = v;
+    if ((e & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (i == (e >> 5)) key[i] = 0ull;
+    }
+    if ((k & 31) == lane) {  // the same lane re-reads this slot below
+      ids_row[k] = e;
+      g_row[k] = v;
+    }
+  }
+  float sum = 0.0f;
+  for (int k = lane; k < K; k += 32) sum += expf(g_row[k] - s0);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+  for (int k = lane; k < K; k += 32) g_row[k] = expf(g_row[k] - s0) / sum;
+}
+
+// ---------------------------------------------------------------- dispatch
+// Phase 1: per-chunk expert histogram (kDispatchChunk tokens per block).
+__global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t *__restrict__ ids,
+                                                             int T, int K, int N,
+                                                             int32_t *__restrict__ counts) {
+  extern __shared__ int32_t cnt[];  // [N]
+  for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kDispatchChunk;
+  const int tn = min(kDispatchChunk, T - t0);
+  const int32_t *base = ids + static_cast<size_t>(t0) * K;
+  for (int i = threadIdx.x; i < tn * K; i += blockDim.x) atomicAdd(&cnt[base[i]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x)
+    counts[static_cast<size_t>(blockIdx.x) * N + e] = cnt[e];
+}
+
+// Inclusive scan across a block of up to 1024 threads; returns the exclusive
+// prefix and writes the total to *total.
+__device__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_sums[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int s = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFull, s, off);
+      if (lane >= off) s += y;
+    }
+    if (lane < nw) warp_sums[lane] = s;  // inclusive warp prefix
+  }
+  __syncthreads();
+  const int before = (w > 0 ? warp_sums[w - 1] : 0) + x - v;
+  *total = warp_sums[nw - 1];
+  __syncthreads();
+  return before;
+}
+
+// Phase 2 (one block of 1024 threads): per-expert exclusive scan over chunks
+// (in place), expert offsets, and the table of tile_m-row M-tiles.
+__global__ void __launch_bounds__(1024) dispatch_scan_kernel(
+    int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
+    TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;  // N <= 1024
+  int tot = 0;
+  if (e < N) {
+    int c = 0;
+    for (; c + 8 <= n_chunks; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = counts[static_cast<size_t>(c + j) * N + e];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        counts[static_cast<size_t>(c + j) * N + e] = tot;
+        tot += v[j];
+      }
+    }
+    for (; c < n_chunks; ++c) {
+      const int v = counts[static_cast<size_t>(c) * N + e];
+      counts[static_cast<size_t>(c) * N + e] = tot;
+      tot += v;
+    }
+  }
+  int all = 0;
+  const int off = block_exclusive_scan(tot, warp_sums, &all);
+  const int mt = (tot + tile_m - 1) / tile_m;
+  int all_tiles = 0;
+  const int tstart = block_exclusive_scan(mt, warp_sums, &all_tiles);
+  if (e < N) {
+    offsets[e] = off;
+    for (int j = 0; j < mt; ++j) {
+      const int idx = tstart + j;
+      if (idx < max_tiles) {
+        TileEntry te;
+        te.row0 = off + j * tile_m;
+        te.row_end = off + tot;
+        te.expert = e;
+        te.pad = 0;
+        tiles[idx] = te;
+      }
+    }
+  }
+  if (threadIdx.x == 0) {
+    offsets[N] = all;
+    *n_tiles = min(all_tiles, max_tiles);
+  }
+}
+
+// Phase 3: stable scatter.  Warp w of a block handles 32 consecutive tokens;
+// a per-warp bitmask per expert gives each (token, slot) its rank among the
+// warp's tokens that chose the same expert (a token picks an expert at most
+// once), the per-warp counts are scanned across the block's warps, and the
+// chunk's base comes from phase 2.  Tokens therefore land in ascending order.
+__global__ void __launch_bounds__(256) dispatch_scatter_kernel(
+    const int32_t *__restrict__ ids, int T, int K, int N, const int32_t *__restrict__ counts,
+    const int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ pos,
+    int32_t *__restrict__ row_expert) {
+  extern __shared__ uint32_t sm[];
+  uint32_t *mask = sm;                                        // [8][N]
+  int32_t *wbase = reinterpret_cast<int32_t *>(sm + 8 * N);  // [8][N]
+  for (int i = threadIdx.x; i < 8 * N; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kDispatchChunk + threadIdx.x;
+  const bool valid = t < T;
+  const int32_t *my_ids = ids + static_cast<size_t>(t) * K;
+  if (valid)
+    for (int k = 0; k < K; ++k) atomicOr(&mask[w * N + my_ids[k]], 1u << lane);
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) {
+      wbase[ww * N + e] = run;
+      run += __popc(mask[ww * N + e]);
+    }
+  }
+  __syncthreads();
+  if (!valid) return;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int32_t *cbase = counts + static_cast<size_t>(blockIdx.x) * N;
+  for (int k = 0; k < K; ++k) {
+    const int e = my_ids[k];
+    const int p = offsets[e] + cbase[e] + wbase[w * N + e] + __popc(mask[w * N + e] & lt);
+    const int flat = t * K + k;
+    perm[p] = flat;
+    pos[flat] = p;
+    row_expert[p] = e;
+  }
+}
+
+// ---------------------------------------------------------------- permute
+__global__ void __launch_bounds__(256) permute_rows_kernel(const uint4 *__restrict__ src,
+                                                           const int32_t *__restrict__ perm,
+                                                           int K, int rows, int vecs_per_row,
+                                                           uint4 *__restrict__ dst) {
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const int tok = perm[r] / K;
+  const uint4 *s = src + static_cast<size_t>(tok) * vecs_per_row;
+  uint4 *d = dst + static_cast<size_t>(r) * vecs_per_row;
+  for (int v = lane; v < vecs_per_row; v += 32) d[v] = s[v];
+}
+
+// ---------------------------------------------------------------- combine
+template <typename Tio>
+__device__ __forceinline__ void accum_vec(float *acc, const uint4 &raw, float g);
+template <>
+__device__ __forceinline__ void accum_vec<__nv_bfloat16>(float *acc, const uint4 &raw, float g) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(h[j]);
+    acc[2 * j] = fmaf(g, f.x, acc[2 * j]);
+    acc[2 * j + 1] = fmaf(g, f.y, acc[2 * j + 1]);
+  }
+}
+template <>
+__device__ __forceinline__ void accum_vec<float>(float *acc, const uint4 &raw, float g) {
+  const float *f = reinterpret_cast<const float *>(&raw);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j] = fmaf(g, f[j], acc[j]);
+}
+template <typename Tio>
+__device__ __forceinline__ uint4 pack_vec(const float *acc);
+template <>
+__device__ __forceinline__ uint4 pack_vec<__nv_bfloat16>(const float *acc) {
+  uint4 r;
+  r.x = pack_bf16x2(acc[0], acc[1]);
+  r.y = pack_bf16x2(acc[2], acc[3]);
+  r.z = pack_bf16x2(acc[4], acc[5]);
+  r.w = pack_bf16x2(acc[6], acc[7]);
+  return r;
+}
+template <>
+__device__ __forceinline__ uint4 pack_vec<float>(const float *acc) {
+  uint4 r;
+  r.x = __float_as_uint(acc[0]);
+  r.y = __float_as_uint(acc[1]);
+  r.z = __float_as_uint(acc[2]);
+  r.w = __float_as_uint(acc[3]);
+  return r;
+}
+
+// One warp per token; 16-byte vectors; slots summed in order 0..K-1 in fp32.
+template <typename Tio>
+__global__ void __launch_bounds__(256) combine_kernel(const Tio *__restrict__ O,
+                                                      const int32_t *__restrict__ pos,
+                                                      const float *__restrict__ gates, int T,
+                                                      int K, int l, Tio *__restrict__ u, int ldu) {
+  constexpr int V = 16 / sizeof(Tio);
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int nvec = l / V;
+  for (int vi = lane; vi < nvec; vi += 32) {
+    float acc[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) acc[j] = 0.0f;
+    for (int k0 = 0; k0 < K; k0 += 32) {
+      const int kk = k0 + lane;
+      const int my_p = kk < K ? pos[static_cast<size_t>(t) * K + kk] : 0;
+      const float my_g = kk < K ? gates[static_cast<size_t>(t) * K + kk] : 0.0f;
+      const int kn = min(32, K - k0);
+      for (int k = 0; k < kn; ++k) {
+        const int p = __shfl_sync(kFull, my_p, k);
+        const float g = __shfl_sync(kFull, my_g, k);
+        const uint4 raw = *reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l + vi * V);
+        accum_vec<Tio>(acc, raw, g);
+      }
+    }
+    *reinterpret_cast<uint4 *>(u + static_cast<size_t>(t) * ldu + vi * V) = pack_vec<Tio>(acc);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, int N, int K,
+                        int32_t *ids, float *gates, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int blocks = (T + 7) / 8;
+  const int vpl = (N + 31) / 32;
+  if (vpl <= 1) topk_kernel<1><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
+  else if (vpl <= 2) topk_kernel<2><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
+  else if (vpl <= 4) topk_kernel<4><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
+  else if (vpl <= 8) topk_kernel<8><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
+  else if (vpl <= 16) topk_kernel<16><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
+  else if (vpl <= 32) topk_kernel<32><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,
+                            int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *row_expert,
+                            TileEntry *tiles, int32_t *n_tiles, int tile_m, int max_tiles,
+                            cudaStream_t s) {
+  if (N > 1024) return cudaErrorInvalidValue;
+  const int nc = dispatch_chunks(T);
+  if (nc > 0) {
+    dispatch_count_kernel<<<nc, 256, N * sizeof(int32_t), s>>>(ids, T, K, N, chunk_counts);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  dispatch_scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, nc, N, offsets, tiles, n_tiles, tile_m,
+                                          max_tiles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || nc == 0) return e;
+  const size_t smem = 16 * static_cast<size_t>(N) * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(dispatch_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dispatch_scatter_kernel<<<nc, 256, smem, s>>>(ids, T, K, N, chunk_counts, offsets, perm, pos,
+                                                row_expert);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
+                                int row_bytes, void *dst, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (row_bytes % 16) return cudaErrorInvalidValue;
+  const int blocks = (rows + 7) / 8;
+  permute_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(src), perm, K, rows,
+                                             row_bytes / 16, static_cast<uint4 *>(dst));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void *O, const int32_t *pos, const float *gates, int T, int K,
+                           int l, void *u, int ldu, bool is_bf16, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int blocks = (T + 7) / 8;
+  if (is_bf16) {
+    if (l % 8 || ldu % 8) return cudaErrorInvalidValue;
+    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(O), pos, gates, T, K, l,
+        static_cast<__nv_bfloat16 *>(u), ldu);
+  } else {
+    if (l % 4 || ldu % 4) return cudaErrorInvalidValue;
+    combine_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float *>(O), pos, gates, T, K,
+                                                 l, static_cast<float *>(u), ldu);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lmoe

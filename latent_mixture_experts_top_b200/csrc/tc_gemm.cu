@@ -1,0 +1,384 @@
+// tc_gemm.cu -- persistent bf16 tcgen05 GEMM for the dense contractions of
+// the LatentMoE layer forward, with four fused epilogues.
+//
+//   TC_X_FUSED     x [T][d] times the stacked matrix [W_r ; W_down ; shared
+//                  gate/up] -> fp32 router logits, bf16 z, and the shared
+//                  experts' SwiGLU hidden (written next to u, so that the
+//                  last GEMM adds the shared output for free).
+//   TC_EXPERT_GU   grouped: permuted z rows of expert e times its gate/up
+//                  rows (interleaved in blocks of 128) -> SwiGLU -> H (bf16).
+//   TC_EXPERT_DOWN grouped: H times W_o[e] -> expert output O (bf16).
+//   TC_OUT         [u | shared hidden] times [W_up | S_o] -> y (bf16).
+//
+// Sources of the maths: "LatentMoE Explained", Figure 3 (router reads the
+// full-width x), Figure 6 (W_down, W_up), Figure 8 (the routed path inside
+// the projections, the shared path at width d), Figure 9 (latent expert
+// l -> m -> l); SwiGLU expert per the paragraph after Figure 1.
+//
+// Structure (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
+//               swizzle, into a 4-stage shared-memory ring (no multicast).
+//   warp 1      TMEM owner and MMA issuer: one thread issues
+//               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into
+//               one of two 256-column fp32 accumulators in TMEM, and
+//               tcgen05.commit frees ring stages / publishes accumulators.
+//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns, fused epilogue,
+//               16-byte global stores; overlaps the next tile's MMAs.
+// Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA records a
+// status, stops its roles, lets in-flight copies and MMAs land, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx_sm100.cuh"
+
+namespace lmoe {
+namespace {
+
+constexpr int TM = 128, TN = 256, TKB = 64;   // tile M, N, K-block
+constexpr int STAGES = 4;
+constexpr int A_BYTES = TM * TKB * 2;         // 16 KB
+constexpr int B_BYTES = TN * TKB * 2;         // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * TN;             // two accumulators
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, TN);
+
+struct __align__(8) SmemCtl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemCtl);
+
+struct Tile {
+  int a_row, b_row, n_tile, row_hi;
+};
+
+__device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles) {
+  Tile tl;
+  if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
+    const int m = t % m_tiles, n = t / m_tiles;  // consecutive CTAs share B
+    tl.a_row = m * TM;
+    tl.b_row = n * TN;
+    tl.n_tile = n;
+    tl.row_hi = p.M;
+  } else {
+    const int mt = t / p.n_tiles_n, n = t % p.n_tiles_n;  // consecutive CTAs share A
+    const TileEntry te = p.tiles[mt];
+    tl.a_row = te.row0;
+    tl.b_row = te.expert * p.b_rows_per_expert + n * TN;
+    tl.n_tile = n;
+    tl.row_hi = te.row_end;
+  }
+  return tl;
+}
+
+__device__ __forceinline__ void record_failure(const TcParams &p, SmemCtl *ctl, int code) {
+  ctl->abort = 1;
+  if (p.status) atomicCAS(p.status, 0, code);
+}
+
+// Bounded wait used only on the abort path (no abort check, shorter limit).
+__device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs / 4) return false;
+  }
+  return true;
+}
+
+// ---- epilogue helpers: one thread = one output row, 32 fp32 columns at a time
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float *v) {
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = w;
+  }
+}
+__device__ __forceinline__ void store_f32x32(float *dst, const float *v) {
+  float4 *d = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// 256 accumulator columns -> bf16 (or f32) row segment, chunks past n_cols skipped.
+template <bool F32OUT, typename OutT>
+__device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_dst, int col0,
+                                          int n_cols) {
+#pragma unroll 1
+  for (int c = 0; c < TN / 32; ++c) {
+    uint32_t r[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+    ptx::tmem_ld_wait();
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    const int col = col0 + c * 32;
+    if (valid && col < n_cols) {
+      if constexpr (F32OUT) store_f32x32(reinterpret_cast<float *>(row_dst) + col, v);
+      else store_bf16x32(reinterpret_cast<__nv_bfloat16 *>(row_dst) + col, v);
+    }
+  }
+}
+
+// Columns [0,128) are gate rows g0..g0+127, [128,256) the matching up rows:
+// h = silu(gate) * up for 128 hidden columns starting at hcol0.
+__device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bfloat16 *row_dst,
+                                           int hcol0) {
+#pragma unroll 1
+  for (int c = 0; c < TN / 64; ++c) {
+    uint32_t g[32], u[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, g);
+    ptx::tmem_ld_32x32b_x32(taddr + TN / 2 + c * 32, u);
+    ptx::tmem_ld_wait();
+    float h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) h[j] = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+    if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *smA = smem;
+  uint8_t *smB = smem + STAGES * A_BYTES;
+  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + STAGES * STAGE_BYTES);
+  volatile int *abort_flag = &ctl->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const bool grouped = (p.mode == TC_EXPERT_GU || p.mode == TC_EXPERT_DOWN);
+  const int m_tiles = grouped ? 0 : (p.M + TM - 1) / TM;
+  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles * p.n_tiles_n;
+  const int nkb = p.Kdim / TKB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&ctl->full[s], 1);
+      ptx::mbar_init(&ctl->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&ctl->acc_full[a], 1);
+      ptx::mbar_init(&ctl->acc_empty[a], 4);  // one arrival per epilogue warp
+    }
+    ptx::mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, t, m_tiles);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
+            record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
+          ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
+          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
+        }
+      }
+      if (!ok) {  // let every copy still in flight land before the CTA exits
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
+            record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, tl_count = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tl_count) {
+        const int acc = tl_count & 1;
+        const uint32_t acc_ph = (tl_count >> 1) & 1;
+        if (!ptx::mbar_wait(&ctl->acc_empty[acc], acc_ph ^ 1, abort_flag)) {
+          record_failure(p, ctl, DEV_TIMEOUT_MMA);
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * TN;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!ptx::mbar_wait(&ctl->full[s], ph, abort_flag)) {
+            record_failure(p, ctl, DEV_TIMEOUT_MMA);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_addr = ptx::smem_u32(smA + s * A_BYTES);
+          const uint32_t b_addr = ptx::smem_u32(smB + s * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < TKB / 16; ++k) {
+            ptx::mma_bf16(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
+                          ptx::smem_desc_sw128(b_addr + k * 32), IDESC, (kb | k) != 0);
+          }
+          ptx::mma_commit(&ctl->empty[s]);  // ring stage free once these MMAs finish
+        }
+        if (!ok) break;
+        ptx::mma_commit(&ctl->acc_full[acc]);  // accumulator ready for the epilogue
+      }
+      if (!ok) {  // let issued MMAs finish before TMEM is freed
+        ptx::mma_commit(&ctl->drain);
+        if (!drain_wait(&ctl->drain, 0)) record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int tl_count = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl_count) {
+      const int acc = tl_count & 1;
+      const uint32_t acc_ph = (tl_count >> 1) & 1;
+      // Lane 0 waits; the verdict is broadcast so the warp stays converged
+      // for the .sync.aligned TMEM loads below.
+      int ok = 1;
+      if (lane == 0) ok = ptx::mbar_wait(&ctl->acc_full[acc], acc_ph, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) {
+        if (lane == 0) record_failure(p, ctl, DEV_TIMEOUT_EPILOGUE);
+        break;
+      }
+      ptx::tc_fence_after();
+      const Tile tl = decode_tile(p, t, m_tiles);
+      const int row = tl.a_row + row_in_tile;
+      const bool valid = row < tl.row_hi;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
+      const int col0 = tl.n_tile * TN;
+      switch (p.mode) {
+        case TC_X_FUSED:
+          if (col0 < p.r_end) {
+            epi_plain<true>(taddr, valid, p.logits + static_cast<size_t>(row) * p.ld_logits, col0,
+                            p.n_routed);
+          } else if (col0 < p.z_end) {
+            epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
+                             col0 - p.r_end, p.l);
+          } else {
+            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
+                       p.out_col0 + (col0 - p.z_end) / 2);
+          }
+          break;
+        case TC_EXPERT_GU:
+          epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2);
+          break;
+        default:  // TC_EXPERT_DOWN, TC_OUT
+          epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
+                           p.ld_out);
+          break;
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace
+
+int make_tmap_bf16(void *tmap_out, const void *base, int64_t rows, int64_t cols,
+                   int64_t row_stride_elems, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0 || cols <= 0) return -1;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_stride_elems * 2) % 16) return -1;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_elems * 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(TKB), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(reinterpret_cast<CUtensorMap *>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+         const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p, int num_sms,
+                           int max_ctas, cudaStream_t s) {
+  static int attr_done = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_done != dev) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    attr_done = dev;
+  }
+  if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
+  const int grid = max_ctas < num_sms ? max_ctas : num_sms;
+  if (grid <= 0) return cudaSuccess;
+  CUtensorMap a, b;
+  memcpy(&a, tmapA, sizeof(a));
+  memcpy(&b, tmapB, sizeof(b));
+  tc_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
+  return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -1,0 +1,225 @@
+"""Thin ctypes binding of ``liblmoe.so`` (include/lmoe.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  The functions keep the C names; torch tensors (device memory)
+are passed as raw pointers, streams as ``torch.cuda.Stream`` or raw handles.
+If the shared library is missing or fails to load, importing this module
+raises -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+from .configs import LayerConfig
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblmoe.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} not built; run `python -m latent_mixture_experts_top_b200.build`")
+_lib = C.CDLL(_LIB_PATH)
+
+LMOE_EFF, LMOE_ACC = 0, 1
+LMOE_F32, LMOE_BF16 = 0, 1
+STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
+          -3: "LMOE_ERR_NOT_LOADED", -4: "LMOE_ERR_TOO_MANY_TOKENS", -5: "LMOE_ERR_CUDA",
+          -6: "LMOE_ERR_DEVICE_TIMEOUT", -7: "LMOE_ERR_UNSUPPORTED",
+          -8: "LMOE_ERR_OUT_OF_MEMORY"}
+EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
+            "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
+            "lmoe_strerror", "lmoe_destroy")
+
+
+class lmoe_config(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in (
+        "d", "m", "n_experts", "top_k", "alpha", "n_shared", "m_shared", "variant", "dtype",
+        "n_routed_override", "top_k_override", "has_router_bias", "max_tokens")]
+
+
+class lmoe_weights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in (
+        "w_router", "b_router", "w_down", "w_up", "w_gate", "w_upx", "w_out", "s_gate",
+        "s_up", "s_out")]
+
+
+P, I32 = C.c_void_p, C.c_int32
+_lib.lmoe_create.argtypes = [C.POINTER(lmoe_config), C.POINTER(C.c_void_p)]
+_lib.lmoe_load_weights.argtypes = [P, C.POINTER(lmoe_weights), P]
+_lib.lmoe_route.argtypes = [P, P, I32, P, P, P, P, P]
+_lib.lmoe_forward.argtypes = [P, P, P, I32, P]
+_lib.lmoe_forward_host.argtypes = [P, P, P, I32, P]
+_lib.lmoe_get_dims.argtypes = [P, C.POINTER(I32), C.POINTER(I32), C.POINTER(I32)]
+_lib.lmoe_device_status.argtypes = [P, P]
+_lib.lmoe_debug_buffer.argtypes = [P, I32, C.POINTER(C.c_void_p), C.POINTER(C.c_int64)]
+_lib.lmoe_strerror.argtypes = [C.c_int]
+_lib.lmoe_strerror.restype = C.c_char_p
+_lib.lmoe_destroy.argtypes = [P]
+for _n in EXPORTED:
+    if _n != "lmoe_strerror":
+        getattr(_lib, _n).restype = C.c_int
+
+
+class LmoeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({lmoe_strerror(code)})")
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise LmoeError(rc, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return t.data_ptr()
+    return int(t)
+
+
+def _stream(s):
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, torch.cuda.Stream):
+        return s.cuda_stream
+    return int(s)
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lmoe_strerror(code: int) -> str:
+    return _lib.lmoe_strerror(code).decode()
+
+
+def config_from(cfg: LayerConfig, max_tokens: int | None = None) -> lmoe_config:
+    return lmoe_config(
+        d=cfg.d, m=cfg.m, n_experts=cfg.n_experts, top_k=cfg.top_k, alpha=cfg.alpha,
+        n_shared=cfg.n_shared, m_shared=cfg.m_shared,
+        variant=LMOE_ACC if cfg.variant == "acc" else LMOE_EFF,
+        dtype=LMOE_BF16 if cfg.dtype == "bf16" else LMOE_F32,
+        n_routed_override=cfg.n_routed_override, top_k_override=cfg.top_k_override,
+        has_router_bias=int(cfg.has_router_bias),
+        max_tokens=cfg.T if max_tokens is None else max_tokens)
+
+
+def lmoe_create(config: lmoe_config) -> int:
+    h = C.c_void_p()
+    _check(_lib.lmoe_create(C.byref(config), C.byref(h)), "lmoe_create")
+    return h.value
+
+
+def lmoe_load_weights(handle: int, weights: dict, stream=None) -> None:
+    w = lmoe_weights(**{k: _ptr(weights.get(k)) for k, _ in lmoe_weights._fields_})
+    _check(_lib.lmoe_load_weights(handle, C.byref(w), _stream(stream)), "lmoe_load_weights")
+
+
+def lmoe_route(handle: int, x, T: int, ids=None, gates=None, offsets=None, perm=None,
+               stream=None) -> None:
+    _check(_lib.lmoe_route(handle, _ptr(x), T, _ptr(ids), _ptr(gates), _ptr(offsets),
+                           _ptr(perm), _stream(stream)), "lmoe_route")
+
+
+def lmoe_forward(handle: int, x, y, T: int, stream=None) -> None:
+    _check(_lib.lmoe_forward(handle, _ptr(x), _ptr(y), T, _stream(stream)), "lmoe_forward")
+
+
+def lmoe_forward_host(handle: int, x_host, y_host, T: int, stream=None) -> None:
+    _check(_lib.lmoe_forward_host(handle, _ptr(x_host), _ptr(y_host), T, _stream(stream)),
+           "lmoe_forward_host")
+
+
+def lmoe_get_dims(handle: int):
+    l, n, k = I32(), I32(), I32()
+    _check(_lib.lmoe_get_dims(handle, C.byref(l), C.byref(n), C.byref(k)), "lmoe_get_dims")
+    return l.value, n.value, k.value
+
+
+def lmoe_device_status(handle: int, stream=None) -> int:
+    return _lib.lmoe_device_status(handle, _stream(stream))
+
+
+def lmoe_debug_buffer(handle: int, which: int):
+    p, n = C.c_void_p(), C.c_int64()
+    _check(_lib.lmoe_debug_buffer(handle, which, C.byref(p), C.byref(n)), "lmoe_debug_buffer")
+    return p.value, n.value
+
+
+def lmoe_destroy(handle: int) -> None:
+    _check(_lib.lmoe_destroy(handle), "lmoe_destroy")
+
+
+class LatentMoELayer:
+    """Convenience owner of one handle: create, load weights, forward.
+
+    Keeps the handle alive and destroys it with the object; every call goes
+    straight through the C ABI above.
+    """
+
+    def __init__(self, cfg: LayerConfig, weights: dict, max_tokens: int | None = None,
+                 stream=None):
+        self.cfg = cfg
+        self.handle = lmoe_create(config_from(cfg, max_tokens))
+        try:
+            lmoe_load_weights(self.handle, weights, stream)
+        except Exception:
+            lmoe_destroy(self.handle)
+            self.handle = None
+            raise
+        self.l, self.n_routed, self.k_active = lmoe_get_dims(self.handle)
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        lmoe_forward(self.handle, x, y, T, stream)
+        return y
+
+    def route(self, x: torch.Tensor, stream=None):
+        T = x.shape[0]
+        dev = x.device
+        ids = torch.empty((T, self.k_active), dtype=torch.int32, device=dev)
+        gates = torch.empty((T, self.k_active), dtype=torch.float32, device=dev)
+        offsets = torch.empty((self.n_routed + 1,), dtype=torch.int32, device=dev)
+        perm = torch.empty((T * self.k_active,), dtype=torch.int32, device=dev)
+        lmoe_route(self.handle, x, T, ids, gates, offsets, perm, stream)
+        return ids, gates, offsets, perm
+
+    def debug_tensor(self, which: int, dtype: torch.dtype, shape) -> torch.Tensor:
+        """A copy of one internal buffer (test hook; see lmoe_debug_buffer)."""
+        ptr, numel = lmoe_debug_buffer(self.handle, which)
+        return device_view(ptr, numel, dtype, shape).clone()
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lmoe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+_TYPESTR = {torch.float32: "<f4", torch.bfloat16: "<u2", torch.int32: "<i4"}
+
+
+def device_view(ptr: int, numel: int, dtype: torch.dtype, shape) -> torch.Tensor:
+    """Zero-copy torch view of `numel` elements at a device address."""
+    n = 1
+    for s in shape:
+        n *= s
+    if n > numel:
+        raise ValueError("view larger than the buffer")
+    holder = type("_DevBuf", (), {})()
+    holder.__cuda_array_interface__ = {"shape": (n,), "typestr": _TYPESTR[dtype],
+                                       "data": (ptr, False), "version": 3}
+    t = torch.as_tensor(holder, device="cuda")
+    if dtype == torch.bfloat16:
+        t = t.view(torch.bfloat16)
+    return t.view(*shape)

@@ -1,0 +1,107 @@
+"""Shared helpers of the GPU parity tests: run the CUDA library and the fp64
+oracle on the same seeded inputs and compare.
+
+Comparison rules (tolerances stated where they are used):
+* routing: the oracle's fp64 logits decide.  A token whose K'-th and
+  (K'+1)-th largest logits are within NEAR_TIE of each other is "near-tie":
+  several selections are correct up to rounding, so only validity is checked
+  there.  Everywhere else the selected set must be identical, and the slot
+  order identical wherever consecutive selected logits differ by more than
+  ORDER_TOL; within ORDER_TOL the GPU order must still be non-increasing in
+  the oracle's logits up to ORDER_TOL.
+* dispatch: offsets / perm must equal the oracle's dispatch of the GPU's own
+  ids exactly (integer work, unique result).
+* y: max|y - y_ref| / max|y_ref| over the compared tokens, where y_ref uses
+  the oracle's routing for tokens whose selection matches and the GPU's ids
+  (oracle forward_given_ids) for near-tie tokens that flipped.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from latent_mixture_experts_top_b200 import synth
+
+NEAR_TIE = 1e-3      # K'-th / (K'+1)-th logit gap below which selection is not unique
+ORDER_TOL = 1e-4     # fp32-accumulated logits differ from fp64 by ~1e-6; 100x margin
+TOL_F32 = 1e-5
+TOL_BF16 = 2e-2
+
+
+def oracle_layer(inputs: dict, k_active: int) -> oracle.Layer:
+    n = {k: (None if v is None else synth.to_numpy(v)) for k, v in inputs.items()}
+    bias = None if n["b_router"] is None else n["b_router"].astype(np.float64)
+    return oracle.Layer(w_router=n["w_router"], b_router=bias, w_down=n["w_down"],
+                        w_up=n["w_up"], w_gate=n["w_gate"], w_upx=n["w_upx"],
+                        w_out=n["w_out"], s_gate=n["s_gate"], s_up=n["s_up"],
+                        s_out=n["s_out"], k_active=k_active)
+
+
+def boundary_gap(s_ref: np.ndarray, K: int) -> np.ndarray:
+    N = s_ref.shape[1]
+    if K >= N:
+        return np.full(s_ref.shape[0], np.inf)
+    part = -np.sort(-s_ref, axis=1)
+    return part[:, K - 1] - part[:, K]
+
+
+def check_routing(ids_gpu: np.ndarray, gates_gpu: np.ndarray, s_ref: np.ndarray, K: int):
+    """Returns (near mask, flipped mask) after asserting the rules above."""
+    T = s_ref.shape[0]
+    ids_ref, g_ref = oracle.select(s_ref, K)
+    near = boundary_gap(s_ref, K) <= NEAR_TIE
+    same_set = np.array([set(a) == set(b) for a, b in zip(ids_gpu.tolist(), ids_ref.tolist())])
+    bad = ~same_set & ~near
+    assert not bad.any(), f"selection differs on {bad.sum()} tokens with a clear gap, e.g. {np.nonzero(bad)[0][:5]}"
+    # every GPU selection is valid: distinct, in range
+    assert ((ids_gpu >= 0) & (ids_gpu < s_ref.shape[1])).all()
+    assert all(len(set(r)) == K for r in ids_gpu.tolist())
+    # order: non-increasing in the oracle's logits (up to ORDER_TOL); identical
+    # where the oracle's consecutive gaps are clear
+    s_sel = np.take_along_axis(s_ref, ids_gpu.astype(np.int64), 1)
+    assert (np.diff(s_sel, axis=1) <= ORDER_TOL).all(), "slot order not by logit"
+    s_ref_sel = np.take_along_axis(s_ref, ids_ref.astype(np.int64), 1)
+    clear = (np.abs(np.diff(s_ref_sel, axis=1)) > ORDER_TOL).all(axis=1) & same_set
+    np.testing.assert_array_equal(ids_gpu[clear], ids_ref[clear])
+    # gates: renormalised softmax of the selected logits (fp32 vs fp64)
+    ids_match = (ids_gpu == ids_ref).all(axis=1)
+    np.testing.assert_allclose(gates_gpu[ids_match], g_ref[ids_match], rtol=0, atol=1e-4)
+    np.testing.assert_allclose(gates_gpu.sum(1), 1.0, rtol=0, atol=1e-5)
+    flipped = ~same_set
+    return near, flipped
+
+
+def check_dispatch(ids_gpu: np.ndarray, offsets: np.ndarray, perm: np.ndarray, N: int):
+    off_ref, perm_ref, _ = oracle.dispatch(ids_gpu, N)
+    np.testing.assert_array_equal(offsets, off_ref)
+    np.testing.assert_array_equal(perm, perm_ref)
+
+
+def rel_err(y: np.ndarray, y_ref: np.ndarray) -> float:
+    return float(np.abs(y - y_ref).max() / max(np.abs(y_ref).max(), 1e-30))
+
+
+def reference_y(L: oracle.Layer, x_np, tokens: np.ndarray, ids_gpu: np.ndarray,
+                flipped: np.ndarray):
+    """y_ref for `tokens`: oracle routing, except GPU ids where the selection flipped."""
+    y = np.empty((len(tokens), L.d))
+    own = ~flipped[tokens]
+    if own.any():
+        y[own], _, _ = oracle.forward(L, x_np, tokens=tokens[own])
+    if (~own).any():
+        y[~own], _, _ = oracle.forward(L, x_np, tokens=tokens[~own], ids=ids_gpu)
+    return y
+
+
+def y_to_numpy(y: torch.Tensor) -> np.ndarray:
+    return y.detach().float().cpu().numpy().astype(np.float64)
+
+
+def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
+    """First and last few tokens, tile boundaries, and a random spread."""
+    rng = np.random.default_rng(seed)
+    fixed = {0, 1, 127, 128, T - 1, T - 2, T // 2}
+    fixed = {t for t in fixed if 0 <= t < T}
+    rest = rng.choice(T, size=min(T, max(0, n - len(fixed))), replace=False)
+    return np.array(sorted(fixed | set(rest.tolist())), dtype=np.int64)

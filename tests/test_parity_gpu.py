@@ -1,0 +1,195 @@
+"""GPU parity: the CUDA library through its C ABI against the fp64 oracle.
+
+Inputs come from latent_mixture_experts_top_b200.synth (seeded, on the GPU);
+the oracle gets host copies of the same rounded values.  Tolerances (from
+the layer's arithmetic): fp32 mode 1e-5 and bf16 mode 2e-2 on
+max|y - y_ref| / max|y_ref|; routing and dispatch exact (see parity_util).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from latent_mixture_experts_top_b200 import configs, synth
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+def _lmoe():
+    from latent_mixture_experts_top_b200 import lmoe
+    return lmoe
+
+
+_INPUT_CACHE = {}
+
+
+def _inputs(cfg, seed=0):
+    key = (cfg.name, seed)
+    if key not in _INPUT_CACHE:
+        _INPUT_CACHE.clear()   # keep at most one big weight set on the device
+        torch.cuda.empty_cache()
+        _INPUT_CACHE[key] = synth.make_inputs(cfg, seed, "cuda")
+    return _INPUT_CACHE[key]
+
+
+def _run(cfg, inp, x=None, max_tokens=None):
+    lm = _lmoe()
+    layer = lm.LatentMoELayer(cfg, inp, max_tokens=max_tokens)
+    x = inp["x"] if x is None else x
+    y = layer.forward(x)
+    ids, gates, offsets, perm = layer.route(x)
+    torch.cuda.synchronize()
+    assert lm.lmoe_device_status(layer.handle) == 0
+    return layer, y, ids, gates, offsets, perm
+
+
+def _check_layer(cfg, n_sample, seed=0):
+    inp = _inputs(cfg, seed)
+    layer, y, ids, gates, offsets, perm = _run(cfg, inp)
+    L = pu.oracle_layer(inp, cfg.k_active)
+    x_np = synth.to_numpy(inp["x"])
+    s_ref = oracle.router_logits(L, x_np)
+    ids_g, gates_g = ids.cpu().numpy(), gates.cpu().numpy()
+    near, flipped = pu.check_routing(ids_g, gates_g, s_ref, cfg.k_active)
+    pu.check_dispatch(ids_g, offsets.cpu().numpy(), perm.cpu().numpy(), cfg.n_routed)
+    if not flipped.any():   # then the oracle's own dispatch must agree too
+        ids_ref, _ = oracle.select(s_ref, cfg.k_active)
+        pu.check_dispatch(ids_ref, offsets.cpu().numpy(), perm.cpu().numpy(), cfg.n_routed)
+    tok = pu.sample_tokens(cfg.T, n_sample) if n_sample < cfg.T else np.arange(cfg.T)
+    y_ref = pu.reference_y(L, x_np, tok, ids_g, flipped)
+    err = pu.rel_err(pu.y_to_numpy(y)[tok], y_ref)
+    tol = pu.TOL_F32 if cfg.dtype == "f32" else pu.TOL_BF16
+    print(f"{cfg.name}: rel err {err:.3e} (tol {tol}), near-tie {near.sum()}, flipped {flipped.sum()}")
+    assert err <= tol
+    layer.close()
+    return err
+
+
+def test_parity_tiny_f32_all_tokens():
+    _check_layer(configs.TINY_F32, n_sample=10 ** 9)
+
+
+def test_parity_readme_acc():
+    _check_layer(configs.README_ACC, n_sample=96)
+
+
+def test_parity_readme_eff():
+    _check_layer(configs.README_EFF, n_sample=96)
+
+
+def test_parity_decode_all_tokens():
+    _check_layer(configs.DECODE, n_sample=10 ** 9)
+
+
+def test_parity_prefill_biased_router():
+    _check_layer(configs.PREFILL, n_sample=48)
+
+
+@pytest.mark.parametrize("cfg", [configs.TINY_F32, configs.README_ACC], ids=["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 5, 129, 333])
+def test_ragged_token_counts(cfg, T):
+    """Token counts that are not a multiple of any tile, in a larger workspace."""
+    inp = _inputs(cfg)
+    x = inp["x"][:T].contiguous()
+    layer, y, ids, gates, offsets, perm = _run(cfg, inp, x=x, max_tokens=cfg.T)
+    L = pu.oracle_layer(inp, cfg.k_active)
+    x_np = synth.to_numpy(x)
+    s_ref = oracle.router_logits(L, x_np)
+    ids_g = ids.cpu().numpy()
+    _, flipped = pu.check_routing(ids_g, gates.cpu().numpy(), s_ref, cfg.k_active)
+    pu.check_dispatch(ids_g, offsets.cpu().numpy(), perm.cpu().numpy(), cfg.n_routed)
+    tok = np.arange(T) if T <= 64 else pu.sample_tokens(T, 48)
+    y_ref = pu.reference_y(L, x_np, tok, ids_g, flipped)
+    tol = pu.TOL_F32 if cfg.dtype == "f32" else pu.TOL_BF16
+    assert pu.rel_err(pu.y_to_numpy(y)[tok], y_ref) <= tol
+    layer.close()
+
+
+@pytest.mark.parametrize("cfg", [configs.TINY_F32, configs.README_ACC], ids=["f32", "bf16"])
+def test_zero_tokens(cfg):
+    lm = _lmoe()
+    inp = _inputs(cfg)
+    layer = lm.LatentMoELayer(cfg, inp)
+    y = torch.full((1, cfg.d), 7.0, device="cuda", dtype=inp["x"].dtype)
+    lm.lmoe_forward(layer.handle, inp["x"], y, 0)
+    offsets = torch.full((cfg.n_routed + 1,), -1, dtype=torch.int32, device="cuda")
+    lm.lmoe_route(layer.handle, inp["x"], 0, None, None, offsets, None)
+    torch.cuda.synchronize()
+    assert (y == 7.0).all()
+    assert (offsets == 0).all()
+    layer.close()
+
+
+def test_hot_expert_and_starved_experts():
+    """A router bias that sends every token to expert 3 (one expert gets all
+    T tokens, several get none): dispatch and output still match."""
+    cfg = configs.README_ACC
+    inp = dict(_inputs(cfg))
+    T = 512
+    bias = torch.zeros(cfg.n_routed, device="cuda")
+    bias[3] = 50.0
+    bias[100:140] = -50.0
+    inp["b_router"] = bias
+    from dataclasses import replace
+    cfgb = replace(cfg, router_bias_std=1.0)
+    x = inp["x"][:T].contiguous()
+    layer, y, ids, gates, offsets, perm = _run(cfgb, inp, x=x, max_tokens=T)
+    off = offsets.cpu().numpy()
+    assert off[4] - off[3] == T
+    assert (np.diff(off)[100:140] == 0).all()
+    L = pu.oracle_layer(inp, cfg.k_active)
+    x_np = synth.to_numpy(x)
+    s_ref = oracle.router_logits(L, x_np)
+    ids_g = ids.cpu().numpy()
+    _, flipped = pu.check_routing(ids_g, gates.cpu().numpy(), s_ref, cfg.k_active)
+    pu.check_dispatch(ids_g, off, perm.cpu().numpy(), cfg.n_routed)
+    tok = pu.sample_tokens(T, 40)
+    y_ref = pu.reference_y(L, x_np, tok, ids_g, flipped)
+    assert pu.rel_err(pu.y_to_numpy(y)[tok], y_ref) <= pu.TOL_BF16
+    layer.close()
+
+
+@pytest.mark.parametrize("cfg", [configs.TINY_F32, configs.README_ACC], ids=["f32", "bf16"])
+def test_deterministic(cfg):
+    inp = _inputs(cfg)
+    lm = _lmoe()
+    layer = lm.LatentMoELayer(cfg, inp)
+    y1 = layer.forward(inp["x"]).clone()
+    y2 = layer.forward(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    layer.close()
+
+
+def test_forward_host_matches_device_path():
+    cfg = configs.README_ACC
+    inp = _inputs(cfg)
+    lm = _lmoe()
+    layer = lm.LatentMoELayer(cfg, inp)
+    y_dev = layer.forward(inp["x"])
+    x_h = inp["x"].cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    lm.lmoe_forward_host(layer.handle, x_h, y_h, cfg.T)
+    torch.cuda.synchronize()
+    assert torch.equal(y_h, y_dev.cpu())
+    layer.close()
+
+
+def test_call_errors_on_device_handle():
+    cfg = configs.TINY_F32
+    lm = _lmoe()
+    h = lm.lmoe_create(lm.config_from(cfg))
+    inp = _inputs(cfg)
+    y = torch.empty_like(inp["x"])
+    with pytest.raises(lm.LmoeError) as e:
+        lm.lmoe_forward(h, inp["x"], y, cfg.T)
+    assert e.value.code == -3     # not loaded
+    lm.lmoe_load_weights(h, inp)
+    with pytest.raises(lm.LmoeError) as e:
+        lm.lmoe_forward(h, inp["x"], y, cfg.T + 1)
+    assert e.value.code == -4     # too many tokens
+    with pytest.raises(lm.LmoeError) as e:
+        lm.lmoe_forward(h, inp["x"], None, cfg.T)
+    assert e.value.code == -2
+    lm.lmoe_destroy(h)

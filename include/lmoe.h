@@ -69,7 +69,8 @@ enum {
  * n_routed_override / top_k_override (0 = derive N' and K' from the variant),
  * has_router_bias, max_tokens (workspace size; forward never allocates).
  * LMOE_BF16 additionally needs d, l, m_shared*n_shared to be multiples of 64,
- * m and m_shared multiples of 128, and N' <= 512 (else LMOE_ERR_UNSUPPORTED). */
+ * m and m_shared multiples of 128, and N' a multiple of 32; every mode needs
+ * N' <= 1024 (else LMOE_ERR_UNSUPPORTED). */
 typedef struct {
   int32_t d, m, n_experts, top_k, alpha, n_shared, m_shared;
   int32_t variant;           /* lmoe_variant */
@@ -152,6 +153,22 @@ int lmoe_device_status(lmoe_handle h, void *stream);
  * of perm), 11 number of 128-row expert tiles).  Errors: NULL_ARG,
  * INVALID_CONFIG (unknown `which`). */
 int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel);
+
+/* Profiling hook.  enable != 0: every later lmoe_forward on this handle also
+ * records a CUDA event on its stream before the first stage and after each
+ * stage (stages, in order: 0 router+down+shared GEMM over x, 1 top-K', 2
+ * dispatch, 3 permute z, 4 expert gate/up GEMM, 5 expert down GEMM, 6
+ * combine, 7 output GEMM; the fp32 mode maps its kernels onto the same
+ * indices).  Events are created here, not in the forward.  Errors: NULL_ARG,
+ * CUDA. */
+int lmoe_profile(lmoe_handle h, int32_t enable);
+
+/* Milliseconds spent in each stage by the most recent profiled lmoe_forward
+ * (waits for its last event).  ms[i] for i < min(n, LMOE_NUM_STAGES);
+ * *launches (may be NULL) = total kernel launches this handle has made.
+ * Errors: NULL_ARG, INVALID_CONFIG (profiling not enabled), CUDA. */
+#define LMOE_NUM_STAGES 8
+int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int64_t *launches);
 
 /* Human-readable name of a status code (static string). */
 const char *lmoe_strerror(int code);

@@ -66,6 +66,10 @@ struct lmoe_layer {
   void *s_gate = nullptr, *s_up = nullptr;   // f32 path: [ns][ms][d]
   void *w_y = nullptr;       // [d][l + ns ms] = [W_up | S_o(0) | S_o(1) ...]
   Workspace ws;
+  // profiling: events around the stages of the last forward; launch counter
+  bool profiling = false;
+  cudaEvent_t ev[LMOE_NUM_STAGES + 1] = {};
+  int64_t launches = 0;
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
 };
 
@@ -309,6 +313,10 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   return LMOE_OK;
 }
 
+static void mark(lmoe_layer *h, int i, cudaStream_t s) {
+  if (h->profiling) cudaEventRecord(h->ev[i], s);
+}
+
 static int check_call(lmoe_handle h, int32_t T) {
   if (!h) return LMOE_ERR_NULL_ARG;
   if (!h->loaded) return LMOE_ERR_NOT_LOADED;
@@ -342,15 +350,35 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.status = w.status;
     const int tiles = (T + kTileM - 1) / kTileM * p.n_tiles_n;
     e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, tiles, s);
+    h->launches += 1;
   } else {
     e = simt_linear(static_cast<const float *>(x), h->d, static_cast<const float *>(h->w_router),
                     h->d, w.logits, h->N, T, h->N, h->d, s);
+    h->launches += 1;
+    if (e == cudaSuccess && full) {  // fp32: z and the shared hidden belong to stage 0 too
+      e = simt_linear(static_cast<const float *>(x), h->d, static_cast<const float *>(h->w_down),
+                      h->d, static_cast<float *>(w.z), h->l, T, h->l, h->d, s);
+      h->launches += 1;
+      if (e == cudaSuccess && h->ns > 0) {
+        e = simt_swiglu(static_cast<const float *>(x), h->d, static_cast<const float *>(h->s_gate),
+                        static_cast<const float *>(h->s_up), h->ms, nullptr,
+                        static_cast<float *>(w.ucat) + h->l, h->ky, T, h->ns * h->ms, h->d, s);
+        h->launches += 1;
+      }
+    }
   }
   if (e != cudaSuccess) return e;
+  if (full) mark(h, 1, s);
   e = launch_topk(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates, s);
+  h->launches += 1;
   if (e != cudaSuccess) return e;
-  return launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, w.offsets, w.perm, w.pos,
-                         w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s);
+  if (full) mark(h, 2, s);
+  e = launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, w.offsets, w.perm, w.pos,
+                      w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s);
+  h->launches += 3;
+  if (e != cudaSuccess) return e;
+  if (full) mark(h, 3, s);
+  return e;
 }
 
 int lmoe_route(lmoe_handle h, const void *x, int32_t T, int32_t *ids, float *gates,
@@ -383,11 +411,14 @@ int lmoe_route(lmoe_handle h, const void *x, int32_t T, int32_t *ids, float *gat
 static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream_t s) {
   Workspace &w = h->ws;
   const int TK = T * h->K;
+  mark(h, 0, s);
   cudaError_t e = run_route(h, x, T, true, s);
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
+  h->launches += 1;
+  if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  mark(h, 4, s);
   if (h->bf16) {
-    e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * 2, w.zp, s);
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
     TcParams p = {};
     p.mode = TC_EXPERT_GU;
     p.Kdim = h->l;
@@ -399,7 +430,9 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.ld_out = h->m;
     p.status = w.status;
     e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
+    h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    mark(h, 5, s);
     p.mode = TC_EXPERT_DOWN;
     p.Kdim = h->m;
     p.n_tiles_n = (h->l + kTileN - 1) / kTileN;
@@ -407,9 +440,13 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.out = static_cast<__nv_bfloat16 *>(w.O);
     p.ld_out = h->l;
     e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, p, h->num_sms, h->num_sms, s);
+    h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    mark(h, 6, s);
     e = launch_combine(w.O, w.pos, w.gates, T, h->K, h->l, w.ucat, h->ky, true, s);
+    h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    mark(h, 7, s);
     TcParams q = {};
     q.mode = TC_OUT;
     q.M = T;
@@ -420,31 +457,32 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     q.status = w.status;
     const int tiles = (T + kTileM - 1) / kTileM * q.n_tiles_n;
     e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, q, h->num_sms, tiles, s);
+    h->launches += 1;
   } else {
-    const float *xf = static_cast<const float *>(x);
-    float *zf = static_cast<float *>(w.z), *zpf = static_cast<float *>(w.zp);
+    float *zpf = static_cast<float *>(w.zp);
     float *Hf = static_cast<float *>(w.H), *Of = static_cast<float *>(w.O);
     float *uf = static_cast<float *>(w.ucat);
-    e = simt_linear(xf, h->d, static_cast<const float *>(h->w_down), h->d, zf, h->l, T, h->l,
-                    h->d, s);
-    if (e == cudaSuccess) e = launch_permute_rows(zf, w.perm, h->K, TK, h->l * 4, zpf, s);
-    if (e == cudaSuccess)
-      e = simt_swiglu(zpf, h->l, static_cast<const float *>(h->w_gate),
-                      static_cast<const float *>(h->w_upx), h->m, w.row_expert, Hf, h->m, TK,
-                      h->m, h->l, s);
+    e = simt_swiglu(zpf, h->l, static_cast<const float *>(h->w_gate),
+                    static_cast<const float *>(h->w_upx), h->m, w.row_expert, Hf, h->m, TK, h->m,
+                    h->l, s);
+    h->launches += 1;
+    mark(h, 5, s);
     if (e == cudaSuccess)
       e = simt_expert_down(Hf, h->m, static_cast<const float *>(h->w_out), w.row_expert, Of, h->l,
                            TK, h->l, h->m, s);
+    h->launches += 1;
+    mark(h, 6, s);
     if (e == cudaSuccess) e = launch_combine(Of, w.pos, w.gates, T, h->K, h->l, uf, h->ky, false, s);
-    if (e == cudaSuccess && h->ns > 0)
-      e = simt_swiglu(xf, h->d, static_cast<const float *>(h->s_gate),
-                      static_cast<const float *>(h->s_up), h->ms, nullptr, uf + h->l, h->ky, T,
-                      h->ns * h->ms, h->d, s);
+    h->launches += 1;
+    mark(h, 7, s);
     if (e == cudaSuccess)
       e = simt_linear(uf, h->ky, static_cast<const float *>(h->w_y), h->ky,
                       static_cast<float *>(y), h->d, T, h->d, h->ky, s);
+    h->launches += 1;
   }
-  return cuda_err(e);
+  if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  mark(h, 8, s);
+  return LMOE_OK;
 }
 
 int lmoe_forward(lmoe_handle h, const void *x, void *y, int32_t T, void *stream) {
@@ -521,12 +559,42 @@ int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *num
   return LMOE_OK;
 }
 
+int lmoe_profile(lmoe_handle h, int32_t enable) {
+  if (!h) return LMOE_ERR_NULL_ARG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  if (enable && !h->ev[0]) {
+    for (int i = 0; i <= LMOE_NUM_STAGES; ++i)
+      if (cudaEventCreate(&h->ev[i]) != cudaSuccess) return LMOE_ERR_CUDA;
+  }
+  h->profiling = enable != 0;
+  return LMOE_OK;
+}
+
+int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int64_t *launches) {
+  if (!h) return LMOE_ERR_NULL_ARG;
+  if (launches) *launches = h->launches;
+  if (!ms || n <= 0) return LMOE_OK;
+  if (!h->profiling || !h->ev[0]) return LMOE_ERR_INVALID_CONFIG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  if (cudaEventSynchronize(h->ev[LMOE_NUM_STAGES]) != cudaSuccess) return LMOE_ERR_CUDA;
+  for (int i = 0; i < n && i < LMOE_NUM_STAGES; ++i) {
+    float t = 0.0f;
+    if (cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]) != cudaSuccess) return LMOE_ERR_CUDA;
+    ms[i] = t;
+  }
+  return LMOE_OK;
+}
+
 int lmoe_destroy(lmoe_handle h) {
   if (!h) return LMOE_OK;
   {
     DeviceGuard g(h->device);
     cudaDeviceSynchronize();
     free_all(h);
+    for (int i = 0; i <= LMOE_NUM_STAGES; ++i)
+      if (h->ev[i]) cudaEventDestroy(h->ev[i]);
   }
   delete h;
   return LMOE_OK;

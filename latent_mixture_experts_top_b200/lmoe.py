@@ -29,7 +29,10 @@ STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -8: "LMOE_ERR_OUT_OF_MEMORY"}
 EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
             "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
-            "lmoe_strerror", "lmoe_destroy")
+            "lmoe_profile", "lmoe_stage_times", "lmoe_strerror", "lmoe_destroy")
+LMOE_NUM_STAGES = 8
+STAGE_NAMES = ("x_gemm_router_down_shared", "topk", "dispatch", "permute_z",
+               "expert_gate_up_gemm", "expert_down_gemm", "combine", "out_gemm")
 
 
 class lmoe_config(C.Structure):
@@ -53,6 +56,8 @@ _lib.lmoe_forward_host.argtypes = [P, P, P, I32, P]
 _lib.lmoe_get_dims.argtypes = [P, C.POINTER(I32), C.POINTER(I32), C.POINTER(I32)]
 _lib.lmoe_device_status.argtypes = [P, P]
 _lib.lmoe_debug_buffer.argtypes = [P, I32, C.POINTER(C.c_void_p), C.POINTER(C.c_int64)]
+_lib.lmoe_profile.argtypes = [P, I32]
+_lib.lmoe_stage_times.argtypes = [P, C.POINTER(C.c_float), I32, C.POINTER(C.c_int64)]
 _lib.lmoe_strerror.argtypes = [C.c_int]
 _lib.lmoe_strerror.restype = C.c_char_p
 _lib.lmoe_destroy.argtypes = [P]
@@ -147,6 +152,24 @@ def lmoe_debug_buffer(handle: int, which: int):
     p, n = C.c_void_p(), C.c_int64()
     _check(_lib.lmoe_debug_buffer(handle, which, C.byref(p), C.byref(n)), "lmoe_debug_buffer")
     return p.value, n.value
+
+
+def lmoe_profile(handle: int, enable: bool) -> None:
+    _check(_lib.lmoe_profile(handle, int(bool(enable))), "lmoe_profile")
+
+
+def lmoe_stage_times(handle: int):
+    """(per-stage milliseconds of the last profiled forward, total launches)."""
+    ms = (C.c_float * LMOE_NUM_STAGES)()
+    n = C.c_int64()
+    _check(_lib.lmoe_stage_times(handle, ms, LMOE_NUM_STAGES, C.byref(n)), "lmoe_stage_times")
+    return list(ms), n.value
+
+
+def lmoe_launches(handle: int) -> int:
+    n = C.c_int64()
+    _check(_lib.lmoe_stage_times(handle, None, 0, C.byref(n)), "lmoe_stage_times")
+    return n.value
 
 
 def lmoe_destroy(handle: int) -> None:

@@ -78,6 +78,23 @@ def check_dispatch(ids_gpu: np.ndarray, offsets: np.ndarray, perm: np.ndarray, N
     np.testing.assert_array_equal(perm, perm_ref)
 
 
+def check_dispatch_against_oracle_ids(ids_ref: np.ndarray, ids_gpu: np.ndarray,
+                                      offsets: np.ndarray, perm: np.ndarray, N: int):
+    """Dispatch vs the oracle's own routing, when both select the same sets.
+
+    perm stores t*K' + k.  Where two selected logits are equal to within
+    rounding, the slot order k may legitimately differ, so the unique part --
+    the token sequence of every expert -- is compared, and the slot part only
+    where the two slot orders agree."""
+    K = ids_ref.shape[1]
+    off_ref, perm_ref, _ = oracle.dispatch(ids_ref, N)
+    np.testing.assert_array_equal(offsets, off_ref)
+    np.testing.assert_array_equal(perm // K, perm_ref // K)
+    same_order = (ids_ref == ids_gpu).all(axis=1)
+    agree = same_order[perm_ref // K]
+    np.testing.assert_array_equal(perm[agree], perm_ref[agree])
+
+
 def rel_err(y: np.ndarray, y_ref: np.ndarray) -> float:
     return float(np.abs(y - y_ref).max() / max(np.abs(y_ref).max(), 1e-30))
 

@@ -55,7 +55,8 @@ def _check_layer(cfg, n_sample, seed=0):
     pu.check_dispatch(ids_g, offsets.cpu().numpy(), perm.cpu().numpy(), cfg.n_routed)
     if not flipped.any():   # then the oracle's own dispatch must agree too
         ids_ref, _ = oracle.select(s_ref, cfg.k_active)
-        pu.check_dispatch(ids_ref, offsets.cpu().numpy(), perm.cpu().numpy(), cfg.n_routed)
+        pu.check_dispatch_against_oracle_ids(ids_ref, ids_g, offsets.cpu().numpy(),
+                                             perm.cpu().numpy(), cfg.n_routed)
     tok = pu.sample_tokens(cfg.T, n_sample) if n_sample < cfg.T else np.arange(cfg.T)
     y_ref = pu.reference_y(L, x_np, tok, ids_g, flipped)
     err = pu.rel_err(pu.y_to_numpy(y)[tok], y_ref)

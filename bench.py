@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Throughput of the LatentMoE layer forward through the C-ABI library.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one lmoe_forward over the README-scale "acc" layer (T=4096 tokens,
+d=2048, l=512, m=1408, N'=256, K'=24, two shared SwiGLU experts of width 1408,
+bf16 operands, fp32 accumulation) on synthetic seeded inputs resident in HBM.
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launch stream, with a 512 MiB write between steps to flush the 126 MB
+L2; barrier + synchronize on both sides; the max over ranks is reported.
+With N > 1 (torchrun) every rank runs an independent replica on its own
+tokens (the layer forward has no exchange step on one GPU): weak scaling.
+
+The JSON line also carries: the roofline of the dominant kernel (per-stage
+CUDA events recorded inside the library over the timed region), the whole
+layer's roofline, an end-to-end number through lmoe_forward_host (host
+buffers, copies inside the timed region), the fp64 oracle timed on a bounded
+sample on the host cores, the launch count, and SM clocks sampled during the
+timed region.  --impl reference times the oracle alone on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LatentMoE fwd tokens/s (1 B200) & % roofline, d2048 l512 N'256 K'24 bf16"
+UNIT = "tokens/s"
+FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="readme_acc",
+                    choices=["readme_acc", "readme_eff", "prefill", "decode"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def workload(name):
+    from latent_mixture_experts_top_b200 import configs
+    return {"readme_acc": configs.README_ACC, "readme_eff": configs.README_EFF,
+            "prefill": configs.PREFILL, "decode": configs.DECODE}[name]
+
+
+def config_json(cfg, n_gpus):
+    return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "l": cfg.l, "m": cfg.m,
+            "n_routed": cfg.n_routed, "k_active": cfg.k_active, "n_shared": cfg.n_shared,
+            "m_shared": cfg.m_shared, "variant": cfg.variant,
+            "router_bias": cfg.has_router_bias, "global_batch": cfg.T * n_gpus,
+            "seq_len": cfg.T, "parallelism": f"replicas x{n_gpus} (no exchange)",
+            "l2": "flushed by a 512 MiB write between timed steps"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic work
+def stage_work(cfg):
+    """Algorithmic FLOPs (tensor stages) or bytes (memory stages) per launch.
+
+    Tensor stages count 2 flops per multiply-add of the layer's definition
+    (no padding, no masked rows).  Memory stages count the bytes the step must
+    read and write once (bf16 activations, int32 indices, fp32 logits/gates).
+    """
+    T, d, l, m, N, K = cfg.T, cfg.d, cfg.l, cfg.m, cfg.n_routed, cfg.k_active
+    ns, ms = cfg.n_shared, cfg.m_shared
+    TK = T * K
+    return {
+        0: ("tensor", 2.0 * T * d * (N + l + 2 * ns * ms)),
+        1: ("hbm", 4.0 * T * N + 8.0 * TK),
+        2: ("hbm", 4.0 * TK * 5),
+        3: ("hbm", 2.0 * TK * l * 2 + 4.0 * TK),
+        4: ("tensor", 2.0 * TK * l * 2 * m),
+        5: ("tensor", 2.0 * TK * m * l),
+        6: ("hbm", 2.0 * TK * l + 8.0 * TK + 2.0 * T * l),
+        7: ("tensor", 2.0 * T * (l + ns * ms) * d),
+    }
+
+
+def layer_flops(cfg):
+    T, d, l, m, N, K = cfg.T, cfg.d, cfg.l, cfg.m, cfg.n_routed, cfg.k_active
+    return 2.0 * T * (d * N + 2 * d * l + 3 * K * l * m + 3 * cfg.n_shared * d * cfg.m_shared)
+
+
+def layer_bytes(cfg, ids=None):
+    """Weights actually touched (router, projections, shared, the distinct
+    experts hit) + x in + y out, bf16."""
+    d, l, m, N = cfg.d, cfg.l, cfg.m, cfg.n_routed
+    touched = N if ids is None else len(set(ids.reshape(-1).tolist()))
+    w = N * d + 2 * d * l + 3 * cfg.n_shared * d * cfg.m_shared + touched * 3 * l * m
+    return 2.0 * (w + 2 * cfg.T * d)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML (read-only)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, index, period=0.02):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = get_r(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml" if self.ok else "unavailable"}
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_rate(cfg, inp_np, budget_s, max_tokens=None):
+    """Tokens/s of the fp64 oracle (full layer incl. router) on the host."""
+    import numpy as np
+    import oracle
+    L = oracle.Layer(w_router=inp_np["w_router"],
+                     b_router=None if inp_np["b_router"] is None else inp_np["b_router"].astype(np.float64),
+                     w_down=inp_np["w_down"], w_up=inp_np["w_up"], w_gate=inp_np["w_gate"],
+                     w_upx=inp_np["w_upx"], w_out=inp_np["w_out"], s_gate=inp_np["s_gate"],
+                     s_up=inp_np["s_up"], s_out=inp_np["s_out"], k_active=cfg.k_active)
+    x = inp_np["x"]
+    cal = min(cfg.T, max(8, oracle.threads()))
+    t0 = time.perf_counter()
+    oracle.forward(L, x, tokens=np.arange(cal))
+    per_tok = (time.perf_counter() - t0) / cal
+    n = int(max(cal, min(cfg.T if max_tokens is None else max_tokens, budget_s / per_tok)))
+    t0 = time.perf_counter()
+    oracle.forward(L, x, tokens=np.arange(n))
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, oracle.threads(), L
+
+
+def numpy_inputs(inp):
+    from latent_mixture_experts_top_b200 import synth
+    return {k: (None if v is None else synth.to_numpy(v)) for k, v in inp.items()}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0      # the oracle runs once, on rank 0; other ranks do no work
+    import numpy as np
+    import torch
+    import oracle
+    from latent_mixture_experts_top_b200 import synth
+    cfg = workload(args.workload)
+    inp = synth.make_inputs(cfg, args.seed, "cpu")
+    n = numpy_inputs(inp)
+    rate_cal, _, _, cores, L = oracle_rate(cfg, n, budget_s=2.0, max_tokens=64)
+    budget = 150.0 / max(1, args.steps + args.warmup)      # whole run within minutes
+    per_step = int(max(1, min(cfg.T, budget * rate_cal)))
+    toks = np.arange(per_step)
+    for _ in range(args.warmup):
+        oracle.forward(L, n["x"], tokens=toks)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(L, n["x"], tokens=toks)
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_json(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} tokens (0..{per_step - 1}) of the "
+                                       f"T={cfg.T} workload per step, full layer incl. router"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def traffic_from_profiles(kernel_key, sha):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
+        return None
+    pat = re.compile(r"traffic_bytes_per_launch\[(\w+)\]\s*=\s*([0-9.eE+]+)\s+source_sha256=(\w+)")
+    for fn in sorted(os.listdir(d)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(d, fn)) as f:
+            for mt in pat.finditer(f.read()):
+                if mt.group(1) == kernel_key and mt.group(3) == sha:
+                    return float(mt.group(2))
+    return None
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for fn in ("tc_gemm.cu", "ptx_sm100.cuh", "common.cuh", "route_kernels.cu"):
+        with open(os.path.join(ROOT, "latent_mixture_experts_top_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from latent_mixture_experts_top_b200 import lmoe, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def allmax(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cfg = workload(args.workload)
+    inp = synth.make_inputs(cfg, args.seed, "cuda")
+    layer = lmoe.LatentMoELayer(cfg, inp)
+    x = inp["x"]
+    y = torch.empty_like(x)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        layer.forward(x, y)
+    torch.cuda.synchronize()
+    if lmoe.lmoe_device_status(layer.handle) != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    lmoe.lmoe_profile(layer.handle, K)
+    launches0 = lmoe.lmoe_launches(layer.handle)
+    clocks = ClockSampler(local).start()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.fill_(1)                    # evict L2 outside the timed window
+        starts[i].record(stream)
+        lmoe.lmoe_forward(layer.handle, x, y, cfg.T, stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    launches = lmoe.lmoe_launches(layer.handle) - launches0
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    stage_ms, n_prof, _ = lmoe.lmoe_stage_times(layer.handle)
+    lmoe.lmoe_profile(layer.handle, 0)
+    if lmoe.lmoe_device_status(layer.handle) != 0:
+        raise RuntimeError("device status error during timing")
+    total_ms = allmax(sum(step_ms))
+    ms_per_step = total_ms / K
+    value = cfg.T * world / (ms_per_step / 1e3)
+
+    peaks, peak_src = load_peaks()
+    work = stage_work(cfg)
+    avg_stage = [t / max(1, n_prof) for t in stage_ms]
+    dom = max(range(len(avg_stage)), key=lambda i: avg_stage[i])
+    kind, amount = work[dom]
+    if kind == "tensor":
+        achieved = amount / (avg_stage[dom] / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        achieved = amount / (avg_stage[dom] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    sha = kernel_source_sha()
+    traffic = traffic_from_profiles(lmoe.STAGE_NAMES[dom], sha)
+    roofline = {"bound": kind, "kernel": lmoe.STAGE_NAMES[dom], "achieved": achieved,
+                "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} (burst)" if kind == "tensor" else peak_src,
+                "algorithmic_per_launch": amount, "avg_launch_ms": avg_stage[dom]}
+    ids = layer.route(x)[0].cpu().numpy()
+    F, B = layer_flops(cfg), layer_bytes(cfg, ids)
+    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+    layer_roof = {"flops": F, "bytes": B, "roofline_ms": 1e3 * t_roof,
+                  "bound": "tensor" if F / (peaks["bf16_tflops"] * 1e12) >= B / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                  "frac": 1e3 * t_roof / ms_per_step,
+                  "achieved_tflops": F / (ms_per_step / 1e3) / 1e12}
+
+    # end to end through the public API with host buffers
+    e2e_steps = args.e2e_steps or max(3, min(K, 50))
+    x_h = x.cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    lmoe.lmoe_forward_host(layer.handle, x_h, y_h, cfg.T)
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        lmoe.lmoe_forward_host(layer.handle, x_h, y_h, cfg.T)
+    e2e_s = allmax(time.perf_counter() - t0)
+    io_bytes = cfg.T * cfg.d * x.element_size()
+    e2e = {"value": cfg.T * world * e2e_steps / e2e_s, "unit": UNIT,
+           "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
+           "steps": e2e_steps, "api": "lmoe_forward_host (pinned host buffers)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n_tok, dt, cores, _ = oracle_rate(cfg, numpy_inputs(inp), budget_s=12.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n_tok} tokens (0..{n_tok - 1}) of the T={cfg.T} workload, full "
+                         f"layer incl. router, fp64, {dt:.1f} s"}
+
+    layer.close()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic: x~N(0,1), weights~N(0,0.02), seeded",
+                "config": config_json(cfg, world), "roofline": roofline,
+                "layer_roofline": layer_roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clk,
+                "stages_ms": {lmoe.STAGE_NAMES[i]: avg_stage[i] for i in range(len(avg_stage))},
+                "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -154,21 +154,23 @@ int lmoe_device_status(lmoe_handle h, void *stream);
  * INVALID_CONFIG (unknown `which`). */
 int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel);
 
-/* Profiling hook.  enable != 0: every later lmoe_forward on this handle also
- * records a CUDA event on its stream before the first stage and after each
+/* Profiling hook.  slots > 0: every later lmoe_forward on this handle also
+ * records CUDA events on its stream before the first stage and after each
  * stage (stages, in order: 0 router+down+shared GEMM over x, 1 top-K', 2
  * dispatch, 3 permute z, 4 expert gate/up GEMM, 5 expert down GEMM, 6
  * combine, 7 output GEMM; the fp32 mode maps its kernels onto the same
- * indices).  Events are created here, not in the forward.  Errors: NULL_ARG,
- * CUDA. */
-int lmoe_profile(lmoe_handle h, int32_t enable);
-
-/* Milliseconds spent in each stage by the most recent profiled lmoe_forward
- * (waits for its last event).  ms[i] for i < min(n, LMOE_NUM_STAGES);
- * *launches (may be NULL) = total kernel launches this handle has made.
- * Errors: NULL_ARG, INVALID_CONFIG (profiling not enabled), CUDA. */
+ * indices), into a ring of `slots` event sets created here (never in the
+ * forward).  slots == 0 turns profiling off.  Errors: NULL_ARG, CUDA. */
 #define LMOE_NUM_STAGES 8
-int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int64_t *launches);
+int lmoe_profile(lmoe_handle h, int32_t slots);
+
+/* Per-stage milliseconds summed over the profiled forwards still in the ring
+ * (the last min(count, slots) since lmoe_profile); waits for their events.
+ * ms[i] for i < min(n, LMOE_NUM_STAGES) (ms may be NULL); *n_forwards = how
+ * many forwards were summed; *launches = kernel launches this handle has made
+ * in total.  Any output may be NULL.  Errors: NULL_ARG, CUDA. */
+int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int32_t *n_forwards,
+                     int64_t *launches);
 
 /* Human-readable name of a status code (static string). */
 const char *lmoe_strerror(int code);

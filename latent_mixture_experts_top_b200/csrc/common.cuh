@@ -36,8 +36,24 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(v);
 }
 
-// silu(a) = a * sigmoid(a) = a / (1 + e^-a), with the CUDA math library's expf.
+// silu(a) = a * sigmoid(a) = a / (1 + e^-a), with the CUDA math library's expf
+// (fp32 mode, held to 1e-5).
 __device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)); }
+
+// Hardware tanh (PTX tanh.approx.f32, one MUFU op; absolute error about 5e-4).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// silu for the bf16 epilogues, from sigmoid(a) = (1 + tanh(a/2)) / 2:
+// silu(a) = h + h * tanh(h) with h = a/2.  Its error (~5e-4 relative) is
+// below half a bf16 ulp of the result, which is rounded to bf16 anyway.
+__device__ __forceinline__ float silu_bf16out(float a) {
+  const float h = 0.5f * a;
+  return fmaf(h, tanh_approx(h), h);
+}
 
 // Two floats -> packed bf16x2 (low half = first), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -66,9 +66,10 @@ struct lmoe_layer {
   void *s_gate = nullptr, *s_up = nullptr;   // f32 path: [ns][ms][d]
   void *w_y = nullptr;       // [d][l + ns ms] = [W_up | S_o(0) | S_o(1) ...]
   Workspace ws;
-  // profiling: events around the stages of the last forward; launch counter
-  bool profiling = false;
-  cudaEvent_t ev[LMOE_NUM_STAGES + 1] = {};
+  // profiling: a ring of event sets (LMOE_NUM_STAGES + 1 per forward)
+  int prof_slots = 0;
+  int64_t prof_count = 0;     // forwards recorded since profiling was enabled
+  cudaEvent_t *ev = nullptr;  // [prof_slots][LMOE_NUM_STAGES + 1]
   int64_t launches = 0;
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
 };
@@ -314,7 +315,10 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
 }
 
 static void mark(lmoe_layer *h, int i, cudaStream_t s) {
-  if (h->profiling) cudaEventRecord(h->ev[i], s);
+  if (h->prof_slots > 0) {
+    const int64_t slot = h->prof_count % h->prof_slots;
+    cudaEventRecord(h->ev[slot * (LMOE_NUM_STAGES + 1) + i], s);
+  }
 }
 
 static int check_call(lmoe_handle h, int32_t T) {
@@ -482,6 +486,7 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   }
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
   mark(h, 8, s);
+  if (h->prof_slots > 0) ++h->prof_count;
   return LMOE_OK;
 }
 
@@ -559,30 +564,55 @@ int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *num
   return LMOE_OK;
 }
 
-int lmoe_profile(lmoe_handle h, int32_t enable) {
+static void free_events(lmoe_layer *h) {
+  if (!h->ev) return;
+  for (int64_t i = 0; i < static_cast<int64_t>(h->prof_slots) * (LMOE_NUM_STAGES + 1); ++i)
+    if (h->ev[i]) cudaEventDestroy(h->ev[i]);
+  free(h->ev);
+  h->ev = nullptr;
+  h->prof_slots = 0;
+}
+
+int lmoe_profile(lmoe_handle h, int32_t slots) {
   if (!h) return LMOE_ERR_NULL_ARG;
+  if (slots < 0) return LMOE_ERR_INVALID_CONFIG;
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
-  if (enable && !h->ev[0]) {
-    for (int i = 0; i <= LMOE_NUM_STAGES; ++i)
-      if (cudaEventCreate(&h->ev[i]) != cudaSuccess) return LMOE_ERR_CUDA;
-  }
-  h->profiling = enable != 0;
+  free_events(h);
+  h->prof_count = 0;
+  if (slots == 0) return LMOE_OK;
+  const int64_t n = static_cast<int64_t>(slots) * (LMOE_NUM_STAGES + 1);
+  h->ev = static_cast<cudaEvent_t *>(calloc(static_cast<size_t>(n), sizeof(cudaEvent_t)));
+  if (!h->ev) return LMOE_ERR_OUT_OF_MEMORY;
+  h->prof_slots = slots;
+  for (int64_t i = 0; i < n; ++i)
+    if (cudaEventCreate(&h->ev[i]) != cudaSuccess) {
+      free_events(h);
+      return LMOE_ERR_CUDA;
+    }
   return LMOE_OK;
 }
 
-int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int64_t *launches) {
+int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int32_t *n_forwards,
+                     int64_t *launches) {
   if (!h) return LMOE_ERR_NULL_ARG;
   if (launches) *launches = h->launches;
+  const int64_t recs = h->prof_slots > 0
+                           ? (h->prof_count < h->prof_slots ? h->prof_count : h->prof_slots)
+                           : 0;
+  if (n_forwards) *n_forwards = static_cast<int32_t>(recs);
   if (!ms || n <= 0) return LMOE_OK;
-  if (!h->profiling || !h->ev[0]) return LMOE_ERR_INVALID_CONFIG;
+  for (int i = 0; i < n; ++i) ms[i] = 0.0f;
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
-  if (cudaEventSynchronize(h->ev[LMOE_NUM_STAGES]) != cudaSuccess) return LMOE_ERR_CUDA;
-  for (int i = 0; i < n && i < LMOE_NUM_STAGES; ++i) {
-    float t = 0.0f;
-    if (cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]) != cudaSuccess) return LMOE_ERR_CUDA;
-    ms[i] = t;
+  for (int64_t r = 0; r < recs; ++r) {
+    cudaEvent_t *e = h->ev + r * (LMOE_NUM_STAGES + 1);
+    if (cudaEventSynchronize(e[LMOE_NUM_STAGES]) != cudaSuccess) return LMOE_ERR_CUDA;
+    for (int i = 0; i < n && i < LMOE_NUM_STAGES; ++i) {
+      float t = 0.0f;
+      if (cudaEventElapsedTime(&t, e[i], e[i + 1]) != cudaSuccess) return LMOE_ERR_CUDA;
+      ms[i] += t;
+    }
   }
   return LMOE_OK;
 }
@@ -593,8 +623,7 @@ int lmoe_destroy(lmoe_handle h) {
     DeviceGuard g(h->device);
     cudaDeviceSynchronize();
     free_all(h);
-    for (int i = 0; i <= LMOE_NUM_STAGES; ++i)
-      if (h->ev[i]) cudaEventDestroy(h->ev[i]);
+    free_events(h);
   }
   delete h;
   return LMOE_OK;

@@ -15,15 +15,17 @@
 // the projections, the shared path at width d), Figure 9 (latent expert
 // l -> m -> l); SwiGLU expert per the paragraph after Figure 1.
 //
-// Structure (one CTA per SM, 192 threads):
+// Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
 //               swizzle, into a 4-stage shared-memory ring (no multicast).
 //   warp 1      TMEM owner and MMA issuer: one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into
 //               one of two 256-column fp32 accumulators in TMEM, and
 //               tcgen05.commit frees ring stages / publishes accumulators.
-//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns, fused epilogue,
-//               16-byte global stores; overlaps the next tile's MMAs.
+//   warps 2-9   epilogue: two warps per TMEM lane quarter, each taking half
+//               of the tile's columns: tcgen05.ld 32 lanes x 32 columns,
+//               fused epilogue, 16-byte global stores; overlaps the next
+//               tile's MMAs.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA records a
 // status, stops its roles, lets in-flight copies and MMAs land, frees TMEM and
 // returns.
@@ -46,7 +48,8 @@ constexpr int A_BYTES = TM * TKB * 2;         // 16 KB
 constexpr int B_BYTES = TN * TKB * 2;         // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * TN;             // two accumulators
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_EPI_WARPS = 8;              // two per TMEM lane quarter
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, TN);
 
 struct __align__(8) SmemCtl {
@@ -119,9 +122,9 @@ __device__ __forceinline__ void store_f32x32(float *dst, const float *v) {
 // 256 accumulator columns -> bf16 (or f32) row segment, chunks past n_cols skipped.
 template <bool F32OUT, typename OutT>
 __device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_dst, int col0,
-                                          int n_cols) {
+                                          int n_cols, int half) {
 #pragma unroll 1
-  for (int c = 0; c < TN / 32; ++c) {
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
     uint32_t r[32];
     ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
     ptx::tmem_ld_wait();
@@ -139,16 +142,16 @@ __device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_
 // Columns [0,128) are gate rows g0..g0+127, [128,256) the matching up rows:
 // h = silu(gate) * up for 128 hidden columns starting at hcol0.
 __device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bfloat16 *row_dst,
-                                           int hcol0) {
+                                           int hcol0, int half) {
 #pragma unroll 1
-  for (int c = 0; c < TN / 64; ++c) {
+  for (int c = half * (TN / 128); c < (half + 1) * (TN / 128); ++c) {
     uint32_t g[32], u[32];
     ptx::tmem_ld_32x32b_x32(taddr + c * 32, g);
     ptx::tmem_ld_32x32b_x32(taddr + TN / 2 + c * 32, u);
     ptx::tmem_ld_wait();
     float h[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) h[j] = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+    for (int j = 0; j < 32; ++j) h[j] = silu_bf16out(__uint_as_float(g[j])) * __uint_as_float(u[j]);
     if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
   }
 }
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&ctl->acc_full[a], 1);
-      ptx::mbar_init(&ctl->acc_empty[a], 4);  // one arrival per epilogue warp
+      ptx::mbar_init(&ctl->acc_empty[a], NUM_EPI_WARPS);  // one arrival per epilogue warp
     }
     ptx::mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -266,7 +269,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row_in_tile = q * 32 + lane;
     int tl_count = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl_count) {
@@ -291,21 +295,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         case TC_X_FUSED:
           if (col0 < p.r_end) {
             epi_plain<true>(taddr, valid, p.logits + static_cast<size_t>(row) * p.ld_logits, col0,
-                            p.n_routed);
+                            p.n_routed, half);
           } else if (col0 < p.z_end) {
             epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
-                             col0 - p.r_end, p.l);
+                             col0 - p.r_end, p.l, half);
           } else {
             epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
-                       p.out_col0 + (col0 - p.z_end) / 2);
+                       p.out_col0 + (col0 - p.z_end) / 2, half);
           }
           break;
         case TC_EXPERT_GU:
-          epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2);
+          epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
           break;
         default:  // TC_EXPERT_DOWN, TC_OUT
           epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
-                           p.ld_out);
+                           p.ld_out, half);
           break;
       }
       ptx::tc_fence_before();

@@ -57,7 +57,8 @@ _lib.lmoe_get_dims.argtypes = [P, C.POINTER(I32), C.POINTER(I32), C.POINTER(I32)
 _lib.lmoe_device_status.argtypes = [P, P]
 _lib.lmoe_debug_buffer.argtypes = [P, I32, C.POINTER(C.c_void_p), C.POINTER(C.c_int64)]
 _lib.lmoe_profile.argtypes = [P, I32]
-_lib.lmoe_stage_times.argtypes = [P, C.POINTER(C.c_float), I32, C.POINTER(C.c_int64)]
+_lib.lmoe_stage_times.argtypes = [P, C.POINTER(C.c_float), I32, C.POINTER(I32),
+                                  C.POINTER(C.c_int64)]
 _lib.lmoe_strerror.argtypes = [C.c_int]
 _lib.lmoe_strerror.restype = C.c_char_p
 _lib.lmoe_destroy.argtypes = [P]
@@ -154,21 +155,23 @@ def lmoe_debug_buffer(handle: int, which: int):
     return p.value, n.value
 
 
-def lmoe_profile(handle: int, enable: bool) -> None:
-    _check(_lib.lmoe_profile(handle, int(bool(enable))), "lmoe_profile")
+def lmoe_profile(handle: int, slots: int) -> None:
+    _check(_lib.lmoe_profile(handle, int(slots)), "lmoe_profile")
 
 
 def lmoe_stage_times(handle: int):
-    """(per-stage milliseconds of the last profiled forward, total launches)."""
+    """(per-stage ms summed over the profiled forwards, their count, launches)."""
     ms = (C.c_float * LMOE_NUM_STAGES)()
+    nf = I32()
     n = C.c_int64()
-    _check(_lib.lmoe_stage_times(handle, ms, LMOE_NUM_STAGES, C.byref(n)), "lmoe_stage_times")
-    return list(ms), n.value
+    _check(_lib.lmoe_stage_times(handle, ms, LMOE_NUM_STAGES, C.byref(nf), C.byref(n)),
+           "lmoe_stage_times")
+    return list(ms), nf.value, n.value
 
 
 def lmoe_launches(handle: int) -> int:
     n = C.c_int64()
-    _check(_lib.lmoe_stage_times(handle, None, 0, C.byref(n)), "lmoe_stage_times")
+    _check(_lib.lmoe_stage_times(handle, None, 0, None, C.byref(n)), "lmoe_stage_times")
     return n.value
 
 

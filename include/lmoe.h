@@ -172,6 +172,38 @@ int lmoe_profile(lmoe_handle h, int32_t slots);
 int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int32_t *n_forwards,
                      int64_t *launches);
 
+/* Dispatch without allocation.  The paper has no counterpart to this call:
+ * it exists for callers that may not call cudaMalloc where they need the
+ * dispatch -- for instance a serving loop whose device memory is entirely
+ * reserved up front by its own pool allocator, or a plugin whose host
+ * framework forbids allocation inside its execute callback.
+ *
+ * Given ids [T][k_active] int32 on the device (as lmoe_route produces them:
+ * every id in [0, n_routed), no id twice in a row -- other values are not
+ * checked and their result is undefined), writes offsets [n_routed+1] and
+ * perm [T*k_active] exactly as lmoe_route does, asynchronously on `stream`.
+ * It needs no handle and calls no cudaMalloc, cudaFree or allocating
+ * routine: its scratch (about 3 MiB) is one fixed file-scope device array
+ * that every GPU loading this library holds until the process exits.
+ *   - Limits: T <= LMOE_NOALLOC_MAX_TOKENS, T*k_active <=
+ *     LMOE_NOALLOC_MAX_PAIRS (else LMOE_ERR_TOO_MANY_TOKENS), n_routed <=
+ *     LMOE_NOALLOC_MAX_EXPERTS (else LMOE_ERR_UNSUPPORTED); k_active outside
+ *     [1, n_routed] or T < 0 gives LMOE_ERR_INVALID_CONFIG; NULL offsets, or
+ *     NULL ids / perm with T > 0, gives LMOE_ERR_NULL_ARG.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, and it keeps the last
+ *     call's contents (each call rewrites every word it reads).  Calls that
+ *     overlap on the GPU -- on different streams, or from different threads
+ *     -- race on it and give wrong results; serialise them.
+ * Errors: as listed above, and LMOE_ERR_CUDA. */
+#define LMOE_NOALLOC_MAX_TOKENS 65536
+#define LMOE_NOALLOC_MAX_PAIRS 262144
+#define LMOE_NOALLOC_MAX_EXPERTS 1024
+int lmoe_dispatch_noalloc(const int32_t *ids, int32_t T, int32_t k_active, int32_t n_routed,
+                          int32_t *offsets, int32_t *perm, void *stream);
+
 /* Human-readable name of a status code (static string). */
 const char *lmoe_strerror(int code);
 

@@ -29,7 +29,8 @@ STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -8: "LMOE_ERR_OUT_OF_MEMORY"}
 EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
             "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
-            "lmoe_profile", "lmoe_stage_times", "lmoe_strerror", "lmoe_destroy")
+            "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc", "lmoe_strerror",
+            "lmoe_destroy")
 LMOE_NUM_STAGES = 8
 STAGE_NAMES = ("x_gemm_router_down_shared", "topk", "dispatch", "permute_z",
                "expert_gate_up_gemm", "expert_down_gemm", "combine", "out_gemm")
@@ -59,6 +60,7 @@ _lib.lmoe_debug_buffer.argtypes = [P, I32, C.POINTER(C.c_void_p), C.POINTER(C.c_
 _lib.lmoe_profile.argtypes = [P, I32]
 _lib.lmoe_stage_times.argtypes = [P, C.POINTER(C.c_float), I32, C.POINTER(I32),
                                   C.POINTER(C.c_int64)]
+_lib.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P]
 _lib.lmoe_strerror.argtypes = [C.c_int]
 _lib.lmoe_strerror.restype = C.c_char_p
 _lib.lmoe_destroy.argtypes = [P]
@@ -173,6 +175,14 @@ def lmoe_launches(handle: int) -> int:
     n = C.c_int64()
     _check(_lib.lmoe_stage_times(handle, None, 0, None, C.byref(n)), "lmoe_stage_times")
     return n.value
+
+
+def lmoe_dispatch_noalloc(ids, T: int, k_active: int, n_routed: int, offsets, perm,
+                          stream=None) -> None:
+    """Dispatch with no allocation (see include/lmoe.h); for callers that may
+    not allocate device memory where they run it."""
+    _check(_lib.lmoe_dispatch_noalloc(_ptr(ids), T, k_active, n_routed, _ptr(offsets),
+                                      _ptr(perm), _stream(stream)), "lmoe_dispatch_noalloc")
 
 
 def lmoe_destroy(handle: int) -> None:

@@ -64,7 +64,8 @@ struct TcParams {
   int mode;
   int M;               // dense: rows (T); grouped: unused (tile table)
   int Kdim;            // reduction length, multiple of 64
-  int n_tiles_n;       // N-tiles of 256 columns
+  int n_tiles_n;       // N-tiles of 256 columns in this launch
+  int n_tile_base;     // dense modes: first N-tile (a launch may cover a column range)
   const TileEntry *tiles;   // grouped modes
   const int32_t *n_mtiles;  // grouped modes: device count of M-tiles
   int b_rows_per_expert;    // grouped modes: B rows per expert (2m or l)

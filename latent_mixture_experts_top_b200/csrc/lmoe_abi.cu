@@ -71,6 +71,10 @@ struct lmoe_layer {
   int64_t prof_count = 0;     // forwards recorded since profiling was enabled
   cudaEvent_t *ev = nullptr;  // [prof_slots][LMOE_NUM_STAGES + 1]
   int64_t launches = 0;
+  // bf16: the shared experts' gate/up GEMM runs on a side stream, forked after
+  // the router/down GEMM and joined before the output GEMM.
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
 };
 
@@ -106,6 +110,11 @@ void free_all(lmoe_layer *h) {
                   h->ws.x_stage, h->ws.y_stage, h->ws.status};
   for (void *p : ptrs)
     if (p) cudaFree(p);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->side) cudaStreamDestroy(h->side);
+  h->ev_fork = h->ev_join = nullptr;
+  h->side = nullptr;
 }
 
 int validate(const lmoe_config *c, lmoe_layer *h) {
@@ -247,6 +256,11 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wo, h->w_out, static_cast<int64_t>(N) * h->l, h->m, h->m, kTileN);
     if (rc == LMOE_OK) rc = make_map(&h->tm_wy, h->w_y, h->d, h->ky, h->ky, kTileN);
+    if (rc == LMOE_OK &&
+        (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
+         cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+         cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess))
+      rc = LMOE_ERR_CUDA;
     if (rc != LMOE_OK) {
       free_all(h);
       delete h;
@@ -339,7 +353,8 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.mode = TC_X_FUSED;
     p.M = T;
     p.Kdim = h->d;
-    p.n_tiles_n = (full ? h->nx_rows : h->n_pad) / kTileN;
+    p.n_tile_base = 0;
+    p.n_tiles_n = (full ? h->n_pad + h->l_pad : h->n_pad) / kTileN;
     p.r_end = h->n_pad;
     p.z_end = h->n_pad + h->l_pad;
     p.n_routed = h->N;
@@ -352,9 +367,24 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.ld_out = h->ky;
     p.out_col0 = h->l;
     p.status = w.status;
-    const int tiles = (T + kTileM - 1) / kTileM * p.n_tiles_n;
-    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, tiles, s);
+    const int m_tiles = (T + kTileM - 1) / kTileM;
+    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, m_tiles * p.n_tiles_n, s);
     h->launches += 1;
+    const int shared_tiles_n = (h->nx_rows - h->n_pad - h->l_pad) / kTileN;
+    if (e == cudaSuccess && full && shared_tiles_n > 0) {
+      // Shared experts' gate/up (same kernel, the shared column range) on the
+      // side stream: it overlaps the routing kernels; the output GEMM joins it.
+      TcParams q = p;
+      q.n_tile_base = (h->n_pad + h->l_pad) / kTileN;
+      q.n_tiles_n = shared_tiles_n;
+      e = cudaEventRecord(h->ev_fork, s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
+      if (e == cudaSuccess)
+        e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, q, h->num_sms, m_tiles * shared_tiles_n,
+                           h->side);
+      if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
+      h->launches += 1;
+    }
   } else {
     e = simt_linear(static_cast<const float *>(x), h->d, static_cast<const float *>(h->w_router),
                     h->d, w.logits, h->N, T, h->N, h->d, s);
@@ -451,6 +481,8 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 7, s);
+    e = cudaStreamWaitEvent(s, h->ev_join, 0);  // shared hidden ready
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
     TcParams q = {};
     q.mode = TC_OUT;
     q.M = T;

@@ -70,11 +70,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
     const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best & 0xFFFFFFFFull));
     const float v = key_float(static_cast<uint32_t>(best >> 32));
     if (k == 0) s0 = v;
-    if ((e & 31) == lane) {
 #pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (i == (e >> 5)) key[i] = 0ull;
-    }
+    for (int i = 0; i < VPL; ++i)  // keys are unique: remove the winner by value
+      if (key[i] == best) key[i] = 0ull;
     if ((k & 31) == lane) {  // the same lane re-reads this slot below
       ids_row[k] = e;
       g_row[k] = v;

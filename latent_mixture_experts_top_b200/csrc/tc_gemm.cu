@@ -70,7 +70,7 @@ struct Tile {
 __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles) {
   Tile tl;
   if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
-    const int m = t % m_tiles, n = t / m_tiles;  // consecutive CTAs share B
+    const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
     tl.a_row = m * TM;
     tl.b_row = n * TN;
     tl.n_tile = n;

@@ -27,11 +27,12 @@ constexpr int kMaxTokens = LMOE_NOALLOC_MAX_TOKENS;
 constexpr int kMaxPairs = LMOE_NOALLOC_MAX_PAIRS;
 constexpr int kMaxExperts = LMOE_NOALLOC_MAX_EXPERTS;
 constexpr int kTileRows = 128;
+constexpr int kChunk = 256;  // tokens per histogram chunk (fewer chunks: smaller scratch)
 constexpr int kMaxTiles = kMaxPairs / kTileRows + kMaxExperts + 1;
 
 constexpr size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 constexpr size_t kCountsBytes =
-    round256(static_cast<size_t>((kMaxTokens + kDispatchChunk - 1) / kDispatchChunk) *
+    round256(static_cast<size_t>((kMaxTokens + kChunk - 1) / kChunk) *
              kMaxExperts * sizeof(int32_t));
 constexpr size_t kPosBytes = round256(static_cast<size_t>(kMaxPairs) * sizeof(int32_t));
 constexpr size_t kTilesBytes = round256(static_cast<size_t>(kMaxTiles) * sizeof(TileEntry));
@@ -94,7 +95,8 @@ extern "C" int lmoe_dispatch_noalloc(const int32_t *ids, int32_t T, int32_t k_ac
   TileEntry *tiles = reinterpret_cast<TileEntry *>(base + kOffTiles);
   int32_t *n_tiles = reinterpret_cast<int32_t *>(base + kOffNTiles);
   const cudaError_t e =
-      launch_dispatch(ids, T, k_active, n_routed, counts, offsets, perm, pos, row_expert, tiles,
-                      n_tiles, kTileRows, kMaxTiles, static_cast<cudaStream_t>(stream));
+      launch_dispatch(ids, T, k_active, n_routed, counts, kChunk, false, offsets, perm, pos,
+                      row_expert, tiles, n_tiles, kTileRows, kMaxTiles,
+                      static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

@@ -14,21 +14,25 @@ struct TileEntry {
 };
 
 // ---- routing (route_kernels.cu)
-// ids/gates from fp32 logits [T][ld] (+ bias [N]); one warp per token.
+// ids/gates from fp32 logits [T][ld] (+ bias [N]); one warp per token.  If
+// counts is non-null ([N][dispatch_chunks(T, chunk)], zeroed beforehand) the
+// kernel also accumulates the dispatch's per-chunk expert histogram.
 cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, int N, int K,
-                        int32_t *ids, float *gates, cudaStream_t s);
+                        int32_t *ids, float *gates, int32_t *counts, int chunk, cudaStream_t s);
 
-// Tokens per dispatch chunk and the per-chunk count matrix size.
-constexpr int kDispatchChunk = 256;
-inline int dispatch_chunks(int T) { return (T + kDispatchChunk - 1) / kDispatchChunk; }
+// Tokens per dispatch chunk on the forward path, and the chunk count.
+constexpr int kDispatchChunk = 64;
+inline int dispatch_chunks(int T, int chunk) { return (T + chunk - 1) / chunk; }
 
-// Histogram -> exclusive scan -> stable scatter.  Writes offsets [N+1],
-// perm / pos / row_expert [T*K], and the M-tile table (tile_m rows per tile;
-// capacity max_tiles entries) plus its length in *n_tiles.
+// Histogram (unless counts_ready) -> exclusive scan -> stable scatter.  The
+// count matrix chunk_counts is [N][dispatch_chunks(T, chunk)] (chunk: a
+// multiple of 32, at most 256).  Writes offsets [N+1], perm / pos /
+// row_expert [T*K], and the M-tile table (tile_m rows per tile; capacity
+// max_tiles entries) plus its length in *n_tiles.
 cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,
-                            int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *row_expert,
-                            TileEntry *tiles, int32_t *n_tiles, int tile_m, int max_tiles,
-                            cudaStream_t s);
+                            int chunk, bool counts_ready, int32_t *offsets, int32_t *perm,
+                            int32_t *pos, int32_t *row_expert, TileEntry *tiles,
+                            int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s);
 
 // dst[p][:] = src[perm[p] / K][:], rows of `row_bytes` (multiple of 16).
 cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
@@ -76,11 +80,17 @@ struct TcParams {
   __nv_bfloat16 *z; int ld_z;
   __nv_bfloat16 *out; int ld_out;   // H, O, y, or Ucat (+ column offset for shared)
   int out_col0;
+  // TC_EXPERT_GU: when gather_perm is set, A row r of a tile is row
+  // gather_perm[row0 + r] / gather_k of the A tensor (z), fetched with TMA
+  // gather4 (rows at or past gather_rows fetch row 0 and are masked).
+  const int32_t *gather_perm;
+  int gather_k, gather_rows;
   int32_t *status;
 };
 
 // Encodes a 2-D bf16 K-major tensor map (rows x cols, row stride in
-// elements) with a {64, box_rows} box and 128-byte swizzle.  Host only.
+// elements) with a {64, box_rows} box and 128-byte swizzle (box_rows = 1 for
+// gather4 maps).  Host only.
 int make_tmap_bf16(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
                    int64_t cols, int64_t row_stride_elems, int box_rows);
 

@@ -75,7 +75,7 @@ struct lmoe_layer {
   // the router/down GEMM and joined before the output GEMM.
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-  TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
+  TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat, tm_zg;
 };
 
 namespace {
@@ -210,7 +210,8 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   h->nx_rows = h->n_pad + h->l_pad + 2 * h->ns * h->ms;
   Workspace &w = h->ws;
   bool ok = dalloc(&w.logits, T * N * 4) && dalloc(&w.ids, TK * 4) && dalloc(&w.gates, TK * 4) &&
-            dalloc(&w.chunk_counts, static_cast<size_t>(dispatch_chunks(h->Tmax)) * N * 4) &&
+            dalloc(&w.chunk_counts,
+                   static_cast<size_t>(dispatch_chunks(h->Tmax, kDispatchChunk)) * N * 4) &&
             dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TK * 4) && dalloc(&w.pos, TK * 4) &&
             dalloc(&w.row_expert, TK * 4) &&
             dalloc(&w.tiles, static_cast<size_t>(h->max_tiles) * sizeof(TileEntry)) &&
@@ -247,6 +248,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   }
   if (h->bf16) {
     rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TK), h->l, h->l, kTileM);
+    if (rc == LMOE_OK) rc = make_map(&h->tm_zg, w.z, h->Tmax, h->l, h->l, 1);  // gather4
     if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, static_cast<int64_t>(TK), h->m, h->m, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_ucat, w.ucat, h->Tmax, h->ky, h->ky, kTileM);
     if (rc == LMOE_OK)
@@ -403,13 +405,18 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
   }
   if (e != cudaSuccess) return e;
   if (full) mark(h, 1, s);
-  e = launch_topk(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates, s);
+  // top-K' also builds the dispatch histogram (into the zeroed count matrix)
+  e = cudaMemsetAsync(w.chunk_counts, 0,
+                      static_cast<size_t>(dispatch_chunks(T, kDispatchChunk)) * h->N * 4, s);
+  if (e != cudaSuccess) return e;
+  e = launch_topk(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates, w.chunk_counts,
+                  kDispatchChunk, s);
   h->launches += 1;
   if (e != cudaSuccess) return e;
   if (full) mark(h, 2, s);
-  e = launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, w.offsets, w.perm, w.pos,
-                      w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s);
-  h->launches += 3;
+  e = launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, kDispatchChunk, true, w.offsets,
+                      w.perm, w.pos, w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s);
+  h->launches += 2;
   if (e != cudaSuccess) return e;
   if (full) mark(h, 3, s);
   return e;
@@ -448,9 +455,11 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   mark(h, 0, s);
   cudaError_t e = run_route(h, x, T, true, s);
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
-  h->launches += 1;
-  if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  if (!h->bf16) {  // the bf16 gate/up GEMM gathers z rows itself
+    e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
+    h->launches += 1;
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  }
   mark(h, 4, s);
   if (h->bf16) {
     TcParams p = {};
@@ -462,8 +471,11 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.b_rows_per_expert = 2 * h->m;
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
+    p.gather_perm = w.perm;
+    p.gather_k = h->K;
+    p.gather_rows = TK;
     p.status = w.status;
-    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
+    e = launch_tc_gemm(h->tm_zg.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 5, s);

@@ -28,54 +28,55 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 }
 
 // ---------------------------------------------------------------- top-K'
-// One warp per token.  Lane j holds experts e = 32 i + j (i < VPL).  A 64-bit
-// key (float key << 32 | ~e) makes one max-reduction pick the largest logit
-// and, among equal logits, the lower expert index.  K' rounds of a warp
-// butterfly max select the slots in order.  Gates: g_k = e^{s_k - s_0} /
+// One warp per token.  Lane j holds experts e = 32 i + j (i < VPL) as 32-bit
+// order-preserving keys of their logits.  Each of the K' rounds takes the
+// warp maximum of the keys (one REDUX), then the smallest expert index holding
+// that maximum (a second REDUX) -- so equal logits go to the lower index --
+// and removes exactly that entry.  Gates: g_k = e^{s_k - s_0} /
 // sum_j e^{s_j - s_0}, which equals softmax(s) at the selected experts
 // renormalised to sum to one (the softmax denominator cancels).
+// If `counts` is given ([N][n_chunks], zeroed), the kernel also builds the
+// per-chunk expert histogram of the dispatch (chunk = `chunk` tokens).
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int ld,
                                                    const float *__restrict__ bias, int T, int N,
                                                    int K, int32_t *__restrict__ ids,
-                                                   float *__restrict__ gates) {
+                                                   float *__restrict__ gates,
+                                                   int32_t *__restrict__ counts, int n_chunks,
+                                                   int chunk) {
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   const float *row = logits + static_cast<size_t>(t) * ld;
-  unsigned long long key[VPL];
+  uint32_t key[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = i * 32 + lane;
-    if (e < N) {
-      const float v = row[e] + (bias ? bias[e] : 0.0f);
-      key[i] = (static_cast<unsigned long long>(float_key(v)) << 32) |
-               static_cast<uint32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
-    } else {
-      key[i] = 0ull;
-    }
+    key[i] = e < N ? float_key(row[e] + (bias ? bias[e] : 0.0f)) : 0u;
   }
   int32_t *ids_row = ids + static_cast<size_t>(t) * K;
   float *g_row = gates + static_cast<size_t>(t) * K;
+  int32_t *my_counts = counts ? counts + t / chunk : nullptr;
   float s0 = 0.0f;
   for (int k = 0; k < K; ++k) {
-    unsigned long long best = key[0];
+    uint32_t m = key[0];
 #pragma unroll
-    for (int i = 1; i < VPL; ++i) best = key[i] > best ? key[i] : best;
+    for (int i = 1; i < VPL; ++i) m = max(m, key[i]);
+    const uint32_t wm = __reduce_max_sync(kFull, m);
+    uint32_t cand = 0xFFFFFFFFu;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const unsigned long long o = __shfl_xor_sync(kFull, best, off);
-      best = o > best ? o : best;
-    }
-    const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best & 0xFFFFFFFFull));
-    const float v = key_float(static_cast<uint32_t>(best >> 32));
+    for (int i = VPL - 1; i >= 0; --i)
+      if (key[i] == wm) cand = static_cast<uint32_t>(i * 32 + lane);
+    const uint32_t e = __reduce_min_sync(kFull, cand);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (static_cast<uint32_t>(i * 32 + lane) == e) key[i] = 0u;
+    const float v = key_float(wm);
     if (k == 0) s0 = v;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i)  // keys are unique: remove the winner by value
-      if (key[i] == best) key[i] = 0ull;
     if ((k & 31) == lane) {  // the same lane re-reads this slot below
-      ids_row[k] = e;
+      ids_row[k] = static_cast<int32_t>(e);
       g_row[k] = v;
+      if (my_counts) atomicAdd(my_counts + static_cast<size_t>(e) * n_chunks, 1);
     }
   }
   float sum = 0.0f;
@@ -86,20 +87,22 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
 }
 
 // ---------------------------------------------------------------- dispatch
-// Phase 1: per-chunk expert histogram (kDispatchChunk tokens per block).
+// Count matrix layout: counts[e][c] (expert-major), c = token chunk.
+// Phase 1 (when the top-K kernel did not count): per-chunk expert histogram.
 __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t *__restrict__ ids,
                                                              int T, int K, int N,
-                                                             int32_t *__restrict__ counts) {
+                                                             int32_t *__restrict__ counts,
+                                                             int n_chunks, int chunk) {
   extern __shared__ int32_t cnt[];  // [N]
   for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
-  const int t0 = blockIdx.x * kDispatchChunk;
-  const int tn = min(kDispatchChunk, T - t0);
+  const int t0 = blockIdx.x * chunk;
+  const int tn = min(chunk, T - t0);
   const int32_t *base = ids + static_cast<size_t>(t0) * K;
   for (int i = threadIdx.x; i < tn * K; i += blockDim.x) atomicAdd(&cnt[base[i]], 1);
   __syncthreads();
   for (int e = threadIdx.x; e < N; e += blockDim.x)
-    counts[static_cast<size_t>(blockIdx.x) * N + e] = cnt[e];
+    counts[static_cast<size_t>(e) * n_chunks + blockIdx.x] = cnt[e];
 }
 
 // Inclusive scan across a block of up to 1024 threads; returns the exclusive
@@ -130,32 +133,36 @@ __device__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
   return before;
 }
 
-// Phase 2 (one block of 1024 threads): per-expert exclusive scan over chunks
-// (in place), expert offsets, and the table of tile_m-row M-tiles.
+// Phase 2 (one block of 1024 threads): each warp scans the chunk counts of
+// its experts (in place: counts[e][c] becomes the number of pairs of expert e
+// in chunks before c); then the expert totals are scanned into offsets and
+// the table of tile_m-row M-tiles is written.
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
     int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
     TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles) {
   __shared__ int warp_sums[32];
-  const int e = threadIdx.x;  // N <= 1024
-  int tot = 0;
-  if (e < N) {
-    int c = 0;
-    for (; c + 8 <= n_chunks; c += 8) {
-      int v[8];
+  __shared__ int tot_s[1024];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int e = w; e < N; e += 32) {
+    int32_t *row = counts + static_cast<size_t>(e) * n_chunks;
+    int carry = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < n_chunks ? row[c] : 0;
+      int x = v;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = counts[static_cast<size_t>(c + j) * N + e];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        counts[static_cast<size_t>(c + j) * N + e] = tot;
-        tot += v[j];
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, off);
+        if (lane >= off) x += y;
       }
+      if (c < n_chunks) row[c] = carry + x - v;
+      carry += __shfl_sync(kFull, x, 31);
     }
-    for (; c < n_chunks; ++c) {
-      const int v = counts[static_cast<size_t>(c) * N + e];
-      counts[static_cast<size_t>(c) * N + e] = tot;
-      tot += v;
-    }
+    if (lane == 0) tot_s[e] = carry;
   }
+  __syncthreads();
+  const int e = threadIdx.x;  // N <= 1024
+  const int tot = e < N ? tot_s[e] : 0;
   int all = 0;
   const int off = block_exclusive_scan(tot, warp_sums, &all);
   const int mt = (tot + tile_m - 1) / tile_m;
@@ -181,22 +188,23 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
   }
 }
 
-// Phase 3: stable scatter.  Warp w of a block handles 32 consecutive tokens;
-// a per-warp bitmask per expert gives each (token, slot) its rank among the
+// Phase 3: stable scatter, one block per chunk, one warp per 32 tokens.  A
+// per-warp bitmask per expert gives each (token, slot) its rank among the
 // warp's tokens that chose the same expert (a token picks an expert at most
-// once), the per-warp counts are scanned across the block's warps, and the
+// once); the per-warp counts are scanned across the block's warps, and the
 // chunk's base comes from phase 2.  Tokens therefore land in ascending order.
 __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
     const int32_t *__restrict__ ids, int T, int K, int N, const int32_t *__restrict__ counts,
-    const int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ pos,
-    int32_t *__restrict__ row_expert) {
+    int n_chunks, int chunk, const int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+    int32_t *__restrict__ pos, int32_t *__restrict__ row_expert) {
   extern __shared__ uint32_t sm[];
-  uint32_t *mask = sm;                                        // [8][N]
-  int32_t *wbase = reinterpret_cast<int32_t *>(sm + 8 * N);  // [8][N]
-  for (int i = threadIdx.x; i < 8 * N; i += blockDim.x) mask[i] = 0u;
+  const int W = blockDim.x >> 5;
+  uint32_t *mask = sm;                                        // [W][N]
+  int32_t *wbase = reinterpret_cast<int32_t *>(sm + W * N);  // [W][N]
+  for (int i = threadIdx.x; i < W * N; i += blockDim.x) mask[i] = 0u;
   __syncthreads();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kDispatchChunk + threadIdx.x;
+  const int t = blockIdx.x * chunk + threadIdx.x;
   const bool valid = t < T;
   const int32_t *my_ids = ids + static_cast<size_t>(t) * K;
   if (valid)
@@ -204,8 +212,7 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
   __syncthreads();
   for (int e = threadIdx.x; e < N; e += blockDim.x) {
     int run = 0;
-#pragma unroll
-    for (int ww = 0; ww < 8; ++ww) {
+    for (int ww = 0; ww < W; ++ww) {
       wbase[ww * N + e] = run;
       run += __popc(mask[ww * N + e]);
     }
@@ -213,10 +220,10 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
   __syncthreads();
   if (!valid) return;
   const uint32_t lt = (1u << lane) - 1u;
-  const int32_t *cbase = counts + static_cast<size_t>(blockIdx.x) * N;
   for (int k = 0; k < K; ++k) {
     const int e = my_ids[k];
-    const int p = offsets[e] + cbase[e] + wbase[w * N + e] + __popc(mask[w * N + e] & lt);
+    const int p = offsets[e] + counts[static_cast<size_t>(e) * n_chunks + blockIdx.x] +
+                  wbase[w * N + e] + __popc(mask[w * N + e] & lt);
     const int flat = t * K + k;
     perm[p] = flat;
     pos[flat] = p;
@@ -312,28 +319,34 @@ __global__ void __launch_bounds__(256) combine_kernel(const Tio *__restrict__ O,
 }  // namespace
 
 cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, int N, int K,
-                        int32_t *ids, float *gates, cudaStream_t s) {
+                        int32_t *ids, float *gates, int32_t *counts, int chunk, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const int blocks = (T + 7) / 8;
   const int vpl = (N + 31) / 32;
-  if (vpl <= 1) topk_kernel<1><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
-  else if (vpl <= 2) topk_kernel<2><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
-  else if (vpl <= 4) topk_kernel<4><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
-  else if (vpl <= 8) topk_kernel<8><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
-  else if (vpl <= 16) topk_kernel<16><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
-  else if (vpl <= 32) topk_kernel<32><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates);
+  const int nc = dispatch_chunks(T, chunk);
+#define LMOE_TOPK(V)                                                                        \
+  topk_kernel<V><<<blocks, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates, counts, nc, \
+                                        chunk)
+  if (vpl <= 1) LMOE_TOPK(1);
+  else if (vpl <= 2) LMOE_TOPK(2);
+  else if (vpl <= 4) LMOE_TOPK(4);
+  else if (vpl <= 8) LMOE_TOPK(8);
+  else if (vpl <= 16) LMOE_TOPK(16);
+  else if (vpl <= 32) LMOE_TOPK(32);
   else return cudaErrorInvalidValue;
+#undef LMOE_TOPK
   return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,
-                            int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *row_expert,
-                            TileEntry *tiles, int32_t *n_tiles, int tile_m, int max_tiles,
-                            cudaStream_t s) {
-  if (N > 1024) return cudaErrorInvalidValue;
-  const int nc = dispatch_chunks(T);
-  if (nc > 0) {
-    dispatch_count_kernel<<<nc, 256, N * sizeof(int32_t), s>>>(ids, T, K, N, chunk_counts);
+                            int chunk, bool counts_ready, int32_t *offsets, int32_t *perm,
+                            int32_t *pos, int32_t *row_expert, TileEntry *tiles,
+                            int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s) {
+  if (N > 1024 || chunk % 32 || chunk < 32 || chunk > 256) return cudaErrorInvalidValue;
+  const int nc = dispatch_chunks(T, chunk);
+  if (nc > 0 && !counts_ready) {
+    dispatch_count_kernel<<<nc, 256, N * sizeof(int32_t), s>>>(ids, T, K, N, chunk_counts, nc,
+                                                               chunk);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -341,14 +354,15 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
                                           max_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || nc == 0) return e;
-  const size_t smem = 16 * static_cast<size_t>(N) * sizeof(uint32_t);
+  const int warps = chunk / 32;
+  const size_t smem = 2 * static_cast<size_t>(warps) * N * sizeof(uint32_t);
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(dispatch_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  dispatch_scatter_kernel<<<nc, 256, smem, s>>>(ids, T, K, N, chunk_counts, offsets, perm, pos,
-                                                row_expert);
+  dispatch_scatter_kernel<<<nc, 32 * warps, smem, s>>>(ids, T, K, N, chunk_counts, nc, chunk,
+                                                       offsets, perm, pos, row_expert);
   return cudaGetLastError();
 }
 

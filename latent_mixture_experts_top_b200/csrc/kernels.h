@@ -80,17 +80,11 @@ struct TcParams {
   __nv_bfloat16 *z; int ld_z;
   __nv_bfloat16 *out; int ld_out;   // H, O, y, or Ucat (+ column offset for shared)
   int out_col0;
-  // TC_EXPERT_GU: when gather_perm is set, A row r of a tile is row
-  // gather_perm[row0 + r] / gather_k of the A tensor (z), fetched with TMA
-  // gather4 (rows at or past gather_rows fetch row 0 and are masked).
-  const int32_t *gather_perm;
-  int gather_k, gather_rows;
   int32_t *status;
 };
 
 // Encodes a 2-D bf16 K-major tensor map (rows x cols, row stride in
-// elements) with a {64, box_rows} box and 128-byte swizzle (box_rows = 1 for
-// gather4 maps).  Host only.
+// elements) with a {64, box_rows} box and 128-byte swizzle.  Host only.
 int make_tmap_bf16(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
                    int64_t cols, int64_t row_stride_elems, int box_rows);
 

@@ -75,7 +75,7 @@ struct lmoe_layer {
   // the router/down GEMM and joined before the output GEMM.
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-  TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat, tm_zg;
+  TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
 };
 
 namespace {
@@ -248,7 +248,6 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   }
   if (h->bf16) {
     rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TK), h->l, h->l, kTileM);
-    if (rc == LMOE_OK) rc = make_map(&h->tm_zg, w.z, h->Tmax, h->l, h->l, 1);  // gather4
     if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, static_cast<int64_t>(TK), h->m, h->m, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_ucat, w.ucat, h->Tmax, h->ky, h->ky, kTileM);
     if (rc == LMOE_OK)
@@ -455,11 +454,9 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   mark(h, 0, s);
   cudaError_t e = run_route(h, x, T, true, s);
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  if (!h->bf16) {  // the bf16 gate/up GEMM gathers z rows itself
-    e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
-    h->launches += 1;
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  }
+  e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
+  h->launches += 1;
+  if (e != cudaSuccess) return LMOE_ERR_CUDA;
   mark(h, 4, s);
   if (h->bf16) {
     TcParams p = {};
@@ -471,11 +468,8 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.b_rows_per_expert = 2 * h->m;
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
-    p.gather_perm = w.perm;
-    p.gather_k = h->K;
-    p.gather_rows = TK;
     p.status = w.status;
-    e = launch_tc_gemm(h->tm_zg.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
+    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 5, s);

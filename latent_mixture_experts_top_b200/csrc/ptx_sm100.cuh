@@ -77,20 +77,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
       : "memory");
 }
 
-// 2-D gather of four rows (r0..r3), columns x .. x+box0, each row landing
-// 128 bytes after the previous one (the tensor map's box is one row high).
-// No multicast.
-__device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, uint64_t *bar,
-                                            int32_t x, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 // TMEM allocation: executed by one full warp; the TMEM base address is written
 // to *smem_dst.  ncols: power of two in [32, 512].

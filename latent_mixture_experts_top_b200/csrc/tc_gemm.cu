@@ -18,9 +18,6 @@
 // Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
 //               swizzle, into a 4-stage shared-memory ring (no multicast).
-//               For the expert gate/up GEMM the A rows are gathered from z
-//               by the dispatch permutation (tile::gather4, 4 rows per lane),
-//               so the permuted copy of z is never materialised.
 //   warp 1      TMEM owner and MMA issuer: one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into
 //               one of two 256-column fp32 accumulators in TMEM, and
@@ -205,47 +202,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // Lane 0 waits for free stages and loads B; A is a plain tile (lane 0) or,
-    // in gather mode, 32 gather4 copies of 4 rows each (one per lane).
-    const bool gather = p.gather_perm != nullptr;
-    int it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const Tile tl = decode_tile(p, t, m_tiles);
-      int32_t rows[4] = {0, 0, 0, 0};
-      if (gather) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = tl.a_row + 4 * lane + j;
-          rows[j] = r < p.gather_rows ? p.gather_perm[r] / p.gather_k : 0;
-        }
-      }
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        int got = 1;
-        if (lane == 0) got = ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag) ? 1 : 0;
-        got = __shfl_sync(0xFFFFFFFFu, got, 0);
-        if (!got) {
-          if (lane == 0) record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
-          ok = false;
-          break;
-        }
-        if (lane == 0) ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
-        __syncwarp();
-        if (gather) {
-          ptx::tma_gather4(smA + s * A_BYTES + lane * 4 * (TKB * 2), &tmA, &ctl->full[s],
-                           kb * TKB, rows[0], rows[1], rows[2], rows[3]);
-        } else if (lane == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, t, m_tiles);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
+            record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
           ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
+          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
         }
-        if (lane == 0) ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
       }
-    }
-    if (!ok && lane == 0) {  // let every copy still in flight land before the CTA exits
-      for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-        if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
-          record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
+      if (!ok) {  // let every copy still in flight land before the CTA exits
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
+            record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

@@ -32,7 +32,7 @@ constexpr int kMaxTiles = kMaxPairs / kTileRows + kMaxExperts + 1;
 
 constexpr size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 constexpr size_t kCountsBytes =
-    round256(static_cast<size_t>((kMaxTokens + kChunk - 1) / kChunk) *
+    round256(static_cast<size_t>(((kMaxTokens + kChunk - 1) / kChunk + 3) / 4 * 4) *
              kMaxExperts * sizeof(int32_t));
 constexpr size_t kPosBytes = round256(static_cast<size_t>(kMaxPairs) * sizeof(int32_t));
 constexpr size_t kTilesBytes = round256(static_cast<size_t>(kMaxTiles) * sizeof(TileEntry));

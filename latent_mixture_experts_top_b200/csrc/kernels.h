@@ -15,18 +15,23 @@ struct TileEntry {
 
 // ---- routing (route_kernels.cu)
 // ids/gates from fp32 logits [T][ld] (+ bias [N]); one warp per token.  If
-// counts is non-null ([N][dispatch_chunks(T, chunk)], zeroed beforehand) the
-// kernel also accumulates the dispatch's per-chunk expert histogram.
+// counts is non-null the
+// kernel also accumulates the dispatch's per-chunk expert histogram (zeroed
+// beforehand, dispatch_count_elems(T, chunk, N) ints).
 cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, int N, int K,
                         int32_t *ids, float *gates, int32_t *counts, int chunk, cudaStream_t s);
 
 // Tokens per dispatch chunk on the forward path, and the chunk count.
 constexpr int kDispatchChunk = 64;
 inline int dispatch_chunks(int T, int chunk) { return (T + chunk - 1) / chunk; }
+// Elements of the [N][chunks] count matrix (rows padded to a multiple of 4).
+inline size_t dispatch_count_elems(int T, int chunk, int N) {
+  return static_cast<size_t>((dispatch_chunks(T, chunk) + 3) & ~3) * N;
+}
 
 // Histogram (unless counts_ready) -> exclusive scan -> stable scatter.  The
-// count matrix chunk_counts is [N][dispatch_chunks(T, chunk)] (chunk: a
-// multiple of 32, at most 256).  Writes offsets [N+1], perm / pos /
+// count matrix chunk_counts holds dispatch_count_elems(T, chunk, N) ints
+// (chunk: a multiple of 32, at most 256).  Writes offsets [N+1], perm / pos /
 // row_expert [T*K], and the M-tile table (tile_m rows per tile; capacity
 // max_tiles entries) plus its length in *n_tiles.
 cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,

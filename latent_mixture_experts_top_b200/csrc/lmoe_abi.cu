@@ -210,8 +210,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   h->nx_rows = h->n_pad + h->l_pad + 2 * h->ns * h->ms;
   Workspace &w = h->ws;
   bool ok = dalloc(&w.logits, T * N * 4) && dalloc(&w.ids, TK * 4) && dalloc(&w.gates, TK * 4) &&
-            dalloc(&w.chunk_counts,
-                   static_cast<size_t>(dispatch_chunks(h->Tmax, kDispatchChunk)) * N * 4) &&
+            dalloc(&w.chunk_counts, dispatch_count_elems(h->Tmax, kDispatchChunk, h->N) * 4) &&
             dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TK * 4) && dalloc(&w.pos, TK * 4) &&
             dalloc(&w.row_expert, TK * 4) &&
             dalloc(&w.tiles, static_cast<size_t>(h->max_tiles) * sizeof(TileEntry)) &&
@@ -405,8 +404,7 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
   if (e != cudaSuccess) return e;
   if (full) mark(h, 1, s);
   // top-K' also builds the dispatch histogram (into the zeroed count matrix)
-  e = cudaMemsetAsync(w.chunk_counts, 0,
-                      static_cast<size_t>(dispatch_chunks(T, kDispatchChunk)) * h->N * 4, s);
+  e = cudaMemsetAsync(w.chunk_counts, 0, dispatch_count_elems(T, kDispatchChunk, h->N) * 4, s);
   if (e != cudaSuccess) return e;
   e = launch_topk(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates, w.chunk_counts,
                   kDispatchChunk, s);

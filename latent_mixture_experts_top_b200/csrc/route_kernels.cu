@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
     if ((k & 31) == lane) {  // the same lane re-reads this slot below
       ids_row[k] = static_cast<int32_t>(e);
       g_row[k] = v;
-      if (my_counts) atomicAdd(my_counts + static_cast<size_t>(e) * n_chunks, 1);
+      if (my_counts) atomicAdd(my_counts + static_cast<size_t>(e) * ((n_chunks + 3) & ~3), 1);
     }
   }
   float sum = 0.0f;
@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
 }
 
 // ---------------------------------------------------------------- dispatch
-// Count matrix layout: counts[e][c] (expert-major), c = token chunk.
+// Count matrix layout: counts[e][c] (expert-major), c = token chunk, row
+// stride n_chunks rounded up to a multiple of 4 (16-byte rows).
 // Phase 1 (when the top-K kernel did not count): per-chunk expert histogram.
 __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t *__restrict__ ids,
                                                              int T, int K, int N,
@@ -101,8 +102,9 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t *__re
   const int32_t *base = ids + static_cast<size_t>(t0) * K;
   for (int i = threadIdx.x; i < tn * K; i += blockDim.x) atomicAdd(&cnt[base[i]], 1);
   __syncthreads();
+  const int ncp = (n_chunks + 3) & ~3;
   for (int e = threadIdx.x; e < N; e += blockDim.x)
-    counts[static_cast<size_t>(e) * n_chunks + blockIdx.x] = cnt[e];
+    counts[static_cast<size_t>(e) * ncp + blockIdx.x] = cnt[e];
 }
 
 // Inclusive scan across a block of up to 1024 threads; returns the exclusive
@@ -133,36 +135,39 @@ __device__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
   return before;
 }
 
-// Phase 2 (one block of 1024 threads): each warp scans the chunk counts of
-// its experts (in place: counts[e][c] becomes the number of pairs of expert e
+// Phase 2 (one block of 1024 threads): each thread scans the chunk counts of
+// its expert (in place: counts[e][c] becomes the number of pairs of expert e
 // in chunks before c); then the expert totals are scanned into offsets and
 // the table of tile_m-row M-tiles is written.
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
     int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
     TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles) {
   __shared__ int warp_sums[32];
-  __shared__ int tot_s[1024];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int e = w; e < N; e += 32) {
-    int32_t *row = counts + static_cast<size_t>(e) * n_chunks;
-    int carry = 0;
-    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < n_chunks ? row[c] : 0;
-      int x = v;
+  const int e = threadIdx.x;  // N <= 1024: one thread per expert row
+  int tot = 0;
+  if (e < N) {
+    // The row is contiguous (row stride n_chunks rounded up to 4): 16-byte
+    // loads, eight in flight at a time.
+    const int ncp = (n_chunks + 3) & ~3;
+    int4 *row = reinterpret_cast<int4 *>(counts + static_cast<size_t>(e) * ncp);
+    const int nv = ncp / 4;
+    for (int v0 = 0; v0 < nv; v0 += 8) {
+      int4 q[8];
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(kFull, x, off);
-        if (lane >= off) x += y;
+      for (int j = 0; j < 8; ++j) q[j] = v0 + j < nv ? row[v0 + j] : make_int4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (v0 + j >= nv) break;
+        const int c = 4 * (v0 + j);
+        int4 o;
+        o.x = tot; tot += c + 0 < n_chunks ? q[j].x : 0;
+        o.y = tot; tot += c + 1 < n_chunks ? q[j].y : 0;
+        o.z = tot; tot += c + 2 < n_chunks ? q[j].z : 0;
+        o.w = tot; tot += c + 3 < n_chunks ? q[j].w : 0;
+        row[v0 + j] = o;
       }
-      if (c < n_chunks) row[c] = carry + x - v;
-      carry += __shfl_sync(kFull, x, 31);
     }
-    if (lane == 0) tot_s[e] = carry;
   }
-  __syncthreads();
-  const int e = threadIdx.x;  // N <= 1024
-  const int tot = e < N ? tot_s[e] : 0;
   int all = 0;
   const int off = block_exclusive_scan(tot, warp_sums, &all);
   const int mt = (tot + tile_m - 1) / tile_m;
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
   const uint32_t lt = (1u << lane) - 1u;
   for (int k = 0; k < K; ++k) {
     const int e = my_ids[k];
-    const int p = offsets[e] + counts[static_cast<size_t>(e) * n_chunks + blockIdx.x] +
+    const int p = offsets[e] + counts[static_cast<size_t>(e) * ((n_chunks + 3) & ~3) + blockIdx.x] +
                   wbase[w * N + e] + __popc(mask[w * N + e] & lt);
     const int flat = t * K + k;
     perm[p] = flat;
@@ -305,11 +310,20 @@ __global__ void __launch_bounds__(256) combine_kernel(const Tio *__restrict__ O,
       const int my_p = kk < K ? pos[static_cast<size_t>(t) * K + kk] : 0;
       const float my_g = kk < K ? gates[static_cast<size_t>(t) * K + kk] : 0.0f;
       const int kn = min(32, K - k0);
-      for (int k = 0; k < kn; ++k) {
-        const int p = __shfl_sync(kFull, my_p, k);
-        const float g = __shfl_sync(kFull, my_g, k);
-        const uint4 raw = *reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l + vi * V);
-        accum_vec<Tio>(acc, raw, g);
+      // Eight slots' loads in flight, then accumulated in slot order.
+      for (int k1 = 0; k1 < kn; k1 += 8) {
+        uint4 raw[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int p = __shfl_sync(kFull, my_p, (k1 + j) & 31);
+          if (k1 + j < kn)
+            raw[j] = __ldcs(reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l + vi * V));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float g = __shfl_sync(kFull, my_g, (k1 + j) & 31);
+          if (k1 + j < kn) accum_vec<Tio>(acc, raw[j], g);
+        }
       }
     }
     *reinterpret_cast<uint4 *>(u + static_cast<size_t>(t) * ldu + vi * V) = pack_vec<Tio>(acc);

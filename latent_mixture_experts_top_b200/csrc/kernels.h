@@ -86,8 +86,8 @@ struct TcParams {
   __nv_bfloat16 *z; int ld_z;
   __nv_bfloat16 *out; int ld_out;   // H, O, y, or Ucat (+ column offset for shared)
   int out_col0;
-  // TC_EXPERT_FUSED: the gate/up tiles of each M-tile, and `group` M-tiles
-  // later the down tiles of that M-tile (second tensor-map pair, Kdim2,
+  // TC_EXPERT_FUSED: the gate/up tiles of a group of `group` M-tiles, then
+  // the down tiles of the previous group (second tensor-map pair, Kdim2,
   // n_tiles_n2, b_rows_per_expert2, out2).  A down tile starts once done[mt]
   // reaches n_tiles_n * (epilogue warps): every gate/up tile of its M-tile has
   // stored its H rows.  done[] is zeroed before the launch.

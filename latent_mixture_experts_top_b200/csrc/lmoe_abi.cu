@@ -476,8 +476,7 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.b_rows_per_expert2 = h->l;
     p.out2 = static_cast<__nv_bfloat16 *>(w.O);
     p.ld_out2 = h->l;
-    // lag: about three waves of tiles between an M-tile's gate/up and down tiles
-    p.group = (3 * h->num_sms + p.n_tiles_n + p.n_tiles_n2 - 1) / (p.n_tiles_n + p.n_tiles_n2);
+    p.group = h->num_sms / p.n_tiles_n > 0 ? h->num_sms / p.n_tiles_n : 1;
     p.done = w.tile_done;
     p.tiles = w.tiles;
     p.n_mtiles = w.n_tiles;

@@ -8,12 +8,12 @@
 //   TC_EXPERT_GU   grouped: permuted z rows of expert e times its gate/up
 //                  rows (interleaved in blocks of 128) -> SwiGLU -> H (bf16).
 //   TC_EXPERT_DOWN grouped: H times W_o[e] -> expert output O (bf16).
-//   TC_EXPERT_FUSED the two grouped modes in one persistent launch: the down
-//                  tiles of an M-tile follow its gate/up tiles with a lag of
-//                  a few waves, so that H is read back while it is still in
-//                  L2 and the down tiles' memory traffic overlaps gate/up
-//                  MMAs.  A down tile waits (bounded) on a per-M-tile
-//                  counter that the gate/up epilogues release.
+//   TC_EXPERT_FUSED the two grouped modes in one persistent launch: gate/up
+//                  tiles of a group of M-tiles, then the down tiles of the
+//                  previous group, so that H is read back while it is still
+//                  in L2 and the down tiles' memory traffic overlaps the
+//                  gate/up tiles' MMAs.  A down tile waits (bounded) on a
+//                  per-M-tile counter that the gate/up epilogues release.
 //   TC_OUT         [u | shared hidden] times [W_up | S_o] -> y (bf16).
 //
 // Sources of the maths: "LatentMoE Explained", Figure 3 (router reads the
@@ -76,29 +76,25 @@ struct Tile {
   int nkb;     // K-blocks of this tile
 };
 
-// Order of the fused expert launch, by M-tile "units": unit u holds the
-// gate/up tiles of M-tile u (if u < M) followed by the down tiles of M-tile
-// u - D (if 0 <= u - D < M).  The lag D (in M-tiles) keeps a down tile
-// several waves of tiles behind the gate/up tiles it reads, so its wait is
-// normally already satisfied, while the H rows in between (D M-tiles) stay in
-// L2.  Every dependency points to an earlier tile.
+// Order of the fused expert launch: block 0 = gate/up tiles of group 0;
+// block b (1..n-1) = gate/up tiles of group b, then down tiles of group b-1;
+// block n = down tiles of group n-1.  Groups hold `group` M-tiles (the last
+// one the remainder); a down tile's gate/up tiles always come earlier.
 struct FusedPlan {
-  int M, D, NG, ND, p1, p2, total;
+  int n, G, c_last, NG, ND, s1, mid, sn, total;
 };
 __device__ __forceinline__ FusedPlan fused_plan(const TcParams &p, int M) {
   FusedPlan f;
-  f.M = M;
-  f.D = p.group;  // lag in M-tiles
+  f.G = p.group;
   f.NG = p.n_tiles_n;
   f.ND = p.n_tiles_n2;
-  if (M <= f.D) {  // all gate/up tiles, then all down tiles
-    f.p1 = M * f.NG;
-    f.p2 = f.p1;
-  } else {
-    f.p1 = f.D * f.NG;
-    f.p2 = f.p1 + (M - f.D) * (f.NG + f.ND);
-  }
-  f.total = M * (f.NG + f.ND);
+  f.n = (M + f.G - 1) / f.G;
+  f.c_last = M - f.G * (f.n - 1);
+  const int c0 = f.n > 1 ? f.G : f.c_last;
+  f.s1 = c0 * f.NG;
+  f.mid = f.G * (f.NG + f.ND);
+  f.sn = f.n > 1 ? f.s1 + (f.n - 2) * f.mid + f.c_last * f.NG + f.G * f.ND : f.s1;
+  f.total = M > 0 ? f.sn + f.c_last * f.ND : 0;
   return f;
 }
 
@@ -118,25 +114,28 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
   }
   int mt, n;
   if (p.mode == TC_EXPERT_FUSED) {
-    if (t < f.p1) {                      // leading gate/up-only units
+    if (t < f.s1) {
       mt = t / f.NG;
       n = t % f.NG;
-    } else if (t < f.p2) {               // units with both parts
-      const int r = t - f.p1, w = r % (f.NG + f.ND);
-      const int u = f.D + r / (f.NG + f.ND);
-      if (w < f.NG) {
-        mt = u;
-        n = w;
-      } else {
-        mt = u - f.D;
-        n = w - f.NG;
-        tl.second = 1;
-      }
-    } else {                             // trailing down-only units
-      const int r = t - f.p2;
-      mt = (f.M > f.D ? f.M - f.D : 0) + r / f.ND;
+    } else if (t >= f.sn) {
+      const int r = t - f.sn;
+      mt = f.G * (f.n - 1) + r / f.ND;
       n = r % f.ND;
       tl.second = 1;
+    } else {
+      int b = 1 + (t - f.s1) / f.mid;
+      if (b > f.n - 1) b = f.n - 1;
+      int r = t - (f.s1 + (b - 1) * f.mid);
+      const int gu = (b < f.n - 1 ? f.G : f.c_last) * f.NG;
+      if (r < gu) {
+        mt = f.G * b + r / f.NG;
+        n = r % f.NG;
+      } else {
+        r -= gu;
+        mt = f.G * (b - 1) + r / f.ND;
+        n = r % f.ND;
+        tl.second = 1;
+      }
     }
   } else {
     mt = t / p.n_tiles_n;  // consecutive CTAs share A

@@ -67,7 +67,6 @@ enum TcMode : int {
   TC_EXPERT_GU = 1, // grouped: permuted z x W_gu[e] -> SwiGLU -> H
   TC_EXPERT_DOWN = 2,  // grouped: H x W_o[e] -> O (bf16)
   TC_OUT = 3,       // [u | shared hidden] x W_y -> y (bf16)
-  TC_EXPERT_FUSED = 4,  // TC_EXPERT_GU and TC_EXPERT_DOWN tiles in one persistent launch
 };
 
 struct TcParams {
@@ -86,15 +85,6 @@ struct TcParams {
   __nv_bfloat16 *z; int ld_z;
   __nv_bfloat16 *out; int ld_out;   // H, O, y, or Ucat (+ column offset for shared)
   int out_col0;
-  // TC_EXPERT_FUSED: the gate/up tiles of a group of `group` M-tiles, then
-  // the down tiles of the previous group (second tensor-map pair, Kdim2,
-  // n_tiles_n2, b_rows_per_expert2, out2).  A down tile starts once done[mt]
-  // reaches n_tiles_n * (epilogue warps): every gate/up tile of its M-tile has
-  // stored its H rows.  done[] is zeroed before the launch.
-  int Kdim2, n_tiles_n2, b_rows_per_expert2;
-  __nv_bfloat16 *out2; int ld_out2;
-  int group;
-  int32_t *done;
   int32_t *status;
 };
 
@@ -103,9 +93,7 @@ struct TcParams {
 int make_tmap_bf16(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
                    int64_t cols, int64_t row_stride_elems, int box_rows);
 
-// tmapA2 / tmapB2: the second operand pair (TC_EXPERT_FUSED), else NULL.
-cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const void *tmapA2,
-                           const void *tmapB2, const TcParams &p, int num_sms, int max_ctas,
-                           cudaStream_t s);
+cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p,
+                           int num_sms, int max_ctas, cudaStream_t s);
 
 }  // namespace lmoe

@@ -37,7 +37,6 @@ struct Workspace {
   int32_t *perm = nullptr, *pos = nullptr, *row_expert = nullptr;
   TileEntry *tiles = nullptr;
   int32_t *n_tiles = nullptr;
-  int32_t *tile_done = nullptr;  // per M-tile: gate/up epilogue warps finished (fused GEMM)
   void *z = nullptr, *zp = nullptr, *H = nullptr, *O = nullptr, *ucat = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
   int32_t *status = nullptr;
@@ -107,7 +106,7 @@ void free_all(lmoe_layer *h) {
   void *ptrs[] = {h->w_router, h->b_router, h->w_x, h->w_down, h->w_gu, h->w_gate, h->w_upx,
                   h->w_out, h->s_gate, h->s_up, h->w_y, h->ws.logits, h->ws.ids, h->ws.gates,
                   h->ws.chunk_counts, h->ws.offsets, h->ws.perm, h->ws.pos, h->ws.row_expert,
-                  h->ws.tiles, h->ws.n_tiles, h->ws.tile_done, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
+                  h->ws.tiles, h->ws.n_tiles, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
                   h->ws.x_stage, h->ws.y_stage, h->ws.status};
   for (void *p : ptrs)
     if (p) cudaFree(p);
@@ -215,9 +214,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
             dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TK * 4) && dalloc(&w.pos, TK * 4) &&
             dalloc(&w.row_expert, TK * 4) &&
             dalloc(&w.tiles, static_cast<size_t>(h->max_tiles) * sizeof(TileEntry)) &&
-            dalloc(&w.n_tiles, 16) &&
-            dalloc(&w.tile_done, static_cast<size_t>(h->max_tiles) * sizeof(int32_t)) &&
-            dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
+            dalloc(&w.n_tiles, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
             dalloc(&w.H, TK * m * es) && dalloc(&w.O, TK * l * es) &&
             dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
             dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16);
@@ -371,8 +368,7 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.out_col0 = h->l;
     p.status = w.status;
     const int m_tiles = (T + kTileM - 1) / kTileM;
-    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, nullptr, nullptr, p, h->num_sms,
-                       m_tiles * p.n_tiles_n, s);
+    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, m_tiles * p.n_tiles_n, s);
     h->launches += 1;
     const int shared_tiles_n = (h->nx_rows - h->n_pad - h->l_pad) / kTileN;
     if (e == cudaSuccess && full && shared_tiles_n > 0) {
@@ -384,8 +380,8 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       e = cudaEventRecord(h->ev_fork, s);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
       if (e == cudaSuccess)
-        e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, nullptr, nullptr, q, h->num_sms,
-                           m_tiles * shared_tiles_n, h->side);
+        e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, q, h->num_sms, m_tiles * shared_tiles_n,
+                           h->side);
       if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
       h->launches += 1;
     }
@@ -461,31 +457,29 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
   mark(h, 4, s);
   if (h->bf16) {
-    // Expert gate/up (SwiGLU -> H) and down (H -> O) in one persistent launch.
-    e = cudaMemsetAsync(w.tile_done, 0, static_cast<size_t>(h->max_tiles) * sizeof(int32_t), s);
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
     TcParams p = {};
-    p.mode = TC_EXPERT_FUSED;
+    p.mode = TC_EXPERT_GU;
     p.Kdim = h->l;
     p.n_tiles_n = 2 * h->m / kTileN;
+    p.tiles = w.tiles;
+    p.n_mtiles = w.n_tiles;
     p.b_rows_per_expert = 2 * h->m;
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
-    p.Kdim2 = h->m;
-    p.n_tiles_n2 = (h->l + kTileN - 1) / kTileN;
-    p.b_rows_per_expert2 = h->l;
-    p.out2 = static_cast<__nv_bfloat16 *>(w.O);
-    p.ld_out2 = h->l;
-    p.group = h->num_sms / p.n_tiles_n > 0 ? h->num_sms / p.n_tiles_n : 1;
-    p.done = w.tile_done;
-    p.tiles = w.tiles;
-    p.n_mtiles = w.n_tiles;
     p.status = w.status;
-    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, h->tm_h.bytes, h->tm_wo.bytes, p,
-                       h->num_sms, h->num_sms, s);
+    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 5, s);
+    p.mode = TC_EXPERT_DOWN;
+    p.Kdim = h->m;
+    p.n_tiles_n = (h->l + kTileN - 1) / kTileN;
+    p.b_rows_per_expert = h->l;
+    p.out = static_cast<__nv_bfloat16 *>(w.O);
+    p.ld_out = h->l;
+    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, p, h->num_sms, h->num_sms, s);
+    h->launches += 1;
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 6, s);
     e = launch_combine(w.O, w.pos, w.gates, T, h->K, h->l, w.ucat, h->ky, true, s);
     h->launches += 1;
@@ -502,8 +496,7 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     q.ld_out = h->d;
     q.status = w.status;
     const int tiles = (T + kTileM - 1) / kTileM * q.n_tiles_n;
-    e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, nullptr, nullptr, q, h->num_sms, tiles,
-                       s);
+    e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, q, h->num_sms, tiles, s);
     h->launches += 1;
   } else {
     float *zpf = static_cast<float *>(w.zp);

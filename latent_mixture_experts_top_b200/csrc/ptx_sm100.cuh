@@ -77,20 +77,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
       : "memory");
 }
 
-// Orders this thread's generic-proxy global accesses with its async-proxy
-// (TMA) accesses.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void red_release_gpu_add(int32_t *p, int v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 // TMEM allocation: executed by one full warp; the TMEM base address is written
 // to *smem_dst.  ncols: power of two in [32, 512].

@@ -8,12 +8,6 @@
 //   TC_EXPERT_GU   grouped: permuted z rows of expert e times its gate/up
 //                  rows (interleaved in blocks of 128) -> SwiGLU -> H (bf16).
 //   TC_EXPERT_DOWN grouped: H times W_o[e] -> expert output O (bf16).
-//   TC_EXPERT_FUSED the two grouped modes in one persistent launch: gate/up
-//                  tiles of a group of M-tiles, then the down tiles of the
-//                  previous group, so that H is read back while it is still
-//                  in L2 and the down tiles' memory traffic overlaps the
-//                  gate/up tiles' MMAs.  A down tile waits (bounded) on a
-//                  per-M-tile counter that the gate/up epilogues release.
 //   TC_OUT         [u | shared hidden] times [W_up | S_o] -> y (bf16).
 //
 // Sources of the maths: "LatentMoE Explained", Figure 3 (router reads the
@@ -71,86 +65,24 @@ constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + size
 
 struct Tile {
   int a_row, b_row, n_tile, row_hi;
-  int second;  // TC_EXPERT_FUSED: 0 gate/up tile, 1 down tile
-  int mt;      // grouped modes: M-tile index
-  int nkb;     // K-blocks of this tile
 };
 
-// Order of the fused expert launch: block 0 = gate/up tiles of group 0;
-// block b (1..n-1) = gate/up tiles of group b, then down tiles of group b-1;
-// block n = down tiles of group n-1.  Groups hold `group` M-tiles (the last
-// one the remainder); a down tile's gate/up tiles always come earlier.
-struct FusedPlan {
-  int n, G, c_last, NG, ND, s1, mid, sn, total;
-};
-__device__ __forceinline__ FusedPlan fused_plan(const TcParams &p, int M) {
-  FusedPlan f;
-  f.G = p.group;
-  f.NG = p.n_tiles_n;
-  f.ND = p.n_tiles_n2;
-  f.n = (M + f.G - 1) / f.G;
-  f.c_last = M - f.G * (f.n - 1);
-  const int c0 = f.n > 1 ? f.G : f.c_last;
-  f.s1 = c0 * f.NG;
-  f.mid = f.G * (f.NG + f.ND);
-  f.sn = f.n > 1 ? f.s1 + (f.n - 2) * f.mid + f.c_last * f.NG + f.G * f.ND : f.s1;
-  f.total = M > 0 ? f.sn + f.c_last * f.ND : 0;
-  return f;
-}
-
-__device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles,
-                                            const FusedPlan &f) {
+__device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles) {
   Tile tl;
-  tl.second = 0;
-  tl.mt = 0;
-  tl.nkb = p.Kdim / TKB;
   if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
     const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
     tl.a_row = m * TM;
     tl.b_row = n * TN;
     tl.n_tile = n;
     tl.row_hi = p.M;
-    return tl;
-  }
-  int mt, n;
-  if (p.mode == TC_EXPERT_FUSED) {
-    if (t < f.s1) {
-      mt = t / f.NG;
-      n = t % f.NG;
-    } else if (t >= f.sn) {
-      const int r = t - f.sn;
-      mt = f.G * (f.n - 1) + r / f.ND;
-      n = r % f.ND;
-      tl.second = 1;
-    } else {
-      int b = 1 + (t - f.s1) / f.mid;
-      if (b > f.n - 1) b = f.n - 1;
-      int r = t - (f.s1 + (b - 1) * f.mid);
-      const int gu = (b < f.n - 1 ? f.G : f.c_last) * f.NG;
-      if (r < gu) {
-        mt = f.G * b + r / f.NG;
-        n = r % f.NG;
-      } else {
-        r -= gu;
-        mt = f.G * (b - 1) + r / f.ND;
-        n = r % f.ND;
-        tl.second = 1;
-      }
-    }
   } else {
-    mt = t / p.n_tiles_n;  // consecutive CTAs share A
-    n = t % p.n_tiles_n;
-    tl.second = p.mode == TC_EXPERT_DOWN;
+    const int mt = t / p.n_tiles_n, n = t % p.n_tiles_n;  // consecutive CTAs share A
+    const TileEntry te = p.tiles[mt];
+    tl.a_row = te.row0;
+    tl.b_row = te.expert * p.b_rows_per_expert + n * TN;
+    tl.n_tile = n;
+    tl.row_hi = te.row_end;
   }
-  const TileEntry te = p.tiles[mt];
-  const bool down = p.mode == TC_EXPERT_DOWN || (p.mode == TC_EXPERT_FUSED && tl.second);
-  tl.a_row = te.row0;
-  tl.b_row = te.expert * (p.mode == TC_EXPERT_FUSED && down ? p.b_rows_per_expert2
-                                                            : p.b_rows_per_expert) + n * TN;
-  tl.n_tile = n;
-  tl.row_hi = te.row_end;
-  tl.mt = mt;
-  if (p.mode == TC_EXPERT_FUSED && down) tl.nkb = p.Kdim2 / TKB;
   return tl;
 }
 
@@ -226,8 +158,7 @@ __device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bflo
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmA2,
-                   const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
+                   const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -238,15 +169,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const bool fused = p.mode == TC_EXPERT_FUSED;
   const bool grouped = (p.mode == TC_EXPERT_GU || p.mode == TC_EXPERT_DOWN);
-  const int m_tiles = (grouped || fused) ? 0 : (p.M + TM - 1) / TM;
-  const FusedPlan plan = fused_plan(p, fused ? *p.n_mtiles : 0);
-  const int total = fused ? plan.total
-                          : (grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles * p.n_tiles_n);
-  // A down tile's H rows are complete once all gate/up epilogue warps of its
-  // M-tile have published them.
-  const int dep_target = p.n_tiles_n * NUM_EPI_WARPS;
+  const int m_tiles = grouped ? 0 : (p.M + TM - 1) / TM;
+  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles * p.n_tiles_n;
+  const int nkb = p.Kdim / TKB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -264,10 +190,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB);
-    if (fused) {
-      ptx::prefetch_tmap(&tmA2);
-      ptx::prefetch_tmap(&tmB2);
-    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(&ctl->tmem_base, TMEM_COLS);
@@ -284,29 +206,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(p, t, m_tiles, plan);
-        const bool second = fused && tl.second;
-        if (second) {  // wait (bounded) until this M-tile's H rows are published
-          const int32_t *flag = p.done + tl.mt;
-          if (ptx::ld_acquire_gpu(flag) < dep_target) {
-            const unsigned long long t0 = globaltimer_ns();
-            while (ptx::ld_acquire_gpu(flag) < dep_target) {
-              if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
-                ok = false;
-                break;
-              }
-              __nanosleep(64);
-            }
-            if (!ok) {
-              record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
-              break;
-            }
-          }
-          ptx::fence_proxy_async_global();  // H was written by generic stores
-        }
-        const void *ta = second ? static_cast<const void *>(&tmA2) : static_cast<const void *>(&tmA);
-        const void *tb = second ? static_cast<const void *>(&tmB2) : static_cast<const void *>(&tmB);
-        for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
+        const Tile tl = decode_tile(p, t, m_tiles);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
@@ -315,8 +216,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
-          ptx::tma_load_2d(smA + s * A_BYTES, ta, &ctl->full[s], kb * TKB, tl.a_row);
-          ptx::tma_load_2d(smB + s * B_BYTES, tb, &ctl->full[s], kb * TKB, tl.b_row);
+          ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
+          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
         }
       }
       if (!ok) {  // let every copy still in flight land before the CTA exits
@@ -340,7 +241,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * TN;
-        const int nkb = decode_tile(p, t, m_tiles, plan).nkb;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -386,7 +286,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      const Tile tl = decode_tile(p, t, m_tiles, plan);
+      const Tile tl = decode_tile(p, t, m_tiles);
       const int row = tl.a_row + row_in_tile;
       const bool valid = row < tl.row_hi;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
@@ -407,17 +307,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         case TC_EXPERT_GU:
           epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
           break;
-        case TC_EXPERT_FUSED:
-          if (!tl.second) {
-            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
-            // Publish this warp's H rows for the down tiles (any SM, read by TMA).
-            ptx::fence_proxy_async_global();
-            __threadfence();
-          } else {
-            epi_plain<false>(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2, col0,
-                             p.ld_out2, half);
-          }
-          break;
         default:  // TC_EXPERT_DOWN, TC_OUT
           epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
                            p.ld_out, half);
@@ -425,10 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(&ctl->acc_empty[acc]);
-        if (fused && !tl.second) ptx::red_release_gpu_add(p.done + tl.mt, 1);
-      }
+      if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
     }
   }
 
@@ -478,9 +364,8 @@ int make_tmap_bf16(void *tmap_out, const void *base, int64_t rows, int64_t cols,
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
-cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const void *tmapA2,
-                           const void *tmapB2, const TcParams &p, int num_sms, int max_ctas,
-                           cudaStream_t s) {
+cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p, int num_sms,
+                           int max_ctas, cudaStream_t s) {
   static int attr_done = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -491,17 +376,12 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const void *tma
     attr_done = dev;
   }
   if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
-  if (p.mode == TC_EXPERT_FUSED &&
-      (!tmapA2 || !tmapB2 || !p.done || p.group < 1 || p.Kdim2 % TKB || p.Kdim2 <= 0))
-    return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
-  CUtensorMap a, b, a2, b2;
+  CUtensorMap a, b;
   memcpy(&a, tmapA, sizeof(a));
   memcpy(&b, tmapB, sizeof(b));
-  memcpy(&a2, tmapA2 ? tmapA2 : tmapA, sizeof(a2));
-  memcpy(&b2, tmapB2 ? tmapB2 : tmapB, sizeof(b2));
-  tc_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, a2, b2, p);
+  tc_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
   return cudaGetLastError();
 }
 

@@ -86,14 +86,15 @@ def stage_work(cfg):
     """Algorithmic FLOPs (tensor stages) or bytes (memory stages) per launch.
 
     Tensor stages count 2 flops per multiply-add of the layer's definition
-    (no padding, no masked rows).  Memory stages count the bytes the step must
+    (no padding, no masked rows).  The shared experts' gate/up GEMM overlaps
+    stages 1-3 on a side stream and is not a stage of its own.  Memory stages count the bytes the step must
     read and write once (bf16 activations, int32 indices, fp32 logits/gates).
     """
     T, d, l, m, N, K = cfg.T, cfg.d, cfg.l, cfg.m, cfg.n_routed, cfg.k_active
     ns, ms = cfg.n_shared, cfg.m_shared
     TK = T * K
     return {
-        0: ("tensor", 2.0 * T * d * (N + l + 2 * ns * ms)),
+        0: ("tensor", 2.0 * T * d * (N + l)),
         1: ("hbm", 4.0 * T * N + 8.0 * TK),
         2: ("hbm", 4.0 * TK * 5),
         3: ("hbm", 2.0 * TK * l * 2 + 4.0 * TK),

@@ -156,11 +156,13 @@ int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *num
 
 /* Profiling hook.  slots > 0: every later lmoe_forward on this handle also
  * records CUDA events on its stream before the first stage and after each
- * stage (stages, in order: 0 router+down+shared GEMM over x, 1 top-K', 2
+ * stage (stages, in order: 0 router + W_down GEMM over x, 1 top-K', 2
  * dispatch, 3 permute z, 4 expert gate/up GEMM, 5 expert down GEMM, 6
  * combine, 7 output GEMM; the fp32 mode maps its kernels onto the same
- * indices), into a ring of `slots` event sets created here (never in the
- * forward).  slots == 0 turns profiling off.  Errors: NULL_ARG, CUDA. */
+ * indices; the bf16 shared experts' gate/up GEMM runs on a side stream during
+ * stages 1-3 and is not timed separately), into a ring of `slots` event sets
+ * created here (never in the forward).  slots == 0 turns profiling off.
+ * Errors: NULL_ARG, CUDA. */
 #define LMOE_NUM_STAGES 8
 int lmoe_profile(lmoe_handle h, int32_t slots);
 

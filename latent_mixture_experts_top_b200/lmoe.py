@@ -32,7 +32,7 @@ EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
             "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc", "lmoe_strerror",
             "lmoe_destroy")
 LMOE_NUM_STAGES = 8
-STAGE_NAMES = ("x_gemm_router_down_shared", "topk", "dispatch", "permute_z",
+STAGE_NAMES = ("x_gemm_router_down", "topk", "dispatch", "permute_z",
                "expert_gate_up_gemm", "expert_down_gemm", "combine", "out_gemm")
 
 

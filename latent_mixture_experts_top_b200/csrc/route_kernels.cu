@@ -291,8 +291,9 @@ __device__ __forceinline__ uint4 pack_vec<float>(const float *acc) {
 }
 
 // One warp per token; 16-byte vectors; slots summed in order 0..K-1 in fp32.
+// (At most 42 registers, so that all token warps are resident at once.)
 template <typename Tio>
-__global__ void __launch_bounds__(256) combine_kernel(const Tio *__restrict__ O,
+__global__ void __launch_bounds__(256, 6) combine_kernel(const Tio *__restrict__ O,
                                                       const int32_t *__restrict__ pos,
                                                       const float *__restrict__ gates, int T,
                                                       int K, int l, Tio *__restrict__ u, int ldu) {
@@ -310,17 +311,17 @@ __global__ void __launch_bounds__(256) combine_kernel(const Tio *__restrict__ O,
       const int my_p = kk < K ? pos[static_cast<size_t>(t) * K + kk] : 0;
       const float my_g = kk < K ? gates[static_cast<size_t>(t) * K + kk] : 0.0f;
       const int kn = min(32, K - k0);
-      // Eight slots' loads in flight, then accumulated in slot order.
-      for (int k1 = 0; k1 < kn; k1 += 8) {
-        uint4 raw[8];
+      // Four slots' loads in flight, then accumulated in slot order.
+      for (int k1 = 0; k1 < kn; k1 += 4) {
+        uint4 raw[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           const int p = __shfl_sync(kFull, my_p, (k1 + j) & 31);
           if (k1 + j < kn)
             raw[j] = __ldcs(reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l + vi * V));
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           const float g = __shfl_sync(kFull, my_g, (k1 + j) & 31);
           if (k1 + j < kn) accum_vec<Tio>(acc, raw[j], g);
         }

@@ -18,6 +18,9 @@
 // Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
 //               swizzle, into a 4-stage shared-memory ring (no multicast).
+//               For the expert gate/up GEMM the whole warp gathers the A rows
+//               from z by the dispatch permutation with 16-byte cp.async,
+//               writing the same 128-byte-swizzled layout the MMA reads.
 //   warp 1      TMEM owner and MMA issuer: one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into
 //               one of two 256-column fp32 accumulators in TMEM, and
@@ -174,9 +177,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles * p.n_tiles_n;
   const int nkb = p.Kdim / TKB;
 
+  const bool gather = p.gather_src != nullptr;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&ctl->full[s], 1);
+      // gather: the B copy's arrival plus one cp.async arrival per producer lane
+      ptx::mbar_init(&ctl->full[s], gather ? 33 : 1);
       ptx::mbar_init(&ctl->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -202,25 +207,75 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (!gather) {
+      if (lane == 0) {
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+          const Tile tl = decode_tile(p, t, m_tiles);
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
+              record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
+              ok = false;
+              break;
+            }
+            ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
+            ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
+            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
+          }
+        }
+        if (!ok) {  // let every copy still in flight land before the CTA exits
+          for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+            if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
+              record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
+        }
+      }
+    } else {
+      // Gather mode: lane L copies rows L, L+32, L+64, L+96 of every A tile
+      // (8 chunks of 16 bytes each per K-block); chunk j of row r goes to
+      // r*128 + ((j ^ (r & 7)) * 16), the 128-byte swizzle that TMA would
+      // produce.  Lane 0 also waits for free stages and loads B with TMA.
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile(p, t, m_tiles);
+        const __nv_bfloat16 *src[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pr = tl.a_row + lane + 32 * i;
+          const int tok = pr < p.gather_rows ? p.gather_perm[pr] / p.gather_k : 0;
+          src[i] = p.gather_src + static_cast<size_t>(tok) * p.gather_ld;
+        }
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
-            record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
+          int got = 1;
+          if (lane == 0) got = ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag) ? 1 : 0;
+          got = __shfl_sync(0xFFFFFFFFu, got, 0);
+          if (!got) {
+            if (lane == 0) record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
-          ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
-          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
+          if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(&ctl->full[s], B_BYTES);
+            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
+          }
+          uint8_t *tile = smA + s * A_BYTES;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = lane + 32 * i;
+            const __nv_bfloat16 *g = src[i] + kb * TKB;
+            uint8_t *row = tile + r * (TKB * 2);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) ptx::cp_async_16(row + ((j ^ (r & 7)) << 4), g + 8 * j);
+          }
+          ptx::cp_async_mbar_arrive_noinc(&ctl->full[s]);
         }
       }
-      if (!ok) {  // let every copy still in flight land before the CTA exits
+      if (!ok && lane == 0) {  // let every copy still in flight land before the CTA exits
         for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
           if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
             record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
@@ -250,6 +305,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           ptx::tc_fence_after();
+          if (gather) ptx::fence_proxy_async_shared();  // A was written by cp.async
           const uint32_t a_addr = ptx::smem_u32(smA + s * A_BYTES);
           const uint32_t b_addr = ptx::smem_u32(smB + s * B_BYTES);
 #pragma unroll

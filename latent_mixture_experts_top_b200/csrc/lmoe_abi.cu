@@ -478,13 +478,17 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 5, s);
-    p.mode = TC_EXPERT_DOWN;
-    p.Kdim = h->m;
-    p.n_tiles_n = (h->l + kTileN - 1) / kTileN;
-    p.b_rows_per_expert = h->l;
-    p.out = static_cast<__nv_bfloat16 *>(w.O);
-    p.ld_out = h->l;
-    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, p, h->num_sms, h->num_sms, s);
+    TcParams pd = {};  // fresh: the down GEMM reads H with TMA (no gather)
+    pd.mode = TC_EXPERT_DOWN;
+    pd.Kdim = h->m;
+    pd.n_tiles_n = (h->l + kTileN - 1) / kTileN;
+    pd.tiles = w.tiles;
+    pd.n_mtiles = w.n_tiles;
+    pd.b_rows_per_expert = h->l;
+    pd.out = static_cast<__nv_bfloat16 *>(w.O);
+    pd.ld_out = h->l;
+    pd.status = w.status;
+    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 6, s);

@@ -432,6 +432,11 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
     attr_done = dev;
   }
   if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
+  // The gather reads Kdim columns of each gathered row: only the gate/up GEMM
+  // (Kdim = row width of z) may gather.
+  if (p.gather_src && (p.mode != TC_EXPERT_GU || p.Kdim > p.gather_ld || !p.gather_perm ||
+                       p.gather_k < 1))
+    return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
   CUtensorMap a, b;

@@ -233,21 +233,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     } else {
-      // Gather mode: lane L copies rows L, L+32, L+64, L+96 of every A tile
-      // (8 chunks of 16 bytes each per K-block); chunk j of row r goes to
-      // r*128 + ((j ^ (r & 7)) * 16), the 128-byte swizzle that TMA would
-      // produce.  Lane 0 also waits for free stages and loads B with TMA.
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(p, t, m_tiles);
-        const __nv_bfloat16 *src[4];
+      // Gather mode (expert gate/up): each A row is one 128-byte line of z.
+      // Eight lanes copy a row together (16 bytes each), four rows per
+      // instruction; chunk j of row r goes to r*128 + ((j ^ (r & 7)) * 16),
+      // the 128-byte swizzle that TMA would produce.  Lane L holds the token
+      // of rows L, L+32, L+64, L+96; other lanes get it by shuffle.  The tile
+      // entry two tiles ahead and the row tokens one tile ahead are loaded
+      // early, so no tile starts with a dependent load.  Lane 0 also waits
+      // for free stages and loads B with TMA.
+      const int q = lane >> 3, j = lane & 7;
+      const int G = gridDim.x;
+      auto entry = [&](int tt) {
+        TileEntry te = {0, 0, 0, 0};
+        if (tt < total) te = p.tiles[tt / p.n_tiles_n];
+        return te;
+      };
+      auto tokens = [&](const TileEntry &te, int tt, int (&tok)[4]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int pr = tl.a_row + lane + 32 * i;
-          const int tok = pr < p.gather_rows ? p.gather_perm[pr] / p.gather_k : 0;
-          src[i] = p.gather_src + static_cast<size_t>(tok) * p.gather_ld;
+          const int pr = te.row0 + lane + 32 * i;
+          tok[i] = (tt < total && pr < p.gather_rows) ? p.gather_perm[pr] / p.gather_k : 0;
         }
+      };
+      int t = blockIdx.x;
+      TileEntry te_cur = entry(t), te_nxt = entry(t + G);
+      int tok_cur[4];
+      tokens(te_cur, t, tok_cur);
+      int it = 0;
+      bool ok = true;
+      for (; t < total && ok; t += G) {
+        int tok_nxt[4];
+        tokens(te_nxt, t + G, tok_nxt);           // in flight during this tile
+        const TileEntry te_nn = entry(t + 2 * G);  // in flight during this tile
+        const int b_row = te_cur.expert * p.b_rows_per_expert + (t % p.n_tiles_n) * TN;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -261,23 +279,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (lane == 0) {
             ptx::mbar_arrive_expect_tx(&ctl->full[s], B_BYTES);
-            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
+            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, b_row);
           }
           uint8_t *tile = smA + s * A_BYTES;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = lane + 32 * i;
-            const __nv_bfloat16 *g = src[i] + kb * TKB;
-            uint8_t *row = tile + r * (TKB * 2);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) ptx::cp_async_16(row + ((j ^ (r & 7)) << 4), g + 8 * j);
+          for (int i = 0; i < 32; ++i) {
+            const int r = 4 * i + q;  // row of this lane's chunk
+            const int tok = __shfl_sync(0xFFFFFFFFu, tok_cur[i >> 3], 4 * (i & 7) + q);
+            const __nv_bfloat16 *g =
+                p.gather_src + static_cast<size_t>(tok) * p.gather_ld + kb * TKB + 8 * j;
+            ptx::cp_async_16(tile + r * (TKB * 2) + ((j ^ (r & 7)) << 4), g);
           }
           ptx::cp_async_mbar_arrive_noinc(&ctl->full[s]);
         }
+        te_cur = te_nxt;
+        te_nxt = te_nn;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tok_cur[i] = tok_nxt[i];
       }
       if (!ok && lane == 0) {  // let every copy still in flight land before the CTA exits
-        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-          if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
+        for (int jj = (it > STAGES ? it - STAGES : 0); jj < it; ++jj)
+          if (!drain_wait(&ctl->full[jj % STAGES], (jj / STAGES) & 1))
             record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
       }
     }

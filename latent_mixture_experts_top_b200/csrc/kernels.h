@@ -85,15 +85,6 @@ struct TcParams {
   __nv_bfloat16 *z; int ld_z;
   __nv_bfloat16 *out; int ld_out;   // H, O, y, or Ucat (+ column offset for shared)
   int out_col0;
-  // TC_EXPERT_GU with gather_src set: A row r of a tile is row
-  // gather_perm[row0 + r] / gather_k of gather_src [*][gather_ld] (z), copied
-  // by the producer warp with cp.async into the swizzled A tile, so the
-  // permuted copy of z is never written.  Rows at or past gather_rows read
-  // row 0 (they are masked in the epilogue).
-  const __nv_bfloat16 *gather_src;
-  int gather_ld;
-  const int32_t *gather_perm;
-  int gather_k, gather_rows;
   int32_t *status;
 };
 

@@ -452,11 +452,9 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   mark(h, 0, s);
   cudaError_t e = run_route(h, x, T, true, s);
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  if (!h->bf16) {  // the bf16 gate/up GEMM gathers the z rows itself
-    e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
-    h->launches += 1;
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  }
+  e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
+  h->launches += 1;
+  if (e != cudaSuccess) return LMOE_ERR_CUDA;
   mark(h, 4, s);
   if (h->bf16) {
     TcParams p = {};
@@ -468,17 +466,12 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.b_rows_per_expert = 2 * h->m;
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
-    p.gather_src = static_cast<const __nv_bfloat16 *>(w.z);
-    p.gather_ld = h->l;
-    p.gather_perm = w.perm;
-    p.gather_k = h->K;
-    p.gather_rows = TK;
     p.status = w.status;
     e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 5, s);
-    TcParams pd = {};  // fresh: the down GEMM reads H with TMA (no gather)
+    TcParams pd = {};
     pd.mode = TC_EXPERT_DOWN;
     pd.Kdim = h->m;
     pd.n_tiles_n = (h->l + kTileN - 1) / kTileN;

@@ -77,25 +77,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
       : "memory");
 }
 
-// ------------------------------------------------------------------ cp.async
-// 16-byte global -> shared copy through L2 (generic proxy).
-__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
-               "l"(gsrc)
-               : "memory");
-}
-// One arrival on `bar` once every cp.async this thread issued so far has
-// landed (counts against the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-// Orders generic-proxy shared-memory writes (cp.async) this thread has
-// observed before its later async-proxy reads (tcgen05.mma operands).
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 // TMEM allocation: executed by one full warp; the TMEM base address is written
 // to *smem_dst.  ncols: power of two in [32, 512].

@@ -18,9 +18,6 @@
 // Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
 //               swizzle, into a 4-stage shared-memory ring (no multicast).
-//               For the expert gate/up GEMM the whole warp gathers the A rows
-//               from z by the dispatch permutation with 16-byte cp.async,
-//               writing the same 128-byte-swizzled layout the MMA reads.
 //   warp 1      TMEM owner and MMA issuer: one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into
 //               one of two 256-column fp32 accumulators in TMEM, and
@@ -177,11 +174,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles * p.n_tiles_n;
   const int nkb = p.Kdim / TKB;
 
-  const bool gather = p.gather_src != nullptr;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // gather: the B copy's arrival plus one cp.async arrival per producer lane
-      ptx::mbar_init(&ctl->full[s], gather ? 33 : 1);
+      ptx::mbar_init(&ctl->full[s], 1);
       ptx::mbar_init(&ctl->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -207,99 +202,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (!gather) {
-      if (lane == 0) {
-        int it = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-          const Tile tl = decode_tile(p, t, m_tiles);
-          for (int kb = 0; kb < nkb; ++kb, ++it) {
-            const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1;
-            if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
-              record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
-              ok = false;
-              break;
-            }
-            ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
-            ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
-            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
-          }
-        }
-        if (!ok) {  // let every copy still in flight land before the CTA exits
-          for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-            if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
-              record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
-        }
-      }
-    } else {
-      // Gather mode (expert gate/up): each A row is one 128-byte line of z.
-      // Eight lanes copy a row together (16 bytes each), four rows per
-      // instruction; chunk j of row r goes to r*128 + ((j ^ (r & 7)) * 16),
-      // the 128-byte swizzle that TMA would produce.  Lane L holds the token
-      // of rows L, L+32, L+64, L+96; other lanes get it by shuffle.  The tile
-      // entry two tiles ahead and the row tokens one tile ahead are loaded
-      // early, so no tile starts with a dependent load.  Lane 0 also waits
-      // for free stages and loads B with TMA.
-      const int q = lane >> 3, j = lane & 7;
-      const int G = gridDim.x;
-      auto entry = [&](int tt) {
-        TileEntry te = {0, 0, 0, 0};
-        if (tt < total) te = p.tiles[tt / p.n_tiles_n];
-        return te;
-      };
-      auto tokens = [&](const TileEntry &te, int tt, int (&tok)[4]) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int pr = te.row0 + lane + 32 * i;
-          tok[i] = (tt < total && pr < p.gather_rows) ? p.gather_perm[pr] / p.gather_k : 0;
-        }
-      };
-      int t = blockIdx.x;
-      TileEntry te_cur = entry(t), te_nxt = entry(t + G);
-      int tok_cur[4];
-      tokens(te_cur, t, tok_cur);
+    if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (; t < total && ok; t += G) {
-        int tok_nxt[4];
-        tokens(te_nxt, t + G, tok_nxt);           // in flight during this tile
-        const TileEntry te_nn = entry(t + 2 * G);  // in flight during this tile
-        const int b_row = te_cur.expert * p.b_rows_per_expert + (t % p.n_tiles_n) * TN;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, t, m_tiles);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          int got = 1;
-          if (lane == 0) got = ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag) ? 1 : 0;
-          got = __shfl_sync(0xFFFFFFFFu, got, 0);
-          if (!got) {
-            if (lane == 0) record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
+          if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
+            record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
             ok = false;
             break;
           }
-          if (lane == 0) {
-            ptx::mbar_arrive_expect_tx(&ctl->full[s], B_BYTES);
-            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, b_row);
-          }
-          uint8_t *tile = smA + s * A_BYTES;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int r = 4 * i + q;  // row of this lane's chunk
-            const int tok = __shfl_sync(0xFFFFFFFFu, tok_cur[i >> 3], 4 * (i & 7) + q);
-            const __nv_bfloat16 *g =
-                p.gather_src + static_cast<size_t>(tok) * p.gather_ld + kb * TKB + 8 * j;
-            ptx::cp_async_16(tile + r * (TKB * 2) + ((j ^ (r & 7)) << 4), g);
-          }
-          ptx::cp_async_mbar_arrive_noinc(&ctl->full[s]);
+          ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
+          ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
+          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
         }
-        te_cur = te_nxt;
-        te_nxt = te_nn;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tok_cur[i] = tok_nxt[i];
       }
-      if (!ok && lane == 0) {  // let every copy still in flight land before the CTA exits
-        for (int jj = (it > STAGES ? it - STAGES : 0); jj < it; ++jj)
-          if (!drain_wait(&ctl->full[jj % STAGES], (jj / STAGES) & 1))
+      if (!ok) {  // let every copy still in flight land before the CTA exits
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          if (!drain_wait(&ctl->full[j % STAGES], (j / STAGES) & 1))
             record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
       }
     }
@@ -327,7 +250,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           ptx::tc_fence_after();
-          if (gather) ptx::fence_proxy_async_shared();  // A was written by cp.async
           const uint32_t a_addr = ptx::smem_u32(smA + s * A_BYTES);
           const uint32_t b_addr = ptx::smem_u32(smB + s * B_BYTES);
 #pragma unroll
@@ -454,11 +376,6 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
     attr_done = dev;
   }
   if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
-  // The gather reads Kdim columns of each gathered row: only the gate/up GEMM
-  // (Kdim = row width of z) may gather.
-  if (p.gather_src && (p.mode != TC_EXPERT_GU || p.Kdim > p.gather_ld || !p.gather_perm ||
-                       p.gather_k < 1))
-    return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
   CUtensorMap a, b;

@@ -106,9 +106,12 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out);
 /* Copies the weights into handle-owned device memory, repacked for the
  * kernels (bf16: router, W_down and the shared gate/up rows stacked into one
  * matrix over x; expert gate/up rows interleaved in blocks of 128; W_up and
- * the shared down-projections concatenated along their input dimension).
- * The caller's buffers may be freed once `stream` has passed this call.
- * Errors: NULL_ARG, CUDA. */
+ * the shared down-projections concatenated along their input dimension; and
+ * every such matrix stored K-block tiled, one contiguous 256 x 64 block per
+ * tile).  bf16 uses temporary device buffers and synchronises `stream`
+ * before returning; fp32 is asynchronous (the caller's buffers may be freed
+ * once `stream` has passed this call).  Errors: NULL_ARG, OUT_OF_MEMORY,
+ * CUDA. */
 int lmoe_load_weights(lmoe_handle h, const lmoe_weights *w, void *stream);
 
 /* Routing only (router GEMM, softmax / top-K' / renormalise, dispatch).

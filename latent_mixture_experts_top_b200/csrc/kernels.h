@@ -77,7 +77,7 @@ struct TcParams {
   int n_tile_base;     // dense modes: first N-tile (a launch may cover a column range)
   const TileEntry *tiles;   // grouped modes
   const int32_t *n_mtiles;  // grouped modes: device count of M-tiles
-  int b_rows_per_expert;    // grouped modes: B rows per expert (2m or l)
+  int b_rows_per_expert;    // unused (B is K-block tiled: see launch_repack_btiles)
   // TC_X_FUSED column regions (multiples of 256): [0, r_end) router logits,
   // [r_end, z_end) z, [z_end, ...) shared gate/up interleaved in blocks of 128.
   int r_end, z_end, n_routed, l;
@@ -87,6 +87,18 @@ struct TcParams {
   int out_col0;
   int32_t *status;
 };
+
+// B operands of the tcgen05 GEMMs are stored K-block tiled: for each group
+// (expert, or the whole matrix), N-tile n of 256 rows and K-block kb of 64
+// columns, one contiguous 256 x 64 bf16 block (32 KB), so that every TMA
+// load of B reads one contiguous range.  Rows past rows_per_group are zero.
+// src: [groups][rows_per_group][cols] row-major; dst holds
+// groups * ceil(rows_per_group/256) * (cols/64) blocks.
+inline int64_t btile_rows(int groups, int rows_per_group, int cols) {
+  return static_cast<int64_t>(groups) * ((rows_per_group + 255) / 256) * (cols / 64) * 256;
+}
+cudaError_t launch_repack_btiles(const __nv_bfloat16 *src, int groups, int rows_per_group,
+                                 int cols, __nv_bfloat16 *dst, cudaStream_t s);
 
 // Encodes a 2-D bf16 K-major tensor map (rows x cols, row stride in
 // elements) with a {64, box_rows} box and 128-byte swizzle.  Host only.

@@ -220,9 +220,11 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
             dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16);
   if (ok) {  // weights
     if (h->bf16) {
-      ok = dalloc(&h->w_x, static_cast<size_t>(h->nx_rows) * d * es) &&
-           dalloc(&h->w_gu, N * 2 * m * l * es) && dalloc(&h->w_out, N * l * m * es) &&
-           dalloc(&h->w_y, d * h->ky * es);
+      // K-block-tiled B operands (see launch_repack_btiles)
+      ok = dalloc(&h->w_x, btile_rows(1, h->nx_rows, h->d) * 64 * es) &&
+           dalloc(&h->w_gu, btile_rows(h->N, 2 * h->m, h->l) * 64 * es) &&
+           dalloc(&h->w_out, btile_rows(h->N, h->l, h->m) * 64 * es) &&
+           dalloc(&h->w_y, btile_rows(1, h->d, h->ky) * 64 * es);
     } else {
       ok = dalloc(&h->w_router, N * d * es) && dalloc(&h->w_down, l * d * es) &&
            dalloc(&h->w_gate, N * m * l * es) && dalloc(&h->w_upx, N * m * l * es) &&
@@ -249,13 +251,15 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TK), h->l, h->l, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, static_cast<int64_t>(TK), h->m, h->m, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_ucat, w.ucat, h->Tmax, h->ky, h->ky, kTileM);
+    // B operands: [tiled rows][64], one {64, 256} box per K-block tile
     if (rc == LMOE_OK)
-      rc = make_map(&h->tm_wx, h->w_x, h->nx_rows, h->d, h->d, kTileN);
+      rc = make_map(&h->tm_wx, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN);
     if (rc == LMOE_OK)
-      rc = make_map(&h->tm_wgu, h->w_gu, static_cast<int64_t>(N) * 2 * h->m, h->l, h->l, kTileN);
+      rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->N, 2 * h->m, h->l), 64, 64, kTileN);
     if (rc == LMOE_OK)
-      rc = make_map(&h->tm_wo, h->w_out, static_cast<int64_t>(N) * h->l, h->m, h->m, kTileN);
-    if (rc == LMOE_OK) rc = make_map(&h->tm_wy, h->w_y, h->d, h->ky, h->ky, kTileN);
+      rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN);
+    if (rc == LMOE_OK)
+      rc = make_map(&h->tm_wy, h->w_y, btile_rows(1, h->d, h->ky), 64, 64, kTileN);
     if (rc == LMOE_OK &&
         (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
          cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
@@ -287,42 +291,79 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
     if (e == cudaSuccess && bytes) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s);
   };
   if (h->cfg.has_router_bias) cp(h->b_router, wt->b_router, N * 4);
-  // W_y = [W_up | S_o(0) | ... ]  ([d][l + ns ms])
-  if (e == cudaSuccess) e = copy2d(h->w_y, ky, wt->w_up, l, l, d, es, s);
-  for (size_t j = 0; j < ns && e == cudaSuccess; ++j)
-    e = copy2d(off(h->w_y, l + j * ms, es), ky, off(const_cast<void *>(wt->s_out), j * d * ms, es),
-               ms, ms, d, es, s);
-  cp(h->w_out, wt->w_out, N * l * m * es);
-  if (h->bf16) {
-    // Stacked x-matrix: rows [0,N) W_r, [n_pad, n_pad+l) W_down, then for each
-    // block b of 128 shared hidden units: 128 gate rows followed by the 128
-    // matching up rows.  Padding rows are zero.
-    if (e == cudaSuccess) e = cudaMemsetAsync(h->w_x, 0, static_cast<size_t>(h->nx_rows) * d * es, s);
-    cp(h->w_x, wt->w_router, N * d * es);
-    cp(off(h->w_x, static_cast<size_t>(h->n_pad) * d, es), wt->w_down, l * d * es);
-    const size_t sh0 = static_cast<size_t>(h->n_pad + h->l_pad);
-    for (size_t b = 0; b < ns * ms / 128; ++b) {
-      cp(off(h->w_x, (sh0 + 256 * b) * d, es), off(const_cast<void *>(wt->s_gate), 128 * b * d, es),
-         128 * d * es);
-      cp(off(h->w_x, (sh0 + 256 * b + 128) * d, es),
-         off(const_cast<void *>(wt->s_up), 128 * b * d, es), 128 * d * es);
-    }
-    // Expert gate/up: per expert, blocks of 128 gate rows then 128 up rows.
-    for (size_t b = 0; b < m / 128 && e == cudaSuccess; ++b) {
-      e = copy2d(off(h->w_gu, 256 * b * l, es), 2 * m * l,
-                 off(const_cast<void *>(wt->w_gate), 128 * b * l, es), m * l, 128 * l, N, es, s);
-      if (e == cudaSuccess)
-        e = copy2d(off(h->w_gu, (256 * b + 128) * l, es), 2 * m * l,
-                   off(const_cast<void *>(wt->w_upx), 128 * b * l, es), m * l, 128 * l, N, es, s);
-    }
-  } else {
+  if (!h->bf16) {
+    // fp32: the CUDA-core kernels read the natural layouts; W_y = [W_up | S_o(0) | ...]
+    if (e == cudaSuccess) e = copy2d(h->w_y, ky, wt->w_up, l, l, d, es, s);
+    for (size_t j = 0; j < ns && e == cudaSuccess; ++j)
+      e = copy2d(off(h->w_y, l + j * ms, es), ky,
+                 off(const_cast<void *>(wt->s_out), j * d * ms, es), ms, ms, d, es, s);
+    cp(h->w_out, wt->w_out, N * l * m * es);
     cp(h->w_router, wt->w_router, N * d * es);
     cp(h->w_down, wt->w_down, l * d * es);
     cp(h->w_gate, wt->w_gate, N * m * l * es);
     cp(h->w_upx, wt->w_upx, N * m * l * es);
     cp(h->s_gate, wt->s_gate, ns * ms * d * es);
     cp(h->s_up, wt->s_up, ns * ms * d * es);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    h->loaded = true;
+    return LMOE_OK;
   }
+  // bf16: assemble each B operand row-major in a temporary, then repack it
+  // K-block tiled into the handle's buffer.
+  void *tx = nullptr, *tgu = nullptr, *ty = nullptr;
+  const size_t bx = static_cast<size_t>(h->nx_rows) * d * es, bgu = N * 2 * m * l * es,
+               by = d * ky * es;
+  if (!dalloc(&tx, bx) || !dalloc(&tgu, bgu) || !dalloc(&ty, by)) {
+    if (tx) cudaFree(tx);
+    if (tgu) cudaFree(tgu);
+    cudaGetLastError();
+    return LMOE_ERR_OUT_OF_MEMORY;
+  }
+  // W_y = [W_up | S_o(0) | S_o(1) ...]  ([d][l + ns ms])
+  if (e == cudaSuccess) e = copy2d(ty, ky, wt->w_up, l, l, d, es, s);
+  for (size_t j = 0; j < ns && e == cudaSuccess; ++j)
+    e = copy2d(off(ty, l + j * ms, es), ky, off(const_cast<void *>(wt->s_out), j * d * ms, es),
+               ms, ms, d, es, s);
+  // Stacked x-matrix: rows [0,N) W_r, [n_pad, n_pad+l) W_down, then for each
+  // block b of 128 shared hidden units: 128 gate rows followed by the 128
+  // matching up rows.  Padding rows are zero.
+  if (e == cudaSuccess) e = cudaMemsetAsync(tx, 0, bx, s);
+  cp(tx, wt->w_router, N * d * es);
+  cp(off(tx, static_cast<size_t>(h->n_pad) * d, es), wt->w_down, l * d * es);
+  const size_t sh0 = static_cast<size_t>(h->n_pad + h->l_pad);
+  for (size_t b = 0; b < ns * ms / 128; ++b) {
+    cp(off(tx, (sh0 + 256 * b) * d, es), off(const_cast<void *>(wt->s_gate), 128 * b * d, es),
+       128 * d * es);
+    cp(off(tx, (sh0 + 256 * b + 128) * d, es), off(const_cast<void *>(wt->s_up), 128 * b * d, es),
+       128 * d * es);
+  }
+  // Expert gate/up: per expert, blocks of 128 gate rows then 128 up rows.
+  for (size_t b = 0; b < m / 128 && e == cudaSuccess; ++b) {
+    e = copy2d(off(tgu, 256 * b * l, es), 2 * m * l,
+               off(const_cast<void *>(wt->w_gate), 128 * b * l, es), m * l, 128 * l, N, es, s);
+    if (e == cudaSuccess)
+      e = copy2d(off(tgu, (256 * b + 128) * l, es), 2 * m * l,
+                 off(const_cast<void *>(wt->w_upx), 128 * b * l, es), m * l, 128 * l, N, es, s);
+  }
+  using bf = __nv_bfloat16;
+  if (e == cudaSuccess)
+    e = launch_repack_btiles(static_cast<const bf *>(tx), 1, h->nx_rows, h->d,
+                             static_cast<bf *>(h->w_x), s);
+  if (e == cudaSuccess)
+    e = launch_repack_btiles(static_cast<const bf *>(tgu), h->N, 2 * h->m, h->l,
+                             static_cast<bf *>(h->w_gu), s);
+  if (e == cudaSuccess)
+    e = launch_repack_btiles(static_cast<const bf *>(wt->w_out), h->N, h->l, h->m,
+                             static_cast<bf *>(h->w_out), s);
+  if (e == cudaSuccess)
+    e = launch_repack_btiles(static_cast<const bf *>(ty), 1, h->d, h->ky,
+                             static_cast<bf *>(h->w_y), s);
+  // the temporaries are freed once the repacks have run
+  const cudaError_t es2 = cudaStreamSynchronize(s);
+  cudaFree(tx);
+  cudaFree(tgu);
+  cudaFree(ty);
+  if (e == cudaSuccess) e = es2;
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
   h->loaded = true;
   return LMOE_OK;

@@ -331,7 +331,41 @@ __global__ void __launch_bounds__(256, 6) combine_kernel(const Tio *__restrict__
   }
 }
 
+// One 16-byte vector per thread: dst vector v -> (group, n-tile, k-block,
+// row, chunk), copied from the row-major source or zero past the group's rows.
+__global__ void __launch_bounds__(256) repack_btiles_kernel(const uint4 *__restrict__ src,
+                                                            int rows_per_group, int cols, int nt,
+                                                            int kb_count, int64_t n_vec,
+                                                            uint4 *__restrict__ dst) {
+  const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (v >= n_vec) return;
+  const int c8 = static_cast<int>(v & 7);
+  const int r = static_cast<int>((v >> 3) & 255);
+  const int64_t blk = v >> 11;  // 256 rows x 8 vectors per block
+  const int kb = static_cast<int>(blk % kb_count);
+  const int64_t gn = blk / kb_count;
+  const int n = static_cast<int>(gn % nt);
+  const int64_t g = gn / nt;
+  const int srow = n * 256 + r;
+  uint4 val = make_uint4(0u, 0u, 0u, 0u);
+  if (srow < rows_per_group)
+    val = src[((g * rows_per_group + srow) * cols + kb * 64) / 8 + c8];
+  dst[v] = val;
+}
+
 }  // namespace
+
+cudaError_t launch_repack_btiles(const __nv_bfloat16 *src, int groups, int rows_per_group,
+                                 int cols, __nv_bfloat16 *dst, cudaStream_t s) {
+  if (cols % 64 || groups <= 0 || rows_per_group <= 0) return cudaErrorInvalidValue;
+  const int nt = (rows_per_group + 255) / 256, kbc = cols / 64;
+  const int64_t n_vec = static_cast<int64_t>(groups) * nt * kbc * 256 * 8;
+  const int64_t blocks = (n_vec + 255) / 256;
+  repack_btiles_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      reinterpret_cast<const uint4 *>(src), rows_per_group, cols, nt, kbc, n_vec,
+      reinterpret_cast<uint4 *>(dst));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, int N, int K,
                         int32_t *ids, float *gates, int32_t *counts, int chunk, cudaStream_t s) {

@@ -15,6 +15,9 @@
 // the projections, the shared path at width d), Figure 9 (latent expert
 // l -> m -> l); SwiGLU expert per the paragraph after Figure 1.
 //
+// B operands are K-block tiled in memory (one contiguous 256 x 64 block per
+// N-tile and K-block), so each B load is one contiguous 32 KB range.
+//
 // Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
 //               swizzle, into a 4-stage shared-memory ring (no multicast).
@@ -74,14 +77,14 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
   if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
     const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
     tl.a_row = m * TM;
-    tl.b_row = n * TN;
+    tl.b_row = n * (p.Kdim / TKB) * TN;  // first K-block tile of B's N-tile n
     tl.n_tile = n;
     tl.row_hi = p.M;
   } else {
     const int mt = t / p.n_tiles_n, n = t % p.n_tiles_n;  // consecutive CTAs share A
     const TileEntry te = p.tiles[mt];
     tl.a_row = te.row0;
-    tl.b_row = te.expert * p.b_rows_per_expert + n * TN;
+    tl.b_row = (te.expert * p.n_tiles_n + n) * (p.Kdim / TKB) * TN;
     tl.n_tile = n;
     tl.row_hi = te.row_end;
   }
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
           ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
-          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kb * TKB, tl.b_row);
+          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
         }
       }
       if (!ok) {  // let every copy still in flight land before the CTA exits

@@ -27,8 +27,8 @@
 //               tcgen05.commit frees ring stages / publishes accumulators.
 //   warps 2-9   epilogue: two warps per TMEM lane quarter, each taking half
 //               of the tile's columns: tcgen05.ld 32 lanes x 32 columns,
-//               fused epilogue, rows staged through shared memory and
-//               stored as full 128-byte lines; overlaps the next tile's MMAs.
+//               fused epilogue, 16-byte global stores; overlaps the next
+//               tile's MMAs.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA records a
 // status, stops its roles, lets in-flight copies and MMAs land, frees TMEM and
 // returns.
@@ -64,9 +64,7 @@ struct __align__(8) SmemCtl {
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES +
-                              NUM_EPI_WARPS * 32 * 128 /*epilogue staging*/ + sizeof(SmemCtl);
-static_assert(SMEM_BYTES <= 232448, "shared memory over the 227 KB per-CTA limit");
+constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemCtl);
 
 struct Tile {
   int a_row, b_row, n_tile, row_hi;
@@ -105,108 +103,60 @@ __device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
   return true;
 }
 
-// ---- epilogue helpers
-// tcgen05.ld gives each thread one output row.  Storing row-per-thread would
-// make every warp store touch 32 rows, so each warp stages a 32-row x
-// 128-byte block in shared memory (16-byte pieces XOR-swizzled by row, so
-// both sides are bank-conflict free) and writes it back with 8 lanes per
-// row: every store instruction then covers four full 128-byte lines.
-constexpr int STAGE_ROW_BYTES = 128;
-constexpr int STAGE_WARP_BYTES = 32 * STAGE_ROW_BYTES;
-
-__device__ __forceinline__ uint4 pack8_bf16(const float *v) {
-  uint4 w;
-  w.x = pack_bf16x2(v[0], v[1]);
-  w.y = pack_bf16x2(v[2], v[3]);
-  w.z = pack_bf16x2(v[4], v[5]);
-  w.w = pack_bf16x2(v[6], v[7]);
-  return w;
-}
-
-// Piece c (16 bytes) of this lane's row of the warp's staged block.
-__device__ __forceinline__ void stage_put(uint8_t *stage, int lane, int c, uint4 v) {
-  *reinterpret_cast<uint4 *>(stage + lane * STAGE_ROW_BYTES + ((c ^ (lane & 7)) << 4)) = v;
-}
-
-// Writes the warp's staged 32 rows x 128 bytes to global memory.  g0 points at
-// row 0 of the block (the segment's first byte); rows past rows_valid and
-// bytes past bytes_valid (a multiple of 16) are not written.
-__device__ __forceinline__ void stage_flush(uint8_t *stage, int lane, uint8_t *g0,
-                                            size_t ld_bytes, int rows_valid, int bytes_valid) {
-  __syncwarp();
-  const int j = lane & 7;
+// ---- epilogue helpers: one thread = one output row, 32 fp32 columns at a time
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float *v) {
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int R = 4 * i + (lane >> 3);
-    const uint4 v =
-        *reinterpret_cast<const uint4 *>(stage + R * STAGE_ROW_BYTES + ((j ^ (R & 7)) << 4));
-    if (R < rows_valid && j * 16 < bytes_valid)
-      *reinterpret_cast<uint4 *>(g0 + R * ld_bytes + j * 16) = v;
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = w;
   }
-  __syncwarp();  // the block is read out before the next one is staged
+}
+__device__ __forceinline__ void store_f32x32(float *dst, const float *v) {
+  float4 *d = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
-__device__ __forceinline__ int clamp_bytes(int b) { return b < 0 ? 0 : (b > 128 ? 128 : b); }
-
-// Half of a 256-column accumulator (128 columns) -> bf16 or f32 output
-// columns col0 + half*128 ..; columns at or past n_cols are not written.
-template <bool F32OUT>
-__device__ __forceinline__ void epi_plain(uint32_t taddr, uint8_t *stage, int lane, void *base,
-                                          size_t ld_elems, int rows_valid, int col0, int n_cols,
-                                          int half) {
-  constexpr int ES = F32OUT ? 4 : 2;
-  constexpr int CHUNKS_PER_SEG = F32OUT ? 1 : 2;  // 32-column chunks per 128-byte segment
-  uint8_t *b = static_cast<uint8_t *>(base);
+// 256 accumulator columns -> bf16 (or f32) row segment, chunks past n_cols skipped.
+template <bool F32OUT, typename OutT>
+__device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_dst, int col0,
+                                          int n_cols, int half) {
 #pragma unroll 1
-  for (int c0 = half * 4; c0 < half * 4 + 4; c0 += CHUNKS_PER_SEG) {
-#pragma unroll 1
-    for (int cc = 0; cc < CHUNKS_PER_SEG; ++cc) {
-      uint32_t r[32];
-      ptx::tmem_ld_32x32b_x32(taddr + (c0 + cc) * 32, r);
-      ptx::tmem_ld_wait();
-      if constexpr (F32OUT) {
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+    uint32_t r[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+    ptx::tmem_ld_wait();
+    float v[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          stage_put(stage, lane, q, make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]));
-      } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float v[8];
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) v[jj] = __uint_as_float(r[8 * q + jj]);
-          stage_put(stage, lane, cc * 4 + q, pack8_bf16(v));
-        }
-      }
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    const int col = col0 + c * 32;
+    if (valid && col < n_cols) {
+      if constexpr (F32OUT) store_f32x32(reinterpret_cast<float *>(row_dst) + col, v);
+      else store_bf16x32(reinterpret_cast<__nv_bfloat16 *>(row_dst) + col, v);
     }
-    const int col = col0 + c0 * 32;
-    stage_flush(stage, lane, b + static_cast<size_t>(col) * ES, ld_elems * ES, rows_valid,
-                clamp_bytes((n_cols - col) * ES));
   }
 }
 
 // Columns [0,128) are gate rows g0..g0+127, [128,256) the matching up rows:
-// this half writes h = silu(gate) * up for 64 hidden columns at hcol0 + half*64.
-__device__ __forceinline__ void epi_swiglu(uint32_t taddr, uint8_t *stage, int lane,
-                                           __nv_bfloat16 *base, size_t ld_elems, int rows_valid,
+// h = silu(gate) * up for 128 hidden columns starting at hcol0.
+__device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bfloat16 *row_dst,
                                            int hcol0, int half) {
 #pragma unroll 1
-  for (int cc = 0; cc < 2; ++cc) {
-    const int c = half * 2 + cc;
+  for (int c = half * (TN / 128); c < (half + 1) * (TN / 128); ++c) {
     uint32_t g[32], u[32];
     ptx::tmem_ld_32x32b_x32(taddr + c * 32, g);
     ptx::tmem_ld_32x32b_x32(taddr + TN / 2 + c * 32, u);
     ptx::tmem_ld_wait();
+    float h[32];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float h[8];
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj)
-        h[jj] = silu_bf16out(__uint_as_float(g[8 * q + jj])) * __uint_as_float(u[8 * q + jj]);
-      stage_put(stage, lane, cc * 4 + q, pack8_bf16(h));
-    }
+    for (int j = 0; j < 32; ++j) h[j] = silu_bf16out(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+    if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
   }
-  stage_flush(stage, lane, reinterpret_cast<uint8_t *>(base + hcol0 + half * 64), ld_elems * 2,
-              rows_valid, 128);
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -217,9 +167,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *smA = smem;
   uint8_t *smB = smem + STAGES * A_BYTES;
-  uint8_t *stage_all = smem + STAGES * STAGE_BYTES;  // epilogue staging, 4 KB per warp
-  SmemCtl *ctl =
-      reinterpret_cast<SmemCtl *>(stage_all + NUM_EPI_WARPS * 32 * 128);
+  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + STAGES * STAGE_BYTES);
   volatile int *abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -326,7 +274,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;   // which half of the tile's columns
-    uint8_t *stage = stage_all + (warp - 2) * STAGE_WARP_BYTES;
+    const int row_in_tile = q * 32 + lane;
     int tl_count = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl_count) {
       const int acc = tl_count & 1;
@@ -342,30 +290,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ptx::tc_fence_after();
       const Tile tl = decode_tile(p, t, m_tiles);
-      const int row0 = tl.a_row + q * 32;  // first of this warp's 32 rows
-      const int rows_valid = max(0, min(32, tl.row_hi - row0));
+      const int row = tl.a_row + row_in_tile;
+      const bool valid = row < tl.row_hi;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
       const int col0 = tl.n_tile * TN;
       switch (p.mode) {
         case TC_X_FUSED:
           if (col0 < p.r_end) {
-            epi_plain<true>(taddr, stage, lane, p.logits + static_cast<size_t>(row0) * p.ld_logits,
-                            p.ld_logits, rows_valid, col0, p.n_routed, half);
+            epi_plain<true>(taddr, valid, p.logits + static_cast<size_t>(row) * p.ld_logits, col0,
+                            p.n_routed, half);
           } else if (col0 < p.z_end) {
-            epi_plain<false>(taddr, stage, lane, p.z + static_cast<size_t>(row0) * p.ld_z, p.ld_z,
-                             rows_valid, col0 - p.r_end, p.l, half);
+            epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
+                             col0 - p.r_end, p.l, half);
           } else {
-            epi_swiglu(taddr, stage, lane, p.out + static_cast<size_t>(row0) * p.ld_out, p.ld_out,
-                       rows_valid, p.out_col0 + (col0 - p.z_end) / 2, half);
+            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
+                       p.out_col0 + (col0 - p.z_end) / 2, half);
           }
           break;
         case TC_EXPERT_GU:
-          epi_swiglu(taddr, stage, lane, p.out + static_cast<size_t>(row0) * p.ld_out, p.ld_out,
-                     rows_valid, col0 / 2, half);
+          epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
           break;
         default:  // TC_EXPERT_DOWN, TC_OUT
-          epi_plain<false>(taddr, stage, lane, p.out + static_cast<size_t>(row0) * p.ld_out,
-                           p.ld_out, rows_valid, col0, p.ld_out, half);
+          epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
+                           p.ld_out, half);
           break;
       }
       ptx::tc_fence_before();

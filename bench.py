@@ -201,7 +201,7 @@ def numpy_inputs(inp):
 
 # ---------------------------------------------------------------- reference arm
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0      # the oracle runs once, on rank 0; other ranks do no work
     import numpy as np
@@ -236,6 +236,32 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- ranks
+def rank_env():
+    """(world size, rank, local rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max_over_ranks(v: float, world: int, device: str) -> float:
+    """Max of a per-rank time over all ranks (the slowest rank sets the job's
+    time); identity on one rank.  Needs an initialised process group."""
+    if world == 1:
+        return float(v)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, max_ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank runs its own replica on its own tokens
+    (no exchange), so the job moves world * tokens_per_rank per step, in the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (max_ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- our arm
 def traffic_from_profiles(kernel_key, sha):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
@@ -268,9 +294,7 @@ def run_ours(args):
     import torch.distributed as dist
     from latent_mixture_experts_top_b200 import lmoe, synth
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -282,11 +306,7 @@ def run_ours(args):
             dist.barrier()
 
     def allmax(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max_over_ranks(v, world, "cuda")
 
     cfg = workload(args.workload)
     inp = synth.make_inputs(cfg, args.seed, "cuda")
@@ -327,7 +347,7 @@ def run_ours(args):
         raise RuntimeError("device status error during timing")
     total_ms = allmax(sum(step_ms))
     ms_per_step = total_ms / K
-    value = cfg.T * world / (ms_per_step / 1e3)
+    value = job_throughput(cfg.T, world, ms_per_step)
 
     peaks, peak_src = load_peaks()
     work = stage_work(cfg)

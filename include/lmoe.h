@@ -148,6 +148,16 @@ int lmoe_get_dims(lmoe_handle h, int32_t *l, int32_t *n_routed, int32_t *k_activ
  * if the stream reports an error. */
 int lmoe_device_status(lmoe_handle h, void *stream);
 
+/* Failure-detection self-test.  Launches one warp that waits on an mbarrier
+ * nothing ever completes, with the same bounded wait the GEMM kernels use
+ * for every pipeline barrier, but limited to limit_ns (1 .. 2e9); when the
+ * wait runs out the kernel records a timeout in the handle's status word and
+ * returns, so the next lmoe_device_status gives LMOE_ERR_DEVICE_TIMEOUT and
+ * the context stays usable.  It does not fault or hang the GPU.  No
+ * counterpart in the pages (test infrastructure for the status word).
+ * Errors: NULL_ARG, INVALID_CONFIG (limit out of range), CUDA. */
+int lmoe_selftest_wait_timeout(lmoe_handle h, int64_t limit_ns, void *stream);
+
 /* Test and profiling hook: the device address and element count of one of
  * the handle's intermediate buffers after the last call on the stream
  * (which: 0 logits f32 [T][N'], 1 z [T][l], 2 permuted z [T*K'][l],

@@ -14,6 +14,7 @@ enum : int {
   DEV_TIMEOUT_MMA = 2,        // MMA issuer waited too long for data / accumulator
   DEV_TIMEOUT_EPILOGUE = 3,   // epilogue waited too long for an accumulator
   DEV_TIMEOUT_DRAIN = 4,      // abort path: in-flight copies did not land
+  DEV_TIMEOUT_SELFTEST = 5,   // the failure-detection self-test's wait ran out
 };
 
 // Every spin-wait in these kernels gives up after this long and records a

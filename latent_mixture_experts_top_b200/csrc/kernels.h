@@ -105,6 +105,9 @@ cudaError_t launch_repack_btiles(const __nv_bfloat16 *src, int groups, int rows_
 int make_tmap_bf16(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
                    int64_t cols, int64_t row_stride_elems, int box_rows);
 
+// Failure-detection self-test (see lmoe_selftest_wait_timeout).
+cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s);
+
 cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p,
                            int num_sms, int max_ctas, cudaStream_t s);
 

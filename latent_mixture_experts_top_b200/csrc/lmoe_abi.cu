@@ -623,6 +623,14 @@ int lmoe_device_status(lmoe_handle h, void *stream) {
   return LMOE_OK;
 }
 
+int lmoe_selftest_wait_timeout(lmoe_handle h, int64_t limit_ns, void *stream) {
+  if (!h) return LMOE_ERR_NULL_ARG;
+  if (limit_ns <= 0 || limit_ns > 2000000000LL) return LMOE_ERR_INVALID_CONFIG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  return cuda_err(launch_wait_selftest(h->ws.status, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
 int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel) {
   if (!h || !dev_ptr || !numel) return LMOE_ERR_NULL_ARG;
   const int64_t T = h->Tmax, TK = static_cast<int64_t>(h->Tmax) * h->K;

@@ -330,6 +330,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// Failure-detection self-test: one warp waits, with the same bounded wait as
+// the GEMM roles, on an mbarrier that nothing ever completes; the wait runs
+// out after limit_ns and the status word records it.  No fault, no hang.
+__global__ void wait_selftest_kernel(int32_t *status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns))
+    atomicCAS(status, 0, DEV_TIMEOUT_SELFTEST);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -385,6 +401,12 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   memcpy(&a, tmapA, sizeof(a));
   memcpy(&b, tmapB, sizeof(b));
   tc_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s) {
+  if (limit_ns <= 0 || limit_ns > static_cast<long long>(kWaitLimitNs)) return cudaErrorInvalidValue;
+  wait_selftest_kernel<<<1, 32, 0, s>>>(status, static_cast<unsigned long long>(limit_ns));
   return cudaGetLastError();
 }
 

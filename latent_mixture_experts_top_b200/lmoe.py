@@ -29,8 +29,8 @@ STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -8: "LMOE_ERR_OUT_OF_MEMORY"}
 EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
             "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
-            "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc", "lmoe_strerror",
-            "lmoe_destroy")
+            "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc",
+            "lmoe_selftest_wait_timeout", "lmoe_strerror", "lmoe_destroy")
 LMOE_NUM_STAGES = 8
 STAGE_NAMES = ("x_gemm_router_down", "topk", "dispatch", "permute_z",
                "expert_gate_up_gemm", "expert_down_gemm", "combine", "out_gemm")
@@ -61,6 +61,7 @@ _lib.lmoe_profile.argtypes = [P, I32]
 _lib.lmoe_stage_times.argtypes = [P, C.POINTER(C.c_float), I32, C.POINTER(I32),
                                   C.POINTER(C.c_int64)]
 _lib.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P]
+_lib.lmoe_selftest_wait_timeout.argtypes = [P, C.c_int64, P]
 _lib.lmoe_strerror.argtypes = [C.c_int]
 _lib.lmoe_strerror.restype = C.c_char_p
 _lib.lmoe_destroy.argtypes = [P]
@@ -183,6 +184,11 @@ def lmoe_dispatch_noalloc(ids, T: int, k_active: int, n_routed: int, offsets, pe
     not allocate device memory where they run it."""
     _check(_lib.lmoe_dispatch_noalloc(_ptr(ids), T, k_active, n_routed, _ptr(offsets),
                                       _ptr(perm), _stream(stream)), "lmoe_dispatch_noalloc")
+
+
+def lmoe_selftest_wait_timeout(handle: int, limit_ns: int, stream=None) -> None:
+    _check(_lib.lmoe_selftest_wait_timeout(handle, int(limit_ns), _stream(stream)),
+           "lmoe_selftest_wait_timeout")
 
 
 def lmoe_destroy(handle: int) -> None:

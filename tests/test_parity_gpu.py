@@ -199,3 +199,27 @@ def test_call_errors_on_device_handle():
         lm.lmoe_forward(h, inp["x"], None, cfg.T)
     assert e.value.code == -2
     lm.lmoe_destroy(h)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """Failure detection without a GPU fault: a wait that nothing completes
+    runs out after 1 ms, the status word reports it, and the next forward on
+    the same context is still correct."""
+    cfg = configs.TINY_F32
+    lm = _lmoe()
+    inp = _inputs(cfg)
+    layer = lm.LatentMoELayer(cfg, inp)
+    assert lm.lmoe_device_status(layer.handle) == 0
+    lm.lmoe_selftest_wait_timeout(layer.handle, 1_000_000)
+    assert lm.lmoe_device_status(layer.handle) == -6      # LMOE_ERR_DEVICE_TIMEOUT
+    assert lm.lmoe_device_status(layer.handle) == 0       # read clears it
+    y = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert lm.lmoe_device_status(layer.handle) == 0
+    L = pu.oracle_layer(inp, cfg.k_active)
+    x_np = synth.to_numpy(inp["x"])
+    y_ref, _, _ = oracle.forward(L, x_np, tokens=np.arange(8))
+    assert pu.rel_err(pu.y_to_numpy(y)[:8], y_ref) <= pu.TOL_F32
+    with pytest.raises(lm.LmoeError):
+        lm.lmoe_selftest_wait_timeout(layer.handle, 0)
+    layer.close()

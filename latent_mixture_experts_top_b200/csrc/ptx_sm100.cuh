@@ -78,15 +78,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
       : "memory");
 }
 
-// Fetches the same box into L2 only (no shared memory, no barrier), so that a
-// later tma_load_2d of it hits L2.
-__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 // TMEM allocation: executed by one full warp; the TMEM base address is written
 // to *smem_dst.  ncols: power of two in [32, 512].

@@ -20,8 +20,7 @@
 //
 // Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
-//               swizzle, into a 4-stage shared-memory ring (no multicast),
-//               with L2 prefetches of the same boxes 8 K-blocks ahead.
+//               swizzle, into a 4-stage shared-memory ring (no multicast).
 //   warp 1      TMEM owner and MMA issuer: one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into
 //               one of two 256-column fp32 accumulators in TMEM, and
@@ -48,7 +47,6 @@ namespace {
 
 constexpr int TM = 128, TN = 256, TKB = 64;   // tile M, N, K-block
 constexpr int STAGES = 4;
-constexpr int PREFETCH_KB = 8;                // L2 prefetch distance, in K-blocks
 constexpr int A_BYTES = TM * TKB * 2;         // 16 KB
 constexpr int B_BYTES = TN * TKB * 2;         // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -208,22 +206,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // L2 prefetch cursor: runs PREFETCH_KB K-blocks ahead of the loads
-      // (into this CTA's next tile), so that the loads mostly hit L2 and the
-      // 4-stage ring covers their latency.
-      int pt = blockIdx.x, pkb = 0;
-      Tile ptl = decode_tile(p, pt < total ? pt : 0, m_tiles);
-      auto prefetch_next = [&]() {
-        if (pt >= total) return;
-        ptx::tma_prefetch_2d(&tmA, pkb * TKB, ptl.a_row);
-        ptx::tma_prefetch_2d(&tmB, 0, ptl.b_row + pkb * TN);
-        if (++pkb == nkb) {
-          pkb = 0;
-          pt += gridDim.x;
-          if (pt < total) ptl = decode_tile(p, pt, m_tiles);
-        }
-      };
-      for (int i = 0; i < PREFETCH_KB; ++i) prefetch_next();
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -231,7 +213,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          prefetch_next();
           if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
             record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
             ok = false;

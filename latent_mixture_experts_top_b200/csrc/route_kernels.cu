@@ -135,57 +135,76 @@ __device__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
   return before;
 }
 
-// Phase 2 (one block of 1024 threads): each thread scans the chunk counts of
-// its expert (in place: counts[e][c] becomes the number of pairs of expert e
-// in chunks before c); then the expert totals are scanned into offsets and
-// the table of tile_m-row M-tiles is written.
-__global__ void __launch_bounds__(1024) dispatch_scan_kernel(
+// Phase 2 (one block of 256 threads, each owning up to four experts -- a block
+// small enough to run beside a GEMM CTA on the same SM): each thread scans the
+// chunk counts of its experts (in place: counts[e][c] becomes the number of
+// pairs of expert e in chunks before c); the expert totals are then scanned
+// into offsets and the table of tile_m-row M-tiles is written.
+constexpr int kScanThreads = 256, kScanPerThread = 4;  // N <= 1024
+
+__device__ int scan_expert_row(int32_t *counts, int e, int n_chunks) {
+  // The row is contiguous (row stride n_chunks rounded up to 4): 16-byte
+  // loads, eight in flight at a time.
+  const int ncp = (n_chunks + 3) & ~3;
+  int4 *row = reinterpret_cast<int4 *>(counts + static_cast<size_t>(e) * ncp);
+  const int nv = ncp / 4;
+  int tot = 0;
+  for (int v0 = 0; v0 < nv; v0 += 8) {
+    int4 q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) q[j] = v0 + j < nv ? row[v0 + j] : make_int4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (v0 + j >= nv) break;
+      const int c = 4 * (v0 + j);
+      int4 o;
+      o.x = tot; tot += c + 0 < n_chunks ? q[j].x : 0;
+      o.y = tot; tot += c + 1 < n_chunks ? q[j].y : 0;
+      o.z = tot; tot += c + 2 < n_chunks ? q[j].z : 0;
+      o.w = tot; tot += c + 3 < n_chunks ? q[j].w : 0;
+      row[v0 + j] = o;
+    }
+  }
+  return tot;
+}
+
+__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
     int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
     TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles) {
   __shared__ int warp_sums[32];
-  const int e = threadIdx.x;  // N <= 1024: one thread per expert row
-  int tot = 0;
-  if (e < N) {
-    // The row is contiguous (row stride n_chunks rounded up to 4): 16-byte
-    // loads, eight in flight at a time.
-    const int ncp = (n_chunks + 3) & ~3;
-    int4 *row = reinterpret_cast<int4 *>(counts + static_cast<size_t>(e) * ncp);
-    const int nv = ncp / 4;
-    for (int v0 = 0; v0 < nv; v0 += 8) {
-      int4 q[8];
+  const int e0 = threadIdx.x * kScanPerThread;  // experts e0 .. e0+3
+  int tot[kScanPerThread], mt[kScanPerThread];
+  int my_tot = 0, my_mt = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) q[j] = v0 + j < nv ? row[v0 + j] : make_int4(0, 0, 0, 0);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (v0 + j >= nv) break;
-        const int c = 4 * (v0 + j);
-        int4 o;
-        o.x = tot; tot += c + 0 < n_chunks ? q[j].x : 0;
-        o.y = tot; tot += c + 1 < n_chunks ? q[j].y : 0;
-        o.z = tot; tot += c + 2 < n_chunks ? q[j].z : 0;
-        o.w = tot; tot += c + 3 < n_chunks ? q[j].w : 0;
-        row[v0 + j] = o;
-      }
-    }
+  for (int i = 0; i < kScanPerThread; ++i) {
+    const int e = e0 + i;
+    tot[i] = e < N ? scan_expert_row(counts, e, n_chunks) : 0;
+    mt[i] = (tot[i] + tile_m - 1) / tile_m;
+    my_tot += tot[i];
+    my_mt += mt[i];
   }
-  int all = 0;
-  const int off = block_exclusive_scan(tot, warp_sums, &all);
-  const int mt = (tot + tile_m - 1) / tile_m;
-  int all_tiles = 0;
-  const int tstart = block_exclusive_scan(mt, warp_sums, &all_tiles);
-  if (e < N) {
-    offsets[e] = off;
-    for (int j = 0; j < mt; ++j) {
-      const int idx = tstart + j;
-      if (idx < max_tiles) {
-        TileEntry te;
-        te.row0 = off + j * tile_m;
-        te.row_end = off + tot;
-        te.expert = e;
-        te.pad = 0;
-        tiles[idx] = te;
+  int all = 0, all_tiles = 0;
+  int off = block_exclusive_scan(my_tot, warp_sums, &all);
+  int tstart = block_exclusive_scan(my_mt, warp_sums, &all_tiles);
+#pragma unroll
+  for (int i = 0; i < kScanPerThread; ++i) {
+    const int e = e0 + i;
+    if (e < N) {
+      offsets[e] = off;
+      for (int j = 0; j < mt[i]; ++j) {
+        const int idx = tstart + j;
+        if (idx < max_tiles) {
+          TileEntry te;
+          te.row0 = off + j * tile_m;
+          te.row_end = off + tot[i];
+          te.expert = e;
+          te.pad = 0;
+          tiles[idx] = te;
+        }
       }
     }
+    off += tot[i];
+    tstart += mt[i];
   }
   if (threadIdx.x == 0) {
     offsets[N] = all;
@@ -291,9 +310,10 @@ __device__ __forceinline__ uint4 pack_vec<float>(const float *acc) {
 }
 
 // One warp per token; 16-byte vectors; slots summed in order 0..K-1 in fp32.
-// (At most 42 registers, so that all token warps are resident at once.)
+// (At most 64 registers: 32 warps per SM keep all token warps of the bench
+// workload resident at once.)
 template <typename Tio>
-__global__ void __launch_bounds__(256, 6) combine_kernel(const Tio *__restrict__ O,
+__global__ void __launch_bounds__(256, 4) combine_kernel(const Tio *__restrict__ O,
                                                       const int32_t *__restrict__ pos,
                                                       const float *__restrict__ gates, int T,
                                                       int K, int l, Tio *__restrict__ u, int ldu) {
@@ -311,17 +331,17 @@ __global__ void __launch_bounds__(256, 6) combine_kernel(const Tio *__restrict__
       const int my_p = kk < K ? pos[static_cast<size_t>(t) * K + kk] : 0;
       const float my_g = kk < K ? gates[static_cast<size_t>(t) * K + kk] : 0.0f;
       const int kn = min(32, K - k0);
-      // Four slots' loads in flight, then accumulated in slot order.
-      for (int k1 = 0; k1 < kn; k1 += 4) {
-        uint4 raw[4];
+      // Eight slots' loads in flight, then accumulated in slot order.
+      for (int k1 = 0; k1 < kn; k1 += 8) {
+        uint4 raw[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const int p = __shfl_sync(kFull, my_p, (k1 + j) & 31);
           if (k1 + j < kn)
             raw[j] = __ldcs(reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l + vi * V));
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const float g = __shfl_sync(kFull, my_g, (k1 + j) & 31);
           if (k1 + j < kn) accum_vec<Tio>(acc, raw[j], g);
         }
@@ -399,8 +419,8 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  dispatch_scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, nc, N, offsets, tiles, n_tiles, tile_m,
-                                          max_tiles);
+  dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_counts, nc, N, offsets, tiles, n_tiles,
+                                                   tile_m, max_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || nc == 0) return e;
   const int warps = chunk / 32;

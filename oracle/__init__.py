@@ -49,6 +49,7 @@ class _Layer(C.Structure):
         ("d", C.c_int32), ("l", C.c_int32), ("m", C.c_int32),
         ("n_routed", C.c_int32), ("k_active", C.c_int32),
         ("n_shared", C.c_int32), ("m_shared", C.c_int32), ("dtype", C.c_int32),
+        ("activation", C.c_int32),
         ("w_router", C.c_void_p), ("b_router", C.c_void_p),
         ("w_down", C.c_void_p), ("w_up", C.c_void_p),
         ("w_gate", C.c_void_p), ("w_upx", C.c_void_p), ("w_out", C.c_void_p),
@@ -122,10 +123,18 @@ class Layer:
     w_router [N'][d], b_router [N'] (float64) or None, w_down [l][d],
     w_up [d][l], w_gate / w_upx [N'][m][l], w_out [N'][l][m],
     s_gate / s_up [n_s][m_s][d], s_out [n_s][d][m_s].
+    activation "swiglu" (three matrices) or "relu2" (squared ReLU, two
+    matrices: w_upx / s_up are the up-projections; w_gate / s_gate unused).
     """
 
     def __init__(self, *, w_router, b_router, w_down, w_up, w_gate, w_upx,
-                 w_out, s_gate, s_up, s_out, k_active):
+                 w_out, s_gate, s_up, s_out, k_active, activation="swiglu"):
+        if activation not in ("swiglu", "relu2"):
+            raise ValueError("activation must be 'swiglu' or 'relu2'")
+        self.activation = activation
+        if activation == "relu2":   # two matrices: the gate weights are unused
+            w_gate = w_upx if w_gate is None else w_gate
+            s_gate = s_up if s_gate is None else s_gate
         arrs = dict(w_router=w_router, w_down=w_down, w_up=w_up, w_gate=w_gate,
                     w_upx=w_upx, w_out=w_out, s_gate=s_gate, s_up=s_up, s_out=s_out)
         self._keep = {k: np.ascontiguousarray(v) for k, v in arrs.items()}
@@ -149,6 +158,7 @@ class Layer:
         assert self._keep["s_out"].shape == (ns, d, ms)
         k = self._keep
         self._c = _Layer(d, l, m, N, k_active, ns, ms, self.dtype,
+                         1 if activation == "relu2" else 0,
                          _ptr(k["w_router"]), _ptr(self.b_router), _ptr(k["w_down"]),
                          _ptr(k["w_up"]), _ptr(k["w_gate"]), _ptr(k["w_upx"]),
                          _ptr(k["w_out"]), _ptr(k["s_gate"]), _ptr(k["s_up"]),

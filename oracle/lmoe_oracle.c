@@ -27,6 +27,9 @@
  *   5. z   = W_down x                                      d -> l, no bias
  *   6. u   = sum_{k=0..K'-1} g_k E_{id_k}(z),  E(v) = W_o (silu(W_g v) * (W_u v))
  *   7. y   = W_up u + sum_{j=0..n_s-1} S_j(x)              S_j: SwiGLU at width d
+ * With activation = squared ReLU (the Expert class of the [Explained] code,
+ * "down(relu(up(x)) ** 2)", two matrices), E(v) = W_o (relu(W_u v))^2 and the
+ * shared experts likewise; W_g is unused.
  * Readings where the pages are silent (each listed in the design doc):
  *   - experts are SwiGLU with three matrices (the pages' code shows squared
  *     ReLU with two; the article says SwiGLU carries over with a third
@@ -50,9 +53,12 @@
 
 enum { ODT_F32 = 0, ODT_BF16 = 1, ODT_F64 = 2 };
 
+enum { OACT_SWIGLU = 0, OACT_RELU2 = 1 };
+
 typedef struct {
   int32_t d, l, m, n_routed, k_active, n_shared, m_shared;
   int32_t dtype;             /* element type of x and every weight below */
+  int32_t activation;        /* OACT_SWIGLU or OACT_RELU2 */
   const void *w_router;      /* [N'][d] */
   const double *b_router;    /* [N'] or NULL */
   const void *w_down;        /* [l][d] */
@@ -89,19 +95,28 @@ static void matvec(const void *W, int dt, size_t off, int rows, int cols,
 }
 
 static double silu(double a) { return a / (1.0 + exp(-a)); }
+static double relu2(double a) { return a > 0.0 ? a * a : 0.0; }
 
-/* One SwiGLU feed-forward: out = W_o (silu(W_g v) * (W_u v)).
- * W_g, W_u: [hid][in_w] at element offset off_in; W_o: [out_w][hid] at off_out.
- * [Explained], paragraph after Figure 1 (gated activation with a third matrix)
- * and Figure 9 (the hidden width is m on both sides). */
+/* One expert feed-forward at the layer's activation.
+ * SwiGLU: out = W_o (silu(W_g v) * (W_u v))  ([Explained], paragraph after
+ * Figure 1: a gated activation adds a third matrix; Figure 9: the hidden
+ * width is m on both sides).
+ * Squared ReLU: out = W_o (relu(W_u v))^2  ([Explained], the Expert class:
+ * up, relu, square, down).
+ * W_g, W_u: [hid][in_w] at element offset off_in; W_o: [out_w][hid] at off_out. */
 static void swiglu_ffn(const oracle_layer *L, const void *Wg, const void *Wu,
                        const void *Wo, size_t off_in, size_t off_out, int in_w,
                        int hid, int out_w, const double *v, double *out,
                        double *scratch /* 2*hid */) {
   double *a = scratch, *b = scratch + hid;
-  matvec(Wg, L->dtype, off_in, hid, in_w, v, a);
-  matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
-  for (int j = 0; j < hid; ++j) a[j] = silu(a[j]) * b[j];
+  if (L->activation == OACT_RELU2) {
+    matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
+    for (int j = 0; j < hid; ++j) a[j] = relu2(b[j]);
+  } else {
+    matvec(Wg, L->dtype, off_in, hid, in_w, v, a);
+    matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
+    for (int j = 0; j < hid; ++j) a[j] = silu(a[j]) * b[j];
+  }
   matvec(Wo, L->dtype, off_out, out_w, hid, a, out);
 }
 

@@ -18,14 +18,16 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "lmoe_oracle.c")
 
 PIN_FUNCS = [
     pins.test_golden_hand_case_b,
+    pins.test_golden_hand_case_relu2,
+    pins.test_alpha_one_relu2_is_the_pages_moe_class,
     pins.test_golden_silu_sign_and_gate_role,
     lambda: pins.test_topk_brute_force(7, 3),
     pins.test_topk_ties_go_to_lower_index,
     pins.test_gates_sum_to_one_and_are_non_increasing,
     pins.test_router_bias_enters_before_softmax,
-    pins.test_dense_limit_K_equals_N,
+    lambda: pins.test_dense_limit_K_equals_N("swiglu"),
     pins.test_alpha_one_identity_projections_is_standard_moe,
-    pins.test_mask_form_over_all_experts,
+    lambda: pins.test_mask_form_over_all_experts("swiglu"),
     lambda: pins.test_dispatch_is_the_unique_stable_grouping(37, 4, 16),
 ]
 
@@ -45,6 +47,10 @@ MUTATIONS = {
                        "for (int i = 0; i < d; ++i) yr[i] += 0.0 * sh[i];"),
     "slot_gate_index": ("for (int i = 0; i < l; ++i) u[i] += g[k] * eo[i];",
                         "for (int i = 0; i < l; ++i) u[i] += g[0] * eo[i];"),
+    "relu2_without_square": ("static double relu2(double a) { return a > 0.0 ? a * a : 0.0; }",
+                             "static double relu2(double a) { return a > 0.0 ? a : 0.0; }"),
+    "relu2_without_relu": ("static double relu2(double a) { return a > 0.0 ? a * a : 0.0; }",
+                           "static double relu2(double a) { return a * a; }"),
     "bias_dropped": ("s[e] = acc + (L->b_router ? L->b_router[e] : 0.0);", "s[e] = acc;"),
     "dispatch_token_descending": ("for (int64_t t = 0; t < T; ++t)\n      for (int k = 0; k < K; ++k)\n        if (ids[t * K + k] == e) {",
                                   "for (int64_t t = T - 1; t >= 0; --t)\n      for (int k = 0; k < K; ++k)\n        if (ids[t * K + k] == e) {"),

@@ -27,31 +27,38 @@ def _golden(name):
 def _layer_from_json(g):
     f64 = lambda k: np.array(g[k], dtype=np.float64)
     d = len(g["x"][0])
-    if "s_gate" in g:
-        sg, su, so = f64("s_gate"), f64("s_up"), f64("s_out")
+    act = g.get("activation", "swiglu")
+    if "s_up" in g:
+        sg = f64("s_gate") if "s_gate" in g else None
+        su, so = f64("s_up"), f64("s_out")
     else:  # no shared expert
         sg, su, so = (np.zeros((0, 1, d)), np.zeros((0, 1, d)), np.zeros((0, d, 1)))
     return oracle.Layer(w_router=f64("w_router"), b_router=None, w_down=f64("w_down"),
-                        w_up=f64("w_up"), w_gate=f64("w_gate"), w_upx=f64("w_upx"),
-                        w_out=f64("w_out"), s_gate=sg, s_up=su, s_out=so,
-                        k_active=g["k_active"])
+                        w_up=f64("w_up"), w_gate=f64("w_gate") if "w_gate" in g else None,
+                        w_upx=f64("w_upx"), w_out=f64("w_out"), s_gate=sg, s_up=su,
+                        s_out=so, k_active=g["k_active"], activation=act)
 
 
-def rand_layer(rng, d, l, m, N, K, ns, ms, dtype=np.float64, bias=False, wstd=0.3):
+def rand_layer(rng, d, l, m, N, K, ns, ms, dtype=np.float64, bias=False, wstd=0.3,
+               activation="swiglu"):
     r = lambda *s: (rng.standard_normal(s) * wstd).astype(dtype)
     return oracle.Layer(
         w_router=r(N, d), b_router=(rng.standard_normal(N) * 0.5 if bias else None),
         w_down=r(l, d), w_up=r(d, l), w_gate=r(N, m, l), w_upx=r(N, m, l),
         w_out=r(N, l, m), s_gate=r(ns, ms, d), s_up=r(ns, ms, d), s_out=r(ns, d, ms),
-        k_active=K)
+        k_active=K, activation=activation)
 
 
 def silu(a):
     return a / (1.0 + np.exp(-a))
 
 
-def ffn(Wg, Wu, Wo, v):
-    """Independent numpy SwiGLU FFN in matrix form (test-side, for reductions)."""
+def ffn(Wg, Wu, Wo, v, activation="swiglu"):
+    """Independent numpy expert FFN in matrix form (test-side, for reductions):
+    SwiGLU W_o (silu(W_g v) * W_u v), or the pages' squared-ReLU Expert class
+    W_o (relu(W_u v))**2 with two matrices."""
+    if activation == "relu2":
+        return Wo @ (np.maximum(Wu @ v, 0.0) ** 2)
     return Wo @ (silu(Wg @ v) * (Wu @ v))
 
 
@@ -64,6 +71,14 @@ def test_golden_hand_case_b():
     y, ids, gates = oracle.forward(L, x)
     assert ids.tolist() == g["expect_ids"]
     np.testing.assert_allclose(gates, g["expect_gates"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(y, g["expect_y"], rtol=0, atol=g["atol"])
+
+
+def test_golden_hand_case_relu2():
+    g = _golden("hand_case_relu2.json")
+    L = _layer_from_json(g)
+    y, ids, gates = oracle.forward(L, np.array(g["x"], dtype=np.float64))
+    assert ids.tolist() == g["expect_ids"]
     np.testing.assert_allclose(y, g["expect_y"], rtol=0, atol=g["atol"])
 
 
@@ -149,11 +164,12 @@ def test_router_bias_enters_before_softmax():
 
 # ------------------------------------------------------- whole-layer pins
 
-def test_dense_limit_K_equals_N():
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_dense_limit_K_equals_N(act):
     """K' = N': no selection is left, y = W_up sum_e softmax(s)_e E_e(z) + shared."""
     rng = np.random.default_rng(4)
     d, l, m, N, ns, ms = 12, 6, 10, 5, 2, 7
-    L = rand_layer(rng, d, l, m, N, N, ns, ms)
+    L = rand_layer(rng, d, l, m, N, N, ns, ms, activation=act)
     k = L._keep
     x = rng.standard_normal((6, d))
     y, _, _ = oracle.forward(L, x)
@@ -161,9 +177,34 @@ def test_dense_limit_K_equals_N():
         s = k["w_router"] @ x[t]
         p = np.exp(s - s.max()); p /= p.sum()
         z = k["w_down"] @ x[t]
-        u = sum(p[e] * ffn(k["w_gate"][e], k["w_upx"][e], k["w_out"][e], z) for e in range(N))
-        ref = k["w_up"] @ u + sum(ffn(k["s_gate"][j], k["s_up"][j], k["s_out"][j], x[t])
+        u = sum(p[e] * ffn(k["w_gate"][e], k["w_upx"][e], k["w_out"][e], z, act)
+                for e in range(N))
+        ref = k["w_up"] @ u + sum(ffn(k["s_gate"][j], k["s_up"][j], k["s_out"][j], x[t], act)
                                   for j in range(ns))
+        np.testing.assert_allclose(y[t], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_alpha_one_relu2_is_the_pages_moe_class():
+    """alpha = 1, identity projections, squared-ReLU experts: the layer is the
+    MoE class of the article's code (router on x, topk of the softmax,
+    renormalise, experts down(relu(up(x))**2), shared experts added)."""
+    rng = np.random.default_rng(15)
+    d, m, N, K, ns = 10, 8, 7, 3, 2
+    L = rand_layer(rng, d, d, m, N, K, ns, m, activation="relu2")
+    k = L._keep
+    k["w_down"][:] = np.eye(d)
+    k["w_up"][:] = np.eye(d)
+    x = rng.standard_normal((9, d))
+    y, ids, _ = oracle.forward(L, x)
+    for t in range(x.shape[0]):
+        scores = k["w_router"] @ x[t]
+        probs = np.exp(scores - scores.max()); probs /= probs.sum()
+        top = np.argsort(-probs, kind="stable")[:K]
+        w = probs[top] / probs[top].sum()
+        expert = lambda up, down, v: down @ (np.maximum(up @ v, 0.0) ** 2)
+        ref = sum(w[i] * expert(k["w_upx"][e], k["w_out"][e], x[t]) for i, e in enumerate(top))
+        ref = ref + sum(expert(k["s_up"][j], k["s_out"][j], x[t]) for j in range(ns))
+        assert sorted(ids[t].tolist()) == sorted(top.tolist())
         np.testing.assert_allclose(y[t], ref, rtol=1e-12, atol=1e-12)
 
 
@@ -205,11 +246,12 @@ def test_combine_then_up_equals_per_expert_up():
         np.testing.assert_allclose(y[t], alt, rtol=1e-12, atol=1e-12)
 
 
-def test_mask_form_over_all_experts():
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_mask_form_over_all_experts(act):
     """y equals the sum over ALL experts with zero gates off the top-K'."""
     rng = np.random.default_rng(7)
     d, l, m, N, K = 12, 4, 6, 9, 3
-    L = rand_layer(rng, d, l, m, N, K, 1, 5)
+    L = rand_layer(rng, d, l, m, N, K, 1, 5, activation=act)
     k = L._keep
     x = rng.standard_normal((8, d))
     y, ids, gates = oracle.forward(L, x)
@@ -217,9 +259,9 @@ def test_mask_form_over_all_experts():
         gate_full = np.zeros(N)
         gate_full[ids[t]] = gates[t]
         z = k["w_down"] @ x[t]
-        u = sum(gate_full[e] * ffn(k["w_gate"][e], k["w_upx"][e], k["w_out"][e], z)
+        u = sum(gate_full[e] * ffn(k["w_gate"][e], k["w_upx"][e], k["w_out"][e], z, act)
                 for e in range(N))
-        ref = k["w_up"] @ u + ffn(k["s_gate"][0], k["s_up"][0], k["s_out"][0], x[t])
+        ref = k["w_up"] @ u + ffn(k["s_gate"][0], k["s_up"][0], k["s_out"][0], x[t], act)
         np.testing.assert_allclose(y[t], ref, rtol=1e-12, atol=1e-12)
 
 

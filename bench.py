@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="readme_acc",
-                    choices=["readme_acc", "readme_eff", "prefill", "decode"])
+                    choices=["readme_acc", "readme_eff", "prefill", "decode", "relu2_95b"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
@@ -60,13 +60,19 @@ def parse_args():
 def workload(name):
     from latent_mixture_experts_top_b200 import configs
     return {"readme_acc": configs.README_ACC, "readme_eff": configs.README_EFF,
-            "prefill": configs.PREFILL, "decode": configs.DECODE}[name]
+            "prefill": configs.PREFILL, "decode": configs.DECODE,
+            "relu2_95b": configs.RELU2_95B}[name]
+
+
+def n_mats(cfg):
+    """Weight matrices per expert: SwiGLU 3 (gate, up, out), squared ReLU 2."""
+    return 2 if cfg.activation == "relu2" else 3
 
 
 def config_json(cfg, n_gpus):
     return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "l": cfg.l, "m": cfg.m,
             "n_routed": cfg.n_routed, "k_active": cfg.k_active, "n_shared": cfg.n_shared,
-            "m_shared": cfg.m_shared, "variant": cfg.variant,
+            "m_shared": cfg.m_shared, "variant": cfg.variant, "activation": cfg.activation,
             "router_bias": cfg.has_router_bias, "global_batch": cfg.T * n_gpus,
             "seq_len": cfg.T, "parallelism": f"replicas x{n_gpus} (no exchange)",
             "l2": "flushed by a 512 MiB write between timed steps"}
@@ -99,7 +105,7 @@ def stage_work(cfg):
         1: ("hbm", 4.0 * T * N + 8.0 * TK),
         2: ("hbm", 4.0 * TK * 5),
         3: ("hbm", 2.0 * TK * l * 2 + 4.0 * TK),
-        4: ("tensor", 2.0 * TK * l * 2 * m),
+        4: ("tensor", 2.0 * TK * l * (n_mats(cfg) - 1) * m),
         5: ("tensor", 2.0 * TK * m * l),
         6: ("hbm", 2.0 * TK * l + 8.0 * TK + 2.0 * T * l),
         7: ("tensor", 2.0 * T * (l + ns * ms) * d),
@@ -108,7 +114,8 @@ def stage_work(cfg):
 
 def layer_flops(cfg):
     T, d, l, m, N, K = cfg.T, cfg.d, cfg.l, cfg.m, cfg.n_routed, cfg.k_active
-    return 2.0 * T * (d * N + 2 * d * l + 3 * K * l * m + 3 * cfg.n_shared * d * cfg.m_shared)
+    nm = n_mats(cfg)
+    return 2.0 * T * (d * N + 2 * d * l + nm * K * l * m + nm * cfg.n_shared * d * cfg.m_shared)
 
 
 def layer_bytes(cfg, ids=None):
@@ -116,7 +123,8 @@ def layer_bytes(cfg, ids=None):
     experts hit) + x in + y out, bf16."""
     d, l, m, N = cfg.d, cfg.l, cfg.m, cfg.n_routed
     touched = N if ids is None else len(set(ids.reshape(-1).tolist()))
-    w = N * d + 2 * d * l + 3 * cfg.n_shared * d * cfg.m_shared + touched * 3 * l * m
+    nm = n_mats(cfg)
+    w = N * d + 2 * d * l + nm * cfg.n_shared * d * cfg.m_shared + touched * nm * l * m
     return 2.0 * (w + 2 * cfg.T * d)
 
 

@@ -51,6 +51,12 @@ typedef enum { LMOE_EFF = 0, LMOE_ACC = 1 } lmoe_variant;
  * combined u, shared hidden). */
 typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
 
+/* Expert activation.  LMOE_SWIGLU: E(v) = W_o (silu(W_g v) * (W_u v)), three
+ * matrices.  LMOE_RELU2: E(v) = W_o (relu(W_u v))^2, two matrices -- the
+ * Expert class of the article's code ("down(relu(up(x)) ** 2)"), the
+ * activation its 95B running example uses.  Shared experts use the same. */
+typedef enum { LMOE_SWIGLU = 0, LMOE_RELU2 = 1 } lmoe_activation;
+
 enum {
   LMOE_OK = 0,
   LMOE_ERR_INVALID_CONFIG = -1,  /* d % alpha != 0, K' outside [1, N'], sizes <= 0 */
@@ -69,8 +75,8 @@ enum {
  * n_routed_override / top_k_override (0 = derive N' and K' from the variant),
  * has_router_bias, max_tokens (workspace size; forward never allocates).
  * LMOE_BF16 additionally needs d, l, m_shared*n_shared to be multiples of 64,
- * m and m_shared multiples of 128, and N' a multiple of 32; every mode needs
- * N' <= 1024 (else LMOE_ERR_UNSUPPORTED). */
+ * N' a multiple of 32, and m, m_shared multiples of 128 (SwiGLU) or of 64
+ * (squared ReLU); every mode needs N' <= 1024 (else LMOE_ERR_UNSUPPORTED). */
 typedef struct {
   int32_t d, m, n_experts, top_k, alpha, n_shared, m_shared;
   int32_t variant;           /* lmoe_variant */
@@ -79,6 +85,7 @@ typedef struct {
   int32_t top_k_override;    /* K' if > 0 */
   int32_t has_router_bias;   /* 1: a float32 bias [N'] is added to the logits */
   int32_t max_tokens;        /* largest T any later call may pass */
+  int32_t activation;        /* lmoe_activation */
 } lmoe_config;
 
 typedef struct lmoe_layer *lmoe_handle;
@@ -88,7 +95,8 @@ typedef struct lmoe_layer *lmoe_handle;
  *   w_router [N'][d], b_router [N'] or NULL, w_down [l][d], w_up [d][l],
  *   w_gate [N'][m][l], w_upx [N'][m][l], w_out [N'][l][m],
  *   s_gate [n_s][m_s][d], s_up [n_s][m_s][d], s_out [n_s][d][m_s]
- * (s_* may be NULL when n_shared == 0). */
+ * (s_* may be NULL when n_shared == 0; w_gate and s_gate are unused, and may
+ * be NULL, for LMOE_RELU2, where w_upx / s_up are the up-projections). */
 typedef struct {
   const void *w_router;
   const float *b_router;

@@ -31,6 +31,7 @@ class LayerConfig:
     n_routed_override: int = 0
     top_k_override: int = 0
     router_bias_std: float = 0.0   # > 0: per-expert router bias ~ N(0, std)
+    activation: str = "swiglu"     # "swiglu" (3 matrices) | "relu2" (2 matrices)
     x_std: float = 1.0
     w_std: float = 0.02
 
@@ -71,5 +72,15 @@ PREFILL = LayerConfig("prefill_T16384_d4096_l1024_m2048_N512_K22_bias", T=16384,
 DECODE = replace(PREFILL, name="decode_T64_d4096_l1024_m2048_N512_K22", T=64,
                  router_bias_std=0.0)
 
+# Squared-ReLU experts ("LatentMoE Explained", the Expert class and the 95B
+# running example: d=4096, l=1024, m=2688, N=128 -> N'=512, K=6 -> K'=24, two
+# shared experts of width m).
+TINY_RELU2_F32 = replace(TINY_F32, name="tiny_relu2_f32_T64_d256_l128_N16_K4",
+                         activation="relu2")
+RELU2_95B = LayerConfig("relu2_95b_T1024_d4096_l1024_m2688_N512_K24", T=1024, d=4096,
+                        m=2688, n_experts=128, top_k=6, alpha=4, n_shared=2, m_shared=2688,
+                        variant="acc", activation="relu2")
+
 CONFIGS = [TINY_F32, README_ACC, README_EFF, PREFILL, DECODE]
-BY_NAME = {c.name: c for c in CONFIGS}
+EXTRA_CONFIGS = [TINY_RELU2_F32, RELU2_95B]
+BY_NAME = {c.name: c for c in CONFIGS + EXTRA_CONFIGS}

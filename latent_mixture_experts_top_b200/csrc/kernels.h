@@ -56,6 +56,10 @@ cudaError_t simt_linear(const float *A, int lda, const float *B, int ldb, float 
 cudaError_t simt_swiglu(const float *A, int lda, const float *Wg, const float *Wu, int mw,
                         const int32_t *row_expert, float *H, int ldh, int M, int Ncols, int Kdim,
                         cudaStream_t s);
+// H[r][c] = relu(A_r . Wu[e][c%mw])^2 (squared-ReLU experts), e as above.
+cudaError_t simt_relu2(const float *A, int lda, const float *Wu, int mw,
+                       const int32_t *row_expert, float *H, int ldh, int M, int Ncols, int Kdim,
+                       cudaStream_t s);
 // O[r][c] = H_r . Wo[row_expert[r]][c]   (Wo [*][Ncols][Kdim])
 cudaError_t simt_expert_down(const float *H, int ldh, const float *Wo,
                              const int32_t *row_expert, float *O, int ldo, int M, int Ncols,
@@ -85,6 +89,10 @@ struct TcParams {
   __nv_bfloat16 *z; int ld_z;
   __nv_bfloat16 *out; int ld_out;   // H, O, y, or Ucat (+ column offset for shared)
   int out_col0;
+  int relu2;           // squared-ReLU experts: TC_EXPERT_GU and the shared
+                       // region of TC_X_FUSED write relu(acc)^2 (no gate/up
+                       // interleave); n_cols2 bounds their output columns
+  int n_cols2;
   int32_t *status;
 };
 

@@ -48,12 +48,14 @@ struct lmoe_layer {
   lmoe_config cfg;
   int d = 0, l = 0, m = 0, N = 0, K = 0, ns = 0, ms = 0, Tmax = 0;
   int bf16 = 0;
+  int relu2 = 0;      // squared-ReLU experts (two matrices)
   size_t esize = 4;
   int device = 0, num_sms = 0;
   bool loaded = false;
   int max_tiles = 0;
-  // bf16 layout of the stacked x-matrix: [W_r | pad][W_down | pad][shared gate/up]
-  int n_pad = 0, l_pad = 0, nx_rows = 0;
+  // bf16 layout of the stacked x-matrix: [W_r | pad][W_down | pad][shared rows | pad]
+  int n_pad = 0, l_pad = 0, sh_rows = 0, nx_rows = 0;
+  int gu_rows = 0;    // B rows per expert of the expert up GEMM: 2m (SwiGLU) or m
   int ky = 0;  // l + n_s * m_s, the reduction length of the last GEMM
   // weights (handle-owned)
   void *w_router = nullptr;  // f32 path: [N][d]
@@ -122,6 +124,7 @@ int validate(const lmoe_config *c, lmoe_layer *h) {
     return LMOE_ERR_INVALID_CONFIG;
   if (c->variant != LMOE_EFF && c->variant != LMOE_ACC) return LMOE_ERR_INVALID_CONFIG;
   if (c->dtype != LMOE_F32 && c->dtype != LMOE_BF16) return LMOE_ERR_INVALID_CONFIG;
+  if (c->activation != LMOE_SWIGLU && c->activation != LMOE_RELU2) return LMOE_ERR_INVALID_CONFIG;
   if (c->d % c->alpha) return LMOE_ERR_INVALID_CONFIG;
   if (c->n_shared > 0 && c->m_shared <= 0) return LMOE_ERR_INVALID_CONFIG;
   const int64_t N = c->n_routed_override > 0 ? c->n_routed_override
@@ -141,11 +144,13 @@ int validate(const lmoe_config *c, lmoe_layer *h) {
   h->ms = c->n_shared > 0 ? c->m_shared : 0;
   h->Tmax = c->max_tokens;
   h->bf16 = c->dtype == LMOE_BF16;
+  h->relu2 = c->activation == LMOE_RELU2;
   h->esize = h->bf16 ? 2 : 4;
   h->ky = h->l + h->ns * h->ms;
   if (static_cast<int64_t>(h->Tmax) * h->K > INT32_MAX / 2) return LMOE_ERR_UNSUPPORTED;
   if (h->bf16) {
-    if (h->d % 64 || h->l % 64 || h->m % 128 || (h->ns > 0 && h->ms % 128) || h->N % 32)
+    const int mq = h->relu2 ? 64 : 128;  // SwiGLU tiles pair 128 gate with 128 up columns
+    if (h->d % 64 || h->l % 64 || h->m % mq || (h->ns > 0 && h->ms % mq) || h->N % 32)
       return LMOE_ERR_UNSUPPORTED;
   } else {
     if (h->l % 4 || h->ky % 4) return LMOE_ERR_UNSUPPORTED;
@@ -207,7 +212,9 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   h->max_tiles = static_cast<int>(TK / kTileM + N + 1);
   h->n_pad = (h->N + kTileN - 1) / kTileN * kTileN;
   h->l_pad = (h->l + kTileN - 1) / kTileN * kTileN;
-  h->nx_rows = h->n_pad + h->l_pad + 2 * h->ns * h->ms;
+  h->sh_rows = h->relu2 ? (h->ns * h->ms + kTileN - 1) / kTileN * kTileN : 2 * h->ns * h->ms;
+  h->nx_rows = h->n_pad + h->l_pad + h->sh_rows;
+  h->gu_rows = h->relu2 ? h->m : 2 * h->m;
   Workspace &w = h->ws;
   bool ok = dalloc(&w.logits, T * N * 4) && dalloc(&w.ids, TK * 4) && dalloc(&w.gates, TK * 4) &&
             dalloc(&w.chunk_counts, dispatch_count_elems(h->Tmax, kDispatchChunk, h->N) * 4) &&
@@ -222,14 +229,14 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     if (h->bf16) {
       // K-block-tiled B operands (see launch_repack_btiles)
       ok = dalloc(&h->w_x, btile_rows(1, h->nx_rows, h->d) * 64 * es) &&
-           dalloc(&h->w_gu, btile_rows(h->N, 2 * h->m, h->l) * 64 * es) &&
+           dalloc(&h->w_gu, btile_rows(h->N, h->gu_rows, h->l) * 64 * es) &&
            dalloc(&h->w_out, btile_rows(h->N, h->l, h->m) * 64 * es) &&
            dalloc(&h->w_y, btile_rows(1, h->d, h->ky) * 64 * es);
     } else {
       ok = dalloc(&h->w_router, N * d * es) && dalloc(&h->w_down, l * d * es) &&
-           dalloc(&h->w_gate, N * m * l * es) && dalloc(&h->w_upx, N * m * l * es) &&
-           dalloc(&h->w_out, N * l * m * es) &&
-           dalloc(&h->s_gate, static_cast<size_t>(h->ns) * h->ms * d * es) &&
+           (h->relu2 || dalloc(&h->w_gate, N * m * l * es)) &&
+           dalloc(&h->w_upx, N * m * l * es) && dalloc(&h->w_out, N * l * m * es) &&
+           (h->relu2 || dalloc(&h->s_gate, static_cast<size_t>(h->ns) * h->ms * d * es)) &&
            dalloc(&h->s_up, static_cast<size_t>(h->ns) * h->ms * d * es) &&
            dalloc(&h->w_y, d * h->ky * es);
     }
@@ -255,7 +262,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wx, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN);
     if (rc == LMOE_OK)
-      rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->N, 2 * h->m, h->l), 64, 64, kTileN);
+      rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->N, h->gu_rows, h->l), 64, 64, kTileN);
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN);
     if (rc == LMOE_OK)
@@ -277,9 +284,11 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
 
 int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   if (!h || !wt) return LMOE_ERR_NULL_ARG;
-  if (!wt->w_router || !wt->w_down || !wt->w_up || !wt->w_gate || !wt->w_upx || !wt->w_out)
+  if (!wt->w_router || !wt->w_down || !wt->w_up || !wt->w_upx || !wt->w_out)
     return LMOE_ERR_NULL_ARG;
-  if (h->ns > 0 && (!wt->s_gate || !wt->s_up || !wt->s_out)) return LMOE_ERR_NULL_ARG;
+  if (!h->relu2 && !wt->w_gate) return LMOE_ERR_NULL_ARG;
+  if (h->ns > 0 && (!wt->s_up || !wt->s_out || (!h->relu2 && !wt->s_gate)))
+    return LMOE_ERR_NULL_ARG;
   if (h->cfg.has_router_bias && !wt->b_router) return LMOE_ERR_NULL_ARG;
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
@@ -300,9 +309,9 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
     cp(h->w_out, wt->w_out, N * l * m * es);
     cp(h->w_router, wt->w_router, N * d * es);
     cp(h->w_down, wt->w_down, l * d * es);
-    cp(h->w_gate, wt->w_gate, N * m * l * es);
+    if (!h->relu2) cp(h->w_gate, wt->w_gate, N * m * l * es);
     cp(h->w_upx, wt->w_upx, N * m * l * es);
-    cp(h->s_gate, wt->s_gate, ns * ms * d * es);
+    if (!h->relu2) cp(h->s_gate, wt->s_gate, ns * ms * d * es);
     cp(h->s_up, wt->s_up, ns * ms * d * es);
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     h->loaded = true;
@@ -313,7 +322,7 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   void *tx = nullptr, *tgu = nullptr, *ty = nullptr;
   const size_t bx = static_cast<size_t>(h->nx_rows) * d * es, bgu = N * 2 * m * l * es,
                by = d * ky * es;
-  if (!dalloc(&tx, bx) || !dalloc(&tgu, bgu) || !dalloc(&ty, by)) {
+  if (!dalloc(&tx, bx) || (!h->relu2 && !dalloc(&tgu, bgu)) || !dalloc(&ty, by)) {
     if (tx) cudaFree(tx);
     if (tgu) cudaFree(tgu);
     cudaGetLastError();
@@ -331,14 +340,17 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   cp(tx, wt->w_router, N * d * es);
   cp(off(tx, static_cast<size_t>(h->n_pad) * d, es), wt->w_down, l * d * es);
   const size_t sh0 = static_cast<size_t>(h->n_pad + h->l_pad);
-  for (size_t b = 0; b < ns * ms / 128; ++b) {
+  if (h->relu2) {  // shared up rows, in expert order (padding rows stay zero)
+    cp(off(tx, sh0 * d, es), wt->s_up, ns * ms * d * es);
+  }
+  for (size_t b = 0; !h->relu2 && b < ns * ms / 128; ++b) {
     cp(off(tx, (sh0 + 256 * b) * d, es), off(const_cast<void *>(wt->s_gate), 128 * b * d, es),
        128 * d * es);
     cp(off(tx, (sh0 + 256 * b + 128) * d, es), off(const_cast<void *>(wt->s_up), 128 * b * d, es),
        128 * d * es);
   }
   // Expert gate/up: per expert, blocks of 128 gate rows then 128 up rows.
-  for (size_t b = 0; b < m / 128 && e == cudaSuccess; ++b) {
+  for (size_t b = 0; !h->relu2 && b < m / 128 && e == cudaSuccess; ++b) {
     e = copy2d(off(tgu, 256 * b * l, es), 2 * m * l,
                off(const_cast<void *>(wt->w_gate), 128 * b * l, es), m * l, 128 * l, N, es, s);
     if (e == cudaSuccess)
@@ -349,9 +361,9 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   if (e == cudaSuccess)
     e = launch_repack_btiles(static_cast<const bf *>(tx), 1, h->nx_rows, h->d,
                              static_cast<bf *>(h->w_x), s);
-  if (e == cudaSuccess)
-    e = launch_repack_btiles(static_cast<const bf *>(tgu), h->N, 2 * h->m, h->l,
-                             static_cast<bf *>(h->w_gu), s);
+  if (e == cudaSuccess)  // expert up rows: interleaved gate/up, or the up-projection itself
+    e = launch_repack_btiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->N,
+                             h->gu_rows, h->l, static_cast<bf *>(h->w_gu), s);
   if (e == cudaSuccess)
     e = launch_repack_btiles(static_cast<const bf *>(wt->w_out), h->N, h->l, h->m,
                              static_cast<bf *>(h->w_out), s);
@@ -361,7 +373,7 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   // the temporaries are freed once the repacks have run
   const cudaError_t es2 = cudaStreamSynchronize(s);
   cudaFree(tx);
-  cudaFree(tgu);
+  if (tgu) cudaFree(tgu);
   cudaFree(ty);
   if (e == cudaSuccess) e = es2;
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
@@ -407,6 +419,8 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.out = static_cast<__nv_bfloat16 *>(w.ucat);
     p.ld_out = h->ky;
     p.out_col0 = h->l;
+    p.relu2 = h->relu2;
+    p.n_cols2 = h->ns * h->ms;
     p.status = w.status;
     const int m_tiles = (T + kTileM - 1) / kTileM;
     e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, m_tiles * p.n_tiles_n, s);
@@ -435,9 +449,13 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
                       h->d, static_cast<float *>(w.z), h->l, T, h->l, h->d, s);
       h->launches += 1;
       if (e == cudaSuccess && h->ns > 0) {
-        e = simt_swiglu(static_cast<const float *>(x), h->d, static_cast<const float *>(h->s_gate),
-                        static_cast<const float *>(h->s_up), h->ms, nullptr,
-                        static_cast<float *>(w.ucat) + h->l, h->ky, T, h->ns * h->ms, h->d, s);
+        const float *xf = static_cast<const float *>(x);
+        float *hs = static_cast<float *>(w.ucat) + h->l;
+        e = h->relu2 ? simt_relu2(xf, h->d, static_cast<const float *>(h->s_up), h->ms, nullptr,
+                                  hs, h->ky, T, h->ns * h->ms, h->d, s)
+                     : simt_swiglu(xf, h->d, static_cast<const float *>(h->s_gate),
+                                   static_cast<const float *>(h->s_up), h->ms, nullptr, hs, h->ky,
+                                   T, h->ns * h->ms, h->d, s);
         h->launches += 1;
       }
     }
@@ -501,10 +519,12 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     TcParams p = {};
     p.mode = TC_EXPERT_GU;
     p.Kdim = h->l;
-    p.n_tiles_n = 2 * h->m / kTileN;
+    p.n_tiles_n = (h->gu_rows + kTileN - 1) / kTileN;
+    p.relu2 = h->relu2;
+    p.n_cols2 = h->m;
     p.tiles = w.tiles;
     p.n_mtiles = w.n_tiles;
-    p.b_rows_per_expert = 2 * h->m;
+    p.b_rows_per_expert = h->gu_rows;
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
     p.status = w.status;
@@ -547,9 +567,11 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     float *zpf = static_cast<float *>(w.zp);
     float *Hf = static_cast<float *>(w.H), *Of = static_cast<float *>(w.O);
     float *uf = static_cast<float *>(w.ucat);
-    e = simt_swiglu(zpf, h->l, static_cast<const float *>(h->w_gate),
-                    static_cast<const float *>(h->w_upx), h->m, w.row_expert, Hf, h->m, TK, h->m,
-                    h->l, s);
+    e = h->relu2 ? simt_relu2(zpf, h->l, static_cast<const float *>(h->w_upx), h->m,
+                              w.row_expert, Hf, h->m, TK, h->m, h->l, s)
+                 : simt_swiglu(zpf, h->l, static_cast<const float *>(h->w_gate),
+                               static_cast<const float *>(h->w_upx), h->m, w.row_expert, Hf,
+                               h->m, TK, h->m, h->l, s);
     h->launches += 1;
     mark(h, 5, s);
     if (e == cudaSuccess)

@@ -89,6 +89,23 @@ __global__ void __launch_bounds__(256) simt_swiglu_kernel(const float *__restric
   H[static_cast<size_t>(r) * ldh + c] = silu_f32(sg) * su;
 }
 
+// Squared-ReLU hidden: H[r][c] = relu(A_r . Wu_row)^2 (the article's Expert class).
+__global__ void __launch_bounds__(256) simt_relu2_kernel(const float *__restrict__ A, int lda,
+                                                         const float *__restrict__ Wu, int mw,
+                                                         const int32_t *__restrict__ row_expert,
+                                                         float *__restrict__ H, int ldh, int M,
+                                                         int Ncols, int Kd) {
+  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
+  const int r = blockIdx.y * 4 + (threadIdx.x >> 6);
+  if (r >= M || c >= Ncols) return;
+  const float *a = A + static_cast<size_t>(r) * lda;
+  const float *u = Wu + wrow(row_expert, r, c, mw, Kd);
+  float su = 0.0f;
+  for (int k = 0; k < Kd; ++k) su = fmaf(a[k], u[k], su);
+  const float h = su > 0.0f ? su : 0.0f;
+  H[static_cast<size_t>(r) * ldh + c] = h * h;
+}
+
 __global__ void __launch_bounds__(256) simt_expert_down_kernel(
     const float *__restrict__ Hm, int ldh, const float *__restrict__ Wo,
     const int32_t *__restrict__ row_expert, float *__restrict__ O, int ldo, int M, int Ncols,
@@ -119,6 +136,15 @@ cudaError_t simt_swiglu(const float *A, int lda, const float *Wg, const float *W
   if (M <= 0 || Ncols <= 0) return cudaSuccess;
   dim3 grid((Ncols + 63) / 64, (M + 3) / 4);
   simt_swiglu_kernel<<<grid, 256, 0, s>>>(A, lda, Wg, Wu, mw, row_expert, H, ldh, M, Ncols, Kdim);
+  return cudaGetLastError();
+}
+
+cudaError_t simt_relu2(const float *A, int lda, const float *Wu, int mw,
+                       const int32_t *row_expert, float *H, int ldh, int M, int Ncols, int Kdim,
+                       cudaStream_t s) {
+  if (M <= 0 || Ncols <= 0) return cudaSuccess;
+  dim3 grid((Ncols + 63) / 64, (M + 3) / 4);
+  simt_relu2_kernel<<<grid, 256, 0, s>>>(A, lda, Wu, mw, row_expert, H, ldh, M, Ncols, Kdim);
   return cudaGetLastError();
 }
 

@@ -6,7 +6,8 @@
 //                  experts' SwiGLU hidden (written next to u, so that the
 //                  last GEMM adds the shared output for free).
 //   TC_EXPERT_GU   grouped: permuted z rows of expert e times its gate/up
-//                  rows (interleaved in blocks of 128) -> SwiGLU -> H (bf16).
+//                  rows (interleaved in blocks of 128) -> SwiGLU -> H (bf16);
+//                  for squared-ReLU experts its up rows -> relu(.)^2 -> H.
 //   TC_EXPERT_DOWN grouped: H times W_o[e] -> expert output O (bf16).
 //   TC_OUT         [u | shared hidden] times [W_up | S_o] -> y (bf16).
 //
@@ -139,6 +140,25 @@ __device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_
       if constexpr (F32OUT) store_f32x32(reinterpret_cast<float *>(row_dst) + col, v);
       else store_bf16x32(reinterpret_cast<__nv_bfloat16 *>(row_dst) + col, v);
     }
+  }
+}
+
+// Squared-ReLU hidden: relu(acc)^2 -> bf16 columns col0 + ..., masked at n_cols.
+__device__ __forceinline__ void epi_relu2(uint32_t taddr, bool valid, __nv_bfloat16 *row_dst,
+                                          int col0, int n_cols, int half) {
+#pragma unroll 1
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+    uint32_t r[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+    ptx::tmem_ld_wait();
+    float h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float a = fmaxf(__uint_as_float(r[j]), 0.0f);
+      h[j] = a * a;
+    }
+    const int col = col0 + c * 32;
+    if (valid && col < n_cols) store_bf16x32(row_dst + col, h);
   }
 }
 
@@ -302,13 +322,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else if (col0 < p.z_end) {
             epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
                              col0 - p.r_end, p.l, half);
+          } else if (p.relu2) {
+            epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
+                      col0 - p.z_end, p.n_cols2, half);
           } else {
             epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
                        p.out_col0 + (col0 - p.z_end) / 2, half);
           }
           break;
         case TC_EXPERT_GU:
-          epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
+          if (p.relu2)
+            epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0, p.n_cols2,
+                      half);
+          else
+            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
           break;
         default:  // TC_EXPERT_DOWN, TC_OUT
           epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,

@@ -23,6 +23,7 @@ _lib = C.CDLL(_LIB_PATH)
 
 LMOE_EFF, LMOE_ACC = 0, 1
 LMOE_F32, LMOE_BF16 = 0, 1
+LMOE_SWIGLU, LMOE_RELU2 = 0, 1
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -3: "LMOE_ERR_NOT_LOADED", -4: "LMOE_ERR_TOO_MANY_TOKENS", -5: "LMOE_ERR_CUDA",
           -6: "LMOE_ERR_DEVICE_TIMEOUT", -7: "LMOE_ERR_UNSUPPORTED",
@@ -39,7 +40,7 @@ STAGE_NAMES = ("x_gemm_router_down", "topk", "dispatch", "permute_z",
 class lmoe_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "d", "m", "n_experts", "top_k", "alpha", "n_shared", "m_shared", "variant", "dtype",
-        "n_routed_override", "top_k_override", "has_router_bias", "max_tokens")]
+        "n_routed_override", "top_k_override", "has_router_bias", "max_tokens", "activation")]
 
 
 class lmoe_weights(C.Structure):
@@ -113,7 +114,8 @@ def config_from(cfg: LayerConfig, max_tokens: int | None = None) -> lmoe_config:
         dtype=LMOE_BF16 if cfg.dtype == "bf16" else LMOE_F32,
         n_routed_override=cfg.n_routed_override, top_k_override=cfg.top_k_override,
         has_router_bias=int(cfg.has_router_bias),
-        max_tokens=cfg.T if max_tokens is None else max_tokens)
+        max_tokens=cfg.T if max_tokens is None else max_tokens,
+        activation=LMOE_RELU2 if cfg.activation == "relu2" else LMOE_SWIGLU)
 
 
 def lmoe_create(config: lmoe_config) -> int:

@@ -8,10 +8,12 @@ Recipe (one torch Philox/MT generator seeded with ``seed``, fixed draw order):
   x ~ N(0, x_std) [T][d]; W_r [N'][d]; b_r [N'] ~ N(0, bias_std) (only when the
   workload has a router bias); W_down [l][d]; W_up [d][l]; W_g, W_u [N'][m][l];
   W_o [N'][l][m]; S_g, S_u [n_s][m_s][d]; S_o [n_s][d][m_s]; every weight
-  ~ N(0, w_std).  Values are drawn in float32 and, for bf16 workloads, rounded
-  to bf16 (round to nearest even, torch's cast).  Large tensors are drawn in
-  slices along their first axis so that the float32 staging stays small; the
-  slicing is part of the recipe (same seed + device -> same values).
+  ~ N(0, w_std).  Squared-ReLU workloads draw no W_g / S_g (two-matrix
+  experts), so their later draws come earlier in the stream.  Values are
+  drawn in float32 and, for bf16 workloads, rounded to bf16 (round to nearest
+  even, torch's cast).  Large tensors are drawn in slices along their first
+  axis so that the float32 staging stays small; the slicing is part of the
+  recipe (same seed + device -> same values).
 The router bias is always float32 (the library takes it in float32).
 """
 from __future__ import annotations
@@ -59,10 +61,11 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, device: str | torch.device = "c
                        if cfg.has_router_bias else None)
     out["w_down"] = _normal(gen, (l, d), w, dt, device)
     out["w_up"] = _normal(gen, (d, l), w, dt, device)
-    out["w_gate"] = _normal(gen, (N, m, l), w, dt, device)
+    relu2 = cfg.activation == "relu2"   # two-matrix experts: no gate weights drawn
+    out["w_gate"] = None if relu2 else _normal(gen, (N, m, l), w, dt, device)
     out["w_upx"] = _normal(gen, (N, m, l), w, dt, device)
     out["w_out"] = _normal(gen, (N, l, m), w, dt, device)
-    out["s_gate"] = _normal(gen, (ns, ms, d), w, dt, device)
+    out["s_gate"] = None if relu2 else _normal(gen, (ns, ms, d), w, dt, device)
     out["s_up"] = _normal(gen, (ns, ms, d), w, dt, device)
     out["s_out"] = _normal(gen, (ns, d, ms), w, dt, device)
     return out

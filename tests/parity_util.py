@@ -29,13 +29,13 @@ TOL_F32 = 1e-5
 TOL_BF16 = 2e-2
 
 
-def oracle_layer(inputs: dict, k_active: int) -> oracle.Layer:
+def oracle_layer(inputs: dict, k_active: int, activation: str = "swiglu") -> oracle.Layer:
     n = {k: (None if v is None else synth.to_numpy(v)) for k, v in inputs.items()}
     bias = None if n["b_router"] is None else n["b_router"].astype(np.float64)
     return oracle.Layer(w_router=n["w_router"], b_router=bias, w_down=n["w_down"],
                         w_up=n["w_up"], w_gate=n["w_gate"], w_upx=n["w_upx"],
                         w_out=n["w_out"], s_gate=n["s_gate"], s_up=n["s_up"],
-                        s_out=n["s_out"], k_active=k_active)
+                        s_out=n["s_out"], k_active=k_active, activation=activation)
 
 
 def boundary_gap(s_ref: np.ndarray, K: int) -> np.ndarray:

@@ -47,7 +47,7 @@ def _run(cfg, inp, x=None, max_tokens=None):
 def _check_layer(cfg, n_sample, seed=0):
     inp = _inputs(cfg, seed)
     layer, y, ids, gates, offsets, perm = _run(cfg, inp)
-    L = pu.oracle_layer(inp, cfg.k_active)
+    L = pu.oracle_layer(inp, cfg.k_active, cfg.activation)
     x_np = synth.to_numpy(inp["x"])
     s_ref = oracle.router_logits(L, x_np)
     ids_g, gates_g = ids.cpu().numpy(), gates.cpu().numpy()
@@ -85,6 +85,15 @@ def test_parity_decode_all_tokens():
 
 def test_parity_prefill_biased_router():
     _check_layer(configs.PREFILL, n_sample=48)
+
+
+def test_parity_relu2_tiny_f32_all_tokens():
+    _check_layer(configs.TINY_RELU2_F32, n_sample=10 ** 9)
+
+
+def test_parity_relu2_95b_shape():
+    """Squared-ReLU experts at the article's 95B running-example layer shape."""
+    _check_layer(configs.RELU2_95B, n_sample=48)
 
 
 @pytest.mark.parametrize("cfg,T", [(configs.TINY_F32, 1), (configs.TINY_F32, 5),

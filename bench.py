@@ -89,27 +89,39 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------- algorithmic work
-def stage_work(cfg):
-    """Algorithmic FLOPs (tensor stages) or bytes (memory stages) per launch.
+def stage_work(cfg, touched=None):
+    """Algorithmic (FLOPs, bytes) of one launch of each profiled stage.
 
-    Tensor stages count 2 flops per multiply-add of the layer's definition
-    (no padding, no masked rows).  The shared experts' gate/up GEMM overlaps
-    stages 1-3 on a side stream and is not a stage of its own.  Memory stages count the bytes the step must
-    read and write once (bf16 activations, int32 indices, fp32 logits/gates).
+    FLOPs count 2 per multiply-add of the layer's definition (no padding, no
+    masked rows); memory-only stages have 0.  Bytes are what the stage must
+    read and write once: bf16 activations and weights, int32 indices, fp32
+    logits and gates; an expert GEMM reads the weights of the ``touched``
+    distinct experts (all N' when not given).  The shared experts' gate/up
+    GEMM overlaps stages 1-3 on a side stream and is not a stage of its own.
     """
     T, d, l, m, N, K = cfg.T, cfg.d, cfg.l, cfg.m, cfg.n_routed, cfg.k_active
     ns, ms = cfg.n_shared, cfg.m_shared
+    E = N if touched is None else touched
     TK = T * K
+    gu = n_mats(cfg) - 1          # gate+up (2) or up (1) rows per hidden column
+    ky = l + ns * ms
     return {
-        0: ("tensor", 2.0 * T * d * (N + l)),
-        1: ("hbm", 4.0 * T * N + 8.0 * TK),
-        2: ("hbm", 4.0 * TK * 5),
-        3: ("hbm", 2.0 * TK * l * 2 + 4.0 * TK),
-        4: ("tensor", 2.0 * TK * l * (n_mats(cfg) - 1) * m),
-        5: ("tensor", 2.0 * TK * m * l),
-        6: ("hbm", 2.0 * TK * l + 8.0 * TK + 2.0 * T * l),
-        7: ("tensor", 2.0 * T * (l + ns * ms) * d),
+        0: (2.0 * T * d * (N + l), 2.0 * T * d + 2.0 * d * (N + l) + 4.0 * T * N + 2.0 * T * l),
+        1: (0.0, 4.0 * T * N + 8.0 * TK),
+        2: (0.0, 4.0 * TK * 5),
+        3: (0.0, 2.0 * TK * l * 2 + 4.0 * TK),
+        4: (2.0 * TK * l * gu * m, 2.0 * TK * l + 2.0 * E * gu * m * l + 2.0 * TK * m),
+        5: (2.0 * TK * m * l, 2.0 * TK * m + 2.0 * E * l * m + 2.0 * TK * l),
+        6: (0.0, 2.0 * TK * l + 8.0 * TK + 2.0 * T * l),
+        7: (2.0 * T * ky * d, 2.0 * T * ky + 2.0 * d * ky + 2.0 * T * d),
     }
+
+
+def stage_bound(flops, nbytes, peaks):
+    """'tensor' or 'hbm': whichever takes longer at the measured peaks."""
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    return "tensor" if t_tensor >= t_hbm else "hbm"
 
 
 def layer_flops(cfg):
@@ -272,20 +284,24 @@ def job_throughput(tokens_per_rank: int, world: int, max_ms_per_step: float) -> 
 
 
 # ---------------------------------------------------------------- our arm
-def traffic_from_profiles(kernel_key, sha):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+def traffic_from_profiles(kernel_key, workload_name, sha):
+    """DRAM bytes per launch of ``kernel_key`` on this workload from a
+    committed ncu summary, if it was taken on the current kernel source (else
+    None).  Summary lines read
+    ``traffic_bytes_per_launch[<kernel>@<workload>] = <bytes> source_sha256=<sha>``."""
     d = os.path.join(ROOT, "profiles")
     if not os.path.isdir(d):
         return None
-    pat = re.compile(r"traffic_bytes_per_launch\[(\w+)\]\s*=\s*([0-9.eE+]+)\s+source_sha256=(\w+)")
+    pat = re.compile(r"traffic_bytes_per_launch\[(\w+)@(\w+)\]\s*=\s*([0-9.eE+]+)"
+                     r"\s+source_sha256=(\w+)")
     for fn in sorted(os.listdir(d)):
         if not fn.endswith((".md", ".txt")):
             continue
         with open(os.path.join(d, fn)) as f:
             for mt in pat.finditer(f.read()):
-                if mt.group(1) == kernel_key and mt.group(3) == sha:
-                    return float(mt.group(2))
+                if (mt.group(1) == kernel_key and mt.group(2) == workload_name
+                        and mt.group(4) == sha):
+                    return float(mt.group(3))
     return None
 
 
@@ -368,25 +384,25 @@ def run_ours(args):
     value = job_throughput(cfg.T, world, ms_per_step)
 
     peaks, peak_src = load_peaks()
-    work = stage_work(cfg)
+    ids = layer.route(x)[0].cpu().numpy()
+    work = stage_work(cfg, touched=len(set(ids.reshape(-1).tolist())))
     avg_stage = [t / max(1, n_prof) for t in stage_ms]
     dom = max(range(len(avg_stage)), key=lambda i: avg_stage[i])
-    kind, amount = work[dom]
+    flops, nbytes = work[dom]
+    kind = stage_bound(flops, nbytes, peaks)
     if kind == "tensor":
+        amount, unit, peak = flops, "TFLOP/s", peaks["bf16_tflops"]
         achieved = amount / (avg_stage[dom] / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
-        unit = "TFLOP/s"
     else:
+        amount, unit, peak = nbytes, "GB/s", peaks["hbm_gbs"]
         achieved = amount / (avg_stage[dom] / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        unit = "GB/s"
     sha = kernel_source_sha()
-    traffic = traffic_from_profiles(lmoe.STAGE_NAMES[dom], sha)
+    traffic = traffic_from_profiles(lmoe.STAGE_NAMES[dom], cfg.name, sha)
     roofline = {"bound": kind, "kernel": lmoe.STAGE_NAMES[dom], "achieved": achieved,
                 "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} (burst)" if kind == "tensor" else peak_src,
-                "algorithmic_per_launch": amount, "avg_launch_ms": avg_stage[dom]}
-    ids = layer.route(x)[0].cpu().numpy()
+                "algorithmic_per_launch": amount, "algorithmic_flops": flops,
+                "algorithmic_bytes": nbytes, "avg_launch_ms": avg_stage[dom]}
     F, B = layer_flops(cfg), layer_bytes(cfg, ids)
     t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
     layer_roof = {"flops": F, "bytes": B, "roofline_ms": 1e3 * t_roof,

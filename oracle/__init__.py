@@ -1,4 +1,5 @@
-"""ctypes binding of the fp64 CPU oracle (``oracle/lmoe_oracle.c``).
+"""ctypes binding of the fp64 CPU oracle (``oracle/lmoe_oracle.c``): the
+LatentMoE layer forward and its backward.
 
 TEST INFRASTRUCTURE ONLY.  The oracle is what the CUDA library is checked
 against.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline /
@@ -79,6 +80,8 @@ def _load():
             lib.oracle_up.restype = None
             lib.oracle_shared.argtypes = [P, P, I64, P]
             lib.oracle_shared.restype = None
+            lib.oracle_backward.argtypes = [P, P, I64, P, I64, P, P, P]
+            lib.oracle_backward.restype = C.c_int
             lib.oracle_threads.argtypes = []
             lib.oracle_threads.restype = C.c_int
             _lib = lib
@@ -256,6 +259,51 @@ def shared(layer: Layer, x, t: int) -> np.ndarray:
     x = layer._x(x)
     out = np.empty(layer.d, dtype=np.float64)
     _load().oracle_shared(layer.cref, _ptr(x), t, _ptr(out))
+    return out
+
+
+class _Grads(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in (
+        "dx", "w_router", "b_router", "w_down", "w_up", "w_gate", "w_upx", "w_out",
+        "s_gate", "s_up", "s_out")]
+
+
+GRAD_NAMES = ("w_router", "b_router", "w_down", "w_up", "w_gate", "w_upx", "w_out",
+              "s_gate", "s_up", "s_out")
+
+
+def backward(layer: Layer, x, dy, tokens=None, ids=None, want=GRAD_NAMES):
+    """Gradients of the layer output for the cotangent dy (fp64).
+
+    dy [n][d] holds the cotangent of the listed tokens' outputs (all tokens if
+    tokens is None).  Weight gradients sum the listed tokens' contributions.
+    ids as in forward().  Returns a dict: "dx" [n][d] and each name in want
+    (weight-gradient arrays in the weights' shapes).
+    """
+    x = layer._x(x)
+    T = x.shape[0]
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+    n = T if tok is None else tok.shape[0]
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    assert dy.shape == (n, layer.d)
+    ids_in = None
+    if ids is not None:
+        ids_in = np.ascontiguousarray(ids, dtype=np.int32)
+        assert ids_in.shape == (T, layer.K)
+    shapes = {"w_router": (layer.N, layer.d), "b_router": (layer.N,),
+              "w_down": (layer.l, layer.d), "w_up": (layer.d, layer.l),
+              "w_gate": (layer.N, layer.m, layer.l), "w_upx": (layer.N, layer.m, layer.l),
+              "w_out": (layer.N, layer.l, layer.m),
+              "s_gate": (layer.n_s, layer.m_s, layer.d), "s_up": (layer.n_s, layer.m_s, layer.d),
+              "s_out": (layer.n_s, layer.d, layer.m_s)}
+    out = {"dx": np.empty((n, layer.d), dtype=np.float64)}
+    for k in want:
+        out[k] = np.zeros(shapes[k], dtype=np.float64)
+    g = _Grads(*[_ptr(out.get(k)) for k in ("dx",) + GRAD_NAMES])
+    rc = _load().oracle_backward(layer.cref, _ptr(x), T, _ptr(tok), n, _ptr(ids_in),
+                                 _ptr(dy), C.byref(g))
+    if rc != 0:
+        raise ValueError(f"oracle_backward failed ({rc})")
     return out
 
 

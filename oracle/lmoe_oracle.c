@@ -1,5 +1,6 @@
 /*
- * lmoe_oracle.c -- plain fp64 CPU oracle of the LatentMoE layer forward.
+ * lmoe_oracle.c -- plain fp64 CPU oracle of the LatentMoE layer forward and
+ * of its backward (the gradient for an output cotangent, after the forward).
  *
  * TEST INFRASTRUCTURE ONLY.  This file is what the CUDA library is checked
  * against; it is never part of the product path.  Only tests/, the smoke
@@ -313,6 +314,287 @@ int oracle_dispatch(const int32_t *ids, int64_t T, int K, int N,
   }
   offsets[N] = (int32_t)cursor;
   return cursor == T * (int64_t)K ? 0 : -1; /* -1: an id outside [0, N) */
+}
+
+/* ---- backward: the gradient of the layer output with respect to x and to
+ * every weight, for a given output cotangent dy (what loss.backward() of the
+ * [README] Usage example computes for this layer).  The pages state no
+ * formulas for it; it is the chain rule through steps 1-7 above, written
+ * out per token:
+ *   du   = W_up^T dy                         dW_up   += dy u^T
+ *   per slot k (expert e, gate g_k, hidden h_k, output o_k):
+ *     dg_k = du . o_k,  do_k = g_k du        dW_o[e] += do_k h_k^T
+ *     dh   = W_o[e]^T do_k
+ *     SwiGLU (a = W_g z, b = W_u z, h = silu(a) b):
+ *       da = dh * b * silu'(a),  db = dh * silu(a)
+ *     squared ReLU (b = W_u z, h = relu(b)^2):  db = dh * 2 relu(b)
+ *     dz  += W_g[e]^T da + W_u[e]^T db       dW_g[e] += da z^T, dW_u[e] += db z^T
+ *   gates g_k = p_{id_k} / sum p over the selected set = exp(s_{id_k}) /
+ *   sum_j exp(s_{id_j}); the selection itself is piecewise constant, so
+ *     ds_{id_k} = g_k (dg_k - sum_j g_j dg_j), ds_e = 0 for unselected e
+ *                                           dW_r += ds x^T, db_r += ds
+ *   dx = W_r^T ds + W_down^T dz + sum_j (S_g[j]^T da_j + S_u[j]^T db_j)
+ *                                           dW_down += dz x^T
+ *   shared expert j (input x, output added to y): dh_j = S_o[j]^T dy,
+ *     da_j, db_j as above                   dS_o[j] += dy h_j^T,
+ *                                           dS_g[j] += da_j x^T, dS_u[j] += db_j x^T
+ * silu'(a) = sigma(a) (1 + a (1 - sigma(a))), sigma(a) = 1 / (1 + e^-a).
+ * Weight gradients sum the listed tokens' contributions in token order. */
+typedef struct {
+  double *dx;        /* [n_tok][d], row n for token tokens[n] */
+  double *w_router;  /* [N'][d]      (each array may be NULL: not computed) */
+  double *b_router;  /* [N'] */
+  double *w_down;    /* [l][d] */
+  double *w_up;      /* [d][l] */
+  double *w_gate;    /* [N'][m][l] */
+  double *w_upx;     /* [N'][m][l] */
+  double *w_out;     /* [N'][l][m] */
+  double *s_gate;    /* [n_s][m_s][d] */
+  double *s_up;      /* [n_s][m_s][d] */
+  double *s_out;     /* [n_s][d][m_s] */
+} oracle_grads;
+
+static double dsilu(double a) {
+  const double sg = 1.0 / (1.0 + exp(-a));
+  return sg * (1.0 + a * (1.0 - sg));
+}
+
+/* Backward of one feed-forward (SwiGLU or squared ReLU) for input v, given
+ * dout: writes the hidden h and the pre-activation gradients da, db (da is
+ * zero for squared ReLU), and ADDS W_g^T da + W_u^T db to dv. */
+static void ffn_backward(const oracle_layer *L, const void *Wg, const void *Wu,
+                         const void *Wo, size_t off_in, size_t off_out, int in_w,
+                         int hid, int out_w, const double *v, const double *dout,
+                         double *h, double *da, double *db, double *dv,
+                         double *scratch /* 2*hid */) {
+  double *a = scratch, *b = scratch + hid;
+  const int dt = L->dtype;
+  matvec(Wu, dt, off_in, hid, in_w, v, b);
+  if (L->activation == OACT_RELU2) {
+    for (int c = 0; c < hid; ++c) h[c] = relu2(b[c]);
+  } else {
+    matvec(Wg, dt, off_in, hid, in_w, v, a);
+    for (int c = 0; c < hid; ++c) h[c] = silu(a[c]) * b[c];
+  }
+  for (int c = 0; c < hid; ++c) { /* dh[c] = sum_j W_o[j][c] dout[j] */
+    double dh = 0.0;
+    for (int j = 0; j < out_w; ++j)
+      dh += elem(Wo, dt, off_out + (size_t)j * hid + c) * dout[j];
+    if (L->activation == OACT_RELU2) {
+      da[c] = 0.0;
+      db[c] = dh * 2.0 * (b[c] > 0.0 ? b[c] : 0.0);
+    } else {
+      da[c] = dh * b[c] * dsilu(a[c]);
+      db[c] = dh * silu(a[c]);
+    }
+  }
+  for (int i = 0; i < in_w; ++i) {
+    double acc = 0.0;
+    for (int c = 0; c < hid; ++c) {
+      const size_t wi = off_in + (size_t)c * in_w + i;
+      if (L->activation != OACT_RELU2) acc += elem(Wg, dt, wi) * da[c];
+      acc += elem(Wu, dt, wi) * db[c];
+    }
+    dv[i] += acc;
+  }
+}
+
+int oracle_backward(const oracle_layer *L, const void *x, int64_t T,
+                    const int64_t *tokens, int64_t n_tok, const int32_t *ids_in,
+                    const double *dy, const oracle_grads *G) {
+  const int d = L->d, l = L->l, m = L->m, N = L->n_routed, K = L->k_active;
+  const int ns = L->n_shared, ms = L->m_shared > 0 ? L->m_shared : 1;
+  const int relu = L->activation == OACT_RELU2;
+  if (K < 1 || K > N || l < 1 || d < 1 || m < 1) return -1;
+  /* per-token and per-slot records for the weight-gradient sums */
+  double *X = (double *)malloc(sizeof(double) * (size_t)n_tok * d);
+  double *Z = (double *)malloc(sizeof(double) * (size_t)n_tok * l);
+  double *U = (double *)malloc(sizeof(double) * (size_t)n_tok * l);
+  double *DZ = (double *)malloc(sizeof(double) * (size_t)n_tok * l);
+  double *DS = (double *)malloc(sizeof(double) * (size_t)n_tok * K);
+  int32_t *ID = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_tok * K);
+  double *DO = (double *)malloc(sizeof(double) * (size_t)n_tok * K * l);
+  double *H = (double *)malloc(sizeof(double) * (size_t)n_tok * K * m);
+  double *DA = (double *)malloc(sizeof(double) * (size_t)n_tok * K * m);
+  double *DB = (double *)malloc(sizeof(double) * (size_t)n_tok * K * m);
+  double *HS = (double *)malloc(sizeof(double) * (size_t)n_tok * ns * ms + 1);
+  double *DAS = (double *)malloc(sizeof(double) * (size_t)n_tok * ns * ms + 1);
+  double *DBS = (double *)malloc(sizeof(double) * (size_t)n_tok * ns * ms + 1);
+  if (!X || !Z || !U || !DZ || !DS || !ID || !DO || !H || !DA || !DB || !HS || !DAS || !DBS) {
+    free(X); free(Z); free(U); free(DZ); free(DS); free(ID); free(DO); free(H);
+    free(DA); free(DB); free(HS); free(DAS); free(DBS);
+    return -3;
+  }
+  int err = 0;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *g = (double *)malloc(sizeof(double) * (size_t)K);
+    double *dg = (double *)malloc(sizeof(double) * (size_t)K);
+    double *du = (double *)malloc(sizeof(double) * (size_t)l);
+    double *eo = (double *)malloc(sizeof(double) * (size_t)l);
+    double *dxs = (double *)malloc(sizeof(double) * (size_t)d);
+    unsigned char *taken = (unsigned char *)malloc((size_t)N);
+    double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)(m > ms ? m : ms));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t n = 0; n < n_tok; ++n) {
+      const int64_t t = tokens ? tokens[n] : n;
+      if (t < 0 || t >= T) { err = -2; continue; }
+      double *xv = X + n * d, *z = Z + n * l, *u = U + n * l, *dz = DZ + n * l;
+      int32_t *ids = ID + n * K;
+      const double *dyr = dy + n * d;
+      router_row(L, x, L->dtype, t, s);
+      if (ids_in) {
+        memcpy(ids, ids_in + t * K, sizeof(int32_t) * (size_t)K);
+        gates_for_ids(s, N, K, ids, g);
+      } else {
+        select_row(s, N, K, ids, g, taken);
+      }
+      for (int i = 0; i < d; ++i) xv[i] = elem(x, L->dtype, (size_t)t * d + i);
+      matvec(L->w_down, L->dtype, 0, l, d, xv, z);
+      /* forward of the slots (o_k is recomputed by ffn_backward's h; keep u) */
+      for (int i = 0; i < l; ++i) u[i] = 0.0;
+      for (int k = 0; k < K; ++k) {
+        const int e = ids[k];
+        swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * m * l,
+                   (size_t)e * l * m, l, m, l, z, eo, scratch);
+        for (int i = 0; i < l; ++i) u[i] += g[k] * eo[i];
+        /* dg_k = du . o_k needs du first: o_k kept in DO for now */
+        memcpy(DO + (n * K + k) * l, eo, sizeof(double) * (size_t)l);
+      }
+      /* du = W_up^T dy */
+      for (int j = 0; j < l; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += elem(L->w_up, L->dtype, (size_t)i * l + j) * dyr[i];
+        du[j] = acc;
+      }
+      double gdg = 0.0;
+      for (int k = 0; k < K; ++k) {
+        double acc = 0.0;
+        const double *ok = DO + (n * K + k) * l;
+        for (int j = 0; j < l; ++j) acc += du[j] * ok[j];
+        dg[k] = acc;
+        gdg += g[k] * acc;
+      }
+      for (int i = 0; i < l; ++i) dz[i] = 0.0;
+      for (int k = 0; k < K; ++k) {
+        const int e = ids[k];
+        double *dok = DO + (n * K + k) * l;
+        for (int j = 0; j < l; ++j) dok[j] = g[k] * du[j];
+        ffn_backward(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * m * l, (size_t)e * l * m,
+                     l, m, l, z, dok, H + (n * K + k) * m, DA + (n * K + k) * m,
+                     DB + (n * K + k) * m, dz, scratch);
+        DS[n * K + k] = g[k] * (dg[k] - gdg);
+      }
+      /* dx = W_r^T ds + W_down^T dz + shared */
+      for (int i = 0; i < d; ++i) dxs[i] = 0.0;
+      for (int k = 0; k < K; ++k)
+        for (int i = 0; i < d; ++i)
+          dxs[i] += elem(L->w_router, L->dtype, (size_t)ids[k] * d + i) * DS[n * K + k];
+      for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < l; ++j) acc += elem(L->w_down, L->dtype, (size_t)j * d + i) * dz[j];
+        dxs[i] += acc;
+      }
+      for (int j = 0; j < ns; ++j)
+        ffn_backward(L, L->s_gate, L->s_up, L->s_out, (size_t)j * L->m_shared * d,
+                     (size_t)j * d * L->m_shared, d, L->m_shared, d, xv, dyr,
+                     HS + (n * ns + j) * ms, DAS + (n * ns + j) * ms, DBS + (n * ns + j) * ms,
+                     dxs, scratch);
+      if (G->dx) memcpy(G->dx + n * d, dxs, sizeof(double) * (size_t)d);
+    }
+    free(s); free(g); free(dg); free(du); free(eo); free(dxs); free(taken); free(scratch);
+  }
+  if (err) goto done;
+  /* weight gradients: each output element sums its tokens in token order */
+  if (G->w_up) {
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < l; ++j) {
+        double acc = 0.0;
+        for (int64_t n = 0; n < n_tok; ++n) acc += dy[n * d + i] * U[n * l + j];
+        G->w_up[(size_t)i * l + j] = acc;
+      }
+  }
+  if (G->w_down) {
+#pragma omp parallel for schedule(static)
+    for (int j = 0; j < l; ++j)
+      for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int64_t n = 0; n < n_tok; ++n) acc += DZ[n * l + j] * X[n * d + i];
+        G->w_down[(size_t)j * d + i] = acc;
+      }
+  }
+  if (G->w_router || G->b_router) {
+#pragma omp parallel for schedule(static)
+    for (int e = 0; e < N; ++e) {
+      double bacc = 0.0;
+      double *row = G->w_router ? G->w_router + (size_t)e * d : NULL;
+      if (row) for (int i = 0; i < d; ++i) row[i] = 0.0;
+      for (int64_t n = 0; n < n_tok; ++n)
+        for (int k = 0; k < K; ++k)
+          if (ID[n * K + k] == e) {
+            const double dsv = DS[n * K + k];
+            bacc += dsv;
+            if (row) for (int i = 0; i < d; ++i) row[i] += dsv * X[n * d + i];
+          }
+      if (G->b_router) G->b_router[e] = bacc;
+    }
+  }
+  if (G->w_out || G->w_gate || G->w_upx) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int e = 0; e < N; ++e) {
+      double *wo = G->w_out ? G->w_out + (size_t)e * l * m : NULL;
+      double *wg = G->w_gate ? G->w_gate + (size_t)e * m * l : NULL;
+      double *wu = G->w_upx ? G->w_upx + (size_t)e * m * l : NULL;
+      if (wo) memset(wo, 0, sizeof(double) * (size_t)l * m);
+      if (wg) memset(wg, 0, sizeof(double) * (size_t)m * l);
+      if (wu) memset(wu, 0, sizeof(double) * (size_t)m * l);
+      for (int64_t n = 0; n < n_tok; ++n)
+        for (int k = 0; k < K; ++k) {
+          if (ID[n * K + k] != e) continue;
+          const double *dok = DO + (n * K + k) * l, *hk = H + (n * K + k) * m;
+          const double *dak = DA + (n * K + k) * m, *dbk = DB + (n * K + k) * m;
+          const double *z = Z + n * l;
+          if (wo)
+            for (int j = 0; j < l; ++j)
+              for (int c = 0; c < m; ++c) wo[(size_t)j * m + c] += dok[j] * hk[c];
+          for (int c = 0; c < m; ++c)
+            for (int j = 0; j < l; ++j) {
+              if (wg && !relu) wg[(size_t)c * l + j] += dak[c] * z[j];
+              if (wu) wu[(size_t)c * l + j] += dbk[c] * z[j];
+            }
+        }
+    }
+  }
+  if (ns > 0 && (G->s_out || G->s_gate || G->s_up)) {
+    const int msr = L->m_shared;
+#pragma omp parallel for schedule(static)
+    for (int j = 0; j < ns; ++j) {
+      double *so = G->s_out ? G->s_out + (size_t)j * d * msr : NULL;
+      double *sg = G->s_gate ? G->s_gate + (size_t)j * msr * d : NULL;
+      double *su = G->s_up ? G->s_up + (size_t)j * msr * d : NULL;
+      if (so) memset(so, 0, sizeof(double) * (size_t)d * msr);
+      if (sg) memset(sg, 0, sizeof(double) * (size_t)msr * d);
+      if (su) memset(su, 0, sizeof(double) * (size_t)msr * d);
+      for (int64_t n = 0; n < n_tok; ++n) {
+        const double *hs = HS + (n * ns + j) * ms, *das = DAS + (n * ns + j) * ms;
+        const double *dbs = DBS + (n * ns + j) * ms, *xv = X + n * d, *dyr = dy + n * d;
+        if (so)
+          for (int i = 0; i < d; ++i)
+            for (int c = 0; c < msr; ++c) so[(size_t)i * msr + c] += dyr[i] * hs[c];
+        for (int c = 0; c < msr; ++c)
+          for (int i = 0; i < d; ++i) {
+            if (sg && !relu) sg[(size_t)c * d + i] += das[c] * xv[i];
+            if (su) su[(size_t)c * d + i] += dbs[c] * xv[i];
+          }
+      }
+    }
+  }
+done:
+  free(X); free(Z); free(U); free(DZ); free(DS); free(ID); free(DO); free(H);
+  free(DA); free(DB); free(HS); free(DAS); free(DBS);
+  return err;
 }
 
 int oracle_threads(void) {

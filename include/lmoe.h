@@ -86,6 +86,9 @@ typedef struct {
   int32_t has_router_bias;   /* 1: a float32 bias [N'] is added to the logits */
   int32_t max_tokens;        /* largest T any later call may pass */
   int32_t activation;        /* lmoe_activation */
+  int32_t training;          /* 1: lmoe_backward is available (the handle
+                                keeps the extra weight layouts and workspace
+                                the backward needs); 0: forward only */
 } lmoe_config;
 
 typedef struct lmoe_layer *lmoe_handle;
@@ -226,6 +229,37 @@ int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int32_t *n_forwards,
 #define LMOE_NOALLOC_MAX_EXPERTS 1024
 int lmoe_dispatch_noalloc(const int32_t *ids, int32_t T, int32_t k_active, int32_t n_routed,
                           int32_t *offsets, int32_t *perm, void *stream);
+
+/* Weight gradients of one lmoe_backward call: float32 device arrays in the
+ * layouts of lmoe_weights (w_router [N'][d], b_router [N'], w_down [l][d],
+ * w_up [d][l], w_gate / w_upx [N'][m][l], w_out [N'][l][m], s_gate / s_up
+ * [n_s][m_s][d], s_out [n_s][d][m_s]), caller-owned, overwritten (not
+ * accumulated).  b_router is required only with has_router_bias; w_gate and
+ * s_gate are unused (may be NULL) for LMOE_RELU2; s_* may be NULL when
+ * n_shared == 0. */
+typedef struct {
+  float *w_router, *b_router, *w_down, *w_up;
+  float *w_gate, *w_upx, *w_out;
+  float *s_gate, *s_up, *s_out;
+} lmoe_grads;
+
+/* The layer backward: for the cotangent dy_dev [T][d] of y = layer(x_dev),
+ * writes dx_dev [T][d] (element type cfg.dtype) and the weight gradients
+ * *grads -- what loss.backward() computes for this layer in the Latent-MoE
+ * README's Usage example.  The pages print no gradient formulas: it is the
+ * chain rule through the forward ("LatentMoE Explained": Figure 3 router,
+ * Figure 6 W_down / W_up, Figure 9 latent expert, the LatentMoE code
+ * module's softmax / top-K / renormalise and slot loop); the top-K
+ * selection is piecewise constant, so the router's gradient flows through
+ * the renormalised gates of the selected experts only.  Stateless: the call
+ * recomputes the forward activations it needs from x_dev (same routing as
+ * lmoe_forward).  Weight gradients sum the T tokens in a fixed order
+ * (deterministic).  Needs a handle created with training = 1.  No host
+ * sync; T == 0 writes zero gradients.  x, dy and dx must not overlap.
+ * Errors: NULL_ARG, NOT_LOADED, TOO_MANY_TOKENS, UNSUPPORTED (handle without
+ * training), CUDA. */
+int lmoe_backward(lmoe_handle h, const void *x_dev, const void *dy_dev, void *dx_dev,
+                  const lmoe_grads *grads, int32_t T, void *stream);
 
 /* Human-readable name of a status code (static string). */
 const char *lmoe_strerror(int code);

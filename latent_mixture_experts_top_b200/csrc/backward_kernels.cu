@@ -1,0 +1,299 @@
+// backward_kernels.cu -- kernels of the layer backward (the gradient for an
+// output cotangent dy), the steps that are not tensor-core GEMMs, plus the
+// fp32 CUDA-core GEMMs of the fp32 mode.
+//
+// The backward is the chain rule through the forward of "LatentMoE
+// Explained" (Figure 3 router, Figure 6 W_down / W_up, Figure 9 latent
+// expert, the LatentMoE code module's softmax / top-K / renormalise and slot
+// loop) for what loss.backward() of the Latent-MoE README's Usage example
+// computes: per token, du = W_up^T dy; per slot dg_k = du . o_k and
+// do_k = g_k du; the expert's hidden gradient; ds_{id_k} = g_k (dg_k -
+// sum_j g_j dg_j) through the renormalised gates; dz = sum over slots of the
+// expert input gradients; dx = W_r^T ds + W_down^T dz + the shared experts'.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lmoe {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float ld(const T *p, size_t i);
+template <>
+__device__ __forceinline__ float ld<float>(const float *p, size_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+template <typename T>
+__device__ __forceinline__ void st(T *p, size_t i, float v);
+template <>
+__device__ __forceinline__ void st<float>(float *p, size_t i, float v) { p[i] = v; }
+template <>
+__device__ __forceinline__ void st<__nv_bfloat16>(__nv_bfloat16 *p, size_t i, float v) {
+  p[i] = __float2bfloat16_rn(v);
+}
+
+// ---------------------------------------------------------------- fp32 GEMM
+// C[g](i, j) (+)= sum_k A[g](i, k) * B[g](j, k) with arbitrary strides, so
+// that transposed operands need no copies; optional per-group ranges of k
+// (grouped weight gradients: the rows of one expert) read from the device.
+constexpr int SBM = 64, SBN = 64, SBK = 16;
+
+__global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemm g) {
+  __shared__ float As[SBK][SBM + 1];
+  __shared__ float Bs[SBK][SBN + 1];
+  const int grp = blockIdx.z;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int r0 = blockIdx.y * SBM, c0 = blockIdx.x * SBN;
+  const float *A = g.A + grp * g.sA_g;
+  const float *B = g.B + grp * g.sB_g;
+  int k_begin = 0, k_end = g.K;
+  if (g.k_off) {
+    k_begin = g.k_off[grp];
+    k_end = g.k_off[grp + 1];
+  }
+  float acc[4][4] = {};
+  for (int k0 = k_begin; k0 < k_end; k0 += SBK) {
+    for (int i = threadIdx.x; i < SBM * SBK; i += 256) {
+      const int rr = i % SBM, kk = i / SBM;
+      const int r = r0 + rr, c = c0 + rr, k = k0 + kk;
+      As[kk][rr] = (r < g.M && k < k_end) ? A[r * g.sA_r + static_cast<long long>(k) * g.sA_k] : 0.0f;
+      Bs[kk][rr] = (c < g.N && k < k_end) ? B[c * g.sB_r + static_cast<long long>(k) * g.sB_k] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SBK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float *C = g.C + grp * g.sC_g;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty * 4 + i;
+    if (r >= g.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx * 4 + j;
+      if (c >= g.N) continue;
+      float *dst = C + r * g.ldc + c;
+      *dst = g.accumulate ? *dst + acc[i][j] : acc[i][j];
+    }
+  }
+}
+
+// C[r][c] (+)= sum_k A[r][k] * W(e, c, k), e = row_expert[r], W(e, c, k) at
+// W[e*sW_e + c*sW_r + k*sW_k]: expert products of permuted rows, any weight
+// orientation.
+__global__ void __launch_bounds__(256) simt_rowexpert_kernel(
+    const float *__restrict__ A, int lda, const float *__restrict__ W, long long sW_e,
+    long long sW_r, long long sW_k, const int32_t *__restrict__ row_expert,
+    float *__restrict__ C, int ldc, int M, int Ncols, int Kd, int accumulate) {
+  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
+  const int r = blockIdx.y * 4 + (threadIdx.x >> 6);
+  if (r >= M || c >= Ncols) return;
+  const float *a = A + static_cast<size_t>(r) * lda;
+  const float *w = W + row_expert[r] * sW_e + c * sW_r;
+  float acc = 0.0f;
+  for (int k = 0; k < Kd; ++k) acc = fmaf(a[k], w[k * sW_k], acc);
+  float *dst = C + static_cast<size_t>(r) * ldc + c;
+  *dst = accumulate ? *dst + acc : acc;
+}
+
+// ------------------------------------------------------- activation backward
+// Per element of [rows][n]: from the pre-activations a (gate), b (up) and the
+// hidden gradient dh, the hidden h and the pre-activation gradients.
+// SwiGLU: h = silu(a) b, da = dh b silu'(a), db = dh silu(a).
+// Squared ReLU: h = relu(b)^2, db = dh 2 relu(b) (a, da unused).
+// silu'(a) = sigma(a) (1 + a (1 - sigma(a))).
+template <typename TI, typename TO>
+__global__ void act_backward_kernel(const TI *__restrict__ a, const TI *__restrict__ b, int ldab,
+                                    const float *__restrict__ dh, int lddh, TO *__restrict__ h,
+                                    int ldh, TO *__restrict__ da, TO *__restrict__ db, int ldd,
+                                    int rows, int n, int relu2) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int r = blockIdx.y;
+  if (r >= rows || c >= n) return;
+  const float bv = ld(b, static_cast<size_t>(r) * ldab + c);
+  const float g = dh ? dh[static_cast<size_t>(r) * lddh + c] : 0.0f;
+  if (relu2) {
+    const float rb = fmaxf(bv, 0.0f);
+    if (h) st(h, static_cast<size_t>(r) * ldh + c, rb * rb);
+    if (db) st(db, static_cast<size_t>(r) * ldd + c, g * 2.0f * rb);
+  } else {
+    const float av = ld(a, static_cast<size_t>(r) * ldab + c);
+    const float sg = 1.0f / (1.0f + expf(-av));
+    const float sl = av * sg;
+    if (h) st(h, static_cast<size_t>(r) * ldh + c, sl * bv);
+    if (da) st(da, static_cast<size_t>(r) * ldd + c, g * bv * sg * (1.0f + av * (1.0f - sg)));
+    if (db) st(db, static_cast<size_t>(r) * ldd + c, g * sl);
+  }
+}
+
+// ------------------------------------------------------------ gate gradient
+// One warp per token t: dg_k = du_t . O[pos(t,k)], gamma = sum_k g_k dg_k,
+// ds_k = g_k (dg_k - gamma); and the expert-output gradient rows
+// DO[pos(t,k)] = g_k du_t.
+template <typename TO>
+__global__ void slot_grad_kernel(const float *__restrict__ du, int lddu,
+                                 const TO *__restrict__ O, int l, const int32_t *__restrict__ pos,
+                                 const float *__restrict__ gates, int T, int K,
+                                 float *__restrict__ ds, TO *__restrict__ DO) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const float *dur = du + static_cast<size_t>(t) * lddu;
+  float gamma = 0.0f;
+  for (int k = 0; k < K; ++k) {
+    const int p = pos[t * K + k];
+    const TO *o = O + static_cast<size_t>(p) * l;
+    float acc = 0.0f;
+    for (int j = lane; j < l; j += 32) acc = fmaf(dur[j], ld(o, j), acc);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+    const float g = gates[t * K + k];
+    gamma = fmaf(g, acc, gamma);
+    if (lane == 0) ds[t * K + k] = acc;  // dg_k for now
+    TO *dor = DO + static_cast<size_t>(p) * l;
+    for (int j = lane; j < l; j += 32) st(dor, j, g * dur[j]);
+  }
+  __syncwarp();
+  if (lane < K) {
+    for (int k = lane; k < K; k += 32) {
+      const float g = gates[t * K + k];
+      ds[t * K + k] = g * (ds[t * K + k] - gamma);
+    }
+  }
+}
+
+// dz[t][:] = sum_k D[pos(t,k)][:] in slot order (fp32 accumulation).
+template <typename TI, typename TO>
+__global__ void gather_sum_kernel(const TI *__restrict__ D, int ldD, const int32_t *__restrict__ pos,
+                                  int T, int K, int n, TO *__restrict__ out, int ldo) {
+  const int t = blockIdx.y;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T || c >= n) return;
+  float acc = 0.0f;
+  for (int k = 0; k < K; ++k) acc += ld(D, static_cast<size_t>(pos[t * K + k]) * ldD + c);
+  st(out, static_cast<size_t>(t) * ldo + c, acc);
+}
+
+// dS[t][e]: the router-logit gradient, ds at the selected experts, 0 elsewhere.
+template <typename TO>
+__global__ void scatter_ds_kernel(const float *__restrict__ ds, const int32_t *__restrict__ ids,
+                                  int T, int K, int N, TO *__restrict__ out, int ldo) {
+  const int t = blockIdx.x;
+  if (t >= T) return;
+  for (int e = threadIdx.x; e < N; e += blockDim.x) st(out, static_cast<size_t>(t) * ldo + e, 0.0f);
+  __syncthreads();
+  for (int k = threadIdx.x; k < K; k += blockDim.x)
+    st(out, static_cast<size_t>(t) * ldo + ids[t * K + k], ds[t * K + k]);
+}
+
+// db_r[e] = sum of ds over the (token, slot) pairs of expert e, in token
+// order (the dispatch's perm lists them so).
+__global__ void bias_grad_kernel(const float *__restrict__ ds, const int32_t *__restrict__ offsets,
+                                 const int32_t *__restrict__ perm, int N, float *__restrict__ db) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= N) return;
+  float acc = 0.0f;
+  for (int p = offsets[e]; p < offsets[e + 1]; ++p) acc += ds[perm[p]];
+  db[e] = acc;
+}
+
+}  // namespace
+
+cudaError_t simt_gemm(const SimtGemm &g, int groups, cudaStream_t s) {
+  if (g.M <= 0 || g.N <= 0 || groups <= 0) return cudaSuccess;
+  dim3 grid((g.N + SBN - 1) / SBN, (g.M + SBM - 1) / SBM, groups);
+  simt_gemm_kernel<<<grid, 256, 0, s>>>(g);
+  return cudaGetLastError();
+}
+
+cudaError_t simt_rowexpert(const float *A, int lda, const float *W, long long sW_e, long long sW_r,
+                           long long sW_k, const int32_t *row_expert, float *C, int ldc, int M,
+                           int Ncols, int Kdim, bool accumulate, cudaStream_t s) {
+  if (M <= 0 || Ncols <= 0) return cudaSuccess;
+  dim3 grid((Ncols + 63) / 64, (M + 3) / 4);
+  simt_rowexpert_kernel<<<grid, 256, 0, s>>>(A, lda, W, sW_e, sW_r, sW_k, row_expert, C, ldc, M,
+                                             Ncols, Kdim, accumulate ? 1 : 0);
+  return cudaGetLastError();
+}
+
+template <typename TI, typename TO>
+cudaError_t launch_act_backward(const TI *a, const TI *b, int ldab, const float *dh, int lddh,
+                                TO *h, int ldh, TO *da, TO *db, int ldd, int rows, int n,
+                                bool relu2, cudaStream_t s) {
+  if (rows <= 0 || n <= 0) return cudaSuccess;
+  dim3 grid((n + 255) / 256, rows);
+  act_backward_kernel<TI, TO><<<grid, 256, 0, s>>>(a, b, ldab, dh, lddh, h, ldh, da, db, ldd, rows,
+                                                   n, relu2 ? 1 : 0);
+  return cudaGetLastError();
+}
+template cudaError_t launch_act_backward<float, float>(const float *, const float *, int,
+                                                       const float *, int, float *, int, float *,
+                                                       float *, int, int, int, bool, cudaStream_t);
+template cudaError_t launch_act_backward<__nv_bfloat16, __nv_bfloat16>(
+    const __nv_bfloat16 *, const __nv_bfloat16 *, int, const float *, int, __nv_bfloat16 *, int,
+    __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, bool, cudaStream_t);
+
+template <typename TO>
+cudaError_t launch_slot_grad(const float *du, int lddu, const TO *O, int l, const int32_t *pos,
+                             const float *gates, int T, int K, float *ds, TO *DO, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  slot_grad_kernel<TO><<<(T + 7) / 8, 256, 0, s>>>(du, lddu, O, l, pos, gates, T, K, ds, DO);
+  return cudaGetLastError();
+}
+template cudaError_t launch_slot_grad<float>(const float *, int, const float *, int,
+                                             const int32_t *, const float *, int, int, float *,
+                                             float *, cudaStream_t);
+template cudaError_t launch_slot_grad<__nv_bfloat16>(const float *, int, const __nv_bfloat16 *, int,
+                                                     const int32_t *, const float *, int, int,
+                                                     float *, __nv_bfloat16 *, cudaStream_t);
+
+template <typename TI, typename TO>
+cudaError_t launch_gather_sum(const TI *D, int ldD, const int32_t *pos, int T, int K, int n, TO *out,
+                              int ldo, cudaStream_t s) {
+  if (T <= 0 || n <= 0) return cudaSuccess;
+  dim3 grid((n + 127) / 128, T);
+  gather_sum_kernel<TI, TO><<<grid, 128, 0, s>>>(D, ldD, pos, T, K, n, out, ldo);
+  return cudaGetLastError();
+}
+template cudaError_t launch_gather_sum<float, float>(const float *, int, const int32_t *, int, int,
+                                                     int, float *, int, cudaStream_t);
+template cudaError_t launch_gather_sum<float, __nv_bfloat16>(const float *, int, const int32_t *,
+                                                             int, int, int, __nv_bfloat16 *, int,
+                                                             cudaStream_t);
+
+template <typename TO>
+cudaError_t launch_scatter_ds(const float *ds, const int32_t *ids, int T, int K, int N, TO *out,
+                              int ldo, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  scatter_ds_kernel<TO><<<T, 128, 0, s>>>(ds, ids, T, K, N, out, ldo);
+  return cudaGetLastError();
+}
+template cudaError_t launch_scatter_ds<float>(const float *, const int32_t *, int, int, int, float *,
+                                              int, cudaStream_t);
+template cudaError_t launch_scatter_ds<__nv_bfloat16>(const float *, const int32_t *, int, int, int,
+                                                      __nv_bfloat16 *, int, cudaStream_t);
+
+cudaError_t launch_bias_grad(const float *ds, const int32_t *offsets, const int32_t *perm, int N,
+                             float *db, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  bias_grad_kernel<<<(N + 127) / 128, 128, 0, s>>>(ds, offsets, perm, N, db);
+  return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -113,6 +113,46 @@ cudaError_t launch_repack_btiles(const __nv_bfloat16 *src, int groups, int rows_
 int make_tmap_bf16(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
                    int64_t cols, int64_t row_stride_elems, int box_rows);
 
+// ---- backward (backward_kernels.cu)
+// fp32 CUDA-core GEMM with arbitrary strides: C[g](i, j) (+)= sum_k
+// A[g](i, k) B[g](j, k), X[g](r, k) at X + g*sX_g + r*sX_r + k*sX_k; k runs
+// over [0, K), or over [k_off[g], k_off[g+1]) when k_off (device) is set.
+struct SimtGemm {
+  const float *A; long long sA_g, sA_r, sA_k;
+  const float *B; long long sB_g, sB_r, sB_k;
+  float *C; long long sC_g, ldc;
+  int M, N, K;
+  const int32_t *k_off;
+  int accumulate;
+};
+cudaError_t simt_gemm(const SimtGemm &g, int groups, cudaStream_t s);
+// C[r][c] (+)= sum_k A[r][k] W[e*sW_e + c*sW_r + k*sW_k], e = row_expert[r].
+cudaError_t simt_rowexpert(const float *A, int lda, const float *W, long long sW_e, long long sW_r,
+                           long long sW_k, const int32_t *row_expert, float *C, int ldc, int M,
+                           int Ncols, int Kdim, bool accumulate, cudaStream_t s);
+// From pre-activations a (gate; unused for squared ReLU), b (up) and the
+// hidden gradient dh (may be null: h only): h, da, db (each may be null).
+template <typename TI, typename TO>
+cudaError_t launch_act_backward(const TI *a, const TI *b, int ldab, const float *dh, int lddh,
+                                TO *h, int ldh, TO *da, TO *db, int ldd, int rows, int n,
+                                bool relu2, cudaStream_t s);
+// Per token: ds[t][k] = g_k (du_t . O[pos] - sum_j g_j du_t . O[pos_j]) and
+// DO[pos(t,k)] = g_k du_t.
+template <typename TO>
+cudaError_t launch_slot_grad(const float *du, int lddu, const TO *O, int l, const int32_t *pos,
+                             const float *gates, int T, int K, float *ds, TO *DO, cudaStream_t s);
+// out[t][:n] = sum_k D[pos(t,k)][:n], slot order.
+template <typename TI, typename TO>
+cudaError_t launch_gather_sum(const TI *D, int ldD, const int32_t *pos, int T, int K, int n, TO *out,
+                              int ldo, cudaStream_t s);
+// out[t][e] = ds of the slot that selected e, 0 for unselected e (e < N).
+template <typename TO>
+cudaError_t launch_scatter_ds(const float *ds, const int32_t *ids, int T, int K, int N, TO *out,
+                              int ldo, cudaStream_t s);
+// db[e] = sum of ds over expert e's pairs, token order.
+cudaError_t launch_bias_grad(const float *ds, const int32_t *offsets, const int32_t *perm, int N,
+                             float *db, cudaStream_t s);
+
 // Failure-detection self-test (see lmoe_selftest_wait_timeout).
 cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s);
 

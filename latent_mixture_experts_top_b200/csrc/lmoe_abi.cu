@@ -42,6 +42,21 @@ struct Workspace {
   int32_t *status = nullptr;
 };
 
+// Backward workspace (handles created with training = 1), sized for Tmax.
+struct BwdWorkspace {
+  void *a = nullptr, *b = nullptr;      // [TK][m] expert pre-activations (gate, up)
+  float *dU = nullptr;                  // [T][ky] dy . [W_up | S_o]
+  float *ds = nullptr;                  // [TK] router-logit gradient per slot
+  void *DO = nullptr;                   // [TK][l] expert-output gradient (permuted)
+  float *dH = nullptr;                  // [TK][m]
+  void *dA = nullptr, *dB = nullptr;    // [TK][m]
+  float *dZp = nullptr;                 // [TK][l]
+  float *dz = nullptr;                  // [T][l]
+  void *as = nullptr, *bs = nullptr;    // [T][ns ms] shared pre-activations
+  void *das = nullptr, *dbs = nullptr;  // [T][ns ms]
+  float *dsfull = nullptr;              // [T][N']
+};
+
 }  // namespace
 
 struct lmoe_layer {
@@ -68,6 +83,8 @@ struct lmoe_layer {
   void *s_gate = nullptr, *s_up = nullptr;   // f32 path: [ns][ms][d]
   void *w_y = nullptr;       // [d][l + ns ms] = [W_up | S_o(0) | S_o(1) ...]
   Workspace ws;
+  BwdWorkspace bw;
+  bool training = false;
   // profiling: a ring of event sets (LMOE_NUM_STAGES + 1 per forward)
   int prof_slots = 0;
   int64_t prof_count = 0;     // forwards recorded since profiling was enabled
@@ -109,7 +126,9 @@ void free_all(lmoe_layer *h) {
                   h->w_out, h->s_gate, h->s_up, h->w_y, h->ws.logits, h->ws.ids, h->ws.gates,
                   h->ws.chunk_counts, h->ws.offsets, h->ws.perm, h->ws.pos, h->ws.row_expert,
                   h->ws.tiles, h->ws.n_tiles, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
-                  h->ws.x_stage, h->ws.y_stage, h->ws.status};
+                  h->ws.x_stage, h->ws.y_stage, h->ws.status, h->bw.a, h->bw.b, h->bw.dU,
+                  h->bw.ds, h->bw.DO, h->bw.dH, h->bw.dA, h->bw.dB, h->bw.dZp, h->bw.dz,
+                  h->bw.as, h->bw.bs, h->bw.das, h->bw.dbs, h->bw.dsfull};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
@@ -241,6 +260,17 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
            dalloc(&h->w_y, d * h->ky * es);
     }
     if (ok && cfg->has_router_bias) ok = dalloc(&h->b_router, N * 4);
+  }
+  h->training = cfg->training != 0;
+  if (ok && h->training) {
+    BwdWorkspace &b = h->bw;
+    const size_t nsms = static_cast<size_t>(h->ns) * h->ms;
+    ok = dalloc(&b.a, TK * m * es) && dalloc(&b.b, TK * m * es) &&
+         dalloc(&b.dU, T * h->ky * 4) && dalloc(&b.ds, TK * 4) && dalloc(&b.DO, TK * l * es) &&
+         dalloc(&b.dH, TK * m * 4) && dalloc(&b.dA, TK * m * es) && dalloc(&b.dB, TK * m * es) &&
+         dalloc(&b.dZp, TK * l * 4) && dalloc(&b.dz, T * l * 4) && dalloc(&b.as, T * nsms * es) &&
+         dalloc(&b.bs, T * nsms * es) && dalloc(&b.das, T * nsms * es) &&
+         dalloc(&b.dbs, T * nsms * es) && dalloc(&b.dsfull, T * N * 4);
   }
   if (!ok) {
     cudaGetLastError();
@@ -601,6 +631,141 @@ int lmoe_forward(lmoe_handle h, const void *x, void *y, int32_t T, void *stream)
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
   return forward_impl(h, x, y, T, static_cast<cudaStream_t>(stream));
+}
+
+// ---- backward (see the declaration of lmoe_backward): fp32 mode on CUDA cores.
+static SimtGemm sg_dense(const float *A, long long sA_r, long long sA_k, const float *B,
+                         long long sB_r, long long sB_k, float *C, long long ldc, int M, int N,
+                         int K, bool accumulate) {
+  SimtGemm q = {};
+  q.A = A; q.sA_r = sA_r; q.sA_k = sA_k;
+  q.B = B; q.sB_r = sB_r; q.sB_k = sB_k;
+  q.C = C; q.ldc = ldc;
+  q.M = M; q.N = N; q.K = K;
+  q.accumulate = accumulate ? 1 : 0;
+  return q;
+}
+
+static cudaError_t backward_f32(lmoe_layer *h, const float *x, const float *dy, float *dx,
+                                const lmoe_grads *g, int T, cudaStream_t s) {
+  Workspace &w = h->ws;
+  BwdWorkspace &b = h->bw;
+  const int d = h->d, l = h->l, m = h->m, N = h->N, K = h->K, ky = h->ky;
+  const int nsms = h->ns * h->ms, TK = T * K;
+  const bool relu2 = h->relu2 != 0;
+  const float *Wr = static_cast<const float *>(h->w_router);
+  const float *Wd = static_cast<const float *>(h->w_down);
+  const float *Wg = static_cast<const float *>(h->w_gate);
+  const float *Wu = static_cast<const float *>(h->w_upx);
+  const float *Wo = static_cast<const float *>(h->w_out);
+  const float *Sg = static_cast<const float *>(h->s_gate);
+  const float *Su = static_cast<const float *>(h->s_up);
+  const float *Wy = static_cast<const float *>(h->w_y);
+  float *zp = static_cast<float *>(w.zp), *H = static_cast<float *>(w.H);
+  float *O = static_cast<float *>(w.O), *ucat = static_cast<float *>(w.ucat);
+  float *A_ = static_cast<float *>(b.a), *B_ = static_cast<float *>(b.b);
+  float *DO = static_cast<float *>(b.DO), *dA = static_cast<float *>(b.dA);
+  float *dB = static_cast<float *>(b.dB);
+  float *as = static_cast<float *>(b.as), *bs = static_cast<float *>(b.bs);
+  float *das = static_cast<float *>(b.das), *dbs = static_cast<float *>(b.dbs);
+  int64_t &L = h->launches;
+#define LMOE_TRY(...) do { cudaError_t e_ = (__VA_ARGS__); ++L; if (e_ != cudaSuccess) return e_; } while (0)
+  // forward activations: routing, z, shared hidden, expert pre-activations, H, O, u
+  cudaError_t e = run_route(h, x, T, true, s);
+  if (e != cudaSuccess) return e;
+  LMOE_TRY(launch_permute_rows(w.z, w.perm, K, TK, l * 4, w.zp, s));
+  if (!relu2) LMOE_TRY(simt_rowexpert(zp, l, Wg, 1LL * m * l, l, 1, w.row_expert, A_, m, TK, m, l, false, s));
+  LMOE_TRY(simt_rowexpert(zp, l, Wu, 1LL * m * l, l, 1, w.row_expert, B_, m, TK, m, l, false, s));
+  LMOE_TRY(launch_act_backward<float, float>(A_, B_, m, nullptr, 0, H, m, nullptr, nullptr, 0, TK,
+                                             m, relu2, s));
+  LMOE_TRY(simt_expert_down(H, m, Wo, w.row_expert, O, l, TK, l, m, s));
+  LMOE_TRY(launch_combine(O, w.pos, w.gates, T, K, l, ucat, ky, false, s));
+  // du | dh_s = dy . [W_up | S_o]   (C[t][c] = sum_i dy[t][i] W_y[i][c])
+  LMOE_TRY(simt_gemm(sg_dense(dy, d, 1, Wy, 1, ky, b.dU, ky, T, ky, d, false), 1, s));
+  // gate gradients and the expert-output gradients
+  LMOE_TRY(launch_slot_grad<float>(b.dU, ky, O, l, w.pos, w.gates, T, K, b.ds, DO, s));
+  // dH[p][c] = sum_j DO[p][j] W_o[e][j][c]
+  LMOE_TRY(simt_rowexpert(DO, l, Wo, 1LL * l * m, 1, m, w.row_expert, b.dH, m, TK, m, l, false, s));
+  LMOE_TRY(launch_act_backward<float, float>(A_, B_, m, b.dH, m, nullptr, 0, dA, dB, m, TK, m,
+                                             relu2, s));
+  // dZp[p][j] = sum_c dA[p][c] W_g[e][c][j] + dB[p][c] W_u[e][c][j]
+  if (!relu2) LMOE_TRY(simt_rowexpert(dA, m, Wg, 1LL * m * l, 1, l, w.row_expert, b.dZp, l, TK, l, m, false, s));
+  LMOE_TRY(simt_rowexpert(dB, m, Wu, 1LL * m * l, 1, l, w.row_expert, b.dZp, l, TK, l, m, !relu2, s));
+  LMOE_TRY(launch_gather_sum<float, float>(b.dZp, l, w.pos, T, K, l, b.dz, l, s));
+  // shared experts: pre-activations and their gradients (dh_s = dU[:, l:])
+  if (nsms > 0) {
+    if (!relu2) LMOE_TRY(simt_gemm(sg_dense(x, d, 1, Sg, d, 1, as, nsms, T, nsms, d, false), 1, s));
+    LMOE_TRY(simt_gemm(sg_dense(x, d, 1, Su, d, 1, bs, nsms, T, nsms, d, false), 1, s));
+    LMOE_TRY(launch_act_backward<float, float>(as, bs, nsms, b.dU + l, ky, nullptr, 0, das, dbs,
+                                               nsms, T, nsms, relu2, s));
+  }
+  LMOE_TRY(launch_scatter_ds<float>(b.ds, w.ids, T, K, N, b.dsfull, N, s));
+  // dx = dz W_down + dS W_r + da_s S_g + db_s S_u
+  LMOE_TRY(simt_gemm(sg_dense(b.dz, l, 1, Wd, 1, d, dx, d, T, d, l, false), 1, s));
+  LMOE_TRY(simt_gemm(sg_dense(b.dsfull, N, 1, Wr, 1, d, dx, d, T, d, N, true), 1, s));
+  if (nsms > 0) {
+    if (!relu2) LMOE_TRY(simt_gemm(sg_dense(das, nsms, 1, Sg, 1, d, dx, d, T, d, nsms, true), 1, s));
+    LMOE_TRY(simt_gemm(sg_dense(dbs, nsms, 1, Su, 1, d, dx, d, T, d, nsms, true), 1, s));
+  }
+  // weight gradients, dense: K runs over the T tokens in order
+  LMOE_TRY(simt_gemm(sg_dense(dy, 1, d, ucat, 1, ky, g->w_up, l, d, l, T, false), 1, s));
+  if (nsms > 0) {
+    SimtGemm q = sg_dense(dy, 1, d, ucat + l, 1, ky, g->s_out, h->ms, d, h->ms, T, false);
+    q.sB_g = h->ms;
+    q.sC_g = 1LL * d * h->ms;
+    LMOE_TRY(simt_gemm(q, h->ns, s));
+    if (!relu2) LMOE_TRY(simt_gemm(sg_dense(das, 1, nsms, x, 1, d, g->s_gate, d, nsms, d, T, false), 1, s));
+    LMOE_TRY(simt_gemm(sg_dense(dbs, 1, nsms, x, 1, d, g->s_up, d, nsms, d, T, false), 1, s));
+  }
+  LMOE_TRY(simt_gemm(sg_dense(b.dz, 1, l, x, 1, d, g->w_down, d, l, d, T, false), 1, s));
+  LMOE_TRY(simt_gemm(sg_dense(b.dsfull, 1, N, x, 1, d, g->w_router, d, N, d, T, false), 1, s));
+  if (g->b_router) LMOE_TRY(launch_bias_grad(b.ds, w.offsets, w.perm, N, g->b_router, s));
+  // weight gradients, grouped: K runs over expert e's permuted rows
+  {
+    SimtGemm q = sg_dense(DO, 1, l, H, 1, m, g->w_out, m, l, m, 0, false);
+    q.k_off = w.offsets;
+    q.sC_g = 1LL * l * m;
+    LMOE_TRY(simt_gemm(q, N, s));
+    q = sg_dense(dB, 1, m, zp, 1, l, g->w_upx, l, m, l, 0, false);
+    q.k_off = w.offsets;
+    q.sC_g = 1LL * m * l;
+    LMOE_TRY(simt_gemm(q, N, s));
+    if (!relu2) {
+      q.A = dA;
+      q.C = g->w_gate;
+      LMOE_TRY(simt_gemm(q, N, s));
+    }
+  }
+#undef LMOE_TRY
+  return cudaSuccess;
+}
+
+int lmoe_backward(lmoe_handle h, const void *x, const void *dy, void *dx, const lmoe_grads *g,
+                  int32_t T, void *stream) {
+  int rc = check_call(h, T);
+  if (rc != LMOE_OK) return rc;
+  if (!h->training) return LMOE_ERR_UNSUPPORTED;
+  if (!g || !g->w_router || !g->w_down || !g->w_up || !g->w_upx || !g->w_out)
+    return LMOE_ERR_NULL_ARG;
+  if (!h->relu2 && !g->w_gate) return LMOE_ERR_NULL_ARG;
+  if (h->cfg.has_router_bias && !g->b_router) return LMOE_ERR_NULL_ARG;
+  if (h->ns > 0 && (!g->s_up || !g->s_out || (!h->relu2 && !g->s_gate))) return LMOE_ERR_NULL_ARG;
+  if (T > 0 && (!x || !dy || !dx)) return LMOE_ERR_NULL_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t N = h->N, d = h->d, l = h->l, m = h->m, nsms = static_cast<size_t>(h->ns) * h->ms;
+  if (T == 0) {  // no tokens: every gradient is zero
+    cudaError_t e = cudaSuccess;
+    auto z = [&](float *p, size_t n) { if (p && e == cudaSuccess) e = cudaMemsetAsync(p, 0, n * 4, s); };
+    z(g->w_router, N * d); z(g->b_router, N); z(g->w_down, l * d); z(g->w_up, d * l);
+    z(g->w_gate, N * m * l); z(g->w_upx, N * m * l); z(g->w_out, N * l * m);
+    z(g->s_gate, nsms * d); z(g->s_up, nsms * d); z(g->s_out, d * nsms);
+    return cuda_err(e);
+  }
+  if (h->bf16) return LMOE_ERR_UNSUPPORTED;
+  return cuda_err(backward_f32(h, static_cast<const float *>(x), static_cast<const float *>(dy),
+                               static_cast<float *>(dx), g, T, s));
 }
 
 int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T, void *stream) {

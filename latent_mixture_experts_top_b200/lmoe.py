@@ -31,7 +31,7 @@ STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
 EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
             "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
             "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc",
-            "lmoe_selftest_wait_timeout", "lmoe_strerror", "lmoe_destroy")
+            "lmoe_selftest_wait_timeout", "lmoe_backward", "lmoe_strerror", "lmoe_destroy")
 LMOE_NUM_STAGES = 8
 STAGE_NAMES = ("x_gemm_router_down", "topk", "dispatch", "permute_z",
                "expert_gate_up_gemm", "expert_down_gemm", "combine", "out_gemm")
@@ -40,13 +40,22 @@ STAGE_NAMES = ("x_gemm_router_down", "topk", "dispatch", "permute_z",
 class lmoe_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "d", "m", "n_experts", "top_k", "alpha", "n_shared", "m_shared", "variant", "dtype",
-        "n_routed_override", "top_k_override", "has_router_bias", "max_tokens", "activation")]
+        "n_routed_override", "top_k_override", "has_router_bias", "max_tokens", "activation",
+        "training")]
 
 
 class lmoe_weights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in (
         "w_router", "b_router", "w_down", "w_up", "w_gate", "w_upx", "w_out", "s_gate",
         "s_up", "s_out")]
+
+
+GRAD_NAMES = ("w_router", "b_router", "w_down", "w_up", "w_gate", "w_upx", "w_out", "s_gate",
+              "s_up", "s_out")
+
+
+class lmoe_grads(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in GRAD_NAMES]
 
 
 P, I32 = C.c_void_p, C.c_int32
@@ -63,6 +72,7 @@ _lib.lmoe_stage_times.argtypes = [P, C.POINTER(C.c_float), I32, C.POINTER(I32),
                                   C.POINTER(C.c_int64)]
 _lib.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P]
 _lib.lmoe_selftest_wait_timeout.argtypes = [P, C.c_int64, P]
+_lib.lmoe_backward.argtypes = [P, P, P, P, C.POINTER(lmoe_grads), I32, P]
 _lib.lmoe_strerror.argtypes = [C.c_int]
 _lib.lmoe_strerror.restype = C.c_char_p
 _lib.lmoe_destroy.argtypes = [P]
@@ -106,7 +116,8 @@ def lmoe_strerror(code: int) -> str:
     return _lib.lmoe_strerror(code).decode()
 
 
-def config_from(cfg: LayerConfig, max_tokens: int | None = None) -> lmoe_config:
+def config_from(cfg: LayerConfig, max_tokens: int | None = None,
+                training: bool = False) -> lmoe_config:
     return lmoe_config(
         d=cfg.d, m=cfg.m, n_experts=cfg.n_experts, top_k=cfg.top_k, alpha=cfg.alpha,
         n_shared=cfg.n_shared, m_shared=cfg.m_shared,
@@ -115,7 +126,8 @@ def config_from(cfg: LayerConfig, max_tokens: int | None = None) -> lmoe_config:
         n_routed_override=cfg.n_routed_override, top_k_override=cfg.top_k_override,
         has_router_bias=int(cfg.has_router_bias),
         max_tokens=cfg.T if max_tokens is None else max_tokens,
-        activation=LMOE_RELU2 if cfg.activation == "relu2" else LMOE_SWIGLU)
+        activation=LMOE_RELU2 if cfg.activation == "relu2" else LMOE_SWIGLU,
+        training=int(training))
 
 
 def lmoe_create(config: lmoe_config) -> int:
@@ -193,6 +205,14 @@ def lmoe_selftest_wait_timeout(handle: int, limit_ns: int, stream=None) -> None:
            "lmoe_selftest_wait_timeout")
 
 
+def lmoe_backward(handle: int, x, dy, dx, grads: dict, T: int, stream=None) -> None:
+    """dx and the weight gradients (dict of float32 device tensors named as
+    GRAD_NAMES; absent names pass NULL) for the cotangent dy of layer(x)."""
+    g = lmoe_grads(**{k: _ptr(grads.get(k)) for k in GRAD_NAMES})
+    _check(_lib.lmoe_backward(handle, _ptr(x), _ptr(dy), _ptr(dx), C.byref(g), T,
+                              _stream(stream)), "lmoe_backward")
+
+
 def lmoe_destroy(handle: int) -> None:
     _check(_lib.lmoe_destroy(handle), "lmoe_destroy")
 
@@ -205,9 +225,9 @@ class LatentMoELayer:
     """
 
     def __init__(self, cfg: LayerConfig, weights: dict, max_tokens: int | None = None,
-                 stream=None):
+                 stream=None, training: bool = False):
         self.cfg = cfg
-        self.handle = lmoe_create(config_from(cfg, max_tokens))
+        self.handle = lmoe_create(config_from(cfg, max_tokens, training))
         try:
             lmoe_load_weights(self.handle, weights, stream)
         except Exception:
@@ -222,6 +242,30 @@ class LatentMoELayer:
             y = torch.empty_like(x)
         lmoe_forward(self.handle, x, y, T, stream)
         return y
+
+    def grad_shapes(self) -> dict:
+        c = self.cfg
+        N, d, l, m, ns, ms = self.n_routed, c.d, self.l, c.m, c.n_shared, c.m_shared
+        shapes = {"w_router": (N, d), "w_down": (l, d), "w_up": (d, l), "w_upx": (N, m, l),
+                  "w_out": (N, l, m)}
+        if c.activation != "relu2":
+            shapes["w_gate"] = (N, m, l)
+        if c.has_router_bias:
+            shapes["b_router"] = (N,)
+        if ns > 0:
+            shapes.update(s_up=(ns, ms, d), s_out=(ns, d, ms))
+            if c.activation != "relu2":
+                shapes["s_gate"] = (ns, ms, d)
+        return shapes
+
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, stream=None):
+        """(dx, dict of float32 weight gradients) for the cotangent dy."""
+        T = x.shape[0]
+        dx = torch.empty_like(x)
+        grads = {k: torch.empty(v, dtype=torch.float32, device=x.device)
+                 for k, v in self.grad_shapes().items()}
+        lmoe_backward(self.handle, x, dy, dx, grads, T, stream)
+        return dx, grads
 
     def route(self, x: torch.Tensor, stream=None):
         T = x.shape[0]

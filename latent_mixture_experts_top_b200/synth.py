@@ -71,6 +71,18 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, device: str | torch.device = "c
     return out
 
 
+def make_cotangent(cfg: LayerConfig, seed: int = 0, device: str | torch.device = "cpu",
+                   T: int | None = None) -> torch.Tensor:
+    """dy [T][d] ~ N(0, 1) in the layer's element type, from its own generator
+    (seed + 1000003), so that x and the weights keep their draws."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 1000003)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    T = cfg.T if T is None else T
+    return _normal(gen, (T, cfg.d), 1.0, dt, device)
+
+
 def to_numpy(t: torch.Tensor):
     """Host numpy copy; bf16 becomes its raw uint16 bit pattern (exact)."""
     t = t.detach().cpu().contiguous()

@@ -1,0 +1,90 @@
+"""GPU parity of the layer backward (lmoe_backward) against the fp64 oracle.
+
+Inputs and the cotangent dy come from latent_mixture_experts_top_b200.synth.
+The routing is checked as in the forward parity tests; the oracle then takes
+the library's own ids (identical off near-ties), so that both sides
+differentiate the same piecewise-smooth branch.  Every array -- dx and each
+weight gradient -- is compared as max|g - g_ref| / max|g_ref| against the
+mode's tolerance: 1e-5 for fp32 (fp32 accumulation of sums over at most a
+few thousand terms of one sign-mixed product), 2e-2 for bf16.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from latent_mixture_experts_top_b200 import configs, synth
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+def _lmoe():
+    from latent_mixture_experts_top_b200 import lmoe
+    return lmoe
+
+
+def _backward_case(cfg, T=None, max_tokens=None, seed=0, tol=None):
+    lm = _lmoe()
+    T = cfg.T if T is None else T
+    inp = synth.make_inputs(cfg, seed, "cuda", T=T)
+    dy = synth.make_cotangent(cfg, seed, "cuda", T=T)
+    layer = lm.LatentMoELayer(cfg, inp, max_tokens=max_tokens or cfg.T, training=True)
+    x = inp["x"]
+    dx, grads = layer.backward(x, dy)
+    ids, gates, offsets, perm = layer.route(x)
+    torch.cuda.synchronize()
+    assert lm.lmoe_device_status(layer.handle) == 0
+    L = pu.oracle_layer(inp, cfg.k_active, cfg.activation)
+    x_np = synth.to_numpy(x)
+    ids_g = ids.cpu().numpy()
+    s_ref = oracle.router_logits(L, x_np)
+    pu.check_routing(ids_g, gates.cpu().numpy(), s_ref, cfg.k_active)
+    dy_np = dy.float().cpu().numpy().astype(np.float64)
+    ref = oracle.backward(L, x_np, dy_np, ids=ids_g, want=tuple(grads))
+    tol = tol or (pu.TOL_F32 if cfg.dtype == "f32" else pu.TOL_BF16)
+    errs = {"dx": pu.rel_err(dx.float().cpu().numpy().astype(np.float64), ref["dx"])}
+    for k, v in grads.items():
+        errs[k] = pu.rel_err(v.cpu().numpy().astype(np.float64), ref[k])
+    print(cfg.name, T, {k: f"{v:.2e}" for k, v in errs.items()})
+    layer.close()
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, bad
+    return errs
+
+
+def test_backward_tiny_f32_swiglu():
+    _backward_case(configs.TINY_F32)
+
+
+def test_backward_tiny_f32_relu2():
+    _backward_case(configs.TINY_RELU2_F32)
+
+
+def test_backward_tiny_f32_ragged_tokens():
+    """T = 37 tokens in a workspace for 64: partial tiles everywhere."""
+    _backward_case(configs.TINY_F32, T=37, max_tokens=64)
+
+
+def test_backward_zero_tokens_gives_zero_gradients():
+    lm = _lmoe()
+    cfg = configs.TINY_F32
+    inp = synth.make_inputs(cfg, 0, "cuda")
+    layer = lm.LatentMoELayer(cfg, inp, training=True)
+    x = inp["x"][:0]
+    dx, grads = layer.backward(x, x.clone())
+    torch.cuda.synchronize()
+    for v in grads.values():
+        assert not torch.any(v)
+    layer.close()
+
+
+def test_backward_needs_a_training_handle():
+    lm = _lmoe()
+    cfg = configs.TINY_F32
+    inp = synth.make_inputs(cfg, 0, "cuda")
+    layer = lm.LatentMoELayer(cfg, inp)   # training off
+    with pytest.raises(lm.LmoeError) as e:
+        layer.backward(inp["x"], inp["x"].clone())
+    assert e.value.code == -7
+    layer.close()

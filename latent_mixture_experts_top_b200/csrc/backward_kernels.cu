@@ -213,7 +213,146 @@ __global__ void bias_grad_kernel(const float *__restrict__ ds, const int32_t *__
   db[e] = acc;
 }
 
+// bf16 mode, gate/up pre-activations as the tensor-core GEMM writes them: in
+// each 256-column block b, columns [0,128) hold the gate of hidden units
+// 128b .. 128b+127 and [128,256) the matching up (squared ReLU: column c is
+// the up of unit c).  Writes h (plain [rows][n]) and dAB (same interleaved
+// layout as AB) from dh (fp32, plain); either output may be null.
+__global__ void act_backward_tiled_kernel(const __nv_bfloat16 *__restrict__ AB, int ldab,
+                                          const float *__restrict__ dh, int lddh,
+                                          __nv_bfloat16 *__restrict__ h, int ldh,
+                                          __nv_bfloat16 *__restrict__ dAB, int lddab, int rows,
+                                          int n, int relu2) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int r = blockIdx.y;
+  if (r >= rows || c >= n) return;
+  const size_t base = static_cast<size_t>(r) * ldab, dbase = static_cast<size_t>(r) * lddab;
+  const float g = dh ? dh[static_cast<size_t>(r) * lddh + c] : 0.0f;
+  if (relu2) {
+    const float rb = fmaxf(__bfloat162float(AB[base + c]), 0.0f);
+    if (h) h[static_cast<size_t>(r) * ldh + c] = __float2bfloat16_rn(rb * rb);
+    if (dAB) dAB[dbase + c] = __float2bfloat16_rn(g * 2.0f * rb);
+  } else {
+    const size_t ia = 256 * (c >> 7) + (c & 127), ib = ia + 128;
+    const float av = __bfloat162float(AB[base + ia]), bv = __bfloat162float(AB[base + ib]);
+    const float sg = 1.0f / (1.0f + expf(-av));
+    const float sl = av * sg;
+    if (h) h[static_cast<size_t>(r) * ldh + c] = __float2bfloat16_rn(sl * bv);
+    if (dAB) {
+      dAB[dbase + ia] = __float2bfloat16_rn(g * bv * sg * (1.0f + av * (1.0f - sg)));
+      dAB[dbase + ib] = __float2bfloat16_rn(g * sl);
+    }
+  }
+}
+
+// dst[c][col(r)] = src[r][c] for r < R, c < C, col(r) = r, or, with
+// row_expert, r + shift[row_expert[r]] (each expert's rows start at a
+// multiple of 64 in dst).  32 x 32 tiles through shared memory.
+__global__ void transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ src, int lds, int R, int C,
+                                      const int32_t *__restrict__ row_expert,
+                                      const int32_t *__restrict__ shift,
+                                      __nv_bfloat16 *__restrict__ dst, long long ldd,
+                                      long long src_batch, long long dst_batch) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  src += blockIdx.z * src_batch;
+  dst += blockIdx.z * dst_batch;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
+  for (int i = ty; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + tx;
+    tile[i][tx] = (r < R && c < C) ? src[static_cast<size_t>(r) * lds + c] : __float2bfloat16_rn(0.0f);
+  }
+  __syncthreads();
+  const int r = r0 + tx;
+  if (r >= R) return;
+  const long long col = row_expert ? r + shift[row_expert[r]] : r;
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i;
+    if (c < C) dst[static_cast<long long>(c) * ldd + col] = tile[tx][i];
+  }
+}
+
+// Zeros the padding columns of a token-major transposed operand: for every
+// row c < n_rows and expert e, columns [kstart[e] + rows_e, kstart[e] +
+// klen[e]) (rows_e = offsets[e+1] - offsets[e]).
+__global__ void zero_pad_cols_kernel(__nv_bfloat16 *__restrict__ dst, long long ldd, int n_rows,
+                                     const int32_t *__restrict__ offsets,
+                                     const int32_t *__restrict__ kstart,
+                                     const int32_t *__restrict__ klen) {
+  const int e = blockIdx.x;
+  const int rows = offsets[e + 1] - offsets[e];
+  const int pad = klen[e] - rows;
+  if (pad <= 0) return;
+  const long long k0 = kstart[e] + rows;
+  for (int i = threadIdx.x; i < n_rows * pad; i += blockDim.x) {
+    const int c = i / pad, k = i % pad;
+    dst[c * ldd + k0 + k] = __float2bfloat16_rn(0.0f);
+  }
+}
+
+// Per-expert K ranges of the token-major transposed operands: klen[e] =
+// rows of e rounded up to 64, kstart = exclusive scan of klen (kstart[N] =
+// total), shift[e] = kstart[e] - offsets[e].  One block, N <= 1024.
+__global__ void padded_offsets_kernel(const int32_t *__restrict__ offsets, int N,
+                                      int32_t *__restrict__ kstart, int32_t *__restrict__ klen,
+                                      int32_t *__restrict__ shift) {
+  __shared__ int buf[1024];
+  const int e = threadIdx.x;
+  const int len = e < N ? ((offsets[e + 1] - offsets[e] + 63) & ~63) : 0;
+  buf[e] = len;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {  // inclusive Hillis-Steele scan
+    const int v = e >= off ? buf[e - off] : 0;
+    __syncthreads();
+    buf[e] += v;
+    __syncthreads();
+  }
+  if (e < N) {
+    const int start = buf[e] - len;
+    kstart[e] = start;
+    klen[e] = len;
+    shift[e] = start - offsets[e];
+  }
+  if (e == N - 1) kstart[N] = buf[e];
+}
+
 }  // namespace
+
+cudaError_t launch_act_backward_tiled(const __nv_bfloat16 *AB, int ldab, const float *dh,
+                                      int lddh, __nv_bfloat16 *h, int ldh, __nv_bfloat16 *dAB,
+                                      int lddab, int rows, int n, bool relu2, cudaStream_t s) {
+  if (rows <= 0 || n <= 0) return cudaSuccess;
+  dim3 grid((n + 255) / 256, rows);
+  act_backward_tiled_kernel<<<grid, 256, 0, s>>>(AB, ldab, dh, lddh, h, ldh, dAB, lddab, rows, n,
+                                                 relu2 ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int lds, int R, int C,
+                                  const int32_t *row_expert, const int32_t *shift,
+                                  __nv_bfloat16 *dst, long long ldd, cudaStream_t s, int batch,
+                                  long long src_batch, long long dst_batch) {
+  if (R <= 0 || C <= 0 || batch <= 0) return cudaSuccess;
+  dim3 grid((C + 31) / 32, (R + 31) / 32, batch);
+  transpose_bf16_kernel<<<grid, 256, 0, s>>>(src, lds, R, C, row_expert, shift, dst, ldd,
+                                             src_batch, dst_batch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_pad_cols(__nv_bfloat16 *dst, long long ldd, int n_rows,
+                                 const int32_t *offsets, const int32_t *kstart,
+                                 const int32_t *klen, int N, cudaStream_t s) {
+  if (N <= 0 || n_rows <= 0) return cudaSuccess;
+  zero_pad_cols_kernel<<<N, 256, 0, s>>>(dst, ldd, n_rows, offsets, kstart, klen);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_padded_offsets(const int32_t *offsets, int N, int32_t *kstart, int32_t *klen,
+                                  int32_t *shift, cudaStream_t s) {
+  if (N <= 0 || N > 1024) return cudaErrorInvalidValue;
+  padded_offsets_kernel<<<1, 1024, 0, s>>>(offsets, N, kstart, klen, shift);
+  return cudaGetLastError();
+}
 
 cudaError_t simt_gemm(const SimtGemm &g, int groups, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0 || groups <= 0) return cudaSuccess;

@@ -71,6 +71,15 @@ enum TcMode : int {
   TC_EXPERT_GU = 1, // grouped: permuted z x W_gu[e] -> SwiGLU -> H
   TC_EXPERT_DOWN = 2,  // grouped: H x W_o[e] -> O (bf16)
   TC_OUT = 3,       // [u | shared hidden] x W_y -> y (bf16)
+  TC_WGRAD = 4,     // weight gradients: dW[g] = A^T B over token-major K ranges (fp32)
+};
+
+// TC_WGRAD destinations (fp32, the caller's gradient layouts).
+enum WgKind {
+  WG_Y = 0,   // rows d, cols l + n_s m_s: [dW_up | dS_o(0) | dS_o(1) ...]
+  WG_X = 1,   // rows = W_x rows (router | W_down | shared gate/up), cols d
+  WG_O = 2,   // per expert: rows l, cols m -> dW_o[e]
+  WG_GU = 3,  // per expert: rows = W_gu rows (gate/up interleaved by 128), cols l
 };
 
 struct TcParams {
@@ -93,6 +102,19 @@ struct TcParams {
                        // region of TC_X_FUSED write relu(acc)^2 (no gate/up
                        // interleave); n_cols2 bounds their output columns
   int n_cols2;
+  // Backward-only options (all zero in the forward):
+  int raw;             // TC_EXPERT_GU and the shared region of TC_X_FUSED write
+                       // the accumulator as is (bf16 gate/up pre-activations)
+  __nv_bfloat16 *out2; int ld_out2;  // TC_X_FUSED shared region, with raw
+  float *out_f32;      // TC_OUT / TC_EXPERT_DOWN: fp32 output [rows][ld_out]
+  // TC_WGRAD: A [M][*] and B [*][*] are plain row-major token-major matrices
+  // (K runs along their rows' contiguous axis); group g reduces over
+  // K-columns [k_start[g], k_start[g] + k_len[g]) (multiples of 64; dense:
+  // k_start == null and K = Kdim); n_tiles_n counts 256-row tiles of B.
+  int wg_kind, groups;
+  const int32_t *k_start, *k_len;
+  int wg_d, wg_l, wg_m, wg_ns, wg_ms, wg_n, wg_npad, wg_lpad;  // layer sizes for the destinations
+  float *g_router, *g_down, *g_up, *g_gate, *g_upx, *g_out, *g_sgate, *g_sup, *g_sout;
   int32_t *status;
 };
 
@@ -152,6 +174,27 @@ cudaError_t launch_scatter_ds(const float *ds, const int32_t *ids, int T, int K,
 // db[e] = sum of ds over expert e's pairs, token order.
 cudaError_t launch_bias_grad(const float *ds, const int32_t *offsets, const int32_t *perm, int N,
                              float *db, cudaStream_t s);
+
+// bf16: gate/up pre-activations AB in the GEMM's 128-interleaved layout
+// (squared ReLU: plain up) -> h (plain) and dAB (interleaved); see the kernel.
+cudaError_t launch_act_backward_tiled(const __nv_bfloat16 *AB, int ldab, const float *dh,
+                                      int lddh, __nv_bfloat16 *h, int ldh, __nv_bfloat16 *dAB,
+                                      int lddab, int rows, int n, bool relu2, cudaStream_t s);
+// dst[c][col(r)] = src[r][c]; col(r) = r, or r + shift[row_expert[r]];
+// `batch` independent matrices, src / dst advanced by src_batch / dst_batch.
+cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int lds, int R, int C,
+                                  const int32_t *row_expert, const int32_t *shift,
+                                  __nv_bfloat16 *dst, long long ldd, cudaStream_t s,
+                                  int batch = 1, long long src_batch = 0,
+                                  long long dst_batch = 0);
+// Zeros dst[c][kstart[e] + rows_e .. kstart[e] + klen[e]) for c < n_rows.
+cudaError_t launch_zero_pad_cols(__nv_bfloat16 *dst, long long ldd, int n_rows,
+                                 const int32_t *offsets, const int32_t *kstart,
+                                 const int32_t *klen, int N, cudaStream_t s);
+// klen[e] = round64(rows of e), kstart = its exclusive scan (kstart[N] =
+// total), shift[e] = kstart[e] - offsets[e].  N <= 1024.
+cudaError_t launch_padded_offsets(const int32_t *offsets, int N, int32_t *kstart, int32_t *klen,
+                                  int32_t *shift, cudaStream_t s);
 
 // Failure-detection self-test (see lmoe_selftest_wait_timeout).
 cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s);

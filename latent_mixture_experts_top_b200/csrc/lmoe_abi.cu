@@ -12,6 +12,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <new>
 
 #include "../../include/lmoe.h"
@@ -55,6 +56,15 @@ struct BwdWorkspace {
   void *as = nullptr, *bs = nullptr;    // [T][ns ms] shared pre-activations
   void *das = nullptr, *dbs = nullptr;  // [T][ns ms]
   float *dsfull = nullptr;              // [T][N']
+  // bf16 mode only
+  void *AB = nullptr;      // [TK][gu_rows] expert gate/up pre-activations (GEMM layout)
+  void *ABs = nullptr;     // [T][sh_rows]  shared gate/up pre-activations (W_x layout)
+  void *dAB = nullptr;     // [TK][gu_rows]
+  void *dXcat = nullptr;   // [T][nx_rows] = [dS (router) | dz | shared dAB], W_x columns
+  void *DOT = nullptr, *HT = nullptr, *dABT = nullptr, *zpT = nullptr;  // [*][Kp] token-major
+  void *dyT = nullptr, *ucatT = nullptr, *dXcatT = nullptr, *xT = nullptr;  // [*][Tp]
+  int32_t *kstart = nullptr, *klen = nullptr, *shift = nullptr;  // [N'+1]
+  int64_t Kp = 0, Tp = 0;
 };
 
 }  // namespace
@@ -95,6 +105,13 @@ struct lmoe_layer {
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
+  // bf16 training: transposed weights (K-block tiled) and backward maps
+  void *w_yT = nullptr;   // [ky][d]
+  void *w_oT = nullptr;   // [N][m][l]
+  void *w_guT = nullptr;  // [N][l][gu_rows]
+  void *w_xT = nullptr;   // [d][nx_rows]
+  TensorMap64 tm_wyT, tm_woT, tm_wguT, tm_wxT, tm_DO, tm_dAB, tm_dXcat;
+  TensorMap64 tm_DOT, tm_HT, tm_dABT, tm_zpT, tm_dyT, tm_ucatT, tm_dXcatT, tm_xT;
 };
 
 namespace {
@@ -128,7 +145,10 @@ void free_all(lmoe_layer *h) {
                   h->ws.tiles, h->ws.n_tiles, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
                   h->ws.x_stage, h->ws.y_stage, h->ws.status, h->bw.a, h->bw.b, h->bw.dU,
                   h->bw.ds, h->bw.DO, h->bw.dH, h->bw.dA, h->bw.dB, h->bw.dZp, h->bw.dz,
-                  h->bw.as, h->bw.bs, h->bw.das, h->bw.dbs, h->bw.dsfull};
+                  h->bw.as, h->bw.bs, h->bw.das, h->bw.dbs, h->bw.dsfull, h->bw.AB,
+                  h->bw.ABs, h->bw.dAB, h->bw.dXcat, h->bw.DOT, h->bw.HT, h->bw.dABT,
+                  h->bw.zpT, h->bw.dyT, h->bw.ucatT, h->bw.dXcatT, h->bw.xT, h->bw.kstart,
+                  h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
@@ -271,6 +291,24 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
          dalloc(&b.dZp, TK * l * 4) && dalloc(&b.dz, T * l * 4) && dalloc(&b.as, T * nsms * es) &&
          dalloc(&b.bs, T * nsms * es) && dalloc(&b.das, T * nsms * es) &&
          dalloc(&b.dbs, T * nsms * es) && dalloc(&b.dsfull, T * N * 4);
+    if (ok && h->bf16) {
+      const size_t gu = h->gu_rows, nx = h->nx_rows, ky = h->ky;
+      b.Kp = static_cast<int64_t>((TK + 63) / 64 * 64 + 64 * N);
+      b.Tp = static_cast<int64_t>((T + 63) / 64 * 64);
+      const size_t Kp = b.Kp, Tp = b.Tp;
+      ok = dalloc(&b.AB, TK * gu * 2) && dalloc(&b.ABs, T * h->sh_rows * 2) &&
+           dalloc(&b.dAB, TK * gu * 2) && dalloc(&b.dXcat, T * nx * 2) &&
+           dalloc(&b.DOT, l * Kp * 2) && dalloc(&b.HT, m * Kp * 2) &&
+           dalloc(&b.dABT, gu * Kp * 2) && dalloc(&b.zpT, l * Kp * 2) &&
+           dalloc(&b.dyT, d * Tp * 2) && dalloc(&b.ucatT, ky * Tp * 2) &&
+           dalloc(&b.dXcatT, nx * Tp * 2) && dalloc(&b.xT, d * Tp * 2) &&
+           dalloc(&b.kstart, (N + 1) * 4) && dalloc(&b.klen, (N + 1) * 4) &&
+           dalloc(&b.shift, (N + 1) * 4) &&
+           dalloc(&h->w_yT, btile_rows(1, h->ky, h->d) * 64 * 2) &&
+           dalloc(&h->w_oT, btile_rows(h->N, h->m, h->l) * 64 * 2) &&
+           dalloc(&h->w_guT, btile_rows(h->N, h->l, h->gu_rows) * 64 * 2) &&
+           dalloc(&h->w_xT, btile_rows(1, h->d, h->nx_rows) * 64 * 2);
+    }
   }
   if (!ok) {
     cudaGetLastError();
@@ -297,6 +335,30 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
       rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN);
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wy, h->w_y, btile_rows(1, h->d, h->ky), 64, 64, kTileN);
+    if (rc == LMOE_OK && h->training) {
+      BwdWorkspace &b = h->bw;
+      const int64_t Kp = b.Kp, Tp = b.Tp;
+      const int gu = h->gu_rows, nx = h->nx_rows;
+      // A operands of the K-major backward GEMMs ({64, 128} boxes)
+      rc = make_map(&h->tm_DO, b.DO, static_cast<int64_t>(TK), h->l, h->l, kTileM);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_dAB, b.dAB, static_cast<int64_t>(TK), gu, gu, kTileM);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_dXcat, b.dXcat, h->Tmax, nx, nx, kTileM);
+      // transposed weights, K-block tiled ({64, 256} boxes)
+      if (rc == LMOE_OK) rc = make_map(&h->tm_wyT, h->w_yT, btile_rows(1, h->ky, h->d), 64, 64, kTileN);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_woT, h->w_oT, btile_rows(h->N, h->m, h->l), 64, 64, kTileN);
+      if (rc == LMOE_OK)
+        rc = make_map(&h->tm_wguT, h->w_guT, btile_rows(h->N, h->l, gu), 64, 64, kTileN);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_wxT, h->w_xT, btile_rows(1, h->d, nx), 64, 64, kTileN);
+      // weight-gradient operands: token-major, A {64, 128}, B {64, 256}
+      if (rc == LMOE_OK) rc = make_map(&h->tm_DOT, b.DOT, h->l, Kp, Kp, kTileM);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_HT, b.HT, h->m, Kp, Kp, kTileN);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_dABT, b.dABT, gu, Kp, Kp, kTileM);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_zpT, b.zpT, h->l, Kp, Kp, kTileN);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_dyT, b.dyT, h->d, Tp, Tp, kTileM);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_ucatT, b.ucatT, h->ky, Tp, Tp, kTileN);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_dXcatT, b.dXcatT, nx, Tp, Tp, kTileM);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_xT, b.xT, h->d, Tp, Tp, kTileN);
+    }
     if (rc == LMOE_OK &&
         (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
          cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
@@ -400,6 +462,41 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   if (e == cudaSuccess)
     e = launch_repack_btiles(static_cast<const bf *>(ty), 1, h->d, h->ky,
                              static_cast<bf *>(h->w_y), s);
+  if (e == cudaSuccess && h->training) {
+    // Backward: the transposed matrices, built in one scratch buffer and
+    // K-block tiled like the forward's.
+    const size_t big = std::max({static_cast<size_t>(h->nx_rows) * d, d * ky,
+                                 N * m * l, N * static_cast<size_t>(h->gu_rows) * l});
+    void *tt = nullptr;
+    if (!dalloc(&tt, big * es)) e = cudaErrorMemoryAllocation;
+    bf *t16 = static_cast<bf *>(tt);
+    const bf *gu_src = static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu);
+    if (e == cudaSuccess)  // [W_up | S_o]^T: [ky][d]
+      e = launch_transpose_bf16(static_cast<const bf *>(ty), static_cast<int>(ky), static_cast<int>(d),
+                                static_cast<int>(ky), nullptr, nullptr, t16, static_cast<long long>(d), s);
+    if (e == cudaSuccess)
+      e = launch_repack_btiles(t16, 1, h->ky, h->d, static_cast<bf *>(h->w_yT), s);
+    if (e == cudaSuccess)  // W_o[e]^T: [m][l] per expert
+      e = launch_transpose_bf16(static_cast<const bf *>(wt->w_out), h->m, h->l, h->m, nullptr,
+                                nullptr, t16, h->l, s, h->N, static_cast<long long>(l * m),
+                                static_cast<long long>(m * l));
+    if (e == cudaSuccess)
+      e = launch_repack_btiles(t16, h->N, h->m, h->l, static_cast<bf *>(h->w_oT), s);
+    if (e == cudaSuccess)  // W_gu[e]^T: [l][gu_rows] per expert
+      e = launch_transpose_bf16(gu_src, h->l, h->gu_rows, h->l, nullptr, nullptr, t16,
+                                h->gu_rows, s, h->N, static_cast<long long>(h->gu_rows) * l,
+                                static_cast<long long>(h->gu_rows) * l);
+    if (e == cudaSuccess)
+      e = launch_repack_btiles(t16, h->N, h->l, h->gu_rows, static_cast<bf *>(h->w_guT), s);
+    if (e == cudaSuccess)  // W_x^T: [d][nx_rows]
+      e = launch_transpose_bf16(static_cast<const bf *>(tx), h->d, h->nx_rows, h->d, nullptr,
+                                nullptr, t16, h->nx_rows, s);
+    if (e == cudaSuccess)
+      e = launch_repack_btiles(t16, 1, h->d, h->nx_rows, static_cast<bf *>(h->w_xT), s);
+    const cudaError_t es3 = cudaStreamSynchronize(s);
+    if (tt) cudaFree(tt);
+    if (e == cudaSuccess) e = es3;
+  }
   // the temporaries are freed once the repacks have run
   const cudaError_t es2 = cudaStreamSynchronize(s);
   cudaFree(tx);
@@ -426,7 +523,11 @@ static int check_call(lmoe_handle h, int32_t T) {
 }
 
 // Router logits (+ z and shared hidden when full) and the routing steps.
-static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cudaStream_t s) {
+// shared_raw (bf16 backward only): the shared experts' gate/up GEMM writes its
+// raw pre-activations there ([T][sh_rows], W_x's shared-row layout) instead
+// of the hidden.
+static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cudaStream_t s,
+                             void *shared_raw = nullptr) {
   Workspace &w = h->ws;
   cudaError_t e = cudaSuccess;
   if (h->bf16) {
@@ -462,6 +563,11 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       TcParams q = p;
       q.n_tile_base = (h->n_pad + h->l_pad) / kTileN;
       q.n_tiles_n = shared_tiles_n;
+      if (shared_raw) {
+        q.raw = 1;
+        q.out2 = static_cast<__nv_bfloat16 *>(shared_raw);
+        q.ld_out2 = h->sh_rows;
+      }
       e = cudaEventRecord(h->ev_fork, s);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
       if (e == cudaSuccess)
@@ -740,6 +846,182 @@ static cudaError_t backward_f32(lmoe_layer *h, const float *x, const float *dy, 
   return cudaSuccess;
 }
 
+// ---- backward, bf16 mode: every contraction on the tcgen05 GEMM.
+static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, void *dx,
+                                 const lmoe_grads *g, int T, cudaStream_t s) {
+  using bf = __nv_bfloat16;
+  Workspace &w = h->ws;
+  BwdWorkspace &b = h->bw;
+  const int d = h->d, l = h->l, m = h->m, N = h->N, K = h->K, ky = h->ky;
+  const int nx = h->nx_rows, gu = h->gu_rows, TK = T * K;
+  const int n_pad = h->n_pad, l_pad = h->l_pad;
+  const bool relu2 = h->relu2 != 0;
+  const int64_t Tp = (T + 63) / 64 * 64, Kp = b.Kp;
+  bf *ucat = static_cast<bf *>(w.ucat), *dXcat = static_cast<bf *>(b.dXcat);
+  int64_t &L = h->launches;
+  auto gemm = [&](const TensorMap64 &ta, const TensorMap64 &tb, const TcParams &p, int tiles) {
+    ++L;
+    return launch_tc_gemm(ta.bytes, tb.bytes, p, h->num_sms, tiles, s);
+  };
+#define LMOE_TRY(...) do { cudaError_t e_ = (__VA_ARGS__); if (e_ != cudaSuccess) return e_; } while (0)
+  TensorMap64 tm_x, tm_dy;
+  if (make_map(&tm_x, x, T, d, d, kTileM) != LMOE_OK ||
+      make_map(&tm_dy, dy, T, d, d, kTileM) != LMOE_OK)
+    return cudaErrorInvalidValue;
+  const int m_tiles_T = (T + kTileM - 1) / kTileM;
+  // ---- forward activations
+  LMOE_TRY(run_route(h, x, T, true, s, b.ABs));
+  ++L;
+  LMOE_TRY(launch_permute_rows(w.z, w.perm, K, TK, l * 2, w.zp, s));
+  {
+    TcParams p = {};  // expert gate/up pre-activations AB
+    p.mode = TC_EXPERT_GU; p.Kdim = l; p.n_tiles_n = (gu + kTileN - 1) / kTileN; p.raw = 1;
+    p.relu2 = h->relu2; p.n_cols2 = m;
+    p.tiles = w.tiles; p.n_mtiles = w.n_tiles;
+    p.out = static_cast<bf *>(b.AB); p.ld_out = gu; p.status = w.status;
+    LMOE_TRY(gemm(h->tm_zp, h->tm_wgu, p, h->num_sms));
+  }
+  ++L;
+  LMOE_TRY(launch_act_backward_tiled(static_cast<bf *>(b.AB), gu, nullptr, 0,
+                                     static_cast<bf *>(w.H), m, nullptr, 0, TK, m, relu2, s));
+  {
+    TcParams p = {};  // expert outputs O
+    p.mode = TC_EXPERT_DOWN; p.Kdim = m; p.n_tiles_n = (l + kTileN - 1) / kTileN;
+    p.tiles = w.tiles; p.n_mtiles = w.n_tiles;
+    p.out = static_cast<bf *>(w.O); p.ld_out = l; p.status = w.status;
+    LMOE_TRY(gemm(h->tm_h, h->tm_wo, p, h->num_sms));
+  }
+  ++L;
+  LMOE_TRY(launch_combine(w.O, w.pos, w.gates, T, K, l, w.ucat, ky, true, s));  // u
+  LMOE_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));  // shared pre-activations ready
+  // ---- dU = dy [W_up | S_o]  (fp32 [T][ky])
+  {
+    TcParams p = {};
+    p.mode = TC_OUT; p.M = T; p.Kdim = d; p.n_tiles_n = (ky + kTileN - 1) / kTileN;
+    p.out_f32 = b.dU; p.ld_out = ky; p.status = w.status;
+    LMOE_TRY(gemm(tm_dy, h->tm_wyT, p, m_tiles_T * p.n_tiles_n));
+  }
+  // shared experts: hidden (for dS_o) into ucat's shared columns, pre-activation
+  // gradients into dXcat's shared columns
+  const int nsms = h->ns * h->ms;
+  if (nsms > 0) {
+    ++L;
+    LMOE_TRY(launch_act_backward_tiled(static_cast<bf *>(b.ABs), h->sh_rows, b.dU + l, ky,
+                                       ucat + l, ky, dXcat + n_pad + l_pad, nx, T, nsms, relu2, s));
+  }
+  // ---- gates, expert-output gradients, expert backward
+  ++L;
+  LMOE_TRY(launch_slot_grad<bf>(b.dU, ky, static_cast<bf *>(w.O), l, w.pos, w.gates, T, K, b.ds,
+                                static_cast<bf *>(b.DO), s));
+  {
+    TcParams p = {};  // dH = DO W_o[e]  (fp32 [TK][m])
+    p.mode = TC_EXPERT_DOWN; p.Kdim = l; p.n_tiles_n = (m + kTileN - 1) / kTileN;
+    p.tiles = w.tiles; p.n_mtiles = w.n_tiles;
+    p.out_f32 = b.dH; p.ld_out = m; p.status = w.status;
+    LMOE_TRY(gemm(h->tm_DO, h->tm_woT, p, h->num_sms));
+  }
+  ++L;
+  LMOE_TRY(launch_act_backward_tiled(static_cast<bf *>(b.AB), gu, b.dH, m, nullptr, 0,
+                                     static_cast<bf *>(b.dAB), gu, TK, m, relu2, s));
+  {
+    TcParams p = {};  // dZp = dAB W_gu[e]  (fp32 [TK][l])
+    p.mode = TC_EXPERT_DOWN; p.Kdim = gu; p.n_tiles_n = (l + kTileN - 1) / kTileN;
+    p.tiles = w.tiles; p.n_mtiles = w.n_tiles;
+    p.out_f32 = b.dZp; p.ld_out = l; p.status = w.status;
+    LMOE_TRY(gemm(h->tm_dAB, h->tm_wguT, p, h->num_sms));
+  }
+  // ---- dXcat = [dS | dz | shared dAB] in W_x's row order, padding zeroed
+  L += 2;
+  LMOE_TRY(launch_gather_sum<float, bf>(b.dZp, l, w.pos, T, K, l, dXcat + n_pad, nx, s));
+  LMOE_TRY(launch_scatter_ds<bf>(b.ds, w.ids, T, K, N, dXcat, nx, s));
+  auto zero_cols = [&](bf *base, int64_t ld, int64_t c0, int64_t c1, int rows) {
+    if (c1 <= c0 || rows <= 0) return cudaSuccess;
+    return cudaMemset2DAsync(base + c0, ld * 2, 0, (c1 - c0) * 2, rows, s);
+  };
+  LMOE_TRY(zero_cols(dXcat, nx, N, n_pad, T));
+  LMOE_TRY(zero_cols(dXcat, nx, n_pad + l, n_pad + l_pad, T));
+  LMOE_TRY(zero_cols(dXcat, nx, n_pad + l_pad + (relu2 ? nsms : 2 * nsms), nx, T));
+  {
+    TcParams p = {};  // dx = dXcat W_x
+    p.mode = TC_OUT; p.M = T; p.Kdim = nx; p.n_tiles_n = (d + kTileN - 1) / kTileN;
+    p.out = static_cast<bf *>(dx); p.ld_out = d; p.status = w.status;
+    LMOE_TRY(gemm(h->tm_dXcat, h->tm_wxT, p, m_tiles_T * p.n_tiles_n));
+  }
+  // ---- weight gradients: token-major transposes, then A^T B per group
+  auto fill_sizes = [&](TcParams &p) {
+    p.wg_d = d; p.wg_l = l; p.wg_m = m; p.wg_ns = h->ns; p.wg_ms = h->ms; p.wg_n = N;
+    p.wg_npad = n_pad; p.wg_lpad = l_pad; p.relu2 = h->relu2; p.status = w.status;
+    p.g_router = g->w_router; p.g_down = g->w_down; p.g_up = g->w_up; p.g_gate = g->w_gate;
+    p.g_upx = g->w_upx; p.g_out = g->w_out; p.g_sgate = g->s_gate; p.g_sup = g->s_up;
+    p.g_sout = g->s_out;
+  };
+  L += 4;
+  // (row stride b.Tp, the maps' width; this call reduces over Tp columns)
+  LMOE_TRY(launch_transpose_bf16(static_cast<const bf *>(dy), d, T, d, nullptr, nullptr,
+                                 static_cast<bf *>(b.dyT), b.Tp, s));
+  LMOE_TRY(launch_transpose_bf16(ucat, ky, T, ky, nullptr, nullptr, static_cast<bf *>(b.ucatT),
+                                 b.Tp, s));
+  LMOE_TRY(launch_transpose_bf16(dXcat, nx, T, nx, nullptr, nullptr, static_cast<bf *>(b.dXcatT),
+                                 b.Tp, s));
+  LMOE_TRY(launch_transpose_bf16(static_cast<const bf *>(x), d, T, d, nullptr, nullptr,
+                                 static_cast<bf *>(b.xT), b.Tp, s));
+  LMOE_TRY(zero_cols(static_cast<bf *>(b.dyT), b.Tp, T, Tp, d));
+  LMOE_TRY(zero_cols(static_cast<bf *>(b.ucatT), b.Tp, T, Tp, ky));
+  LMOE_TRY(zero_cols(static_cast<bf *>(b.dXcatT), b.Tp, T, Tp, nx));
+  LMOE_TRY(zero_cols(static_cast<bf *>(b.xT), b.Tp, T, Tp, d));
+  {
+    TcParams p = {};  // [dW_up | dS_o] = dy^T [u | h_s]
+    p.mode = TC_WGRAD; p.wg_kind = WG_Y; p.groups = 1; p.M = d; p.Kdim = static_cast<int>(Tp);
+    p.n_tiles_n = (ky + kTileN - 1) / kTileN;
+    fill_sizes(p);
+    LMOE_TRY(gemm(h->tm_dyT, h->tm_ucatT, p, (d + kTileM - 1) / kTileM * p.n_tiles_n));
+  }
+  {
+    TcParams p = {};  // [dW_r ; dW_down ; dS_g / dS_u] = dXcat^T x
+    p.mode = TC_WGRAD; p.wg_kind = WG_X; p.groups = 1; p.M = nx; p.Kdim = static_cast<int>(Tp);
+    p.n_tiles_n = (d + kTileN - 1) / kTileN;
+    fill_sizes(p);
+    LMOE_TRY(gemm(h->tm_dXcatT, h->tm_xT, p, (nx + kTileM - 1) / kTileM * p.n_tiles_n));
+  }
+  if (g->b_router) {
+    ++L;
+    LMOE_TRY(launch_bias_grad(b.ds, w.offsets, w.perm, N, g->b_router, s));
+  }
+  // grouped: each expert's rows at a 64-aligned K range of the transposes
+  L += 9;
+  LMOE_TRY(launch_padded_offsets(w.offsets, N, b.kstart, b.klen, b.shift, s));
+  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(b.DO), l, TK, l, w.row_expert, b.shift,
+                                 static_cast<bf *>(b.DOT), Kp, s));
+  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(w.H), m, TK, m, w.row_expert, b.shift,
+                                 static_cast<bf *>(b.HT), Kp, s));
+  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(b.dAB), gu, TK, gu, w.row_expert, b.shift,
+                                 static_cast<bf *>(b.dABT), Kp, s));
+  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(w.zp), l, TK, l, w.row_expert, b.shift,
+                                 static_cast<bf *>(b.zpT), Kp, s));
+  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.DOT), Kp, l, w.offsets, b.kstart, b.klen, N, s));
+  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.HT), Kp, m, w.offsets, b.kstart, b.klen, N, s));
+  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.dABT), Kp, gu, w.offsets, b.kstart, b.klen, N, s));
+  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.zpT), Kp, l, w.offsets, b.kstart, b.klen, N, s));
+  {
+    TcParams p = {};  // dW_o[e] = DO_e^T H_e
+    p.mode = TC_WGRAD; p.wg_kind = WG_O; p.groups = N; p.M = l; p.Kdim = 64;
+    p.k_start = b.kstart; p.k_len = b.klen;
+    p.n_tiles_n = (m + kTileN - 1) / kTileN;
+    fill_sizes(p);
+    LMOE_TRY(gemm(h->tm_DOT, h->tm_HT, p, N * ((l + kTileM - 1) / kTileM) * p.n_tiles_n));
+  }
+  {
+    TcParams p = {};  // [dW_g ; dW_u][e] = dAB_e^T zp_e
+    p.mode = TC_WGRAD; p.wg_kind = WG_GU; p.groups = N; p.M = gu; p.Kdim = 64;
+    p.k_start = b.kstart; p.k_len = b.klen;
+    p.n_tiles_n = (l + kTileN - 1) / kTileN;
+    fill_sizes(p);
+    LMOE_TRY(gemm(h->tm_dABT, h->tm_zpT, p, N * ((gu + kTileM - 1) / kTileM) * p.n_tiles_n));
+  }
+#undef LMOE_TRY
+  return cudaSuccess;
+}
+
 int lmoe_backward(lmoe_handle h, const void *x, const void *dy, void *dx, const lmoe_grads *g,
                   int32_t T, void *stream) {
   int rc = check_call(h, T);
@@ -763,7 +1045,7 @@ int lmoe_backward(lmoe_handle h, const void *x, const void *dy, void *dx, const 
     z(g->s_gate, nsms * d); z(g->s_up, nsms * d); z(g->s_out, d * nsms);
     return cuda_err(e);
   }
-  if (h->bf16) return LMOE_ERR_UNSUPPORTED;
+  if (h->bf16) return cuda_err(backward_bf16(h, x, dy, dx, g, T, s));
   return cuda_err(backward_f32(h, static_cast<const float *>(x), static_cast<const float *>(dy),
                                static_cast<float *>(dx), g, T, s));
 }

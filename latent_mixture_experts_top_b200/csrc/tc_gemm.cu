@@ -69,11 +69,33 @@ constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + size
 
 struct Tile {
   int a_row, b_row, n_tile, row_hi;
+  int k0;     // first K column (A, and B when b_plain)
+  int nkb;    // K-blocks of this tile
+  int group;  // TC_WGRAD group
+  bool b_plain;  // B is a plain row-major matrix (else K-block tiled)
 };
 
 __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles) {
   Tile tl;
-  if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
+  tl.k0 = 0;
+  tl.nkb = p.Kdim / TKB;
+  tl.group = 0;
+  tl.b_plain = false;
+  if (p.mode == TC_WGRAD) {
+    const int per = m_tiles * p.n_tiles_n;
+    const int g = t / per, r = t % per;
+    const int m = r % m_tiles, n = r / m_tiles;  // consecutive CTAs share B
+    tl.a_row = m * TM;
+    tl.b_row = n * TN;
+    tl.n_tile = n;
+    tl.row_hi = p.M;
+    tl.group = g;
+    tl.b_plain = true;
+    if (p.k_start) {
+      tl.k0 = p.k_start[g];
+      tl.nkb = p.k_len[g] / TKB;
+    }
+  } else if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
     const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
     tl.a_row = m * TM;
     tl.b_row = n * (p.Kdim / TKB) * TN;  // first K-block tile of B's N-tile n
@@ -162,6 +184,81 @@ __device__ __forceinline__ void epi_relu2(uint32_t taddr, bool valid, __nv_bfloa
   }
 }
 
+// Weight-gradient tile row `row` (an A row), output columns col0 .. col0+255
+// (B rows): fp32 into the caller's gradient arrays; zeros when the tile had
+// no K-blocks (an expert no token chose).
+__device__ __forceinline__ float *wgrad_row_dst(const TcParams &p, int row, int group,
+                                                int *ld_or_skip) {
+  const int d = p.wg_d, l = p.wg_l, m = p.wg_m;
+  switch (p.wg_kind) {
+    case WG_X: {
+      *ld_or_skip = d;
+      if (row < p.wg_n) return p.g_router + static_cast<size_t>(row) * d;
+      if (row >= p.wg_npad && row < p.wg_npad + l)
+        return p.g_down + static_cast<size_t>(row - p.wg_npad) * d;
+      const int r = row - p.wg_npad - p.wg_lpad;
+      const int nsms = p.wg_ns * p.wg_ms;
+      if (r < 0) return nullptr;
+      if (p.relu2) return r < nsms ? p.g_sup + static_cast<size_t>(r) * d : nullptr;
+      const int b = r >> 8, i = r & 255;
+      const int unit = 128 * b + (i & 127);
+      if (unit >= nsms) return nullptr;
+      return (i < 128 ? p.g_sgate : p.g_sup) + static_cast<size_t>(unit) * d;
+    }
+    case WG_O:
+      *ld_or_skip = m;
+      return row < l ? p.g_out + (static_cast<size_t>(group) * l + row) * m : nullptr;
+    case WG_GU: {
+      *ld_or_skip = l;
+      if (p.relu2) return row < m ? p.g_upx + (static_cast<size_t>(group) * m + row) * l : nullptr;
+      const int b = row >> 8, i = row & 255;
+      const int unit = 128 * b + (i & 127);
+      if (unit >= m) return nullptr;
+      return (i < 128 ? p.g_gate : p.g_upx) + (static_cast<size_t>(group) * m + unit) * l;
+    }
+    default:
+      return nullptr;
+  }
+}
+
+__device__ __forceinline__ void epi_wgrad(uint32_t taddr, bool valid, const TcParams &p, int row,
+                                          int group, int col0, bool empty, int half) {
+  const int ky = p.wg_l + p.wg_ns * p.wg_ms;
+  int ld = 0;
+  float *rowp = nullptr;
+  if (p.wg_kind != WG_Y && valid) rowp = wgrad_row_dst(p, row, group, &ld);
+  const int n_cols = p.wg_kind == WG_Y ? ky : ld;
+#pragma unroll 1
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+    float v[32];
+    if (empty) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+    } else {
+      uint32_t r[32];
+      ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+      ptx::tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    }
+    const int col = col0 + c * 32;
+    if (!valid || col >= n_cols) continue;
+    float *dst;
+    if (p.wg_kind == WG_Y) {  // columns [0, l): dW_up; then each shared expert's dS_o
+      if (col < p.wg_l) {
+        dst = p.g_up + static_cast<size_t>(row) * p.wg_l + col;
+      } else {
+        const int cc = col - p.wg_l, j = cc / p.wg_ms;
+        dst = p.g_sout + (static_cast<size_t>(j) * p.wg_d + row) * p.wg_ms + (cc - j * p.wg_ms);
+      }
+    } else {
+      if (!rowp) continue;
+      dst = rowp + col;
+    }
+    store_f32x32(dst, v);
+  }
+}
+
 // Columns [0,128) are gate rows g0..g0+127, [128,256) the matching up rows:
 // h = silu(gate) * up for 128 hidden columns starting at hcol0.
 __device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bfloat16 *row_dst,
@@ -194,8 +291,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const bool grouped = (p.mode == TC_EXPERT_GU || p.mode == TC_EXPERT_DOWN);
   const int m_tiles = grouped ? 0 : (p.M + TM - 1) / TM;
-  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles * p.n_tiles_n;
-  const int nkb = p.Kdim / TKB;
+  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n
+                            : m_tiles * p.n_tiles_n * (p.mode == TC_WGRAD ? p.groups : 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -230,7 +327,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile(p, t, m_tiles);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
@@ -239,8 +336,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
-          ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kb * TKB, tl.a_row);
-          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
+          const int kx = tl.k0 + kb * TKB;
+          ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kx, tl.a_row);
+          if (tl.b_plain)
+            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kx, tl.b_row);
+          else
+            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
         }
       }
       if (!ok) {  // let every copy still in flight land before the CTA exits
@@ -264,6 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * TN;
+        const int nkb = decode_tile(p, t, m_tiles).nkb;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -322,6 +424,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else if (col0 < p.z_end) {
             epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
                              col0 - p.r_end, p.l, half);
+          } else if (p.raw) {
+            epi_plain<false>(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2,
+                             col0 - p.z_end, p.ld_out2, half);
           } else if (p.relu2) {
             epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
                       col0 - p.z_end, p.n_cols2, half);
@@ -331,15 +436,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           break;
         case TC_EXPERT_GU:
-          if (p.relu2)
+          if (p.raw)
+            epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
+                             p.ld_out, half);
+          else if (p.relu2)
             epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0, p.n_cols2,
                       half);
           else
             epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
           break;
+        case TC_WGRAD:
+          epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
+          break;
         default:  // TC_EXPERT_DOWN, TC_OUT
-          epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
-                           p.ld_out, half);
+          if (p.out_f32)
+            epi_plain<true>(taddr, valid, p.out_f32 + static_cast<size_t>(row) * p.ld_out, col0,
+                            p.ld_out, half);
+          else
+            epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
+                             p.ld_out, half);
           break;
       }
       ptx::tc_fence_before();

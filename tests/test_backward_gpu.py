@@ -8,6 +8,8 @@ weight gradient -- is compared as max|g - g_ref| / max|g_ref| against the
 mode's tolerance: 1e-5 for fp32 (fp32 accumulation of sums over at most a
 few thousand terms of one sign-mixed product), 2e-2 for bf16.
 """
+from dataclasses import replace
+
 import numpy as np
 import pytest
 import torch
@@ -64,6 +66,28 @@ def test_backward_tiny_f32_relu2():
 def test_backward_tiny_f32_ragged_tokens():
     """T = 37 tokens in a workspace for 64: partial tiles everywhere."""
     _backward_case(configs.TINY_F32, T=37, max_tokens=64)
+
+
+# bf16 cases: a mid-size layer that spans several tiles of every GEMM with
+# ragged tails (T*K' = 2400 rows over 32 experts), both expert activations,
+# with a router bias; and the README acc layer's full shape at T = 256.
+MID_BF16 = configs.LayerConfig("mid_bf16_T300_d512_l256_m256_N32_K8_bias", T=300, d=512, m=256,
+                               n_experts=16, top_k=4, alpha=2, n_shared=1, m_shared=256,
+                               variant="acc", router_bias_std=0.5)
+MID_RELU2_BF16 = replace(MID_BF16, name="mid_relu2_bf16_T300_d512_l256_m192_N32_K8", m=192,
+                         m_shared=192, activation="relu2", router_bias_std=0.0)
+
+
+def test_backward_bf16_mid_swiglu_bias():
+    _backward_case(MID_BF16)
+
+
+def test_backward_bf16_mid_relu2():
+    _backward_case(MID_RELU2_BF16)
+
+
+def test_backward_bf16_readme_acc_shape():
+    _backward_case(configs.README_ACC, T=256, max_tokens=256)
 
 
 def test_backward_zero_tokens_gives_zero_gradients():

@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
+                    help="backward: time lmoe_backward (dx and every weight gradient, "
+                         "forward activations recomputed) instead of the forward")
     return ap.parse_args()
 
 
@@ -122,6 +125,23 @@ def stage_bound(flops, nbytes, peaks):
     t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     return "tensor" if t_tensor >= t_hbm else "hbm"
+
+
+def backward_flops(cfg):
+    """Algorithmic FLOPs of one lmoe_backward call: the recomputed forward
+    activations (x-GEMM, expert gate/up and down), the data gradients (dy W_y,
+    DO W_o, dAB W_gu, dXcat W_x) and the weight gradients (dy^T [u|h_s],
+    dXcat^T x, DO^T H, dAB^T zp), 2 flops per multiply-add."""
+    T, d, l, m, N, K = cfg.T, cfg.d, cfg.l, cfg.m, cfg.n_routed, cfg.k_active
+    gu = n_mats(cfg) - 1
+    nsms = cfg.n_shared * cfg.m_shared
+    TK = T * K
+    xrows = N + l + gu * nsms        # router, W_down and shared gate/up rows
+    ky = l + nsms
+    fwd = 2.0 * T * d * xrows + 2.0 * TK * l * gu * m + 2.0 * TK * m * l
+    data = 2.0 * T * d * ky + 2.0 * TK * l * m + 2.0 * TK * gu * m * l + 2.0 * T * xrows * d
+    wgt = 2.0 * T * d * ky + 2.0 * T * xrows * d + 2.0 * TK * l * m + 2.0 * TK * gu * m * l
+    return fwd + data + wgt
 
 
 def layer_flops(cfg):
@@ -202,7 +222,8 @@ def oracle_rate(cfg, inp_np, budget_s, max_tokens=None):
                      b_router=None if inp_np["b_router"] is None else inp_np["b_router"].astype(np.float64),
                      w_down=inp_np["w_down"], w_up=inp_np["w_up"], w_gate=inp_np["w_gate"],
                      w_upx=inp_np["w_upx"], w_out=inp_np["w_out"], s_gate=inp_np["s_gate"],
-                     s_up=inp_np["s_up"], s_out=inp_np["s_out"], k_active=cfg.k_active)
+                     s_up=inp_np["s_up"], s_out=inp_np["s_out"], k_active=cfg.k_active,
+                     activation=cfg.activation)
     x = inp_np["x"]
     cal = min(cfg.T, max(8, oracle.threads()))
     t0 = time.perf_counter()
@@ -451,10 +472,120 @@ def run_ours(args):
     return 0
 
 
+def oracle_backward_rate(cfg, inp_np, dy_np, budget_s):
+    """Tokens/s of the fp64 oracle's backward (dx and every weight gradient)."""
+    import numpy as np
+    import oracle
+    L = oracle.Layer(w_router=inp_np["w_router"],
+                     b_router=None if inp_np["b_router"] is None else inp_np["b_router"].astype(np.float64),
+                     w_down=inp_np["w_down"], w_up=inp_np["w_up"], w_gate=inp_np["w_gate"],
+                     w_upx=inp_np["w_upx"], w_out=inp_np["w_out"], s_gate=inp_np["s_gate"],
+                     s_up=inp_np["s_up"], s_out=inp_np["s_out"], k_active=cfg.k_active,
+                     activation=cfg.activation)
+    x = inp_np["x"]
+    cal = min(cfg.T, max(8, oracle.threads()))
+    t0 = time.perf_counter()
+    oracle.backward(L, x, dy_np[:cal], tokens=np.arange(cal))
+    per_tok = (time.perf_counter() - t0) / cal
+    n = int(max(cal, min(cfg.T, budget_s / per_tok)))
+    t0 = time.perf_counter()
+    oracle.backward(L, x, dy_np[:n], tokens=np.arange(n))
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, oracle.threads()
+
+
+def run_backward(args):
+    """One step = one lmoe_backward over the workload (the forward
+    activations it needs are recomputed inside the call)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from latent_mixture_experts_top_b200 import lmoe, synth
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    cfg = workload(args.workload)
+    inp = synth.make_inputs(cfg, args.seed, "cuda")
+    dy = synth.make_cotangent(cfg, args.seed, "cuda")
+    layer = lmoe.LatentMoELayer(cfg, inp, training=True)
+    x = inp["x"]
+    dx = torch.empty_like(x)
+    grads = {k: torch.empty(v, dtype=torch.float32, device="cuda")
+             for k, v in layer.grad_shapes().items()}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        lmoe.lmoe_backward(layer.handle, x, dy, dx, grads, cfg.T, stream)
+    torch.cuda.synchronize()
+    if lmoe.lmoe_device_status(layer.handle) != 0:
+        raise RuntimeError("device status error during warm-up")
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    launches0 = lmoe.lmoe_launches(layer.handle)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local).start()
+    for i in range(K):
+        flush.fill_(1)
+        starts[i].record(stream)
+        lmoe.lmoe_backward(layer.handle, x, dy, dx, grads, cfg.T, stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    launches = lmoe.lmoe_launches(layer.handle) - launches0
+    if lmoe.lmoe_device_status(layer.handle) != 0:
+        raise RuntimeError("device status error during timing")
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms_per_step = reduce_max_over_ranks(sum(step_ms), world, "cuda") / K
+    value = job_throughput(cfg.T, world, ms_per_step)
+    peaks, peak_src = load_peaks()
+    F = backward_flops(cfg)
+    achieved = F / (ms_per_step / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "lmoe_backward (every launch of the call)",
+                "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peak_src} (burst)", "algorithmic_per_launch": F,
+                "avg_launch_ms": ms_per_step}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dy_np = dy.float().cpu().numpy().astype(np.float64)
+        rate, n_tok, dt, cores = oracle_backward_rate(cfg, numpy_inputs(inp), dy_np, 12.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n_tok} tokens (0..{n_tok - 1}) of the T={cfg.T} workload, dx and "
+                         f"every weight gradient, fp64, {dt:.1f} s"}
+    layer.close()
+    if rank == 0:
+        line = {"metric": "LatentMoE layer backward tokens/s (1 B200), dx + all weight gradients",
+                "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic: x~N(0,1), dy~N(0,1), weights~N(0,0.02), seeded",
+                "config": dict(config_json(cfg, world), which="backward"),
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": None, "note": "no host-buffer backward call in the API"},
+                "gpu_launches": launches, "clocks": clk,
+                "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.which == "backward":
+        return run_backward(args)
     return run_ours(args)
 
 

@@ -101,8 +101,8 @@ __global__ void __launch_bounds__(256) simt_rowexpert_kernel(
     const float *__restrict__ A, int lda, const float *__restrict__ W, long long sW_e,
     long long sW_r, long long sW_k, const int32_t *__restrict__ row_expert,
     float *__restrict__ C, int ldc, int M, int Ncols, int Kd, int accumulate) {
-  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
-  const int r = blockIdx.y * 4 + (threadIdx.x >> 6);
+  const int c = blockIdx.y * 64 + (threadIdx.x & 63);
+  const int r = blockIdx.x * 4 + (threadIdx.x >> 6);
   if (r >= M || c >= Ncols) return;
   const float *a = A + static_cast<size_t>(r) * lda;
   const float *w = W + row_expert[r] * sW_e + c * sW_r;
@@ -123,8 +123,8 @@ __global__ void act_backward_kernel(const TI *__restrict__ a, const TI *__restri
                                     const float *__restrict__ dh, int lddh, TO *__restrict__ h,
                                     int ldh, TO *__restrict__ da, TO *__restrict__ db, int ldd,
                                     int rows, int n, int relu2) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  const int r = blockIdx.y;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;  // rows on x: up to 2^31 - 1
+  const int r = blockIdx.x;
   if (r >= rows || c >= n) return;
   const float bv = ld(b, static_cast<size_t>(r) * ldab + c);
   const float g = dh ? dh[static_cast<size_t>(r) * lddh + c] : 0.0f;
@@ -182,8 +182,8 @@ __global__ void slot_grad_kernel(const float *__restrict__ du, int lddu,
 template <typename TI, typename TO>
 __global__ void gather_sum_kernel(const TI *__restrict__ D, int ldD, const int32_t *__restrict__ pos,
                                   int T, int K, int n, TO *__restrict__ out, int ldo) {
-  const int t = blockIdx.y;
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int t = blockIdx.x;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
   if (t >= T || c >= n) return;
   float acc = 0.0f;
   for (int k = 0; k < K; ++k) acc += ld(D, static_cast<size_t>(pos[t * K + k]) * ldD + c);
@@ -223,8 +223,8 @@ __global__ void act_backward_tiled_kernel(const __nv_bfloat16 *__restrict__ AB, 
                                           __nv_bfloat16 *__restrict__ h, int ldh,
                                           __nv_bfloat16 *__restrict__ dAB, int lddab, int rows,
                                           int n, int relu2) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  const int r = blockIdx.y;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;  // rows on x: up to 2^31 - 1
+  const int r = blockIdx.x;
   if (r >= rows || c >= n) return;
   const size_t base = static_cast<size_t>(r) * ldab, dbase = static_cast<size_t>(r) * lddab;
   const float g = dh ? dh[static_cast<size_t>(r) * lddh + c] : 0.0f;
@@ -322,7 +322,7 @@ cudaError_t launch_act_backward_tiled(const __nv_bfloat16 *AB, int ldab, const f
                                       int lddh, __nv_bfloat16 *h, int ldh, __nv_bfloat16 *dAB,
                                       int lddab, int rows, int n, bool relu2, cudaStream_t s) {
   if (rows <= 0 || n <= 0) return cudaSuccess;
-  dim3 grid((n + 255) / 256, rows);
+  dim3 grid(rows, (n + 255) / 256);
   act_backward_tiled_kernel<<<grid, 256, 0, s>>>(AB, ldab, dh, lddh, h, ldh, dAB, lddab, rows, n,
                                                  relu2 ? 1 : 0);
   return cudaGetLastError();
@@ -365,7 +365,7 @@ cudaError_t simt_rowexpert(const float *A, int lda, const float *W, long long sW
                            long long sW_k, const int32_t *row_expert, float *C, int ldc, int M,
                            int Ncols, int Kdim, bool accumulate, cudaStream_t s) {
   if (M <= 0 || Ncols <= 0) return cudaSuccess;
-  dim3 grid((Ncols + 63) / 64, (M + 3) / 4);
+  dim3 grid((M + 3) / 4, (Ncols + 63) / 64);
   simt_rowexpert_kernel<<<grid, 256, 0, s>>>(A, lda, W, sW_e, sW_r, sW_k, row_expert, C, ldc, M,
                                              Ncols, Kdim, accumulate ? 1 : 0);
   return cudaGetLastError();
@@ -376,7 +376,7 @@ cudaError_t launch_act_backward(const TI *a, const TI *b, int ldab, const float 
                                 TO *h, int ldh, TO *da, TO *db, int ldd, int rows, int n,
                                 bool relu2, cudaStream_t s) {
   if (rows <= 0 || n <= 0) return cudaSuccess;
-  dim3 grid((n + 255) / 256, rows);
+  dim3 grid(rows, (n + 255) / 256);
   act_backward_kernel<TI, TO><<<grid, 256, 0, s>>>(a, b, ldab, dh, lddh, h, ldh, da, db, ldd, rows,
                                                    n, relu2 ? 1 : 0);
   return cudaGetLastError();
@@ -406,7 +406,7 @@ template <typename TI, typename TO>
 cudaError_t launch_gather_sum(const TI *D, int ldD, const int32_t *pos, int T, int K, int n, TO *out,
                               int ldo, cudaStream_t s) {
   if (T <= 0 || n <= 0) return cudaSuccess;
-  dim3 grid((n + 127) / 128, T);
+  dim3 grid(T, (n + 127) / 128);
   gather_sum_kernel<TI, TO><<<grid, 128, 0, s>>>(D, ldD, pos, T, K, n, out, ldo);
   return cudaGetLastError();
 }

@@ -75,8 +75,8 @@ __global__ void __launch_bounds__(256) simt_swiglu_kernel(const float *__restric
                                                           const int32_t *__restrict__ row_expert,
                                                           float *__restrict__ H, int ldh, int M,
                                                           int Ncols, int Kd) {
-  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
-  const int r = blockIdx.y * 4 + (threadIdx.x >> 6);
+  const int c = blockIdx.y * 64 + (threadIdx.x & 63);  // rows on x: up to 2^31 - 1
+  const int r = blockIdx.x * 4 + (threadIdx.x >> 6);
   if (r >= M || c >= Ncols) return;
   const float *a = A + static_cast<size_t>(r) * lda;
   const size_t wr = wrow(row_expert, r, c, mw, Kd);
@@ -95,8 +95,8 @@ __global__ void __launch_bounds__(256) simt_relu2_kernel(const float *__restrict
                                                          const int32_t *__restrict__ row_expert,
                                                          float *__restrict__ H, int ldh, int M,
                                                          int Ncols, int Kd) {
-  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
-  const int r = blockIdx.y * 4 + (threadIdx.x >> 6);
+  const int c = blockIdx.y * 64 + (threadIdx.x & 63);  // rows on x: up to 2^31 - 1
+  const int r = blockIdx.x * 4 + (threadIdx.x >> 6);
   if (r >= M || c >= Ncols) return;
   const float *a = A + static_cast<size_t>(r) * lda;
   const float *u = Wu + wrow(row_expert, r, c, mw, Kd);
@@ -110,8 +110,8 @@ __global__ void __launch_bounds__(256) simt_expert_down_kernel(
     const float *__restrict__ Hm, int ldh, const float *__restrict__ Wo,
     const int32_t *__restrict__ row_expert, float *__restrict__ O, int ldo, int M, int Ncols,
     int Kd) {
-  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
-  const int r = blockIdx.y * 4 + (threadIdx.x >> 6);
+  const int c = blockIdx.y * 64 + (threadIdx.x & 63);  // rows on x: up to 2^31 - 1
+  const int r = blockIdx.x * 4 + (threadIdx.x >> 6);
   if (r >= M || c >= Ncols) return;
   const float *h = Hm + static_cast<size_t>(r) * ldh;
   const float *w = Wo + (static_cast<size_t>(row_expert[r]) * Ncols + c) * Kd;
@@ -134,7 +134,7 @@ cudaError_t simt_swiglu(const float *A, int lda, const float *Wg, const float *W
                         const int32_t *row_expert, float *H, int ldh, int M, int Ncols, int Kdim,
                         cudaStream_t s) {
   if (M <= 0 || Ncols <= 0) return cudaSuccess;
-  dim3 grid((Ncols + 63) / 64, (M + 3) / 4);
+  dim3 grid((M + 3) / 4, (Ncols + 63) / 64);
   simt_swiglu_kernel<<<grid, 256, 0, s>>>(A, lda, Wg, Wu, mw, row_expert, H, ldh, M, Ncols, Kdim);
   return cudaGetLastError();
 }
@@ -143,7 +143,7 @@ cudaError_t simt_relu2(const float *A, int lda, const float *Wu, int mw,
                        const int32_t *row_expert, float *H, int ldh, int M, int Ncols, int Kdim,
                        cudaStream_t s) {
   if (M <= 0 || Ncols <= 0) return cudaSuccess;
-  dim3 grid((Ncols + 63) / 64, (M + 3) / 4);
+  dim3 grid((M + 3) / 4, (Ncols + 63) / 64);
   simt_relu2_kernel<<<grid, 256, 0, s>>>(A, lda, Wu, mw, row_expert, H, ldh, M, Ncols, Kdim);
   return cudaGetLastError();
 }
@@ -151,7 +151,7 @@ cudaError_t simt_relu2(const float *A, int lda, const float *Wu, int mw,
 cudaError_t simt_expert_down(const float *H, int ldh, const float *Wo, const int32_t *row_expert,
                              float *O, int ldo, int M, int Ncols, int Kdim, cudaStream_t s) {
   if (M <= 0 || Ncols <= 0) return cudaSuccess;
-  dim3 grid((Ncols + 63) / 64, (M + 3) / 4);
+  dim3 grid((M + 3) / 4, (Ncols + 63) / 64);
   simt_expert_down_kernel<<<grid, 256, 0, s>>>(H, ldh, Wo, row_expert, O, ldo, M, Ncols, Kdim);
   return cudaGetLastError();
 }

@@ -143,39 +143,80 @@ __global__ void act_backward_kernel(const TI *__restrict__ a, const TI *__restri
 }
 
 // ------------------------------------------------------------ gate gradient
-// One warp per token t: dg_k = du_t . O[pos(t,k)], gamma = sum_k g_k dg_k,
-// ds_k = g_k (dg_k - gamma); and the expert-output gradient rows
-// DO[pos(t,k)] = g_k du_t.
+// Phase 1, one warp per (token, slot) pair: dg = du_t . O[pos(t,k)] (into
+// ds for now) and the expert-output gradient row DO[pos(t,k)] = g_k du_t.
 template <typename TO>
 __global__ void slot_grad_kernel(const float *__restrict__ du, int lddu,
                                  const TO *__restrict__ O, int l, const int32_t *__restrict__ pos,
-                                 const float *__restrict__ gates, int T, int K,
+                                 const float *__restrict__ gates, int TK, int K,
                                  float *__restrict__ ds, TO *__restrict__ DO) {
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (t >= T) return;
+  if (pair >= TK) return;
+  const int t = pair / K;
   const float *dur = du + static_cast<size_t>(t) * lddu;
-  float gamma = 0.0f;
-  for (int k = 0; k < K; ++k) {
-    const int p = pos[t * K + k];
-    const TO *o = O + static_cast<size_t>(p) * l;
-    float acc = 0.0f;
-    for (int j = lane; j < l; j += 32) acc = fmaf(dur[j], ld(o, j), acc);
+  const int p = pos[pair];
+  const float g = gates[pair];
+  const TO *o = O + static_cast<size_t>(p) * l;
+  TO *dor = DO + static_cast<size_t>(p) * l;
+  float acc = 0.0f;
+  for (int j = lane; j < l; j += 32) {
+    const float dv = dur[j];
+    acc = fmaf(dv, ld(o, j), acc);
+    st(dor, j, g * dv);
+  }
 #pragma unroll
-    for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-    const float g = gates[t * K + k];
-    gamma = fmaf(g, acc, gamma);
-    if (lane == 0) ds[t * K + k] = acc;  // dg_k for now
-    TO *dor = DO + static_cast<size_t>(p) * l;
-    for (int j = lane; j < l; j += 32) st(dor, j, g * dur[j]);
-  }
-  __syncwarp();
-  if (lane < K) {
-    for (int k = lane; k < K; k += 32) {
-      const float g = gates[t * K + k];
-      ds[t * K + k] = g * (ds[t * K + k] - gamma);
+  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+  if (lane == 0) ds[pair] = acc;
+}
+
+// Phase 2, one thread per token: ds_k = g_k (dg_k - sum_j g_j dg_j).
+__global__ void gate_grad_kernel(const float *__restrict__ gates, int T, int K,
+                                 float *__restrict__ ds) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  float gamma = 0.0f;
+  for (int k = 0; k < K; ++k) gamma = fmaf(gates[t * K + k], ds[t * K + k], gamma);
+  for (int k = 0; k < K; ++k) ds[t * K + k] = gates[t * K + k] * (ds[t * K + k] - gamma);
+}
+
+// bf16 specialisation of phase 1: each lane moves 8 columns (16 bytes of O
+// and DO) at a time; l % 8 == 0.
+template <>
+__global__ void slot_grad_kernel<__nv_bfloat16>(const float *__restrict__ du, int lddu,
+                                                const __nv_bfloat16 *__restrict__ O, int l,
+                                                const int32_t *__restrict__ pos,
+                                                const float *__restrict__ gates, int TK, int K,
+                                                float *__restrict__ ds,
+                                                __nv_bfloat16 *__restrict__ DO) {
+  const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (pair >= TK) return;
+  const int t = pair / K;
+  const float *dur = du + static_cast<size_t>(t) * lddu;
+  const int p = pos[pair];
+  const float g = gates[pair];
+  const uint4 *o = reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l);
+  uint4 *dor = reinterpret_cast<uint4 *>(DO + static_cast<size_t>(p) * l);
+  float acc = 0.0f;
+  for (int v = lane; v < l / 8; v += 32) {
+    const uint4 ov = o[v];
+    const float4 d0 = *reinterpret_cast<const float4 *>(dur + 8 * v);
+    const float4 d1 = *reinterpret_cast<const float4 *>(dur + 8 * v + 4);
+    const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+    uint32_t outw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(dv[2 * i], __uint_as_float(ow[i] << 16), acc);
+      acc = fmaf(dv[2 * i + 1], __uint_as_float(ow[i] & 0xFFFF0000u), acc);
+      outw[i] = pack_bf16x2(g * dv[2 * i], g * dv[2 * i + 1]);
     }
+    dor[v] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
   }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+  if (lane == 0) ds[pair] = acc;
 }
 
 // dz[t][:] = sum_k D[pos(t,k)][:] in slot order (fp32 accumulation).
@@ -269,6 +310,57 @@ __global__ void transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ src, int
   for (int i = ty; i < 32; i += 8) {
     const int c = c0 + i;
     if (c < C) dst[static_cast<long long>(c) * ldd + col] = tile[tx][i];
+  }
+}
+
+// Token-major transpose for the weight-gradient GEMMs: dst[c][kstart[e] + j]
+// = src[offsets[e] + j][c] for the j < rows_e rows of expert e, and 0 for
+// rows_e <= j < klen[e] (the padding each expert's K range runs over).
+// Dense form (kstart == null): one block of T rows, zero-padded to a
+// multiple of 64.  One CTA per 64 tokens x 64 columns, 16-byte global loads
+// and stores on both sides.  C, lds, ldd multiples of 8.
+__global__ void __launch_bounds__(256) transpose_tokens_kernel(
+    const __nv_bfloat16 *__restrict__ src, int lds, int C, const int32_t *__restrict__ offsets,
+    const int32_t *__restrict__ kstart, int N, int T_dense, __nv_bfloat16 *__restrict__ dst,
+    long long ldd) {
+  __shared__ uint32_t tile[64][33];  // 64 tokens x 64 bf16 (33-word rows)
+  const int k0 = blockIdx.x * 64, c0 = blockIdx.y * 64;
+  int row0, rows;
+  if (kstart) {
+    if (k0 >= kstart[N]) return;
+    int lo = 0, hi = N;  // expert e with kstart[e] <= k0 < kstart[e+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (kstart[mid] <= k0) lo = mid; else hi = mid;
+    }
+    row0 = offsets[lo] + (k0 - kstart[lo]);
+    rows = offsets[lo + 1] - row0;
+  } else {
+    row0 = k0;
+    rows = T_dense - k0;
+  }
+  for (int v = threadIdx.x; v < 512; v += 256) {  // 64 tokens x 8 vectors of 8 columns
+    const int rr = v >> 3, cv = (v & 7) * 8;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (rr < rows && c0 + cv < C)
+      val = *reinterpret_cast<const uint4 *>(src + static_cast<size_t>(row0 + rr) * lds + c0 + cv);
+    uint32_t *t = &tile[rr][cv >> 1];
+    t[0] = val.x; t[1] = val.y; t[2] = val.z; t[3] = val.w;
+  }
+  __syncthreads();
+  const unsigned short *t16 = reinterpret_cast<const unsigned short *>(&tile[0][0]);
+  for (int v = threadIdx.x; v < 512; v += 256) {  // 64 columns x 8 vectors of 8 tokens
+    const int cc = v >> 3, kv = (v & 7) * 8;
+    if (c0 + cc >= C) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo16 = t16[(kv + 2 * i) * 66 + cc];
+      const uint32_t hi16 = t16[(kv + 2 * i + 1) * 66 + cc];
+      w[i] = lo16 | (hi16 << 16);
+    }
+    *reinterpret_cast<uint4 *>(dst + static_cast<long long>(c0 + cc) * ldd + k0 + kv) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -392,7 +484,22 @@ template <typename TO>
 cudaError_t launch_slot_grad(const float *du, int lddu, const TO *O, int l, const int32_t *pos,
                              const float *gates, int T, int K, float *ds, TO *DO, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  slot_grad_kernel<TO><<<(T + 7) / 8, 256, 0, s>>>(du, lddu, O, l, pos, gates, T, K, ds, DO);
+  const int TK = T * K;
+  slot_grad_kernel<TO><<<(TK + 7) / 8, 256, 0, s>>>(du, lddu, O, l, pos, gates, TK, K, ds, DO);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  gate_grad_kernel<<<(T + 255) / 256, 256, 0, s>>>(gates, T, K, ds);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_tokens(const __nv_bfloat16 *src, int lds, int C,
+                                    const int32_t *offsets, const int32_t *kstart, int N,
+                                    int64_t k_cols, int T_dense, __nv_bfloat16 *dst, long long ldd,
+                                    cudaStream_t s) {
+  if (C <= 0 || k_cols <= 0) return cudaSuccess;
+  if (C % 8 || lds % 8 || ldd % 8) return cudaErrorInvalidValue;
+  dim3 grid(static_cast<unsigned>((k_cols + 63) / 64), (C + 63) / 64);
+  transpose_tokens_kernel<<<grid, 256, 0, s>>>(src, lds, C, offsets, kstart, N, T_dense, dst, ldd);
   return cudaGetLastError();
 }
 template cudaError_t launch_slot_grad<float>(const float *, int, const float *, int,

@@ -107,6 +107,11 @@ struct TcParams {
                        // the accumulator as is (bf16 gate/up pre-activations)
   __nv_bfloat16 *out2; int ld_out2;  // TC_X_FUSED shared region, with raw
   float *out_f32;      // TC_OUT / TC_EXPERT_DOWN: fp32 output [rows][ld_out]
+  __nv_bfloat16 *out_h; int ld_h;  // TC_EXPERT_GU with raw: the hidden h as well
+  // TC_EXPERT_DOWN computing dH = DO W_o[e]: instead of storing dH, the
+  // epilogue applies the activation backward with the pre-activations
+  // act_ab [rows][ld_ab] (gate/up layout of the GU GEMM) and writes act_dab.
+  const __nv_bfloat16 *act_ab; __nv_bfloat16 *act_dab; int ld_ab;
   // TC_WGRAD: A [M][*] and B [*][*] are plain row-major token-major matrices
   // (K runs along their rows' contiguous axis); group g reduces over
   // K-columns [k_start[g], k_start[g] + k_len[g]) (multiples of 64; dense:
@@ -187,6 +192,14 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int lds, int R, int 
                                   __nv_bfloat16 *dst, long long ldd, cudaStream_t s,
                                   int batch = 1, long long src_batch = 0,
                                   long long dst_batch = 0);
+// Token-major transpose for the weight gradients: dst[c][kstart[e] + j] =
+// src[offsets[e] + j][c] (zeros up to klen[e]); dense (kstart null): T_dense
+// rows, zero-padded to a multiple of 64.  k_cols: the destination columns to
+// cover (grouped: the workspace width; dense: round64(T)).
+cudaError_t launch_transpose_tokens(const __nv_bfloat16 *src, int lds, int C,
+                                    const int32_t *offsets, const int32_t *kstart, int N,
+                                    int64_t k_cols, int T_dense, __nv_bfloat16 *dst, long long ldd,
+                                    cudaStream_t s);
 // Zeros dst[c][kstart[e] + rows_e .. kstart[e] + klen[e]) for c < n_rows.
 cudaError_t launch_zero_pad_cols(__nv_bfloat16 *dst, long long ldd, int n_rows,
                                  const int32_t *offsets, const int32_t *kstart,

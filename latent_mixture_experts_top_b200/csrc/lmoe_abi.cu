@@ -878,12 +878,11 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
     p.mode = TC_EXPERT_GU; p.Kdim = l; p.n_tiles_n = (gu + kTileN - 1) / kTileN; p.raw = 1;
     p.relu2 = h->relu2; p.n_cols2 = m;
     p.tiles = w.tiles; p.n_mtiles = w.n_tiles;
-    p.out = static_cast<bf *>(b.AB); p.ld_out = gu; p.status = w.status;
+    p.out = static_cast<bf *>(b.AB); p.ld_out = gu;
+    p.out_h = static_cast<bf *>(w.H); p.ld_h = m;  // and the hidden
+    p.status = w.status;
     LMOE_TRY(gemm(h->tm_zp, h->tm_wgu, p, h->num_sms));
   }
-  ++L;
-  LMOE_TRY(launch_act_backward_tiled(static_cast<bf *>(b.AB), gu, nullptr, 0,
-                                     static_cast<bf *>(w.H), m, nullptr, 0, TK, m, relu2, s));
   {
     TcParams p = {};  // expert outputs O
     p.mode = TC_EXPERT_DOWN; p.Kdim = m; p.n_tiles_n = (l + kTileN - 1) / kTileN;
@@ -907,22 +906,20 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
   if (nsms > 0) {
     ++L;
     LMOE_TRY(launch_act_backward_tiled(static_cast<bf *>(b.ABs), h->sh_rows, b.dU + l, ky,
-                                       ucat + l, ky, dXcat + n_pad + l_pad, nx, T, nsms, relu2, s));
+                                       nullptr, 0, dXcat + n_pad + l_pad, nx, T, nsms, relu2, s));
   }
   // ---- gates, expert-output gradients, expert backward
   ++L;
   LMOE_TRY(launch_slot_grad<bf>(b.dU, ky, static_cast<bf *>(w.O), l, w.pos, w.gates, T, K, b.ds,
                                 static_cast<bf *>(b.DO), s));
   {
-    TcParams p = {};  // dH = DO W_o[e]  (fp32 [TK][m])
+    TcParams p = {};  // dH = DO W_o[e], then dAB = activation backward (in the epilogue)
     p.mode = TC_EXPERT_DOWN; p.Kdim = l; p.n_tiles_n = (m + kTileN - 1) / kTileN;
     p.tiles = w.tiles; p.n_mtiles = w.n_tiles;
-    p.out_f32 = b.dH; p.ld_out = m; p.status = w.status;
+    p.ld_out = m; p.relu2 = h->relu2; p.status = w.status;
+    p.act_ab = static_cast<const bf *>(b.AB); p.act_dab = static_cast<bf *>(b.dAB); p.ld_ab = gu;
     LMOE_TRY(gemm(h->tm_DO, h->tm_woT, p, h->num_sms));
   }
-  ++L;
-  LMOE_TRY(launch_act_backward_tiled(static_cast<bf *>(b.AB), gu, b.dH, m, nullptr, 0,
-                                     static_cast<bf *>(b.dAB), gu, TK, m, relu2, s));
   {
     TcParams p = {};  // dZp = dAB W_gu[e]  (fp32 [TK][l])
     p.mode = TC_EXPERT_DOWN; p.Kdim = gu; p.n_tiles_n = (l + kTileN - 1) / kTileN;
@@ -957,18 +954,14 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
   };
   L += 4;
   // (row stride b.Tp, the maps' width; this call reduces over Tp columns)
-  LMOE_TRY(launch_transpose_bf16(static_cast<const bf *>(dy), d, T, d, nullptr, nullptr,
-                                 static_cast<bf *>(b.dyT), b.Tp, s));
-  LMOE_TRY(launch_transpose_bf16(ucat, ky, T, ky, nullptr, nullptr, static_cast<bf *>(b.ucatT),
-                                 b.Tp, s));
-  LMOE_TRY(launch_transpose_bf16(dXcat, nx, T, nx, nullptr, nullptr, static_cast<bf *>(b.dXcatT),
-                                 b.Tp, s));
-  LMOE_TRY(launch_transpose_bf16(static_cast<const bf *>(x), d, T, d, nullptr, nullptr,
-                                 static_cast<bf *>(b.xT), b.Tp, s));
-  LMOE_TRY(zero_cols(static_cast<bf *>(b.dyT), b.Tp, T, Tp, d));
-  LMOE_TRY(zero_cols(static_cast<bf *>(b.ucatT), b.Tp, T, Tp, ky));
-  LMOE_TRY(zero_cols(static_cast<bf *>(b.dXcatT), b.Tp, T, Tp, nx));
-  LMOE_TRY(zero_cols(static_cast<bf *>(b.xT), b.Tp, T, Tp, d));
+  LMOE_TRY(launch_transpose_tokens(static_cast<const bf *>(dy), d, d, nullptr, nullptr, 0, Tp, T,
+                                   static_cast<bf *>(b.dyT), b.Tp, s));
+  LMOE_TRY(launch_transpose_tokens(ucat, ky, ky, nullptr, nullptr, 0, Tp, T,
+                                   static_cast<bf *>(b.ucatT), b.Tp, s));
+  LMOE_TRY(launch_transpose_tokens(dXcat, nx, nx, nullptr, nullptr, 0, Tp, T,
+                                   static_cast<bf *>(b.dXcatT), b.Tp, s));
+  LMOE_TRY(launch_transpose_tokens(static_cast<const bf *>(x), d, d, nullptr, nullptr, 0, Tp, T,
+                                   static_cast<bf *>(b.xT), b.Tp, s));
   {
     TcParams p = {};  // [dW_up | dS_o] = dy^T [u | h_s]
     p.mode = TC_WGRAD; p.wg_kind = WG_Y; p.groups = 1; p.M = d; p.Kdim = static_cast<int>(Tp);
@@ -988,20 +981,16 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
     LMOE_TRY(launch_bias_grad(b.ds, w.offsets, w.perm, N, g->b_router, s));
   }
   // grouped: each expert's rows at a 64-aligned K range of the transposes
-  L += 9;
+  L += 5;
   LMOE_TRY(launch_padded_offsets(w.offsets, N, b.kstart, b.klen, b.shift, s));
-  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(b.DO), l, TK, l, w.row_expert, b.shift,
-                                 static_cast<bf *>(b.DOT), Kp, s));
-  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(w.H), m, TK, m, w.row_expert, b.shift,
-                                 static_cast<bf *>(b.HT), Kp, s));
-  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(b.dAB), gu, TK, gu, w.row_expert, b.shift,
-                                 static_cast<bf *>(b.dABT), Kp, s));
-  LMOE_TRY(launch_transpose_bf16(static_cast<bf *>(w.zp), l, TK, l, w.row_expert, b.shift,
-                                 static_cast<bf *>(b.zpT), Kp, s));
-  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.DOT), Kp, l, w.offsets, b.kstart, b.klen, N, s));
-  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.HT), Kp, m, w.offsets, b.kstart, b.klen, N, s));
-  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.dABT), Kp, gu, w.offsets, b.kstart, b.klen, N, s));
-  LMOE_TRY(launch_zero_pad_cols(static_cast<bf *>(b.zpT), Kp, l, w.offsets, b.kstart, b.klen, N, s));
+  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(b.DO), l, l, w.offsets, b.kstart, N, Kp, 0,
+                                   static_cast<bf *>(b.DOT), Kp, s));
+  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(w.H), m, m, w.offsets, b.kstart, N, Kp, 0,
+                                   static_cast<bf *>(b.HT), Kp, s));
+  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(b.dAB), gu, gu, w.offsets, b.kstart, N, Kp, 0,
+                                   static_cast<bf *>(b.dABT), Kp, s));
+  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(w.zp), l, l, w.offsets, b.kstart, N, Kp, 0,
+                                   static_cast<bf *>(b.zpT), Kp, s));
   {
     TcParams p = {};  // dW_o[e] = DO_e^T H_e
     p.mode = TC_WGRAD; p.wg_kind = WG_O; p.groups = N; p.M = l; p.Kdim = 64;

@@ -276,6 +276,111 @@ __device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bflo
   }
 }
 
+// Raw gate/up pre-activations (row segment raw_dst, 256 columns as in the
+// accumulator) and the SwiGLU hidden (h_dst + hcol0) of one tile.
+__device__ __forceinline__ void epi_swiglu_raw(uint32_t taddr, bool valid,
+                                               __nv_bfloat16 *raw_dst, __nv_bfloat16 *h_dst,
+                                               int half) {
+#pragma unroll 1
+  for (int c = half * (TN / 128); c < (half + 1) * (TN / 128); ++c) {
+    uint32_t g[32], u[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, g);
+    ptx::tmem_ld_32x32b_x32(taddr + TN / 2 + c * 32, u);
+    ptx::tmem_ld_wait();
+    float gv[32], uv[32], h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      gv[j] = __uint_as_float(g[j]);
+      uv[j] = __uint_as_float(u[j]);
+      h[j] = silu_bf16out(gv[j]) * uv[j];
+    }
+    if (valid) {
+      store_bf16x32(raw_dst + c * 32, gv);
+      store_bf16x32(raw_dst + TN / 2 + c * 32, uv);
+      store_bf16x32(h_dst + c * 32, h);
+    }
+  }
+}
+
+// Squared ReLU: raw up pre-activation and h = relu(b)^2, masked at n_cols.
+__device__ __forceinline__ void epi_relu2_raw(uint32_t taddr, bool valid, __nv_bfloat16 *raw_dst,
+                                              __nv_bfloat16 *h_dst, int col0, int n_cols,
+                                              int half) {
+#pragma unroll 1
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+    uint32_t r[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+    ptx::tmem_ld_wait();
+    float bv[32], h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      bv[j] = __uint_as_float(r[j]);
+      const float a = fmaxf(bv[j], 0.0f);
+      h[j] = a * a;
+    }
+    const int col = col0 + c * 32;
+    if (valid && col < n_cols) {
+      store_bf16x32(raw_dst + col, bv);
+      store_bf16x32(h_dst + col, h);
+    }
+  }
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16 *src, float *v) {
+  const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 w = s4[q];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * q + 2 * i] = __uint_as_float(ws[i] << 16);
+      v[8 * q + 2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// dh (accumulator) of hidden units col0 .. col0+255 of row `row` -> the
+// pre-activation gradients, written in the GU GEMM's layout:
+// SwiGLU da = dh b silu'(a), db = dh silu(a); squared ReLU db = dh 2 relu(b).
+__device__ __forceinline__ void epi_act_backward(uint32_t taddr, bool valid, const TcParams &p,
+                                                 int row, int col0, int n_units, int half) {
+#pragma unroll 1
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+    uint32_t r[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+    ptx::tmem_ld_wait();
+    const int col = col0 + c * 32;
+    if (!valid || col >= n_units) continue;
+    const size_t base = static_cast<size_t>(row) * p.ld_ab;
+    if (p.relu2) {
+      float bv[32], db[32];
+      load_bf16x32(p.act_ab + base + col, bv);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) db[j] = __uint_as_float(r[j]) * 2.0f * fmaxf(bv[j], 0.0f);
+      store_bf16x32(p.act_dab + base + col, db);
+    } else {
+      const size_t ia = base + 256 * (col >> 7) + (col & 127), ib = ia + 128;
+      float av[32], bv[32], da[32], db[32];
+      load_bf16x32(p.act_ab + ia, av);
+      load_bf16x32(p.act_ab + ib, bv);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float dh = __uint_as_float(r[j]);
+        const float sg = 1.0f / (1.0f + __expf(-av[j]));
+        da[j] = dh * bv[j] * sg * (1.0f + av[j] * (1.0f - sg));
+        db[j] = dh * av[j] * sg;
+      }
+      store_bf16x32(p.act_dab + ia, da);
+      store_bf16x32(p.act_dab + ib, db);
+    }
+  }
+}
+
+// kBwd: the instantiation with the backward's epilogues and the TC_WGRAD
+// mode; the forward launches the other one, whose smaller register budget
+// leaves room for the routing kernels that run beside it.
+template <bool kBwd>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcParams p) {
@@ -424,9 +529,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else if (col0 < p.z_end) {
             epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
                              col0 - p.r_end, p.l, half);
-          } else if (p.raw) {
-            epi_plain<false>(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2,
-                             col0 - p.z_end, p.ld_out2, half);
+          } else if (kBwd && p.raw) {  // pre-activations and the hidden
+            if (p.relu2)
+              epi_relu2_raw(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2,
+                            p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
+                            col0 - p.z_end, p.n_cols2, half);
+            else
+              epi_swiglu_raw(taddr, valid,
+                             p.out2 + static_cast<size_t>(row) * p.ld_out2 + (col0 - p.z_end),
+                             p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0 +
+                                 (col0 - p.z_end) / 2,
+                             half);
           } else if (p.relu2) {
             epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
                       col0 - p.z_end, p.n_cols2, half);
@@ -436,9 +549,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           break;
         case TC_EXPERT_GU:
-          if (p.raw)
-            epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
-                             p.ld_out, half);
+          if (kBwd && p.raw && p.relu2)
+            epi_relu2_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
+                          p.out_h + static_cast<size_t>(row) * p.ld_h, col0, p.n_cols2, half);
+          else if (kBwd && p.raw)
+            epi_swiglu_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + col0,
+                           p.out_h + static_cast<size_t>(row) * p.ld_h + col0 / 2, half);
           else if (p.relu2)
             epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0, p.n_cols2,
                       half);
@@ -446,10 +562,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
           break;
         case TC_WGRAD:
-          epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
+          if constexpr (kBwd) epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
           break;
         default:  // TC_EXPERT_DOWN, TC_OUT
-          if (p.out_f32)
+          if (kBwd && p.act_dab)
+            epi_act_backward(taddr, valid, p, row, col0, p.ld_out, half);
+          else if (kBwd && p.out_f32)
             epi_plain<true>(taddr, valid, p.out_f32 + static_cast<size_t>(row) * p.ld_out, col0,
                             p.ld_out, half);
           else
@@ -531,18 +649,26 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_done != dev) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     attr_done = dev;
   }
+  const bool bwd = p.mode == TC_WGRAD || p.raw || p.act_dab || p.out_f32 || p.out_h;
   if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
   CUtensorMap a, b;
   memcpy(&a, tmapA, sizeof(a));
   memcpy(&b, tmapB, sizeof(b));
-  tc_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
+  if (bwd)
+    tc_gemm_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
+  else
+    tc_gemm_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
   return cudaGetLastError();
 }
 

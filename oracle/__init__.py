@@ -82,6 +82,8 @@ def _load():
             lib.oracle_shared.restype = None
             lib.oracle_backward.argtypes = [P, P, I64, P, I64, P, P, P]
             lib.oracle_backward.restype = C.c_int
+            lib.oracle_fp8_rows.argtypes = [P, I32, I64, I32, P, P]
+            lib.oracle_fp8_rows.restype = None
             lib.oracle_threads.argtypes = []
             lib.oracle_threads.restype = C.c_int
             _lib = lib
@@ -305,6 +307,19 @@ def backward(layer: Layer, x, dy, tokens=None, ids=None, want=GRAD_NAMES):
     if rc != 0:
         raise ValueError(f"oracle_backward failed ({rc})")
     return out
+
+
+def fp8_rows(w):
+    """Row-wise E4M3 quantisation with power-of-two scales (see the C source):
+    returns (W' dequantised, float64, same shape; scales [rows])."""
+    w = np.ascontiguousarray(w)
+    code = _dtype_code(w)
+    cols = w.shape[-1]
+    rows = w.size // cols
+    wq = np.empty(w.shape, dtype=np.float64)
+    sc = np.empty(rows, dtype=np.float64)
+    _load().oracle_fp8_rows(_ptr(w), code, rows, cols, _ptr(wq), _ptr(sc))
+    return wq, sc
 
 
 def threads() -> int:

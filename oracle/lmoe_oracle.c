@@ -597,6 +597,63 @@ done:
   return err;
 }
 
+/* ---- FP8 expert weights (the "LatentMoE Explained" remark that an expert
+ * is 22 MB in FP8, and the models' NVFP4 pretraining; the pages give no
+ * scaling recipe, so this one is chosen and stated): every weight row r of
+ * an expert matrix gets a power-of-two scale s_r = 2^e_r, the smallest with
+ * max_c |W[r][c]| <= 448 s_r (448 = the largest finite E4M3 value), and each
+ * element is stored as q = E4M3(W[r][c] / s_r); the layer then uses
+ * W'[r][c] = q * s_r.  E4M3 (the OCP 8-bit floating point format, E4M3
+ * variant): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; normal values 2^(E-7) (1 + M/8) for E in 1..15 (E = 15, M = 7
+ * is NaN, so the largest is 2^8 * 1.75 = 448); subnormals 2^-6 * M/8 (spacing
+ * 2^-9).  Rounding is to nearest, ties to even mantissa, and out-of-range
+ * magnitudes saturate to 448.  A row of zeros gets s = 1. */
+static double e4m3_round(double v) {
+  const double a = fabs(v);
+  if (a == 0.0) return 0.0 * v;
+  double r;
+  if (a >= 448.0) {
+    r = 448.0;
+  } else {
+    int e;
+    frexp(a, &e);               /* a = f * 2^e, f in [0.5, 1): a in [2^(e-1), 2^e) */
+    int ex = e - 1;             /* a in [2^ex, 2^(ex+1)) */
+    if (ex < -6) ex = -6;       /* below the normal range: subnormal spacing */
+    const double q = ldexp(1.0, ex - 3);  /* spacing of 3 mantissa bits */
+    const double n = a / q;     /* exact: q is a power of two */
+    double k = floor(n);
+    const double frac = n - k;
+    if (frac > 0.5 || (frac == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0;
+    r = k * q;
+    if (r > 448.0) r = 448.0;
+  }
+  return v < 0.0 ? -r : r;
+}
+
+/* W [rows][cols] (any element type) -> W' (double) and the row scales. */
+void oracle_fp8_rows(const void *W, int dt, int64_t rows, int cols, double *Wq,
+                     double *scales) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    double amax = 0.0;
+    for (int c = 0; c < cols; ++c) {
+      const double v = fabs(elem(W, dt, (size_t)r * cols + c));
+      if (v > amax) amax = v;
+    }
+    int e = 0;  /* smallest e with amax <= 448 * 2^e */
+    if (amax > 0.0) {
+      e = (int)ceil(log2(amax / 448.0));
+      while (ldexp(448.0, e) < amax) ++e;
+      while (e > -200 && ldexp(448.0, e - 1) >= amax) --e;
+    }
+    const double s = ldexp(1.0, e);
+    scales[r] = s;
+    for (int c = 0; c < cols; ++c)
+      Wq[(size_t)r * cols + c] = e4m3_round(elem(W, dt, (size_t)r * cols + c) / s) * s;
+  }
+}
+
 int oracle_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -50,7 +50,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="readme_acc",
-                    choices=["readme_acc", "readme_eff", "prefill", "decode", "relu2_95b"])
+                    choices=["readme_acc", "readme_eff", "prefill", "decode", "relu2_95b",
+                             "decode_fp8", "relu2_95b_fp8"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
@@ -64,7 +65,8 @@ def workload(name):
     from latent_mixture_experts_top_b200 import configs
     return {"readme_acc": configs.README_ACC, "readme_eff": configs.README_EFF,
             "prefill": configs.PREFILL, "decode": configs.DECODE,
-            "relu2_95b": configs.RELU2_95B}[name]
+            "relu2_95b": configs.RELU2_95B, "decode_fp8": configs.DECODE_FP8,
+            "relu2_95b_fp8": configs.RELU2_95B_FP8}[name]
 
 
 def n_mats(cfg):
@@ -76,6 +78,7 @@ def config_json(cfg, n_gpus):
     return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "l": cfg.l, "m": cfg.m,
             "n_routed": cfg.n_routed, "k_active": cfg.k_active, "n_shared": cfg.n_shared,
             "m_shared": cfg.m_shared, "variant": cfg.variant, "activation": cfg.activation,
+            "expert_weights": cfg.weights,
             "router_bias": cfg.has_router_bias, "global_batch": cfg.T * n_gpus,
             "seq_len": cfg.T, "parallelism": f"replicas x{n_gpus} (no exchange)",
             "l2": "flushed by a 512 MiB write between timed steps"}
@@ -107,14 +110,15 @@ def stage_work(cfg, touched=None):
     E = N if touched is None else touched
     TK = T * K
     gu = n_mats(cfg) - 1          # gate+up (2) or up (1) rows per hidden column
+    ew = expert_weight_bytes(cfg)
     ky = l + ns * ms
     return {
         0: (2.0 * T * d * (N + l), 2.0 * T * d + 2.0 * d * (N + l) + 4.0 * T * N + 2.0 * T * l),
         1: (0.0, 4.0 * T * N + 8.0 * TK),
         2: (0.0, 4.0 * TK * 5),
         3: (0.0, 2.0 * TK * l * 2 + 4.0 * TK),
-        4: (2.0 * TK * l * gu * m, 2.0 * TK * l + 2.0 * E * gu * m * l + 2.0 * TK * m),
-        5: (2.0 * TK * m * l, 2.0 * TK * m + 2.0 * E * l * m + 2.0 * TK * l),
+        4: (2.0 * TK * l * gu * m, 2.0 * TK * l + ew * E * gu * m * l + 2.0 * TK * m),
+        5: (2.0 * TK * m * l, 2.0 * TK * m + ew * E * l * m + 2.0 * TK * l),
         6: (0.0, 2.0 * TK * l + 8.0 * TK + 2.0 * T * l),
         7: (2.0 * T * ky * d, 2.0 * T * ky + 2.0 * d * ky + 2.0 * T * d),
     }
@@ -150,14 +154,21 @@ def layer_flops(cfg):
     return 2.0 * T * (d * N + 2 * d * l + nm * K * l * m + nm * cfg.n_shared * d * cfg.m_shared)
 
 
+def expert_weight_bytes(cfg):
+    """Bytes per routed-expert weight: 2 (bf16), or 1 (E4M3) plus one f32
+    scale per weight row (row length >= 512, so < 0.01 byte per weight)."""
+    return 1.0 if cfg.weights == "fp8" else 2.0
+
+
 def layer_bytes(cfg, ids=None):
     """Weights actually touched (router, projections, shared, the distinct
-    experts hit) + x in + y out, bf16."""
+    experts hit) + x in + y out; bf16 except E4M3 routed experts."""
     d, l, m, N = cfg.d, cfg.l, cfg.m, cfg.n_routed
     touched = N if ids is None else len(set(ids.reshape(-1).tolist()))
     nm = n_mats(cfg)
-    w = N * d + 2 * d * l + nm * cfg.n_shared * d * cfg.m_shared + touched * nm * l * m
-    return 2.0 * (w + 2 * cfg.T * d)
+    w = N * d + 2 * d * l + nm * cfg.n_shared * d * cfg.m_shared
+    experts = touched * nm * l * m * expert_weight_bytes(cfg)
+    return 2.0 * (w + 2 * cfg.T * d) + experts
 
 
 # ---------------------------------------------------------------- clocks

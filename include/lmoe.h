@@ -57,6 +57,15 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
  * activation its 95B running example uses.  Shared experts use the same. */
 typedef enum { LMOE_SWIGLU = 0, LMOE_RELU2 = 1 } lmoe_activation;
 
+/* Storage of the routed experts' weights (W_g, W_u, W_o) in LMOE_BF16 mode.
+ * LMOE_WEIGHTS_FP8: E4M3 with one power-of-two scale per weight row (the
+ * smallest that brings the row's largest magnitude within 448), for the
+ * weight-streaming decode regime ("LatentMoE Explained" puts an expert at
+ * about 22 MB in FP8; the pages give no scaling recipe, this is the one
+ * chosen).  The layer then computes exactly with W' = E4M3(W / s) * s.
+ * Not with training = 1. */
+typedef enum { LMOE_WEIGHTS_BF16 = 0, LMOE_WEIGHTS_FP8 = 1 } lmoe_weight_format;
+
 enum {
   LMOE_OK = 0,
   LMOE_ERR_INVALID_CONFIG = -1,  /* d % alpha != 0, K' outside [1, N'], sizes <= 0 */
@@ -89,6 +98,7 @@ typedef struct {
   int32_t training;          /* 1: lmoe_backward is available (the handle
                                 keeps the extra weight layouts and workspace
                                 the backward needs); 0: forward only */
+  int32_t weight_format;     /* lmoe_weight_format (bf16 dtype only) */
 } lmoe_config;
 
 typedef struct lmoe_layer *lmoe_handle;
@@ -174,7 +184,11 @@ int lmoe_selftest_wait_timeout(lmoe_handle h, int64_t limit_ns, void *stream);
  * (which: 0 logits f32 [T][N'], 1 z [T][l], 2 permuted z [T*K'][l],
  * 3 expert hidden [T*K'][m], 4 expert out [T*K'][l], 5 [u | shared hidden]
  * [T][l + n_s m_s], 6 ids, 7 gates, 8 offsets, 9 perm, 10 pos [T*K'] (inverse
- * of perm), 11 number of 128-row expert tiles).  Errors: NULL_ARG,
+ * of perm), 11 number of 128-row expert tiles; with LMOE_WEIGHTS_FP8 also
+ * 12 gate/up E4M3 codes and 14 W_o E4M3 codes (bytes, in 256 x 64 tiles:
+ * expert, 256-row tile, 64-column block, row, column), 13 gate/up row scales
+ * [N'][2m, gate and up rows interleaved in blocks of 128; m rows of W_u for
+ * squared ReLU] and 15 W_o row scales [N'][l], f32).  Errors: NULL_ARG,
  * INVALID_CONFIG (unknown `which`). */
 int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel);
 

@@ -32,6 +32,7 @@ class LayerConfig:
     top_k_override: int = 0
     router_bias_std: float = 0.0   # > 0: per-expert router bias ~ N(0, std)
     activation: str = "swiglu"     # "swiglu" (3 matrices) | "relu2" (2 matrices)
+    weights: str = "bf16"          # routed experts' weights: "bf16" | "fp8" (E4M3, row scales)
     x_std: float = 1.0
     w_std: float = 0.02
 
@@ -81,6 +82,12 @@ RELU2_95B = LayerConfig("relu2_95b_T1024_d4096_l1024_m2688_N512_K24", T=1024, d=
                         m=2688, n_experts=128, top_k=6, alpha=4, n_shared=2, m_shared=2688,
                         variant="acc", activation="relu2")
 
+# The decode workload with E4M3 routed-expert weights ("LatentMoE Explained":
+# an expert is about 22 MB in FP8), and the 95B squared-ReLU shape likewise.
+DECODE_FP8 = replace(DECODE, name="decode_fp8_T64_d4096_l1024_m2048_N512_K22", weights="fp8")
+RELU2_95B_FP8 = replace(RELU2_95B, name="relu2_95b_fp8_T1024_d4096_l1024_m2688_N512_K24",
+                        weights="fp8")
+
 CONFIGS = [TINY_F32, README_ACC, README_EFF, PREFILL, DECODE]
-EXTRA_CONFIGS = [TINY_RELU2_F32, RELU2_95B]
+EXTRA_CONFIGS = [TINY_RELU2_F32, RELU2_95B, DECODE_FP8, RELU2_95B_FP8]
 BY_NAME = {c.name: c for c in CONFIGS + EXTRA_CONFIGS}

@@ -112,6 +112,10 @@ struct TcParams {
   // epilogue applies the activation backward with the pre-activations
   // act_ab [rows][ld_ab] (gate/up layout of the GU GEMM) and writes act_dab.
   const __nv_bfloat16 *act_ab; __nv_bfloat16 *act_dab; int ld_ab;
+  // FP8 expert weights (TC_EXPERT_GU / TC_EXPERT_DOWN): B is E4M3 (tiled like
+  // the bf16 weights, 1 byte per element) and b_scale [expert][b_scale_ld]
+  // holds each weight row's scale.
+  const float *b_scale; int b_scale_ld;
   // TC_WGRAD: A [M][*] and B [*][*] are plain row-major token-major matrices
   // (K runs along their rows' contiguous axis); group g reduces over
   // K-columns [k_start[g], k_start[g] + k_len[g]) (multiples of 64; dense:
@@ -134,6 +138,17 @@ inline int64_t btile_rows(int groups, int rows_per_group, int cols) {
 }
 cudaError_t launch_repack_btiles(const __nv_bfloat16 *src, int groups, int rows_per_group,
                                  int cols, __nv_bfloat16 *dst, cudaStream_t s);
+
+// E4M3 expert weights (fp8_weights.cu): src [groups][rows][cols] bf16 ->
+// per-row power-of-two scales [groups][rows] and E4M3 codes, K-block tiled
+// like launch_repack_btiles (1 byte per element; padding rows zero).
+cudaError_t launch_quantize_e4m3_tiles(const __nv_bfloat16 *src, int groups, int rows_per_group,
+                                       int cols, float *scales, uint8_t *dst, cudaStream_t s);
+
+// Encodes a 2-D byte tensor map (rows x cols bytes, row stride in bytes)
+// with a {64, box_rows} box and no swizzle.  Host only.
+int make_tmap_u8(void *tmap_out, const void *base, int64_t rows, int64_t cols,
+                 int64_t row_stride_bytes, int box_rows);
 
 // Encodes a 2-D bf16 K-major tensor map (rows x cols, row stride in
 // elements) with a {64, box_rows} box and 128-byte swizzle.  Host only.
@@ -212,7 +227,10 @@ cudaError_t launch_padded_offsets(const int32_t *offsets, int N, int32_t *kstart
 // Failure-detection self-test (see lmoe_selftest_wait_timeout).
 cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s);
 
+// tmapA32: with E4M3 weights (p.b_scale set), the same A matrix with a
+// {64, 32} box, used for tiles of at most 32 token rows.
 cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p,
-                           int num_sms, int max_ctas, cudaStream_t s);
+                           int num_sms, int max_ctas, cudaStream_t s,
+                           const void *tmapA32 = nullptr);
 
 }  // namespace lmoe

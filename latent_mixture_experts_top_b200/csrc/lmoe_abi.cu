@@ -74,6 +74,7 @@ struct lmoe_layer {
   int d = 0, l = 0, m = 0, N = 0, K = 0, ns = 0, ms = 0, Tmax = 0;
   int bf16 = 0;
   int relu2 = 0;      // squared-ReLU experts (two matrices)
+  int fp8 = 0;        // E4M3 routed-expert weights
   size_t esize = 4;
   int device = 0, num_sms = 0;
   bool loaded = false;
@@ -105,6 +106,10 @@ struct lmoe_layer {
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
+  TensorMap64 tm_zp32, tm_h32;  // E4M3 weights: {64, 32} boxes for small tiles
+  // E4M3 expert weights (tiled like w_gu / w_out) and their row scales
+  uint8_t *w_gu8 = nullptr, *w_o8 = nullptr;
+  float *gu_scale = nullptr, *o_scale = nullptr;
   // bf16 training: transposed weights (K-block tiled) and backward maps
   void *w_yT = nullptr;   // [ky][d]
   void *w_oT = nullptr;   // [N][m][l]
@@ -148,7 +153,8 @@ void free_all(lmoe_layer *h) {
                   h->bw.as, h->bw.bs, h->bw.das, h->bw.dbs, h->bw.dsfull, h->bw.AB,
                   h->bw.ABs, h->bw.dAB, h->bw.dXcat, h->bw.DOT, h->bw.HT, h->bw.dABT,
                   h->bw.zpT, h->bw.dyT, h->bw.ucatT, h->bw.dXcatT, h->bw.xT, h->bw.kstart,
-                  h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT};
+                  h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT, h->w_gu8,
+                  h->w_o8, h->gu_scale, h->o_scale};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
@@ -184,6 +190,10 @@ int validate(const lmoe_config *c, lmoe_layer *h) {
   h->Tmax = c->max_tokens;
   h->bf16 = c->dtype == LMOE_BF16;
   h->relu2 = c->activation == LMOE_RELU2;
+  if (c->weight_format != LMOE_WEIGHTS_BF16 && c->weight_format != LMOE_WEIGHTS_FP8)
+    return LMOE_ERR_INVALID_CONFIG;
+  h->fp8 = c->weight_format == LMOE_WEIGHTS_FP8;
+  if (h->fp8 && (c->dtype != LMOE_BF16 || c->training)) return LMOE_ERR_UNSUPPORTED;
   h->esize = h->bf16 ? 2 : 4;
   h->ky = h->l + h->ns * h->ms;
   if (static_cast<int64_t>(h->Tmax) * h->K > INT32_MAX / 2) return LMOE_ERR_UNSUPPORTED;
@@ -268,9 +278,14 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     if (h->bf16) {
       // K-block-tiled B operands (see launch_repack_btiles)
       ok = dalloc(&h->w_x, btile_rows(1, h->nx_rows, h->d) * 64 * es) &&
-           dalloc(&h->w_gu, btile_rows(h->N, h->gu_rows, h->l) * 64 * es) &&
-           dalloc(&h->w_out, btile_rows(h->N, h->l, h->m) * 64 * es) &&
            dalloc(&h->w_y, btile_rows(1, h->d, h->ky) * 64 * es);
+      if (ok && h->fp8)
+        ok = dalloc(&h->w_gu8, btile_rows(h->N, h->gu_rows, h->l) * 64) &&
+             dalloc(&h->w_o8, btile_rows(h->N, h->l, h->m) * 64) &&
+             dalloc(&h->gu_scale, N * h->gu_rows * 4) && dalloc(&h->o_scale, N * l * 4);
+      else if (ok)
+        ok = dalloc(&h->w_gu, btile_rows(h->N, h->gu_rows, h->l) * 64 * es) &&
+             dalloc(&h->w_out, btile_rows(h->N, h->l, h->m) * 64 * es);
     } else {
       ok = dalloc(&h->w_router, N * d * es) && dalloc(&h->w_down, l * d * es) &&
            (h->relu2 || dalloc(&h->w_gate, N * m * l * es)) &&
@@ -329,10 +344,21 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     // B operands: [tiled rows][64], one {64, 256} box per K-block tile
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wx, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN);
-    if (rc == LMOE_OK)
-      rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->N, h->gu_rows, h->l), 64, 64, kTileN);
-    if (rc == LMOE_OK)
-      rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN);
+    if (rc == LMOE_OK && h->fp8) {
+      rc = make_map(&h->tm_zp32, w.zp, static_cast<int64_t>(TK), h->l, h->l, 32);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_h32, w.H, static_cast<int64_t>(TK), h->m, h->m, 32);
+    }
+    if (rc == LMOE_OK && h->fp8) {  // E4M3 tiles: {64 bytes, 256 rows}, no swizzle
+      if (make_tmap_u8(h->tm_wgu.bytes, h->w_gu8, btile_rows(h->N, h->gu_rows, h->l), 64, 64,
+                       kTileN) != 0 ||
+          make_tmap_u8(h->tm_wo.bytes, h->w_o8, btile_rows(h->N, h->l, h->m), 64, 64, kTileN) != 0)
+        rc = LMOE_ERR_CUDA;
+    } else {
+      if (rc == LMOE_OK)
+        rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->N, h->gu_rows, h->l), 64, 64, kTileN);
+      if (rc == LMOE_OK)
+        rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN);
+    }
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wy, h->w_y, btile_rows(1, h->d, h->ky), 64, 64, kTileN);
     if (rc == LMOE_OK && h->training) {
@@ -453,12 +479,21 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   if (e == cudaSuccess)
     e = launch_repack_btiles(static_cast<const bf *>(tx), 1, h->nx_rows, h->d,
                              static_cast<bf *>(h->w_x), s);
-  if (e == cudaSuccess)  // expert up rows: interleaved gate/up, or the up-projection itself
-    e = launch_repack_btiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->N,
-                             h->gu_rows, h->l, static_cast<bf *>(h->w_gu), s);
-  if (e == cudaSuccess)
-    e = launch_repack_btiles(static_cast<const bf *>(wt->w_out), h->N, h->l, h->m,
-                             static_cast<bf *>(h->w_out), s);
+  if (h->fp8) {  // E4M3 codes + row scales, tiled like the bf16 weights
+    if (e == cudaSuccess)
+      e = launch_quantize_e4m3_tiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->N,
+                                     h->gu_rows, h->l, h->gu_scale, h->w_gu8, s);
+    if (e == cudaSuccess)
+      e = launch_quantize_e4m3_tiles(static_cast<const bf *>(wt->w_out), h->N, h->l, h->m,
+                                     h->o_scale, h->w_o8, s);
+  } else {
+    if (e == cudaSuccess)  // expert up rows: interleaved gate/up, or the up-projection itself
+      e = launch_repack_btiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->N,
+                               h->gu_rows, h->l, static_cast<bf *>(h->w_gu), s);
+    if (e == cudaSuccess)
+      e = launch_repack_btiles(static_cast<const bf *>(wt->w_out), h->N, h->l, h->m,
+                               static_cast<bf *>(h->w_out), s);
+  }
   if (e == cudaSuccess)
     e = launch_repack_btiles(static_cast<const bf *>(ty), 1, h->d, h->ky,
                              static_cast<bf *>(h->w_y), s);
@@ -660,11 +695,16 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.n_cols2 = h->m;
     p.tiles = w.tiles;
     p.n_mtiles = w.n_tiles;
+    if (h->fp8) {
+      p.b_scale = h->gu_scale;
+      p.b_scale_ld = h->gu_rows;
+    }
     p.b_rows_per_expert = h->gu_rows;
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
     p.status = w.status;
-    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s);
+    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s,
+                       h->tm_zp32.bytes);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 5, s);
@@ -678,7 +718,12 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     pd.out = static_cast<__nv_bfloat16 *>(w.O);
     pd.ld_out = h->l;
     pd.status = w.status;
-    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s);
+    if (h->fp8) {
+      pd.b_scale = h->o_scale;
+      pd.b_scale_ld = h->l;
+    }
+    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s,
+                       h->tm_h32.bytes);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 6, s);
@@ -1106,6 +1151,13 @@ int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *num
     case 9: *dev_ptr = w.perm; *numel = TK; break;
     case 10: *dev_ptr = w.pos; *numel = TK; break;
     case 11: *dev_ptr = w.n_tiles; *numel = 1; break;
+    case 12: case 13: case 14: case 15:
+      if (!h->fp8) return LMOE_ERR_INVALID_CONFIG;
+      if (which == 12) { *dev_ptr = h->w_gu8; *numel = btile_rows(h->N, h->gu_rows, h->l) * 64; }
+      if (which == 13) { *dev_ptr = h->gu_scale; *numel = static_cast<int64_t>(h->N) * h->gu_rows; }
+      if (which == 14) { *dev_ptr = h->w_o8; *numel = btile_rows(h->N, h->l, h->m) * 64; }
+      if (which == 15) { *dev_ptr = h->o_scale; *numel = static_cast<int64_t>(h->N) * h->l; }
+      break;
     default: return LMOE_ERR_INVALID_CONFIG;
   }
   return LMOE_OK;

@@ -47,31 +47,56 @@ namespace lmoe {
 namespace {
 
 constexpr int TM = 128, TN = 256, TKB = 64;   // tile M, N, K-block
-constexpr int STAGES = 4;
 constexpr int A_BYTES = TM * TKB * 2;         // 16 KB
-constexpr int B_BYTES = TN * TKB * 2;         // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int B_BYTES = TN * TKB * 2;         // 32 KB (16-bit B tile)
 constexpr int TMEM_COLS = 2 * TN;             // two accumulators
 constexpr int NUM_EPI_WARPS = 8;              // two per TMEM lane quarter
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, TN);
 
+// Pipeline shape.  Default: a STAGES-deep ring of (A, B) tiles filled by TMA
+// and read by the MMA.  kFp8 (weights in E4M3): the same ring carries A and
+// the E4M3 weight tile (16 KB instead of 32 KB), four converter warps move
+// each weight tile to bf16 in the 128-byte-swizzled layout into a second,
+// S2-deep ring, and the MMA reads A from the first ring and B from the
+// second.  A first-ring slot is free once the converters and the MMAs are
+// both done with it.
+template <bool kFp8>
+struct Cfg {
+  static constexpr int STAGES = 4;
+  static constexpr int S2 = kFp8 ? 3 : 0;           // kFp8: converted-B ring
+  static constexpr int B_LOAD = kFp8 ? TN * TKB : B_BYTES;  // weight bytes per TMA stage
+  // kFp8 (weight streaming, few rows per tile): four epilogue warps, one per
+  // TMEM lane quarter covering both column halves, and eight converter
+  // warps, two per scheduler, so that the conversion's latency is hidden.
+  static constexpr int EPI_WARPS = kFp8 ? 4 : NUM_EPI_WARPS;
+  static constexpr int CONV_WARPS = kFp8 ? 8 : 0;
+  static constexpr int NUM_THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
+  static constexpr int RING_BYTES = STAGES * (A_BYTES + B_LOAD) + S2 * B_BYTES;
+};
+
+constexpr int MAX_STAGES = 8;
 struct __align__(8) SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
+  uint64_t conv[MAX_STAGES];    // kFp8: ring-2 slot holds A and the converted B
+  uint64_t conv_empty[MAX_STAGES];  // kFp8: the MMAs have read the ring-2 slot
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemCtl);
+template <bool kFp8>
+constexpr size_t smem_bytes() {
+  return 1024 /*align slack*/ + Cfg<kFp8>::RING_BYTES + sizeof(SmemCtl);
+}
 
 struct Tile {
   int a_row, b_row, n_tile, row_hi;
   int k0;     // first K column (A, and B when b_plain)
   int nkb;    // K-blocks of this tile
   int group;  // TC_WGRAD group
+  int expert; // grouped modes: the expert of the tile
   bool b_plain;  // B is a plain row-major matrix (else K-block tiled)
 };
 
@@ -80,6 +105,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
   tl.k0 = 0;
   tl.nkb = p.Kdim / TKB;
   tl.group = 0;
+  tl.expert = 0;
   tl.b_plain = false;
   if (p.mode == TC_WGRAD) {
     const int per = m_tiles * p.n_tiles_n;
@@ -104,6 +130,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
   } else {
     const int mt = t / p.n_tiles_n, n = t % p.n_tiles_n;  // consecutive CTAs share A
     const TileEntry te = p.tiles[mt];
+    tl.expert = te.expert;
     tl.a_row = te.row0;
     tl.b_row = (te.expert * p.n_tiles_n + n) * (p.Kdim / TKB) * TN;
     tl.n_tile = n;
@@ -377,19 +404,128 @@ __device__ __forceinline__ void epi_act_backward(uint32_t taddr, bool valid, con
   }
 }
 
+// ---- epilogues of the FP8-weight variant: the accumulator column c holds
+// 2^-120 times the product with the E4M3 codes (see convert_stage), so it is
+// scaled by the weight row's scale scl[c] times 2^120.
+constexpr float kTwo120 = 1.329227995784916e36f;  // 2^120, exact in f32
+
+__device__ __forceinline__ void epi_swiglu_scaled(uint32_t taddr, bool valid,
+                                                  __nv_bfloat16 *row_dst, int hcol0,
+                                                  const float *scl, int half) {
+#pragma unroll 1
+  for (int c = half * (TN / 128); c < (half + 1) * (TN / 128); ++c) {
+    uint32_t g[32], u[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, g);
+    ptx::tmem_ld_32x32b_x32(taddr + TN / 2 + c * 32, u);
+    ptx::tmem_ld_wait();
+    float h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      h[j] = silu_bf16out(__uint_as_float(g[j]) * (scl[c * 32 + j] * kTwo120)) *
+             (__uint_as_float(u[j]) * (scl[TN / 2 + c * 32 + j] * kTwo120));
+    if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
+  }
+}
+
+__device__ __forceinline__ void epi_relu2_scaled(uint32_t taddr, bool valid,
+                                                 __nv_bfloat16 *row_dst, int col0, int n_cols,
+                                                 const float *scl, int half) {
+#pragma unroll 1
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+    const int col = col0 + c * 32;
+    uint32_t r[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+    ptx::tmem_ld_wait();
+    if (!valid || col >= n_cols) continue;
+    float h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float a = fmaxf(__uint_as_float(r[j]) * (scl[c * 32 + j] * kTwo120), 0.0f);
+      h[j] = a * a;
+    }
+    store_bf16x32(row_dst + col, h);
+  }
+}
+
+__device__ __forceinline__ void epi_plain_scaled(uint32_t taddr, bool valid,
+                                                 __nv_bfloat16 *row_dst, int col0, int n_cols,
+                                                 const float *scl, int half) {
+#pragma unroll 1
+  for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+    const int col = col0 + c * 32;
+    uint32_t r[32];
+    ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+    ptx::tmem_ld_wait();
+    if (!valid || col >= n_cols) continue;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * (scl[c * 32 + j] * kTwo120);
+    store_bf16x32(row_dst + col, v);
+  }
+}
+
+constexpr int CONV_THREADS = 256;  // Cfg<true>::CONV_WARPS * 32
+
+// Converter role (kFp8): moves one stage's E4M3 B tile (256 rows x 64
+// bytes, TMA-loaded without swizzle) into bf16 in the 128-byte-swizzled
+// K-major layout: element (r, k) at byte r*128 + (((k/8) ^ (r%8)) * 16) +
+// (k%8)*2.  No arithmetic conversion: an E4M3 code (sign s, exponent field
+// E, mantissa M) with its sign moved to bit 15 and its 7 magnitude bits to
+// bits 4..10 is the bf16 bit pattern of (its value) * 2^-120 exactly -- for
+// E >= 1 a normal bf16 with exponent field E and mantissa M/8, for E = 0
+// (the E4M3 subnormals M/8 * 2^-6) the bf16 subnormal M/8 * 2^-126.  The
+// epilogue multiplies by the row scale times 2^120.  Each of the 256 threads
+// moves 4 groups of 16 codes; the reads, and each 8-thread phase of the
+// writes, hit distinct banks.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_scaled(uint32_t t) {
+  // t: code 0 in bits 0..7, code 1 in bits 16..23 (other bits zero).
+  // (t << 4) puts the magnitudes at bits 4..10 / 20..26 and the signs at
+  // bits 11 / 27; adding sign * (2^8 - 2^4) moves each sign to bit 15 / 31.
+  return (t << 4) + (t & 0x00800080u) * 240u;
+}
+
+__device__ __forceinline__ void convert_stage(const uint8_t *b8, uint8_t *b16, int ctid) {
+#pragma unroll
+  for (int i = 0; i < 1024 / CONV_THREADS; ++i) {
+    const int item = ctid + CONV_THREADS * i;
+    const int r = item >> 2, j = item & 3;
+    const uint4 q = *reinterpret_cast<const uint4 *>(b8 + r * 64 + j * 16);
+    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+    uint32_t hw[8];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      hw[2 * w] = e4m3x2_to_bf16x2_scaled(__byte_perm(qw[w], 0u, 0x4140));
+      hw[2 * w + 1] = e4m3x2_to_bf16x2_scaled(__byte_perm(qw[w], 0u, 0x4342));
+    }
+    const int c0 = 2 * j, sw = r & 7;
+    *reinterpret_cast<uint4 *>(b16 + r * 128 + ((c0 ^ sw) << 4)) =
+        make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4 *>(b16 + r * 128 + (((c0 + 1) ^ sw) << 4)) =
+        make_uint4(hw[4], hw[5], hw[6], hw[7]);
+  }
+}
+
 // kBwd: the instantiation with the backward's epilogues and the TC_WGRAD
 // mode; the forward launches the other one, whose smaller register budget
 // leaves room for the routing kernels that run beside it.
-template <bool kBwd>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// kFp8: expert weights in E4M3 (TC_EXPERT_GU / TC_EXPERT_DOWN with b_scale):
+// four more warps convert each stage's weight tile to f16 for the MMA.
+template <bool kBwd, bool kFp8>
+__global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmA32, const TcParams p) {
+  constexpr int STAGES = Cfg<kFp8>::STAGES;
+  constexpr int S2 = Cfg<kFp8>::S2;
+  constexpr int S2M = S2 > 0 ? S2 : 1;  // ring-2 index arithmetic (kFp8 only)
+  constexpr int B_LOAD = Cfg<kFp8>::B_LOAD;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // [A ring][B ring (E4M3 if kFp8)][kFp8: converted-B ring]
   uint8_t *smA = smem;
   uint8_t *smB = smem + STAGES * A_BYTES;
-  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + STAGES * STAGE_BYTES);
+  uint8_t *smBc = smB + STAGES * B_LOAD;
+  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + Cfg<kFp8>::RING_BYTES);
   volatile int *abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -402,11 +538,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&ctl->full[s], 1);
-      ptx::mbar_init(&ctl->empty[s], 1);
+      // freed by the MMA commit (kFp8: and by each converter warp)
+      ptx::mbar_init(&ctl->empty[s], 1 + Cfg<kFp8>::CONV_WARPS);
+    }
+    for (int s = 0; s < S2; ++s) {
+      ptx::mbar_init(&ctl->conv[s], Cfg<kFp8>::CONV_WARPS);
+      ptx::mbar_init(&ctl->conv_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&ctl->acc_full[a], 1);
-      ptx::mbar_init(&ctl->acc_empty[a], NUM_EPI_WARPS);  // one arrival per epilogue warp
+      ptx::mbar_init(&ctl->acc_empty[a], Cfg<kFp8>::EPI_WARPS);  // one per epilogue warp
     }
     ptx::mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -414,6 +555,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&tmA);
+    if (kFp8) ptx::prefetch_tmap(&tmA32);
     ptx::prefetch_tmap(&tmB);
   }
   if (warp == 1) {
@@ -440,13 +582,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
           const int kx = tl.k0 + kb * TKB;
-          ptx::tma_load_2d(smA + s * A_BYTES, &tmA, &ctl->full[s], kx, tl.a_row);
+          // kFp8 (weight streaming): a tile of at most 32 token rows loads
+          // only those rows of A (the MMA's other rows are never stored)
+          const bool a32 = kFp8 && tl.row_hi - tl.a_row <= 32;
+          ptx::mbar_arrive_expect_tx(&ctl->full[s], (a32 ? A_BYTES / 4 : A_BYTES) + B_LOAD);
+          ptx::tma_load_2d(smA + s * A_BYTES, a32 ? &tmA32 : &tmA, &ctl->full[s], kx, tl.a_row);
           if (tl.b_plain)
-            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kx, tl.b_row);
+            ptx::tma_load_2d(smB + s * B_LOAD, &tmB, &ctl->full[s], kx, tl.b_row);
           else
-            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
+            ptx::tma_load_2d(smB + s * B_LOAD, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
         }
       }
       if (!ok) {  // let every copy still in flight land before the CTA exits
@@ -472,22 +617,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + acc * TN;
         const int nkb = decode_tile(p, t, m_tiles).nkb;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!ptx::mbar_wait(&ctl->full[s], ph, abort_flag)) {
+          const int s = it % STAGES, s2 = it % S2M;
+          const uint32_t ph = (it / STAGES) & 1, ph2 = (it / S2M) & 1;
+          // kFp8: the converted B of this K-block (its A landed before it)
+          if (!ptx::mbar_wait(kFp8 ? &ctl->conv[s2] : &ctl->full[s], kFp8 ? ph2 : ph,
+                              abort_flag)) {
             record_failure(p, ctl, DEV_TIMEOUT_MMA);
             ok = false;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(smA + s * A_BYTES);
-          const uint32_t b_addr = ptx::smem_u32(smB + s * B_BYTES);
+          const uint32_t b_addr =
+              ptx::smem_u32(kFp8 ? smBc + s2 * B_BYTES : smB + s * B_LOAD);
 #pragma unroll
           for (int k = 0; k < TKB / 16; ++k) {
             ptx::mma_bf16(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
                           ptx::smem_desc_sw128(b_addr + k * 32), IDESC, (kb | k) != 0);
           }
-          ptx::mma_commit(&ctl->empty[s]);  // ring stage free once these MMAs finish
+          // the stage (kFp8: and the converted-B slot) is free once these MMAs finish
+          ptx::mma_commit(&ctl->empty[s]);
+          if constexpr (kFp8) ptx::mma_commit(&ctl->conv_empty[s2]);
         }
         if (!ok) break;
         ptx::mma_commit(&ctl->acc_full[acc]);  // accumulator ready for the epilogue
@@ -497,10 +647,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!drain_wait(&ctl->drain, 0)) record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
       }
     }
+  } else if (kFp8 && warp >= 2 + Cfg<kFp8>::EPI_WARPS) {
+    // ------------------------------------------------------------ converters
+    const int ctid = threadIdx.x - 32 * (2 + Cfg<kFp8>::EPI_WARPS);
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int nkb = decode_tile(p, t, m_tiles).nkb;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % STAGES, s2 = it % S2M;
+        const uint32_t ph = (it / STAGES) & 1, ph2 = (it / S2M) & 1;
+        int w_ok = 1;
+        if (lane == 0) {  // converted-B slot free, then this stage's tiles landed
+          w_ok = ptx::mbar_wait(&ctl->conv_empty[s2], ph2 ^ 1, abort_flag) ? 1 : 0;
+          if (w_ok) w_ok = ptx::mbar_wait(&ctl->full[s], ph, abort_flag) ? 1 : 0;
+        }
+        w_ok = __shfl_sync(0xFFFFFFFFu, w_ok, 0);
+        if (!w_ok) {
+          if (lane == 0) record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
+          ok = false;
+          break;
+        }
+        convert_stage(smB + s * B_LOAD, smBc + s2 * B_BYTES, ctid);
+        // generic-proxy writes -> visible to the tensor core's async-proxy reads
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(&ctl->conv[s2]);
+          ptx::mbar_arrive(&ctl->empty[s]);  // done with the stage's E4M3 tile
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;   // which half of the tile's columns
+    // which half of the tile's columns (both, one after the other, when the
+    // variant has one epilogue warp per lane quarter)
+    constexpr int kHalfStep = Cfg<kFp8>::EPI_WARPS / 4;
+    const int half0 = (warp - 2) >> 2;
     const int row_in_tile = q * 32 + lane;
     int tl_count = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl_count) {
@@ -521,6 +705,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool valid = row < tl.row_hi;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
       const int col0 = tl.n_tile * TN;
+      for (int half = half0; half < 2; half += kHalfStep) {
       switch (p.mode) {
         case TC_X_FUSED:
           if (col0 < p.r_end) {
@@ -549,7 +734,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           break;
         case TC_EXPERT_GU:
-          if (kBwd && p.raw && p.relu2)
+          if constexpr (kFp8) {
+            const float *scl = p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0;
+            __nv_bfloat16 *hrow = p.out + static_cast<size_t>(row) * p.ld_out;
+            if (p.relu2) epi_relu2_scaled(taddr, valid, hrow, col0, p.n_cols2, scl, half);
+            else epi_swiglu_scaled(taddr, valid, hrow, col0 / 2, scl, half);
+          } else if (kBwd && p.raw && p.relu2)
             epi_relu2_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
                           p.out_h + static_cast<size_t>(row) * p.ld_h, col0, p.n_cols2, half);
           else if (kBwd && p.raw)
@@ -565,7 +755,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if constexpr (kBwd) epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
           break;
         default:  // TC_EXPERT_DOWN, TC_OUT
-          if (kBwd && p.act_dab)
+          if constexpr (kFp8) {
+            epi_plain_scaled(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
+                             p.ld_out,
+                             p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0,
+                             half);
+          } else if (kBwd && p.act_dab)
             epi_act_backward(taddr, valid, p, row, col0, p.ld_out, half);
           else if (kBwd && p.out_f32)
             epi_plain<true>(taddr, valid, p.out_f32 + static_cast<size_t>(row) * p.ld_out, col0,
@@ -575,6 +770,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                              p.ld_out, half);
           break;
       }
+      }  // halves
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
@@ -643,32 +839,64 @@ int make_tmap_bf16(void *tmap_out, const void *base, int64_t rows, int64_t cols,
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
+int make_tmap_u8(void *tmap_out, const void *base, int64_t rows, int64_t cols,
+                 int64_t row_stride_bytes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0 || cols <= 0) return -1;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || row_stride_bytes % 16) return -1;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(TKB), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(reinterpret_cast<CUtensorMap *>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+         const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
 cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p, int num_sms,
-                           int max_ctas, cudaStream_t s) {
+                           int max_ctas, cudaStream_t s, const void *tmapA32) {
   static int attr_done = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_done != dev) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<false>,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<false, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SMEM_BYTES));
+                                         static_cast<int>(smem_bytes<false>()));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(SMEM_BYTES));
+      e = cudaFuncSetAttribute(tc_gemm_kernel<true, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes<false>()));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_gemm_kernel<false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes<true>()));
     if (e != cudaSuccess) return e;
     attr_done = dev;
   }
   const bool bwd = p.mode == TC_WGRAD || p.raw || p.act_dab || p.out_f32 || p.out_h;
+  const bool fp8 = p.b_scale != nullptr;
+  if (fp8 && (bwd || (p.mode != TC_EXPERT_GU && p.mode != TC_EXPERT_DOWN)))
+    return cudaErrorInvalidValue;
   if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
-  CUtensorMap a, b;
+  if (fp8 && !tmapA32) return cudaErrorInvalidValue;
+  CUtensorMap a, b, a32;
   memcpy(&a, tmapA, sizeof(a));
   memcpy(&b, tmapB, sizeof(b));
-  if (bwd)
-    tc_gemm_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
+  memcpy(&a32, fp8 ? tmapA32 : tmapA, sizeof(a32));
+  if (fp8)
+    tc_gemm_kernel<false, true>
+        <<<grid, Cfg<true>::NUM_THREADS, smem_bytes<true>(), s>>>(a, b, a32, p);
+  else if (bwd)
+    tc_gemm_kernel<true, false>
+        <<<grid, Cfg<false>::NUM_THREADS, smem_bytes<false>(), s>>>(a, b, a32, p);
   else
-    tc_gemm_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b, p);
+    tc_gemm_kernel<false, false>
+        <<<grid, Cfg<false>::NUM_THREADS, smem_bytes<false>(), s>>>(a, b, a32, p);
   return cudaGetLastError();
 }
 

@@ -24,6 +24,7 @@ _lib = C.CDLL(_LIB_PATH)
 LMOE_EFF, LMOE_ACC = 0, 1
 LMOE_F32, LMOE_BF16 = 0, 1
 LMOE_SWIGLU, LMOE_RELU2 = 0, 1
+LMOE_WEIGHTS_BF16, LMOE_WEIGHTS_FP8 = 0, 1
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -3: "LMOE_ERR_NOT_LOADED", -4: "LMOE_ERR_TOO_MANY_TOKENS", -5: "LMOE_ERR_CUDA",
           -6: "LMOE_ERR_DEVICE_TIMEOUT", -7: "LMOE_ERR_UNSUPPORTED",
@@ -41,7 +42,7 @@ class lmoe_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "d", "m", "n_experts", "top_k", "alpha", "n_shared", "m_shared", "variant", "dtype",
         "n_routed_override", "top_k_override", "has_router_bias", "max_tokens", "activation",
-        "training")]
+        "training", "weight_format")]
 
 
 class lmoe_weights(C.Structure):
@@ -127,7 +128,8 @@ def config_from(cfg: LayerConfig, max_tokens: int | None = None,
         has_router_bias=int(cfg.has_router_bias),
         max_tokens=cfg.T if max_tokens is None else max_tokens,
         activation=LMOE_RELU2 if cfg.activation == "relu2" else LMOE_SWIGLU,
-        training=int(training))
+        training=int(training),
+        weight_format=LMOE_WEIGHTS_FP8 if cfg.weights == "fp8" else LMOE_WEIGHTS_BF16)
 
 
 def lmoe_create(config: lmoe_config) -> int:
@@ -294,7 +296,7 @@ class LatentMoELayer:
             pass
 
 
-_TYPESTR = {torch.float32: "<f4", torch.bfloat16: "<u2", torch.int32: "<i4"}
+_TYPESTR = {torch.float32: "<f4", torch.bfloat16: "<u2", torch.int32: "<i4", torch.uint8: "|u1"}
 
 
 def device_view(ptr: int, numel: int, dtype: torch.dtype, shape) -> torch.Tensor:

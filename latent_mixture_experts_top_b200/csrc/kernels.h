@@ -124,6 +124,12 @@ struct TcParams {
   const int32_t *k_start, *k_len;
   int wg_d, wg_l, wg_m, wg_ns, wg_ms, wg_n, wg_npad, wg_lpad;  // layer sizes for the destinations
   float *g_router, *g_down, *g_up, *g_gate, *g_upx, *g_out, *g_sgate, *g_sup, *g_sout;
+  // Forward bf16 outputs (z, H, O, y; not the fp32 router logits): with
+  // tma_out set, an epilogue warp whose 32 rows are all valid stages each
+  // 32 x 32 block in shared memory and writes it with one TMA store through
+  // the launch's output tensor map (launch_tc_gemm's tmapOut); other warps
+  // store directly.
+  int tma_out;
   int32_t *status;
 };
 
@@ -154,6 +160,12 @@ int make_tmap_u8(void *tmap_out, const void *base, int64_t rows, int64_t cols,
 // elements) with a {64, box_rows} box and 128-byte swizzle.  Host only.
 int make_tmap_bf16(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
                    int64_t cols, int64_t row_stride_elems, int box_rows);
+
+// Encodes a 2-D bf16 tensor map of an output matrix (rows x cols, row stride
+// in elements) with a {32, 32} box and 64-byte swizzle, for the GEMM
+// epilogue's TMA stores.  Host only.
+int make_tmap_bf16_out(void *tmap_out /*CUtensorMap, 64 B*/, const void *base, int64_t rows,
+                       int64_t cols, int64_t row_stride_elems);
 
 // ---- backward (backward_kernels.cu)
 // fp32 CUDA-core GEMM with arbitrary strides: C[g](i, j) (+)= sum_k
@@ -229,8 +241,10 @@ cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream
 
 // tmapA32: with E4M3 weights (p.b_scale set), the same A matrix with a
 // {64, 32} box, used for tiles of at most 32 token rows.
+// tmapOut: with p.tma_out set (forward bf16 modes only), the bf16 output
+// matrix's map from make_tmap_bf16_out (z for TC_X_FUSED).
 cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p,
                            int num_sms, int max_ctas, cudaStream_t s,
-                           const void *tmapA32 = nullptr);
+                           const void *tmapA32 = nullptr, const void *tmapOut = nullptr);
 
 }  // namespace lmoe

@@ -106,6 +106,7 @@ struct lmoe_layer {
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
+  TensorMap64 tm_out_z, tm_out_h, tm_out_o;  // epilogue TMA stores: z, H, O
   TensorMap64 tm_zp32, tm_h32;  // E4M3 weights: {64, 32} boxes for small tiles
   // E4M3 expert weights (tiled like w_gu / w_out) and their row scales
   uint8_t *w_gu8 = nullptr, *w_o8 = nullptr;
@@ -341,6 +342,11 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TK), h->l, h->l, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, static_cast<int64_t>(TK), h->m, h->m, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_ucat, w.ucat, h->Tmax, h->ky, h->ky, kTileM);
+    if (rc == LMOE_OK &&
+        (make_tmap_bf16_out(h->tm_out_z.bytes, w.z, h->Tmax, h->l, h->l) != 0 ||
+         make_tmap_bf16_out(h->tm_out_h.bytes, w.H, static_cast<int64_t>(TK), h->m, h->m) != 0 ||
+         make_tmap_bf16_out(h->tm_out_o.bytes, w.O, static_cast<int64_t>(TK), h->l, h->l) != 0))
+      rc = LMOE_ERR_CUDA;
     // B operands: [tiled rows][64], one {64, 256} box per K-block tile
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wx, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN);
@@ -588,8 +594,10 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.relu2 = h->relu2;
     p.n_cols2 = h->ns * h->ms;
     p.status = w.status;
+    p.tma_out = 1;  // z through TMA stores (the logits are stored directly)
     const int m_tiles = (T + kTileM - 1) / kTileM;
-    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, m_tiles * p.n_tiles_n, s);
+    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, m_tiles * p.n_tiles_n, s,
+                       nullptr, h->tm_out_z.bytes);
     h->launches += 1;
     const int shared_tiles_n = (h->nx_rows - h->n_pad - h->l_pad) / kTileN;
     if (e == cudaSuccess && full && shared_tiles_n > 0) {
@@ -598,6 +606,9 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       TcParams q = p;
       q.n_tile_base = (h->n_pad + h->l_pad) / kTileN;
       q.n_tiles_n = shared_tiles_n;
+      // direct stores: the smaller shared-memory footprint lets the routing
+      // kernels run beside this launch's CTAs
+      q.tma_out = 0;
       if (shared_raw) {
         q.raw = 1;
         q.out2 = static_cast<__nv_bfloat16 *>(shared_raw);
@@ -703,8 +714,9 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
     p.status = w.status;
+    p.tma_out = h->fp8 ? 0 : 1;
     e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s,
-                       h->tm_zp32.bytes);
+                       h->tm_zp32.bytes, h->tm_out_h.bytes);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 5, s);
@@ -722,8 +734,9 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
       pd.b_scale = h->o_scale;
       pd.b_scale_ld = h->l;
     }
+    pd.tma_out = h->fp8 ? 0 : 1;
     e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s,
-                       h->tm_h32.bytes);
+                       h->tm_h32.bytes, h->tm_out_o.bytes);
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 6, s);
@@ -741,8 +754,12 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     q.out = static_cast<__nv_bfloat16 *>(y);
     q.ld_out = h->d;
     q.status = w.status;
+    // y through TMA stores when its address allows a tensor map (16-byte aligned)
+    TensorMap64 tm_y;
+    q.tma_out = make_tmap_bf16_out(tm_y.bytes, y, T, h->d, h->d) == 0 ? 1 : 0;
     const int tiles = (T + kTileM - 1) / kTileM * q.n_tiles_n;
-    e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, q, h->num_sms, tiles, s);
+    e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, q, h->num_sms, tiles, s, nullptr,
+                       tm_y.bytes);
     h->launches += 1;
   } else {
     float *zpf = static_cast<float *>(w.zp);

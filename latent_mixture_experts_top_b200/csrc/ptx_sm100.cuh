@@ -1,6 +1,6 @@
 // ptx_sm100.cuh -- inline-PTX wrappers for the sm_100a data path:
-// mbarriers, TMA tiled loads (no multicast), and the tcgen05 tensor-core
-// instructions (TMEM alloc, MMA kind::f16, commit, TMEM loads, fences).
+// mbarriers, TMA tiled loads (no multicast) and stores, and the tcgen05
+// tensor-core instructions (TMEM alloc, MMA kind::f16, commit, TMEM loads, fences).
 //
 // Shared-memory operand descriptors follow the sm_100 UMMA descriptor format:
 // start address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30),
@@ -76,6 +76,34 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// 2-D tiled store of a shared-memory box to global memory, tracked as one
+// bulk async-group of the issuing thread.  Rows and columns past the tensor's
+// extent are not written.
+__device__ __forceinline__ void tma_store_2d(const void *tmap, const void *smem_src, int32_t x,
+                                             int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Until all of this thread's bulk groups have completed (writes performed).
+__device__ __forceinline__ void bulk_wait_group_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA, tensor core) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

@@ -86,10 +86,19 @@ struct __align__(8) SmemCtl {
   uint32_t tmem_base;
   int abort;
 };
+// TMA-store epilogue (forward bf16 outputs): each epilogue warp owns two
+// staging buffers of one 32 x 32 bf16 block; they follow the control block.
+constexpr int OUT_BOX = 32;
+constexpr int OUT_BOX_BYTES = OUT_BOX * OUT_BOX * 2;                // 2 KB
+constexpr int CTL_BYTES = 1024;                                     // SmemCtl, padded
+constexpr int STAGING_BYTES = NUM_EPI_WARPS * 2 * OUT_BOX_BYTES;    // 32 KB
+static_assert(sizeof(SmemCtl) <= CTL_BYTES, "control block");
 template <bool kFp8>
-constexpr size_t smem_bytes() {
-  return 1024 /*align slack*/ + Cfg<kFp8>::RING_BYTES + sizeof(SmemCtl);
+constexpr size_t smem_bytes(bool staging) {
+  return 1024 /*align slack*/ + Cfg<kFp8>::RING_BYTES +
+         (staging ? CTL_BYTES + STAGING_BYTES : sizeof(SmemCtl));
 }
+static_assert(smem_bytes<false>(true) <= 232448, "shared memory per CTA");
 
 struct Tile {
   int a_row, b_row, n_tile, row_hi;
@@ -172,10 +181,53 @@ __device__ __forceinline__ void store_f32x32(float *dst, const float *v) {
   for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
+// Per-warp state of the TMA-store epilogue.  map == null: the warp stores
+// its rows directly (one 16-byte store per lane and 8 columns).
+struct OutSink {
+  const CUtensorMap *map;
+  uint8_t *buf;  // the warp's two staging buffers
+  int x0;        // output column of the epilogue's column 0
+  int y;         // output row of lane 0
+  int issued;    // blocks stored so far (selects the buffer)
+};
+
+// Row `lane` of the warp's 32-row block, columns x .. x+31: the 32 values go,
+// as bf16, into a staging buffer in the 64-byte-swizzled layout of the output
+// map (16-byte chunk j of row r at chunk position j ^ ((r >> 1) & 3), which
+// also keeps each 8-lane phase of the writes on distinct banks), and lane 0
+// stores the block with one TMA store.  A buffer is refilled only once the
+// store issued two blocks earlier has finished reading it.  All 32 lanes call
+// this together.
+__device__ __forceinline__ void sink_store(OutSink &o, const float *v, int x) {
+  const int lane = threadIdx.x & 31;
+  uint8_t *b = o.buf + (o.issued & 1) * OUT_BOX_BYTES;
+  if (o.issued >= 2) {
+    if (lane == 0) ptx::bulk_wait_group_read<1>();
+    __syncwarp();
+  }
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+    w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+    w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+    w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+    *reinterpret_cast<uint4 *>(b + lane * 64 + ((j ^ sw) << 4)) = w;
+  }
+  ptx::fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    ptx::tma_store_2d(o.map, b, o.x0 + x, o.y);
+    ptx::bulk_commit_group();
+  }
+  ++o.issued;
+}
+
 // 256 accumulator columns -> bf16 (or f32) row segment, chunks past n_cols skipped.
 template <bool F32OUT, typename OutT>
 __device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_dst, int col0,
-                                          int n_cols, int half) {
+                                          int n_cols, int half, OutSink *sink = nullptr) {
 #pragma unroll 1
   for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
     uint32_t r[32];
@@ -185,6 +237,12 @@ __device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
     const int col = col0 + c * 32;
+    if constexpr (!F32OUT) {
+      if (sink && sink->map) {
+        if (col < n_cols) sink_store(*sink, v, col);
+        continue;
+      }
+    }
     if (valid && col < n_cols) {
       if constexpr (F32OUT) store_f32x32(reinterpret_cast<float *>(row_dst) + col, v);
       else store_bf16x32(reinterpret_cast<__nv_bfloat16 *>(row_dst) + col, v);
@@ -194,7 +252,8 @@ __device__ __forceinline__ void epi_plain(uint32_t taddr, bool valid, OutT *row_
 
 // Squared-ReLU hidden: relu(acc)^2 -> bf16 columns col0 + ..., masked at n_cols.
 __device__ __forceinline__ void epi_relu2(uint32_t taddr, bool valid, __nv_bfloat16 *row_dst,
-                                          int col0, int n_cols, int half) {
+                                          int col0, int n_cols, int half,
+                                          OutSink *sink = nullptr) {
 #pragma unroll 1
   for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
     uint32_t r[32];
@@ -207,7 +266,11 @@ __device__ __forceinline__ void epi_relu2(uint32_t taddr, bool valid, __nv_bfloa
       h[j] = a * a;
     }
     const int col = col0 + c * 32;
-    if (valid && col < n_cols) store_bf16x32(row_dst + col, h);
+    if (sink && sink->map) {
+      if (col < n_cols) sink_store(*sink, h, col);
+    } else if (valid && col < n_cols) {
+      store_bf16x32(row_dst + col, h);
+    }
   }
 }
 
@@ -289,7 +352,7 @@ __device__ __forceinline__ void epi_wgrad(uint32_t taddr, bool valid, const TcPa
 // Columns [0,128) are gate rows g0..g0+127, [128,256) the matching up rows:
 // h = silu(gate) * up for 128 hidden columns starting at hcol0.
 __device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bfloat16 *row_dst,
-                                           int hcol0, int half) {
+                                           int hcol0, int half, OutSink *sink = nullptr) {
 #pragma unroll 1
   for (int c = half * (TN / 128); c < (half + 1) * (TN / 128); ++c) {
     uint32_t g[32], u[32];
@@ -299,7 +362,8 @@ __device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bflo
     float h[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) h[j] = silu_bf16out(__uint_as_float(g[j])) * __uint_as_float(u[j]);
-    if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
+    if (sink && sink->map) sink_store(*sink, h, hcol0 + c * 32);
+    else if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
   }
 }
 
@@ -513,7 +577,8 @@ __device__ __forceinline__ void convert_stage(const uint8_t *b8, uint8_t *b16, i
 template <bool kBwd, bool kFp8>
 __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmA32, const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmA32, const __grid_constant__ CUtensorMap tmO,
+                   const TcParams p) {
   constexpr int STAGES = Cfg<kFp8>::STAGES;
   constexpr int S2 = Cfg<kFp8>::S2;
   constexpr int S2M = S2 > 0 ? S2 : 1;  // ring-2 index arithmetic (kFp8 only)
@@ -521,11 +586,15 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // [A ring][B ring (E4M3 if kFp8)][kFp8: converted-B ring]
+  // [A ring][B ring (E4M3 if kFp8)][kFp8: converted-B ring][control block]
+  // [tma_out: the epilogue warps' staging buffers]
   uint8_t *smA = smem;
   uint8_t *smB = smem + STAGES * A_BYTES;
   uint8_t *smBc = smB + STAGES * B_LOAD;
   SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + Cfg<kFp8>::RING_BYTES);
+  uint8_t *staging = smem + Cfg<kFp8>::RING_BYTES + CTL_BYTES;
+  // TMA stores: the forward instantiation with a bf16-output mode
+  const bool use_tma_out = !kBwd && !kFp8 && p.tma_out != 0;
   volatile int *abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -686,6 +755,12 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
     constexpr int kHalfStep = Cfg<kFp8>::EPI_WARPS / 4;
     const int half0 = (warp - 2) >> 2;
     const int row_in_tile = q * 32 + lane;
+    OutSink sink;
+    sink.map = nullptr;
+    sink.buf = staging + (warp - 2) * 2 * OUT_BOX_BYTES;
+    sink.x0 = 0;
+    sink.y = 0;
+    sink.issued = 0;
     int tl_count = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl_count) {
       const int acc = tl_count & 1;
@@ -705,6 +780,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
       const bool valid = row < tl.row_hi;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
       const int col0 = tl.n_tile * TN;
+      // TMA stores only for a warp whose 32 rows are all valid: a grouped
+      // tile's rows past its expert's end belong to the next tile.
+      sink.y = tl.a_row + q * 32;
+      sink.map = (use_tma_out && sink.y + 31 < tl.row_hi) ? &tmO : nullptr;
       for (int half = half0; half < 2; half += kHalfStep) {
       switch (p.mode) {
         case TC_X_FUSED:
@@ -713,7 +792,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
                             p.n_routed, half);
           } else if (col0 < p.z_end) {
             epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
-                             col0 - p.r_end, p.l, half);
+                             col0 - p.r_end, p.l, half, &sink);
           } else if (kBwd && p.raw) {  // pre-activations and the hidden
             if (p.relu2)
               epi_relu2_raw(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2,
@@ -747,9 +826,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
                            p.out_h + static_cast<size_t>(row) * p.ld_h + col0 / 2, half);
           else if (p.relu2)
             epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0, p.n_cols2,
-                      half);
+                      half, &sink);
           else
-            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half);
+            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half,
+                       &sink);
           break;
         case TC_WGRAD:
           if constexpr (kBwd) epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
@@ -767,7 +847,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
                             p.ld_out, half);
           else
             epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
-                             p.ld_out, half);
+                             p.ld_out, half, &sink);
           break;
       }
       }  // halves
@@ -775,6 +855,8 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
     }
+    // the staging buffers stay allocated until this warp's stores are done
+    if (use_tma_out && lane == 0) ptx::bulk_wait_group_all();
   }
 
   ptx::tc_fence_before();
@@ -839,6 +921,23 @@ int make_tmap_bf16(void *tmap_out, const void *base, int64_t rows, int64_t cols,
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
+int make_tmap_bf16_out(void *tmap_out, const void *base, int64_t rows, int64_t cols,
+                       int64_t row_stride_elems) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0 || cols <= 0) return -1;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_stride_elems * 2) % 16) return -1;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_elems * 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(OUT_BOX), static_cast<cuuint32_t>(OUT_BOX)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(reinterpret_cast<CUtensorMap *>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+         const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
 int make_tmap_u8(void *tmap_out, const void *base, int64_t rows, int64_t cols,
                  int64_t row_stride_bytes, int box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -857,22 +956,23 @@ int make_tmap_u8(void *tmap_out, const void *base, int64_t rows, int64_t cols,
 }
 
 cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p, int num_sms,
-                           int max_ctas, cudaStream_t s, const void *tmapA32) {
+                           int max_ctas, cudaStream_t s, const void *tmapA32,
+                           const void *tmapOut) {
   static int attr_done = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_done != dev) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<false, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes<false>()));
+                                         static_cast<int>(smem_bytes<false>(true)));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(tc_gemm_kernel<true, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes<false>()));
+                               static_cast<int>(smem_bytes<false>(false)));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(tc_gemm_kernel<false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes<true>()));
+                               static_cast<int>(smem_bytes<true>(false)));
     if (e != cudaSuccess) return e;
     attr_done = dev;
   }
@@ -880,23 +980,25 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   const bool fp8 = p.b_scale != nullptr;
   if (fp8 && (bwd || (p.mode != TC_EXPERT_GU && p.mode != TC_EXPERT_DOWN)))
     return cudaErrorInvalidValue;
+  if (p.tma_out && (bwd || fp8 || p.mode == TC_WGRAD || !tmapOut)) return cudaErrorInvalidValue;
   if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
   if (fp8 && !tmapA32) return cudaErrorInvalidValue;
-  CUtensorMap a, b, a32;
+  CUtensorMap a, b, a32, o;
   memcpy(&a, tmapA, sizeof(a));
   memcpy(&b, tmapB, sizeof(b));
   memcpy(&a32, fp8 ? tmapA32 : tmapA, sizeof(a32));
+  memcpy(&o, p.tma_out ? tmapOut : tmapA, sizeof(o));
   if (fp8)
     tc_gemm_kernel<false, true>
-        <<<grid, Cfg<true>::NUM_THREADS, smem_bytes<true>(), s>>>(a, b, a32, p);
+        <<<grid, Cfg<true>::NUM_THREADS, smem_bytes<true>(false), s>>>(a, b, a32, o, p);
   else if (bwd)
     tc_gemm_kernel<true, false>
-        <<<grid, Cfg<false>::NUM_THREADS, smem_bytes<false>(), s>>>(a, b, a32, p);
+        <<<grid, Cfg<false>::NUM_THREADS, smem_bytes<false>(false), s>>>(a, b, a32, o, p);
   else
-    tc_gemm_kernel<false, false>
-        <<<grid, Cfg<false>::NUM_THREADS, smem_bytes<false>(), s>>>(a, b, a32, p);
+    tc_gemm_kernel<false, false><<<grid, Cfg<false>::NUM_THREADS,
+                                   smem_bytes<false>(p.tma_out != 0), s>>>(a, b, a32, o, p);
   return cudaGetLastError();
 }
 

@@ -33,11 +33,14 @@ inline size_t dispatch_count_elems(int T, int chunk, int N) {
 // count matrix chunk_counts holds dispatch_count_elems(T, chunk, N) ints
 // (chunk: a multiple of 32, at most 256).  Writes offsets [N+1], perm / pos /
 // row_expert [T*K], and the M-tile table (tile_m rows per tile; capacity
-// max_tiles entries) plus its length in *n_tiles.
+// max_tiles entries) plus its length in *n_tiles; with tiles2, also a second
+// table of tile_m2-row M-tiles (capacity max_tiles2) and its length.
 cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,
                             int chunk, bool counts_ready, int32_t *offsets, int32_t *perm,
                             int32_t *pos, int32_t *row_expert, TileEntry *tiles,
-                            int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s);
+                            int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s,
+                            TileEntry *tiles2 = nullptr, int32_t *n_tiles2 = nullptr,
+                            int tile_m2 = 0, int max_tiles2 = 0);
 
 // dst[p][:] = src[perm[p] / K][:], rows of `row_bytes` (multiple of 16).
 cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
@@ -246,5 +249,15 @@ cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream
 cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p,
                            int num_sms, int max_ctas, cudaStream_t s,
                            const void *tmapA32 = nullptr, const void *tmapOut = nullptr);
+
+// The forward's bf16 GEMMs (TC_X_FUSED, TC_EXPERT_GU, TC_EXPERT_DOWN, TC_OUT;
+// bf16 weights, no backward options) on CTA pairs: 256 x 256 output tiles,
+// tcgen05.mma.cta_group::2.  tmapA: A with a {64, 128} box (as for
+// launch_tc_gemm); tmapB2: the K-block-tiled B with a {64, 128} box (each CTA
+// loads half of a 256-row block); grouped modes read 256-row M-tiles
+// (p.tiles / p.n_mtiles from launch_dispatch's second table).  At most
+// max_pairs clusters of two CTAs are launched.
+cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcParams &p,
+                                int max_pairs, cudaStream_t s, const void *tmapOut = nullptr);
 
 }  // namespace lmoe

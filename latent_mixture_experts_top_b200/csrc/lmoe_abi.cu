@@ -36,8 +36,10 @@ struct Workspace {
   int32_t *chunk_counts = nullptr;
   int32_t *offsets = nullptr;
   int32_t *perm = nullptr, *pos = nullptr, *row_expert = nullptr;
-  TileEntry *tiles = nullptr;
+  TileEntry *tiles = nullptr;     // 128-row M-tiles (single-CTA GEMMs)
   int32_t *n_tiles = nullptr;
+  TileEntry *tiles2 = nullptr;    // 256-row M-tiles (CTA-pair GEMMs)
+  int32_t *n_tiles2 = nullptr;
   void *z = nullptr, *zp = nullptr, *H = nullptr, *O = nullptr, *ucat = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
   int32_t *status = nullptr;
@@ -78,7 +80,7 @@ struct lmoe_layer {
   size_t esize = 4;
   int device = 0, num_sms = 0;
   bool loaded = false;
-  int max_tiles = 0;
+  int max_tiles = 0, max_tiles2 = 0;
   // bf16 layout of the stacked x-matrix: [W_r | pad][W_down | pad][shared rows | pad]
   int n_pad = 0, l_pad = 0, sh_rows = 0, nx_rows = 0;
   int gu_rows = 0;    // B rows per expert of the expert up GEMM: 2m (SwiGLU) or m
@@ -107,6 +109,8 @@ struct lmoe_layer {
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
   TensorMap64 tm_out_z, tm_out_h, tm_out_o;  // epilogue TMA stores: z, H, O
+  // B operands of the CTA-pair GEMMs: the same tiled matrices, {64, 128} boxes
+  TensorMap64 tm_wx2, tm_wo2, tm_wy2;
   TensorMap64 tm_zp32, tm_h32;  // E4M3 weights: {64, 32} boxes for small tiles
   // E4M3 expert weights (tiled like w_gu / w_out) and their row scales
   uint8_t *w_gu8 = nullptr, *w_o8 = nullptr;
@@ -148,7 +152,7 @@ void free_all(lmoe_layer *h) {
   void *ptrs[] = {h->w_router, h->b_router, h->w_x, h->w_down, h->w_gu, h->w_gate, h->w_upx,
                   h->w_out, h->s_gate, h->s_up, h->w_y, h->ws.logits, h->ws.ids, h->ws.gates,
                   h->ws.chunk_counts, h->ws.offsets, h->ws.perm, h->ws.pos, h->ws.row_expert,
-                  h->ws.tiles, h->ws.n_tiles, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
+                  h->ws.tiles, h->ws.n_tiles, h->ws.tiles2, h->ws.n_tiles2, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
                   h->ws.x_stage, h->ws.y_stage, h->ws.status, h->bw.a, h->bw.b, h->bw.dU,
                   h->bw.ds, h->bw.DO, h->bw.dH, h->bw.dA, h->bw.dB, h->bw.dZp, h->bw.dz,
                   h->bw.as, h->bw.bs, h->bw.das, h->bw.dbs, h->bw.dsfull, h->bw.AB,
@@ -260,6 +264,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   const size_t T = h->Tmax, TK = static_cast<size_t>(h->Tmax) * h->K, es = h->esize;
   const size_t N = h->N, d = h->d, l = h->l, m = h->m;
   h->max_tiles = static_cast<int>(TK / kTileM + N + 1);
+  h->max_tiles2 = static_cast<int>(TK / (2 * kTileM) + N + 1);
   h->n_pad = (h->N + kTileN - 1) / kTileN * kTileN;
   h->l_pad = (h->l + kTileN - 1) / kTileN * kTileN;
   h->sh_rows = h->relu2 ? (h->ns * h->ms + kTileN - 1) / kTileN * kTileN : 2 * h->ns * h->ms;
@@ -271,7 +276,9 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
             dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TK * 4) && dalloc(&w.pos, TK * 4) &&
             dalloc(&w.row_expert, TK * 4) &&
             dalloc(&w.tiles, static_cast<size_t>(h->max_tiles) * sizeof(TileEntry)) &&
-            dalloc(&w.n_tiles, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
+            dalloc(&w.n_tiles, 16) &&
+            dalloc(&w.tiles2, static_cast<size_t>(h->max_tiles2) * sizeof(TileEntry)) &&
+            dalloc(&w.n_tiles2, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
             dalloc(&w.H, TK * m * es) && dalloc(&w.O, TK * l * es) &&
             dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
             dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16);
@@ -333,6 +340,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     return LMOE_ERR_OUT_OF_MEMORY;
   }
   if (cudaMemset(w.status, 0, 16) != cudaSuccess || cudaMemset(w.n_tiles, 0, 16) != cudaSuccess ||
+      cudaMemset(w.n_tiles2, 0, 16) != cudaSuccess ||
       cudaMemset(w.ucat, 0, T * h->ky * es) != cudaSuccess) {
     free_all(h);
     delete h;
@@ -350,6 +358,8 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     // B operands: [tiled rows][64], one {64, 256} box per K-block tile
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wx, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN);
+    if (rc == LMOE_OK)
+      rc = make_map(&h->tm_wx2, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN / 2);
     if (rc == LMOE_OK && h->fp8) {
       rc = make_map(&h->tm_zp32, w.zp, static_cast<int64_t>(TK), h->l, h->l, 32);
       if (rc == LMOE_OK) rc = make_map(&h->tm_h32, w.H, static_cast<int64_t>(TK), h->m, h->m, 32);
@@ -364,9 +374,13 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
         rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->N, h->gu_rows, h->l), 64, 64, kTileN);
       if (rc == LMOE_OK)
         rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN);
+      if (rc == LMOE_OK)
+        rc = make_map(&h->tm_wo2, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN / 2);
     }
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wy, h->w_y, btile_rows(1, h->d, h->ky), 64, 64, kTileN);
+    if (rc == LMOE_OK)
+      rc = make_map(&h->tm_wy2, h->w_y, btile_rows(1, h->d, h->ky), 64, 64, kTileN / 2);
     if (rc == LMOE_OK && h->training) {
       BwdWorkspace &b = h->bw;
       const int64_t Kp = b.Kp, Tp = b.Tp;
@@ -596,8 +610,9 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.status = w.status;
     p.tma_out = 1;  // z through TMA stores (the logits are stored directly)
     const int m_tiles = (T + kTileM - 1) / kTileM;
-    e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, m_tiles * p.n_tiles_n, s,
-                       nullptr, h->tm_out_z.bytes);
+    const int m_tiles2 = (T + 2 * kTileM - 1) / (2 * kTileM);
+    e = launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, p, m_tiles2 * p.n_tiles_n, s,
+                            h->tm_out_z.bytes);
     h->launches += 1;
     const int shared_tiles_n = (h->nx_rows - h->n_pad - h->l_pad) / kTileN;
     if (e == cudaSuccess && full && shared_tiles_n > 0) {
@@ -617,8 +632,10 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       e = cudaEventRecord(h->ev_fork, s);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
       if (e == cudaSuccess)
-        e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, q, h->num_sms, m_tiles * shared_tiles_n,
-                           h->side);
+        e = shared_raw ? launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, q, h->num_sms,
+                                        m_tiles * shared_tiles_n, h->side)
+                       : launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, q,
+                                             m_tiles2 * shared_tiles_n, h->side);
       if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
       h->launches += 1;
     }
@@ -653,7 +670,8 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
   if (e != cudaSuccess) return e;
   if (full) mark(h, 2, s);
   e = launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, kDispatchChunk, true, w.offsets,
-                      w.perm, w.pos, w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s);
+                      w.perm, w.pos, w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s,
+                      w.tiles2, w.n_tiles2, 2 * kTileM, h->max_tiles2);
   h->launches += 2;
   if (e != cudaSuccess) return e;
   if (full) mark(h, 3, s);
@@ -714,6 +732,9 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     p.out = static_cast<__nv_bfloat16 *>(w.H);
     p.ld_out = h->m;
     p.status = w.status;
+    // Single-CTA tiles of 128 rows: measured at least as fast as CTA pairs for
+    // the gate/up GEMM (K = l is short, the SwiGLU epilogue is the heavier)
+    // and much faster when experts hold few tokens.
     p.tma_out = h->fp8 ? 0 : 1;
     e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s,
                        h->tm_zp32.bytes, h->tm_out_h.bytes);
@@ -734,9 +755,20 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
       pd.b_scale = h->o_scale;
       pd.b_scale_ld = h->l;
     }
+    // CTA pairs (256-row M-tiles) when experts average at least 256 rows: the
+    // long reduction (K = m) then gains from the smaller per-SM operand feed;
+    // with fewer rows the pair's half-empty tiles cost more than that.
+    const bool pair_down = !h->fp8 && static_cast<int64_t>(T) * h->K >= 256LL * h->N;
     pd.tma_out = h->fp8 ? 0 : 1;
-    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s,
-                       h->tm_h32.bytes, h->tm_out_o.bytes);
+    if (pair_down) {
+      pd.tiles = w.tiles2;
+      pd.n_mtiles = w.n_tiles2;
+      e = launch_tc_gemm_pair(h->tm_h.bytes, h->tm_wo2.bytes, pd, h->num_sms, s,
+                              h->tm_out_o.bytes);
+    } else {
+      e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s,
+                         h->tm_h32.bytes, h->tm_out_o.bytes);
+    }
     h->launches += 1;
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     mark(h, 6, s);
@@ -757,9 +789,8 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     // y through TMA stores when its address allows a tensor map (16-byte aligned)
     TensorMap64 tm_y;
     q.tma_out = make_tmap_bf16_out(tm_y.bytes, y, T, h->d, h->d) == 0 ? 1 : 0;
-    const int tiles = (T + kTileM - 1) / kTileM * q.n_tiles_n;
-    e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, q, h->num_sms, tiles, s, nullptr,
-                       tm_y.bytes);
+    const int tiles2 = (T + 2 * kTileM - 1) / (2 * kTileM) * q.n_tiles_n;
+    e = launch_tc_gemm_pair(h->tm_ucat.bytes, h->tm_wy2.bytes, q, tiles2, s, tm_y.bytes);
     h->launches += 1;
   } else {
     float *zpf = static_cast<float *>(w.zp);

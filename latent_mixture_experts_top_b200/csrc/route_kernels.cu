@@ -139,7 +139,8 @@ __device__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
 // small enough to run beside a GEMM CTA on the same SM): each thread scans the
 // chunk counts of its experts (in place: counts[e][c] becomes the number of
 // pairs of expert e in chunks before c); the expert totals are then scanned
-// into offsets and the table of tile_m-row M-tiles is written.
+// into offsets and the table of tile_m-row M-tiles is written, and, when
+// tiles2 is given, a second table of tile_m2-row M-tiles (the CTA-pair GEMM's).
 constexpr int kScanThreads = 256, kScanPerThread = 4;  // N <= 1024
 
 __device__ int scan_expert_row(int32_t *counts, int e, int n_chunks) {
@@ -168,47 +169,63 @@ __device__ int scan_expert_row(int32_t *counts, int e, int n_chunks) {
   return tot;
 }
 
+// Writes the table entries of expert e's M-tiles (tile_m rows each, the last
+// one ragged) from index tstart on.
+__device__ void write_tiles(TileEntry *tiles, int tstart, int max_tiles, int e, int off, int tot,
+                            int tile_m) {
+  const int mt = (tot + tile_m - 1) / tile_m;
+  for (int j = 0; j < mt; ++j) {
+    const int idx = tstart + j;
+    if (idx < max_tiles) {
+      TileEntry te;
+      te.row0 = off + j * tile_m;
+      te.row_end = off + tot;
+      te.expert = e;
+      te.pad = 0;
+      tiles[idx] = te;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
     int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
-    TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles) {
+    TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+    TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2, int tile_m2,
+    int max_tiles2) {
   __shared__ int warp_sums[32];
   const int e0 = threadIdx.x * kScanPerThread;  // experts e0 .. e0+3
-  int tot[kScanPerThread], mt[kScanPerThread];
-  int my_tot = 0, my_mt = 0;
+  int tot[kScanPerThread], mt[kScanPerThread], mt2[kScanPerThread];
+  int my_tot = 0, my_mt = 0, my_mt2 = 0;
 #pragma unroll
   for (int i = 0; i < kScanPerThread; ++i) {
     const int e = e0 + i;
     tot[i] = e < N ? scan_expert_row(counts, e, n_chunks) : 0;
     mt[i] = (tot[i] + tile_m - 1) / tile_m;
+    mt2[i] = tiles2 ? (tot[i] + tile_m2 - 1) / tile_m2 : 0;
     my_tot += tot[i];
     my_mt += mt[i];
+    my_mt2 += mt2[i];
   }
-  int all = 0, all_tiles = 0;
+  int all = 0, all_tiles = 0, all_tiles2 = 0;
   int off = block_exclusive_scan(my_tot, warp_sums, &all);
   int tstart = block_exclusive_scan(my_mt, warp_sums, &all_tiles);
+  int tstart2 = block_exclusive_scan(my_mt2, warp_sums, &all_tiles2);
 #pragma unroll
   for (int i = 0; i < kScanPerThread; ++i) {
     const int e = e0 + i;
     if (e < N) {
       offsets[e] = off;
-      for (int j = 0; j < mt[i]; ++j) {
-        const int idx = tstart + j;
-        if (idx < max_tiles) {
-          TileEntry te;
-          te.row0 = off + j * tile_m;
-          te.row_end = off + tot[i];
-          te.expert = e;
-          te.pad = 0;
-          tiles[idx] = te;
-        }
-      }
+      write_tiles(tiles, tstart, max_tiles, e, off, tot[i], tile_m);
+      if (tiles2) write_tiles(tiles2, tstart2, max_tiles2, e, off, tot[i], tile_m2);
     }
     off += tot[i];
     tstart += mt[i];
+    tstart2 += mt2[i];
   }
   if (threadIdx.x == 0) {
     offsets[N] = all;
     *n_tiles = min(all_tiles, max_tiles);
+    if (tiles2) *n_tiles2 = min(all_tiles2, max_tiles2);
   }
 }
 
@@ -410,7 +427,8 @@ cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, i
 cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,
                             int chunk, bool counts_ready, int32_t *offsets, int32_t *perm,
                             int32_t *pos, int32_t *row_expert, TileEntry *tiles,
-                            int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s) {
+                            int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s,
+                            TileEntry *tiles2, int32_t *n_tiles2, int tile_m2, int max_tiles2) {
   if (N > 1024 || chunk % 32 || chunk < 32 || chunk > 256) return cudaErrorInvalidValue;
   const int nc = dispatch_chunks(T, chunk);
   if (nc > 0 && !counts_ready) {
@@ -419,8 +437,10 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  if (tiles2 && (!n_tiles2 || tile_m2 <= 0)) return cudaErrorInvalidValue;
   dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_counts, nc, N, offsets, tiles, n_tiles,
-                                                   tile_m, max_tiles);
+                                                   tile_m, max_tiles, tiles2, n_tiles2, tile_m2,
+                                                   max_tiles2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || nc == 0) return e;
   const int warps = chunk / 32;

@@ -569,6 +569,84 @@ __device__ __forceinline__ void convert_stage(const uint8_t *b8, uint8_t *b16, i
   }
 }
 
+// One tile's epilogue for the calling warp: its 32 accumulator lanes (output
+// rows row = lane's row, valid when inside the tile) and its column halves,
+// by mode.  Shared by the single-CTA and the CTA-pair kernels.
+template <bool kBwd, bool kFp8>
+__device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl, uint32_t taddr,
+                                              int row, bool valid, int col0, int half0,
+                                              OutSink &sink) {
+  // one epilogue warp per lane quarter covers both halves, two take one each
+  constexpr int kHalfStep = Cfg<kFp8>::EPI_WARPS / 4;
+  for (int half = half0; half < 2; half += kHalfStep) {
+    switch (p.mode) {
+      case TC_X_FUSED:
+        if (col0 < p.r_end) {
+          epi_plain<true>(taddr, valid, p.logits + static_cast<size_t>(row) * p.ld_logits, col0,
+                          p.n_routed, half);
+        } else if (col0 < p.z_end) {
+          epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
+                           col0 - p.r_end, p.l, half, &sink);
+        } else if (kBwd && p.raw) {  // pre-activations and the hidden
+          if (p.relu2)
+            epi_relu2_raw(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2,
+                          p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
+                          col0 - p.z_end, p.n_cols2, half);
+          else
+            epi_swiglu_raw(taddr, valid,
+                           p.out2 + static_cast<size_t>(row) * p.ld_out2 + (col0 - p.z_end),
+                           p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0 +
+                               (col0 - p.z_end) / 2,
+                           half);
+        } else if (p.relu2) {
+          epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
+                    col0 - p.z_end, p.n_cols2, half);
+        } else {
+          epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
+                     p.out_col0 + (col0 - p.z_end) / 2, half);
+        }
+        break;
+      case TC_EXPERT_GU:
+        if constexpr (kFp8) {
+          const float *scl = p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0;
+          __nv_bfloat16 *hrow = p.out + static_cast<size_t>(row) * p.ld_out;
+          if (p.relu2) epi_relu2_scaled(taddr, valid, hrow, col0, p.n_cols2, scl, half);
+          else epi_swiglu_scaled(taddr, valid, hrow, col0 / 2, scl, half);
+        } else if (kBwd && p.raw && p.relu2)
+          epi_relu2_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
+                        p.out_h + static_cast<size_t>(row) * p.ld_h, col0, p.n_cols2, half);
+        else if (kBwd && p.raw)
+          epi_swiglu_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + col0,
+                         p.out_h + static_cast<size_t>(row) * p.ld_h + col0 / 2, half);
+        else if (p.relu2)
+          epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0, p.n_cols2,
+                    half, &sink);
+        else
+          epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half,
+                     &sink);
+        break;
+      case TC_WGRAD:
+        if constexpr (kBwd) epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
+        break;
+      default:  // TC_EXPERT_DOWN, TC_OUT
+        if constexpr (kFp8) {
+          epi_plain_scaled(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
+                           p.ld_out,
+                           p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0,
+                           half);
+        } else if (kBwd && p.act_dab)
+          epi_act_backward(taddr, valid, p, row, col0, p.ld_out, half);
+        else if (kBwd && p.out_f32)
+          epi_plain<true>(taddr, valid, p.out_f32 + static_cast<size_t>(row) * p.ld_out, col0,
+                          p.ld_out, half);
+        else
+          epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
+                           p.ld_out, half, &sink);
+        break;
+    }
+  }  // halves
+}
+
 // kBwd: the instantiation with the backward's epilogues and the TC_WGRAD
 // mode; the forward launches the other one, whose smaller register budget
 // leaves room for the routing kernels that run beside it.
@@ -752,7 +830,6 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     // which half of the tile's columns (both, one after the other, when the
     // variant has one epilogue warp per lane quarter)
-    constexpr int kHalfStep = Cfg<kFp8>::EPI_WARPS / 4;
     const int half0 = (warp - 2) >> 2;
     const int row_in_tile = q * 32 + lane;
     OutSink sink;
@@ -784,73 +861,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
       // tile's rows past its expert's end belong to the next tile.
       sink.y = tl.a_row + q * 32;
       sink.map = (use_tma_out && sink.y + 31 < tl.row_hi) ? &tmO : nullptr;
-      for (int half = half0; half < 2; half += kHalfStep) {
-      switch (p.mode) {
-        case TC_X_FUSED:
-          if (col0 < p.r_end) {
-            epi_plain<true>(taddr, valid, p.logits + static_cast<size_t>(row) * p.ld_logits, col0,
-                            p.n_routed, half);
-          } else if (col0 < p.z_end) {
-            epi_plain<false>(taddr, valid, p.z + static_cast<size_t>(row) * p.ld_z,
-                             col0 - p.r_end, p.l, half, &sink);
-          } else if (kBwd && p.raw) {  // pre-activations and the hidden
-            if (p.relu2)
-              epi_relu2_raw(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2,
-                            p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
-                            col0 - p.z_end, p.n_cols2, half);
-            else
-              epi_swiglu_raw(taddr, valid,
-                             p.out2 + static_cast<size_t>(row) * p.ld_out2 + (col0 - p.z_end),
-                             p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0 +
-                                 (col0 - p.z_end) / 2,
-                             half);
-          } else if (p.relu2) {
-            epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
-                      col0 - p.z_end, p.n_cols2, half);
-          } else {
-            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
-                       p.out_col0 + (col0 - p.z_end) / 2, half);
-          }
-          break;
-        case TC_EXPERT_GU:
-          if constexpr (kFp8) {
-            const float *scl = p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0;
-            __nv_bfloat16 *hrow = p.out + static_cast<size_t>(row) * p.ld_out;
-            if (p.relu2) epi_relu2_scaled(taddr, valid, hrow, col0, p.n_cols2, scl, half);
-            else epi_swiglu_scaled(taddr, valid, hrow, col0 / 2, scl, half);
-          } else if (kBwd && p.raw && p.relu2)
-            epi_relu2_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
-                          p.out_h + static_cast<size_t>(row) * p.ld_h, col0, p.n_cols2, half);
-          else if (kBwd && p.raw)
-            epi_swiglu_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + col0,
-                           p.out_h + static_cast<size_t>(row) * p.ld_h + col0 / 2, half);
-          else if (p.relu2)
-            epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0, p.n_cols2,
-                      half, &sink);
-          else
-            epi_swiglu(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0 / 2, half,
-                       &sink);
-          break;
-        case TC_WGRAD:
-          if constexpr (kBwd) epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
-          break;
-        default:  // TC_EXPERT_DOWN, TC_OUT
-          if constexpr (kFp8) {
-            epi_plain_scaled(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
-                             p.ld_out,
-                             p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0,
-                             half);
-          } else if (kBwd && p.act_dab)
-            epi_act_backward(taddr, valid, p, row, col0, p.ld_out, half);
-          else if (kBwd && p.out_f32)
-            epi_plain<true>(taddr, valid, p.out_f32 + static_cast<size_t>(row) * p.ld_out, col0,
-                            p.ld_out, half);
-          else
-            epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
-                             p.ld_out, half, &sink);
-          break;
-      }
-      }  // halves
+      epilogue_tile<kBwd, kFp8>(p, tl, taddr, row, valid, col0, half0, sink);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
@@ -865,6 +876,271 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
     __syncwarp();
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- CTA pairs
+// The forward's bf16 GEMMs run on CTA pairs: a cluster of two CTAs on two SMs
+// computes a 256 x 256 output tile with tcgen05.mma.cta_group::2 (M = 256).
+// Each CTA stages its own 128 A rows and one half (128 rows) of the tile's
+// 256 B rows, so a K-block moves 32 KB through each SM's shared memory for
+// 128 x 256 x 64 multiply-adds, where the single-CTA tile needs 48 KB: the
+// L2-to-SM feed, not the tensor pipe, limits the 128 x 256 tile.  Each CTA's
+// TMEM holds its 128 rows of the accumulator, so the epilogue is the
+// single-CTA one.  Grouped modes take 256-row M-tiles from their own table
+// (an expert's last tile may leave rank 1 without rows: it then loads no A).
+//
+// Roles as in the single-CTA kernel, in both CTAs; rank 0 (the leader)
+// alone issues the MMAs.  Both CTAs' TMA loads complete on the leader's
+// `full` barrier; the leader's commits free both CTAs' ring stages and
+// publish both halves of an accumulator; both CTAs' epilogue warps release
+// it on the leader's `acc_empty`.  No load uses multicast.
+constexpr int P_STAGES = 6;
+constexpr int P_B_BYTES = (TN / 2) * TKB * 2;             // 16 KB: this CTA's half of B
+constexpr int P_RING_BYTES = P_STAGES * (A_BYTES + P_B_BYTES);  // 192 KB
+constexpr uint32_t P_IDESC = ptx::idesc_bf16_f32(2 * TM, TN);
+
+struct __align__(8) PairCtl {
+  uint64_t full[P_STAGES];   // leader: both CTAs' bytes of a stage landed
+  uint64_t empty[P_STAGES];  // each CTA: its ring stage may be refilled
+  uint64_t acc_full[2];      // each CTA: its half of an accumulator is ready
+  uint64_t acc_empty[2];     // leader: both CTAs' epilogue warps are done with it
+  uint64_t drain;            // leader, abort path: issued MMAs finished
+  uint64_t peer_done;        // exit handshake
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(PairCtl) <= CTL_BYTES, "pair control block");
+constexpr size_t pair_smem_bytes(bool staging) {
+  return 1024 /*align slack*/ + P_RING_BYTES + (staging ? CTL_BYTES + STAGING_BYTES : sizeof(PairCtl));
+}
+static_assert(pair_smem_bytes(true) <= 232448, "shared memory per CTA");
+
+// Pair tile t as seen by CTA `rank`: its 128 A rows (a_row, row_hi as in the
+// single-CTA tile) and its half of the B block (b_row, K-block 0);
+// *rank1_rows: whether rank 1 has any valid rows in the tile.
+__device__ __forceinline__ Tile decode_pair_tile(const TcParams &p, int t, int m_tiles2,
+                                                 uint32_t rank, bool *rank1_rows) {
+  Tile tl;
+  tl.k0 = 0;
+  tl.nkb = p.Kdim / TKB;
+  tl.group = 0;
+  tl.expert = 0;
+  tl.b_plain = false;
+  int row0, b0;
+  if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
+    const int m = t % m_tiles2, n = p.n_tile_base + t / m_tiles2;  // consecutive pairs share B
+    row0 = m * 2 * TM;
+    b0 = n * tl.nkb * TN;
+    tl.n_tile = n;
+    tl.row_hi = p.M;
+  } else {
+    const int mt = t / p.n_tiles_n, n = t % p.n_tiles_n;  // consecutive pairs share A
+    const TileEntry te = p.tiles[mt];
+    row0 = te.row0;
+    b0 = (te.expert * p.n_tiles_n + n) * tl.nkb * TN;
+    tl.n_tile = n;
+    tl.row_hi = te.row_end;
+    tl.expert = te.expert;
+  }
+  tl.a_row = row0 + static_cast<int>(rank) * TM;
+  tl.b_row = b0 + static_cast<int>(rank) * (TN / 2);
+  *rank1_rows = row0 + TM < tl.row_hi;
+  return tl;
+}
+
+__device__ __forceinline__ void record_failure_pair(const TcParams &p, PairCtl *ctl,
+                                                    uint32_t peer, int code) {
+  ctl->abort = 1;
+  ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(&ctl->abort), peer), 1u);
+  if (p.status) atomicCAS(p.status, 0, code);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<false>::NUM_THREADS, 1)
+    tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // [A ring][B-half ring][control block][tma_out: staging buffers]
+  uint8_t *smA = smem;
+  uint8_t *smB = smem + P_STAGES * A_BYTES;
+  PairCtl *ctl = reinterpret_cast<PairCtl *>(smem + P_RING_BYTES);
+  uint8_t *staging = smem + P_RING_BYTES + CTL_BYTES;
+  volatile int *abort_flag = &ctl->abort;
+  const bool use_tma_out = p.tma_out != 0;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const bool leader = rank == 0;
+  const int cid = static_cast<int>(ptx::cluster_id_x());
+  const int ncl = static_cast<int>(ptx::cluster_count_x());
+
+  const bool grouped = (p.mode == TC_EXPERT_GU || p.mode == TC_EXPERT_DOWN);
+  const int m_tiles2 = grouped ? 0 : (p.M + 2 * TM - 1) / (2 * TM);
+  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles2 * p.n_tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      ptx::mbar_init(&ctl->full[s], 1);
+      ptx::mbar_init(&ctl->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&ctl->acc_full[a], 1);
+      ptx::mbar_init(&ctl->acc_empty[a], 2 * NUM_EPI_WARPS);
+    }
+    ptx::mbar_init(&ctl->drain, 1);
+    ptx::mbar_init(&ctl->peer_done, 1);
+    ctl->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint32_t full0 = ptx::map_to_rank(ptx::smem_u32(&ctl->full[0]), 0);
+      int it = 0;
+      bool ok = true;
+      for (int t = cid; t < total && ok; t += ncl) {
+        bool rank1_rows;
+        const Tile tl = decode_pair_tile(p, t, m_tiles2, rank, &rank1_rows);
+        const bool load_a = leader || rank1_rows;
+        const uint32_t tx = 2 * P_B_BYTES + (rank1_rows ? 2 * A_BYTES : A_BYTES);
+        for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (!ptx::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag)) {
+            record_failure_pair(p, ctl, peer, DEV_TIMEOUT_PRODUCER);
+            ok = false;
+            break;
+          }
+          if (leader) ptx::mbar_arrive_expect_tx(&ctl->full[s], tx);
+          const uint32_t bar = full0 + s * 8;
+          if (load_a) ptx::tma_load_2d_pair(smA + s * A_BYTES, &tmA, bar, kb * TKB, tl.a_row);
+          ptx::tma_load_2d_pair(smB + s * P_B_BYTES, &tmB, bar, 0, tl.b_row + kb * TN);
+        }
+      }
+      if (!ok && leader) {  // let every copy of both CTAs still in flight land
+        for (int j = (it > P_STAGES ? it - P_STAGES : 0); j < it; ++j)
+          if (!drain_wait(&ctl->full[j % P_STAGES], (j / P_STAGES) & 1))
+            record_failure_pair(p, ctl, peer, DEV_TIMEOUT_DRAIN);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
+      const uint32_t empty_me = ptx::smem_u32(&ctl->empty[0]);
+      const uint32_t empty_peer = ptx::map_to_rank(empty_me, peer);
+      const uint32_t accf_me = ptx::smem_u32(&ctl->acc_full[0]);
+      const uint32_t accf_peer = ptx::map_to_rank(accf_me, peer);
+      const int nkb = p.Kdim / TKB;
+      int it = 0, tl_count = 0;
+      bool ok = true;
+      for (int t = cid; t < total && ok; t += ncl, ++tl_count) {
+        const int acc = tl_count & 1;
+        const uint32_t acc_ph = (tl_count >> 1) & 1;
+        if (!ptx::mbar_wait(&ctl->acc_empty[acc], acc_ph ^ 1, abort_flag)) {
+          record_failure_pair(p, ctl, peer, DEV_TIMEOUT_MMA);
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * TN;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (!ptx::mbar_wait(&ctl->full[s], ph, abort_flag)) {
+            record_failure_pair(p, ctl, peer, DEV_TIMEOUT_MMA);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_addr = ptx::smem_u32(smA + s * A_BYTES);
+          const uint32_t b_addr = ptx::smem_u32(smB + s * P_B_BYTES);
+#pragma unroll
+          for (int k = 0; k < TKB / 16; ++k)
+            ptx::mma_bf16_pair(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
+                               ptx::smem_desc_sw128(b_addr + k * 32), P_IDESC, (kb | k) != 0);
+          // both CTAs' stage s is free once these MMAs finish
+          ptx::mma_commit_pair(empty_me + s * 8);
+          ptx::mma_commit_pair(empty_peer + s * 8);
+        }
+        if (!ok) break;
+        ptx::mma_commit_pair(accf_me + acc * 8);  // both halves of the accumulator ready
+        ptx::mma_commit_pair(accf_peer + acc * 8);
+      }
+      if (!ok) {  // let issued MMAs finish before TMEM is freed
+        ptx::mma_commit_pair(ptx::smem_u32(&ctl->drain));
+        if (!drain_wait(&ctl->drain, 0)) record_failure_pair(p, ctl, peer, DEV_TIMEOUT_DRAIN);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int half0 = (warp - 2) >> 2;
+    const uint32_t acc_empty0 = ptx::map_to_rank(ptx::smem_u32(&ctl->acc_empty[0]), 0);
+    OutSink sink;
+    sink.map = nullptr;
+    sink.buf = staging + (warp - 2) * 2 * OUT_BOX_BYTES;
+    sink.x0 = 0;
+    sink.y = 0;
+    sink.issued = 0;
+    int tl_count = 0;
+    for (int t = cid; t < total; t += ncl, ++tl_count) {
+      const int acc = tl_count & 1;
+      const uint32_t acc_ph = (tl_count >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = ptx::mbar_wait(&ctl->acc_full[acc], acc_ph, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) {
+        if (lane == 0) record_failure_pair(p, ctl, peer, DEV_TIMEOUT_EPILOGUE);
+        break;
+      }
+      ptx::tc_fence_after();
+      bool rank1_rows;
+      const Tile tl = decode_pair_tile(p, t, m_tiles2, rank, &rank1_rows);
+      if (tl.a_row < tl.row_hi) {  // rank 1 of an expert's last tile may have no rows
+        const int row = tl.a_row + q * 32 + lane;
+        const bool valid = row < tl.row_hi;
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
+        sink.y = tl.a_row + q * 32;
+        sink.map = (use_tma_out && sink.y + 31 < tl.row_hi) ? &tmO : nullptr;
+        epilogue_tile<false, false>(p, tl, taddr, row, valid, tl.n_tile * TN, half0, sink);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(acc_empty0 + acc * 8);
+    }
+    if (use_tma_out && lane == 0) ptx::bulk_wait_group_all();
+  }
+
+  // Exit: meet the peer (the leader's MMAs write this CTA's TMEM and its
+  // loads complete on the leader's barriers; the peer's epilogue arrives on
+  // the leader's), then free TMEM.
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_u32(&ctl->peer_done), peer));
+    if (!drain_wait(&ctl->peer_done, 0) && p.status) atomicCAS(p.status, 0, DEV_TIMEOUT_DRAIN);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -999,6 +1275,42 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   else
     tc_gemm_kernel<false, false><<<grid, Cfg<false>::NUM_THREADS,
                                    smem_bytes<false>(p.tma_out != 0), s>>>(a, b, a32, o, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcParams &p,
+                                int max_pairs, cudaStream_t s, const void *tmapOut) {
+  static int attr_dev = -1, dev_pairs = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(pair_smem_bytes(true)));
+    if (e != cudaSuccess) return e;
+    // pairs resident at once (one CTA per SM; a GPC with an odd number of
+    // free SMs leaves one idle)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(Cfg<false>::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = pair_smem_bytes(true);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, tc_pair_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n <= 0) return cudaErrorInvalidConfiguration;
+    dev_pairs = n;
+    attr_dev = dev;
+  }
+  const bool bwd = p.mode == TC_WGRAD || p.raw || p.act_dab || p.out_f32 || p.out_h;
+  if (bwd || p.b_scale || (p.tma_out && !tmapOut)) return cudaErrorInvalidValue;
+  if (p.Kdim % TKB || p.Kdim <= 0 || p.n_tiles_n <= 0) return cudaErrorInvalidValue;
+  const int pairs = max_pairs < dev_pairs ? max_pairs : dev_pairs;
+  if (pairs <= 0) return cudaSuccess;
+  CUtensorMap a, b, o;
+  memcpy(&a, tmapA, sizeof(a));
+  memcpy(&b, tmapB2, sizeof(b));
+  memcpy(&o, p.tma_out ? tmapOut : tmapA, sizeof(o));
+  tc_pair_kernel<<<2 * pairs, Cfg<false>::NUM_THREADS, pair_smem_bytes(p.tma_out != 0), s>>>(a, b, o,
+                                                                                           p);
   return cudaGetLastError();
 }
 

@@ -87,6 +87,21 @@ def test_parity_prefill_biased_router():
     _check_layer(configs.PREFILL, n_sample=48)
 
 
+# A mid-size layer whose experts average 275 rows (T K / N = 1100 * 8 / 32),
+# so that the expert down GEMM runs on CTA pairs over 256-row M-tiles: with
+# the router bias the counts spread, giving full pair tiles, ragged ones and
+# tiles whose second CTA has no rows; T = 1100 also leaves the dense GEMMs a
+# ragged last pair tile.  Every token is compared.
+MID_PAIR = configs.LayerConfig("mid_pair_T1100_d512_l256_m256_N32_K8_bias", T=1100, d=512,
+                               m=256, n_experts=16, top_k=4, alpha=2, n_shared=1, m_shared=256,
+                               variant="acc", router_bias_std=0.5)
+
+
+def test_parity_pair_down_gemm_all_tokens():
+    assert MID_PAIR.T * MID_PAIR.k_active >= 256 * MID_PAIR.n_routed
+    _check_layer(MID_PAIR, n_sample=10 ** 9)
+
+
 def test_parity_relu2_tiny_f32_all_tokens():
     _check_layer(configs.TINY_RELU2_F32, n_sample=10 ** 9)
 

@@ -28,11 +28,15 @@
 //               tcgen05.commit frees ring stages / publishes accumulators.
 //   warps 2-9   epilogue: two warps per TMEM lane quarter, each taking half
 //               of the tile's columns: tcgen05.ld 32 lanes x 32 columns,
-//               fused epilogue, 16-byte global stores; overlaps the next
-//               tile's MMAs.
+//               fused epilogue, then (forward bf16 outputs) a TMA store of
+//               each 32 x 32 block staged in shared memory, or 16-byte
+//               global stores; overlaps the next tile's MMAs.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA records a
 // status, stops its roles, lets in-flight copies and MMAs land, frees TMEM and
 // returns.
+//
+// tc_pair_kernel (further down) runs the same forward modes on CTA pairs
+// (tcgen05.mma.cta_group::2, 256 x 256 tiles) with the same epilogue.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>

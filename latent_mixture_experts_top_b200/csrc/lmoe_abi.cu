@@ -616,8 +616,9 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     h->launches += 1;
     const int shared_tiles_n = (h->nx_rows - h->n_pad - h->l_pad) / kTileN;
     if (e == cudaSuccess && full && shared_tiles_n > 0) {
-      // Shared experts' gate/up (same kernel, the shared column range) on the
-      // side stream: it overlaps the routing kernels; the output GEMM joins it.
+      // Shared experts' gate/up (the shared column range of the same matrix) on
+      // the side stream: it overlaps the routing kernels; the output GEMM joins
+      // it.  The backward's raw variant runs on the single-CTA kernel.
       TcParams q = p;
       q.n_tile_base = (h->n_pad + h->l_pad) / kTileN;
       q.n_tiles_n = shared_tiles_n;

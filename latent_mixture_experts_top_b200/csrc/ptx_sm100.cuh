@@ -1,5 +1,5 @@
 // ptx_sm100.cuh -- inline-PTX wrappers for the sm_100a data path:
-// mbarriers, TMA tiled loads (no multicast) and stores, the tcgen05
+// mbarriers, TMA tiled loads (each CTA its own) and stores, the tcgen05
 // tensor-core instructions (TMEM alloc, MMA kind::f16, commit, TMEM loads,
 // fences), and their CTA-pair (cta_group::2) forms.
 //
@@ -228,7 +228,8 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 // Tiled load into this CTA's shared memory whose bytes complete on the
-// mbarrier at bar_cluster, which may be the other CTA's (no multicast).
+// mbarrier at bar_cluster, which may be the other CTA's; the data lands
+// only in this CTA.
 __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const void *tmap,
                                                  uint32_t bar_cluster, int32_t x, int32_t y) {
   asm volatile(

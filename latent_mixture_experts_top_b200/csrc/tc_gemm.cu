@@ -21,7 +21,7 @@
 //
 // Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
-//               swizzle, into a 4-stage shared-memory ring (no multicast).
+//               swizzle, into a 4-stage shared-memory ring of this CTA.
 //   warp 1      TMEM owner and MMA issuer: one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into
 //               one of two 256-column fp32 accumulators in TMEM, and
@@ -898,7 +898,8 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
 // alone issues the MMAs.  Both CTAs' TMA loads complete on the leader's
 // `full` barrier; the leader's commits free both CTAs' ring stages and
 // publish both halves of an accumulator; both CTAs' epilogue warps release
-// it on the leader's `acc_empty`.  No load uses multicast.
+// it on the leader's `acc_empty`.  Every load fills only the issuing CTA's
+// shared memory.
 constexpr int P_STAGES = 6;
 constexpr int P_B_BYTES = (TN / 2) * TKB * 2;             // 16 KB: this CTA's half of B
 constexpr int P_RING_BYTES = P_STAGES * (A_BYTES + P_B_BYTES);  // 192 KB

@@ -75,7 +75,10 @@ enum {
   LMOE_ERR_CUDA = -5,            /* a CUDA runtime / driver call failed */
   LMOE_ERR_DEVICE_TIMEOUT = -6,  /* a kernel's bounded wait ran out (status word) */
   LMOE_ERR_UNSUPPORTED = -7,     /* valid layer, but a shape this build does not tile */
-  LMOE_ERR_OUT_OF_MEMORY = -8    /* workspace or weight allocation failed */
+  LMOE_ERR_OUT_OF_MEMORY = -8,   /* workspace or weight allocation failed */
+  LMOE_ERR_MISALIGNED = -9       /* a device array does not start on a 16-byte
+                                    boundary (cudaMalloc and torch allocations
+                                    always do); refused before any launch */
 };
 
 /* Layer hyper-parameters.  Field names follow LatentMoEConfig of the
@@ -104,7 +107,8 @@ typedef struct {
 typedef struct lmoe_layer *lmoe_handle;
 
 /* Device pointers to the caller's weights, element type = cfg.dtype (the
- * router bias is always float32), nn.Linear [out][in] row-major:
+ * router bias is always float32), nn.Linear [out][in] row-major, each used
+ * matrix starting on a 16-byte boundary (else LMOE_ERR_MISALIGNED):
  *   w_router [N'][d], b_router [N'] or NULL, w_down [l][d], w_up [d][l],
  *   w_gate [N'][m][l], w_upx [N'][m][l], w_out [N'][l][m],
  *   s_gate [n_s][m_s][d], s_up [n_s][m_s][d], s_out [n_s][d][m_s]
@@ -131,8 +135,8 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out);
  * every such matrix stored K-block tiled, one contiguous 256 x 64 block per
  * tile).  bf16 uses temporary device buffers and synchronises `stream`
  * before returning; fp32 is asynchronous (the caller's buffers may be freed
- * once `stream` has passed this call).  Errors: NULL_ARG, OUT_OF_MEMORY,
- * CUDA. */
+ * once `stream` has passed this call).  Errors: NULL_ARG, MISALIGNED,
+ * OUT_OF_MEMORY, CUDA. */
 int lmoe_load_weights(lmoe_handle h, const lmoe_weights *w, void *stream);
 
 /* Routing only (router GEMM, softmax / top-K' / renormalise, dispatch).
@@ -143,15 +147,16 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *w, void *stream);
  *     to experts < e (exclusive scan of the per-expert histogram);
  *   perm [T*K'] int32: perm[offsets[e] + r] = t*K' + k for the r-th token
  *     (ascending t) that chose expert e, in slot k.
- * T == 0 is allowed (offsets all 0).  Errors: NULL_ARG, NOT_LOADED,
- * TOO_MANY_TOKENS, CUDA. */
+ * x_dev starts on a 16-byte boundary.  T == 0 is allowed (offsets all 0).
+ * Errors: NULL_ARG, NOT_LOADED, TOO_MANY_TOKENS, MISALIGNED, CUDA. */
 int lmoe_route(lmoe_handle h, const void *x_dev, int32_t T, int32_t *ids,
                float *gates, int32_t *offsets, int32_t *perm, void *stream);
 
 /* The layer forward: y_dev [T][d] = layer(x_dev [T][d]), element type
- * cfg.dtype.  x and y must not overlap.  Graph-capturable: no host sync, no
- * allocation.  T == 0 is a no-op.  Errors: NULL_ARG, NOT_LOADED,
- * TOO_MANY_TOKENS, CUDA. */
+ * cfg.dtype.  x and y must not overlap and must start on 16-byte boundaries
+ * (the kernels move them with 16-byte vectors and TMA).  Graph-capturable:
+ * no host sync, no allocation.  T == 0 is a no-op.  Errors: NULL_ARG,
+ * NOT_LOADED, TOO_MANY_TOKENS, MISALIGNED, CUDA. */
 int lmoe_forward(lmoe_handle h, const void *x_dev, void *y_dev, int32_t T, void *stream);
 
 /* End-to-end variant with HOST buffers: copies x_host to a handle-owned
@@ -269,9 +274,10 @@ typedef struct {
  * recomputes the forward activations it needs from x_dev (same routing as
  * lmoe_forward).  Weight gradients sum the T tokens in a fixed order
  * (deterministic).  Needs a handle created with training = 1.  No host
- * sync; T == 0 writes zero gradients.  x, dy and dx must not overlap.
+ * sync; T == 0 writes zero gradients.  x, dy and dx must not overlap; they
+ * and the gradient arrays (b_router excepted) start on 16-byte boundaries.
  * Errors: NULL_ARG, NOT_LOADED, TOO_MANY_TOKENS, UNSUPPORTED (handle without
- * training), CUDA. */
+ * training), MISALIGNED, CUDA. */
 int lmoe_backward(lmoe_handle h, const void *x_dev, const void *dy_dev, void *dx_dev,
                   const lmoe_grads *grads, int32_t T, void *stream);
 

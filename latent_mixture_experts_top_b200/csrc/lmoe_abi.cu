@@ -232,6 +232,11 @@ char *off(void *base, size_t elems, size_t es) { return static_cast<char *>(base
 
 extern "C" {
 
+// The kernels move activations, weights and gradients with 16-byte vectors
+// and TMA, so every such array must start on a 16-byte boundary; the calls
+// check this before launching anything.
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 const char *lmoe_strerror(int code) {
   switch (code) {
     case LMOE_OK: return "ok";
@@ -243,6 +248,7 @@ const char *lmoe_strerror(int code) {
     case LMOE_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait ran out";
     case LMOE_ERR_UNSUPPORTED: return "shape not supported by this build";
     case LMOE_ERR_OUT_OF_MEMORY: return "device allocation failed";
+    case LMOE_ERR_MISALIGNED: return "device array not 16-byte aligned";
     default: return "unknown status";
   }
 }
@@ -428,6 +434,14 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   if (h->ns > 0 && (!wt->s_up || !wt->s_out || (!h->relu2 && !wt->s_gate)))
     return LMOE_ERR_NULL_ARG;
   if (h->cfg.has_router_bias && !wt->b_router) return LMOE_ERR_NULL_ARG;
+  {
+    const void *used[] = {wt->w_router, wt->w_down, wt->w_up, wt->w_upx, wt->w_out,
+                          h->relu2 ? nullptr : wt->w_gate,
+                          h->ns > 0 ? wt->s_up : nullptr, h->ns > 0 ? wt->s_out : nullptr,
+                          (h->ns > 0 && !h->relu2) ? wt->s_gate : nullptr};
+    for (const void *q : used)
+      if (q && !aligned16(q)) return LMOE_ERR_MISALIGNED;
+  }
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -684,6 +698,7 @@ int lmoe_route(lmoe_handle h, const void *x, int32_t T, int32_t *ids, float *gat
   int rc = check_call(h, T);
   if (rc != LMOE_OK) return rc;
   if (T > 0 && !x) return LMOE_ERR_NULL_ARG;
+  if (T > 0 && !aligned16(x)) return LMOE_ERR_MISALIGNED;
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -828,6 +843,7 @@ int lmoe_forward(lmoe_handle h, const void *x, void *y, int32_t T, void *stream)
   if (rc != LMOE_OK) return rc;
   if (T == 0) return LMOE_OK;
   if (!x || !y) return LMOE_ERR_NULL_ARG;
+  if (!aligned16(x) || !aligned16(y)) return LMOE_ERR_MISALIGNED;
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
   return forward_impl(h, x, y, T, static_cast<cudaStream_t>(stream));
@@ -1116,6 +1132,15 @@ int lmoe_backward(lmoe_handle h, const void *x, const void *dy, void *dx, const 
   if (h->cfg.has_router_bias && !g->b_router) return LMOE_ERR_NULL_ARG;
   if (h->ns > 0 && (!g->s_up || !g->s_out || (!h->relu2 && !g->s_gate))) return LMOE_ERR_NULL_ARG;
   if (T > 0 && (!x || !dy || !dx)) return LMOE_ERR_NULL_ARG;
+  if (T > 0 && (!aligned16(x) || !aligned16(dy) || !aligned16(dx))) return LMOE_ERR_MISALIGNED;
+  {
+    const float *used[] = {g->w_router, g->w_down, g->w_up, g->w_upx, g->w_out,
+                           h->relu2 ? nullptr : g->w_gate,
+                           h->ns > 0 ? g->s_up : nullptr, h->ns > 0 ? g->s_out : nullptr,
+                           (h->ns > 0 && !h->relu2) ? g->s_gate : nullptr};
+    for (const float *q : used)
+      if (q && !aligned16(q)) return LMOE_ERR_MISALIGNED;
+  }
   DeviceGuard guard(h->device);
   if (!guard.ok) return LMOE_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -28,7 +28,7 @@ LMOE_WEIGHTS_BF16, LMOE_WEIGHTS_FP8 = 0, 1
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -3: "LMOE_ERR_NOT_LOADED", -4: "LMOE_ERR_TOO_MANY_TOKENS", -5: "LMOE_ERR_CUDA",
           -6: "LMOE_ERR_DEVICE_TIMEOUT", -7: "LMOE_ERR_UNSUPPORTED",
-          -8: "LMOE_ERR_OUT_OF_MEMORY"}
+          -8: "LMOE_ERR_OUT_OF_MEMORY", -9: "LMOE_ERR_MISALIGNED"}
 EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
             "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
             "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc",

@@ -46,6 +46,13 @@ def test_binding_has_the_same_names(lib):
     assert set(lmoe.EXPORTED) >= set(_declared())
 
 
+def test_binding_status_names_match_the_header():
+    from latent_mixture_experts_top_b200 import lmoe
+    codes = {int(v): k for k, v in re.findall(r"(LMOE_(?:OK|ERR_\w+))\s*=\s*(-?\d+)",
+                                              open(HEADER).read())}
+    assert codes == lmoe.STATUS
+
+
 def _cfg(**kw):
     from latent_mixture_experts_top_b200 import lmoe
     base = dict(d=256, m=256, n_experts=8, top_k=2, alpha=2, n_shared=1, m_shared=256,
@@ -87,11 +94,11 @@ def test_null_arguments(lib):
 def test_strerror_names_every_code(lib):
     lib.lmoe_strerror.restype = C.c_char_p
     seen = set()
-    for code in range(0, -9, -1):
+    for code in range(0, -10, -1):
         s = lib.lmoe_strerror(code).decode()
         assert s and s != "unknown status"
         seen.add(s)
-    assert len(seen) == 9
+    assert len(seen) == 10
     assert lib.lmoe_strerror(-99).decode() == "unknown status"
 
 

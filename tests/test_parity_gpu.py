@@ -225,6 +225,36 @@ def test_call_errors_on_device_handle():
     lm.lmoe_destroy(h)
 
 
+def test_misaligned_device_arrays_are_refused_before_any_launch():
+    """x or y a few bytes off a 16-byte boundary (2 bytes for bf16, 4 for
+    fp32): route and forward return LMOE_ERR_MISALIGNED without launching
+    anything, and the same handle then runs a normal forward."""
+    lm = _lmoe()
+    for cfg in (configs.TINY_F32, MID_PAIR):
+        inp = _inputs(cfg)
+        x = inp["x"]
+        T, d = x.shape
+        layer = lm.LatentMoELayer(cfg, inp)
+        buf = torch.empty(2 * T * d + 16, dtype=x.dtype, device=x.device)
+        x_bad = buf[1:1 + T * d].view(T, d)
+        y_bad = buf[T * d + 9:2 * T * d + 9].view(T, d)
+        assert x_bad.data_ptr() % 16 != 0 and y_bad.data_ptr() % 16 != 0
+        x_bad.copy_(x)
+        y = torch.empty_like(x)
+        for xx, yy in ((x_bad, y), (x, y_bad)):
+            with pytest.raises(lm.LmoeError) as e:
+                lm.lmoe_forward(layer.handle, xx, yy, T)
+            assert e.value.code == -9
+        with pytest.raises(lm.LmoeError) as e:
+            lm.lmoe_route(layer.handle, x_bad, T)
+        assert e.value.code == -9
+        y_ok = layer.forward(x)
+        torch.cuda.synchronize()
+        assert lm.lmoe_device_status(layer.handle) == 0
+        assert torch.isfinite(y_ok.float()).all()
+        layer.close()
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     """Failure detection without a GPU fault: a wait that nothing completes
     runs out after 1 ms, the status word reports it, and the next forward on

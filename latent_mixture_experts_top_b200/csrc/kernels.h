@@ -91,7 +91,8 @@ struct TcParams {
   int Kdim;            // reduction length, multiple of 64
   int n_tiles_n;       // N-tiles of 256 columns in this launch
   int n_tile_base;     // dense modes: first N-tile (a launch may cover a column range)
-  const TileEntry *tiles;   // grouped modes
+  const TileEntry *tiles;   // grouped modes: the M-tile table (128-row tiles for
+                            // launch_tc_gemm, 256-row tiles for launch_tc_gemm_pair)
   const int32_t *n_mtiles;  // grouped modes: device count of M-tiles
   int b_rows_per_expert;    // unused (B is K-block tiled: see launch_repack_btiles)
   // TC_X_FUSED column regions (multiples of 256): [0, r_end) router logits,

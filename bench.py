@@ -96,14 +96,20 @@ def load_peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 def stage_work(cfg, touched=None):
-    """Algorithmic (FLOPs, bytes) of one launch of each profiled stage.
+    """(FLOPs, algorithmic bytes, intermediate bytes) of one launch of each
+    profiled stage.
 
     FLOPs count 2 per multiply-add of the layer's definition (no padding, no
-    masked rows); memory-only stages have 0.  Bytes are what the stage must
-    read and write once: bf16 activations and weights, int32 indices, fp32
-    logits and gates; an expert GEMM reads the weights of the ``touched``
-    distinct experts (all N' when not given).  The shared experts' gate/up
-    GEMM overlaps stages 1-3 on a side stream and is not a stage of its own.
+    masked rows); memory-only stages have 0.  Algorithmic bytes are the
+    layer's own inputs and outputs that the stage must move once: the weights
+    it multiplies by (for an expert GEMM, those of the ``touched`` distinct
+    experts, all N' when not given), x into the first GEMM and y out of the
+    last.  Intermediates (logits, ids, gates, dispatch indices, z, the
+    permuted z, H, O, u and the shared hidden) are not algorithmic bytes:
+    their traffic depends on how the path is cut into kernels, so it is
+    reported apart, in the third entry.  The shared experts' gate/up GEMM
+    overlaps stages 1-3 on a side stream and is not a stage of its own (see
+    shared_gate_up_work).
     """
     T, d, l, m, N, K = cfg.T, cfg.d, cfg.l, cfg.m, cfg.n_routed, cfg.k_active
     ns, ms = cfg.n_shared, cfg.m_shared
@@ -113,19 +119,32 @@ def stage_work(cfg, touched=None):
     ew = expert_weight_bytes(cfg)
     ky = l + ns * ms
     return {
-        0: (2.0 * T * d * (N + l), 2.0 * T * d + 2.0 * d * (N + l) + 4.0 * T * N + 2.0 * T * l),
-        1: (0.0, 4.0 * T * N + 8.0 * TK),
-        2: (0.0, 4.0 * TK * 5),
-        3: (0.0, 2.0 * TK * l * 2 + 4.0 * TK),
-        4: (2.0 * TK * l * gu * m, 2.0 * TK * l + ew * E * gu * m * l + 2.0 * TK * m),
-        5: (2.0 * TK * m * l, 2.0 * TK * m + ew * E * l * m + 2.0 * TK * l),
-        6: (0.0, 2.0 * TK * l + 8.0 * TK + 2.0 * T * l),
-        7: (2.0 * T * ky * d, 2.0 * T * ky + 2.0 * d * ky + 2.0 * T * d),
+        0: (2.0 * T * d * (N + l), 2.0 * T * d + 2.0 * d * (N + l), 4.0 * T * N + 2.0 * T * l),
+        1: (0.0, 0.0, 4.0 * T * N + 8.0 * TK),
+        2: (0.0, 0.0, 4.0 * TK * 5),
+        3: (0.0, 0.0, 2.0 * TK * l * 2 + 4.0 * TK),
+        4: (2.0 * TK * l * gu * m, ew * E * gu * m * l, 2.0 * TK * l + 2.0 * TK * m),
+        5: (2.0 * TK * m * l, ew * E * l * m, 2.0 * TK * m + 2.0 * TK * l),
+        6: (0.0, 0.0, 2.0 * TK * l + 8.0 * TK + 2.0 * T * l),
+        7: (2.0 * T * ky * d, 2.0 * d * ky + 2.0 * T * d, 2.0 * T * ky),
     }
 
 
+def shared_gate_up_work(cfg):
+    """(FLOPs, algorithmic bytes, intermediate bytes) of the side-stream
+    shared-expert gate/up GEMM: its weights are algorithmic; x is counted
+    once, by stage 0; the shared hidden it writes is an intermediate."""
+    gu = n_mats(cfg) - 1
+    nsms = cfg.n_shared * cfg.m_shared
+    return (2.0 * cfg.T * cfg.d * gu * nsms, 2.0 * cfg.d * gu * nsms, 2.0 * cfg.T * nsms)
+
+
 def stage_bound(flops, nbytes, peaks):
-    """'tensor' or 'hbm': whichever takes longer at the measured peaks."""
+    """'tensor' or 'hbm': whichever takes longer at the measured peaks (a
+    stage with neither FLOPs nor algorithmic bytes is a memory-bound helper:
+    'hbm')."""
+    if flops <= 0.0 and nbytes <= 0.0:
+        return "hbm"
     t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     return "tensor" if t_tensor >= t_hbm else "hbm"
@@ -178,7 +197,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x2: "applications_clocks_setting", 0x10: "sync_boost"}
 
-    def __init__(self, index, period=0.02):
+    def __init__(self, index, period=0.002):
         self.index, self.period = index, period
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -420,7 +439,7 @@ def run_ours(args):
     work = stage_work(cfg, touched=len(set(ids.reshape(-1).tolist())))
     avg_stage = [t / max(1, n_prof) for t in stage_ms]
     dom = max(range(len(avg_stage)), key=lambda i: avg_stage[i])
-    flops, nbytes = work[dom]
+    flops, nbytes, inter = work[dom]
     kind = stage_bound(flops, nbytes, peaks)
     if kind == "tensor":
         amount, unit, peak = flops, "TFLOP/s", peaks["bf16_tflops"]
@@ -434,7 +453,9 @@ def run_ours(args):
                 "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} (burst)" if kind == "tensor" else peak_src,
                 "algorithmic_per_launch": amount, "algorithmic_flops": flops,
-                "algorithmic_bytes": nbytes, "avg_launch_ms": avg_stage[dom]}
+                "algorithmic_bytes": nbytes, "intermediate_bytes": inter,
+                "bytes_ratio_with_intermediates": (nbytes + inter) / nbytes if nbytes else None,
+                "avg_launch_ms": avg_stage[dom]}
     F, B = layer_flops(cfg), layer_bytes(cfg, ids)
     t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
     layer_roof = {"flops": F, "bytes": B, "roofline_ms": 1e3 * t_roof,

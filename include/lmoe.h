@@ -53,8 +53,8 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
 
 /* Expert activation.  LMOE_SWIGLU: E(v) = W_o (silu(W_g v) * (W_u v)), three
  * matrices.  LMOE_RELU2: E(v) = W_o (relu(W_u v))^2, two matrices -- the
- * Expert class of the article's code ("down(relu(up(x)) ** 2)"), the
- * activation its 95B running example uses.  Shared experts use the same. */
+ * Expert class of the article's code module, the activation its 95B running
+ * example uses.  Shared experts use the same. */
 typedef enum { LMOE_SWIGLU = 0, LMOE_RELU2 = 1 } lmoe_activation;
 
 /* Storage of the routed experts' weights (W_g, W_u, W_o) in LMOE_BF16 mode.
@@ -224,9 +224,14 @@ int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int32_t *n_forwards,
  * framework forbids allocation inside its execute callback.
  *
  * Given ids [T][k_active] int32 on the device (as lmoe_route produces them:
- * every id in [0, n_routed), no id twice in a row -- other values are not
- * checked and their result is undefined), writes offsets [n_routed+1] and
- * perm [T*k_active] exactly as lmoe_route does, asynchronously on `stream`.
+ * every id in [0, n_routed), no id twice in a row), writes offsets
+ * [n_routed+1] and perm [T*k_active] exactly as lmoe_route does,
+ * asynchronously on `stream`.  Other ids are tolerated without any
+ * out-of-bounds access: a pair whose id lies outside [0, n_routed) is
+ * skipped (not counted in offsets, not placed in perm), so offsets[n_routed]
+ * is the number of pairs placed and perm from that index on holds -1; a row
+ * that names one expert twice places both pairs at one position of that
+ * expert's range, and the position left over holds -1.
  * It needs no handle and calls no cudaMalloc, cudaFree or allocating
  * routine: its scratch (about 3 MiB) is one fixed file-scope device array
  * that every GPU loading this library holds until the process exits.
@@ -237,7 +242,8 @@ int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int32_t *n_forwards,
  *     NULL ids / perm with T > 0, gives LMOE_ERR_NULL_ARG.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept until the process
+ *     exits, so do not call this after cudaDeviceReset on that device.
  *   - All calls on a device share the one array, and it keeps the last
  *     call's contents (each call rewrites every word it reads).  Calls that
  *     overlap on the GPU -- on different streams, or from different threads

@@ -47,7 +47,9 @@ constexpr size_t kScratchBytes = kOffNTiles + 256;
 static __device__ __align__(256) unsigned char g_dispatch_scratch[kScratchBytes];
 
 // Device address of g_dispatch_scratch, looked up once per device with that
-// device current (the first call on the device does it).
+// device current (the first call on the device does it) and kept for the
+// life of the process: after a cudaDeviceReset the module may load at another
+// address, so the entry point must not be called after a reset.
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void *g_scratch_addr[kMaxDevices] = {};
@@ -94,9 +96,16 @@ extern "C" int lmoe_dispatch_noalloc(const int32_t *ids, int32_t T, int32_t k_ac
   int32_t *row_expert = reinterpret_cast<int32_t *>(base + kOffRowExpert);
   TileEntry *tiles = reinterpret_cast<TileEntry *>(base + kOffTiles);
   int32_t *n_tiles = reinterpret_cast<int32_t *>(base + kOffNTiles);
-  const cudaError_t e =
-      launch_dispatch(ids, T, k_active, n_routed, counts, kChunk, false, offsets, perm, pos,
-                      row_expert, tiles, n_tiles, kTileRows, kMaxTiles,
-                      static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The ids come from the caller: the kernels skip any outside [0, n_routed)
+  // (check_ids), and perm starts as -1 so that the entries such pairs would
+  // have filled are defined.
+  cudaError_t e = cudaSuccess;
+  if (T > 0)
+    e = cudaMemsetAsync(perm, 0xFF, static_cast<size_t>(T) * k_active * sizeof(int32_t), s);
+  if (e == cudaSuccess)
+    e = launch_dispatch(ids, T, k_active, n_routed, counts, kChunk, false, offsets, perm, pos,
+                        row_expert, tiles, n_tiles, kTileRows, kMaxTiles, s, nullptr, nullptr,
+                        0, 0, /*check_ids=*/true);
   return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

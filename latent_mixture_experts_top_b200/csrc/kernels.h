@@ -35,12 +35,15 @@ inline size_t dispatch_count_elems(int T, int chunk, int N) {
 // row_expert [T*K], and the M-tile table (tile_m rows per tile; capacity
 // max_tiles entries) plus its length in *n_tiles; with tiles2, also a second
 // table of tile_m2-row M-tiles (capacity max_tiles2) and its length.
+// check_ids (ids from a caller rather than the top-K kernel): pairs whose id
+// lies outside [0, N) are skipped -- not counted, not placed -- so that no
+// kernel indexes memory with them; without it every id must be in range.
 cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *chunk_counts,
                             int chunk, bool counts_ready, int32_t *offsets, int32_t *perm,
                             int32_t *pos, int32_t *row_expert, TileEntry *tiles,
                             int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s,
                             TileEntry *tiles2 = nullptr, int32_t *n_tiles2 = nullptr,
-                            int tile_m2 = 0, int max_tiles2 = 0);
+                            int tile_m2 = 0, int max_tiles2 = 0, bool check_ids = false);
 
 // dst[p][:] = src[perm[p] / K][:], rows of `row_bytes` (multiple of 16).
 cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,

@@ -1,9 +1,10 @@
 // route_kernels.cu -- routing, dispatch, permutation and combine kernels.
 //
 // Sources: "LatentMoE Explained" (Towards AI), Figure 3 (router: one score
-// per expert, softmax, top-K), the LatentMoE code module (top-k of the
-// softmax, w / w.sum(), the slot loop "for e in e_ids.unique(): sel = e_ids
-// == e; out[sel] += gate[sel] * expert(z[sel])").  The pages' masked loop is
+// per expert, softmax, top-K), the LatentMoE code module (top-K of the
+// softmax, the selected weights renormalised to sum to one, and a slot loop
+// that masks, expert by expert, the tokens that chose it and adds the gated
+// expert output to theirs).  The pages' masked loop is
 // replaced by a histogram -> exclusive scan -> stable scatter that yields the
 // same grouping (experts in index order, tokens ascending within an expert)
 // in three launches and no host synchronisation.
@@ -90,17 +91,23 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
 // Count matrix layout: counts[e][c] (expert-major), c = token chunk, row
 // stride n_chunks rounded up to a multiple of 4 (16-byte rows).
 // Phase 1 (when the top-K kernel did not count): per-chunk expert histogram.
+// check_ids: ids come from the caller, not from the top-K kernel, so an id
+// outside [0, N) is skipped instead of indexing the histogram with it.
 __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t *__restrict__ ids,
                                                              int T, int K, int N,
                                                              int32_t *__restrict__ counts,
-                                                             int n_chunks, int chunk) {
+                                                             int n_chunks, int chunk,
+                                                             int check_ids) {
   extern __shared__ int32_t cnt[];  // [N]
   for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   const int t0 = blockIdx.x * chunk;
   const int tn = min(chunk, T - t0);
   const int32_t *base = ids + static_cast<size_t>(t0) * K;
-  for (int i = threadIdx.x; i < tn * K; i += blockDim.x) atomicAdd(&cnt[base[i]], 1);
+  for (int i = threadIdx.x; i < tn * K; i += blockDim.x) {
+    const int e = base[i];
+    if (!check_ids || static_cast<unsigned>(e) < static_cast<unsigned>(N)) atomicAdd(&cnt[e], 1);
+  }
   __syncthreads();
   const int ncp = (n_chunks + 3) & ~3;
   for (int e = threadIdx.x; e < N; e += blockDim.x)
@@ -234,10 +241,11 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
 // warp's tokens that chose the same expert (a token picks an expert at most
 // once); the per-warp counts are scanned across the block's warps, and the
 // chunk's base comes from phase 2.  Tokens therefore land in ascending order.
+// check_ids: as in phase 1, pairs whose id lies outside [0, N) are skipped.
 __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
     const int32_t *__restrict__ ids, int T, int K, int N, const int32_t *__restrict__ counts,
     int n_chunks, int chunk, const int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
-    int32_t *__restrict__ pos, int32_t *__restrict__ row_expert) {
+    int32_t *__restrict__ pos, int32_t *__restrict__ row_expert, int check_ids) {
   extern __shared__ uint32_t sm[];
   const int W = blockDim.x >> 5;
   uint32_t *mask = sm;                                        // [W][N]
@@ -249,7 +257,11 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
   const bool valid = t < T;
   const int32_t *my_ids = ids + static_cast<size_t>(t) * K;
   if (valid)
-    for (int k = 0; k < K; ++k) atomicOr(&mask[w * N + my_ids[k]], 1u << lane);
+    for (int k = 0; k < K; ++k) {
+      const int e = my_ids[k];
+      if (!check_ids || static_cast<unsigned>(e) < static_cast<unsigned>(N))
+        atomicOr(&mask[w * N + e], 1u << lane);
+    }
   __syncthreads();
   for (int e = threadIdx.x; e < N; e += blockDim.x) {
     int run = 0;
@@ -263,6 +275,7 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
   const uint32_t lt = (1u << lane) - 1u;
   for (int k = 0; k < K; ++k) {
     const int e = my_ids[k];
+    if (check_ids && static_cast<unsigned>(e) >= static_cast<unsigned>(N)) continue;
     const int p = offsets[e] + counts[static_cast<size_t>(e) * ((n_chunks + 3) & ~3) + blockIdx.x] +
                   wbase[w * N + e] + __popc(mask[w * N + e] & lt);
     const int flat = t * K + k;
@@ -428,12 +441,13 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
                             int chunk, bool counts_ready, int32_t *offsets, int32_t *perm,
                             int32_t *pos, int32_t *row_expert, TileEntry *tiles,
                             int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s,
-                            TileEntry *tiles2, int32_t *n_tiles2, int tile_m2, int max_tiles2) {
+                            TileEntry *tiles2, int32_t *n_tiles2, int tile_m2, int max_tiles2,
+                            bool check_ids) {
   if (N > 1024 || chunk % 32 || chunk < 32 || chunk > 256) return cudaErrorInvalidValue;
   const int nc = dispatch_chunks(T, chunk);
   if (nc > 0 && !counts_ready) {
     dispatch_count_kernel<<<nc, 256, N * sizeof(int32_t), s>>>(ids, T, K, N, chunk_counts, nc,
-                                                               chunk);
+                                                               chunk, check_ids ? 1 : 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -451,7 +465,8 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
     if (e != cudaSuccess) return e;
   }
   dispatch_scatter_kernel<<<nc, 32 * warps, smem, s>>>(ids, T, K, N, chunk_counts, nc, chunk,
-                                                       offsets, perm, pos, row_expert);
+                                                       offsets, perm, pos, row_expert,
+                                                       check_ids ? 1 : 0);
   return cudaGetLastError();
 }
 

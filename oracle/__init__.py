@@ -68,6 +68,8 @@ def _load():
             lib.oracle_router_logits.restype = None
             lib.oracle_select.argtypes = [P, I64, I32, I32, P, P]
             lib.oracle_select.restype = C.c_int
+            lib.oracle_gates.argtypes = [P, I64, I32, I32, P, P]
+            lib.oracle_gates.restype = C.c_int
             lib.oracle_forward.argtypes = [P, P, I64, P, I64, P, P, P, P]
             lib.oracle_forward.restype = C.c_int
             lib.oracle_dispatch.argtypes = [P, I64, I32, I32, P, P, P]
@@ -198,6 +200,20 @@ def select(logits: np.ndarray, k: int):
     if _load().oracle_select(_ptr(s), T, N, k, _ptr(ids), _ptr(g)) != 0:
         raise ValueError("k must be in [1, N']")
     return ids, g
+
+
+def gates_for_ids(logits: np.ndarray, ids: np.ndarray) -> np.ndarray:
+    """Gates of given selections: softmax at ``ids`` renormalised over them (fp64)."""
+    s = np.ascontiguousarray(logits, dtype=np.float64)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, N = s.shape
+    assert ids.shape[0] == T
+    k = ids.shape[1]
+    g = np.empty((T, k), dtype=np.float64)
+    rc = _load().oracle_gates(_ptr(s), T, N, k, _ptr(ids), _ptr(g))
+    if rc != 0:
+        raise ValueError("k must be in [1, N'] and every id in [0, N')")
+    return g
 
 
 def forward(layer: Layer, x, tokens=None, ids=None):

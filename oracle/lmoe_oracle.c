@@ -28,10 +28,10 @@
  *   5. z   = W_down x                                      d -> l, no bias
  *   6. u   = sum_{k=0..K'-1} g_k E_{id_k}(z),  E(v) = W_o (silu(W_g v) * (W_u v))
  *   7. y   = W_up u + sum_{j=0..n_s-1} S_j(x)              S_j: SwiGLU at width d
- * With activation = squared ReLU (the Expert class of the [Explained] code,
- * "down(relu(up(x)) ** 2)", two matrices), E(v) = W_o (relu(W_u v))^2 and the
- * shared experts likewise; W_g is unused.
- * Readings where the pages are silent (each listed in the design doc):
+ * With activation = squared ReLU (the Expert class of the [Explained] code:
+ * two matrices, the up-projection's output passed through relu and squared),
+ * E(v) = W_o (relu(W_u v))^2 and the shared experts likewise; W_g is unused.
+ * Readings where the pages are silent:
  *   - experts are SwiGLU with three matrices (the pages' code shows squared
  *     ReLU with two; the article says SwiGLU carries over with a third
  *     matrix, and [Shaping] Table 9 names W_g, W_u, W_o); silu(a)=a/(1+e^-a);
@@ -141,7 +141,8 @@ void oracle_router_logits(const oracle_layer *L, const void *x, int64_t T,
 }
 
 /* ---- steps 2-4 for one token: softmax, top-K', renormalised gates.
- * [Explained] LatentMoE code: topk(softmax(scores)), then w / w.sum(). */
+ * [Explained] LatentMoE code module: the top-K' of the softmax of the
+ * scores, then the selected weights divided by their sum. */
 static void select_row(const double *s, int N, int K, int32_t *ids,
                        double *gates, unsigned char *taken) {
   double smax = s[0];
@@ -193,6 +194,20 @@ static void gates_for_ids(const double *s, int N, int K, const int32_t *ids,
     psum += gates[k];
   }
   for (int k = 0; k < K; ++k) gates[k] /= psum;
+}
+
+/* Gates of caller-given selections, row by row: step 4's rule (softmax at
+ * the selected ids, renormalised over them) applied to any K'-subset, e.g.
+ * a selection that differs from ours only on a near-tie. */
+int oracle_gates(const double *s, int64_t T, int N, int K, const int32_t *ids,
+                 double *gates) {
+  if (K < 1 || K > N) return -1;
+  for (int64_t i = 0; i < T * K; ++i)
+    if (ids[i] < 0 || ids[i] >= N) return -2;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t)
+    gates_for_ids(s + t * N, N, K, ids + t * K, gates + t * K);
+  return 0;
 }
 
 /* ---- components, exposed so tests can recompose the layer another way */
@@ -294,8 +309,9 @@ int oracle_forward(const oracle_layer *L, const void *x, int64_t T,
 }
 
 /* ---- dispatch: group the (token, slot) pairs by expert.
- * [Explained] code: "for e in e_ids.unique(): sel = e_ids == e" visits, per
- * expert, the tokens that chose it in token order.  Written out plainly:
+ * [Explained] LatentMoE code module: its slot loop visits each distinct
+ * expert once and takes, through a boolean mask, the tokens that chose it,
+ * in token order.  Written out plainly:
  * offsets[e] = number of pairs with expert < e (exclusive prefix count);
  * perm lists, expert by expert, the flat pair index t*K+k with t ascending;
  * pos is the inverse of perm. */

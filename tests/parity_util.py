@@ -4,8 +4,9 @@ oracle on the same seeded inputs and compare.
 Comparison rules (tolerances stated where they are used):
 * routing: the oracle's fp64 logits decide.  A token whose K'-th and
   (K'+1)-th largest logits are within NEAR_TIE of each other is "near-tie":
-  several selections are correct up to rounding, so only validity is checked
-  there.  Everywhere else the selected set must be identical, and the slot
+  several selections are correct up to rounding, so there the GPU's set must
+  be a correct top-K' of the fp64 logits (up to ORDER_TOL) with every
+  differing expert inside the tie band.  Everywhere else the selected set must be identical, and the slot
   order identical wherever consecutive selected logits differ by more than
   ORDER_TOL; within ORDER_TOL the GPU order must still be non-increasing in
   the oracle's logits up to ORDER_TOL.
@@ -47,16 +48,38 @@ def boundary_gap(s_ref: np.ndarray, K: int) -> np.ndarray:
 
 
 def check_routing(ids_gpu: np.ndarray, gates_gpu: np.ndarray, s_ref: np.ndarray, K: int):
-    """Returns (near mask, flipped mask) after asserting the rules above."""
-    T = s_ref.shape[0]
+    """Returns (near mask, flipped mask) after asserting the rules above.
+
+    Where the GPU's set differs from the oracle's (possible only on near-tie
+    tokens), the GPU's set must itself be a correct top-K' of the fp64
+    logits: its smallest selected logit is not below the largest unselected
+    one (up to ORDER_TOL, the fp32-vs-fp64 logit error), and every expert
+    that is in one set but not the other lies within NEAR_TIE of the K'-th
+    largest logit.  Gates are checked on every token against the oracle's
+    gates for the GPU's own ids."""
+    T, N = s_ref.shape
     ids_ref, g_ref = oracle.select(s_ref, K)
     near = boundary_gap(s_ref, K) <= NEAR_TIE
+    # every GPU selection is well formed: in range, K' distinct experts
+    assert ((ids_gpu >= 0) & (ids_gpu < N)).all()
+    assert all(len(set(r)) == K for r in ids_gpu.tolist())
     same_set = np.array([set(a) == set(b) for a, b in zip(ids_gpu.tolist(), ids_ref.tolist())])
     bad = ~same_set & ~near
     assert not bad.any(), f"selection differs on {bad.sum()} tokens with a clear gap, e.g. {np.nonzero(bad)[0][:5]}"
-    # every GPU selection is valid: distinct, in range
-    assert ((ids_gpu >= 0) & (ids_gpu < s_ref.shape[1])).all()
-    assert all(len(set(r)) == K for r in ids_gpu.tolist())
+    # the GPU's set is a top-K' of the fp64 logits on every token
+    if K < N:
+        chosen = np.zeros((T, N), dtype=bool)
+        chosen[np.arange(T)[:, None], ids_gpu.astype(np.int64)] = True
+        sel_min = np.where(chosen, s_ref, np.inf).min(axis=1)
+        unsel_max = np.where(chosen, -np.inf, s_ref).max(axis=1)
+        worst = np.nonzero(sel_min < unsel_max - ORDER_TOL)[0]
+        assert worst.size == 0, f"not a top-K' selection on tokens {worst[:5]}"
+        # flipped experts sit in the near-tie band around the K'-th logit
+        kth = -np.sort(-s_ref, axis=1)[:, K - 1]
+        for t in np.nonzero(~same_set)[0]:
+            diff = set(ids_gpu[t].tolist()) ^ set(ids_ref[t].tolist())
+            for e in diff:
+                assert abs(s_ref[t, e] - kth[t]) <= NEAR_TIE, (t, e, s_ref[t, e] - kth[t])
     # order: non-increasing in the oracle's logits (up to ORDER_TOL); identical
     # where the oracle's consecutive gaps are clear
     s_sel = np.take_along_axis(s_ref, ids_gpu.astype(np.int64), 1)
@@ -64,7 +87,10 @@ def check_routing(ids_gpu: np.ndarray, gates_gpu: np.ndarray, s_ref: np.ndarray,
     s_ref_sel = np.take_along_axis(s_ref, ids_ref.astype(np.int64), 1)
     clear = (np.abs(np.diff(s_ref_sel, axis=1)) > ORDER_TOL).all(axis=1) & same_set
     np.testing.assert_array_equal(ids_gpu[clear], ids_ref[clear])
-    # gates: renormalised softmax of the selected logits (fp32 vs fp64)
+    # gates: renormalised softmax at the GPU's own ids (fp32 vs fp64), on every
+    # token; where the ids are the oracle's own, also its own gates
+    g_for_gpu_ids = oracle.gates_for_ids(s_ref, ids_gpu)
+    np.testing.assert_allclose(gates_gpu, g_for_gpu_ids, rtol=0, atol=1e-4)
     ids_match = (ids_gpu == ids_ref).all(axis=1)
     np.testing.assert_allclose(gates_gpu[ids_match], g_ref[ids_match], rtol=0, atol=1e-4)
     np.testing.assert_allclose(gates_gpu.sum(1), 1.0, rtol=0, atol=1e-5)
@@ -113,6 +139,24 @@ def reference_y(L: oracle.Layer, x_np, tokens: np.ndarray, ids_gpu: np.ndarray,
 
 def y_to_numpy(y: torch.Tensor) -> np.ndarray:
     return y.detach().float().cpu().numpy().astype(np.float64)
+
+
+def tile_cover_tokens(offsets: np.ndarray, perm: np.ndarray, K: int,
+                      tile_rows=(128, 256)) -> np.ndarray:
+    """Tokens that put at least one compared row into every expert's first
+    and last M-tile, for each grouped-GEMM tile height: per expert, the first
+    row of its range, the first row of its last tile and its last row (the
+    ragged tail)."""
+    rows = set()
+    for e in range(len(offsets) - 1):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 <= r0:
+            continue
+        rows.update((r0, r1 - 1))
+        for tm in tile_rows:
+            rows.add(r0 + (r1 - 1 - r0) // tm * tm)
+    rows = np.array(sorted(rows), dtype=np.int64)
+    return np.unique(perm[rows] // K).astype(np.int64)
 
 
 def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:

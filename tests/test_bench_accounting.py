@@ -45,10 +45,22 @@ def test_squared_relu_layer_flops_drop_one_matrix_per_expert():
 @pytest.mark.parametrize("cfg", ALL, ids=lambda c: c.name)
 def test_stage_flops_add_up_to_the_layer(cfg):
     work = bench.stage_work(cfg)
-    staged = sum(f for f, _ in work.values())
+    staged = sum(w[0] for w in work.values())
+    assert bench.shared_gate_up_work(cfg)[0] == _shared_gate_up_flops(cfg)
     assert staged + _shared_gate_up_flops(cfg) == pytest.approx(bench.layer_flops(cfg), rel=1e-12)
-    for stage in (1, 2, 3, 6):   # routing, dispatch, permute, combine move bytes only
-        assert work[stage][0] == 0.0 and work[stage][1] > 0.0
+    for stage in (1, 2, 3, 6):   # routing, dispatch, permute, combine: intermediates only
+        assert work[stage][0] == 0.0 and work[stage][1] == 0.0 and work[stage][2] > 0.0
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=lambda c: c.name)
+def test_stage_bytes_add_up_to_the_layer(cfg):
+    """Algorithmic bytes are touched weights + x + y only: summed over the
+    stages and the side-stream shared GEMM they give layer_bytes exactly."""
+    for touched in (None, 37):
+        work = bench.stage_work(cfg, touched=touched)
+        staged = sum(w[1] for w in work.values()) + bench.shared_gate_up_work(cfg)[1]
+        ids = None if touched is None else __import__("numpy").arange(touched)
+        assert staged == pytest.approx(bench.layer_bytes(cfg, ids), rel=1e-12)
 
 
 def test_readme_acc_figures_quoted_in_the_design_notes():
@@ -57,9 +69,15 @@ def test_readme_acc_figures_quoted_in_the_design_notes():
     assert round(bench.layer_flops(cfg) / 1e9, 1) == 588.4
     assert round(work[4][0] / 1e9, 1) == 283.5      # expert gate/up GEMM
     assert round(work[5][0] / 1e9, 1) == 141.7      # expert down GEMM
-    # gate/up bytes: permuted z in, the 256 experts' gate/up weights, H out
+    # gate/up: algorithmic bytes are the 256 experts' gate/up weights; the
+    # permuted z in and H out are intermediates
     TK = cfg.T * cfg.k_active
-    assert work[4][1] == 2 * TK * cfg.l + 2 * 256 * 2 * cfg.m * cfg.l + 2 * TK * cfg.m
+    assert work[4][1] == 2 * 256 * 2 * cfg.m * cfg.l
+    assert round(work[4][1] / 1e6, 1) == 738.2
+    assert work[4][2] == 2 * TK * cfg.l + 2 * TK * cfg.m
+    # so the stage is tensor-bound at the measured peaks
+    peaks = {"bf16_tflops": 1640.9, "hbm_gbs": 6441.9}
+    assert bench.stage_bound(work[4][0], work[4][1], peaks) == "tensor"
 
 
 def test_touched_experts_scale_only_the_weight_bytes():
@@ -83,3 +101,4 @@ def test_stage_bound_picks_the_slower_roof():
     peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 1000.0}
     assert bench.stage_bound(2e12, 1e9, peaks) == "tensor"    # 2 ms of math, 1 ms of bytes
     assert bench.stage_bound(1e12, 2e9, peaks) == "hbm"
+    assert bench.stage_bound(0.0, 0.0, peaks) == "hbm"     # a memory-only helper

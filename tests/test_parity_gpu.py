@@ -45,6 +45,9 @@ def _run(cfg, inp, x=None, max_tokens=None):
 
 
 def _check_layer(cfg, n_sample, seed=0):
+    """n_sample: compare that many sampled tokens, every token (>= T), or
+    "tiles": the tokens that put a compared row into every expert's first and
+    last grouped-GEMM M-tile (128- and 256-row tiles), plus a random spread."""
     inp = _inputs(cfg, seed)
     layer, y, ids, gates, offsets, perm = _run(cfg, inp)
     L = pu.oracle_layer(inp, cfg.k_active, cfg.activation)
@@ -57,11 +60,18 @@ def _check_layer(cfg, n_sample, seed=0):
         ids_ref, _ = oracle.select(s_ref, cfg.k_active)
         pu.check_dispatch_against_oracle_ids(ids_ref, ids_g, offsets.cpu().numpy(),
                                              perm.cpu().numpy(), cfg.n_routed)
-    tok = pu.sample_tokens(cfg.T, n_sample) if n_sample < cfg.T else np.arange(cfg.T)
+    if n_sample == "tiles":
+        cover = pu.tile_cover_tokens(offsets.cpu().numpy(), perm.cpu().numpy(), cfg.k_active)
+        tok = np.union1d(cover, pu.sample_tokens(cfg.T, 64))
+    elif n_sample < cfg.T:
+        tok = pu.sample_tokens(cfg.T, n_sample)
+    else:
+        tok = np.arange(cfg.T)
     y_ref = pu.reference_y(L, x_np, tok, ids_g, flipped)
     err = pu.rel_err(pu.y_to_numpy(y)[tok], y_ref)
     tol = pu.TOL_F32 if cfg.dtype == "f32" else pu.TOL_BF16
-    print(f"{cfg.name}: rel err {err:.3e} (tol {tol}), near-tie {near.sum()}, flipped {flipped.sum()}")
+    print(f"{cfg.name}: rel err {err:.3e} (tol {tol}) over {len(tok)} tokens, "
+          f"near-tie {near.sum()}, flipped {flipped.sum()}")
     assert err <= tol
     layer.close()
     return err
@@ -71,12 +81,12 @@ def test_parity_tiny_f32_all_tokens():
     _check_layer(configs.TINY_F32, n_sample=10 ** 9)
 
 
-def test_parity_readme_acc():
-    _check_layer(configs.README_ACC, n_sample=96)
+def test_parity_readme_acc_all_tokens():
+    _check_layer(configs.README_ACC, n_sample=10 ** 9)
 
 
-def test_parity_readme_eff():
-    _check_layer(configs.README_EFF, n_sample=96)
+def test_parity_readme_eff_all_tokens():
+    _check_layer(configs.README_EFF, n_sample=10 ** 9)
 
 
 def test_parity_decode_all_tokens():
@@ -84,7 +94,9 @@ def test_parity_decode_all_tokens():
 
 
 def test_parity_prefill_biased_router():
-    _check_layer(configs.PREFILL, n_sample=48)
+    """Every expert's first and last 128-row (gate/up) and 256-row (down, CTA
+    pairs) M-tile holds a compared row."""
+    _check_layer(configs.PREFILL, n_sample="tiles")
 
 
 # A mid-size layer whose experts average 275 rows (T K / N = 1100 * 8 / 32),
@@ -108,7 +120,7 @@ def test_parity_relu2_tiny_f32_all_tokens():
 
 def test_parity_relu2_95b_shape():
     """Squared-ReLU experts at the article's 95B running-example layer shape."""
-    _check_layer(configs.RELU2_95B, n_sample=48)
+    _check_layer(configs.RELU2_95B, n_sample=96)
 
 
 @pytest.mark.parametrize("cfg,T", [(configs.TINY_F32, 1), (configs.TINY_F32, 5),

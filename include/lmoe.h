@@ -102,6 +102,9 @@ typedef struct {
                                 keeps the extra weight layouts and workspace
                                 the backward needs); 0: forward only */
   int32_t weight_format;     /* lmoe_weight_format (bf16 dtype only) */
+  int32_t ep_rank;           /* expert parallelism: this rank, in [0, ep_world) */
+  int32_t ep_world;          /* ranks the N' routed experts are split over; 0 or
+                                1 = no expert parallelism (see lmoe_ep_dispatch) */
 } lmoe_config;
 
 typedef struct lmoe_layer *lmoe_handle;
@@ -216,6 +219,70 @@ int lmoe_profile(lmoe_handle h, int32_t slots);
  * in total.  Any output may be NULL.  Errors: NULL_ARG, CUDA. */
 int lmoe_stage_times(lmoe_handle h, float *ms, int32_t n, int32_t *n_forwards,
                      int64_t *launches);
+
+/* ---- Expert parallelism ("Shaping Latent MoE", Figure 6: the routed experts
+ * sit between W_down and W_up, so the tokens cross between devices in the
+ * latent width l; "LatentMoE Explained", Figure 12 and the passage on the
+ * all-to-all that runs twice per expert layer).
+ *
+ * A handle created with ep_world = W > 1 and ep_rank = r holds the router,
+ * W_down, W_up and the shared experts (replicated on every rank) and the
+ * routed experts [r * N'/W, (r+1) * N'/W) only: in lmoe_load_weights,
+ * w_gate / w_upx / w_out then point at those N'/W experts ([N'/W][m][l],
+ * [N'/W][m][l], [N'/W][l][m]).  N' must be a multiple of W; bf16 dtype,
+ * bf16 expert weights, no training.  lmoe_forward and lmoe_backward return
+ * LMOE_ERR_UNSUPPORTED on such a handle; lmoe_route works.  One forward of
+ * the layer on rank r is, in order on one stream:
+ *
+ *   1. lmoe_ep_dispatch(x [T][d]) -> send rows + expert counts
+ *   2. (caller) exchange: every rank sends its rows for rank q's experts to
+ *      rank q -- counts first, then the rows (an all-to-all with splits) --
+ *      so that rank q receives, source rank by source rank, the rows for its
+ *      experts;
+ *   3. lmoe_ep_experts(received rows) -> expert outputs, same row order
+ *   4. (caller) exchange back: the outputs return to their source ranks in
+ *      the order they were sent;
+ *   5. lmoe_ep_combine(returned rows) -> y [T][d].
+ *
+ * The exchanged rows are l wide (not d): z rows go out, expert-output rows
+ * come back.  Steps 1 and 5 must use the same handle, with no other call on
+ * it in between: the routing (ids, gates, positions) and the shared experts'
+ * hidden of step 1 stay in the handle's workspace for step 5.  Step 3 uses
+ * its own workspace, so it may run between them on the same stream. */
+
+/* Step 1.  Routes x_dev [T][d] over all N' experts and writes
+ * send_rows_dev [T*K'][l] (bf16): row p is z of the token in dispatch
+ * position p (lmoe_route's perm order: experts ascending, tokens ascending
+ * within an expert), so the rows for rank q are the contiguous range of
+ * experts [q N'/W, (q+1) N'/W); and expert_counts_dev [N'] int32, the
+ * number of rows per expert.  Rows past the T*K' actually routed are not
+ * written.  x and send_rows start on 16-byte boundaries.  Errors: NULL_ARG,
+ * NOT_LOADED, TOO_MANY_TOKENS, MISALIGNED, UNSUPPORTED (not an
+ * expert-parallel handle), CUDA. */
+int lmoe_ep_dispatch(lmoe_handle h, const void *x_dev, int32_t T, void *send_rows_dev,
+                     int32_t *expert_counts_dev, void *stream);
+
+/* Step 3.  recv_rows_dev [R][l] (bf16): the rows received from every source
+ * rank s = 0..W-1 in turn, each source's rows grouped by this rank's local
+ * experts in order (exactly what step 1's send rows give after the
+ * exchange); recv_counts_dev [W][N'/W] int32 on the device: rows from source
+ * s for local expert e.  Writes out_rows_dev [R][l] (bf16), row i =
+ * E_e(row i) for the row's expert e, the latent expert l -> m -> l ("LatentMoE
+ * Explained", Figure 9), not yet gate-weighted.  R = the sum of
+ * recv_counts, at most W * max_tokens * K'.  Buffers start on 16-byte
+ * boundaries.  Errors: NULL_ARG, NOT_LOADED, TOO_MANY_TOKENS (R out of
+ * range), MISALIGNED, UNSUPPORTED, CUDA. */
+int lmoe_ep_experts(lmoe_handle h, const void *recv_rows_dev, const int32_t *recv_counts_dev,
+                    int32_t R, void *out_rows_dev, void *stream);
+
+/* Step 5.  back_rows_dev [T*K'][l] (bf16): the expert outputs returned to
+ * this rank, in the order of step 1's send rows.  Combines them with the
+ * gates of step 1 in slot order and writes y_dev [T][d] = u W_up^T + the
+ * shared experts of x (T must equal step 1's).  Buffers start on 16-byte
+ * boundaries.  Errors: NULL_ARG, NOT_LOADED, TOO_MANY_TOKENS, MISALIGNED,
+ * UNSUPPORTED, CUDA. */
+int lmoe_ep_combine(lmoe_handle h, const void *back_rows_dev, void *y_dev, int32_t T,
+                    void *stream);
 
 /* Dispatch without allocation.  The paper has no counterpart to this call:
  * it exists for callers that may not call cudaMalloc where they need the

@@ -45,6 +45,21 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
                             TileEntry *tiles2 = nullptr, int32_t *n_tiles2 = nullptr,
                             int tile_m2 = 0, int max_tiles2 = 0, bool check_ids = false);
 
+// Expert parallelism, receiving side.  recv_counts [W][NL]: rows that source
+// rank s sent for local expert e; the received rows lie source-major and,
+// within a source, expert-grouped in expert order.  Writes the M-tile tables
+// (tile_m and tile_m2 rows per tile, entries ordered by expert, then source,
+// so that tiles sharing an expert's weights run together) and their lengths.
+// Row ranges are clipped at R (the rows actually received).  W * NL <= 65536,
+// NL <= 1024.
+cudaError_t launch_ep_tiles(const int32_t *recv_counts, int W, int NL, int R, TileEntry *tiles,
+                            int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
+                            int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s);
+
+// counts[e] = offsets[e+1] - offsets[e] for e < N.
+cudaError_t launch_counts_from_offsets(const int32_t *offsets, int N, int32_t *counts,
+                                       cudaStream_t s);
+
 // dst[p][:] = src[perm[p] / K][:], rows of `row_bytes` (multiple of 16).
 cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
                                 int row_bytes, void *dst, cudaStream_t s);

@@ -43,6 +43,9 @@ struct Workspace {
   void *z = nullptr, *zp = nullptr, *H = nullptr, *O = nullptr, *ucat = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
   int32_t *status = nullptr;
+  // expert parallelism: M-tile tables of the received rows (128- and 256-row)
+  TileEntry *ep_tiles = nullptr, *ep_tiles2 = nullptr;
+  int32_t *ep_n_tiles = nullptr, *ep_n_tiles2 = nullptr;
 };
 
 // Backward workspace (handles created with training = 1), sized for Tmax.
@@ -81,6 +84,14 @@ struct lmoe_layer {
   int device = 0, num_sms = 0;
   bool loaded = false;
   int max_tiles = 0, max_tiles2 = 0;
+  // Expert parallelism: ep_world ranks share the N routed experts; this
+  // handle holds NE = N / ep_world of them (NE = N without it), experts
+  // [ep_rank * NE, (ep_rank + 1) * NE).  R_max: rows lmoe_ep_experts may
+  // receive (ep_world * Tmax * K); h_rows: rows of the H workspace.
+  int ep_world = 1, ep_rank = 0, NE = 0;
+  int ep_T = -1;  // tokens of the last lmoe_ep_dispatch (its combine must match)
+  int64_t R_max = 0, h_rows = 0;
+  int max_tiles_ep = 0, max_tiles2_ep = 0;
   // bf16 layout of the stacked x-matrix: [W_r | pad][W_down | pad][shared rows | pad]
   int n_pad = 0, l_pad = 0, sh_rows = 0, nx_rows = 0;
   int gu_rows = 0;    // B rows per expert of the expert up GEMM: 2m (SwiGLU) or m
@@ -159,7 +170,8 @@ void free_all(lmoe_layer *h) {
                   h->bw.ABs, h->bw.dAB, h->bw.dXcat, h->bw.DOT, h->bw.HT, h->bw.dABT,
                   h->bw.zpT, h->bw.dyT, h->bw.ucatT, h->bw.dXcatT, h->bw.xT, h->bw.kstart,
                   h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT, h->w_gu8,
-                  h->w_o8, h->gu_scale, h->o_scale};
+                  h->w_o8, h->gu_scale, h->o_scale, h->ws.ep_tiles, h->ws.ep_tiles2,
+                  h->ws.ep_n_tiles, h->ws.ep_n_tiles2};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
@@ -185,6 +197,16 @@ int validate(const lmoe_config *c, lmoe_layer *h) {
                                                   : c->top_k);
   if (N < 1 || K < 1 || K > N) return LMOE_ERR_INVALID_CONFIG;
   if (N > 1024) return LMOE_ERR_UNSUPPORTED;
+  const int W = c->ep_world > 1 ? c->ep_world : 1;
+  if (c->ep_world < 0 || c->ep_rank < 0 || c->ep_rank >= W) return LMOE_ERR_INVALID_CONFIG;
+  if (W > 1) {
+    if (N % W) return LMOE_ERR_INVALID_CONFIG;
+    if (c->dtype != LMOE_BF16 || c->weight_format != LMOE_WEIGHTS_BF16 || c->training)
+      return LMOE_ERR_UNSUPPORTED;
+  }
+  h->ep_world = W;
+  h->ep_rank = c->ep_rank;
+  h->NE = static_cast<int>(N / W);
   h->d = c->d;
   h->l = c->d / c->alpha;
   h->m = c->m;
@@ -201,7 +223,9 @@ int validate(const lmoe_config *c, lmoe_layer *h) {
   if (h->fp8 && (c->dtype != LMOE_BF16 || c->training)) return LMOE_ERR_UNSUPPORTED;
   h->esize = h->bf16 ? 2 : 4;
   h->ky = h->l + h->ns * h->ms;
-  if (static_cast<int64_t>(h->Tmax) * h->K > INT32_MAX / 2) return LMOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(h->Tmax) * h->K * W > INT32_MAX / 2) return LMOE_ERR_UNSUPPORTED;
+  h->R_max = W > 1 ? static_cast<int64_t>(W) * h->Tmax * h->K : 0;
+  h->h_rows = std::max(static_cast<int64_t>(h->Tmax) * h->K, h->R_max);
   if (h->bf16) {
     const int mq = h->relu2 ? 64 : 128;  // SwiGLU tiles pair 128 gate with 128 up columns
     if (h->d % 64 || h->l % 64 || h->m % mq || (h->ns > 0 && h->ms % mq) || h->N % 32)
@@ -285,7 +309,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
             dalloc(&w.n_tiles, 16) &&
             dalloc(&w.tiles2, static_cast<size_t>(h->max_tiles2) * sizeof(TileEntry)) &&
             dalloc(&w.n_tiles2, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
-            dalloc(&w.H, TK * m * es) && dalloc(&w.O, TK * l * es) &&
+            dalloc(&w.H, static_cast<size_t>(h->h_rows) * m * es) && dalloc(&w.O, TK * l * es) &&
             dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
             dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16);
   if (ok) {  // weights
@@ -298,8 +322,16 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
              dalloc(&h->w_o8, btile_rows(h->N, h->l, h->m) * 64) &&
              dalloc(&h->gu_scale, N * h->gu_rows * 4) && dalloc(&h->o_scale, N * l * 4);
       else if (ok)
-        ok = dalloc(&h->w_gu, btile_rows(h->N, h->gu_rows, h->l) * 64 * es) &&
-             dalloc(&h->w_out, btile_rows(h->N, h->l, h->m) * 64 * es);
+        ok = dalloc(&h->w_gu, btile_rows(h->NE, h->gu_rows, h->l) * 64 * es) &&
+             dalloc(&h->w_out, btile_rows(h->NE, h->l, h->m) * 64 * es);
+      if (ok && h->ep_world > 1) {
+        h->max_tiles_ep = static_cast<int>(h->R_max / kTileM + static_cast<int64_t>(h->ep_world) * h->NE + 1);
+        h->max_tiles2_ep =
+            static_cast<int>(h->R_max / (2 * kTileM) + static_cast<int64_t>(h->ep_world) * h->NE + 1);
+        ok = dalloc(&w.ep_tiles, static_cast<size_t>(h->max_tiles_ep) * sizeof(TileEntry)) &&
+             dalloc(&w.ep_tiles2, static_cast<size_t>(h->max_tiles2_ep) * sizeof(TileEntry)) &&
+             dalloc(&w.ep_n_tiles, 16) && dalloc(&w.ep_n_tiles2, 16);
+      }
     } else {
       ok = dalloc(&h->w_router, N * d * es) && dalloc(&h->w_down, l * d * es) &&
            (h->relu2 || dalloc(&h->w_gate, N * m * l * es)) &&
@@ -354,11 +386,11 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   }
   if (h->bf16) {
     rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TK), h->l, h->l, kTileM);
-    if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, static_cast<int64_t>(TK), h->m, h->m, kTileM);
+    if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, h->h_rows, h->m, h->m, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_ucat, w.ucat, h->Tmax, h->ky, h->ky, kTileM);
     if (rc == LMOE_OK &&
         (make_tmap_bf16_out(h->tm_out_z.bytes, w.z, h->Tmax, h->l, h->l) != 0 ||
-         make_tmap_bf16_out(h->tm_out_h.bytes, w.H, static_cast<int64_t>(TK), h->m, h->m) != 0 ||
+         make_tmap_bf16_out(h->tm_out_h.bytes, w.H, h->h_rows, h->m, h->m) != 0 ||
          make_tmap_bf16_out(h->tm_out_o.bytes, w.O, static_cast<int64_t>(TK), h->l, h->l) != 0))
       rc = LMOE_ERR_CUDA;
     // B operands: [tiled rows][64], one {64, 256} box per K-block tile
@@ -377,11 +409,11 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
         rc = LMOE_ERR_CUDA;
     } else {
       if (rc == LMOE_OK)
-        rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->N, h->gu_rows, h->l), 64, 64, kTileN);
+        rc = make_map(&h->tm_wgu, h->w_gu, btile_rows(h->NE, h->gu_rows, h->l), 64, 64, kTileN);
       if (rc == LMOE_OK)
-        rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN);
+        rc = make_map(&h->tm_wo, h->w_out, btile_rows(h->NE, h->l, h->m), 64, 64, kTileN);
       if (rc == LMOE_OK)
-        rc = make_map(&h->tm_wo2, h->w_out, btile_rows(h->N, h->l, h->m), 64, 64, kTileN / 2);
+        rc = make_map(&h->tm_wo2, h->w_out, btile_rows(h->NE, h->l, h->m), 64, 64, kTileN / 2);
     }
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wy, h->w_y, btile_rows(1, h->d, h->ky), 64, 64, kTileN);
@@ -472,7 +504,8 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   // bf16: assemble each B operand row-major in a temporary, then repack it
   // K-block tiled into the handle's buffer.
   void *tx = nullptr, *tgu = nullptr, *ty = nullptr;
-  const size_t bx = static_cast<size_t>(h->nx_rows) * d * es, bgu = N * 2 * m * l * es,
+  const size_t NE = h->NE;
+  const size_t bx = static_cast<size_t>(h->nx_rows) * d * es, bgu = NE * 2 * m * l * es,
                by = d * ky * es;
   if (!dalloc(&tx, bx) || (!h->relu2 && !dalloc(&tgu, bgu)) || !dalloc(&ty, by)) {
     if (tx) cudaFree(tx);
@@ -504,10 +537,10 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   // Expert gate/up: per expert, blocks of 128 gate rows then 128 up rows.
   for (size_t b = 0; !h->relu2 && b < m / 128 && e == cudaSuccess; ++b) {
     e = copy2d(off(tgu, 256 * b * l, es), 2 * m * l,
-               off(const_cast<void *>(wt->w_gate), 128 * b * l, es), m * l, 128 * l, N, es, s);
+               off(const_cast<void *>(wt->w_gate), 128 * b * l, es), m * l, 128 * l, NE, es, s);
     if (e == cudaSuccess)
       e = copy2d(off(tgu, (256 * b + 128) * l, es), 2 * m * l,
-                 off(const_cast<void *>(wt->w_upx), 128 * b * l, es), m * l, 128 * l, N, es, s);
+                 off(const_cast<void *>(wt->w_upx), 128 * b * l, es), m * l, 128 * l, NE, es, s);
   }
   using bf = __nv_bfloat16;
   if (e == cudaSuccess)
@@ -522,10 +555,10 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
                                      h->o_scale, h->w_o8, s);
   } else {
     if (e == cudaSuccess)  // expert up rows: interleaved gate/up, or the up-projection itself
-      e = launch_repack_btiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->N,
+      e = launch_repack_btiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->NE,
                                h->gu_rows, h->l, static_cast<bf *>(h->w_gu), s);
     if (e == cudaSuccess)
-      e = launch_repack_btiles(static_cast<const bf *>(wt->w_out), h->N, h->l, h->m,
+      e = launch_repack_btiles(static_cast<const bf *>(wt->w_out), h->NE, h->l, h->m,
                                static_cast<bf *>(h->w_out), s);
   }
   if (e == cudaSuccess)
@@ -596,7 +629,7 @@ static int check_call(lmoe_handle h, int32_t T) {
 // raw pre-activations there ([T][sh_rows], W_x's shared-row layout) instead
 // of the hidden.
 static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cudaStream_t s,
-                             void *shared_raw = nullptr) {
+                             void *shared_raw = nullptr, bool marks = true) {
   Workspace &w = h->ws;
   cudaError_t e = cudaSuccess;
   if (h->bf16) {
@@ -675,7 +708,7 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     }
   }
   if (e != cudaSuccess) return e;
-  if (full) mark(h, 1, s);
+  if (full && marks) mark(h, 1, s);
   // top-K' also builds the dispatch histogram (into the zeroed count matrix)
   e = cudaMemsetAsync(w.chunk_counts, 0, dispatch_count_elems(T, kDispatchChunk, h->N) * 4, s);
   if (e != cudaSuccess) return e;
@@ -683,13 +716,13 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
                   kDispatchChunk, s);
   h->launches += 1;
   if (e != cudaSuccess) return e;
-  if (full) mark(h, 2, s);
+  if (full && marks) mark(h, 2, s);
   e = launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, kDispatchChunk, true, w.offsets,
                       w.perm, w.pos, w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s,
                       w.tiles2, w.n_tiles2, 2 * kTileM, h->max_tiles2);
   h->launches += 2;
   if (e != cudaSuccess) return e;
-  if (full) mark(h, 3, s);
+  if (full && marks) mark(h, 3, s);
   return e;
 }
 
@@ -721,6 +754,99 @@ int lmoe_route(lmoe_handle h, const void *x, int32_t T, int32_t *ids, float *gat
   return cuda_err(e);
 }
 
+// bf16 expert GEMMs over grouped rows: A rows through tm_a ({64, 128} boxes;
+// tm_a32: {64, 32} boxes, E4M3 weights only), the M-tile tables (128-row
+// tiles, and 256-row tiles for the pair down GEMM), H in the workspace, and
+// the expert outputs through the store map tm_o.  pair_down: the down GEMM
+// runs on CTA pairs.  stage_gu / stage_down: profiling marks after each.
+static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
+                                    const TensorMap64 &tm_a32, const TileEntry *tiles,
+                                    const int32_t *n_tiles, const TileEntry *tiles2,
+                                    const int32_t *n_tiles2, bool pair_down, void *O,
+                                    const TensorMap64 &tm_o, cudaStream_t s, bool marks) {
+  Workspace &w = h->ws;
+  TcParams p = {};
+  p.mode = TC_EXPERT_GU;
+  p.Kdim = h->l;
+  p.n_tiles_n = (h->gu_rows + kTileN - 1) / kTileN;
+  p.relu2 = h->relu2;
+  p.n_cols2 = h->m;
+  p.tiles = tiles;
+  p.n_mtiles = n_tiles;
+  if (h->fp8) {
+    p.b_scale = h->gu_scale;
+    p.b_scale_ld = h->gu_rows;
+  }
+  p.b_rows_per_expert = h->gu_rows;
+  p.out = static_cast<__nv_bfloat16 *>(w.H);
+  p.ld_out = h->m;
+  p.status = w.status;
+  // Single-CTA tiles of 128 rows: measured at least as fast as CTA pairs for
+  // the gate/up GEMM (K = l is short, the SwiGLU epilogue is the heavier)
+  // and much faster when experts hold few tokens.
+  p.tma_out = h->fp8 ? 0 : 1;
+  cudaError_t e = launch_tc_gemm(tm_a.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s,
+                                 tm_a32.bytes, h->tm_out_h.bytes);
+  h->launches += 1;
+  if (e != cudaSuccess) return e;
+  if (marks) mark(h, 5, s);
+  TcParams pd = {};
+  pd.mode = TC_EXPERT_DOWN;
+  pd.Kdim = h->m;
+  pd.n_tiles_n = (h->l + kTileN - 1) / kTileN;
+  pd.tiles = tiles;
+  pd.n_mtiles = n_tiles;
+  pd.b_rows_per_expert = h->l;
+  pd.out = static_cast<__nv_bfloat16 *>(O);
+  pd.ld_out = h->l;
+  pd.status = w.status;
+  if (h->fp8) {
+    pd.b_scale = h->o_scale;
+    pd.b_scale_ld = h->l;
+  }
+  pd.tma_out = h->fp8 ? 0 : 1;
+  if (pair_down) {
+    pd.tiles = tiles2;
+    pd.n_mtiles = n_tiles2;
+    e = launch_tc_gemm_pair(h->tm_h.bytes, h->tm_wo2.bytes, pd, h->num_sms, s, tm_o.bytes);
+  } else {
+    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s,
+                       h->tm_h32.bytes, tm_o.bytes);
+  }
+  h->launches += 1;
+  if (e == cudaSuccess && marks) mark(h, 6, s);
+  return e;
+}
+
+// bf16: u = the gate-weighted combine of the expert outputs O (dispatch
+// order) into Ucat's first l columns, then y = [u | shared hidden] W_y^T
+// once the side stream's shared gate/up GEMM has joined.
+static cudaError_t run_combine_out_bf16(lmoe_layer *h, const void *O, void *y, int T,
+                                        cudaStream_t s, bool marks) {
+  Workspace &w = h->ws;
+  cudaError_t e = launch_combine(O, w.pos, w.gates, T, h->K, h->l, w.ucat, h->ky, true, s);
+  h->launches += 1;
+  if (e != cudaSuccess) return e;
+  if (marks) mark(h, 7, s);
+  e = cudaStreamWaitEvent(s, h->ev_join, 0);  // shared hidden ready
+  if (e != cudaSuccess) return e;
+  TcParams q = {};
+  q.mode = TC_OUT;
+  q.M = T;
+  q.Kdim = h->ky;
+  q.n_tiles_n = (h->d + kTileN - 1) / kTileN;
+  q.out = static_cast<__nv_bfloat16 *>(y);
+  q.ld_out = h->d;
+  q.status = w.status;
+  // y through TMA stores when its address allows a tensor map (16-byte aligned)
+  TensorMap64 tm_y;
+  q.tma_out = make_tmap_bf16_out(tm_y.bytes, y, T, h->d, h->d) == 0 ? 1 : 0;
+  const int tiles2 = (T + 2 * kTileM - 1) / (2 * kTileM) * q.n_tiles_n;
+  e = launch_tc_gemm_pair(h->tm_ucat.bytes, h->tm_wy2.bytes, q, tiles2, s, tm_y.bytes);
+  h->launches += 1;
+  return e;
+}
+
 static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream_t s) {
   Workspace &w = h->ws;
   const int TK = T * h->K;
@@ -732,82 +858,14 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
   mark(h, 4, s);
   if (h->bf16) {
-    TcParams p = {};
-    p.mode = TC_EXPERT_GU;
-    p.Kdim = h->l;
-    p.n_tiles_n = (h->gu_rows + kTileN - 1) / kTileN;
-    p.relu2 = h->relu2;
-    p.n_cols2 = h->m;
-    p.tiles = w.tiles;
-    p.n_mtiles = w.n_tiles;
-    if (h->fp8) {
-      p.b_scale = h->gu_scale;
-      p.b_scale_ld = h->gu_rows;
-    }
-    p.b_rows_per_expert = h->gu_rows;
-    p.out = static_cast<__nv_bfloat16 *>(w.H);
-    p.ld_out = h->m;
-    p.status = w.status;
-    // Single-CTA tiles of 128 rows: measured at least as fast as CTA pairs for
-    // the gate/up GEMM (K = l is short, the SwiGLU epilogue is the heavier)
-    // and much faster when experts hold few tokens.
-    p.tma_out = h->fp8 ? 0 : 1;
-    e = launch_tc_gemm(h->tm_zp.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s,
-                       h->tm_zp32.bytes, h->tm_out_h.bytes);
-    h->launches += 1;
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
-    mark(h, 5, s);
-    TcParams pd = {};
-    pd.mode = TC_EXPERT_DOWN;
-    pd.Kdim = h->m;
-    pd.n_tiles_n = (h->l + kTileN - 1) / kTileN;
-    pd.tiles = w.tiles;
-    pd.n_mtiles = w.n_tiles;
-    pd.b_rows_per_expert = h->l;
-    pd.out = static_cast<__nv_bfloat16 *>(w.O);
-    pd.ld_out = h->l;
-    pd.status = w.status;
-    if (h->fp8) {
-      pd.b_scale = h->o_scale;
-      pd.b_scale_ld = h->l;
-    }
-    // CTA pairs (256-row M-tiles) when experts average at least 256 rows: the
-    // long reduction (K = m) then gains from the smaller per-SM operand feed;
-    // with fewer rows the pair's half-empty tiles cost more than that.
+    // CTA pairs (256-row M-tiles) for the down GEMM when experts average at
+    // least 256 rows: the long reduction (K = m) then gains from the smaller
+    // per-SM operand feed; with fewer rows the pair's half-empty tiles cost
+    // more than that.
     const bool pair_down = !h->fp8 && static_cast<int64_t>(T) * h->K >= 256LL * h->N;
-    pd.tma_out = h->fp8 ? 0 : 1;
-    if (pair_down) {
-      pd.tiles = w.tiles2;
-      pd.n_mtiles = w.n_tiles2;
-      e = launch_tc_gemm_pair(h->tm_h.bytes, h->tm_wo2.bytes, pd, h->num_sms, s,
-                              h->tm_out_o.bytes);
-    } else {
-      e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s,
-                         h->tm_h32.bytes, h->tm_out_o.bytes);
-    }
-    h->launches += 1;
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
-    mark(h, 6, s);
-    e = launch_combine(w.O, w.pos, w.gates, T, h->K, h->l, w.ucat, h->ky, true, s);
-    h->launches += 1;
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
-    mark(h, 7, s);
-    e = cudaStreamWaitEvent(s, h->ev_join, 0);  // shared hidden ready
-    if (e != cudaSuccess) return LMOE_ERR_CUDA;
-    TcParams q = {};
-    q.mode = TC_OUT;
-    q.M = T;
-    q.Kdim = h->ky;
-    q.n_tiles_n = (h->d + kTileN - 1) / kTileN;
-    q.out = static_cast<__nv_bfloat16 *>(y);
-    q.ld_out = h->d;
-    q.status = w.status;
-    // y through TMA stores when its address allows a tensor map (16-byte aligned)
-    TensorMap64 tm_y;
-    q.tma_out = make_tmap_bf16_out(tm_y.bytes, y, T, h->d, h->d) == 0 ? 1 : 0;
-    const int tiles2 = (T + 2 * kTileM - 1) / (2 * kTileM) * q.n_tiles_n;
-    e = launch_tc_gemm_pair(h->tm_ucat.bytes, h->tm_wy2.bytes, q, tiles2, s, tm_y.bytes);
-    h->launches += 1;
+    e = run_experts_bf16(h, h->tm_zp, h->tm_zp32, w.tiles, w.n_tiles, w.tiles2, w.n_tiles2,
+                         pair_down, w.O, h->tm_out_o, s, true);
+    if (e == cudaSuccess) e = run_combine_out_bf16(h, w.O, y, T, s, true);
   } else {
     float *zpf = static_cast<float *>(w.zp);
     float *Hf = static_cast<float *>(w.H), *Of = static_cast<float *>(w.O);
@@ -841,12 +899,85 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
 int lmoe_forward(lmoe_handle h, const void *x, void *y, int32_t T, void *stream) {
   int rc = check_call(h, T);
   if (rc != LMOE_OK) return rc;
+  if (h->ep_world > 1) return LMOE_ERR_UNSUPPORTED;  // this rank holds a slice of the experts
   if (T == 0) return LMOE_OK;
   if (!x || !y) return LMOE_ERR_NULL_ARG;
   if (!aligned16(x) || !aligned16(y)) return LMOE_ERR_MISALIGNED;
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
   return forward_impl(h, x, y, T, static_cast<cudaStream_t>(stream));
+}
+
+// ---- expert parallelism (see the declarations of lmoe_ep_*)
+static int check_ep(lmoe_handle h, int32_t T) {
+  const int rc = check_call(h, T);
+  if (rc != LMOE_OK) return rc;
+  return h->ep_world > 1 ? LMOE_OK : LMOE_ERR_UNSUPPORTED;
+}
+
+int lmoe_ep_dispatch(lmoe_handle h, const void *x, int32_t T, void *send_rows,
+                     int32_t *expert_counts, void *stream) {
+  int rc = check_ep(h, T);
+  if (rc != LMOE_OK) return rc;
+  if (!expert_counts || (T > 0 && (!x || !send_rows))) return LMOE_ERR_NULL_ARG;
+  if (T > 0 && (!aligned16(x) || !aligned16(send_rows))) return LMOE_ERR_MISALIGNED;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace &w = h->ws;
+  h->ep_T = T;
+  if (T == 0) return cuda_err(cudaMemsetAsync(expert_counts, 0, h->N * sizeof(int32_t), s));
+  // routing over all N' experts, z, and the shared hidden (side stream)
+  cudaError_t e = run_route(h, x, T, true, s, nullptr, false);
+  // z rows in dispatch order: expert-grouped, hence destination-rank grouped
+  if (e == cudaSuccess)
+    e = launch_permute_rows(w.z, w.perm, h->K, T * h->K, h->l * 2, send_rows, s);
+  if (e == cudaSuccess) e = launch_counts_from_offsets(w.offsets, h->N, expert_counts, s);
+  h->launches += 2;
+  return cuda_err(e);
+}
+
+int lmoe_ep_experts(lmoe_handle h, const void *recv_rows, const int32_t *recv_counts, int32_t R,
+                    void *out_rows, void *stream) {
+  if (!h) return LMOE_ERR_NULL_ARG;
+  if (!h->loaded) return LMOE_ERR_NOT_LOADED;
+  if (h->ep_world <= 1) return LMOE_ERR_UNSUPPORTED;
+  if (R < 0 || R > h->R_max) return LMOE_ERR_TOO_MANY_TOKENS;
+  if (!recv_counts || (R > 0 && (!recv_rows || !out_rows))) return LMOE_ERR_NULL_ARG;
+  if (R > 0 && (!aligned16(recv_rows) || !aligned16(out_rows))) return LMOE_ERR_MISALIGNED;
+  if (R == 0) return LMOE_OK;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace &w = h->ws;
+  TensorMap64 tm_a, tm_o;
+  if (make_map(&tm_a, recv_rows, R, h->l, h->l, kTileM) != LMOE_OK ||
+      make_tmap_bf16_out(tm_o.bytes, out_rows, R, h->l, h->l) != 0)
+    return LMOE_ERR_CUDA;
+  // tile tables of the received rows; rows past R (counts that sum to more)
+  // are clipped, so no tile reaches past the caller's buffers
+  cudaError_t e = launch_ep_tiles(recv_counts, h->ep_world, h->NE, R, w.ep_tiles, w.ep_n_tiles,
+                                  kTileM, h->max_tiles_ep, w.ep_tiles2, w.ep_n_tiles2, 2 * kTileM,
+                                  h->max_tiles2_ep, s);
+  h->launches += 1;
+  const bool pair_down = static_cast<int64_t>(R) >= 256LL * h->NE;
+  if (e == cudaSuccess)
+    e = run_experts_bf16(h, tm_a, tm_a, w.ep_tiles, w.ep_n_tiles, w.ep_tiles2, w.ep_n_tiles2,
+                         pair_down, out_rows, tm_o, s, false);
+  return cuda_err(e);
+}
+
+int lmoe_ep_combine(lmoe_handle h, const void *back_rows, void *y, int32_t T, void *stream) {
+  int rc = check_ep(h, T);
+  if (rc != LMOE_OK) return rc;
+  if (T != h->ep_T) return LMOE_ERR_INVALID_CONFIG;  // not the dispatched batch
+  if (T == 0) return LMOE_OK;
+  if (!back_rows || !y) return LMOE_ERR_NULL_ARG;
+  if (!aligned16(back_rows) || !aligned16(y)) return LMOE_ERR_MISALIGNED;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  return cuda_err(run_combine_out_bf16(h, back_rows, y, T, static_cast<cudaStream_t>(stream),
+                                       false));
 }
 
 // ---- backward (see the declaration of lmoe_backward): fp32 mode on CUDA cores.
@@ -1161,6 +1292,7 @@ int lmoe_backward(lmoe_handle h, const void *x, const void *dy, void *dx, const 
 int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T, void *stream) {
   int rc = check_call(h, T);
   if (rc != LMOE_OK) return rc;
+  if (h->ep_world > 1) return LMOE_ERR_UNSUPPORTED;
   if (T == 0) return LMOE_OK;
   if (!x_host || !y_host) return LMOE_ERR_NULL_ARG;
   DeviceGuard g(h->device);

@@ -285,6 +285,77 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
   }
 }
 
+// ---------------------------------------------------------------- expert parallelism
+// As write_tiles, for rows [off, off + tot) of which only those below R
+// exist: a tile starting at or past R gets an empty range (row_end = row0:
+// the GEMMs store nothing for it), the others end at min(row_end, R).
+__device__ void write_tiles_clipped(TileEntry *tiles, int tstart, int max_tiles, int e, int off,
+                                    int tot, int tile_m, int R) {
+  const int mt = (tot + tile_m - 1) / tile_m;
+  for (int j = 0; j < mt; ++j) {
+    const int idx = tstart + j;
+    if (idx < max_tiles) {
+      TileEntry te;
+      te.row0 = min(off + j * tile_m, R);
+      te.row_end = min(off + tot, R);
+      te.expert = e;
+      te.pad = 0;
+      tiles[idx] = te;
+    }
+  }
+}
+
+// Receiving side of the expert-parallel exchange: one block, thread e owns
+// local expert e.  Segment (s, e) -- the rows source s sent for expert e --
+// starts at the sum of every earlier source's rows plus source s's rows for
+// experts before e.  Tiles are numbered expert by expert, sources in order
+// within an expert.
+__global__ void __launch_bounds__(1024) ep_tiles_kernel(
+    const int32_t *__restrict__ recv_counts, int W, int NL, int R, TileEntry *__restrict__ tiles,
+    int32_t *__restrict__ n_tiles, int tile_m, int max_tiles, TileEntry *__restrict__ tiles2,
+    int32_t *__restrict__ n_tiles2, int tile_m2, int max_tiles2) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  const bool mine = e < NL;
+  // count of segment (s, e): clipped to non-negative; rows past R are dropped
+  // below, so inconsistent counts cannot send a tile past the buffers
+  auto count = [&](int s) {
+    return mine ? max(0, recv_counts[static_cast<size_t>(s) * NL + e]) : 0;
+  };
+  int my_t = 0, my_t2 = 0;
+  for (int s = 0; s < W; ++s) {
+    const int c = count(s);
+    my_t += (c + tile_m - 1) / tile_m;
+    my_t2 += (c + tile_m2 - 1) / tile_m2;
+  }
+  int all_t = 0, all_t2 = 0;
+  int t_at = block_exclusive_scan(my_t, warp_sums, &all_t);
+  int t2_at = block_exclusive_scan(my_t2, warp_sums, &all_t2);
+  int base = 0;  // rows of the sources before s
+  for (int s = 0; s < W; ++s) {
+    const int c = count(s);
+    int src_rows = 0;
+    const int r0 = base + block_exclusive_scan(c, warp_sums, &src_rows);
+    if (mine) {
+      write_tiles_clipped(tiles, t_at, max_tiles, e, r0, c, tile_m, R);
+      write_tiles_clipped(tiles2, t2_at, max_tiles2, e, r0, c, tile_m2, R);
+    }
+    t_at += (c + tile_m - 1) / tile_m;
+    t2_at += (c + tile_m2 - 1) / tile_m2;
+    base += src_rows;
+  }
+  if (threadIdx.x == 0) {
+    *n_tiles = min(all_t, max_tiles);
+    *n_tiles2 = min(all_t2, max_tiles2);
+  }
+}
+
+__global__ void counts_from_offsets_kernel(const int32_t *__restrict__ offsets, int N,
+                                           int32_t *__restrict__ counts) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < N) counts[e] = offsets[e + 1] - offsets[e];
+}
+
 // ---------------------------------------------------------------- permute
 __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4 *__restrict__ src,
                                                            const int32_t *__restrict__ perm,
@@ -467,6 +538,25 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
   dispatch_scatter_kernel<<<nc, 32 * warps, smem, s>>>(ids, T, K, N, chunk_counts, nc, chunk,
                                                        offsets, perm, pos, row_expert,
                                                        check_ids ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_tiles(const int32_t *recv_counts, int W, int NL, int R, TileEntry *tiles,
+                            int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
+                            int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s) {
+  if (W < 1 || NL < 1 || NL > 1024 || static_cast<int64_t>(W) * NL > 65536 || tile_m <= 0 ||
+      tile_m2 <= 0)
+    return cudaErrorInvalidValue;
+  const int threads = (NL + 31) / 32 * 32;
+  ep_tiles_kernel<<<1, threads, 0, s>>>(recv_counts, W, NL, R, tiles, n_tiles, tile_m,
+                                        max_tiles, tiles2, n_tiles2, tile_m2, max_tiles2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_counts_from_offsets(const int32_t *offsets, int N, int32_t *counts,
+                                       cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  counts_from_offsets_kernel<<<(N + 255) / 256, 256, 0, s>>>(offsets, N, counts);
   return cudaGetLastError();
 }
 

@@ -32,7 +32,8 @@ STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
 EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
             "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
             "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc",
-            "lmoe_selftest_wait_timeout", "lmoe_backward", "lmoe_strerror", "lmoe_destroy")
+            "lmoe_selftest_wait_timeout", "lmoe_backward", "lmoe_ep_dispatch", "lmoe_ep_experts",
+            "lmoe_ep_combine", "lmoe_strerror", "lmoe_destroy")
 LMOE_NUM_STAGES = 8
 STAGE_NAMES = ("x_gemm_router_down", "topk", "dispatch", "permute_z",
                "expert_gate_up_gemm", "expert_down_gemm", "combine", "out_gemm")
@@ -42,7 +43,7 @@ class lmoe_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "d", "m", "n_experts", "top_k", "alpha", "n_shared", "m_shared", "variant", "dtype",
         "n_routed_override", "top_k_override", "has_router_bias", "max_tokens", "activation",
-        "training", "weight_format")]
+        "training", "weight_format", "ep_rank", "ep_world")]
 
 
 class lmoe_weights(C.Structure):
@@ -74,6 +75,9 @@ _lib.lmoe_stage_times.argtypes = [P, C.POINTER(C.c_float), I32, C.POINTER(I32),
 _lib.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P]
 _lib.lmoe_selftest_wait_timeout.argtypes = [P, C.c_int64, P]
 _lib.lmoe_backward.argtypes = [P, P, P, P, C.POINTER(lmoe_grads), I32, P]
+_lib.lmoe_ep_dispatch.argtypes = [P, P, I32, P, P, P]
+_lib.lmoe_ep_experts.argtypes = [P, P, P, I32, P, P]
+_lib.lmoe_ep_combine.argtypes = [P, P, P, I32, P]
 _lib.lmoe_strerror.argtypes = [C.c_int]
 _lib.lmoe_strerror.restype = C.c_char_p
 _lib.lmoe_destroy.argtypes = [P]
@@ -118,7 +122,7 @@ def lmoe_strerror(code: int) -> str:
 
 
 def config_from(cfg: LayerConfig, max_tokens: int | None = None,
-                training: bool = False) -> lmoe_config:
+                training: bool = False, ep_rank: int = 0, ep_world: int = 0) -> lmoe_config:
     return lmoe_config(
         d=cfg.d, m=cfg.m, n_experts=cfg.n_experts, top_k=cfg.top_k, alpha=cfg.alpha,
         n_shared=cfg.n_shared, m_shared=cfg.m_shared,
@@ -129,7 +133,8 @@ def config_from(cfg: LayerConfig, max_tokens: int | None = None,
         max_tokens=cfg.T if max_tokens is None else max_tokens,
         activation=LMOE_RELU2 if cfg.activation == "relu2" else LMOE_SWIGLU,
         training=int(training),
-        weight_format=LMOE_WEIGHTS_FP8 if cfg.weights == "fp8" else LMOE_WEIGHTS_BF16)
+        weight_format=LMOE_WEIGHTS_FP8 if cfg.weights == "fp8" else LMOE_WEIGHTS_BF16,
+        ep_rank=ep_rank, ep_world=ep_world)
 
 
 def lmoe_create(config: lmoe_config) -> int:
@@ -215,6 +220,21 @@ def lmoe_backward(handle: int, x, dy, dx, grads: dict, T: int, stream=None) -> N
                               _stream(stream)), "lmoe_backward")
 
 
+def lmoe_ep_dispatch(handle: int, x, T: int, send_rows, expert_counts, stream=None) -> None:
+    _check(_lib.lmoe_ep_dispatch(handle, _ptr(x), T, _ptr(send_rows), _ptr(expert_counts),
+                                 _stream(stream)), "lmoe_ep_dispatch")
+
+
+def lmoe_ep_experts(handle: int, recv_rows, recv_counts, R: int, out_rows, stream=None) -> None:
+    _check(_lib.lmoe_ep_experts(handle, _ptr(recv_rows), _ptr(recv_counts), R, _ptr(out_rows),
+                                _stream(stream)), "lmoe_ep_experts")
+
+
+def lmoe_ep_combine(handle: int, back_rows, y, T: int, stream=None) -> None:
+    _check(_lib.lmoe_ep_combine(handle, _ptr(back_rows), _ptr(y), T, _stream(stream)),
+           "lmoe_ep_combine")
+
+
 def lmoe_destroy(handle: int) -> None:
     _check(_lib.lmoe_destroy(handle), "lmoe_destroy")
 
@@ -227,9 +247,19 @@ class LatentMoELayer:
     """
 
     def __init__(self, cfg: LayerConfig, weights: dict, max_tokens: int | None = None,
-                 stream=None, training: bool = False):
+                 stream=None, training: bool = False, ep_rank: int = 0, ep_world: int = 0):
+        """ep_world > 1: an expert-parallel rank (see lmoe_ep_dispatch) holding
+        experts [ep_rank * N'/ep_world, (ep_rank + 1) * N'/ep_world) of the full
+        expert weights in ``weights``."""
         self.cfg = cfg
-        self.handle = lmoe_create(config_from(cfg, max_tokens, training))
+        self.ep_rank, self.ep_world = ep_rank, ep_world
+        self.handle = lmoe_create(config_from(cfg, max_tokens, training, ep_rank, ep_world))
+        if ep_world > 1:
+            nl = cfg.n_routed // ep_world
+            weights = dict(weights)
+            for k in ("w_gate", "w_upx", "w_out"):
+                if weights.get(k) is not None:
+                    weights[k] = weights[k][ep_rank * nl:(ep_rank + 1) * nl]
         try:
             lmoe_load_weights(self.handle, weights, stream)
         except Exception:

@@ -68,6 +68,10 @@ def _cfg(**kw):
     (dict(dtype=5), -1), (dict(max_tokens=0), -1), (dict(n_shared=1, m_shared=0), -1),
     (dict(n_routed_override=2048, top_k_override=4), -7),
     (dict(dtype=1), -7),  # bf16 tiles need d, l multiples of 64 and m multiple of 128 ...
+    # expert parallelism: N' = 16 experts over 3 ranks, a rank outside the
+    # world, a negative world, and the fp32 mode (bf16 only)
+    (dict(dtype=1, ep_world=3, ep_rank=0), -1), (dict(dtype=1, ep_world=2, ep_rank=2), -1),
+    (dict(ep_world=-1), -1), (dict(ep_world=2, ep_rank=1), -7),
 ])
 def test_create_rejects_bad_configs_on_host(lib, kw, code):
     from latent_mixture_experts_top_b200 import lmoe
@@ -89,6 +93,9 @@ def test_null_arguments(lib):
     assert lib.lmoe_load_weights(None, None, None) == -2
     assert lib.lmoe_get_dims(None, None, None, None) == -2
     assert lib.lmoe_destroy(None) == 0
+    assert lib.lmoe_ep_dispatch(None, None, 0, None, None, None) == -2
+    assert lib.lmoe_ep_experts(None, None, None, 0, None, None) == -2
+    assert lib.lmoe_ep_combine(None, None, None, 0, None) == -2
 
 
 def test_strerror_names_every_code(lib):

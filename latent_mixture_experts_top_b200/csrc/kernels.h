@@ -60,6 +60,26 @@ cudaError_t launch_ep_tiles(const int32_t *recv_counts, int W, int NL, int R, Ti
 cudaError_t launch_counts_from_offsets(const int32_t *offsets, int N, int32_t *counts,
                                        cudaStream_t s);
 
+// Routing and dispatch in two launches.  launch_route_select: top-K' with
+// the per-chunk histogram and, in the grid's last block, the scan (outputs of
+// launch_topk + the offsets and tile tables of launch_dispatch); counts holds
+// dispatch_count_elems(T, chunk, N) ints and needs no clearing; arrivals is
+// one int, zero before the first launch and left zero by each.
+// launch_scatter_permute: the stable scatter (perm, pos, row_expert) and,
+// when src is given, the row permutation dst[p] = src[perm[p] / K] (rows of
+// row_bytes, a multiple of 16), with `shares` blocks per chunk splitting the
+// copies.  Valid when fused_route_ok(N, K, chunk).
+bool fused_route_ok(int N, int K, int chunk);
+cudaError_t launch_route_select(const float *logits, int ld, const float *bias, int T, int N,
+                                int K, int32_t *ids, float *gates, int32_t *counts, int chunk,
+                                int32_t *arrivals, int32_t *offsets, TileEntry *tiles,
+                                int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
+                                int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s);
+cudaError_t launch_scatter_permute(const int32_t *ids, int T, int K, int N, const int32_t *counts,
+                                   int chunk, const int32_t *offsets, int32_t *perm, int32_t *pos,
+                                   int32_t *row_expert, const void *src, int row_bytes, void *dst,
+                                   int shares, cudaStream_t s);
+
 // dst[p][:] = src[perm[p] / K][:], rows of `row_bytes` (multiple of 16).
 cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
                                 int row_bytes, void *dst, cudaStream_t s);

@@ -43,6 +43,7 @@ struct Workspace {
   void *z = nullptr, *zp = nullptr, *H = nullptr, *O = nullptr, *ucat = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
   int32_t *status = nullptr;
+  int32_t *arrivals = nullptr;  // fused routing: the last-block counter (zero between launches)
   // expert parallelism: M-tile tables of the received rows (128- and 256-row)
   TileEntry *ep_tiles = nullptr, *ep_tiles2 = nullptr;
   int32_t *ep_n_tiles = nullptr, *ep_n_tiles2 = nullptr;
@@ -90,6 +91,10 @@ struct lmoe_layer {
   // receive (ep_world * Tmax * K); h_rows: rows of the H workspace.
   int ep_world = 1, ep_rank = 0, NE = 0;
   int ep_T = -1;  // tokens of the last lmoe_ep_dispatch (its combine must match)
+  // Routing in two launches (top-K' + histogram + scan, then scatter + the
+  // permutation of z) when the shapes allow; else four (see run_route).
+  bool fused_route = false;
+  int route_shares = 1;  // blocks per dispatch chunk that split the permutation copies
   int64_t R_max = 0, h_rows = 0;
   int max_tiles_ep = 0, max_tiles2_ep = 0;
   // bf16 layout of the stacked x-matrix: [W_r | pad][W_down | pad][shared rows | pad]
@@ -171,7 +176,7 @@ void free_all(lmoe_layer *h) {
                   h->bw.zpT, h->bw.dyT, h->bw.ucatT, h->bw.dXcatT, h->bw.xT, h->bw.kstart,
                   h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT, h->w_gu8,
                   h->w_o8, h->gu_scale, h->o_scale, h->ws.ep_tiles, h->ws.ep_tiles2,
-                  h->ws.ep_n_tiles, h->ws.ep_n_tiles2};
+                  h->ws.ep_n_tiles, h->ws.ep_n_tiles2, h->ws.arrivals};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
@@ -300,6 +305,9 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   h->sh_rows = h->relu2 ? (h->ns * h->ms + kTileN - 1) / kTileN * kTileN : 2 * h->ns * h->ms;
   h->nx_rows = h->n_pad + h->l_pad + h->sh_rows;
   h->gu_rows = h->relu2 ? h->m : 2 * h->m;
+  h->fused_route = fused_route_ok(h->N, h->K, kDispatchChunk);
+  h->route_shares = std::max(1, std::min(16, (2 * h->num_sms + dispatch_chunks(h->Tmax, kDispatchChunk) - 1) /
+                                                 dispatch_chunks(h->Tmax, kDispatchChunk)));
   Workspace &w = h->ws;
   bool ok = dalloc(&w.logits, T * N * 4) && dalloc(&w.ids, TK * 4) && dalloc(&w.gates, TK * 4) &&
             dalloc(&w.chunk_counts, dispatch_count_elems(h->Tmax, kDispatchChunk, h->N) * 4) &&
@@ -311,7 +319,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
             dalloc(&w.n_tiles2, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
             dalloc(&w.H, static_cast<size_t>(h->h_rows) * m * es) && dalloc(&w.O, TK * l * es) &&
             dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
-            dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16);
+            dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16) && dalloc(&w.arrivals, 16);
   if (ok) {  // weights
     if (h->bf16) {
       // K-block-tiled B operands (see launch_repack_btiles)
@@ -378,6 +386,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     return LMOE_ERR_OUT_OF_MEMORY;
   }
   if (cudaMemset(w.status, 0, 16) != cudaSuccess || cudaMemset(w.n_tiles, 0, 16) != cudaSuccess ||
+      cudaMemset(w.arrivals, 0, 16) != cudaSuccess ||
       cudaMemset(w.n_tiles2, 0, 16) != cudaSuccess ||
       cudaMemset(w.ucat, 0, T * h->ky * es) != cudaSuccess) {
     free_all(h);
@@ -628,8 +637,10 @@ static int check_call(lmoe_handle h, int32_t T) {
 // shared_raw (bf16 backward only): the shared experts' gate/up GEMM writes its
 // raw pre-activations there ([T][sh_rows], W_x's shared-row layout) instead
 // of the hidden.
+// permute_dst: also write the z rows in dispatch order there (full only).
 static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cudaStream_t s,
-                             void *shared_raw = nullptr, bool marks = true) {
+                             void *shared_raw = nullptr, bool marks = true,
+                             void *permute_dst = nullptr) {
   Workspace &w = h->ws;
   cudaError_t e = cudaSuccess;
   if (h->bf16) {
@@ -709,6 +720,26 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
   }
   if (e != cudaSuccess) return e;
   if (full && marks) mark(h, 1, s);
+  const int rb = h->l * static_cast<int>(h->esize);
+  if (h->fused_route) {
+    e = launch_route_select(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates,
+                            w.chunk_counts, kDispatchChunk, w.arrivals, w.offsets, w.tiles,
+                            w.n_tiles, kTileM, h->max_tiles, w.tiles2, w.n_tiles2, 2 * kTileM,
+                            h->max_tiles2, s);
+    h->launches += 1;
+    if (e != cudaSuccess) return e;
+    if (full && marks) mark(h, 2, s);
+    e = launch_scatter_permute(w.ids, T, h->K, h->N, w.chunk_counts, kDispatchChunk, w.offsets,
+                               w.perm, w.pos, w.row_expert, permute_dst ? w.z : nullptr, rb,
+                               permute_dst, h->route_shares, s);
+    h->launches += 1;
+    if (e != cudaSuccess) return e;
+    if (full && marks) {
+      mark(h, 3, s);  // the permutation ran inside the scatter: stage 3 is empty
+      mark(h, 4, s);
+    }
+    return e;
+  }
   // top-K' also builds the dispatch histogram (into the zeroed count matrix)
   e = cudaMemsetAsync(w.chunk_counts, 0, dispatch_count_elems(T, kDispatchChunk, h->N) * 4, s);
   if (e != cudaSuccess) return e;
@@ -723,6 +754,12 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
   h->launches += 2;
   if (e != cudaSuccess) return e;
   if (full && marks) mark(h, 3, s);
+  if (permute_dst) {
+    e = launch_permute_rows(w.z, w.perm, h->K, T * h->K, rb, permute_dst, s);
+    h->launches += 1;
+    if (e != cudaSuccess) return e;
+    if (full && marks) mark(h, 4, s);
+  }
   return e;
 }
 
@@ -851,12 +888,8 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   Workspace &w = h->ws;
   const int TK = T * h->K;
   mark(h, 0, s);
-  cudaError_t e = run_route(h, x, T, true, s);
+  cudaError_t e = run_route(h, x, T, true, s, nullptr, true, w.zp);
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  e = launch_permute_rows(w.z, w.perm, h->K, TK, h->l * static_cast<int>(h->esize), w.zp, s);
-  h->launches += 1;
-  if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  mark(h, 4, s);
   if (h->bf16) {
     // CTA pairs (256-row M-tiles) for the down GEMM when experts average at
     // least 256 rows: the long reduction (K = m) then gains from the smaller
@@ -928,12 +961,10 @@ int lmoe_ep_dispatch(lmoe_handle h, const void *x, int32_t T, void *send_rows,
   h->ep_T = T;
   if (T == 0) return cuda_err(cudaMemsetAsync(expert_counts, 0, h->N * sizeof(int32_t), s));
   // routing over all N' experts, z, and the shared hidden (side stream)
-  cudaError_t e = run_route(h, x, T, true, s, nullptr, false);
-  // z rows in dispatch order: expert-grouped, hence destination-rank grouped
-  if (e == cudaSuccess)
-    e = launch_permute_rows(w.z, w.perm, h->K, T * h->K, h->l * 2, send_rows, s);
+  // (z rows in dispatch order: expert-grouped, hence destination-rank grouped)
+  cudaError_t e = run_route(h, x, T, true, s, nullptr, false, send_rows);
   if (e == cudaSuccess) e = launch_counts_from_offsets(w.offsets, h->N, expert_counts, s);
-  h->launches += 2;
+  h->launches += 1;
   return cuda_err(e);
 }
 

@@ -36,18 +36,15 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 // and removes exactly that entry.  Gates: g_k = e^{s_k - s_0} /
 // sum_j e^{s_j - s_0}, which equals softmax(s) at the selected experts
 // renormalised to sum to one (the softmax denominator cancels).
-// If `counts` is given ([N][n_chunks], zeroed), the kernel also builds the
-// per-chunk expert histogram of the dispatch (chunk = `chunk` tokens).
+// select_token: one token's selection by the calling warp.  The chosen
+// expert of each slot is counted in hist[e] (shared memory) when hist is
+// given, else in gcount[e * gstride] (global) when gcount is given.
 template <int VPL>
-__global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int ld,
-                                                   const float *__restrict__ bias, int T, int N,
-                                                   int K, int32_t *__restrict__ ids,
-                                                   float *__restrict__ gates,
-                                                   int32_t *__restrict__ counts, int n_chunks,
-                                                   int chunk) {
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+__device__ __forceinline__ void select_token(const float *__restrict__ logits, int ld,
+                                             const float *__restrict__ bias, int N, int K, int t,
+                                             int32_t *__restrict__ ids, float *__restrict__ gates,
+                                             int *hist, int32_t *gcount, int gstride) {
   const int lane = threadIdx.x & 31;
-  if (t >= T) return;
   const float *row = logits + static_cast<size_t>(t) * ld;
   uint32_t key[VPL];
 #pragma unroll
@@ -57,7 +54,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
   }
   int32_t *ids_row = ids + static_cast<size_t>(t) * K;
   float *g_row = gates + static_cast<size_t>(t) * K;
-  int32_t *my_counts = counts ? counts + t / chunk : nullptr;
   float s0 = 0.0f;
   for (int k = 0; k < K; ++k) {
     uint32_t m = key[0];
@@ -77,7 +73,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
     if ((k & 31) == lane) {  // the same lane re-reads this slot below
       ids_row[k] = static_cast<int32_t>(e);
       g_row[k] = v;
-      if (my_counts) atomicAdd(my_counts + static_cast<size_t>(e) * ((n_chunks + 3) & ~3), 1);
+      if (hist) atomicAdd(hist + e, 1);
+      else if (gcount) atomicAdd(gcount + static_cast<size_t>(e) * gstride, 1);
     }
   }
   float sum = 0.0f;
@@ -85,6 +82,22 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
   for (int k = lane; k < K; k += 32) g_row[k] = expf(g_row[k] - s0) / sum;
+}
+
+// topk_kernel: one warp per token.  If `counts` is given ([N][n_chunks],
+// zeroed), it also builds the per-chunk expert histogram of the dispatch
+// (chunk = `chunk` tokens).
+template <int VPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int ld,
+                                                   const float *__restrict__ bias, int T, int N,
+                                                   int K, int32_t *__restrict__ ids,
+                                                   float *__restrict__ gates,
+                                                   int32_t *__restrict__ counts, int n_chunks,
+                                                   int chunk) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  select_token<VPL>(logits, ld, bias, N, K, t, ids, gates, nullptr,
+                    counts ? counts + t / chunk : nullptr, (n_chunks + 3) & ~3);
 }
 
 // ---------------------------------------------------------------- dispatch
@@ -160,7 +173,7 @@ __device__ int scan_expert_row(int32_t *counts, int e, int n_chunks) {
   for (int v0 = 0; v0 < nv; v0 += 8) {
     int4 q[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) q[j] = v0 + j < nv ? row[v0 + j] : make_int4(0, 0, 0, 0);
+    for (int j = 0; j < 8; ++j) q[j] = v0 + j < nv ? __ldcg(row + v0 + j) : make_int4(0, 0, 0, 0);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (v0 + j >= nv) break;
@@ -194,11 +207,12 @@ __device__ void write_tiles(TileEntry *tiles, int tstart, int max_tiles, int e, 
   }
 }
 
-__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
-    int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
-    TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
-    TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2, int tile_m2,
-    int max_tiles2) {
+// Phase 2 body, run by one block of kScanThreads threads.
+__device__ void scan_and_tables(int32_t *__restrict__ counts, int n_chunks, int N,
+                                int32_t *__restrict__ offsets, TileEntry *__restrict__ tiles,
+                                int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+                                TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2,
+                                int tile_m2, int max_tiles2) {
   __shared__ int warp_sums[32];
   const int e0 = threadIdx.x * kScanPerThread;  // experts e0 .. e0+3
   int tot[kScanPerThread], mt[kScanPerThread], mt2[kScanPerThread];
@@ -233,6 +247,115 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
     offsets[N] = all;
     *n_tiles = min(all_tiles, max_tiles);
     if (tiles2) *n_tiles2 = min(all_tiles2, max_tiles2);
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
+    int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
+    TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+    TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2, int tile_m2,
+    int max_tiles2) {
+  scan_and_tables(counts, n_chunks, N, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
+                  n_tiles2, tile_m2, max_tiles2);
+}
+
+// ---------------------------------------------------------------- fused routing
+// Top-K', dispatch histogram and scan in one launch.  Block c takes the
+// chunk of `chunk` tokens starting at c * chunk; its warps select the tokens
+// in turn (select_token) and count the chosen experts in shared memory, which
+// becomes column c of the count matrix (every entry written: no clearing
+// needed).  The block that arrives last on the arrival counter (after a
+// fence, so it sees every column) runs the scan of phase 2 and resets the
+// counter to zero for the next launch.
+template <int VPL>
+__global__ void __launch_bounds__(256) route_select_kernel(
+    const float *__restrict__ logits, int ld, const float *__restrict__ bias, int T, int N, int K,
+    int32_t *__restrict__ ids, float *__restrict__ gates, int32_t *__restrict__ counts,
+    int n_chunks, int chunk, int32_t *__restrict__ arrivals, int32_t *__restrict__ offsets,
+    TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+    TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2, int tile_m2,
+    int max_tiles2) {
+  __shared__ int hist[1024];
+  __shared__ int is_last;
+  const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * chunk, t1 = min(T, t0 + chunk);
+  for (int t = t0 + warp; t < t1; t += nwarps)
+    select_token<VPL>(logits, ld, bias, N, K, t, ids, gates, hist, nullptr, 0);
+  __syncthreads();
+  const int ncp = (n_chunks + 3) & ~3;
+  for (int e = threadIdx.x; e < N; e += blockDim.x)
+    counts[static_cast<size_t>(e) * ncp + blockIdx.x] = hist[e];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(arrivals, 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  scan_and_tables(counts, n_chunks, N, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
+                  n_tiles2, tile_m2, max_tiles2);
+  if (threadIdx.x == 0) *arrivals = 0;
+}
+
+// Stable scatter and row permutation in one launch.  Block (c, share) with
+// c = blockIdx.x / S: chunk c's first chunk/32 warps place its (token, slot)
+// pairs exactly as dispatch_scatter_kernel does (share 0 also writes perm,
+// pos and row_expert); then every warp of the block copies the source rows of
+// the share's pairs (pair i of the chunk with i % S == share) to their
+// permuted rows, 16 bytes per lane.  src == nullptr: positions only.
+__global__ void __launch_bounds__(256) scatter_permute_kernel(
+    const int32_t *__restrict__ ids, int T, int K, int N, const int32_t *__restrict__ counts,
+    int n_chunks, int chunk, const int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+    int32_t *__restrict__ pos, int32_t *__restrict__ row_expert, const uint4 *__restrict__ src,
+    int vecs_per_row, uint4 *__restrict__ dst, int S) {
+  extern __shared__ uint32_t sm[];
+  const int W = chunk >> 5;
+  uint32_t *mask = sm;                                            // [W][N]
+  int32_t *wbase = reinterpret_cast<int32_t *>(sm + W * N);      // [W][N]
+  int32_t *ppos = reinterpret_cast<int32_t *>(sm + 2 * W * N);   // [chunk][K]
+  const int c = blockIdx.x / S, share = blockIdx.x - c * S;
+  for (int i = threadIdx.x; i < W * N; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = c * chunk + threadIdx.x;
+  const bool tok = threadIdx.x < chunk && t < T;
+  const int32_t *my_ids = ids + static_cast<size_t>(t) * K;
+  if (tok)
+    for (int k = 0; k < K; ++k) atomicOr(&mask[w * N + my_ids[k]], 1u << lane);
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int run = 0;
+    for (int ww = 0; ww < W; ++ww) {
+      wbase[ww * N + e] = run;
+      run += __popc(mask[ww * N + e]);
+    }
+  }
+  __syncthreads();
+  if (tok) {
+    const uint32_t lt = (1u << lane) - 1u;
+    const int ncp = (n_chunks + 3) & ~3;
+    for (int k = 0; k < K; ++k) {
+      const int e = my_ids[k];
+      const int p = offsets[e] + counts[static_cast<size_t>(e) * ncp + c] + wbase[w * N + e] +
+                    __popc(mask[w * N + e] & lt);
+      ppos[threadIdx.x * K + k] = p;
+      if (share == 0) {
+        const int flat = t * K + k;
+        perm[p] = flat;
+        pos[flat] = p;
+        row_expert[p] = e;
+      }
+    }
+  }
+  if (!src) return;
+  __syncthreads();
+  const int npairs = min(chunk, T - c * chunk) * K;
+  const int nwarps = blockDim.x >> 5;
+  for (int i = share + S * w; i < npairs; i += S * nwarps) {
+    const uint4 *sr = src + static_cast<size_t>(c * chunk + i / K) * vecs_per_row;
+    uint4 *dr = dst + static_cast<size_t>(ppos[i]) * vecs_per_row;
+    for (int v = lane; v < vecs_per_row; v += 32) dr[v] = sr[v];
   }
 }
 
@@ -557,6 +680,52 @@ cudaError_t launch_counts_from_offsets(const int32_t *offsets, int N, int32_t *c
                                        cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   counts_from_offsets_kernel<<<(N + 255) / 256, 256, 0, s>>>(offsets, N, counts);
+  return cudaGetLastError();
+}
+
+bool fused_route_ok(int N, int K, int chunk) {
+  return N <= 1024 && chunk % 32 == 0 && chunk >= 32 && chunk <= 256 && chunk * K <= 4096;
+}
+
+cudaError_t launch_route_select(const float *logits, int ld, const float *bias, int T, int N,
+                                int K, int32_t *ids, float *gates, int32_t *counts, int chunk,
+                                int32_t *arrivals, int32_t *offsets, TileEntry *tiles,
+                                int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
+                                int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  if (!fused_route_ok(N, K, chunk) || !tiles2 || !n_tiles2 || tile_m2 <= 0)
+    return cudaErrorInvalidValue;
+  const int nc = dispatch_chunks(T, chunk);
+  const int vpl = (N + 31) / 32;
+#define LMOE_ROUTE(V)                                                                          \
+  route_select_kernel<V><<<nc, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates, counts, nc, \
+                                            chunk, arrivals, offsets, tiles, n_tiles, tile_m,  \
+                                            max_tiles, tiles2, n_tiles2, tile_m2, max_tiles2)
+  if (vpl <= 1) LMOE_ROUTE(1);
+  else if (vpl <= 2) LMOE_ROUTE(2);
+  else if (vpl <= 4) LMOE_ROUTE(4);
+  else if (vpl <= 8) LMOE_ROUTE(8);
+  else if (vpl <= 16) LMOE_ROUTE(16);
+  else LMOE_ROUTE(32);
+#undef LMOE_ROUTE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_permute(const int32_t *ids, int T, int K, int N, const int32_t *counts,
+                                   int chunk, const int32_t *offsets, int32_t *perm, int32_t *pos,
+                                   int32_t *row_expert, const void *src, int row_bytes, void *dst,
+                                   int shares, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  if (!fused_route_ok(N, K, chunk) || shares < 1) return cudaErrorInvalidValue;
+  if (src && (row_bytes % 16 || !dst)) return cudaErrorInvalidValue;
+  const int nc = dispatch_chunks(T, chunk);
+  const int W = chunk / 32;
+  const size_t smem = (2 * static_cast<size_t>(W) * N + static_cast<size_t>(chunk) * K) * 4;
+  const int S = src ? shares : 1;
+  scatter_permute_kernel<<<nc * S, 256, smem, s>>>(ids, T, K, N, counts, nc, chunk, offsets, perm,
+                                                   pos, row_expert,
+                                                   static_cast<const uint4 *>(src),
+                                                   row_bytes / 16, static_cast<uint4 *>(dst), S);
   return cudaGetLastError();
 }
 

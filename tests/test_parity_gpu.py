@@ -114,6 +114,22 @@ def test_parity_pair_down_gemm_all_tokens():
     _check_layer(MID_PAIR, n_sample=10 ** 9)
 
 
+# K' = 72 > 64: routing takes the four-launch path (top-K', histogram scan,
+# scatter, then the permutation) instead of the fused two-launch one.
+WIDE_K_F32 = configs.LayerConfig("wide_k_f32_T64_d256_l128_N128_K72", T=64, d=256, m=256,
+                                 n_experts=64, top_k=36, alpha=2, n_shared=1, m_shared=256,
+                                 variant="acc", dtype="f32")
+WIDE_K_BF16 = configs.LayerConfig("wide_k_bf16_T300_d256_l128_N128_K72", T=300, d=256, m=256,
+                                  n_experts=64, top_k=36, alpha=2, n_shared=1, m_shared=256,
+                                  variant="acc")
+
+
+@pytest.mark.parametrize("cfg", [WIDE_K_F32, WIDE_K_BF16], ids=["f32", "bf16"])
+def test_parity_wide_k_four_launch_routing(cfg):
+    assert cfg.k_active == 72
+    _check_layer(cfg, n_sample=10 ** 9)
+
+
 def test_parity_relu2_tiny_f32_all_tokens():
     _check_layer(configs.TINY_RELU2_F32, n_sample=10 ** 9)
 

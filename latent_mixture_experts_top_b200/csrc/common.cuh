@@ -21,6 +21,35 @@ enum : int {
 // status instead of hanging the GPU.  Healthy waits last microseconds.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of its stream is still
+// running; griddep_wait blocks until that kernel has completed and its
+// memory is visible (it returns at once in a kernel launched without it), so
+// every kernel calls it before its first global-memory access.
+// griddep_launch_dependents lets the next kernel be scheduled early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
+// Host: launches `kernel` on `s`, with programmatic stream serialization
+// when pdl is set (see griddep_wait).
+template <typename... Params, typename... Args>
+inline cudaError_t launch_ex(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t s, bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

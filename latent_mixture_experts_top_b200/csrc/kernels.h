@@ -74,11 +74,12 @@ cudaError_t launch_route_select(const float *logits, int ld, const float *bias, 
                                 int K, int32_t *ids, float *gates, int32_t *counts, int chunk,
                                 int32_t *arrivals, int32_t *offsets, TileEntry *tiles,
                                 int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
-                                int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s);
+                                int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s,
+                                bool pdl = false);
 cudaError_t launch_scatter_permute(const int32_t *ids, int T, int K, int N, const int32_t *counts,
                                    int chunk, const int32_t *offsets, int32_t *perm, int32_t *pos,
                                    int32_t *row_expert, const void *src, int row_bytes, void *dst,
-                                   int shares, cudaStream_t s);
+                                   int shares, cudaStream_t s, bool pdl = false);
 
 // dst[p][:] = src[perm[p] / K][:], rows of `row_bytes` (multiple of 16).
 cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
@@ -87,7 +88,8 @@ cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int
 // u[t][0:l] (row stride ldu) = sum_k gates[t][k] * O[pos[t*K+k]][0:l] in slot
 // order, fp32 accumulation; element type bf16 (is_bf16) or f32.
 cudaError_t launch_combine(const void *O, const int32_t *pos, const float *gates, int T, int K,
-                           int l, void *u, int ldu, bool is_bf16, cudaStream_t s);
+                           int l, void *u, int ldu, bool is_bf16, cudaStream_t s,
+                           bool pdl = false);
 
 // ---- fp32 CUDA-core path (simt_kernels.cu)
 cudaError_t simt_linear(const float *A, int lda, const float *B, int ldb, float *C, int ldc,
@@ -172,6 +174,11 @@ struct TcParams {
   // the launch's output tensor map (launch_tc_gemm's tmapOut); other warps
   // store directly.
   int tma_out;
+  // Launch with programmatic stream serialization (the kernel may start while
+  // the previous kernel of the stream drains; it waits for it before touching
+  // global memory).  Only for a launch that directly follows another kernel
+  // on the same stream.
+  int pdl;
   int32_t *status;
 };
 

@@ -722,16 +722,19 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
   if (full && marks) mark(h, 1, s);
   const int rb = h->l * static_cast<int>(h->esize);
   if (h->fused_route) {
+    // programmatic launches: each follows the previous kernel of the stream
+    // (bf16: the router GEMM; fp32: the CUDA-core router) and waits for it on
+    // the device before touching memory
     e = launch_route_select(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates,
                             w.chunk_counts, kDispatchChunk, w.arrivals, w.offsets, w.tiles,
                             w.n_tiles, kTileM, h->max_tiles, w.tiles2, w.n_tiles2, 2 * kTileM,
-                            h->max_tiles2, s);
+                            h->max_tiles2, s, true);
     h->launches += 1;
     if (e != cudaSuccess) return e;
     if (full && marks) mark(h, 2, s);
     e = launch_scatter_permute(w.ids, T, h->K, h->N, w.chunk_counts, kDispatchChunk, w.offsets,
                                w.perm, w.pos, w.row_expert, permute_dst ? w.z : nullptr, rb,
-                               permute_dst, h->route_shares, s);
+                               permute_dst, h->route_shares, s, true);
     h->launches += 1;
     if (e != cudaSuccess) return e;
     if (full && marks) {
@@ -796,11 +799,14 @@ int lmoe_route(lmoe_handle h, const void *x, int32_t T, int32_t *ids, float *gat
 // tiles, and 256-row tiles for the pair down GEMM), H in the workspace, and
 // the expert outputs through the store map tm_o.  pair_down: the down GEMM
 // runs on CTA pairs.  stage_gu / stage_down: profiling marks after each.
+// pdl: the gate/up launch directly follows another kernel on s (the down
+// GEMM always follows the gate/up GEMM).
 static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
                                     const TensorMap64 &tm_a32, const TileEntry *tiles,
                                     const int32_t *n_tiles, const TileEntry *tiles2,
                                     const int32_t *n_tiles2, bool pair_down, void *O,
-                                    const TensorMap64 &tm_o, cudaStream_t s, bool marks) {
+                                    const TensorMap64 &tm_o, cudaStream_t s, bool marks,
+                                    bool pdl) {
   Workspace &w = h->ws;
   TcParams p = {};
   p.mode = TC_EXPERT_GU;
@@ -822,6 +828,7 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
   // the gate/up GEMM (K = l is short, the SwiGLU epilogue is the heavier)
   // and much faster when experts hold few tokens.
   p.tma_out = h->fp8 ? 0 : 1;
+  p.pdl = pdl && !marks ? 1 : 0;
   cudaError_t e = launch_tc_gemm(tm_a.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s,
                                  tm_a32.bytes, h->tm_out_h.bytes);
   h->launches += 1;
@@ -842,6 +849,7 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
     pd.b_scale_ld = h->l;
   }
   pd.tma_out = h->fp8 ? 0 : 1;
+  pd.pdl = marks ? 0 : 1;
   if (pair_down) {
     pd.tiles = tiles2;
     pd.n_mtiles = n_tiles2;
@@ -858,10 +866,12 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
 // bf16: u = the gate-weighted combine of the expert outputs O (dispatch
 // order) into Ucat's first l columns, then y = [u | shared hidden] W_y^T
 // once the side stream's shared gate/up GEMM has joined.
+// pdl: the combine directly follows another kernel on s.
 static cudaError_t run_combine_out_bf16(lmoe_layer *h, const void *O, void *y, int T,
-                                        cudaStream_t s, bool marks) {
+                                        cudaStream_t s, bool marks, bool pdl) {
   Workspace &w = h->ws;
-  cudaError_t e = launch_combine(O, w.pos, w.gates, T, h->K, h->l, w.ucat, h->ky, true, s);
+  cudaError_t e =
+      launch_combine(O, w.pos, w.gates, T, h->K, h->l, w.ucat, h->ky, true, s, pdl && !marks);
   h->launches += 1;
   if (e != cudaSuccess) return e;
   if (marks) mark(h, 7, s);
@@ -896,9 +906,10 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     // per-SM operand feed; with fewer rows the pair's half-empty tiles cost
     // more than that.
     const bool pair_down = !h->fp8 && static_cast<int64_t>(T) * h->K >= 256LL * h->N;
+    const bool marks = h->prof_slots > 0;
     e = run_experts_bf16(h, h->tm_zp, h->tm_zp32, w.tiles, w.n_tiles, w.tiles2, w.n_tiles2,
-                         pair_down, w.O, h->tm_out_o, s, true);
-    if (e == cudaSuccess) e = run_combine_out_bf16(h, w.O, y, T, s, true);
+                         pair_down, w.O, h->tm_out_o, s, marks, true);
+    if (e == cudaSuccess) e = run_combine_out_bf16(h, w.O, y, T, s, marks, true);
   } else {
     float *zpf = static_cast<float *>(w.zp);
     float *Hf = static_cast<float *>(w.H), *Of = static_cast<float *>(w.O);
@@ -994,7 +1005,7 @@ int lmoe_ep_experts(lmoe_handle h, const void *recv_rows, const int32_t *recv_co
   const bool pair_down = static_cast<int64_t>(R) >= 256LL * h->NE;
   if (e == cudaSuccess)
     e = run_experts_bf16(h, tm_a, tm_a, w.ep_tiles, w.ep_n_tiles, w.ep_tiles2, w.ep_n_tiles2,
-                         pair_down, out_rows, tm_o, s, false);
+                         pair_down, out_rows, tm_o, s, false, true);
   return cuda_err(e);
 }
 
@@ -1008,7 +1019,7 @@ int lmoe_ep_combine(lmoe_handle h, const void *back_rows, void *y, int32_t T, vo
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
   return cuda_err(run_combine_out_bf16(h, back_rows, y, T, static_cast<cudaStream_t>(stream),
-                                       false));
+                                       false, false));
 }
 
 // ---- backward (see the declaration of lmoe_backward): fp32 mode on CUDA cores.

@@ -279,6 +279,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(
   __shared__ int is_last;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
+  griddep_wait();
   __syncthreads();
   const int t0 = blockIdx.x * chunk, t1 = min(T, t0 + chunk);
   for (int t = t0 + warp; t < t1; t += nwarps)
@@ -316,6 +317,7 @@ __global__ void __launch_bounds__(256) scatter_permute_kernel(
   int32_t *ppos = reinterpret_cast<int32_t *>(sm + 2 * W * N);   // [chunk][K]
   const int c = blockIdx.x / S, share = blockIdx.x - c * S;
   for (int i = threadIdx.x; i < W * N; i += blockDim.x) mask[i] = 0u;
+  griddep_wait();
   __syncthreads();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = c * chunk + threadIdx.x;
@@ -544,6 +546,7 @@ __global__ void __launch_bounds__(256, 4) combine_kernel(const Tio *__restrict__
   constexpr int V = 16 / sizeof(Tio);
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  griddep_wait();
   if (t >= T) return;
   const int nvec = l / V;
   for (int vi = lane; vi < nvec; vi += 32) {
@@ -691,16 +694,18 @@ cudaError_t launch_route_select(const float *logits, int ld, const float *bias, 
                                 int K, int32_t *ids, float *gates, int32_t *counts, int chunk,
                                 int32_t *arrivals, int32_t *offsets, TileEntry *tiles,
                                 int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
-                                int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s) {
+                                int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s,
+                                bool pdl) {
   if (T <= 0) return cudaSuccess;
   if (!fused_route_ok(N, K, chunk) || !tiles2 || !n_tiles2 || tile_m2 <= 0)
     return cudaErrorInvalidValue;
   const int nc = dispatch_chunks(T, chunk);
   const int vpl = (N + 31) / 32;
-#define LMOE_ROUTE(V)                                                                          \
-  route_select_kernel<V><<<nc, 256, 0, s>>>(logits, ld, bias, T, N, K, ids, gates, counts, nc, \
-                                            chunk, arrivals, offsets, tiles, n_tiles, tile_m,  \
-                                            max_tiles, tiles2, n_tiles2, tile_m2, max_tiles2)
+  cudaError_t e;
+#define LMOE_ROUTE(V)                                                                            \
+  e = launch_ex(route_select_kernel<V>, dim3(nc), dim3(256), 0, s, pdl, logits, ld, bias, T, N, \
+                K, ids, gates, counts, nc, chunk, arrivals, offsets, tiles, n_tiles, tile_m,     \
+                max_tiles, tiles2, n_tiles2, tile_m2, max_tiles2)
   if (vpl <= 1) LMOE_ROUTE(1);
   else if (vpl <= 2) LMOE_ROUTE(2);
   else if (vpl <= 4) LMOE_ROUTE(4);
@@ -708,13 +713,13 @@ cudaError_t launch_route_select(const float *logits, int ld, const float *bias, 
   else if (vpl <= 16) LMOE_ROUTE(16);
   else LMOE_ROUTE(32);
 #undef LMOE_ROUTE
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_scatter_permute(const int32_t *ids, int T, int K, int N, const int32_t *counts,
                                    int chunk, const int32_t *offsets, int32_t *perm, int32_t *pos,
                                    int32_t *row_expert, const void *src, int row_bytes, void *dst,
-                                   int shares, cudaStream_t s) {
+                                   int shares, cudaStream_t s, bool pdl) {
   if (T <= 0) return cudaSuccess;
   if (!fused_route_ok(N, K, chunk) || shares < 1) return cudaErrorInvalidValue;
   if (src && (row_bytes % 16 || !dst)) return cudaErrorInvalidValue;
@@ -722,11 +727,11 @@ cudaError_t launch_scatter_permute(const int32_t *ids, int T, int K, int N, cons
   const int W = chunk / 32;
   const size_t smem = (2 * static_cast<size_t>(W) * N + static_cast<size_t>(chunk) * K) * 4;
   const int S = src ? shares : 1;
-  scatter_permute_kernel<<<nc * S, 256, smem, s>>>(ids, T, K, N, counts, nc, chunk, offsets, perm,
-                                                   pos, row_expert,
-                                                   static_cast<const uint4 *>(src),
-                                                   row_bytes / 16, static_cast<uint4 *>(dst), S);
-  return cudaGetLastError();
+  const cudaError_t e = launch_ex(scatter_permute_kernel, dim3(nc * S), dim3(256), smem, s, pdl,
+                                  ids, T, K, N, counts, nc, chunk, offsets, perm, pos, row_expert,
+                                  static_cast<const uint4 *>(src), row_bytes / 16,
+                                  static_cast<uint4 *>(dst), S);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int rows,
@@ -740,18 +745,21 @@ cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int
 }
 
 cudaError_t launch_combine(const void *O, const int32_t *pos, const float *gates, int T, int K,
-                           int l, void *u, int ldu, bool is_bf16, cudaStream_t s) {
+                           int l, void *u, int ldu, bool is_bf16, cudaStream_t s, bool pdl) {
   if (T <= 0) return cudaSuccess;
   const int blocks = (T + 7) / 8;
   if (is_bf16) {
     if (l % 8 || ldu % 8) return cudaErrorInvalidValue;
-    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(O), pos, gates, T, K, l,
-        static_cast<__nv_bfloat16 *>(u), ldu);
+    const cudaError_t e = launch_ex(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, s,
+                                    pdl, static_cast<const __nv_bfloat16 *>(O), pos, gates, T, K,
+                                    l, static_cast<__nv_bfloat16 *>(u), ldu);
+    if (e != cudaSuccess) return e;
   } else {
     if (l % 4 || ldu % 4) return cudaErrorInvalidValue;
-    combine_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float *>(O), pos, gates, T, K,
-                                                 l, static_cast<float *>(u), ldu);
+    const cudaError_t e = launch_ex(combine_kernel<float>, dim3(blocks), dim3(256), 0, s, pdl,
+                                    static_cast<const float *>(O), pos, gates, T, K, l,
+                                    static_cast<float *>(u), ldu);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

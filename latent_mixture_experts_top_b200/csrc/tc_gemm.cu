@@ -683,8 +683,6 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
 
   const bool grouped = (p.mode == TC_EXPERT_GU || p.mode == TC_EXPERT_DOWN);
   const int m_tiles = grouped ? 0 : (p.M + TM - 1) / TM;
-  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n
-                            : m_tiles * p.n_tiles_n * (p.mode == TC_WGRAD ? p.groups : 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -717,6 +715,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+  // everything above touched only shared memory, TMEM and the parameters
+  griddep_wait();
+  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n
+                            : m_tiles * p.n_tiles_n * (p.mode == TC_WGRAD ? p.groups : 1);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -798,6 +800,8 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
         if (!drain_wait(&ctl->drain, 0)) record_failure(p, ctl, DEV_TIMEOUT_DRAIN);
       }
     }
+    // every MMA is issued: the next kernel of the stream may be scheduled
+    if (lane == 0) griddep_launch_dependents();
   } else if (kFp8 && warp >= 2 + Cfg<kFp8>::EPI_WARPS) {
     // ------------------------------------------------------------ converters
     const int ctid = threadIdx.x - 32 * (2 + Cfg<kFp8>::EPI_WARPS);
@@ -984,7 +988,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<false>::NUM_THRE
 
   const bool grouped = (p.mode == TC_EXPERT_GU || p.mode == TC_EXPERT_DOWN);
   const int m_tiles2 = grouped ? 0 : (p.M + 2 * TM - 1) / (2 * TM);
-  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles2 * p.n_tiles_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < P_STAGES; ++s) {
@@ -1012,6 +1015,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<false>::NUM_THRE
   ptx::cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
   ptx::tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+  // everything above touched only shared memory, TMEM and the parameters
+  griddep_wait();
+  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles2 * p.n_tiles_n;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1092,6 +1098,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<false>::NUM_THRE
         if (!drain_wait(&ctl->drain, 0)) record_failure_pair(p, ctl, peer, DEV_TIMEOUT_DRAIN);
       }
     }
+    // every MMA of the pair is issued: the next kernel may be scheduled
+    if (lane == 0) griddep_launch_dependents();
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
@@ -1271,16 +1279,18 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   memcpy(&b, tmapB, sizeof(b));
   memcpy(&a32, fp8 ? tmapA32 : tmapA, sizeof(a32));
   memcpy(&o, p.tma_out ? tmapOut : tmapA, sizeof(o));
+  const bool pdl = p.pdl != 0;
+  cudaError_t e;
   if (fp8)
-    tc_gemm_kernel<false, true>
-        <<<grid, Cfg<true>::NUM_THREADS, smem_bytes<true>(false), s>>>(a, b, a32, o, p);
+    e = launch_ex(tc_gemm_kernel<false, true>, dim3(grid), dim3(Cfg<true>::NUM_THREADS),
+                  smem_bytes<true>(false), s, pdl, a, b, a32, o, p);
   else if (bwd)
-    tc_gemm_kernel<true, false>
-        <<<grid, Cfg<false>::NUM_THREADS, smem_bytes<false>(false), s>>>(a, b, a32, o, p);
+    e = launch_ex(tc_gemm_kernel<true, false>, dim3(grid), dim3(Cfg<false>::NUM_THREADS),
+                  smem_bytes<false>(false), s, pdl, a, b, a32, o, p);
   else
-    tc_gemm_kernel<false, false><<<grid, Cfg<false>::NUM_THREADS,
-                                   smem_bytes<false>(p.tma_out != 0), s>>>(a, b, a32, o, p);
-  return cudaGetLastError();
+    e = launch_ex(tc_gemm_kernel<false, false>, dim3(grid), dim3(Cfg<false>::NUM_THREADS),
+                  smem_bytes<false>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcParams &p,
@@ -1314,9 +1324,10 @@ cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcP
   memcpy(&a, tmapA, sizeof(a));
   memcpy(&b, tmapB2, sizeof(b));
   memcpy(&o, p.tma_out ? tmapOut : tmapA, sizeof(o));
-  tc_pair_kernel<<<2 * pairs, Cfg<false>::NUM_THREADS, pair_smem_bytes(p.tma_out != 0), s>>>(a, b, o,
-                                                                                           p);
-  return cudaGetLastError();
+  const cudaError_t e =
+      launch_ex(tc_pair_kernel, dim3(2 * pairs), dim3(Cfg<false>::NUM_THREADS),
+                pair_smem_bytes(p.tma_out != 0), s, p.pdl != 0, a, b, o, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s) {

@@ -55,6 +55,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ep", type=int, default=0,
+                    help="expert parallelism over this many ranks: under torchrun with as many "
+                         "GPUs, one rank per GPU with NCCL all-to-alls; on one GPU, that many "
+                         "ranks emulated in one process (copies for the exchange)")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
                     help="backward: time lmoe_backward (dx and every weight gradient, "
                          "forward activations recomputed) instead of the forward")
@@ -612,10 +616,93 @@ def run_backward(args):
     return 0
 
 
+def run_ep(args):
+    """One step = one expert-parallel forward of T tokens per rank (the
+    phases of lmoe_ep_* with the two l-wide all-to-alls between them)."""
+    import torch
+    import torch.distributed as dist
+    from latent_mixture_experts_top_b200 import ep, lmoe, synth
+
+    W = args.ep
+    if W < 2:
+        raise SystemExit("--ep needs at least 2 ranks")
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    emulated = world == 1
+    if not emulated and world != W:
+        raise SystemExit(f"--ep {W} needs {W} ranks (got {world}) or one (emulated)")
+    if not emulated:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    cfg = workload(args.workload)
+    inp = synth.make_inputs(cfg, args.seed, "cuda")       # same weights on every rank
+    ranks = range(W) if emulated else [rank]
+    layers = [lmoe.LatentMoELayer(cfg, inp, ep_rank=r, ep_world=W) for r in ranks]
+    backends = [ep.CudaBackend(L) for L in layers]
+    g = torch.Generator(device="cuda").manual_seed(1000 + rank)
+    xs = [(torch.randn((cfg.T, cfg.d), generator=g, device="cuda")).to(inp["x"].dtype)
+          for _ in ranks]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        if emulated:
+            return ep.forward_emulated(backends, xs)
+        return [ep.forward(backends[0], xs[0], W)]
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if not emulated:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local).start()
+    for i in range(K):
+        flush.fill_(1)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total = sum(step_ms)
+    if not emulated:
+        total = reduce_max_over_ranks(total, world, "cuda")
+        dist.barrier()
+    ms_per_step = total / K
+    for L in layers:
+        if lmoe.lmoe_device_status(L.handle) != 0:
+            raise RuntimeError("device status error")
+        L.close()
+    if rank == 0:
+        line = {"metric": f"LatentMoE expert-parallel fwd tokens/s, {W} ranks",
+                "value": cfg.T * W / (ms_per_step / 1e3), "unit": UNIT, "n_gpus": world,
+                "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic: x~N(0,1) per rank, weights~N(0,0.02), seeded",
+                "config": dict(config_json(cfg, W),
+                               parallelism=f"expert-parallel x{W}" +
+                               (" (emulated on one GPU: phases of every rank in turn, "
+                                "exchange by device copies)" if emulated else " (NCCL)")),
+                "gpu_launches": None, "clocks": clk,
+                "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
+        print(json.dumps(line), flush=True)
+    if not emulated:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.ep:
+        return run_ep(args)
     if args.which == "backward":
         return run_backward(args)
     return run_ours(args)

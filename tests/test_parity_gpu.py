@@ -130,6 +130,37 @@ def test_parity_wide_k_four_launch_routing(cfg):
     _check_layer(cfg, n_sample=10 ** 9)
 
 
+# The method's degenerate cases and the largest expert count, every token
+# compared: K' = 1 (the gate is 1), K' = N' (every expert: the dense limit),
+# alpha = 1 (l = d, no compression), and N' = 1024 (the library's maximum;
+# top-K' keys 32 per lane).
+EDGE = [
+    configs.LayerConfig("k1_f32_T64_d256_l128_N16_K1", T=64, d=256, m=256, n_experts=16, top_k=1,
+                        alpha=2, n_shared=1, m_shared=256, variant="eff", dtype="f32",
+                        n_routed_override=16),
+    configs.LayerConfig("k1_bf16_T200_d256_l128_N32_K1", T=200, d=256, m=256, n_experts=32,
+                        top_k=1, alpha=2, n_shared=1, m_shared=256, variant="eff",
+                        n_routed_override=32),
+    configs.LayerConfig("dense_f32_T64_d256_l128_N16_K16", T=64, d=256, m=256, n_experts=16,
+                        top_k=16, alpha=2, n_shared=1, m_shared=256, variant="eff", dtype="f32",
+                        n_routed_override=16),
+    configs.LayerConfig("dense_bf16_T200_d256_l128_N32_K32", T=200, d=256, m=256, n_experts=32,
+                        top_k=32, alpha=2, n_shared=1, m_shared=256, variant="eff",
+                        n_routed_override=32),
+    configs.LayerConfig("alpha1_f32_T64_d128_l128_N8_K2", T=64, d=128, m=128, n_experts=8, top_k=2,
+                        alpha=1, n_shared=1, m_shared=128, variant="acc", dtype="f32"),
+    configs.LayerConfig("alpha1_bf16_T300_d256_l256_N32_K4", T=300, d=256, m=256, n_experts=32,
+                        top_k=4, alpha=1, n_shared=1, m_shared=256, variant="acc"),
+    configs.LayerConfig("n1024_bf16_T512_d256_l128_N1024_K8", T=512, d=256, m=128, n_experts=512,
+                        top_k=4, alpha=2, n_shared=1, m_shared=256, variant="acc"),
+]
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=lambda c: c.name)
+def test_parity_degenerate_and_extreme_layers(cfg):
+    _check_layer(cfg, n_sample=10 ** 9)
+
+
 def test_parity_relu2_tiny_f32_all_tokens():
     _check_layer(configs.TINY_RELU2_F32, n_sample=10 ** 9)
 

@@ -21,7 +21,9 @@ struct TileEntry {
 cudaError_t launch_topk(const float *logits, int ld, const float *bias, int T, int N, int K,
                         int32_t *ids, float *gates, int32_t *counts, int chunk, cudaStream_t s);
 
-// Tokens per dispatch chunk on the forward path, and the chunk count.
+// Tokens per dispatch chunk on the forward path (the two-launch routing, and
+// the four-launch one), and the chunk count.
+constexpr int kFusedChunk = 32;
 constexpr int kDispatchChunk = 64;
 inline int dispatch_chunks(int T, int chunk) { return (T + chunk - 1) / chunk; }
 // Elements of the [N][chunks] count matrix (rows padded to a multiple of 4).

@@ -94,6 +94,7 @@ struct lmoe_layer {
   // Routing in two launches (top-K' + histogram + scan, then scatter + the
   // permutation of z) when the shapes allow; else four (see run_route).
   bool fused_route = false;
+  int route_chunk = kDispatchChunk;  // tokens per dispatch chunk of the path taken
   int route_shares = 1;  // blocks per dispatch chunk that split the permutation copies
   int64_t R_max = 0, h_rows = 0;
   int max_tiles_ep = 0, max_tiles2_ep = 0;
@@ -305,12 +306,15 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   h->sh_rows = h->relu2 ? (h->ns * h->ms + kTileN - 1) / kTileN * kTileN : 2 * h->ns * h->ms;
   h->nx_rows = h->n_pad + h->l_pad + h->sh_rows;
   h->gu_rows = h->relu2 ? h->m : 2 * h->m;
-  h->fused_route = fused_route_ok(h->N, h->K, kDispatchChunk);
-  h->route_shares = std::max(1, std::min(16, (2 * h->num_sms + dispatch_chunks(h->Tmax, kDispatchChunk) - 1) /
-                                                 dispatch_chunks(h->Tmax, kDispatchChunk)));
+  h->fused_route = fused_route_ok(h->N, h->K, kFusedChunk);
+  h->route_chunk = h->fused_route ? kFusedChunk : kDispatchChunk;
+  {  // blocks per chunk for the permutation copies: about four per SM in all
+    const int nc = dispatch_chunks(h->Tmax, kFusedChunk);
+    h->route_shares = std::max(1, std::min(64, (4 * h->num_sms + nc - 1) / nc));
+  }
   Workspace &w = h->ws;
   bool ok = dalloc(&w.logits, T * N * 4) && dalloc(&w.ids, TK * 4) && dalloc(&w.gates, TK * 4) &&
-            dalloc(&w.chunk_counts, dispatch_count_elems(h->Tmax, kDispatchChunk, h->N) * 4) &&
+            dalloc(&w.chunk_counts, dispatch_count_elems(h->Tmax, h->route_chunk, h->N) * 4) &&
             dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TK * 4) && dalloc(&w.pos, TK * 4) &&
             dalloc(&w.row_expert, TK * 4) &&
             dalloc(&w.tiles, static_cast<size_t>(h->max_tiles) * sizeof(TileEntry)) &&
@@ -726,13 +730,13 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     // (bf16: the router GEMM; fp32: the CUDA-core router) and waits for it on
     // the device before touching memory
     e = launch_route_select(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates,
-                            w.chunk_counts, kDispatchChunk, w.arrivals, w.offsets, w.tiles,
+                            w.chunk_counts, kFusedChunk, w.arrivals, w.offsets, w.tiles,
                             w.n_tiles, kTileM, h->max_tiles, w.tiles2, w.n_tiles2, 2 * kTileM,
                             h->max_tiles2, s, true);
     h->launches += 1;
     if (e != cudaSuccess) return e;
     if (full && marks) mark(h, 2, s);
-    e = launch_scatter_permute(w.ids, T, h->K, h->N, w.chunk_counts, kDispatchChunk, w.offsets,
+    e = launch_scatter_permute(w.ids, T, h->K, h->N, w.chunk_counts, kFusedChunk, w.offsets,
                                w.perm, w.pos, w.row_expert, permute_dst ? w.z : nullptr, rb,
                                permute_dst, h->route_shares, s, true);
     h->launches += 1;

@@ -261,14 +261,15 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
 
 // ---------------------------------------------------------------- fused routing
 // Top-K', dispatch histogram and scan in one launch.  Block c takes the
-// chunk of `chunk` tokens starting at c * chunk; its warps select the tokens
-// in turn (select_token) and count the chosen experts in shared memory, which
-// becomes column c of the count matrix (every entry written: no clearing
-// needed).  The block that arrives last on the arrival counter (after a
+// chunk of `chunk` tokens starting at c * chunk, one warp per token (the
+// selection is a chain of dependent warp reductions, so every token runs in
+// its own warp at once), and counts the chosen experts in shared memory,
+// which becomes column c of the count matrix (every entry written: no
+// clearing needed).  The block that arrives last on the arrival counter (after a
 // fence, so it sees every column) runs the scan of phase 2 and resets the
 // counter to zero for the next launch.
 template <int VPL>
-__global__ void __launch_bounds__(256) route_select_kernel(
+__global__ void __launch_bounds__(1024) route_select_kernel(
     const float *__restrict__ logits, int ld, const float *__restrict__ bias, int T, int N, int K,
     int32_t *__restrict__ ids, float *__restrict__ gates, int32_t *__restrict__ counts,
     int n_chunks, int chunk, int32_t *__restrict__ arrivals, int32_t *__restrict__ offsets,
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(
   griddep_wait();
   __syncthreads();
   const int t0 = blockIdx.x * chunk, t1 = min(T, t0 + chunk);
-  for (int t = t0 + warp; t < t1; t += nwarps)
+  for (int t = t0 + warp; t < t1; t += nwarps)  // one pass: nwarps == chunk
     select_token<VPL>(logits, ld, bias, N, K, t, ids, gates, hist, nullptr, 0);
   __syncthreads();
   const int ncp = (n_chunks + 3) & ~3;
@@ -352,12 +353,29 @@ __global__ void __launch_bounds__(256) scatter_permute_kernel(
   }
   if (!src) return;
   __syncthreads();
+  // The share's pairs are i = share, share + S, ...; item j = (its q-th pair,
+  // vector v) with q = j / vecs_per_row: consecutive threads copy consecutive
+  // 16-byte vectors of a row, four items in flight per thread.
   const int npairs = min(chunk, T - c * chunk) * K;
-  const int nwarps = blockDim.x >> 5;
-  for (int i = share + S * w; i < npairs; i += S * nwarps) {
-    const uint4 *sr = src + static_cast<size_t>(c * chunk + i / K) * vecs_per_row;
-    uint4 *dr = dst + static_cast<size_t>(ppos[i]) * vecs_per_row;
-    for (int v = lane; v < vecs_per_row; v += 32) dr[v] = sr[v];
+  const int my_pairs = npairs > share ? (npairs - share + S - 1) / S : 0;
+  const int items = my_pairs * vecs_per_row;
+  for (int j0 = threadIdx.x; j0 < items; j0 += 4 * blockDim.x) {
+    uint4 v[4];
+    int64_t dst_at[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * blockDim.x;
+      dst_at[u] = -1;
+      if (j < items) {
+        const int q = j / vecs_per_row, vv = j - q * vecs_per_row;
+        const int i = share + q * S;
+        v[u] = src[static_cast<size_t>(c * chunk + i / K) * vecs_per_row + vv];
+        dst_at[u] = static_cast<int64_t>(ppos[i]) * vecs_per_row + vv;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (dst_at[u] >= 0) dst[dst_at[u]] = v[u];
   }
 }
 
@@ -535,47 +553,51 @@ __device__ __forceinline__ uint4 pack_vec<float>(const float *acc) {
   return r;
 }
 
-// One warp per token; 16-byte vectors; slots summed in order 0..K-1 in fp32.
-// (At most 64 registers: 32 warps per SM keep all token warps of the bench
-// workload resident at once.)
+// One warp per (token, 32 vectors of its row): a row of l elements takes
+// ceil(l / (32 V)) warps, so that every vector of every token has its loads in
+// flight at once; 16-byte vectors; the K' slots are summed in slot order
+// 0..K'-1 in fp32 (eight slots' loads in flight, then accumulated in order).
+// (At most 64 registers: 32 warps per SM.)
 template <typename Tio>
 __global__ void __launch_bounds__(256, 4) combine_kernel(const Tio *__restrict__ O,
                                                       const int32_t *__restrict__ pos,
                                                       const float *__restrict__ gates, int T,
                                                       int K, int l, Tio *__restrict__ u, int ldu) {
   constexpr int V = 16 / sizeof(Tio);
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nvec = l / V;
+  const int wpt = (nvec + 31) / 32;  // warps per token
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   griddep_wait();
+  const int t = gw / wpt;
   if (t >= T) return;
-  const int nvec = l / V;
-  for (int vi = lane; vi < nvec; vi += 32) {
-    float acc[V];
+  const int vi = (gw - t * wpt) * 32 + lane;
+  const bool active = vi < nvec;
+  float acc[V];
 #pragma unroll
-    for (int j = 0; j < V; ++j) acc[j] = 0.0f;
-    for (int k0 = 0; k0 < K; k0 += 32) {
-      const int kk = k0 + lane;
-      const int my_p = kk < K ? pos[static_cast<size_t>(t) * K + kk] : 0;
-      const float my_g = kk < K ? gates[static_cast<size_t>(t) * K + kk] : 0.0f;
-      const int kn = min(32, K - k0);
-      // Eight slots' loads in flight, then accumulated in slot order.
-      for (int k1 = 0; k1 < kn; k1 += 8) {
-        uint4 raw[8];
+  for (int j = 0; j < V; ++j) acc[j] = 0.0f;
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    const int kk = k0 + lane;
+    const int my_p = kk < K ? pos[static_cast<size_t>(t) * K + kk] : 0;
+    const float my_g = kk < K ? gates[static_cast<size_t>(t) * K + kk] : 0.0f;
+    const int kn = min(32, K - k0);
+    for (int k1 = 0; k1 < kn; k1 += 8) {
+      uint4 raw[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int p = __shfl_sync(kFull, my_p, (k1 + j) & 31);
-          if (k1 + j < kn)
-            raw[j] = __ldcs(reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l + vi * V));
-        }
+      for (int j = 0; j < 8; ++j) {
+        const int p = __shfl_sync(kFull, my_p, (k1 + j) & 31);
+        if (active && k1 + j < kn)
+          raw[j] = __ldcs(reinterpret_cast<const uint4 *>(O + static_cast<size_t>(p) * l + vi * V));
+      }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float g = __shfl_sync(kFull, my_g, (k1 + j) & 31);
-          if (k1 + j < kn) accum_vec<Tio>(acc, raw[j], g);
-        }
+      for (int j = 0; j < 8; ++j) {
+        const float g = __shfl_sync(kFull, my_g, (k1 + j) & 31);
+        if (active && k1 + j < kn) accum_vec<Tio>(acc, raw[j], g);
       }
     }
-    *reinterpret_cast<uint4 *>(u + static_cast<size_t>(t) * ldu + vi * V) = pack_vec<Tio>(acc);
   }
+  if (active)
+    *reinterpret_cast<uint4 *>(u + static_cast<size_t>(t) * ldu + vi * V) = pack_vec<Tio>(acc);
 }
 
 // One 16-byte vector per thread: dst vector v -> (group, n-tile, k-block,
@@ -687,7 +709,9 @@ cudaError_t launch_counts_from_offsets(const int32_t *offsets, int N, int32_t *c
 }
 
 bool fused_route_ok(int N, int K, int chunk) {
-  return N <= 1024 && chunk % 32 == 0 && chunk >= 32 && chunk <= 256 && chunk * K <= 4096;
+  // route_select_kernel: one warp per token of a chunk (at most 1024 threads);
+  // scatter_permute_kernel: chunk * K positions in shared memory
+  return N <= 1024 && chunk == 32 && chunk * K <= 4096;
 }
 
 cudaError_t launch_route_select(const float *logits, int ld, const float *bias, int T, int N,
@@ -703,7 +727,7 @@ cudaError_t launch_route_select(const float *logits, int ld, const float *bias, 
   const int vpl = (N + 31) / 32;
   cudaError_t e;
 #define LMOE_ROUTE(V)                                                                            \
-  e = launch_ex(route_select_kernel<V>, dim3(nc), dim3(256), 0, s, pdl, logits, ld, bias, T, N, \
+  e = launch_ex(route_select_kernel<V>, dim3(nc), dim3(32 * chunk), 0, s, pdl, logits, ld, bias, T, N, \
                 K, ids, gates, counts, nc, chunk, arrivals, offsets, tiles, n_tiles, tile_m,     \
                 max_tiles, tiles2, n_tiles2, tile_m2, max_tiles2)
   if (vpl <= 1) LMOE_ROUTE(1);
@@ -747,7 +771,9 @@ cudaError_t launch_permute_rows(const void *src, const int32_t *perm, int K, int
 cudaError_t launch_combine(const void *O, const int32_t *pos, const float *gates, int T, int K,
                            int l, void *u, int ldu, bool is_bf16, cudaStream_t s, bool pdl) {
   if (T <= 0) return cudaSuccess;
-  const int blocks = (T + 7) / 8;
+  const int nvec = l / (is_bf16 ? 8 : 4);
+  const int64_t warps = static_cast<int64_t>(T) * ((nvec + 31) / 32);
+  const int blocks = static_cast<int>((warps + 7) / 8);
   if (is_bf16) {
     if (l % 8 || ldu % 8) return cudaErrorInvalidValue;
     const cudaError_t e = launch_ex(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, s,

@@ -55,6 +55,7 @@ class _Layer(C.Structure):
         ("w_down", C.c_void_p), ("w_up", C.c_void_p),
         ("w_gate", C.c_void_p), ("w_upx", C.c_void_p), ("w_out", C.c_void_p),
         ("s_gate", C.c_void_p), ("s_up", C.c_void_p), ("s_out", C.c_void_p),
+        ("act_fp8", C.c_int32),
     ]
 
 
@@ -132,10 +133,15 @@ class Layer:
     s_gate / s_up [n_s][m_s][d], s_out [n_s][d][m_s].
     activation "swiglu" (three matrices) or "relu2" (squared ReLU, two
     matrices: w_upx / s_up are the up-projections; w_gate / s_gate unused).
+    act_fp8: the routed experts multiply E4M3 activations -- each token's z
+    and each expert's hidden vector quantised with the weight rows' rule (a
+    power-of-two scale, the smallest that brings the largest magnitude
+    within 448); the backward is then not defined.
     """
 
     def __init__(self, *, w_router, b_router, w_down, w_up, w_gate, w_upx,
-                 w_out, s_gate, s_up, s_out, k_active, activation="swiglu"):
+                 w_out, s_gate, s_up, s_out, k_active, activation="swiglu",
+                 act_fp8=False):
         if activation not in ("swiglu", "relu2"):
             raise ValueError("activation must be 'swiglu' or 'relu2'")
         self.activation = activation
@@ -169,7 +175,8 @@ class Layer:
                          _ptr(k["w_router"]), _ptr(self.b_router), _ptr(k["w_down"]),
                          _ptr(k["w_up"]), _ptr(k["w_gate"]), _ptr(k["w_upx"]),
                          _ptr(k["w_out"]), _ptr(k["s_gate"]), _ptr(k["s_up"]),
-                         _ptr(k["s_out"]))
+                         _ptr(k["s_out"]), 1 if act_fp8 else 0)
+        self.act_fp8 = bool(act_fp8)
 
     @property
     def cref(self):

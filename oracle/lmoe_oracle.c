@@ -70,6 +70,7 @@ typedef struct {
   const void *s_gate;        /* [n_s][m_s][d] */
   const void *s_up;          /* [n_s][m_s][d] */
   const void *s_out;         /* [n_s][d][m_s] */
+  int32_t act_fp8;           /* 1: routed experts run on E4M3 activations (see q_vec_e4m3) */
 } oracle_layer;
 
 /* Exact widening of one stored element to double. */
@@ -105,10 +106,14 @@ static double relu2(double a) { return a > 0.0 ? a * a : 0.0; }
  * Squared ReLU: out = W_o (relu(W_u v))^2  ([Explained], the Expert class:
  * up, relu, square, down).
  * W_g, W_u: [hid][in_w] at element offset off_in; W_o: [out_w][hid] at off_out. */
+static void q_vec_e4m3(double *v, int n);
+
+/* quant_hidden: the hidden vector is replaced by its E4M3 row quantisation
+ * before the down-projection (routed experts with act_fp8). */
 static void swiglu_ffn(const oracle_layer *L, const void *Wg, const void *Wu,
                        const void *Wo, size_t off_in, size_t off_out, int in_w,
                        int hid, int out_w, const double *v, double *out,
-                       double *scratch /* 2*hid */) {
+                       double *scratch /* 2*hid */, int quant_hidden) {
   double *a = scratch, *b = scratch + hid;
   if (L->activation == OACT_RELU2) {
     matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
@@ -118,6 +123,7 @@ static void swiglu_ffn(const oracle_layer *L, const void *Wg, const void *Wu,
     matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
     for (int j = 0; j < hid; ++j) a[j] = silu(a[j]) * b[j];
   }
+  if (quant_hidden) q_vec_e4m3(a, hid);
   matvec(Wo, L->dtype, off_out, out_w, hid, a, out);
 }
 
@@ -224,7 +230,7 @@ void oracle_down(const oracle_layer *L, const void *x, int64_t t, double *z) {
 void oracle_expert(const oracle_layer *L, int e, const double *z, double *out) {
   double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)L->m);
   swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * L->m * L->l,
-             (size_t)e * L->l * L->m, L->l, L->m, L->l, z, out, scratch);
+             (size_t)e * L->l * L->m, L->l, L->m, L->l, z, out, scratch, L->act_fp8);
   free(scratch);
 }
 
@@ -242,7 +248,7 @@ void oracle_shared(const oracle_layer *L, const void *x, int64_t t, double *out)
   for (int i = 0; i < d; ++i) { xv[i] = elem(x, L->dtype, (size_t)t * d + i); out[i] = 0.0; }
   for (int j = 0; j < L->n_shared; ++j) {
     swiglu_ffn(L, L->s_gate, L->s_up, L->s_out, (size_t)j * ms * d,
-               (size_t)j * d * ms, d, ms, d, xv, tmp, scratch);
+               (size_t)j * d * ms, d, ms, d, xv, tmp, scratch, 0);
     for (int i = 0; i < d; ++i) out[i] += tmp[i];
   }
   free(xv); free(tmp); free(scratch);
@@ -285,18 +291,19 @@ int oracle_forward(const oracle_layer *L, const void *x, int64_t T,
       }
       for (int i = 0; i < d; ++i) xv[i] = elem(x, L->dtype, (size_t)t * d + i);
       matvec(L->w_down, L->dtype, 0, l, d, xv, z);
+      if (L->act_fp8) q_vec_e4m3(z, l);  /* the experts read z in E4M3 */
       for (int i = 0; i < l; ++i) u[i] = 0.0;
       for (int k = 0; k < K; ++k) { /* slot loop, in slot order */
         const int e = ids[k];
         swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * m * l,
-                   (size_t)e * l * m, l, m, l, z, eo, scratch);
+                   (size_t)e * l * m, l, m, l, z, eo, scratch, L->act_fp8);
         for (int i = 0; i < l; ++i) u[i] += g[k] * eo[i];
       }
       double *yr = y + n * d;
       matvec(L->w_up, L->dtype, 0, d, l, u, yr);
       for (int j = 0; j < L->n_shared; ++j) {
         swiglu_ffn(L, L->s_gate, L->s_up, L->s_out, (size_t)j * L->m_shared * d,
-                   (size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch);
+                   (size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, 0);
         for (int i = 0; i < d; ++i) yr[i] += sh[i];
       }
       if (ids_out) memcpy(ids_out + n * K, ids, sizeof(int32_t) * (size_t)K);
@@ -422,6 +429,7 @@ int oracle_backward(const oracle_layer *L, const void *x, int64_t T,
   const int ns = L->n_shared, ms = L->m_shared > 0 ? L->m_shared : 1;
   const int relu = L->activation == OACT_RELU2;
   if (K < 1 || K > N || l < 1 || d < 1 || m < 1) return -1;
+  if (L->act_fp8) return -3;  /* no gradient through the activation quantiser */
   /* per-token and per-slot records for the weight-gradient sums */
   double *X = (double *)malloc(sizeof(double) * (size_t)n_tok * d);
   double *Z = (double *)malloc(sizeof(double) * (size_t)n_tok * l);
@@ -473,7 +481,7 @@ int oracle_backward(const oracle_layer *L, const void *x, int64_t T,
       for (int k = 0; k < K; ++k) {
         const int e = ids[k];
         swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * m * l,
-                   (size_t)e * l * m, l, m, l, z, eo, scratch);
+                   (size_t)e * l * m, l, m, l, z, eo, scratch, 0);
         for (int i = 0; i < l; ++i) u[i] += g[k] * eo[i];
         /* dg_k = du . o_k needs du first: o_k kept in DO for now */
         memcpy(DO + (n * K + k) * l, eo, sizeof(double) * (size_t)l);
@@ -647,6 +655,18 @@ static double e4m3_round(double v) {
   return v < 0.0 ? -r : r;
 }
 
+/* The row scale: the smallest power of two s with amax <= 448 s (1 for a
+ * row of zeros). */
+static double e4m3_row_scale(double amax) {
+  int e = 0;
+  if (amax > 0.0) {
+    e = (int)ceil(log2(amax / 448.0));
+    while (ldexp(448.0, e) < amax) ++e;
+    while (e > -200 && ldexp(448.0, e - 1) >= amax) --e;
+  }
+  return ldexp(1.0, e);
+}
+
 /* W [rows][cols] (any element type) -> W' (double) and the row scales. */
 void oracle_fp8_rows(const void *W, int dt, int64_t rows, int cols, double *Wq,
                      double *scales) {
@@ -657,17 +677,26 @@ void oracle_fp8_rows(const void *W, int dt, int64_t rows, int cols, double *Wq,
       const double v = fabs(elem(W, dt, (size_t)r * cols + c));
       if (v > amax) amax = v;
     }
-    int e = 0;  /* smallest e with amax <= 448 * 2^e */
-    if (amax > 0.0) {
-      e = (int)ceil(log2(amax / 448.0));
-      while (ldexp(448.0, e) < amax) ++e;
-      while (e > -200 && ldexp(448.0, e - 1) >= amax) --e;
-    }
-    const double s = ldexp(1.0, e);
+    const double s = e4m3_row_scale(amax);
     scales[r] = s;
     for (int c = 0; c < cols; ++c)
       Wq[(size_t)r * cols + c] = e4m3_round(elem(W, dt, (size_t)r * cols + c) / s) * s;
   }
+}
+
+/* ---- E4M3 activations (act_fp8; a reading chosen here, the pages give no
+ * FP8 activation recipe): the same rule as the weight rows, applied to each
+ * activation vector the routed experts multiply -- a token's z (its row of
+ * the expert GEMMs' first operand) and each expert's hidden h (its row of the
+ * down-projection's first operand): v <- E4M3(v / s) * s with s the row
+ * scale of v.  The router, W_down, the combine, W_up and the shared experts
+ * stay as they are. */
+static void q_vec_e4m3(double *v, int n) {
+  double amax = 0.0;
+  for (int i = 0; i < n; ++i)
+    if (fabs(v[i]) > amax) amax = fabs(v[i]);
+  const double s = e4m3_row_scale(amax);
+  for (int i = 0; i < n; ++i) v[i] = e4m3_round(v[i] / s) * s;
 }
 
 int oracle_threads(void) {

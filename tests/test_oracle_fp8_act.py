@@ -1,0 +1,128 @@
+"""Pins of the oracle's E4M3-activation reading (act_fp8), CPU only.
+
+The pages put the experts in FP8 ("LatentMoE Explained": an expert is about
+22 MB in FP8; the models are pretrained in NVFP4) but print no recipe for the
+activations.  The reading taken: the routed experts multiply E4M3 activations
+-- each token's z and each expert's hidden vector h are quantised with the
+rule of the weight rows (power-of-two scale, E4M3 round-to-nearest-even,
+saturating; pinned in tests/test_oracle_fp8.py) -- while the router, W_down,
+the combine, W_up and the shared experts are unchanged.  Here the oracle's
+forward with act_fp8 is held to the definition recomposed with numpy from the
+pinned quantiser and the pinned router: a missing, misplaced or extra
+quantisation step fails.
+"""
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+
+D, L_, M, N, K, NS, MS = 64, 32, 48, 6, 2, 1, 32
+
+
+def _weights(seed, activation):
+    rng = np.random.default_rng(seed)
+    w = lambda *s: rng.normal(0.0, 0.3, size=s)
+    kw = dict(w_router=w(N, D), b_router=None, w_down=w(L_, D), w_up=w(D, L_),
+              w_gate=w(N, M, L_), w_upx=w(N, M, L_), w_out=w(N, L_, M), s_gate=w(NS, MS, D),
+              s_up=w(NS, MS, D), s_out=w(NS, D, MS), k_active=K, activation=activation)
+    x = rng.normal(0.0, 1.0, size=(9, D))
+    return kw, x
+
+
+def _q(v):
+    q, _ = oracle.fp8_rows(np.asarray(v, dtype=np.float64)[None, :])
+    return q[0]
+
+
+def _silu(a):
+    return a / (1.0 + np.exp(-a))
+
+
+def _recompose(kw, x, act_fp8):
+    Lp = oracle.Layer(**kw)                        # unquantised: router and ids only
+    s = oracle.router_logits(Lp, x)
+    ids, g = oracle.select(s, K)
+    relu2 = kw["activation"] == "relu2"
+    y = np.zeros((x.shape[0], D))
+    for t in range(x.shape[0]):
+        z = kw["w_down"] @ x[t]
+        if act_fp8:
+            z = _q(z)
+        u = np.zeros(L_)
+        for k in range(K):
+            e = ids[t, k]
+            b = kw["w_upx"][e] @ z
+            h = np.maximum(b, 0.0) ** 2 if relu2 else _silu(kw["w_gate"][e] @ z) * b
+            if act_fp8:
+                h = _q(h)
+            u += g[t, k] * (kw["w_out"][e] @ h)
+        y[t] = kw["w_up"] @ u
+        for j in range(NS):
+            b = kw["s_up"][j] @ x[t]
+            h = np.maximum(b, 0.0) ** 2 if relu2 else _silu(kw["s_gate"][j] @ x[t]) * b
+            y[t] += kw["s_out"][j] @ h
+    return y
+
+
+@pytest.mark.parametrize("activation", ["swiglu", "relu2"])
+def test_act_fp8_forward_is_the_quantised_recomposition(activation):
+    kw, x = _weights(1, activation)
+    y, _, _ = oracle.forward(oracle.Layer(**kw, act_fp8=True), x)
+    y_ref = _recompose(kw, x, True)
+    np.testing.assert_allclose(y, y_ref, rtol=0, atol=1e-12 * np.abs(y_ref).max())
+    # and it is not the unquantised layer
+    y0 = _recompose(kw, x, False)
+    assert np.abs(y - y0).max() > 1e-4 * np.abs(y0).max()
+
+
+def test_act_fp8_off_leaves_the_layer_unchanged():
+    kw, x = _weights(2, "swiglu")
+    y, _, _ = oracle.forward(oracle.Layer(**kw, act_fp8=False), x)
+    np.testing.assert_allclose(y, _recompose(kw, x, False), rtol=0, atol=1e-12)
+
+
+def test_act_fp8_error_is_that_of_a_few_e4m3_roundings():
+    kw, x = _weights(3, "swiglu")
+    y8, _, _ = oracle.forward(oracle.Layer(**kw, act_fp8=True), x)
+    y, _, _ = oracle.forward(oracle.Layer(**kw), x)
+    rel = np.abs(y8 - y).max() / np.abs(y).max()
+    assert 1e-4 < rel < 0.1, rel
+
+
+def test_backward_refuses_act_fp8():
+    kw, x = _weights(4, "swiglu")
+    with pytest.raises(Exception):
+        oracle.backward(oracle.Layer(**kw, act_fp8=True), x, np.ones((x.shape[0], D)))
+
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "lmoe_oracle.c")
+MUTATIONS = {
+    "no_hidden_quantisation": ("  if (quant_hidden) q_vec_e4m3(a, hid);\n", "\n"),
+    "no_z_quantisation": ("      if (L->act_fp8) q_vec_e4m3(z, l);  /* the experts read z in E4M3 */\n",
+                          "\n"),
+    "shared_quantised_too": ("(size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, 0);",
+                             "(size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, L->act_fp8);"),
+    "quantised_after_down": ("  if (quant_hidden) q_vec_e4m3(a, hid);\n  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);",
+                             "  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);\n  if (quant_hidden) q_vec_e4m3(out, out_w);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_act_fp8_pins_catch_mutation(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-std=c11", "-O2", "-fopenmp", "-fPIC", "-shared",
+                           "-o", str(lib), str(mutated), "-lm"])
+    oracle._swap_library(str(lib))
+    try:
+        with pytest.raises(AssertionError):
+            test_act_fp8_forward_is_the_quantised_recomposition("swiglu")
+    finally:
+        oracle._swap_library(None)

@@ -57,13 +57,17 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
  * example uses.  Shared experts use the same. */
 typedef enum { LMOE_SWIGLU = 0, LMOE_RELU2 = 1 } lmoe_activation;
 
-/* Storage of the routed experts' weights (W_g, W_u, W_o) in LMOE_BF16 mode.
- * LMOE_WEIGHTS_FP8: E4M3 with one power-of-two scale per weight row (the
- * smallest that brings the row's largest magnitude within 448), for the
- * weight-streaming decode regime ("LatentMoE Explained" puts an expert at
- * about 22 MB in FP8; the pages give no scaling recipe, this is the one
- * chosen).  The layer then computes exactly with W' = E4M3(W / s) * s.
- * Not with training = 1. */
+/* Element type of the routed experts in LMOE_BF16 mode.
+ * LMOE_WEIGHTS_FP8: the expert GEMMs run in E4M3 on both operands
+ * (tcgen05 kind::f8f6f4, fp32 accumulation), for the weight-streaming decode
+ * regime ("LatentMoE Explained" puts an expert at about 22 MB in FP8; the
+ * pages give no scaling recipe, this is the one chosen).  W_g, W_u and W_o
+ * are stored as E4M3 with one power-of-two scale per weight row (the smallest
+ * that brings the row's largest magnitude within 448); each token's z and
+ * each expert's hidden vector are quantised the same way, per row, before
+ * they are multiplied.  The layer then computes exactly with those quantised
+ * operands.  Needs l and m multiples of 128.  Not with training = 1, not
+ * with expert parallelism. */
 typedef enum { LMOE_WEIGHTS_BF16 = 0, LMOE_WEIGHTS_FP8 = 1 } lmoe_weight_format;
 
 enum {
@@ -193,11 +197,14 @@ int lmoe_selftest_wait_timeout(lmoe_handle h, int64_t limit_ns, void *stream);
  * 3 expert hidden [T*K'][m], 4 expert out [T*K'][l], 5 [u | shared hidden]
  * [T][l + n_s m_s], 6 ids, 7 gates, 8 offsets, 9 perm, 10 pos [T*K'] (inverse
  * of perm), 11 number of 128-row expert tiles; with LMOE_WEIGHTS_FP8 also
- * 12 gate/up E4M3 codes and 14 W_o E4M3 codes (bytes, in 256 x 64 tiles:
- * expert, 256-row tile, 64-column block, row, column), 13 gate/up row scales
+ * 12 gate/up E4M3 codes and 14 W_o E4M3 codes (bytes, in 256 x 128 blocks:
+ * expert, 256-row tile, 128-column block, row, column), 13 gate/up row scales
  * [N'][2m, gate and up rows interleaved in blocks of 128; m rows of W_u for
- * squared ReLU] and 15 W_o row scales [N'][l], f32).  Errors: NULL_ARG,
- * INVALID_CONFIG (unknown `which`). */
+ * squared ReLU] and 15 W_o row scales [N'][l], f32; 16 the E4M3 codes of the
+ * experts' input rows [T*K'][l] (z in dispatch order) and 17 their row scales
+ * [T*K'] f32; 18 the E4M3 codes of the expert hidden rows [T*K'][m] and 19
+ * their row scales [T*K'] f32).  Errors: NULL_ARG, INVALID_CONFIG (unknown
+ * `which`). */
 int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel);
 
 /* Profiling hook.  slots > 0: every later lmoe_forward on this handle also

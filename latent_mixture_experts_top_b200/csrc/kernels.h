@@ -158,9 +158,12 @@ struct TcParams {
   // epilogue applies the activation backward with the pre-activations
   // act_ab [rows][ld_ab] (gate/up layout of the GU GEMM) and writes act_dab.
   const __nv_bfloat16 *act_ab; __nv_bfloat16 *act_dab; int ld_ab;
-  // FP8 expert weights (TC_EXPERT_GU / TC_EXPERT_DOWN): B is E4M3 (tiled like
-  // the bf16 weights, 1 byte per element) and b_scale [expert][b_scale_ld]
-  // holds each weight row's scale.
+  // E4M3 operands (TC_EXPERT_GU / TC_EXPERT_DOWN with b_scale set): A is
+  // E4M3 [rows][Kdim] with one scale per row in a_scale, B is the E4M3 weight
+  // tiled in 256-row x 128-byte blocks (launch_quantize_e4m3_tiles) and
+  // b_scale [expert][b_scale_ld] holds each weight row's scale; the MMA is
+  // kind::f8f6f4 over 128-element K-blocks.
+  const float *a_scale;
   const float *b_scale; int b_scale_ld;
   // TC_WGRAD: A [M][*] and B [*][*] are plain row-major token-major matrices
   // (K runs along their rows' contiguous axis); group g reduces over
@@ -197,13 +200,25 @@ cudaError_t launch_repack_btiles(const __nv_bfloat16 *src, int groups, int rows_
                                  int cols, __nv_bfloat16 *dst, cudaStream_t s);
 
 // E4M3 expert weights (fp8_weights.cu): src [groups][rows][cols] bf16 ->
-// per-row power-of-two scales [groups][rows] and E4M3 codes, K-block tiled
-// like launch_repack_btiles (1 byte per element; padding rows zero).
+// per-row power-of-two scales [groups][rows] and E4M3 codes stored in blocks
+// of 256 rows x 128 bytes (per group, 256-row tile n and 128-column block kb:
+// one contiguous block; padding rows zero).  cols % 128 == 0.  The same byte
+// count as btile_rows(groups, rows_per_group, cols) * 64.
 cudaError_t launch_quantize_e4m3_tiles(const __nv_bfloat16 *src, int groups, int rows_per_group,
                                        int cols, float *scales, uint8_t *dst, cudaStream_t s);
 
+// E4M3 activations: row r of dst [rows][cols] (bytes) and scales[r] from the
+// bf16 row src[gather ? gather[r] / K : r] (row stride cols): the smallest
+// power-of-two scale with max |row| <= 448 scale, then each element's E4M3
+// code, rounded to nearest even and saturating (the weights' rule).  One warp
+// per row.  cols % 8 == 0.
+cudaError_t launch_quantize_rows_e4m3(const __nv_bfloat16 *src, const int32_t *gather, int K,
+                                      int rows, int cols, uint8_t *dst, float *scales,
+                                      cudaStream_t s, bool pdl = false);
+
 // Encodes a 2-D byte tensor map (rows x cols bytes, row stride in bytes)
-// with a {64, box_rows} box and no swizzle.  Host only.
+// with a {128, box_rows} box and 128-byte swizzle (E4M3 GEMM operands).
+// Host only.
 int make_tmap_u8(void *tmap_out, const void *base, int64_t rows, int64_t cols,
                  int64_t row_stride_bytes, int box_rows);
 
@@ -290,8 +305,8 @@ cudaError_t launch_padded_offsets(const int32_t *offsets, int N, int32_t *kstart
 // Failure-detection self-test (see lmoe_selftest_wait_timeout).
 cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s);
 
-// tmapA32: with E4M3 weights (p.b_scale set), the same A matrix with a
-// {64, 32} box, used for tiles of at most 32 token rows.
+// tmapA32: with E4M3 operands (p.b_scale set), the same A matrix with a
+// {128, 32} box, used for tiles of at most 32 token rows.
 // tmapOut: with p.tma_out set (forward bf16 modes only), the bf16 output
 // matrix's map from make_tmap_bf16_out (z for TC_X_FUSED).
 cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams &p,

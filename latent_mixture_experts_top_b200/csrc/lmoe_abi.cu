@@ -44,6 +44,9 @@ struct Workspace {
   void *x_stage = nullptr, *y_stage = nullptr;
   int32_t *status = nullptr;
   int32_t *arrivals = nullptr;  // fused routing: the last-block counter (zero between launches)
+  // E4M3 routed experts: the expert GEMMs' A operands in E4M3 with row scales
+  uint8_t *zq = nullptr, *hq = nullptr;  // [TK][l], [TK][m]
+  float *zq_scale = nullptr, *hq_scale = nullptr;  // [TK]
   // expert parallelism: M-tile tables of the received rows (128- and 256-row)
   TileEntry *ep_tiles = nullptr, *ep_tiles2 = nullptr;
   int32_t *ep_n_tiles = nullptr, *ep_n_tiles2 = nullptr;
@@ -80,7 +83,7 @@ struct lmoe_layer {
   int d = 0, l = 0, m = 0, N = 0, K = 0, ns = 0, ms = 0, Tmax = 0;
   int bf16 = 0;
   int relu2 = 0;      // squared-ReLU experts (two matrices)
-  int fp8 = 0;        // E4M3 routed-expert weights
+  int fp8 = 0;        // E4M3 routed experts (weights and the activations they multiply)
   size_t esize = 4;
   int device = 0, num_sms = 0;
   bool loaded = false;
@@ -128,7 +131,7 @@ struct lmoe_layer {
   TensorMap64 tm_out_z, tm_out_h, tm_out_o;  // epilogue TMA stores: z, H, O
   // B operands of the CTA-pair GEMMs: the same tiled matrices, {64, 128} boxes
   TensorMap64 tm_wx2, tm_wo2, tm_wy2;
-  TensorMap64 tm_zp32, tm_h32;  // E4M3 weights: {64, 32} boxes for small tiles
+  TensorMap64 tm_zq, tm_zq32, tm_hq, tm_hq32;  // E4M3 activations ({128, 128}, {128, 32})
   // E4M3 expert weights (tiled like w_gu / w_out) and their row scales
   uint8_t *w_gu8 = nullptr, *w_o8 = nullptr;
   float *gu_scale = nullptr, *o_scale = nullptr;
@@ -177,7 +180,8 @@ void free_all(lmoe_layer *h) {
                   h->bw.zpT, h->bw.dyT, h->bw.ucatT, h->bw.dXcatT, h->bw.xT, h->bw.kstart,
                   h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT, h->w_gu8,
                   h->w_o8, h->gu_scale, h->o_scale, h->ws.ep_tiles, h->ws.ep_tiles2,
-                  h->ws.ep_n_tiles, h->ws.ep_n_tiles2, h->ws.arrivals};
+                  h->ws.ep_n_tiles, h->ws.ep_n_tiles2, h->ws.arrivals, h->ws.zq, h->ws.hq,
+                  h->ws.zq_scale, h->ws.hq_scale};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
@@ -227,6 +231,8 @@ int validate(const lmoe_config *c, lmoe_layer *h) {
     return LMOE_ERR_INVALID_CONFIG;
   h->fp8 = c->weight_format == LMOE_WEIGHTS_FP8;
   if (h->fp8 && (c->dtype != LMOE_BF16 || c->training)) return LMOE_ERR_UNSUPPORTED;
+  // E4M3 GEMMs run 128-element K-blocks: l and m must be multiples of 128
+  if (h->fp8 && ((c->d / c->alpha) % 128 || c->m % 128)) return LMOE_ERR_UNSUPPORTED;
   h->esize = h->bf16 ? 2 : 4;
   h->ky = h->l + h->ns * h->ms;
   if (static_cast<int64_t>(h->Tmax) * h->K * W > INT32_MAX / 2) return LMOE_ERR_UNSUPPORTED;
@@ -332,7 +338,9 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
       if (ok && h->fp8)
         ok = dalloc(&h->w_gu8, btile_rows(h->N, h->gu_rows, h->l) * 64) &&
              dalloc(&h->w_o8, btile_rows(h->N, h->l, h->m) * 64) &&
-             dalloc(&h->gu_scale, N * h->gu_rows * 4) && dalloc(&h->o_scale, N * l * 4);
+             dalloc(&h->gu_scale, N * h->gu_rows * 4) && dalloc(&h->o_scale, N * l * 4) &&
+             dalloc(&w.zq, TK * l) && dalloc(&w.hq, TK * m) && dalloc(&w.zq_scale, TK * 4) &&
+             dalloc(&w.hq_scale, TK * 4);
       else if (ok)
         ok = dalloc(&h->w_gu, btile_rows(h->NE, h->gu_rows, h->l) * 64 * es) &&
              dalloc(&h->w_out, btile_rows(h->NE, h->l, h->m) * 64 * es);
@@ -412,13 +420,16 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wx2, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN / 2);
     if (rc == LMOE_OK && h->fp8) {
-      rc = make_map(&h->tm_zp32, w.zp, static_cast<int64_t>(TK), h->l, h->l, 32);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_h32, w.H, static_cast<int64_t>(TK), h->m, h->m, 32);
-    }
-    if (rc == LMOE_OK && h->fp8) {  // E4M3 tiles: {64 bytes, 256 rows}, no swizzle
-      if (make_tmap_u8(h->tm_wgu.bytes, h->w_gu8, btile_rows(h->N, h->gu_rows, h->l), 64, 64,
-                       kTileN) != 0 ||
-          make_tmap_u8(h->tm_wo.bytes, h->w_o8, btile_rows(h->N, h->l, h->m), 64, 64, kTileN) != 0)
+      // E4M3 operands, 128-byte swizzle: A rows {128, 128} (and {128, 32} for
+      // tiles of at most 32 rows); the weights in 256-row x 128-byte blocks
+      const int64_t gu8_rows = btile_rows(h->N, h->gu_rows, h->l) / 2;
+      const int64_t o8_rows = btile_rows(h->N, h->l, h->m) / 2;
+      if (make_tmap_u8(h->tm_zq.bytes, w.zq, static_cast<int64_t>(TK), h->l, h->l, kTileM) != 0 ||
+          make_tmap_u8(h->tm_zq32.bytes, w.zq, static_cast<int64_t>(TK), h->l, h->l, 32) != 0 ||
+          make_tmap_u8(h->tm_hq.bytes, w.hq, static_cast<int64_t>(TK), h->m, h->m, kTileM) != 0 ||
+          make_tmap_u8(h->tm_hq32.bytes, w.hq, static_cast<int64_t>(TK), h->m, h->m, 32) != 0 ||
+          make_tmap_u8(h->tm_wgu.bytes, h->w_gu8, gu8_rows, 128, 128, kTileN) != 0 ||
+          make_tmap_u8(h->tm_wo.bytes, h->w_o8, o8_rows, 128, 128, kTileN) != 0)
         rc = LMOE_ERR_CUDA;
     } else {
       if (rc == LMOE_OK)
@@ -804,13 +815,15 @@ int lmoe_route(lmoe_handle h, const void *x, int32_t T, int32_t *ids, float *gat
 // the expert outputs through the store map tm_o.  pair_down: the down GEMM
 // runs on CTA pairs.  stage_gu / stage_down: profiling marks after each.
 // pdl: the gate/up launch directly follows another kernel on s (the down
-// GEMM always follows the gate/up GEMM).
+// GEMM always follows the gate/up GEMM).  a_rows: rows of A (and of H, O).
+// E4M3 experts: A is the E4M3 copy of the rows (tm_a over zq), H is
+// quantised to hq between the two GEMMs.
 static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
                                     const TensorMap64 &tm_a32, const TileEntry *tiles,
                                     const int32_t *n_tiles, const TileEntry *tiles2,
                                     const int32_t *n_tiles2, bool pair_down, void *O,
                                     const TensorMap64 &tm_o, cudaStream_t s, bool marks,
-                                    bool pdl) {
+                                    bool pdl, int a_rows) {
   Workspace &w = h->ws;
   TcParams p = {};
   p.mode = TC_EXPERT_GU;
@@ -821,6 +834,7 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
   p.tiles = tiles;
   p.n_mtiles = n_tiles;
   if (h->fp8) {
+    p.a_scale = h->ws.zq_scale;
     p.b_scale = h->gu_scale;
     p.b_scale_ld = h->gu_rows;
   }
@@ -831,12 +845,18 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
   // Single-CTA tiles of 128 rows: measured at least as fast as CTA pairs for
   // the gate/up GEMM (K = l is short, the SwiGLU epilogue is the heavier)
   // and much faster when experts hold few tokens.
-  p.tma_out = h->fp8 ? 0 : 1;
+  p.tma_out = 1;
   p.pdl = pdl && !marks ? 1 : 0;
   cudaError_t e = launch_tc_gemm(tm_a.bytes, h->tm_wgu.bytes, p, h->num_sms, h->num_sms, s,
                                  tm_a32.bytes, h->tm_out_h.bytes);
   h->launches += 1;
   if (e != cudaSuccess) return e;
+  if (h->fp8) {  // H rows -> E4M3 with row scales, the down GEMM's A operand
+    e = launch_quantize_rows_e4m3(static_cast<const __nv_bfloat16 *>(w.H), nullptr, 1, a_rows,
+                                  h->m, w.hq, w.hq_scale, s, !marks);
+    h->launches += 1;
+    if (e != cudaSuccess) return e;
+  }
   if (marks) mark(h, 5, s);
   TcParams pd = {};
   pd.mode = TC_EXPERT_DOWN;
@@ -849,18 +869,19 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
   pd.ld_out = h->l;
   pd.status = w.status;
   if (h->fp8) {
+    pd.a_scale = w.hq_scale;
     pd.b_scale = h->o_scale;
     pd.b_scale_ld = h->l;
   }
-  pd.tma_out = h->fp8 ? 0 : 1;
+  pd.tma_out = 1;
   pd.pdl = marks ? 0 : 1;
   if (pair_down) {
     pd.tiles = tiles2;
     pd.n_mtiles = n_tiles2;
     e = launch_tc_gemm_pair(h->tm_h.bytes, h->tm_wo2.bytes, pd, h->num_sms, s, tm_o.bytes);
   } else {
-    e = launch_tc_gemm(h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms, h->num_sms, s,
-                       h->tm_h32.bytes, tm_o.bytes);
+    e = launch_tc_gemm(h->fp8 ? h->tm_hq.bytes : h->tm_h.bytes, h->tm_wo.bytes, pd, h->num_sms,
+                       h->num_sms, s, h->tm_hq32.bytes, tm_o.bytes);
   }
   h->launches += 1;
   if (e == cudaSuccess && marks) mark(h, 6, s);
@@ -902,8 +923,17 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   Workspace &w = h->ws;
   const int TK = T * h->K;
   mark(h, 0, s);
-  cudaError_t e = run_route(h, x, T, true, s, nullptr, true, w.zp);
+  // the experts' rows: permuted z (bf16, fp32), or its E4M3 copy with row
+  // scales, gathered straight from z through perm
+  cudaError_t e = run_route(h, x, T, true, s, nullptr, true, h->fp8 ? nullptr : w.zp);
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
+  if (h->fp8) {
+    e = launch_quantize_rows_e4m3(static_cast<const __nv_bfloat16 *>(w.z), w.perm, h->K, TK, h->l,
+                                  w.zq, w.zq_scale, s, h->prof_slots == 0);
+    h->launches += 1;
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    mark(h, 4, s);
+  }
   if (h->bf16) {
     // CTA pairs (256-row M-tiles) for the down GEMM when experts average at
     // least 256 rows: the long reduction (K = m) then gains from the smaller
@@ -911,8 +941,8 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
     // more than that.
     const bool pair_down = !h->fp8 && static_cast<int64_t>(T) * h->K >= 256LL * h->N;
     const bool marks = h->prof_slots > 0;
-    e = run_experts_bf16(h, h->tm_zp, h->tm_zp32, w.tiles, w.n_tiles, w.tiles2, w.n_tiles2,
-                         pair_down, w.O, h->tm_out_o, s, marks, true);
+    e = run_experts_bf16(h, h->fp8 ? h->tm_zq : h->tm_zp, h->tm_zq32, w.tiles, w.n_tiles,
+                         w.tiles2, w.n_tiles2, pair_down, w.O, h->tm_out_o, s, marks, true, TK);
     if (e == cudaSuccess) e = run_combine_out_bf16(h, w.O, y, T, s, marks, true);
   } else {
     float *zpf = static_cast<float *>(w.zp);
@@ -1009,7 +1039,7 @@ int lmoe_ep_experts(lmoe_handle h, const void *recv_rows, const int32_t *recv_co
   const bool pair_down = static_cast<int64_t>(R) >= 256LL * h->NE;
   if (e == cudaSuccess)
     e = run_experts_bf16(h, tm_a, tm_a, w.ep_tiles, w.ep_n_tiles, w.ep_tiles2, w.ep_n_tiles2,
-                         pair_down, out_rows, tm_o, s, false, true);
+                         pair_down, out_rows, tm_o, s, false, true, R);
   return cuda_err(e);
 }
 
@@ -1409,6 +1439,13 @@ int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *num
       if (which == 13) { *dev_ptr = h->gu_scale; *numel = static_cast<int64_t>(h->N) * h->gu_rows; }
       if (which == 14) { *dev_ptr = h->w_o8; *numel = btile_rows(h->N, h->l, h->m) * 64; }
       if (which == 15) { *dev_ptr = h->o_scale; *numel = static_cast<int64_t>(h->N) * h->l; }
+      break;
+    case 16: case 17: case 18: case 19:
+      if (!h->fp8) return LMOE_ERR_INVALID_CONFIG;
+      if (which == 16) { *dev_ptr = w.zq; *numel = TK * h->l; }
+      if (which == 17) { *dev_ptr = w.zq_scale; *numel = TK; }
+      if (which == 18) { *dev_ptr = w.hq; *numel = TK * h->m; }
+      if (which == 19) { *dev_ptr = w.hq_scale; *numel = TK; }
       break;
     default: return LMOE_ERR_INVALID_CONFIG;
   }

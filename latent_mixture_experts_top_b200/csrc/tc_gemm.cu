@@ -37,6 +37,12 @@
 //
 // tc_pair_kernel (further down) runs the same forward modes on CTA pairs
 // (tcgen05.mma.cta_group::2, 256 x 256 tiles) with the same epilogue.
+//
+// kF8 (E4M3 routed experts): the expert GEMMs take both operands in E4M3
+// (tcgen05.mma kind::f8f6f4, fp32 accumulation): a K-block is 128 elements,
+// so every row of a staged tile is still 128 bytes and the shared-memory
+// layout, descriptors and pipeline are those of the bf16 tiles; the epilogue
+// multiplies the accumulator by the A row's scale and the weight row's scale.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -56,34 +62,25 @@ constexpr int B_BYTES = TN * TKB * 2;         // 32 KB (16-bit B tile)
 constexpr int TMEM_COLS = 2 * TN;             // two accumulators
 constexpr int NUM_EPI_WARPS = 8;              // two per TMEM lane quarter
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, TN);
+constexpr uint32_t IDESC8 = ptx::idesc_e4m3_f32(TM, TN);
 
-// Pipeline shape.  Default: a STAGES-deep ring of (A, B) tiles filled by TMA
-// and read by the MMA.  kFp8 (weights in E4M3): the same ring carries A and
-// the E4M3 weight tile (16 KB instead of 32 KB), four converter warps move
-// each weight tile to bf16 in the 128-byte-swizzled layout into a second,
-// S2-deep ring, and the MMA reads A from the first ring and B from the
-// second.  A first-ring slot is free once the converters and the MMAs are
-// both done with it.
-template <bool kFp8>
+// Pipeline shape: a STAGES-deep ring of (A, B) tiles filled by TMA and read
+// by the MMA.  Both element types stage 128-byte K-block rows: 64 bf16, or
+// (kF8) 128 E4M3 codes.
+constexpr int TKB8 = 128;  // K-block of the E4M3 GEMM (elements = bytes)
+template <bool kF8>
 struct Cfg {
   static constexpr int STAGES = 4;
-  static constexpr int S2 = kFp8 ? 3 : 0;           // kFp8: converted-B ring
-  static constexpr int B_LOAD = kFp8 ? TN * TKB : B_BYTES;  // weight bytes per TMA stage
-  // kFp8 (weight streaming, few rows per tile): four epilogue warps, one per
-  // TMEM lane quarter covering both column halves, and eight converter
-  // warps, two per scheduler, so that the conversion's latency is hidden.
-  static constexpr int EPI_WARPS = kFp8 ? 4 : NUM_EPI_WARPS;
-  static constexpr int CONV_WARPS = kFp8 ? 8 : 0;
-  static constexpr int NUM_THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
-  static constexpr int RING_BYTES = STAGES * (A_BYTES + B_LOAD) + S2 * B_BYTES;
+  static constexpr int KB = kF8 ? TKB8 : TKB;  // elements per K-block
+  static constexpr int EPI_WARPS = NUM_EPI_WARPS;
+  static constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int RING_BYTES = STAGES * (A_BYTES + B_BYTES);
 };
 
 constexpr int MAX_STAGES = 8;
 struct __align__(8) SmemCtl {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
-  uint64_t conv[MAX_STAGES];    // kFp8: ring-2 slot holds A and the converted B
-  uint64_t conv_empty[MAX_STAGES];  // kFp8: the MMAs have read the ring-2 slot
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
@@ -97,9 +94,9 @@ constexpr int OUT_BOX_BYTES = OUT_BOX * OUT_BOX * 2;                // 2 KB
 constexpr int CTL_BYTES = 1024;                                     // SmemCtl, padded
 constexpr int STAGING_BYTES = NUM_EPI_WARPS * 2 * OUT_BOX_BYTES;    // 32 KB
 static_assert(sizeof(SmemCtl) <= CTL_BYTES, "control block");
-template <bool kFp8>
+template <bool kF8>
 constexpr size_t smem_bytes(bool staging) {
-  return 1024 /*align slack*/ + Cfg<kFp8>::RING_BYTES +
+  return 1024 /*align slack*/ + Cfg<kF8>::RING_BYTES +
          (staging ? CTL_BYTES + STAGING_BYTES : sizeof(SmemCtl));
 }
 static_assert(smem_bytes<false>(true) <= 232448, "shared memory per CTA");
@@ -113,10 +110,11 @@ struct Tile {
   bool b_plain;  // B is a plain row-major matrix (else K-block tiled)
 };
 
-__device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles) {
+__device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles,
+                                           int kb_elems = TKB) {
   Tile tl;
   tl.k0 = 0;
-  tl.nkb = p.Kdim / TKB;
+  tl.nkb = p.Kdim / kb_elems;
   tl.group = 0;
   tl.expert = 0;
   tl.b_plain = false;
@@ -132,12 +130,12 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
     tl.b_plain = true;
     if (p.k_start) {
       tl.k0 = p.k_start[g];
-      tl.nkb = p.k_len[g] / TKB;
+      tl.nkb = p.k_len[g] / kb_elems;
     }
   } else if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
     const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
     tl.a_row = m * TM;
-    tl.b_row = n * (p.Kdim / TKB) * TN;  // first K-block tile of B's N-tile n
+    tl.b_row = n * (p.Kdim / kb_elems) * TN;  // first K-block tile of B's N-tile n
     tl.n_tile = n;
     tl.row_hi = p.M;
   } else {
@@ -145,7 +143,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
     const TileEntry te = p.tiles[mt];
     tl.expert = te.expert;
     tl.a_row = te.row0;
-    tl.b_row = (te.expert * p.n_tiles_n + n) * (p.Kdim / TKB) * TN;
+    tl.b_row = (te.expert * p.n_tiles_n + n) * (p.Kdim / kb_elems) * TN;
     tl.n_tile = n;
     tl.row_hi = te.row_end;
   }
@@ -472,14 +470,12 @@ __device__ __forceinline__ void epi_act_backward(uint32_t taddr, bool valid, con
   }
 }
 
-// ---- epilogues of the FP8-weight variant: the accumulator column c holds
-// 2^-120 times the product with the E4M3 codes (see convert_stage), so it is
-// scaled by the weight row's scale scl[c] times 2^120.
-constexpr float kTwo120 = 1.329227995784916e36f;  // 2^120, exact in f32
-
+// ---- epilogues of the E4M3 GEMM (kF8): the accumulator holds products of
+// E4M3 codes, so column c is multiplied by the A row's scale sa and the
+// weight row's scale scl[c] (both powers of two).
 __device__ __forceinline__ void epi_swiglu_scaled(uint32_t taddr, bool valid,
-                                                  __nv_bfloat16 *row_dst, int hcol0,
-                                                  const float *scl, int half) {
+                                                  __nv_bfloat16 *row_dst, int hcol0, float sa,
+                                                  const float *scl, int half, OutSink *sink) {
 #pragma unroll 1
   for (int c = half * (TN / 128); c < (half + 1) * (TN / 128); ++c) {
     uint32_t g[32], u[32];
@@ -489,99 +485,69 @@ __device__ __forceinline__ void epi_swiglu_scaled(uint32_t taddr, bool valid,
     float h[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      h[j] = silu_bf16out(__uint_as_float(g[j]) * (scl[c * 32 + j] * kTwo120)) *
-             (__uint_as_float(u[j]) * (scl[TN / 2 + c * 32 + j] * kTwo120));
-    if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
+      h[j] = silu_bf16out(__uint_as_float(g[j]) * (sa * scl[c * 32 + j])) *
+             (__uint_as_float(u[j]) * (sa * scl[TN / 2 + c * 32 + j]));
+    if (sink && sink->map) sink_store(*sink, h, hcol0 + c * 32);
+    else if (valid) store_bf16x32(row_dst + hcol0 + c * 32, h);
   }
 }
 
 __device__ __forceinline__ void epi_relu2_scaled(uint32_t taddr, bool valid,
                                                  __nv_bfloat16 *row_dst, int col0, int n_cols,
-                                                 const float *scl, int half) {
+                                                 float sa, const float *scl, int half,
+                                                 OutSink *sink) {
 #pragma unroll 1
   for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
     const int col = col0 + c * 32;
     uint32_t r[32];
     ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
     ptx::tmem_ld_wait();
-    if (!valid || col >= n_cols) continue;
     float h[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const float a = fmaxf(__uint_as_float(r[j]) * (scl[c * 32 + j] * kTwo120), 0.0f);
+      const float a = fmaxf(__uint_as_float(r[j]) * (sa * scl[c * 32 + j]), 0.0f);
       h[j] = a * a;
     }
-    store_bf16x32(row_dst + col, h);
+    if (sink && sink->map) {
+      if (col < n_cols) sink_store(*sink, h, col);
+    } else if (valid && col < n_cols) {
+      store_bf16x32(row_dst + col, h);
+    }
   }
 }
 
 __device__ __forceinline__ void epi_plain_scaled(uint32_t taddr, bool valid,
                                                  __nv_bfloat16 *row_dst, int col0, int n_cols,
-                                                 const float *scl, int half) {
+                                                 float sa, const float *scl, int half,
+                                                 OutSink *sink) {
 #pragma unroll 1
   for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
     const int col = col0 + c * 32;
     uint32_t r[32];
     ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
     ptx::tmem_ld_wait();
-    if (!valid || col >= n_cols) continue;
     float v[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * (scl[c * 32 + j] * kTwo120);
-    store_bf16x32(row_dst + col, v);
-  }
-}
-
-constexpr int CONV_THREADS = 256;  // Cfg<true>::CONV_WARPS * 32
-
-// Converter role (kFp8): moves one stage's E4M3 B tile (256 rows x 64
-// bytes, TMA-loaded without swizzle) into bf16 in the 128-byte-swizzled
-// K-major layout: element (r, k) at byte r*128 + (((k/8) ^ (r%8)) * 16) +
-// (k%8)*2.  No arithmetic conversion: an E4M3 code (sign s, exponent field
-// E, mantissa M) with its sign moved to bit 15 and its 7 magnitude bits to
-// bits 4..10 is the bf16 bit pattern of (its value) * 2^-120 exactly -- for
-// E >= 1 a normal bf16 with exponent field E and mantissa M/8, for E = 0
-// (the E4M3 subnormals M/8 * 2^-6) the bf16 subnormal M/8 * 2^-126.  The
-// epilogue multiplies by the row scale times 2^120.  Each of the 256 threads
-// moves 4 groups of 16 codes; the reads, and each 8-thread phase of the
-// writes, hit distinct banks.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_scaled(uint32_t t) {
-  // t: code 0 in bits 0..7, code 1 in bits 16..23 (other bits zero).
-  // (t << 4) puts the magnitudes at bits 4..10 / 20..26 and the signs at
-  // bits 11 / 27; adding sign * (2^8 - 2^4) moves each sign to bit 15 / 31.
-  return (t << 4) + (t & 0x00800080u) * 240u;
-}
-
-__device__ __forceinline__ void convert_stage(const uint8_t *b8, uint8_t *b16, int ctid) {
-#pragma unroll
-  for (int i = 0; i < 1024 / CONV_THREADS; ++i) {
-    const int item = ctid + CONV_THREADS * i;
-    const int r = item >> 2, j = item & 3;
-    const uint4 q = *reinterpret_cast<const uint4 *>(b8 + r * 64 + j * 16);
-    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-    uint32_t hw[8];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      hw[2 * w] = e4m3x2_to_bf16x2_scaled(__byte_perm(qw[w], 0u, 0x4140));
-      hw[2 * w + 1] = e4m3x2_to_bf16x2_scaled(__byte_perm(qw[w], 0u, 0x4342));
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * (sa * scl[c * 32 + j]);
+    if (sink && sink->map) {
+      if (col < n_cols) sink_store(*sink, v, col);
+    } else if (valid && col < n_cols) {
+      store_bf16x32(row_dst + col, v);
     }
-    const int c0 = 2 * j, sw = r & 7;
-    *reinterpret_cast<uint4 *>(b16 + r * 128 + ((c0 ^ sw) << 4)) =
-        make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *reinterpret_cast<uint4 *>(b16 + r * 128 + (((c0 + 1) ^ sw) << 4)) =
-        make_uint4(hw[4], hw[5], hw[6], hw[7]);
   }
 }
 
 // One tile's epilogue for the calling warp: its 32 accumulator lanes (output
 // rows row = lane's row, valid when inside the tile) and its column halves,
 // by mode.  Shared by the single-CTA and the CTA-pair kernels.
-template <bool kBwd, bool kFp8>
+template <bool kBwd, bool kF8>
 __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl, uint32_t taddr,
                                               int row, bool valid, int col0, int half0,
                                               OutSink &sink) {
   // one epilogue warp per lane quarter covers both halves, two take one each
-  constexpr int kHalfStep = Cfg<kFp8>::EPI_WARPS / 4;
+  constexpr int kHalfStep = Cfg<kF8>::EPI_WARPS / 4;
+  // kF8: the A row's scale (rows past the tile's end are not stored)
+  const float sa = (kF8 && valid) ? p.a_scale[row] : 0.0f;
   for (int half = half0; half < 2; half += kHalfStep) {
     switch (p.mode) {
       case TC_X_FUSED:
@@ -611,11 +577,11 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
         }
         break;
       case TC_EXPERT_GU:
-        if constexpr (kFp8) {
+        if constexpr (kF8) {
           const float *scl = p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0;
           __nv_bfloat16 *hrow = p.out + static_cast<size_t>(row) * p.ld_out;
-          if (p.relu2) epi_relu2_scaled(taddr, valid, hrow, col0, p.n_cols2, scl, half);
-          else epi_swiglu_scaled(taddr, valid, hrow, col0 / 2, scl, half);
+          if (p.relu2) epi_relu2_scaled(taddr, valid, hrow, col0, p.n_cols2, sa, scl, half, &sink);
+          else epi_swiglu_scaled(taddr, valid, hrow, col0 / 2, sa, scl, half, &sink);
         } else if (kBwd && p.raw && p.relu2)
           epi_relu2_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
                         p.out_h + static_cast<size_t>(row) * p.ld_h, col0, p.n_cols2, half);
@@ -633,11 +599,11 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
         if constexpr (kBwd) epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
         break;
       default:  // TC_EXPERT_DOWN, TC_OUT
-        if constexpr (kFp8) {
+        if constexpr (kF8) {
           epi_plain_scaled(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
-                           p.ld_out,
+                           p.ld_out, sa,
                            p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0,
-                           half);
+                           half, &sink);
         } else if (kBwd && p.act_dab)
           epi_act_backward(taddr, valid, p, row, col0, p.ld_out, half);
         else if (kBwd && p.out_f32)
@@ -654,29 +620,25 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
 // kBwd: the instantiation with the backward's epilogues and the TC_WGRAD
 // mode; the forward launches the other one, whose smaller register budget
 // leaves room for the routing kernels that run beside it.
-// kFp8: expert weights in E4M3 (TC_EXPERT_GU / TC_EXPERT_DOWN with b_scale):
-// four more warps convert each stage's weight tile to f16 for the MMA.
-template <bool kBwd, bool kFp8>
-__global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
+// kF8: the expert GEMMs with E4M3 operands (TC_EXPERT_GU / TC_EXPERT_DOWN with
+// a_scale and b_scale): tcgen05.mma kind::f8f6f4 over 128-element K-blocks.
+template <bool kBwd, bool kF8>
+__global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA32, const __grid_constant__ CUtensorMap tmO,
                    const TcParams p) {
-  constexpr int STAGES = Cfg<kFp8>::STAGES;
-  constexpr int S2 = Cfg<kFp8>::S2;
-  constexpr int S2M = S2 > 0 ? S2 : 1;  // ring-2 index arithmetic (kFp8 only)
-  constexpr int B_LOAD = Cfg<kFp8>::B_LOAD;
+  constexpr int STAGES = Cfg<kF8>::STAGES;
+  constexpr int KB = Cfg<kF8>::KB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // [A ring][B ring (E4M3 if kFp8)][kFp8: converted-B ring][control block]
-  // [tma_out: the epilogue warps' staging buffers]
+  // [A ring][B ring][control block][tma_out: the epilogue warps' staging buffers]
   uint8_t *smA = smem;
   uint8_t *smB = smem + STAGES * A_BYTES;
-  uint8_t *smBc = smB + STAGES * B_LOAD;
-  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + Cfg<kFp8>::RING_BYTES);
-  uint8_t *staging = smem + Cfg<kFp8>::RING_BYTES + CTL_BYTES;
-  // TMA stores: the forward instantiation with a bf16-output mode
-  const bool use_tma_out = !kBwd && !kFp8 && p.tma_out != 0;
+  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + Cfg<kF8>::RING_BYTES);
+  uint8_t *staging = smem + Cfg<kF8>::RING_BYTES + CTL_BYTES;
+  // TMA stores: the forward instantiations with a bf16-output mode
+  const bool use_tma_out = !kBwd && p.tma_out != 0;
   volatile int *abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -687,16 +649,11 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&ctl->full[s], 1);
-      // freed by the MMA commit (kFp8: and by each converter warp)
-      ptx::mbar_init(&ctl->empty[s], 1 + Cfg<kFp8>::CONV_WARPS);
-    }
-    for (int s = 0; s < S2; ++s) {
-      ptx::mbar_init(&ctl->conv[s], Cfg<kFp8>::CONV_WARPS);
-      ptx::mbar_init(&ctl->conv_empty[s], 1);
+      ptx::mbar_init(&ctl->empty[s], 1);  // freed by the MMA commit
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&ctl->acc_full[a], 1);
-      ptx::mbar_init(&ctl->acc_empty[a], Cfg<kFp8>::EPI_WARPS);  // one per epilogue warp
+      ptx::mbar_init(&ctl->acc_empty[a], Cfg<kF8>::EPI_WARPS);  // one per epilogue warp
     }
     ptx::mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -704,7 +661,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&tmA);
-    if (kFp8) ptx::prefetch_tmap(&tmA32);
+    if (kF8) ptx::prefetch_tmap(&tmA32);
     ptx::prefetch_tmap(&tmB);
   }
   if (warp == 1) {
@@ -726,7 +683,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(p, t, m_tiles);
+        const Tile tl = decode_tile(p, t, m_tiles, KB);
         for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -735,16 +692,16 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
             ok = false;
             break;
           }
-          const int kx = tl.k0 + kb * TKB;
-          // kFp8 (weight streaming): a tile of at most 32 token rows loads
+          const int kx = tl.k0 + kb * KB;  // elements = bytes for kF8
+          // kF8 (weight streaming): a tile of at most 32 token rows loads
           // only those rows of A (the MMA's other rows are never stored)
-          const bool a32 = kFp8 && tl.row_hi - tl.a_row <= 32;
-          ptx::mbar_arrive_expect_tx(&ctl->full[s], (a32 ? A_BYTES / 4 : A_BYTES) + B_LOAD);
+          const bool a32 = kF8 && tl.row_hi - tl.a_row <= 32;
+          ptx::mbar_arrive_expect_tx(&ctl->full[s], (a32 ? A_BYTES / 4 : A_BYTES) + B_BYTES);
           ptx::tma_load_2d(smA + s * A_BYTES, a32 ? &tmA32 : &tmA, &ctl->full[s], kx, tl.a_row);
           if (tl.b_plain)
-            ptx::tma_load_2d(smB + s * B_LOAD, &tmB, &ctl->full[s], kx, tl.b_row);
+            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kx, tl.b_row);
           else
-            ptx::tma_load_2d(smB + s * B_LOAD, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
+            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
         }
       }
       if (!ok) {  // let every copy still in flight land before the CTA exits
@@ -768,29 +725,29 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * TN;
-        const int nkb = decode_tile(p, t, m_tiles).nkb;
+        const int nkb = decode_tile(p, t, m_tiles, KB).nkb;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES, s2 = it % S2M;
-          const uint32_t ph = (it / STAGES) & 1, ph2 = (it / S2M) & 1;
-          // kFp8: the converted B of this K-block (its A landed before it)
-          if (!ptx::mbar_wait(kFp8 ? &ctl->conv[s2] : &ctl->full[s], kFp8 ? ph2 : ph,
-                              abort_flag)) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!ptx::mbar_wait(&ctl->full[s], ph, abort_flag)) {
             record_failure(p, ctl, DEV_TIMEOUT_MMA);
             ok = false;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(smA + s * A_BYTES);
-          const uint32_t b_addr =
-              ptx::smem_u32(kFp8 ? smBc + s2 * B_BYTES : smB + s * B_LOAD);
+          const uint32_t b_addr = ptx::smem_u32(smB + s * B_BYTES);
+          // four MMAs per K-block: K = 16 bf16 or 32 E4M3 elements, 32 bytes each
 #pragma unroll
-          for (int k = 0; k < TKB / 16; ++k) {
-            ptx::mma_bf16(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
-                          ptx::smem_desc_sw128(b_addr + k * 32), IDESC, (kb | k) != 0);
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (kF8)
+              ptx::mma_e4m3(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
+                            ptx::smem_desc_sw128(b_addr + k * 32), IDESC8, (kb | k) != 0);
+            else
+              ptx::mma_bf16(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
+                            ptx::smem_desc_sw128(b_addr + k * 32), IDESC, (kb | k) != 0);
           }
-          // the stage (kFp8: and the converted-B slot) is free once these MMAs finish
-          ptx::mma_commit(&ctl->empty[s]);
-          if constexpr (kFp8) ptx::mma_commit(&ctl->conv_empty[s2]);
+          ptx::mma_commit(&ctl->empty[s]);  // the stage is free once these MMAs finish
         }
         if (!ok) break;
         ptx::mma_commit(&ctl->acc_full[acc]);  // accumulator ready for the epilogue
@@ -802,37 +759,6 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
     }
     // every MMA is issued: the next kernel of the stream may be scheduled
     if (lane == 0) griddep_launch_dependents();
-  } else if (kFp8 && warp >= 2 + Cfg<kFp8>::EPI_WARPS) {
-    // ------------------------------------------------------------ converters
-    const int ctid = threadIdx.x - 32 * (2 + Cfg<kFp8>::EPI_WARPS);
-    int it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const int nkb = decode_tile(p, t, m_tiles).nkb;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % STAGES, s2 = it % S2M;
-        const uint32_t ph = (it / STAGES) & 1, ph2 = (it / S2M) & 1;
-        int w_ok = 1;
-        if (lane == 0) {  // converted-B slot free, then this stage's tiles landed
-          w_ok = ptx::mbar_wait(&ctl->conv_empty[s2], ph2 ^ 1, abort_flag) ? 1 : 0;
-          if (w_ok) w_ok = ptx::mbar_wait(&ctl->full[s], ph, abort_flag) ? 1 : 0;
-        }
-        w_ok = __shfl_sync(0xFFFFFFFFu, w_ok, 0);
-        if (!w_ok) {
-          if (lane == 0) record_failure(p, ctl, DEV_TIMEOUT_PRODUCER);
-          ok = false;
-          break;
-        }
-        convert_stage(smB + s * B_LOAD, smBc + s2 * B_BYTES, ctid);
-        // generic-proxy writes -> visible to the tensor core's async-proxy reads
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(&ctl->conv[s2]);
-          ptx::mbar_arrive(&ctl->empty[s]);  // done with the stage's E4M3 tile
-        }
-      }
-    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quarter this warp may access
@@ -860,7 +786,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      const Tile tl = decode_tile(p, t, m_tiles);
+      const Tile tl = decode_tile(p, t, m_tiles, KB);
       const int row = tl.a_row + row_in_tile;
       const bool valid = row < tl.row_hi;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
@@ -869,7 +795,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::NUM_THREADS, 1)
       // tile's rows past its expert's end belong to the next tile.
       sink.y = tl.a_row + q * 32;
       sink.map = (use_tma_out && sink.y + 31 < tl.row_hi) ? &tmO : nullptr;
-      epilogue_tile<kBwd, kFp8>(p, tl, taddr, row, valid, col0, half0, sink);
+      epilogue_tile<kBwd, kF8>(p, tl, taddr, row, valid, col0, half0, sink);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
@@ -1234,12 +1160,12 @@ int make_tmap_u8(void *tmap_out, const void *base, int64_t rows, int64_t cols,
   if ((reinterpret_cast<uintptr_t>(base) & 15) || row_stride_bytes % 16) return -1;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(TKB), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(TKB8), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r =
       fn(reinterpret_cast<CUtensorMap *>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
          const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -1;
 }
@@ -1261,16 +1187,16 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(tc_gemm_kernel<false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes<true>(false)));
+                               static_cast<int>(smem_bytes<true>(true)));
     if (e != cudaSuccess) return e;
     attr_done = dev;
   }
   const bool bwd = p.mode == TC_WGRAD || p.raw || p.act_dab || p.out_f32 || p.out_h;
   const bool fp8 = p.b_scale != nullptr;
-  if (fp8 && (bwd || (p.mode != TC_EXPERT_GU && p.mode != TC_EXPERT_DOWN)))
+  if (fp8 && (bwd || !p.a_scale || (p.mode != TC_EXPERT_GU && p.mode != TC_EXPERT_DOWN)))
     return cudaErrorInvalidValue;
-  if (p.tma_out && (bwd || fp8 || p.mode == TC_WGRAD || !tmapOut)) return cudaErrorInvalidValue;
-  if (p.Kdim % TKB || p.Kdim <= 0) return cudaErrorInvalidValue;
+  if (p.tma_out && (bwd || p.mode == TC_WGRAD || !tmapOut)) return cudaErrorInvalidValue;
+  if (p.Kdim % (fp8 ? TKB8 : TKB) || p.Kdim <= 0) return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
   if (fp8 && !tmapA32) return cudaErrorInvalidValue;
@@ -1283,7 +1209,7 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   cudaError_t e;
   if (fp8)
     e = launch_ex(tc_gemm_kernel<false, true>, dim3(grid), dim3(Cfg<true>::NUM_THREADS),
-                  smem_bytes<true>(false), s, pdl, a, b, a32, o, p);
+                  smem_bytes<true>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
   else if (bwd)
     e = launch_ex(tc_gemm_kernel<true, false>, dim3(grid), dim3(Cfg<false>::NUM_THREADS),
                   smem_bytes<false>(false), s, pdl, a, b, a32, o, p);

@@ -1,12 +1,18 @@
-"""GPU checks of the E4M3 routed-expert weights (LMOE_WEIGHTS_FP8).
+"""GPU checks of the E4M3 routed experts (LMOE_WEIGHTS_FP8): both operands
+of the expert GEMMs in E4M3 with power-of-two row scales.
 
-1. The library's codes and row scales, decoded on the host from the E4M3
-   definition, equal the oracle's quantisation of the same bf16 weights
+1. The library's weight codes and row scales, decoded on the host from the
+   E4M3 definition, equal the oracle's quantisation of the same bf16 weights
    bit for bit (both round W / s to nearest-even with saturation, s a power
    of two, so there is one right answer).
-2. The layer output matches the fp64 oracle run with the dequantised expert
-   weights W' = E4M3(W / s) s and every other weight widened from bf16
-   (tolerance 2e-2, the bf16 mode's: the GPU computes exactly with W').
+2. The same holds for the activation rows the library quantises on the fly
+   (each expert input row z, each hidden row h), taken from the library's
+   own bf16 z and H: the quantiser sees the same values on both sides.
+3. The layer output matches the fp64 oracle run with the dequantised expert
+   weights, every other weight widened from bf16 and act_fp8 (z and h
+   quantised per row); tolerance 2e-2, the bf16 mode's (the oracle quantises
+   its fp64 z and h, the library its bf16-rounded ones, so a code may differ
+   by one step).
 """
 from dataclasses import replace
 
@@ -23,8 +29,8 @@ pytestmark = pytest.mark.gpu
 MID_FP8 = configs.LayerConfig("mid_fp8_T300_d512_l256_m256_N32_K8", T=300, d=512, m=256,
                               n_experts=16, top_k=4, alpha=2, n_shared=1, m_shared=256,
                               variant="acc", weights="fp8")
-MID_RELU2_FP8 = replace(MID_FP8, name="mid_relu2_fp8_T300_d512_l256_m192_N32_K8", m=192,
-                        m_shared=192, activation="relu2")
+MID_RELU2_FP8 = replace(MID_FP8, name="mid_relu2_fp8_T300_d512_l256_m384_N32_K8", m=384,
+                        m_shared=384, activation="relu2")
 
 
 def _e4m3_table():
@@ -42,8 +48,8 @@ def _e4m3_table():
 
 
 def _detile(codes, groups, rows, cols):
-    nt, kbc = (rows + 255) // 256, cols // 64
-    a = codes.reshape(groups, nt, kbc, 256, 64).transpose(0, 1, 3, 2, 4)
+    nt, kbc = (rows + 255) // 256, cols // 128
+    a = codes.reshape(groups, nt, kbc, 256, 128).transpose(0, 1, 3, 2, 4)
     return a.reshape(groups, nt * 256, cols)[:, :rows]
 
 
@@ -108,7 +114,8 @@ def _fp8_layer_case(cfg, n_sample):
     L = oracle.Layer(w_router=wide["w_router"], b_router=bias, w_down=wide["w_down"],
                      w_up=wide["w_up"], w_gate=wide["w_gate"], w_upx=wide["w_upx"],
                      w_out=wide["w_out"], s_gate=wide["s_gate"], s_up=wide["s_up"],
-                     s_out=wide["s_out"], k_active=cfg.k_active, activation=cfg.activation)
+                     s_out=wide["s_out"], k_active=cfg.k_active, activation=cfg.activation,
+                     act_fp8=True)
     x64 = wide["x"]
     ids_g = ids.cpu().numpy()
     s_ref = oracle.router_logits(L, x64)
@@ -120,6 +127,34 @@ def _fp8_layer_case(cfg, n_sample):
           f"flipped {flipped.sum()}")
     layer.close()
     assert err <= pu.TOL_BF16
+
+
+@pytest.mark.parametrize("cfg", [MID_FP8, MID_RELU2_FP8], ids=lambda c: c.name)
+def test_activation_codes_equal_the_oracle_quantisation(cfg):
+    """The E4M3 rows the expert GEMMs read, from the library's own z (in
+    dispatch order) and hidden H: codes and row scales bit for bit."""
+    lm = _lmoe()
+    inp = synth.make_inputs(cfg, 0, "cuda")
+    layer = lm.LatentMoELayer(cfg, inp)
+    layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    T, K, l, m = cfg.T, cfg.k_active, cfg.l, cfg.m
+    TK = T * K
+    table = _e4m3_table()
+    z = layer.debug_tensor(1, torch.bfloat16, (T, l)).view(torch.int16).cpu().numpy().view(np.uint16)
+    perm = layer.debug_tensor(9, torch.int32, (TK,)).cpu().numpy()
+    H = layer.debug_tensor(3, torch.bfloat16, (TK, m)).view(torch.int16).cpu().numpy().view(np.uint16)
+    zq = table[layer.debug_tensor(16, torch.uint8, (TK, l)).cpu().numpy()]
+    zs = layer.debug_tensor(17, torch.float32, (TK,)).cpu().numpy().astype(np.float64)
+    hq = table[layer.debug_tensor(18, torch.uint8, (TK, m)).cpu().numpy()]
+    hs = layer.debug_tensor(19, torch.float32, (TK,)).cpu().numpy().astype(np.float64)
+    zref, zref_s = oracle.fp8_rows(z[perm // K])
+    np.testing.assert_array_equal(zq * zs[:, None], zref)
+    np.testing.assert_array_equal(zs, zref_s)
+    href, href_s = oracle.fp8_rows(H)
+    np.testing.assert_array_equal(hq * hs[:, None], href)
+    np.testing.assert_array_equal(hs, href_s)
+    layer.close()
 
 
 def test_fp8_mid_swiglu_all_tokens():

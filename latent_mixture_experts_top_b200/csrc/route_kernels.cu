@@ -260,6 +260,95 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
 }
 
 // ---------------------------------------------------------------- fused routing
+// Phase 2 with one warp per expert row (any number of warps): lane j takes a
+// contiguous run of the row's chunk counts, the warp scans the runs' sums, and
+// each count becomes the exclusive prefix within its row, as in
+// scan_and_tables.  A row costs two short passes over one run per lane
+// instead of one thread walking the whole row in dependent groups.  Expert
+// totals go through shared memory to the block-wide scans of offsets and
+// tile starts.  N <= 1024.
+__device__ void scan_and_tables_warps(int32_t *__restrict__ counts, int n_chunks, int N,
+                                      int32_t *__restrict__ offsets, TileEntry *__restrict__ tiles,
+                                      int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+                                      TileEntry *__restrict__ tiles2,
+                                      int32_t *__restrict__ n_tiles2, int tile_m2,
+                                      int max_tiles2) {
+  __shared__ int totals[1024];
+  __shared__ int warp_sums[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int ncp = (n_chunks + 3) & ~3;
+  const int nv = ncp / 4;                       // int4 vectors per row
+  const int per = (nv + 31) / 32;               // vectors per lane (contiguous)
+  for (int e = warp; e < N; e += nwarps) {
+    int4 *row = reinterpret_cast<int4 *>(counts + static_cast<size_t>(e) * ncp);
+    const int v0 = lane * per, v1 = min(nv, v0 + per);
+    // pass 1: the lane's sum (its run of chunk counts; entries past n_chunks
+    // are row padding and count as zero)
+    int sum = 0;
+    for (int v = v0; v < v1; ++v) {
+      const int4 q = __ldcg(row + v);
+      const int c = 4 * v;
+      sum += (c + 0 < n_chunks ? q.x : 0) + (c + 1 < n_chunks ? q.y : 0) +
+             (c + 2 < n_chunks ? q.z : 0) + (c + 3 < n_chunks ? q.w : 0);
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += y;
+    }
+    // pass 2: each count becomes the number of pairs in the chunks before it
+    int run = incl - sum;
+    for (int v = v0; v < v1; ++v) {
+      const int4 q = __ldcg(row + v);
+      const int c = 4 * v;
+      int4 o;
+      o.x = run; run += c + 0 < n_chunks ? q.x : 0;
+      o.y = run; run += c + 1 < n_chunks ? q.y : 0;
+      o.z = run; run += c + 2 < n_chunks ? q.z : 0;
+      o.w = run; run += c + 3 < n_chunks ? q.w : 0;
+      row[v] = o;
+    }
+    if (lane == 31) totals[e] = incl;
+  }
+  __syncthreads();
+  // experts e0 .. e0+3 per thread, as in scan_and_tables
+  const int e0 = threadIdx.x * kScanPerThread;
+  int tot[kScanPerThread], mt[kScanPerThread], mt2[kScanPerThread];
+  int my_tot = 0, my_mt = 0, my_mt2 = 0;
+#pragma unroll
+  for (int i = 0; i < kScanPerThread; ++i) {
+    const int e = e0 + i;
+    tot[i] = e < N ? totals[e] : 0;
+    mt[i] = (tot[i] + tile_m - 1) / tile_m;
+    mt2[i] = tiles2 ? (tot[i] + tile_m2 - 1) / tile_m2 : 0;
+    my_tot += tot[i];
+    my_mt += mt[i];
+    my_mt2 += mt2[i];
+  }
+  int all = 0, all_tiles = 0, all_tiles2 = 0;
+  int off = block_exclusive_scan(my_tot, warp_sums, &all);
+  int tstart = block_exclusive_scan(my_mt, warp_sums, &all_tiles);
+  int tstart2 = block_exclusive_scan(my_mt2, warp_sums, &all_tiles2);
+#pragma unroll
+  for (int i = 0; i < kScanPerThread; ++i) {
+    const int e = e0 + i;
+    if (e < N) {
+      offsets[e] = off;
+      write_tiles(tiles, tstart, max_tiles, e, off, tot[i], tile_m);
+      if (tiles2) write_tiles(tiles2, tstart2, max_tiles2, e, off, tot[i], tile_m2);
+    }
+    off += tot[i];
+    tstart += mt[i];
+    tstart2 += mt2[i];
+  }
+  if (threadIdx.x == 0) {
+    offsets[N] = all;
+    *n_tiles = min(all_tiles, max_tiles);
+    if (tiles2) *n_tiles2 = min(all_tiles2, max_tiles2);
+  }
+}
+
 // Top-K', dispatch histogram and scan in one launch.  Block c takes the
 // chunk of `chunk` tokens starting at c * chunk, one warp per token (the
 // selection is a chain of dependent warp reductions, so every token runs in
@@ -295,8 +384,8 @@ __global__ void __launch_bounds__(1024) route_select_kernel(
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  scan_and_tables(counts, n_chunks, N, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
-                  n_tiles2, tile_m2, max_tiles2);
+  scan_and_tables_warps(counts, n_chunks, N, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
+                        n_tiles2, tile_m2, max_tiles2);
   if (threadIdx.x == 0) *arrivals = 0;
 }
 
@@ -338,16 +427,26 @@ __global__ void __launch_bounds__(256) scatter_permute_kernel(
   if (tok) {
     const uint32_t lt = (1u << lane) - 1u;
     const int ncp = (n_chunks + 3) & ~3;
-    for (int k = 0; k < K; ++k) {
-      const int e = my_ids[k];
-      const int p = offsets[e] + counts[static_cast<size_t>(e) * ncp + c] + wbase[w * N + e] +
-                    __popc(mask[w * N + e] & lt);
-      ppos[threadIdx.x * K + k] = p;
-      if (share == 0) {
-        const int flat = t * K + k;
-        perm[p] = flat;
-        pos[flat] = p;
-        row_expert[p] = e;
+    for (int k0 = 0; k0 < K; k0 += 8) {  // eight slots' loads in flight, then the stores
+      int ev[8], base[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ev[j] = k0 + j < K ? my_ids[k0 + j] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        base[j] = k0 + j < K ? offsets[ev[j]] + counts[static_cast<size_t>(ev[j]) * ncp + c] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int k = k0 + j;
+        if (k >= K) break;
+        const int e = ev[j];
+        const int p = base[j] + wbase[w * N + e] + __popc(mask[w * N + e] & lt);
+        ppos[threadIdx.x * K + k] = p;
+        if (share == 0) {
+          const int flat = t * K + k;
+          perm[p] = flat;
+          pos[flat] = p;
+          row_expert[p] = e;
+        }
       }
     }
   }
@@ -355,15 +454,15 @@ __global__ void __launch_bounds__(256) scatter_permute_kernel(
   __syncthreads();
   // The share's pairs are i = share, share + S, ...; item j = (its q-th pair,
   // vector v) with q = j / vecs_per_row: consecutive threads copy consecutive
-  // 16-byte vectors of a row, four items in flight per thread.
+  // 16-byte vectors of a row, eight items in flight per thread.
   const int npairs = min(chunk, T - c * chunk) * K;
   const int my_pairs = npairs > share ? (npairs - share + S - 1) / S : 0;
   const int items = my_pairs * vecs_per_row;
-  for (int j0 = threadIdx.x; j0 < items; j0 += 4 * blockDim.x) {
-    uint4 v[4];
-    int64_t dst_at[4];
+  for (int j0 = threadIdx.x; j0 < items; j0 += 8 * blockDim.x) {
+    uint4 v[8];
+    int64_t dst_at[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       const int j = j0 + u * blockDim.x;
       dst_at[u] = -1;
       if (j < items) {
@@ -374,7 +473,7 @@ __global__ void __launch_bounds__(256) scatter_permute_kernel(
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 8; ++u)
       if (dst_at[u] >= 0) dst[dst_at[u]] = v[u];
   }
 }

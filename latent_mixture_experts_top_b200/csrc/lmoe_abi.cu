@@ -696,7 +696,9 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       q.n_tile_base = (h->n_pad + h->l_pad) / kTileN;
       q.n_tiles_n = shared_tiles_n;
       // direct stores: the smaller shared-memory footprint lets the routing
-      // kernels run beside this launch's CTAs
+      // kernels run beside this launch's CTAs.  The paired launch is capped at
+      // a third of the SMs (each CTA pair loops over its tiles), so that the
+      // routing kernels and the first expert tiles find free SMs.
       q.tma_out = 0;
       if (shared_raw) {
         q.raw = 1;
@@ -709,7 +711,9 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
         e = shared_raw ? launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, q, h->num_sms,
                                         m_tiles * shared_tiles_n, h->side)
                        : launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, q,
-                                             m_tiles2 * shared_tiles_n, h->side);
+                                             std::min(m_tiles2 * shared_tiles_n,
+                                                      std::max(1, h->num_sms / 3)),
+                                             h->side);
       if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
       h->launches += 1;
     }

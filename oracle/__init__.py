@@ -55,7 +55,7 @@ class _Layer(C.Structure):
         ("w_down", C.c_void_p), ("w_up", C.c_void_p),
         ("w_gate", C.c_void_p), ("w_upx", C.c_void_p), ("w_out", C.c_void_p),
         ("s_gate", C.c_void_p), ("s_up", C.c_void_p), ("s_out", C.c_void_p),
-        ("act_fp8", C.c_int32),
+        ("act_quant", C.c_int32),
     ]
 
 
@@ -87,6 +87,8 @@ def _load():
             lib.oracle_backward.restype = C.c_int
             lib.oracle_fp8_rows.argtypes = [P, I32, I64, I32, P, P]
             lib.oracle_fp8_rows.restype = None
+            lib.oracle_nvfp4_rows.argtypes = [P, I32, I64, I32, P, P, P]
+            lib.oracle_nvfp4_rows.restype = I32
             lib.oracle_threads.argtypes = []
             lib.oracle_threads.restype = C.c_int
             _lib = lib
@@ -137,11 +139,16 @@ class Layer:
     and each expert's hidden vector quantised with the weight rows' rule (a
     power-of-two scale, the smallest that brings the largest magnitude
     within 448); the backward is then not defined.
+    act_fp4: the same with NVFP4 activations (nvfp4_rows' rule: E2M1 codes,
+    an E4M3 scale per 16 elements, a power-of-two row scale); l and m must
+    be multiples of 16.
     """
 
     def __init__(self, *, w_router, b_router, w_down, w_up, w_gate, w_upx,
                  w_out, s_gate, s_up, s_out, k_active, activation="swiglu",
-                 act_fp8=False):
+                 act_fp8=False, act_fp4=False):
+        if act_fp8 and act_fp4:
+            raise ValueError("act_fp8 and act_fp4 are exclusive")
         if activation not in ("swiglu", "relu2"):
             raise ValueError("activation must be 'swiglu' or 'relu2'")
         self.activation = activation
@@ -175,8 +182,9 @@ class Layer:
                          _ptr(k["w_router"]), _ptr(self.b_router), _ptr(k["w_down"]),
                          _ptr(k["w_up"]), _ptr(k["w_gate"]), _ptr(k["w_upx"]),
                          _ptr(k["w_out"]), _ptr(k["s_gate"]), _ptr(k["s_up"]),
-                         _ptr(k["s_out"]), 1 if act_fp8 else 0)
+                         _ptr(k["s_out"]), 1 if act_fp8 else (2 if act_fp4 else 0))
         self.act_fp8 = bool(act_fp8)
+        self.act_fp4 = bool(act_fp4)
 
     @property
     def cref(self):
@@ -343,6 +351,26 @@ def fp8_rows(w):
     sc = np.empty(rows, dtype=np.float64)
     _load().oracle_fp8_rows(_ptr(w), code, rows, cols, _ptr(wq), _ptr(sc))
     return wq, sc
+
+
+def nvfp4_rows(w):
+    """Row-wise NVFP4 quantisation (E2M1 codes, an E4M3 scale per 16
+    elements, a power-of-two row scale; see the C source): returns (W'
+    dequantised, float64, same shape; row scales [rows]; block scales
+    [rows][cols/16])."""
+    w = np.ascontiguousarray(w)
+    code = _dtype_code(w)
+    cols = w.shape[-1]
+    if cols % 16:
+        raise ValueError("NVFP4 rows need a multiple of 16 columns")
+    rows = w.size // cols
+    wq = np.empty(w.shape, dtype=np.float64)
+    sc = np.empty(rows, dtype=np.float64)
+    bs = np.empty((rows, cols // 16), dtype=np.float64)
+    rc = _load().oracle_nvfp4_rows(_ptr(w), code, rows, cols, _ptr(wq), _ptr(sc), _ptr(bs))
+    if rc != 0:
+        raise ValueError(f"oracle_nvfp4_rows failed ({rc})")
+    return wq, sc, bs
 
 
 def threads() -> int:

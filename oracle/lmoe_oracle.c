@@ -55,6 +55,7 @@
 enum { ODT_F32 = 0, ODT_BF16 = 1, ODT_F64 = 2 };
 
 enum { OACT_SWIGLU = 0, OACT_RELU2 = 1 };
+enum { OQ_NONE = 0, OQ_E4M3 = 1, OQ_NVFP4 = 2 };  /* activation quantisation */
 
 typedef struct {
   int32_t d, l, m, n_routed, k_active, n_shared, m_shared;
@@ -70,7 +71,8 @@ typedef struct {
   const void *s_gate;        /* [n_s][m_s][d] */
   const void *s_up;          /* [n_s][m_s][d] */
   const void *s_out;         /* [n_s][d][m_s] */
-  int32_t act_fp8;           /* 1: routed experts run on E4M3 activations (see q_vec_e4m3) */
+  int32_t act_quant;         /* routed experts' activations: OQ_NONE, OQ_E4M3 (q_vec_e4m3)
+                                or OQ_NVFP4 (q_vec_nvfp4) */
 } oracle_layer;
 
 /* Exact widening of one stored element to double. */
@@ -106,10 +108,11 @@ static double relu2(double a) { return a > 0.0 ? a * a : 0.0; }
  * Squared ReLU: out = W_o (relu(W_u v))^2  ([Explained], the Expert class:
  * up, relu, square, down).
  * W_g, W_u: [hid][in_w] at element offset off_in; W_o: [out_w][hid] at off_out. */
-static void q_vec_e4m3(double *v, int n);
+static void q_act(int mode, double *v, int n);
 
-/* quant_hidden: the hidden vector is replaced by its E4M3 row quantisation
- * before the down-projection (routed experts with act_fp8). */
+/* quant_hidden: the hidden vector is replaced by its row quantisation in
+ * that mode (OQ_E4M3 or OQ_NVFP4) before the down-projection (the routed
+ * experts when act_quant is set). */
 static void swiglu_ffn(const oracle_layer *L, const void *Wg, const void *Wu,
                        const void *Wo, size_t off_in, size_t off_out, int in_w,
                        int hid, int out_w, const double *v, double *out,
@@ -123,7 +126,7 @@ static void swiglu_ffn(const oracle_layer *L, const void *Wg, const void *Wu,
     matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
     for (int j = 0; j < hid; ++j) a[j] = silu(a[j]) * b[j];
   }
-  if (quant_hidden) q_vec_e4m3(a, hid);
+  if (quant_hidden) q_act(quant_hidden, a, hid);
   matvec(Wo, L->dtype, off_out, out_w, hid, a, out);
 }
 
@@ -230,7 +233,7 @@ void oracle_down(const oracle_layer *L, const void *x, int64_t t, double *z) {
 void oracle_expert(const oracle_layer *L, int e, const double *z, double *out) {
   double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)L->m);
   swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * L->m * L->l,
-             (size_t)e * L->l * L->m, L->l, L->m, L->l, z, out, scratch, L->act_fp8);
+             (size_t)e * L->l * L->m, L->l, L->m, L->l, z, out, scratch, L->act_quant);
   free(scratch);
 }
 
@@ -264,6 +267,8 @@ int oracle_forward(const oracle_layer *L, const void *x, int64_t T,
                    double *y, int32_t *ids_out, double *gates_out) {
   const int d = L->d, l = L->l, m = L->m, N = L->n_routed, K = L->k_active;
   if (K < 1 || K > N || l < 1 || d < 1 || m < 1) return -1;
+  if (L->act_quant < OQ_NONE || L->act_quant > OQ_NVFP4) return -1;
+  if (L->act_quant == OQ_NVFP4 && (l % 16 || m % 16)) return -1;  /* whole 16-blocks */
   int err = 0;
 #pragma omp parallel
   {
@@ -291,12 +296,12 @@ int oracle_forward(const oracle_layer *L, const void *x, int64_t T,
       }
       for (int i = 0; i < d; ++i) xv[i] = elem(x, L->dtype, (size_t)t * d + i);
       matvec(L->w_down, L->dtype, 0, l, d, xv, z);
-      if (L->act_fp8) q_vec_e4m3(z, l);  /* the experts read z in E4M3 */
+      if (L->act_quant) q_act(L->act_quant, z, l);  /* the experts read z quantised */
       for (int i = 0; i < l; ++i) u[i] = 0.0;
       for (int k = 0; k < K; ++k) { /* slot loop, in slot order */
         const int e = ids[k];
         swiglu_ffn(L, L->w_gate, L->w_upx, L->w_out, (size_t)e * m * l,
-                   (size_t)e * l * m, l, m, l, z, eo, scratch, L->act_fp8);
+                   (size_t)e * l * m, l, m, l, z, eo, scratch, L->act_quant);
         for (int i = 0; i < l; ++i) u[i] += g[k] * eo[i];
       }
       double *yr = y + n * d;
@@ -429,7 +434,7 @@ int oracle_backward(const oracle_layer *L, const void *x, int64_t T,
   const int ns = L->n_shared, ms = L->m_shared > 0 ? L->m_shared : 1;
   const int relu = L->activation == OACT_RELU2;
   if (K < 1 || K > N || l < 1 || d < 1 || m < 1) return -1;
-  if (L->act_fp8) return -3;  /* no gradient through the activation quantiser */
+  if (L->act_quant) return -3;  /* no gradient through the activation quantiser */
   /* per-token and per-slot records for the weight-gradient sums */
   double *X = (double *)malloc(sizeof(double) * (size_t)n_tok * d);
   double *Z = (double *)malloc(sizeof(double) * (size_t)n_tok * l);
@@ -684,7 +689,7 @@ void oracle_fp8_rows(const void *W, int dt, int64_t rows, int cols, double *Wq,
   }
 }
 
-/* ---- E4M3 activations (act_fp8; a reading chosen here, the pages give no
+/* ---- E4M3 activations (act_quant = OQ_E4M3; a reading chosen here, the pages give no
  * FP8 activation recipe): the same rule as the weight rows, applied to each
  * activation vector the routed experts multiply -- a token's z (its row of
  * the expert GEMMs' first operand) and each expert's hidden h (its row of the
@@ -697,6 +702,114 @@ static void q_vec_e4m3(double *v, int n) {
     if (fabs(v[i]) > amax) amax = fabs(v[i]);
   const double s = e4m3_row_scale(amax);
   for (int i = 0; i < n; ++i) v[i] = e4m3_round(v[i] / s) * s;
+}
+
+/* ---- NVFP4 (a reading chosen here: the pages say only that the models were
+ * pretrained in NVFP4; the format is NVIDIA's published 4-bit floating
+ * point).  Elements are E2M1 -- 1 sign bit, 2 exponent bits with bias 1, 1
+ * mantissa bit, magnitudes 0, 0.5, 1, 1.5 (subnormal 0.5 and normals
+ * 2^(E-1) (1 + M/2) for E = 1..3) up to 6 -- and every run of 16 consecutive
+ * elements of a row (along the reduction dimension of the GEMM that reads
+ * the row) shares one E4M3 block scale.  The second-level scale is taken per
+ * row: s_r, the smallest power of two with amax_r <= 6 * 448 * s_r, so that
+ * every block scale falls in E4M3's range.  Block j of the row gets
+ *   b_j = E4M3(amax_j / (6 s_r)),
+ * each of its elements the code q = E2M1(x / (b_j s_r)) (0 for the whole
+ * block when b_j = 0), and the value the layer uses is q b_j s_r.  Both
+ * divisions decide codes, so they are taken in IEEE single precision (round
+ * to nearest) on the elements' single-precision values: the precision the
+ * GPU's quantisers take them in.  (b_j s_r is exact in single precision: a
+ * 4-significant-bit value times a power of two.)  E2M1 rounding is to
+ * nearest, ties to the even mantissa, and magnitudes above 6 saturate. */
+static double e2m1_round(double v) {
+  const double a = fabs(v);
+  double r;
+  if (a >= 6.0) {
+    r = 6.0;
+  } else {
+    /* grid spacing: 0.5 below 2 (0, 0.5, 1, 1.5), 1 in [2, 4), 2 in [4, 6] */
+    const double q = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);
+    const double n = a / q;   /* exact */
+    double k = floor(n);
+    const double frac = n - k;
+    /* an even k is an even mantissa on every segment of the grid */
+    if (frac > 0.5 || (frac == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0;
+    r = k * q;
+  }
+  return v < 0.0 ? -r : r;
+}
+
+/* The second-level row scale: the smallest power of two s with
+ * amax <= 2688 s (2688 = 6 * 448), 1 for a row of zeros. */
+static double nvfp4_row_scale(double amax) {
+  int e = 0;
+  if (amax > 0.0) {
+    e = (int)ceil(log2(amax / 2688.0));
+    while (ldexp(2688.0, e) < amax) ++e;
+    while (e > -200 && ldexp(2688.0, e - 1) >= amax) --e;
+  }
+  return ldexp(1.0, e);
+}
+
+/* One row of n (a multiple of 16) single-precision values -> the values the
+ * layer uses (out), the row scale and the n/16 block scales. */
+static void nvfp4_row(const float *x, int n, double *out, double *row_scale,
+                      double *block_scales) {
+  double amax = 0.0;
+  for (int i = 0; i < n; ++i)
+    if (fabs((double)x[i]) > amax) amax = fabs((double)x[i]);
+  const double sr = nvfp4_row_scale(amax);
+  *row_scale = sr;
+  const float six_sr = (float)(6.0 * sr);
+  for (int j = 0; j < n / 16; ++j) {
+    float am = 0.0f;
+    for (int i = 16 * j; i < 16 * j + 16; ++i)
+      if (fabsf(x[i]) > am) am = fabsf(x[i]);
+    const float t = am / six_sr;                         /* single precision */
+    const double b = e4m3_round((double)t);
+    if (block_scales) block_scales[j] = b;
+    const float den = (float)(b * sr);                   /* exact */
+    for (int i = 16 * j; i < 16 * j + 16; ++i) {
+      if (b == 0.0) { out[i] = 0.0; continue; }
+      const float y = x[i] / den;                        /* single precision */
+      out[i] = e2m1_round((double)y) * b * sr;
+    }
+  }
+}
+
+/* W [rows][cols] (any element type, cols a multiple of 16) -> W' (double),
+ * the row scales [rows] and the block scales [rows][cols/16].  -1 when cols
+ * is not a multiple of 16. */
+int oracle_nvfp4_rows(const void *W, int dt, int64_t rows, int cols, double *Wq,
+                      double *row_scales, double *block_scales) {
+  if (cols <= 0 || cols % 16) return -1;
+#pragma omp parallel
+  {
+    float *xf = (float *)malloc(sizeof(float) * (size_t)cols);
+#pragma omp for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+      for (int c = 0; c < cols; ++c) xf[c] = (float)elem(W, dt, (size_t)r * cols + c);
+      nvfp4_row(xf, cols, Wq + (size_t)r * cols, row_scales + r,
+                block_scales ? block_scales + (size_t)r * (cols / 16) : NULL);
+    }
+    free(xf);
+  }
+  return 0;
+}
+
+/* NVFP4 activations (act_quant = OQ_NVFP4): z and h quantised with the row
+ * rule above, on their single-precision values. */
+static void q_vec_nvfp4(double *v, int n) {
+  float *xf = (float *)malloc(sizeof(float) * (size_t)n);
+  for (int i = 0; i < n; ++i) xf[i] = (float)v[i];
+  double sr;
+  nvfp4_row(xf, n, v, &sr, NULL);
+  free(xf);
+}
+
+static void q_act(int mode, double *v, int n) {
+  if (mode == OQ_E4M3) q_vec_e4m3(v, n);
+  else if (mode == OQ_NVFP4) q_vec_nvfp4(v, n);
 }
 
 int oracle_threads(void) {

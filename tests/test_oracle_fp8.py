@@ -90,8 +90,8 @@ import pytest
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "lmoe_oracle.c")
 MUTATIONS = {
-    "ties_away_from_zero": ("if (frac > 0.5 || (frac == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0;",
-                            "if (frac >= 0.5) k += 1.0;"),
+    "ties_away_from_zero": ("const double frac = n - k;\n    if (frac > 0.5 || (frac == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0;",
+                            "const double frac = n - k;\n    if (frac >= 0.5) k += 1.0;"),
     "scale_one_step_too_large": ("while (e > -200 && ldexp(448.0, e - 1) >= amax) --e;",
                                  "while (e > -200 && ldexp(448.0, e - 1) >= amax) --e;\n    ++e;"),
     "no_subnormals": ("if (ex < -6) ex = -6;", "if (ex < -6) return 0.0;"),

@@ -1,4 +1,5 @@
-"""Pins of the oracle's E4M3-activation reading (act_fp8), CPU only.
+"""Pins of the oracle's quantised-activation readings (act_fp8: E4M3;
+act_fp4: NVFP4), CPU only.
 
 The pages put the experts in FP8 ("LatentMoE Explained": an expert is about
 22 MB in FP8; the models are pretrained in NVFP4) but print no recipe for the
@@ -9,7 +10,8 @@ saturating; pinned in tests/test_oracle_fp8.py) -- while the router, W_down,
 the combine, W_up and the shared experts are unchanged.  Here the oracle's
 forward with act_fp8 is held to the definition recomposed with numpy from the
 pinned quantiser and the pinned router: a missing, misplaced or extra
-quantisation step fails.
+quantisation step fails.  The NVFP4 reading is the same with the NVFP4 row
+quantiser (pinned in tests/test_oracle_nvfp4.py) in place of E4M3.
 """
 import os
 import subprocess
@@ -32,16 +34,16 @@ def _weights(seed, activation):
     return kw, x
 
 
-def _q(v):
-    q, _ = oracle.fp8_rows(np.asarray(v, dtype=np.float64)[None, :])
-    return q[0]
+def _q(v, mode="e4m3"):
+    v = np.asarray(v, dtype=np.float64)[None, :]
+    return (oracle.fp8_rows(v) if mode == "e4m3" else oracle.nvfp4_rows(v))[0][0]
 
 
 def _silu(a):
     return a / (1.0 + np.exp(-a))
 
 
-def _recompose(kw, x, act_fp8):
+def _recompose(kw, x, act_fp8, mode="e4m3"):
     Lp = oracle.Layer(**kw)                        # unquantised: router and ids only
     s = oracle.router_logits(Lp, x)
     ids, g = oracle.select(s, K)
@@ -50,14 +52,14 @@ def _recompose(kw, x, act_fp8):
     for t in range(x.shape[0]):
         z = kw["w_down"] @ x[t]
         if act_fp8:
-            z = _q(z)
+            z = _q(z, mode)
         u = np.zeros(L_)
         for k in range(K):
             e = ids[t, k]
             b = kw["w_upx"][e] @ z
             h = np.maximum(b, 0.0) ** 2 if relu2 else _silu(kw["w_gate"][e] @ z) * b
             if act_fp8:
-                h = _q(h)
+                h = _q(h, mode)
             u += g[t, k] * (kw["w_out"][e] @ h)
         y[t] = kw["w_up"] @ u
         for j in range(NS):
@@ -67,11 +69,16 @@ def _recompose(kw, x, act_fp8):
     return y
 
 
+def _flag(mode):
+    return {"act_fp8": True} if mode == "e4m3" else {"act_fp4": True}
+
+
+@pytest.mark.parametrize("mode", ["e4m3", "nvfp4"])
 @pytest.mark.parametrize("activation", ["swiglu", "relu2"])
-def test_act_fp8_forward_is_the_quantised_recomposition(activation):
+def test_act_fp8_forward_is_the_quantised_recomposition(activation, mode):
     kw, x = _weights(1, activation)
-    y, _, _ = oracle.forward(oracle.Layer(**kw, act_fp8=True), x)
-    y_ref = _recompose(kw, x, True)
+    y, _, _ = oracle.forward(oracle.Layer(**kw, **_flag(mode)), x)
+    y_ref = _recompose(kw, x, True, mode)
     np.testing.assert_allclose(y, y_ref, rtol=0, atol=1e-12 * np.abs(y_ref).max())
     # and it is not the unquantised layer
     y0 = _recompose(kw, x, False)
@@ -84,34 +91,47 @@ def test_act_fp8_off_leaves_the_layer_unchanged():
     np.testing.assert_allclose(y, _recompose(kw, x, False), rtol=0, atol=1e-12)
 
 
-def test_act_fp8_error_is_that_of_a_few_e4m3_roundings():
+@pytest.mark.parametrize("mode,hi", [("e4m3", 0.1), ("nvfp4", 0.4)])
+def test_act_fp8_error_is_that_of_a_few_roundings(mode, hi):
     kw, x = _weights(3, "swiglu")
-    y8, _, _ = oracle.forward(oracle.Layer(**kw, act_fp8=True), x)
+    y8, _, _ = oracle.forward(oracle.Layer(**kw, **_flag(mode)), x)
     y, _, _ = oracle.forward(oracle.Layer(**kw), x)
     rel = np.abs(y8 - y).max() / np.abs(y).max()
-    assert 1e-4 < rel < 0.1, rel
+    assert 1e-4 < rel < hi, rel
 
 
-def test_backward_refuses_act_fp8():
+def test_nvfp4_activations_need_whole_blocks():
+    kw, x = _weights(5, "swiglu")          # m = 48, l = 32: whole 16-blocks
+    oracle.forward(oracle.Layer(**kw, act_fp4=True), x)
+    kw["w_gate"], kw["w_upx"], kw["w_out"] = kw["w_gate"][:, :40], kw["w_upx"][:, :40], kw["w_out"][:, :, :40]
+    with pytest.raises(ValueError):
+        oracle.forward(oracle.Layer(**kw, act_fp4=True), x)
+
+
+@pytest.mark.parametrize("mode", ["e4m3", "nvfp4"])
+def test_backward_refuses_quantised_activations(mode):
     kw, x = _weights(4, "swiglu")
     with pytest.raises(Exception):
-        oracle.backward(oracle.Layer(**kw, act_fp8=True), x, np.ones((x.shape[0], D)))
+        oracle.backward(oracle.Layer(**kw, **_flag(mode)), x, np.ones((x.shape[0], D)))
 
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "lmoe_oracle.c")
 MUTATIONS = {
-    "no_hidden_quantisation": ("  if (quant_hidden) q_vec_e4m3(a, hid);\n", "\n"),
-    "no_z_quantisation": ("      if (L->act_fp8) q_vec_e4m3(z, l);  /* the experts read z in E4M3 */\n",
+    "no_hidden_quantisation": ("  if (quant_hidden) q_act(quant_hidden, a, hid);\n", "\n"),
+    "no_z_quantisation": ("      if (L->act_quant) q_act(L->act_quant, z, l);  /* the experts read z quantised */\n",
                           "\n"),
     "shared_quantised_too": ("(size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, 0);",
-                             "(size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, L->act_fp8);"),
-    "quantised_after_down": ("  if (quant_hidden) q_vec_e4m3(a, hid);\n  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);",
-                             "  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);\n  if (quant_hidden) q_vec_e4m3(out, out_w);"),
+                             "(size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, L->act_quant);"),
+    "quantised_after_down": ("  if (quant_hidden) q_act(quant_hidden, a, hid);\n  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);",
+                             "  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);\n  if (quant_hidden) q_act(quant_hidden, out, out_w);"),
+    "modes_swapped": ("  if (mode == OQ_E4M3) q_vec_e4m3(v, n);\n  else if (mode == OQ_NVFP4) q_vec_nvfp4(v, n);",
+                      "  if (mode == OQ_NVFP4) q_vec_e4m3(v, n);\n  else if (mode == OQ_E4M3) q_vec_nvfp4(v, n);"),
 }
 
 
+@pytest.mark.parametrize("mode", ["e4m3", "nvfp4"])
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
-def test_act_fp8_pins_catch_mutation(name, tmp_path):
+def test_act_fp8_pins_catch_mutation(name, mode, tmp_path):
     old, new = MUTATIONS[name]
     src = open(SRC).read()
     assert src.count(old) == 1, f"mutation anchor for {name} not unique"
@@ -123,6 +143,6 @@ def test_act_fp8_pins_catch_mutation(name, tmp_path):
     oracle._swap_library(str(lib))
     try:
         with pytest.raises(AssertionError):
-            test_act_fp8_forward_is_the_quantised_recomposition("swiglu")
+            test_act_fp8_forward_is_the_quantised_recomposition("swiglu", mode)
     finally:
         oracle._swap_library(None)

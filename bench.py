@@ -51,7 +51,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="readme_acc",
                     choices=["readme_acc", "readme_eff", "prefill", "decode", "relu2_95b",
-                             "decode_fp8", "relu2_95b_fp8"])
+                             "decode_fp8", "relu2_95b_fp8", "decode_nvfp4",
+                             "relu2_95b_nvfp4"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
@@ -70,7 +71,8 @@ def workload(name):
     return {"readme_acc": configs.README_ACC, "readme_eff": configs.README_EFF,
             "prefill": configs.PREFILL, "decode": configs.DECODE,
             "relu2_95b": configs.RELU2_95B, "decode_fp8": configs.DECODE_FP8,
-            "relu2_95b_fp8": configs.RELU2_95B_FP8}[name]
+            "relu2_95b_fp8": configs.RELU2_95B_FP8, "decode_nvfp4": configs.DECODE_NVFP4,
+            "relu2_95b_nvfp4": configs.RELU2_95B_NVFP4}[name]
 
 
 def n_mats(cfg):
@@ -178,9 +180,11 @@ def layer_flops(cfg):
 
 
 def expert_weight_bytes(cfg):
-    """Bytes per routed-expert weight: 2 (bf16), or 1 (E4M3) plus one f32
-    scale per weight row (row length >= 512, so < 0.01 byte per weight)."""
-    return 1.0 if cfg.weights == "fp8" else 2.0
+    """Bytes per routed-expert weight: 2 (bf16); 1 (E4M3); NVFP4 half a byte
+    of E2M1 code plus one E4M3 block scale per 16 weights.  The f32 row
+    scales (one per weight row of length >= 512, < 0.01 byte per weight) are
+    left out."""
+    return {"fp8": 1.0, "nvfp4": 0.5 + 1.0 / 16}.get(cfg.weights, 2.0)
 
 
 def layer_bytes(cfg, ids=None):
@@ -257,7 +261,8 @@ def oracle_rate(cfg, inp_np, budget_s, max_tokens=None):
                      w_down=inp_np["w_down"], w_up=inp_np["w_up"], w_gate=inp_np["w_gate"],
                      w_upx=inp_np["w_upx"], w_out=inp_np["w_out"], s_gate=inp_np["s_gate"],
                      s_up=inp_np["s_up"], s_out=inp_np["s_out"], k_active=cfg.k_active,
-                     activation=cfg.activation)
+                     activation=cfg.activation, act_fp8=cfg.weights == "fp8",
+                     act_fp4=cfg.weights == "nvfp4")
     x = inp_np["x"]
     cal = min(cfg.T, max(8, oracle.threads()))
     t0 = time.perf_counter()

@@ -67,8 +67,21 @@ typedef enum { LMOE_SWIGLU = 0, LMOE_RELU2 = 1 } lmoe_activation;
  * each expert's hidden vector are quantised the same way, per row, before
  * they are multiplied.  The layer then computes exactly with those quantised
  * operands.  Needs l and m multiples of 128.  Not with training = 1, not
- * with expert parallelism. */
-typedef enum { LMOE_WEIGHTS_BF16 = 0, LMOE_WEIGHTS_FP8 = 1 } lmoe_weight_format;
+ * with expert parallelism.
+ * LMOE_WEIGHTS_NVFP4: the same with NVFP4 on both operands (the pages say
+ * the shipped models were pretrained in NVFP4; the format is NVIDIA's
+ * published one): E2M1 codes, one E4M3 scale per 16 consecutive elements of
+ * a row, and a second-level power-of-two scale per row (the smallest with
+ * the row's largest magnitude within 6 * 448).  Block scale b =
+ * E4M3(block max / (6 s_row)), code = E2M1(x / (b s_row)), both divisions in
+ * IEEE single precision, rounding to nearest even with saturation.  The
+ * expert GEMMs run tcgen05 kind::mxf4nvf4 (the tensor cores apply the block
+ * scales, fp32 accumulation).  Same limits as LMOE_WEIGHTS_FP8. */
+typedef enum {
+  LMOE_WEIGHTS_BF16 = 0,
+  LMOE_WEIGHTS_FP8 = 1,
+  LMOE_WEIGHTS_NVFP4 = 2
+} lmoe_weight_format;
 
 enum {
   LMOE_OK = 0,
@@ -203,8 +216,19 @@ int lmoe_selftest_wait_timeout(lmoe_handle h, int64_t limit_ns, void *stream);
  * squared ReLU] and 15 W_o row scales [N'][l], f32; 16 the E4M3 codes of the
  * experts' input rows [T*K'][l] (z in dispatch order) and 17 their row scales
  * [T*K'] f32; 18 the E4M3 codes of the expert hidden rows [T*K'][m] and 19
- * their row scales [T*K'] f32).  Errors: NULL_ARG, INVALID_CONFIG (unknown
- * `which`). */
+ * their row scales [T*K'] f32).  With LMOE_WEIGHTS_NVFP4 the same ids hold
+ * the NVFP4 counterparts -- 12 / 14 the packed E2M1 weight codes (two per
+ * byte, element 2i in the low nibble of byte i) in 256-row x 128-byte blocks
+ * (expert, 256-row tile, 256-element K-block, row, byte), 13 / 15 the row
+ * scales, 16 / 18 the packed activation codes [T*K'][l / 2] and [T*K'][m / 2],
+ * 17 / 19 their row scales -- and also 20 / 21 the weights' E4M3 block scales
+ * (bytes; per expert, 256-row tile and K-block 4 KB: for each 128-row half
+ * and each 64-element slice of the K-block a 512-byte atom in which row
+ * r0 + 32 r1 (r0 < 32, r1 < 4) holds its four scales at bytes 16 r0 + 4 r1
+ * .. + 3) and 22 / 23 the activations' block scales (per 128-row tile of
+ * debug buffer 11's count, in dispatch order of the experts, and K-block
+ * 2 KB: the four slices' atoms of the tile's rows).  Errors: NULL_ARG,
+ * INVALID_CONFIG (unknown `which`). */
 int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *numel);
 
 /* Profiling hook.  slots > 0: every later lmoe_forward on this handle also

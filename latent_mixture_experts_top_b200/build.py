@@ -18,7 +18,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblmoe.so")
 SOURCES = ["route_kernels.cu", "simt_kernels.cu", "tc_gemm.cu", "lmoe_abi.cu",
            "dispatch_noalloc.cu", "backward_kernels.cu",
-           "fp8_weights.cu"]
+           "fp8_weights.cu", "fp4_quant.cu"]
 HEADERS = ["common.cuh", "ptx_sm100.cuh", "kernels.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

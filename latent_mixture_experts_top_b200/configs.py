@@ -32,7 +32,7 @@ class LayerConfig:
     top_k_override: int = 0
     router_bias_std: float = 0.0   # > 0: per-expert router bias ~ N(0, std)
     activation: str = "swiglu"     # "swiglu" (3 matrices) | "relu2" (2 matrices)
-    weights: str = "bf16"          # routed experts' weights: "bf16" | "fp8" (E4M3, row scales)
+    weights: str = "bf16"          # routed experts: "bf16" | "fp8" (E4M3, row scales) | "nvfp4"
     x_std: float = 1.0
     w_std: float = 0.02
 
@@ -87,7 +87,15 @@ RELU2_95B = LayerConfig("relu2_95b_T1024_d4096_l1024_m2688_N512_K24", T=1024, d=
 DECODE_FP8 = replace(DECODE, name="decode_fp8_T64_d4096_l1024_m2048_N512_K22", weights="fp8")
 RELU2_95B_FP8 = replace(RELU2_95B, name="relu2_95b_fp8_T1024_d4096_l1024_m2688_N512_K24",
                         weights="fp8")
+# The same two with NVFP4 routed experts ("LatentMoE Explained": the shipped
+# models were pretrained in NVFP4): E2M1 codes, an E4M3 scale per 16 elements
+# and a power-of-two scale per row, on weights and activations alike.
+DECODE_NVFP4 = replace(DECODE, name="decode_nvfp4_T64_d4096_l1024_m2048_N512_K22",
+                       weights="nvfp4")
+RELU2_95B_NVFP4 = replace(RELU2_95B, name="relu2_95b_nvfp4_T1024_d4096_l1024_m2688_N512_K24",
+                          weights="nvfp4")
 
 CONFIGS = [TINY_F32, README_ACC, README_EFF, PREFILL, DECODE]
-EXTRA_CONFIGS = [TINY_RELU2_F32, RELU2_95B, DECODE_FP8, RELU2_95B_FP8]
+EXTRA_CONFIGS = [TINY_RELU2_F32, RELU2_95B, DECODE_FP8, RELU2_95B_FP8, DECODE_NVFP4,
+                 RELU2_95B_NVFP4]
 BY_NAME = {c.name: c for c in CONFIGS + EXTRA_CONFIGS}

@@ -165,6 +165,14 @@ struct TcParams {
   // kind::f8f6f4 over 128-element K-blocks.
   const float *a_scale;
   const float *b_scale; int b_scale_ld;
+  // NVFP4 operands (a_sf and b_sf set as well as the row scales): A is packed
+  // E2M1 [rows][Kdim / 2], B the packed weight tiled in 256-row x 128-byte
+  // blocks (launch_quantize_nvfp4_tiles); a_sf holds the E4M3 block scales of
+  // A by M-tile of the tile table and K-block (2 KB each), b_sf those of B by
+  // expert, N-tile and K-block (4 KB each), in the layout the MMA reads from
+  // TMEM (see launch_quantize_nvfp4_tiles); the MMA is kind::mxf4nvf4 over
+  // 256-element K-blocks.
+  const uint8_t *a_sf, *b_sf;
   // TC_WGRAD: A [M][*] and B [*][*] are plain row-major token-major matrices
   // (K runs along their rows' contiguous axis); group g reduces over
   // K-columns [k_start[g], k_start[g] + k_len[g]) (multiples of 64; dense:
@@ -215,6 +223,30 @@ cudaError_t launch_quantize_e4m3_tiles(const __nv_bfloat16 *src, int groups, int
 cudaError_t launch_quantize_rows_e4m3(const __nv_bfloat16 *src, const int32_t *gather, int K,
                                       int rows, int cols, uint8_t *dst, float *scales,
                                       cudaStream_t s, bool pdl = false);
+
+// NVFP4 expert weights (fp4_quant.cu): src [groups][rows_per_group][cols]
+// bf16 -> packed E2M1 codes in 256-row x 128-byte blocks per (group, 256-row
+// tile, 256-element K-block), E4M3 block scales in 4 KB per such block (two
+// 128-row halves x four 64-element slices x one 512-byte atom: row r0 + 32 r1
+// at bytes 16 r0 + 4 r1 .. + 3), and the power-of-two row scales [groups]
+// [rows_per_group].  Padding rows, columns and scales are zero.  cols % 32 == 0.
+size_t nvfp4_weight_code_bytes(int groups, int rows_per_group, int cols);
+size_t nvfp4_weight_sf_bytes(int groups, int rows_per_group, int cols);
+cudaError_t launch_quantize_nvfp4_tiles(const __nv_bfloat16 *src, int groups, int rows_per_group,
+                                        int cols, float *scales, uint8_t *codes, uint8_t *sf,
+                                        cudaStream_t s);
+
+// NVFP4 activations, one block per M-tile of the table (tiles, device count
+// n_tiles, grid max_tiles): tile row p reads the bf16 row src[gather ?
+// gather[p] / K : p] (row stride cols) and writes the packed codes row p of
+// codes [rows][cols / 2], scales[p] and, per K-block, the tile's four 512-byte
+// block-scale atoms (sf: nvfp4_act_sf_bytes(max_tiles, cols) bytes; scales of
+// rows past the tile's expert and of blocks past cols are zero).
+size_t nvfp4_act_sf_bytes(int max_tiles, int cols);
+cudaError_t launch_quantize_act_nvfp4(const __nv_bfloat16 *src, const int32_t *gather, int K,
+                                      const TileEntry *tiles, const int32_t *n_tiles,
+                                      int max_tiles, int cols, uint8_t *codes, float *scales,
+                                      uint8_t *sf, cudaStream_t s, bool pdl = false);
 
 // Encodes a 2-D byte tensor map (rows x cols bytes, row stride in bytes)
 // with a {128, box_rows} box and 128-byte swizzle (E4M3 GEMM operands).

@@ -44,9 +44,10 @@ struct Workspace {
   void *x_stage = nullptr, *y_stage = nullptr;
   int32_t *status = nullptr;
   int32_t *arrivals = nullptr;  // fused routing: the last-block counter (zero between launches)
-  // E4M3 routed experts: the expert GEMMs' A operands in E4M3 with row scales
-  uint8_t *zq = nullptr, *hq = nullptr;  // [TK][l], [TK][m]
+  // E4M3 / NVFP4 routed experts: the expert GEMMs' A operands with row scales
+  uint8_t *zq = nullptr, *hq = nullptr;  // [TK][l], [TK][m] (NVFP4: packed, half the bytes)
   float *zq_scale = nullptr, *hq_scale = nullptr;  // [TK]
+  uint8_t *zq_sf = nullptr, *hq_sf = nullptr;  // NVFP4 block scales, by M-tile and K-block
   // expert parallelism: M-tile tables of the received rows (128- and 256-row)
   TileEntry *ep_tiles = nullptr, *ep_tiles2 = nullptr;
   int32_t *ep_n_tiles = nullptr, *ep_n_tiles2 = nullptr;
@@ -83,7 +84,8 @@ struct lmoe_layer {
   int d = 0, l = 0, m = 0, N = 0, K = 0, ns = 0, ms = 0, Tmax = 0;
   int bf16 = 0;
   int relu2 = 0;      // squared-ReLU experts (two matrices)
-  int fp8 = 0;        // E4M3 routed experts (weights and the activations they multiply)
+  int fp8 = 0;        // quantised routed experts (weights and the activations they multiply)
+  int fp4 = 0;        // ... in NVFP4 (else E4M3)
   size_t esize = 4;
   int device = 0, num_sms = 0;
   bool loaded = false;
@@ -132,9 +134,11 @@ struct lmoe_layer {
   // B operands of the CTA-pair GEMMs: the same tiled matrices, {64, 128} boxes
   TensorMap64 tm_wx2, tm_wo2, tm_wy2;
   TensorMap64 tm_zq, tm_zq32, tm_hq, tm_hq32;  // E4M3 activations ({128, 128}, {128, 32})
-  // E4M3 expert weights (tiled like w_gu / w_out) and their row scales
+  // E4M3 / NVFP4 expert weights (256-row x 128-byte blocks) and their row
+  // scales; NVFP4 block scales (4 KB per 256-row tile and K-block)
   uint8_t *w_gu8 = nullptr, *w_o8 = nullptr;
   float *gu_scale = nullptr, *o_scale = nullptr;
+  uint8_t *gu_sf = nullptr, *o_sf = nullptr;
   // bf16 training: transposed weights (K-block tiled) and backward maps
   void *w_yT = nullptr;   // [ky][d]
   void *w_oT = nullptr;   // [N][m][l]
@@ -179,7 +183,8 @@ void free_all(lmoe_layer *h) {
                   h->bw.ABs, h->bw.dAB, h->bw.dXcat, h->bw.DOT, h->bw.HT, h->bw.dABT,
                   h->bw.zpT, h->bw.dyT, h->bw.ucatT, h->bw.dXcatT, h->bw.xT, h->bw.kstart,
                   h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT, h->w_gu8,
-                  h->w_o8, h->gu_scale, h->o_scale, h->ws.ep_tiles, h->ws.ep_tiles2,
+                  h->w_o8, h->gu_scale, h->o_scale, h->gu_sf, h->o_sf, h->ws.zq_sf, h->ws.hq_sf,
+                  h->ws.ep_tiles, h->ws.ep_tiles2,
                   h->ws.ep_n_tiles, h->ws.ep_n_tiles2, h->ws.arrivals, h->ws.zq, h->ws.hq,
                   h->ws.zq_scale, h->ws.hq_scale};
   for (void *p : ptrs)
@@ -227,11 +232,14 @@ int validate(const lmoe_config *c, lmoe_layer *h) {
   h->Tmax = c->max_tokens;
   h->bf16 = c->dtype == LMOE_BF16;
   h->relu2 = c->activation == LMOE_RELU2;
-  if (c->weight_format != LMOE_WEIGHTS_BF16 && c->weight_format != LMOE_WEIGHTS_FP8)
+  if (c->weight_format != LMOE_WEIGHTS_BF16 && c->weight_format != LMOE_WEIGHTS_FP8 &&
+      c->weight_format != LMOE_WEIGHTS_NVFP4)
     return LMOE_ERR_INVALID_CONFIG;
-  h->fp8 = c->weight_format == LMOE_WEIGHTS_FP8;
+  h->fp8 = c->weight_format != LMOE_WEIGHTS_BF16;
+  h->fp4 = c->weight_format == LMOE_WEIGHTS_NVFP4;
   if (h->fp8 && (c->dtype != LMOE_BF16 || c->training)) return LMOE_ERR_UNSUPPORTED;
   // E4M3 GEMMs run 128-element K-blocks: l and m must be multiples of 128
+  // (NVFP4, 256-element K-blocks, reads a ragged last one as zeros)
   if (h->fp8 && ((c->d / c->alpha) % 128 || c->m % 128)) return LMOE_ERR_UNSUPPORTED;
   h->esize = h->bf16 ? 2 : 4;
   h->ky = h->l + h->ns * h->ms;
@@ -335,7 +343,17 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
       // K-block-tiled B operands (see launch_repack_btiles)
       ok = dalloc(&h->w_x, btile_rows(1, h->nx_rows, h->d) * 64 * es) &&
            dalloc(&h->w_y, btile_rows(1, h->d, h->ky) * 64 * es);
-      if (ok && h->fp8)
+      if (ok && h->fp4)
+        ok = dalloc(&h->w_gu8, nvfp4_weight_code_bytes(h->N, h->gu_rows, h->l)) &&
+             dalloc(&h->w_o8, nvfp4_weight_code_bytes(h->N, h->l, h->m)) &&
+             dalloc(&h->gu_sf, nvfp4_weight_sf_bytes(h->N, h->gu_rows, h->l)) &&
+             dalloc(&h->o_sf, nvfp4_weight_sf_bytes(h->N, h->l, h->m)) &&
+             dalloc(&h->gu_scale, N * h->gu_rows * 4) && dalloc(&h->o_scale, N * l * 4) &&
+             dalloc(&w.zq, TK * l / 2) && dalloc(&w.hq, TK * m / 2) &&
+             dalloc(&w.zq_scale, TK * 4) && dalloc(&w.hq_scale, TK * 4) &&
+             dalloc(&w.zq_sf, nvfp4_act_sf_bytes(h->max_tiles, h->l)) &&
+             dalloc(&w.hq_sf, nvfp4_act_sf_bytes(h->max_tiles, h->m));
+      else if (ok && h->fp8)
         ok = dalloc(&h->w_gu8, btile_rows(h->N, h->gu_rows, h->l) * 64) &&
              dalloc(&h->w_o8, btile_rows(h->N, h->l, h->m) * 64) &&
              dalloc(&h->gu_scale, N * h->gu_rows * 4) && dalloc(&h->o_scale, N * l * 4) &&
@@ -420,14 +438,20 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     if (rc == LMOE_OK)
       rc = make_map(&h->tm_wx2, h->w_x, btile_rows(1, h->nx_rows, h->d), 64, 64, kTileN / 2);
     if (rc == LMOE_OK && h->fp8) {
-      // E4M3 operands, 128-byte swizzle: A rows {128, 128} (and {128, 32} for
-      // tiles of at most 32 rows); the weights in 256-row x 128-byte blocks
-      const int64_t gu8_rows = btile_rows(h->N, h->gu_rows, h->l) / 2;
-      const int64_t o8_rows = btile_rows(h->N, h->l, h->m) / 2;
-      if (make_tmap_u8(h->tm_zq.bytes, w.zq, static_cast<int64_t>(TK), h->l, h->l, kTileM) != 0 ||
-          make_tmap_u8(h->tm_zq32.bytes, w.zq, static_cast<int64_t>(TK), h->l, h->l, 32) != 0 ||
-          make_tmap_u8(h->tm_hq.bytes, w.hq, static_cast<int64_t>(TK), h->m, h->m, kTileM) != 0 ||
-          make_tmap_u8(h->tm_hq32.bytes, w.hq, static_cast<int64_t>(TK), h->m, h->m, 32) != 0 ||
+      // E4M3 / NVFP4 operands, 128-byte swizzle: A rows {128, 128} (and
+      // {128, 32} for tiles of at most 32 rows); the weights in 256-row x
+      // 128-byte blocks.  NVFP4 rows hold half as many bytes.
+      const int64_t gu8_rows = h->fp4 ? static_cast<int64_t>(
+                                            nvfp4_weight_code_bytes(h->N, h->gu_rows, h->l) / 128)
+                                      : btile_rows(h->N, h->gu_rows, h->l) / 2;
+      const int64_t o8_rows = h->fp4 ? static_cast<int64_t>(
+                                           nvfp4_weight_code_bytes(h->N, h->l, h->m) / 128)
+                                     : btile_rows(h->N, h->l, h->m) / 2;
+      const int lb = h->fp4 ? h->l / 2 : h->l, mb = h->fp4 ? h->m / 2 : h->m;  // row bytes
+      if (make_tmap_u8(h->tm_zq.bytes, w.zq, static_cast<int64_t>(TK), lb, lb, kTileM) != 0 ||
+          make_tmap_u8(h->tm_zq32.bytes, w.zq, static_cast<int64_t>(TK), lb, lb, 32) != 0 ||
+          make_tmap_u8(h->tm_hq.bytes, w.hq, static_cast<int64_t>(TK), mb, mb, kTileM) != 0 ||
+          make_tmap_u8(h->tm_hq32.bytes, w.hq, static_cast<int64_t>(TK), mb, mb, 32) != 0 ||
           make_tmap_u8(h->tm_wgu.bytes, h->w_gu8, gu8_rows, 128, 128, kTileN) != 0 ||
           make_tmap_u8(h->tm_wo.bytes, h->w_o8, o8_rows, 128, 128, kTileN) != 0)
         rc = LMOE_ERR_CUDA;
@@ -570,7 +594,14 @@ int lmoe_load_weights(lmoe_handle h, const lmoe_weights *wt, void *stream) {
   if (e == cudaSuccess)
     e = launch_repack_btiles(static_cast<const bf *>(tx), 1, h->nx_rows, h->d,
                              static_cast<bf *>(h->w_x), s);
-  if (h->fp8) {  // E4M3 codes + row scales, tiled like the bf16 weights
+  if (h->fp4) {  // NVFP4 codes, block scales and row scales in GEMM tiles
+    if (e == cudaSuccess)
+      e = launch_quantize_nvfp4_tiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->N,
+                                      h->gu_rows, h->l, h->gu_scale, h->w_gu8, h->gu_sf, s);
+    if (e == cudaSuccess)
+      e = launch_quantize_nvfp4_tiles(static_cast<const bf *>(wt->w_out), h->N, h->l, h->m,
+                                      h->o_scale, h->w_o8, h->o_sf, s);
+  } else if (h->fp8) {  // E4M3 codes + row scales, tiled like the bf16 weights
     if (e == cudaSuccess)
       e = launch_quantize_e4m3_tiles(static_cast<const bf *>(h->relu2 ? wt->w_upx : tgu), h->N,
                                      h->gu_rows, h->l, h->gu_scale, h->w_gu8, s);
@@ -841,6 +872,10 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
     p.a_scale = h->ws.zq_scale;
     p.b_scale = h->gu_scale;
     p.b_scale_ld = h->gu_rows;
+    if (h->fp4) {
+      p.a_sf = h->ws.zq_sf;
+      p.b_sf = h->gu_sf;
+    }
   }
   p.b_rows_per_expert = h->gu_rows;
   p.out = static_cast<__nv_bfloat16 *>(w.H);
@@ -855,7 +890,13 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
                                  tm_a32.bytes, h->tm_out_h.bytes);
   h->launches += 1;
   if (e != cudaSuccess) return e;
-  if (h->fp8) {  // H rows -> E4M3 with row scales, the down GEMM's A operand
+  if (h->fp4) {  // H rows -> NVFP4 codes and scales, the down GEMM's A operand
+    e = launch_quantize_act_nvfp4(static_cast<const __nv_bfloat16 *>(w.H), nullptr, 1, tiles,
+                                  n_tiles, h->max_tiles, h->m, w.hq, w.hq_scale, w.hq_sf, s,
+                                  !marks);
+    h->launches += 1;
+    if (e != cudaSuccess) return e;
+  } else if (h->fp8) {  // H rows -> E4M3 with row scales, the down GEMM's A operand
     e = launch_quantize_rows_e4m3(static_cast<const __nv_bfloat16 *>(w.H), nullptr, 1, a_rows,
                                   h->m, w.hq, w.hq_scale, s, !marks);
     h->launches += 1;
@@ -876,6 +917,10 @@ static cudaError_t run_experts_bf16(lmoe_layer *h, const TensorMap64 &tm_a,
     pd.a_scale = w.hq_scale;
     pd.b_scale = h->o_scale;
     pd.b_scale_ld = h->l;
+    if (h->fp4) {
+      pd.a_sf = w.hq_sf;
+      pd.b_sf = h->o_sf;
+    }
   }
   pd.tma_out = 1;
   pd.pdl = marks ? 0 : 1;
@@ -931,7 +976,14 @@ static int forward_impl(lmoe_layer *h, const void *x, void *y, int T, cudaStream
   // scales, gathered straight from z through perm
   cudaError_t e = run_route(h, x, T, true, s, nullptr, true, h->fp8 ? nullptr : w.zp);
   if (e != cudaSuccess) return LMOE_ERR_CUDA;
-  if (h->fp8) {
+  if (h->fp4) {
+    e = launch_quantize_act_nvfp4(static_cast<const __nv_bfloat16 *>(w.z), w.perm, h->K, w.tiles,
+                                  w.n_tiles, h->max_tiles, h->l, w.zq, w.zq_scale, w.zq_sf, s,
+                                  h->prof_slots == 0);
+    h->launches += 1;
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    mark(h, 4, s);
+  } else if (h->fp8) {
     e = launch_quantize_rows_e4m3(static_cast<const __nv_bfloat16 *>(w.z), w.perm, h->K, TK, h->l,
                                   w.zq, w.zq_scale, s, h->prof_slots == 0);
     h->launches += 1;
@@ -1437,19 +1489,46 @@ int lmoe_debug_buffer(lmoe_handle h, int32_t which, void **dev_ptr, int64_t *num
     case 9: *dev_ptr = w.perm; *numel = TK; break;
     case 10: *dev_ptr = w.pos; *numel = TK; break;
     case 11: *dev_ptr = w.n_tiles; *numel = 1; break;
-    case 12: case 13: case 14: case 15:
+    case 12: case 13: case 14: case 15: {
       if (!h->fp8) return LMOE_ERR_INVALID_CONFIG;
-      if (which == 12) { *dev_ptr = h->w_gu8; *numel = btile_rows(h->N, h->gu_rows, h->l) * 64; }
+      const int64_t gu_bytes = h->fp4 ? static_cast<int64_t>(
+                                            nvfp4_weight_code_bytes(h->N, h->gu_rows, h->l))
+                                      : btile_rows(h->N, h->gu_rows, h->l) * 64;
+      const int64_t o_bytes = h->fp4 ? static_cast<int64_t>(nvfp4_weight_code_bytes(h->N, h->l, h->m))
+                                     : btile_rows(h->N, h->l, h->m) * 64;
+      if (which == 12) { *dev_ptr = h->w_gu8; *numel = gu_bytes; }
       if (which == 13) { *dev_ptr = h->gu_scale; *numel = static_cast<int64_t>(h->N) * h->gu_rows; }
-      if (which == 14) { *dev_ptr = h->w_o8; *numel = btile_rows(h->N, h->l, h->m) * 64; }
+      if (which == 14) { *dev_ptr = h->w_o8; *numel = o_bytes; }
       if (which == 15) { *dev_ptr = h->o_scale; *numel = static_cast<int64_t>(h->N) * h->l; }
       break;
-    case 16: case 17: case 18: case 19:
+    }
+    case 16: case 17: case 18: case 19: {
       if (!h->fp8) return LMOE_ERR_INVALID_CONFIG;
-      if (which == 16) { *dev_ptr = w.zq; *numel = TK * h->l; }
+      const int64_t div = h->fp4 ? 2 : 1;  // packed NVFP4 rows
+      if (which == 16) { *dev_ptr = w.zq; *numel = TK * h->l / div; }
       if (which == 17) { *dev_ptr = w.zq_scale; *numel = TK; }
-      if (which == 18) { *dev_ptr = w.hq; *numel = TK * h->m; }
+      if (which == 18) { *dev_ptr = w.hq; *numel = TK * h->m / div; }
       if (which == 19) { *dev_ptr = w.hq_scale; *numel = TK; }
+      break;
+    }
+    case 20: case 21: case 22: case 23:
+      if (!h->fp4) return LMOE_ERR_INVALID_CONFIG;
+      if (which == 20) {
+        *dev_ptr = h->gu_sf;
+        *numel = static_cast<int64_t>(nvfp4_weight_sf_bytes(h->N, h->gu_rows, h->l));
+      }
+      if (which == 21) {
+        *dev_ptr = h->o_sf;
+        *numel = static_cast<int64_t>(nvfp4_weight_sf_bytes(h->N, h->l, h->m));
+      }
+      if (which == 22) {
+        *dev_ptr = w.zq_sf;
+        *numel = static_cast<int64_t>(nvfp4_act_sf_bytes(h->max_tiles, h->l));
+      }
+      if (which == 23) {
+        *dev_ptr = w.hq_sf;
+        *numel = static_cast<int64_t>(nvfp4_act_sf_bytes(h->max_tiles, h->m));
+      }
       break;
     default: return LMOE_ERR_INVALID_CONFIG;
   }

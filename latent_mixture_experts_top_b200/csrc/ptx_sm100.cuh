@@ -79,6 +79,17 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
       : "memory");
 }
 
+// Plain (non-tensor) bulk copy global -> shared, completing on `bar` like a
+// TMA load: both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 2-D tiled store of a shared-memory box to global memory, tracked as one
 // bulk async-group of the issuing thread.  Rows and columns past the tensor's
 // extent are not written.
@@ -151,6 +162,30 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= (A . SFA)[smem] * (B . SFB)[smem]^T with NVFP4 operands:
+// packed E2M1 codes (two per byte, K-major, 64 elements = 32 bytes of a row
+// per instruction) and one E4M3 scale per 16 elements of a row, read from
+// TMEM at sfa / sfb (kind::mxf4nvf4, 16-element scale blocks), f32 accumulate.
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;"
+      "\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// 32 TMEM lanes x 128 bits from shared memory (32 rows of 16 bytes, described
+// by smem_desc_rows16), written to lanes 0-31 of each of the four lane
+// quarters at columns taddr .. taddr + 3.  Ordered before the tcgen05.mma
+// this thread issues next.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
 // The mbarrier receives one arrival once every tcgen05 op this thread issued
 // before the commit has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -192,6 +227,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   return desc;
 }
 
+// 32 rows of 16 bytes, contiguous, no swizzle: the source of a 32x128b
+// tcgen05.cp.  8-row core matrices of 128 bytes follow one another (stride
+// byte offset 128); there is one core matrix along the row.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t addr) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);  // start address
+  desc |= static_cast<uint64_t>(1u) << 16;                // leading byte offset (unused here)
+  desc |= static_cast<uint64_t>(128u >> 4) << 32;         // stride byte offset: 8 rows
+  desc |= static_cast<uint64_t>(1u) << 46;                // descriptor version (sm_100)
+  return desc;                                            // layout: no swizzle
+}
+
 // Instruction descriptor: bf16 A/B, f32 accumulate, K-major A and B.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
@@ -201,6 +248,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // and [10,13)), f32 accumulate, K-major A and B.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Block-scaled instruction descriptor (kind::mxf4nvf4): E2M1 A and B (format
+// 1 in bits [7,10) and [10,13)), K-major, N >> 3 in bits [17,23), E4M3 scale
+// factors (bit 23 clear), M >> 4 in bits [24,29); scale-factor ids and the
+// sparsity fields 0, K = 64 per instruction (bit 31 clear).
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

@@ -454,15 +454,16 @@ __global__ void __launch_bounds__(256) scatter_permute_kernel(
   __syncthreads();
   // The share's pairs are i = share, share + S, ...; item j = (its q-th pair,
   // vector v) with q = j / vecs_per_row: consecutive threads copy consecutive
-  // 16-byte vectors of a row, eight items in flight per thread.
+  // 16-byte vectors of a row, four items in flight per thread (eight measured
+  // slower).
   const int npairs = min(chunk, T - c * chunk) * K;
   const int my_pairs = npairs > share ? (npairs - share + S - 1) / S : 0;
   const int items = my_pairs * vecs_per_row;
-  for (int j0 = threadIdx.x; j0 < items; j0 += 8 * blockDim.x) {
-    uint4 v[8];
-    int64_t dst_at[8];
+  for (int j0 = threadIdx.x; j0 < items; j0 += 4 * blockDim.x) {
+    uint4 v[4];
+    int64_t dst_at[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 4; ++u) {
       const int j = j0 + u * blockDim.x;
       dst_at[u] = -1;
       if (j < items) {
@@ -473,7 +474,7 @@ __global__ void __launch_bounds__(256) scatter_permute_kernel(
       }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < 4; ++u)
       if (dst_at[u] >= 0) dst[dst_at[u]] = v[u];
   }
 }

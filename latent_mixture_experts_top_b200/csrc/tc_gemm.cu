@@ -43,6 +43,16 @@
 // so every row of a staged tile is still 128 bytes and the shared-memory
 // layout, descriptors and pipeline are those of the bf16 tiles; the epilogue
 // multiplies the accumulator by the A row's scale and the weight row's scale.
+//
+// kQ = kNvf4 (NVFP4 routed experts): both operands are packed E2M1 codes with
+// one E4M3 scale per 16 elements of a row (tcgen05.mma kind::mxf4nvf4, block
+// size 16): a K-block is 256 elements, again 128 bytes per staged row.  Each
+// stage also carries the two operands' scale blocks (2 KB for the 128 A rows,
+// 4 KB for the 256 B rows), laid out as the MMA reads them from TMEM; the
+// MMA warp copies them into TMEM (tcgen05.cp) ahead of the stage's four
+// MMAs.  The per-row second-level scales are applied in the epilogue, as for
+// E4M3.  The scale blocks take 48 TMEM columns, so this variant keeps one
+// accumulator (256 columns) instead of two.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -63,18 +73,29 @@ constexpr int TMEM_COLS = 2 * TN;             // two accumulators
 constexpr int NUM_EPI_WARPS = 8;              // two per TMEM lane quarter
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, TN);
 constexpr uint32_t IDESC8 = ptx::idesc_e4m3_f32(TM, TN);
+constexpr uint32_t IDESC4 = ptx::idesc_nvf4(TM, TN);
+// operand formats of the single-CTA kernel
+constexpr int kBf16 = 0, kE4m3 = 1, kNvf4 = 2;
+// NVFP4 scale blocks of one stage: A 128 rows x 16 scales, B 256 rows x 16,
+// as 512-byte atoms (32 rows x 4 scales of one MMA; row r0 + 32 r1 at byte
+// 16 r0 + 4 r1); TMEM columns of the A atoms (4 per MMA) and the B atoms (8)
+constexpr int SFA_BYTES = 2048, SFB_BYTES = 4096;
+constexpr int SFA_COL = 256, SFB_COL = 288;
 
 // Pipeline shape: a STAGES-deep ring of (A, B) tiles filled by TMA and read
 // by the MMA.  Both element types stage 128-byte K-block rows: 64 bf16, or
 // (kF8) 128 E4M3 codes.
 constexpr int TKB8 = 128;  // K-block of the E4M3 GEMM (elements = bytes)
-template <bool kF8>
+constexpr int TKB4 = 256;  // K-block of the NVFP4 GEMM (two elements per byte)
+template <int kQ>
 struct Cfg {
-  static constexpr int STAGES = 4;
-  static constexpr int KB = kF8 ? TKB8 : TKB;  // elements per K-block
+  static constexpr int STAGES = kQ == kNvf4 ? 3 : 4;
+  static constexpr int KB = kQ == kNvf4 ? TKB4 : kQ == kE4m3 ? TKB8 : TKB;  // elements per K-block
   static constexpr int EPI_WARPS = NUM_EPI_WARPS;
   static constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int RING_BYTES = STAGES * (A_BYTES + B_BYTES);
+  static constexpr int SF_BYTES = kQ == kNvf4 ? SFA_BYTES + SFB_BYTES : 0;  // per stage
+  static constexpr int RING_BYTES = STAGES * (A_BYTES + B_BYTES + SF_BYTES);
+  static constexpr int ACC_BUFS = kQ == kNvf4 ? 1 : 2;  // accumulators in TMEM
 };
 
 constexpr int MAX_STAGES = 8;
@@ -94,15 +115,18 @@ constexpr int OUT_BOX_BYTES = OUT_BOX * OUT_BOX * 2;                // 2 KB
 constexpr int CTL_BYTES = 1024;                                     // SmemCtl, padded
 constexpr int STAGING_BYTES = NUM_EPI_WARPS * 2 * OUT_BOX_BYTES;    // 32 KB
 static_assert(sizeof(SmemCtl) <= CTL_BYTES, "control block");
-template <bool kF8>
+template <int kQ>
 constexpr size_t smem_bytes(bool staging) {
-  return 1024 /*align slack*/ + Cfg<kF8>::RING_BYTES +
+  return 1024 /*align slack*/ + Cfg<kQ>::RING_BYTES +
          (staging ? CTL_BYTES + STAGING_BYTES : sizeof(SmemCtl));
 }
-static_assert(smem_bytes<false>(true) <= 232448, "shared memory per CTA");
+static_assert(smem_bytes<kBf16>(true) <= 232448, "shared memory per CTA");
+static_assert(smem_bytes<kE4m3>(true) <= 232448, "shared memory per CTA");
+static_assert(smem_bytes<kNvf4>(true) <= 232448, "shared memory per CTA");
 
 struct Tile {
   int a_row, b_row, n_tile, row_hi;
+  int mt;     // grouped modes: the M-tile's index in the tile table
   int k0;     // first K column (A, and B when b_plain)
   int nkb;    // K-blocks of this tile
   int group;  // TC_WGRAD group
@@ -114,7 +138,10 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
                                            int kb_elems = TKB) {
   Tile tl;
   tl.k0 = 0;
-  tl.nkb = p.Kdim / kb_elems;
+  // a ragged last K-block (NVFP4 only) reads zero codes past Kdim
+  const int nkb_all = (p.Kdim + kb_elems - 1) / kb_elems;
+  tl.nkb = nkb_all;
+  tl.mt = 0;
   tl.group = 0;
   tl.expert = 0;
   tl.b_plain = false;
@@ -135,15 +162,16 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
   } else if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
     const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
     tl.a_row = m * TM;
-    tl.b_row = n * (p.Kdim / kb_elems) * TN;  // first K-block tile of B's N-tile n
+    tl.b_row = n * nkb_all * TN;  // first K-block tile of B's N-tile n
     tl.n_tile = n;
     tl.row_hi = p.M;
   } else {
     const int mt = t / p.n_tiles_n, n = t % p.n_tiles_n;  // consecutive CTAs share A
     const TileEntry te = p.tiles[mt];
     tl.expert = te.expert;
+    tl.mt = mt;
     tl.a_row = te.row0;
-    tl.b_row = (te.expert * p.n_tiles_n + n) * (p.Kdim / kb_elems) * TN;
+    tl.b_row = (te.expert * p.n_tiles_n + n) * nkb_all * TN;
     tl.n_tile = n;
     tl.row_hi = te.row_end;
   }
@@ -540,12 +568,15 @@ __device__ __forceinline__ void epi_plain_scaled(uint32_t taddr, bool valid,
 // One tile's epilogue for the calling warp: its 32 accumulator lanes (output
 // rows row = lane's row, valid when inside the tile) and its column halves,
 // by mode.  Shared by the single-CTA and the CTA-pair kernels.
-template <bool kBwd, bool kF8>
+template <bool kBwd, int kQ>
 __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl, uint32_t taddr,
                                               int row, bool valid, int col0, int half0,
                                               OutSink &sink) {
+  // kF8: a quantised-operand GEMM (E4M3 or NVFP4): the accumulator is scaled
+  // by the A row's and the weight row's second-level scales
+  constexpr bool kF8 = kQ != kBf16;
   // one epilogue warp per lane quarter covers both halves, two take one each
-  constexpr int kHalfStep = Cfg<kF8>::EPI_WARPS / 4;
+  constexpr int kHalfStep = Cfg<kQ>::EPI_WARPS / 4;
   // kF8: the A row's scale (rows past the tile's end are not stored)
   const float sa = (kF8 && valid) ? p.a_scale[row] : 0.0f;
   for (int half = half0; half < 2; half += kHalfStep) {
@@ -620,23 +651,29 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
 // kBwd: the instantiation with the backward's epilogues and the TC_WGRAD
 // mode; the forward launches the other one, whose smaller register budget
 // leaves room for the routing kernels that run beside it.
-// kF8: the expert GEMMs with E4M3 operands (TC_EXPERT_GU / TC_EXPERT_DOWN with
-// a_scale and b_scale): tcgen05.mma kind::f8f6f4 over 128-element K-blocks.
-template <bool kBwd, bool kF8>
-__global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
+// kQ: the operand format.  kE4m3 / kNvf4: the expert GEMMs with E4M3 or
+// NVFP4 operands (TC_EXPERT_GU / TC_EXPERT_DOWN with a_scale and b_scale):
+// tcgen05.mma kind::f8f6f4 over 128-element K-blocks, or kind::mxf4nvf4 with
+// 16-element scale blocks over 256-element K-blocks.
+template <bool kBwd, int kQ>
+__global__ void __launch_bounds__(Cfg<kQ>::NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA32, const __grid_constant__ CUtensorMap tmO,
                    const TcParams p) {
-  constexpr int STAGES = Cfg<kF8>::STAGES;
-  constexpr int KB = Cfg<kF8>::KB;
+  constexpr bool kF8 = kQ != kBf16;  // quantised operands with row scales
+  constexpr int STAGES = Cfg<kQ>::STAGES;
+  constexpr int KB = Cfg<kQ>::KB;
+  constexpr int ACC_BUFS = Cfg<kQ>::ACC_BUFS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // [A ring][B ring][control block][tma_out: the epilogue warps' staging buffers]
+  // [A ring][B ring][NVFP4: scale-block ring][control block]
+  // [tma_out: the epilogue warps' staging buffers]
   uint8_t *smA = smem;
   uint8_t *smB = smem + STAGES * A_BYTES;
-  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + Cfg<kF8>::RING_BYTES);
-  uint8_t *staging = smem + Cfg<kF8>::RING_BYTES + CTL_BYTES;
+  uint8_t *smSF = smem + STAGES * (A_BYTES + B_BYTES);
+  SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + Cfg<kQ>::RING_BYTES);
+  uint8_t *staging = smem + Cfg<kQ>::RING_BYTES + CTL_BYTES;
   // TMA stores: the forward instantiations with a bf16-output mode
   const bool use_tma_out = !kBwd && p.tma_out != 0;
   volatile int *abort_flag = &ctl->abort;
@@ -653,7 +690,7 @@ __global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&ctl->acc_full[a], 1);
-      ptx::mbar_init(&ctl->acc_empty[a], Cfg<kF8>::EPI_WARPS);  // one per epilogue warp
+      ptx::mbar_init(&ctl->acc_empty[a], Cfg<kQ>::EPI_WARPS);  // one per epilogue warp
     }
     ptx::mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -692,12 +729,27 @@ __global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
             ok = false;
             break;
           }
-          const int kx = tl.k0 + kb * KB;  // elements = bytes for kF8
+          // A's K coordinate in bytes: elements for bf16 (the map's unit) and
+          // E4M3, half the elements for packed NVFP4
+          const int kx = kQ == kNvf4 ? (tl.k0 + kb * KB) / 2 : tl.k0 + kb * KB;
           // kF8 (weight streaming): a tile of at most 32 token rows loads
           // only those rows of A (the MMA's other rows are never stored)
           const bool a32 = kF8 && tl.row_hi - tl.a_row <= 32;
-          ptx::mbar_arrive_expect_tx(&ctl->full[s], (a32 ? A_BYTES / 4 : A_BYTES) + B_BYTES);
+          ptx::mbar_arrive_expect_tx(&ctl->full[s], (a32 ? A_BYTES / 4 : A_BYTES) + B_BYTES +
+                                                        Cfg<kQ>::SF_BYTES);
           ptx::tma_load_2d(smA + s * A_BYTES, a32 ? &tmA32 : &tmA, &ctl->full[s], kx, tl.a_row);
+          if constexpr (kQ == kNvf4) {
+            // this stage's scale blocks: the A tile's (by M-tile) and the B
+            // tile's (by expert and N-tile), 2 KB and 4 KB, contiguous
+            const int nkb_all = (p.Kdim + KB - 1) / KB;
+            uint8_t *sf = smSF + s * Cfg<kQ>::SF_BYTES;
+            ptx::bulk_load(sf, p.a_sf + (static_cast<size_t>(tl.mt) * nkb_all + kb) * SFA_BYTES,
+                           SFA_BYTES, &ctl->full[s]);
+            ptx::bulk_load(sf + SFA_BYTES,
+                           p.b_sf + ((static_cast<size_t>(tl.expert) * p.n_tiles_n + tl.n_tile) *
+                                         nkb_all + kb) * SFB_BYTES,
+                           SFB_BYTES, &ctl->full[s]);
+          }
           if (tl.b_plain)
             ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kx, tl.b_row);
           else
@@ -716,8 +768,8 @@ __global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
       int it = 0, tl_count = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tl_count) {
-        const int acc = tl_count & 1;
-        const uint32_t acc_ph = (tl_count >> 1) & 1;
+        const int acc = tl_count % ACC_BUFS;
+        const uint32_t acc_ph = (tl_count / ACC_BUFS) & 1;
         if (!ptx::mbar_wait(&ctl->acc_empty[acc], acc_ph ^ 1, abort_flag)) {
           record_failure(p, ctl, DEV_TIMEOUT_MMA);
           ok = false;
@@ -737,10 +789,32 @@ __global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(smA + s * A_BYTES);
           const uint32_t b_addr = ptx::smem_u32(smB + s * B_BYTES);
-          // four MMAs per K-block: K = 16 bf16 or 32 E4M3 elements, 32 bytes each
+          if constexpr (kQ == kNvf4) {
+            // scale blocks into TMEM: MMA k reads A's at SFA_COL + 4k and B's
+            // (two 128-row atoms) at SFB_COL + 8k; executed before the MMAs
+            // below, which this thread issues after them
+            const uint32_t sfa = ptx::smem_u32(smSF + s * Cfg<kQ>::SF_BYTES);
+            const uint32_t sfb = sfa + SFA_BYTES;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              ptx::tmem_cp_32x128b_x4(tmem_base + SFA_COL + 4 * k,
+                                      ptx::smem_desc_rows16(sfa + 512 * k));
+              ptx::tmem_cp_32x128b_x4(tmem_base + SFB_COL + 8 * k,
+                                      ptx::smem_desc_rows16(sfb + 512 * k));
+              ptx::tmem_cp_32x128b_x4(tmem_base + SFB_COL + 8 * k + 4,
+                                      ptx::smem_desc_rows16(sfb + SFA_BYTES + 512 * k));
+            }
+          }
+          // four MMAs per K-block: K = 16 bf16, 32 E4M3 or 64 E2M1 elements,
+          // 32 bytes of each row
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            if constexpr (kF8)
+            if constexpr (kQ == kNvf4)
+              ptx::mma_nvf4(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
+                            ptx::smem_desc_sw128(b_addr + k * 32), IDESC4,
+                            tmem_base + SFA_COL + 4 * k, tmem_base + SFB_COL + 8 * k,
+                            (kb | k) != 0);
+            else if constexpr (kQ == kE4m3)
               ptx::mma_e4m3(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
                             ptx::smem_desc_sw128(b_addr + k * 32), IDESC8, (kb | k) != 0);
             else
@@ -774,8 +848,8 @@ __global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
     sink.issued = 0;
     int tl_count = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl_count) {
-      const int acc = tl_count & 1;
-      const uint32_t acc_ph = (tl_count >> 1) & 1;
+      const int acc = tl_count % ACC_BUFS;
+      const uint32_t acc_ph = (tl_count / ACC_BUFS) & 1;
       // Lane 0 waits; the verdict is broadcast so the warp stays converged
       // for the .sync.aligned TMEM loads below.
       int ok = 1;
@@ -795,7 +869,7 @@ __global__ void __launch_bounds__(Cfg<kF8>::NUM_THREADS, 1)
       // tile's rows past its expert's end belong to the next tile.
       sink.y = tl.a_row + q * 32;
       sink.map = (use_tma_out && sink.y + 31 < tl.row_hi) ? &tmO : nullptr;
-      epilogue_tile<kBwd, kF8>(p, tl, taddr, row, valid, col0, half0, sink);
+      epilogue_tile<kBwd, kQ>(p, tl, taddr, row, valid, col0, half0, sink);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
@@ -891,7 +965,7 @@ __device__ __forceinline__ void record_failure_pair(const TcParams &p, PairCtl *
   if (p.status) atomicCAS(p.status, 0, code);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<false>::NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kBf16>::NUM_THREADS, 1)
     tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -1057,7 +1131,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<false>::NUM_THRE
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * TN;
         sink.y = tl.a_row + q * 32;
         sink.map = (use_tma_out && sink.y + 31 < tl.row_hi) ? &tmO : nullptr;
-        epilogue_tile<false, false>(p, tl, taddr, row, valid, tl.n_tile * TN, half0, sink);
+        epilogue_tile<false, kBf16>(p, tl, taddr, row, valid, tl.n_tile * TN, half0, sink);
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -1177,26 +1251,34 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_done != dev) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<false, false>,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<false, kBf16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes<false>(true)));
+                                         static_cast<int>(smem_bytes<kBf16>(true)));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(tc_gemm_kernel<true, false>,
+      e = cudaFuncSetAttribute(tc_gemm_kernel<true, kBf16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes<false>(false)));
+                               static_cast<int>(smem_bytes<kBf16>(false)));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(tc_gemm_kernel<false, true>,
+      e = cudaFuncSetAttribute(tc_gemm_kernel<false, kE4m3>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes<true>(true)));
+                               static_cast<int>(smem_bytes<kE4m3>(true)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_gemm_kernel<false, kNvf4>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes<kNvf4>(true)));
     if (e != cudaSuccess) return e;
     attr_done = dev;
   }
   const bool bwd = p.mode == TC_WGRAD || p.raw || p.act_dab || p.out_f32 || p.out_h;
-  const bool fp8 = p.b_scale != nullptr;
+  const bool fp8 = p.b_scale != nullptr;      // quantised operands (E4M3 or NVFP4)
+  const bool fp4 = fp8 && p.b_sf != nullptr;  // NVFP4: block scales as well
   if (fp8 && (bwd || !p.a_scale || (p.mode != TC_EXPERT_GU && p.mode != TC_EXPERT_DOWN)))
     return cudaErrorInvalidValue;
+  if (fp4 != (p.a_sf != nullptr)) return cudaErrorInvalidValue;
   if (p.tma_out && (bwd || p.mode == TC_WGRAD || !tmapOut)) return cudaErrorInvalidValue;
-  if (p.Kdim % (fp8 ? TKB8 : TKB) || p.Kdim <= 0) return cudaErrorInvalidValue;
+  // NVFP4: whole 16-element scale blocks and 16-byte rows (a ragged last
+  // K-block is read as zero codes); else whole K-blocks
+  if (p.Kdim <= 0 || (fp4 ? p.Kdim % 32 : p.Kdim % (fp8 ? TKB8 : TKB))) return cudaErrorInvalidValue;
   const int grid = max_ctas < num_sms ? max_ctas : num_sms;
   if (grid <= 0) return cudaSuccess;
   if (fp8 && !tmapA32) return cudaErrorInvalidValue;
@@ -1207,15 +1289,18 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   memcpy(&o, p.tma_out ? tmapOut : tmapA, sizeof(o));
   const bool pdl = p.pdl != 0;
   cudaError_t e;
-  if (fp8)
-    e = launch_ex(tc_gemm_kernel<false, true>, dim3(grid), dim3(Cfg<true>::NUM_THREADS),
-                  smem_bytes<true>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
+  if (fp4)
+    e = launch_ex(tc_gemm_kernel<false, kNvf4>, dim3(grid), dim3(Cfg<kNvf4>::NUM_THREADS),
+                  smem_bytes<kNvf4>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
+  else if (fp8)
+    e = launch_ex(tc_gemm_kernel<false, kE4m3>, dim3(grid), dim3(Cfg<kE4m3>::NUM_THREADS),
+                  smem_bytes<kE4m3>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
   else if (bwd)
-    e = launch_ex(tc_gemm_kernel<true, false>, dim3(grid), dim3(Cfg<false>::NUM_THREADS),
-                  smem_bytes<false>(false), s, pdl, a, b, a32, o, p);
+    e = launch_ex(tc_gemm_kernel<true, kBf16>, dim3(grid), dim3(Cfg<kBf16>::NUM_THREADS),
+                  smem_bytes<kBf16>(false), s, pdl, a, b, a32, o, p);
   else
-    e = launch_ex(tc_gemm_kernel<false, false>, dim3(grid), dim3(Cfg<false>::NUM_THREADS),
-                  smem_bytes<false>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
+    e = launch_ex(tc_gemm_kernel<false, kBf16>, dim3(grid), dim3(Cfg<kBf16>::NUM_THREADS),
+                  smem_bytes<kBf16>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1232,7 +1317,7 @@ cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcP
     // free SMs leaves one idle)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(Cfg<false>::NUM_THREADS, 1, 1);
+    cfg.blockDim = dim3(Cfg<kBf16>::NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = pair_smem_bytes(true);
     int n = 0;
     e = cudaOccupancyMaxActiveClusters(&n, tc_pair_kernel, &cfg);
@@ -1251,7 +1336,7 @@ cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcP
   memcpy(&b, tmapB2, sizeof(b));
   memcpy(&o, p.tma_out ? tmapOut : tmapA, sizeof(o));
   const cudaError_t e =
-      launch_ex(tc_pair_kernel, dim3(2 * pairs), dim3(Cfg<false>::NUM_THREADS),
+      launch_ex(tc_pair_kernel, dim3(2 * pairs), dim3(Cfg<kBf16>::NUM_THREADS),
                 pair_smem_bytes(p.tma_out != 0), s, p.pdl != 0, a, b, o, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -24,7 +24,7 @@ _lib = C.CDLL(_LIB_PATH)
 LMOE_EFF, LMOE_ACC = 0, 1
 LMOE_F32, LMOE_BF16 = 0, 1
 LMOE_SWIGLU, LMOE_RELU2 = 0, 1
-LMOE_WEIGHTS_BF16, LMOE_WEIGHTS_FP8 = 0, 1
+LMOE_WEIGHTS_BF16, LMOE_WEIGHTS_FP8, LMOE_WEIGHTS_NVFP4 = 0, 1, 2
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -3: "LMOE_ERR_NOT_LOADED", -4: "LMOE_ERR_TOO_MANY_TOKENS", -5: "LMOE_ERR_CUDA",
           -6: "LMOE_ERR_DEVICE_TIMEOUT", -7: "LMOE_ERR_UNSUPPORTED",
@@ -133,7 +133,8 @@ def config_from(cfg: LayerConfig, max_tokens: int | None = None,
         max_tokens=cfg.T if max_tokens is None else max_tokens,
         activation=LMOE_RELU2 if cfg.activation == "relu2" else LMOE_SWIGLU,
         training=int(training),
-        weight_format=LMOE_WEIGHTS_FP8 if cfg.weights == "fp8" else LMOE_WEIGHTS_BF16,
+        weight_format={"fp8": LMOE_WEIGHTS_FP8, "nvfp4": LMOE_WEIGHTS_NVFP4}.get(
+            cfg.weights, LMOE_WEIGHTS_BF16),
         ep_rank=ep_rank, ep_world=ep_world)
 
 

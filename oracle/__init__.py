@@ -142,11 +142,13 @@ class Layer:
     act_fp4: the same with NVFP4 activations (nvfp4_rows' rule: E2M1 codes,
     an E4M3 scale per 16 elements, a power-of-two row scale); l and m must
     be multiples of 16.
+    act_bf16: the quantised rows are rounded to bf16 first, as a bf16 layer
+    always does (for a float64 layer standing for a bf16 one).
     """
 
     def __init__(self, *, w_router, b_router, w_down, w_up, w_gate, w_upx,
                  w_out, s_gate, s_up, s_out, k_active, activation="swiglu",
-                 act_fp8=False, act_fp4=False):
+                 act_fp8=False, act_fp4=False, act_bf16=False):
         if act_fp8 and act_fp4:
             raise ValueError("act_fp8 and act_fp4 are exclusive")
         if activation not in ("swiglu", "relu2"):
@@ -182,7 +184,8 @@ class Layer:
                          _ptr(k["w_router"]), _ptr(self.b_router), _ptr(k["w_down"]),
                          _ptr(k["w_up"]), _ptr(k["w_gate"]), _ptr(k["w_upx"]),
                          _ptr(k["w_out"]), _ptr(k["s_gate"]), _ptr(k["s_up"]),
-                         _ptr(k["s_out"]), 1 if act_fp8 else (2 if act_fp4 else 0))
+                         _ptr(k["s_out"]),
+                         (1 if act_fp8 else (2 if act_fp4 else 0)) | (16 if act_bf16 else 0))
         self.act_fp8 = bool(act_fp8)
         self.act_fp4 = bool(act_fp4)
 
@@ -356,8 +359,8 @@ def fp8_rows(w):
 def nvfp4_rows(w):
     """Row-wise NVFP4 quantisation (E2M1 codes, an E4M3 scale per 16
     elements, a power-of-two row scale; see the C source): returns (W'
-    dequantised, float64, same shape; row scales [rows]; block scales
-    [rows][cols/16])."""
+    dequantised, float64, same shape; row scales [rows]; block scales, the
+    shape of W with cols/16 in place of cols)."""
     w = np.ascontiguousarray(w)
     code = _dtype_code(w)
     cols = w.shape[-1]
@@ -366,7 +369,7 @@ def nvfp4_rows(w):
     rows = w.size // cols
     wq = np.empty(w.shape, dtype=np.float64)
     sc = np.empty(rows, dtype=np.float64)
-    bs = np.empty((rows, cols // 16), dtype=np.float64)
+    bs = np.empty(w.shape[:-1] + (cols // 16,), dtype=np.float64)
     rc = _load().oracle_nvfp4_rows(_ptr(w), code, rows, cols, _ptr(wq), _ptr(sc), _ptr(bs))
     if rc != 0:
         raise ValueError(f"oracle_nvfp4_rows failed ({rc})")

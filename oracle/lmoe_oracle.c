@@ -55,7 +55,7 @@
 enum { ODT_F32 = 0, ODT_BF16 = 1, ODT_F64 = 2 };
 
 enum { OACT_SWIGLU = 0, OACT_RELU2 = 1 };
-enum { OQ_NONE = 0, OQ_E4M3 = 1, OQ_NVFP4 = 2 };  /* activation quantisation */
+enum { OQ_NONE = 0, OQ_E4M3 = 1, OQ_NVFP4 = 2, OQ_MODE = 3, OQ_BF16_ROWS = 16 };
 
 typedef struct {
   int32_t d, l, m, n_routed, k_active, n_shared, m_shared;
@@ -72,7 +72,8 @@ typedef struct {
   const void *s_up;          /* [n_s][m_s][d] */
   const void *s_out;         /* [n_s][d][m_s] */
   int32_t act_quant;         /* routed experts' activations: OQ_NONE, OQ_E4M3 (q_vec_e4m3)
-                                or OQ_NVFP4 (q_vec_nvfp4) */
+                                or OQ_NVFP4 (q_vec_nvfp4), plus OQ_BF16_ROWS: the rows
+                                are rounded to bf16 first (see q_act) */
 } oracle_layer;
 
 /* Exact widening of one stored element to double. */
@@ -108,7 +109,7 @@ static double relu2(double a) { return a > 0.0 ? a * a : 0.0; }
  * Squared ReLU: out = W_o (relu(W_u v))^2  ([Explained], the Expert class:
  * up, relu, square, down).
  * W_g, W_u: [hid][in_w] at element offset off_in; W_o: [out_w][hid] at off_out. */
-static void q_act(int mode, double *v, int n);
+static void q_act(const oracle_layer *L, int mode, double *v, int n);
 
 /* quant_hidden: the hidden vector is replaced by its row quantisation in
  * that mode (OQ_E4M3 or OQ_NVFP4) before the down-projection (the routed
@@ -126,7 +127,7 @@ static void swiglu_ffn(const oracle_layer *L, const void *Wg, const void *Wu,
     matvec(Wu, L->dtype, off_in, hid, in_w, v, b);
     for (int j = 0; j < hid; ++j) a[j] = silu(a[j]) * b[j];
   }
-  if (quant_hidden) q_act(quant_hidden, a, hid);
+  if (quant_hidden) q_act(L, quant_hidden, a, hid);
   matvec(Wo, L->dtype, off_out, out_w, hid, a, out);
 }
 
@@ -267,8 +268,8 @@ int oracle_forward(const oracle_layer *L, const void *x, int64_t T,
                    double *y, int32_t *ids_out, double *gates_out) {
   const int d = L->d, l = L->l, m = L->m, N = L->n_routed, K = L->k_active;
   if (K < 1 || K > N || l < 1 || d < 1 || m < 1) return -1;
-  if (L->act_quant < OQ_NONE || L->act_quant > OQ_NVFP4) return -1;
-  if (L->act_quant == OQ_NVFP4 && (l % 16 || m % 16)) return -1;  /* whole 16-blocks */
+  if (L->act_quant & ~(OQ_MODE | OQ_BF16_ROWS) || (L->act_quant & OQ_MODE) == OQ_MODE) return -1;
+  if ((L->act_quant & OQ_MODE) == OQ_NVFP4 && (l % 16 || m % 16)) return -1;  /* 16-blocks */
   int err = 0;
 #pragma omp parallel
   {
@@ -296,7 +297,7 @@ int oracle_forward(const oracle_layer *L, const void *x, int64_t T,
       }
       for (int i = 0; i < d; ++i) xv[i] = elem(x, L->dtype, (size_t)t * d + i);
       matvec(L->w_down, L->dtype, 0, l, d, xv, z);
-      if (L->act_quant) q_act(L->act_quant, z, l);  /* the experts read z quantised */
+      if (L->act_quant) q_act(L, L->act_quant, z, l);  /* the experts read z quantised */
       for (int i = 0; i < l; ++i) u[i] = 0.0;
       for (int k = 0; k < K; ++k) { /* slot loop, in slot order */
         const int e = ids[k];
@@ -807,7 +808,27 @@ static void q_vec_nvfp4(double *v, int n) {
   free(xf);
 }
 
-static void q_act(int mode, double *v, int n) {
+/* v rounded to the nearest bf16 value (through single precision, ties to
+ * even): the precision in which a bf16 layer holds z and h. */
+static double round_bf16(double v) {
+  float f = (float)v;
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  if ((u & 0x7F800000u) != 0x7F800000u) u += 0x7FFFu + ((u >> 16) & 1u);
+  u &= 0xFFFF0000u;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* The quantisation of an expert's activation row.  A code is an integer that
+ * floating point decides, so it is decided on the values in the precision
+ * the layer holds them in: for a bf16 layer (or with OQ_BF16_ROWS, a layer
+ * whose other weights stand for bf16 ones) the row is first rounded to bf16
+ * (z and h are bf16 vectors there). */
+static void q_act(const oracle_layer *L, int mode, double *v, int n) {
+  if (L->dtype == ODT_BF16 || (L->act_quant & OQ_BF16_ROWS))
+    for (int i = 0; i < n; ++i) v[i] = round_bf16(v[i]);
+  mode &= OQ_MODE;
   if (mode == OQ_E4M3) q_vec_e4m3(v, n);
   else if (mode == OQ_NVFP4) q_vec_nvfp4(v, n);
 }

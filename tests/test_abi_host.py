@@ -72,6 +72,10 @@ def _cfg(**kw):
     # world, a negative world, and the fp32 mode (bf16 only)
     (dict(dtype=1, ep_world=3, ep_rank=0), -1), (dict(dtype=1, ep_world=2, ep_rank=2), -1),
     (dict(ep_world=-1), -1), (dict(ep_world=2, ep_rank=1), -7),
+    # routed-expert formats: unknown; NVFP4 in the fp32 mode; NVFP4 with
+    # l = 64 (quantised experts need l and m multiples of 128)
+    (dict(weight_format=3), -1), (dict(weight_format=2), -7),
+    (dict(dtype=1, weight_format=2, alpha=4), -7),
 ])
 def test_create_rejects_bad_configs_on_host(lib, kw, code):
     from latent_mixture_experts_top_b200 import lmoe

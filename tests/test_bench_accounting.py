@@ -16,7 +16,8 @@ from latent_mixture_experts_top_b200 import configs
 from oracle import costs
 
 SWIGLU = [configs.README_ACC, configs.README_EFF, configs.PREFILL, configs.DECODE]
-ALL = SWIGLU + [configs.RELU2_95B, configs.DECODE_FP8, configs.RELU2_95B_FP8]
+ALL = SWIGLU + [configs.RELU2_95B, configs.DECODE_FP8, configs.RELU2_95B_FP8,
+               configs.DECODE_NVFP4, configs.RELU2_95B_NVFP4]
 
 
 def _shared_gate_up_flops(cfg):
@@ -102,3 +103,13 @@ def test_stage_bound_picks_the_slower_roof():
     assert bench.stage_bound(2e12, 1e9, peaks) == "tensor"    # 2 ms of math, 1 ms of bytes
     assert bench.stage_bound(1e12, 2e9, peaks) == "hbm"
     assert bench.stage_bound(0.0, 0.0, peaks) == "hbm"     # a memory-only helper
+
+
+def test_nvfp4_experts_take_half_a_byte_and_a_sixteenth_per_weight():
+    """E2M1 codes (4 bits) plus one E4M3 block scale per 16 weights."""
+    bf, f4 = configs.DECODE, configs.DECODE_NVFP4
+    per_weight = 0.5 + 1.0 / 16
+    assert bench.layer_bytes(bf) - bench.layer_bytes(f4) == pytest.approx(
+        bf.n_routed * 3 * bf.l * bf.m * (2.0 - per_weight))
+    w4 = bench.stage_work(f4)
+    assert w4[4][1] == pytest.approx(f4.n_routed * 2 * f4.m * f4.l * per_weight)

@@ -39,11 +39,22 @@ def _q(v, mode="e4m3"):
     return (oracle.fp8_rows(v) if mode == "e4m3" else oracle.nvfp4_rows(v))[0][0]
 
 
+def _bf16(a):
+    """float64 -> bf16 bit patterns, rounded to nearest even through float32."""
+    u = np.asarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _widen(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 def _silu(a):
     return a / (1.0 + np.exp(-a))
 
 
-def _recompose(kw, x, act_fp8, mode="e4m3"):
+def _recompose(kw, x, act_fp8, mode="e4m3", rnd=False):
+    r = (lambda v: _widen(_bf16(v))) if rnd else (lambda v: v)
     Lp = oracle.Layer(**kw)                        # unquantised: router and ids only
     s = oracle.router_logits(Lp, x)
     ids, g = oracle.select(s, K)
@@ -52,14 +63,14 @@ def _recompose(kw, x, act_fp8, mode="e4m3"):
     for t in range(x.shape[0]):
         z = kw["w_down"] @ x[t]
         if act_fp8:
-            z = _q(z, mode)
+            z = _q(r(z), mode)
         u = np.zeros(L_)
         for k in range(K):
             e = ids[t, k]
             b = kw["w_upx"][e] @ z
             h = np.maximum(b, 0.0) ** 2 if relu2 else _silu(kw["w_gate"][e] @ z) * b
             if act_fp8:
-                h = _q(h, mode)
+                h = _q(r(h), mode)
             u += g[t, k] * (kw["w_out"][e] @ h)
         y[t] = kw["w_up"] @ u
         for j in range(NS):
@@ -83,6 +94,25 @@ def test_act_fp8_forward_is_the_quantised_recomposition(activation, mode):
     # and it is not the unquantised layer
     y0 = _recompose(kw, x, False)
     assert np.abs(y - y0).max() > 1e-4 * np.abs(y0).max()
+
+
+@pytest.mark.parametrize("mode", ["e4m3", "nvfp4"])
+def test_bf16_layer_quantises_the_bf16_rounding_of_each_row(mode):
+    """In a bf16 layer z and h are bf16 vectors: their codes are decided on
+    the bf16 values (the precision the layer holds them in)."""
+    kw, x = _weights(6, "swiglu")
+    bits = {k: (_bf16(v) if isinstance(v, np.ndarray) else v) for k, v in kw.items()}
+    xb = _bf16(x)
+    y, _, _ = oracle.forward(oracle.Layer(**bits, **_flag(mode)), xb)
+    wide = {k: (_widen(v) if isinstance(v, np.ndarray) else v) for k, v in bits.items()}
+    y_ref = _recompose(wide, _widen(xb), True, mode, rnd=True)
+    np.testing.assert_allclose(y, y_ref, rtol=0, atol=1e-12 * np.abs(y_ref).max())
+    # a float64 layer with act_bf16 is the same layer
+    y64, _, _ = oracle.forward(oracle.Layer(**wide, **_flag(mode), act_bf16=True), _widen(xb))
+    np.testing.assert_allclose(y64, y_ref, rtol=0, atol=1e-12 * np.abs(y_ref).max())
+    # and the rounding decides some codes: without it the result differs
+    y_unrounded = _recompose(wide, _widen(xb), True, mode, rnd=False)
+    assert np.abs(y_unrounded - y_ref).max() > 1e-9 * np.abs(y_ref).max()
 
 
 def test_act_fp8_off_leaves_the_layer_unchanged():
@@ -117,13 +147,15 @@ def test_backward_refuses_quantised_activations(mode):
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "lmoe_oracle.c")
 MUTATIONS = {
-    "no_hidden_quantisation": ("  if (quant_hidden) q_act(quant_hidden, a, hid);\n", "\n"),
-    "no_z_quantisation": ("      if (L->act_quant) q_act(L->act_quant, z, l);  /* the experts read z quantised */\n",
+    "no_hidden_quantisation": ("  if (quant_hidden) q_act(L, quant_hidden, a, hid);\n", "\n"),
+    "no_z_quantisation": ("      if (L->act_quant) q_act(L, L->act_quant, z, l);  /* the experts read z quantised */\n",
                           "\n"),
     "shared_quantised_too": ("(size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, 0);",
                              "(size_t)j * d * L->m_shared, d, L->m_shared, d, xv, sh, scratch, L->act_quant);"),
-    "quantised_after_down": ("  if (quant_hidden) q_act(quant_hidden, a, hid);\n  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);",
-                             "  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);\n  if (quant_hidden) q_act(quant_hidden, out, out_w);"),
+    "quantised_after_down": ("  if (quant_hidden) q_act(L, quant_hidden, a, hid);\n  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);",
+                             "  matvec(Wo, L->dtype, off_out, out_w, hid, a, out);\n  if (quant_hidden) q_act(L, quant_hidden, out, out_w);"),
+    "no_bf16_rounding": ("  if (L->dtype == ODT_BF16 || (L->act_quant & OQ_BF16_ROWS))\n    for (int i = 0; i < n; ++i) v[i] = round_bf16(v[i]);\n",
+                         "\n"),
     "modes_swapped": ("  if (mode == OQ_E4M3) q_vec_e4m3(v, n);\n  else if (mode == OQ_NVFP4) q_vec_nvfp4(v, n);",
                       "  if (mode == OQ_NVFP4) q_vec_e4m3(v, n);\n  else if (mode == OQ_E4M3) q_vec_nvfp4(v, n);"),
 }
@@ -144,5 +176,6 @@ def test_act_fp8_pins_catch_mutation(name, mode, tmp_path):
     try:
         with pytest.raises(AssertionError):
             test_act_fp8_forward_is_the_quantised_recomposition("swiglu", mode)
+            test_bf16_layer_quantises_the_bf16_rounding_of_each_row(mode)
     finally:
         oracle._swap_library(None)

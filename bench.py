@@ -60,19 +60,26 @@ def parse_args():
                     help="expert parallelism over this many ranks: under torchrun with as many "
                          "GPUs, one rank per GPU with NCCL all-to-alls; on one GPU, that many "
                          "ranks emulated in one process (copies for the exchange)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count T (a smaller case of the same "
+                         "layer, e.g. for a profiler capture); the line's config names it")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
                     help="backward: time lmoe_backward (dx and every weight gradient, "
                          "forward activations recomputed) instead of the forward")
     return ap.parse_args()
 
 
-def workload(name):
+def workload(name, tokens=None):
+    from dataclasses import replace
     from latent_mixture_experts_top_b200 import configs
-    return {"readme_acc": configs.README_ACC, "readme_eff": configs.README_EFF,
-            "prefill": configs.PREFILL, "decode": configs.DECODE,
-            "relu2_95b": configs.RELU2_95B, "decode_fp8": configs.DECODE_FP8,
-            "relu2_95b_fp8": configs.RELU2_95B_FP8, "decode_nvfp4": configs.DECODE_NVFP4,
-            "relu2_95b_nvfp4": configs.RELU2_95B_NVFP4}[name]
+    cfg = {"readme_acc": configs.README_ACC, "readme_eff": configs.README_EFF,
+           "prefill": configs.PREFILL, "decode": configs.DECODE,
+           "relu2_95b": configs.RELU2_95B, "decode_fp8": configs.DECODE_FP8,
+           "relu2_95b_fp8": configs.RELU2_95B_FP8, "decode_nvfp4": configs.DECODE_NVFP4,
+           "relu2_95b_nvfp4": configs.RELU2_95B_NVFP4}[name]
+    if tokens is not None and tokens != cfg.T:
+        cfg = replace(cfg, name=f"{cfg.name}@T{tokens}", T=tokens)
+    return cfg
 
 
 def n_mats(cfg):
@@ -289,7 +296,7 @@ def run_reference(args):
     import torch
     import oracle
     from latent_mixture_experts_top_b200 import synth
-    cfg = workload(args.workload)
+    cfg = workload(args.workload, args.tokens)
     inp = synth.make_inputs(cfg, args.seed, "cpu")
     n = numpy_inputs(inp)
     rate_cal, _, _, cores, L = oracle_rate(cfg, n, budget_s=2.0, max_tokens=64)
@@ -393,7 +400,7 @@ def run_ours(args):
     def allmax(v):
         return reduce_max_over_ranks(v, world, "cuda")
 
-    cfg = workload(args.workload)
+    cfg = workload(args.workload, args.tokens)
     inp = synth.make_inputs(cfg, args.seed, "cuda")
     layer = lmoe.LatentMoELayer(cfg, inp)
     x = inp["x"]
@@ -549,7 +556,7 @@ def run_backward(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    cfg = workload(args.workload)
+    cfg = workload(args.workload, args.tokens)
     inp = synth.make_inputs(cfg, args.seed, "cuda")
     dy = synth.make_cotangent(cfg, args.seed, "cuda")
     layer = lmoe.LatentMoELayer(cfg, inp, training=True)
@@ -640,7 +647,7 @@ def run_ep(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    cfg = workload(args.workload)
+    cfg = workload(args.workload, args.tokens)
     inp = synth.make_inputs(cfg, args.seed, "cuda")       # same weights on every rank
     ranks = range(W) if emulated else [rank]
     layers = [lmoe.LatentMoELayer(cfg, inp, ep_rank=r, ep_world=W) for r in ranks]

@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(256) quantize_w_nvfp4_kernel(
 // One block per M-tile of the tile table, one warp per row in turn: the row
 // p = row0 + i of the tile reads src row (gather ? gather[p] / K : p) and
 // writes codes row p, scales[p] and the tile's block-scale atoms (scales of
-// 16-blocks past cols as zero, so a ragged last K-block adds nothing).
+// 16-blocks past cols as zero: the ragged last K-block's zero codes then add
+// nothing).
 __global__ void __launch_bounds__(256) quantize_act_nvfp4_kernel(
     const __nv_bfloat16 *__restrict__ src, const int32_t *__restrict__ gather, int K,
     const TileEntry *__restrict__ tiles, const int32_t *__restrict__ n_tiles, int cols,
@@ -152,15 +153,11 @@ __global__ void __launch_bounds__(256) quantize_act_nvfp4_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = (cols + kKb - 1) / kKb, nblk = cols / 16;
   uint8_t *tsf = sf + static_cast<size_t>(mt) * nkb * 4 * kAtom;
-  for (int i = warp; i < 128; i += 8) {
+  // Rows past the expert's end are left as they are: an accumulator row
+  // depends only on its own A row and scales, and those rows are never stored.
+  const int n_rows = min(128, te.row_end - te.row0);
+  for (int i = warp; i < n_rows; i += 8) {
     const int p = te.row0 + i;
-    if (p >= te.row_end) {
-      // rows past the expert's end: their accumulator rows are never stored,
-      // but keep the scales finite
-      for (int blk = lane; blk < nkb * 16; blk += 32)
-        tsf[((blk >> 4) * 4 + ((blk >> 2) & 3)) * kAtom + atom_byte(i, blk & 3)] = 0;
-      continue;
-    }
     const int srow = gather ? gather[p] / K : p;
     const uint4 *w = reinterpret_cast<const uint4 *>(src + static_cast<size_t>(srow) * cols);
     const int e = nvfp4_row_exp(row_amax(w, cols / 8, lane));

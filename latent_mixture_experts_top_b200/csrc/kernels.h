@@ -241,7 +241,8 @@ cudaError_t launch_quantize_nvfp4_tiles(const __nv_bfloat16 *src, int groups, in
 // gather[p] / K : p] (row stride cols) and writes the packed codes row p of
 // codes [rows][cols / 2], scales[p] and, per K-block, the tile's four 512-byte
 // block-scale atoms (sf: nvfp4_act_sf_bytes(max_tiles, cols) bytes; scales of
-// rows past the tile's expert and of blocks past cols are zero).
+// blocks past cols are zero; the atoms' rows past the tile's expert are not
+// written).
 size_t nvfp4_act_sf_bytes(int max_tiles, int cols);
 cudaError_t launch_quantize_act_nvfp4(const __nv_bfloat16 *src, const int32_t *gather, int K,
                                       const TileEntry *tiles, const int32_t *n_tiles,

@@ -97,16 +97,22 @@ __device__ __forceinline__ uint8_t nvfp4_block(const uint4 lo, const uint4 hi, i
 // of its 64-element slice.
 __device__ __forceinline__ int atom_byte(int i, int q) { return 16 * (i & 31) + 4 * (i >> 5) + q; }
 
-// Warp-wide max |x| over one bf16 row of nv 16-byte vectors.
+// Warp-wide max |x| over one bf16 row of nv 16-byte vectors (four loads in
+// flight per lane).
 __device__ __forceinline__ float row_amax(const uint4 *w, int nv, int lane) {
   float amax = 0.0f;
-  for (int v = lane; v < nv; v += 32) {
-    const uint4 q = w[v];
-    const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+  for (int v0 = lane; v0 < nv; v0 += 128) {
+    uint4 q[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] << 16)));
-      amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] & 0xFFFF0000u)));
+    for (int u = 0; u < 4; ++u) q[u] = v0 + 32 * u < nv ? w[v0 + 32 * u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t qs[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] << 16)));
+        amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] & 0xFFFF0000u)));
+      }
     }
   }
 #pragma unroll
@@ -137,7 +143,8 @@ __global__ void __launch_bounds__(256) quantize_w_nvfp4_kernel(
   }
 }
 
-// One block per M-tile of the tile table, one warp per row in turn: the row
+// Block (mt, j) takes rows 8j .. 8j + 7 of M-tile mt of the tile table, one
+// warp per row (every row of the layer in flight at once): the row
 // p = row0 + i of the tile reads src row (gather ? gather[p] / K : p) and
 // writes codes row p, scales[p] and the tile's block-scale atoms (scales of
 // 16-blocks past cols as zero: the ragged last K-block's zero codes then add
@@ -155,8 +162,8 @@ __global__ void __launch_bounds__(256) quantize_act_nvfp4_kernel(
   uint8_t *tsf = sf + static_cast<size_t>(mt) * nkb * 4 * kAtom;
   // Rows past the expert's end are left as they are: an accumulator row
   // depends only on its own A row and scales, and those rows are never stored.
-  const int n_rows = min(128, te.row_end - te.row0);
-  for (int i = warp; i < n_rows; i += 8) {
+  const int i = blockIdx.y * 8 + warp;
+  if (i < min(128, te.row_end - te.row0)) {
     const int p = te.row0 + i;
     const int srow = gather ? gather[p] / K : p;
     const uint4 *w = reinterpret_cast<const uint4 *>(src + static_cast<size_t>(srow) * cols);
@@ -212,7 +219,7 @@ cudaError_t launch_quantize_act_nvfp4(const __nv_bfloat16 *src, const int32_t *g
                                       uint8_t *sf, cudaStream_t s, bool pdl) {
   if (max_tiles <= 0) return cudaSuccess;
   if (cols % 32 || cols <= 0 || (gather && K <= 0)) return cudaErrorInvalidValue;
-  const cudaError_t e = launch_ex(quantize_act_nvfp4_kernel, dim3(max_tiles), dim3(256), 0, s, pdl,
+  const cudaError_t e = launch_ex(quantize_act_nvfp4_kernel, dim3(max_tiles, 16), dim3(256), 0, s, pdl,
                                   src, gather, K, tiles, n_tiles, cols, codes, scales, sf);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -46,16 +46,22 @@ __device__ __forceinline__ uint2 e4m3x8(const uint4 q, float inv) {
   return make_uint2(out[0], out[1]);
 }
 
-// Warp-wide max |x| over one bf16 row of nv 16-byte vectors.
+// Warp-wide max |x| over one bf16 row of nv 16-byte vectors (four loads in
+// flight per lane).
 __device__ __forceinline__ float row_amax(const uint4 *w, int nv, int lane) {
   float amax = 0.0f;
-  for (int v = lane; v < nv; v += 32) {
-    const uint4 q = w[v];
-    const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+  for (int v0 = lane; v0 < nv; v0 += 128) {
+    uint4 q[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] << 16)));
-      amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] & 0xFFFF0000u)));
+    for (int u = 0; u < 4; ++u) q[u] = v0 + 32 * u < nv ? w[v0 + 32 * u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t qs[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] << 16)));
+        amax = fmaxf(amax, fabsf(__uint_as_float(qs[i] & 0xFFFF0000u)));
+      }
     }
   }
 #pragma unroll

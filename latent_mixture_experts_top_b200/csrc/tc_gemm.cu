@@ -565,6 +565,65 @@ __device__ __forceinline__ void epi_plain_scaled(uint32_t taddr, bool valid,
   }
 }
 
+// NVFP4 GEMM (one accumulator): the calling warp copies its half of the tile
+// (128 accumulator columns of its 32 lanes) into registers and releases the
+// accumulator at once, so that the next tile's MMAs overlap the scaling,
+// activation and stores that follow.  Modes: TC_EXPERT_GU (SwiGLU or squared
+// ReLU) and TC_EXPERT_DOWN, as in the kF8 branches of epilogue_tile.
+__device__ __forceinline__ void epilogue_tile_release_early(const TcParams &p, const Tile &tl,
+                                                            uint32_t taddr, int row, bool valid,
+                                                            int col0, int half, OutSink &sink,
+                                                            uint64_t *acc_empty, int lane) {
+  const bool gu = p.mode == TC_EXPERT_GU, swiglu = gu && !p.relu2;
+  // register block j: SwiGLU gate, up, gate, up of chunks 2h, 2h + 1
+  // (columns c 32 and TN / 2 + c 32); else chunks 4h .. 4h + 3
+  uint32_t a[4][32];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int col = swiglu ? (2 * half + (j >> 1)) * 32 + (j & 1) * (TN / 2) : (4 * half + j) * 32;
+    ptx::tmem_ld_32x32b_x32(taddr + col, a[j]);
+  }
+  ptx::tmem_ld_wait();
+  ptx::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) ptx::mbar_arrive(acc_empty);
+  const float sa = valid ? p.a_scale[row] : 0.0f;
+  const float *scl = p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0;
+  __nv_bfloat16 *dst = p.out + static_cast<size_t>(row) * p.ld_out;
+  if (swiglu) {
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int c = 2 * half + c2;
+      float h[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        h[j] = silu_bf16out(__uint_as_float(a[2 * c2][j]) * (sa * scl[c * 32 + j])) *
+               (__uint_as_float(a[2 * c2 + 1][j]) * (sa * scl[TN / 2 + c * 32 + j]));
+      const int hcol = col0 / 2 + c * 32;
+      if (sink.map) sink_store(sink, h, hcol);
+      else if (valid) store_bf16x32(dst + hcol, h);
+    }
+  } else {
+    const int n_cols = gu ? p.n_cols2 : p.ld_out;
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const int c = 4 * half + j4, col = col0 + c * 32;
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float t = __uint_as_float(a[j4][j]) * (sa * scl[c * 32 + j]);
+        const float r = fmaxf(t, 0.0f);
+        v[j] = gu ? r * r : t;  // squared ReLU hidden, or the plain output
+      }
+      if (sink.map) {
+        if (col < n_cols) sink_store(sink, v, col);
+      } else if (valid && col < n_cols) {
+        store_bf16x32(dst + col, v);
+      }
+    }
+  }
+}
+
 // One tile's epilogue for the calling warp: its 32 accumulator lanes (output
 // rows row = lane's row, valid when inside the tile) and its column halves,
 // by mode.  Shared by the single-CTA and the CTA-pair kernels.
@@ -869,10 +928,17 @@ __global__ void __launch_bounds__(Cfg<kQ>::NUM_THREADS, 1)
       // tile's rows past its expert's end belong to the next tile.
       sink.y = tl.a_row + q * 32;
       sink.map = (use_tma_out && sink.y + 31 < tl.row_hi) ? &tmO : nullptr;
-      epilogue_tile<kBwd, kQ>(p, tl, taddr, row, valid, col0, half0, sink);
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
+      if constexpr (kQ == kNvf4) {
+        // one warp per half of the tile (two per lane quarter); the
+        // accumulator is released inside, as soon as it is in registers
+        epilogue_tile_release_early(p, tl, taddr, row, valid, col0, half0, sink,
+                                    &ctl->acc_empty[acc], lane);
+      } else {
+        epilogue_tile<kBwd, kQ>(p, tl, taddr, row, valid, col0, half0, sink);
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
+      }
     }
     // the staging buffers stay allocated until this warp's stores are done
     if (use_tma_out && lane == 0) ptx::bulk_wait_group_all();

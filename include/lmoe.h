@@ -73,8 +73,9 @@ typedef enum { LMOE_SWIGLU = 0, LMOE_RELU2 = 1 } lmoe_activation;
  * published one): E2M1 codes, one E4M3 scale per 16 consecutive elements of
  * a row, and a second-level power-of-two scale per row (the smallest with
  * the row's largest magnitude within 6 * 448).  Block scale b =
- * E4M3(block max / (6 s_row)), code = E2M1(x / (b s_row)), both divisions in
- * IEEE single precision, rounding to nearest even with saturation.  The
+ * E4M3(block max / (6 s_row)), code = E2M1(x * rcp) with rcp = 1 / (b s_row)
+ * rounded once, all in IEEE single precision, rounding to nearest even with
+ * saturation.  The
  * expert GEMMs run tcgen05 kind::mxf4nvf4 (the tensor cores apply the block
  * scales, fp32 accumulation).  Same limits as LMOE_WEIGHTS_FP8. */
 typedef enum {

@@ -7,9 +7,11 @@
 // consecutive elements of a row.  The second-level scale is taken per row
 // here: s_r = 2^e_r, the smallest power of two with max |row| <= 6 * 448 s_r.
 // Block j of the row: b_j = E4M3(amax_j / (6 s_r)); each element's code is
-// E2M1(x / (b_j s_r)), both rounded to nearest even with saturation, both
-// divisions IEEE single precision (they decide codes); a block with b_j = 0
-// has all-zero codes.  The GEMM's tensor cores apply b_j (kind::mxf4nvf4),
+// E2M1(x * rcp_j) with rcp_j = 1 / (b_j s_r) rounded once (the element scaled
+// by the reciprocal of its decoded block scale), both roundings to nearest
+// even with saturation; the division, the reciprocal and the product are IEEE
+// single precision (they decide codes).  A block with b_j = 0 has all-zero
+// codes.  The GEMM's tensor cores apply b_j (kind::mxf4nvf4),
 // its epilogue s_r.
 //
 // Layouts (the GEMM's, see TcParams):
@@ -85,10 +87,10 @@ __device__ __forceinline__ uint8_t nvfp4_block(const uint4 lo, const uint4 hi, i
     *codes = make_uint2(0u, 0u);
     return 0;
   }
-  const float den = ldexpf(b, e);  // exact: 4 significant bits times 2^e
+  const float rcp = __frcp_rn(ldexpf(b, e));  // b 2^e is exact: 4 significant bits
   float y[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(v[i], den);
+  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(v[i], rcp);
   *codes = make_uint2(e2m1x8(y), e2m1x8(y + 8));
   return static_cast<uint8_t>(bc);
 }

@@ -715,13 +715,16 @@ static void q_vec_e4m3(double *v, int n) {
  * row: s_r, the smallest power of two with amax_r <= 6 * 448 * s_r, so that
  * every block scale falls in E4M3's range.  Block j of the row gets
  *   b_j = E4M3(amax_j / (6 s_r)),
- * each of its elements the code q = E2M1(x / (b_j s_r)) (0 for the whole
- * block when b_j = 0), and the value the layer uses is q b_j s_r.  Both
- * divisions decide codes, so they are taken in IEEE single precision (round
- * to nearest) on the elements' single-precision values: the precision the
- * GPU's quantisers take them in.  (b_j s_r is exact in single precision: a
- * 4-significant-bit value times a power of two.)  E2M1 rounding is to
- * nearest, ties to the even mantissa, and magnitudes above 6 saturate. */
+ * each of its elements the code q = E2M1(x * rcp_j) with rcp_j = 1 / (b_j
+ * s_r) rounded once (0 for the whole block when b_j = 0): the element is
+ * scaled by the reciprocal of its decoded block scale, as scaling to a
+ * low-precision format is done in practice; the value the layer uses is
+ * q b_j s_r.  The division, the reciprocal and the product decide codes, so
+ * they are taken in IEEE single precision (round to nearest) on the
+ * elements' single-precision values: the precision the GPU's quantisers
+ * take them in.  (b_j s_r is exact in single precision: a 4-significant-bit
+ * value times a power of two.)  E2M1 rounding is to nearest, ties to the
+ * even mantissa, and magnitudes above 6 saturate. */
 static double e2m1_round(double v) {
   const double a = fabs(v);
   double r;
@@ -770,9 +773,10 @@ static void nvfp4_row(const float *x, int n, double *out, double *row_scale,
     const double b = e4m3_round((double)t);
     if (block_scales) block_scales[j] = b;
     const float den = (float)(b * sr);                   /* exact */
+    const float rcp = b == 0.0 ? 0.0f : 1.0f / den;      /* single precision */
     for (int i = 16 * j; i < 16 * j + 16; ++i) {
       if (b == 0.0) { out[i] = 0.0; continue; }
-      const float y = x[i] / den;                        /* single precision */
+      const float y = x[i] * rcp;                        /* single precision */
       out[i] = e2m1_round((double)y) * b * sr;
     }
   }

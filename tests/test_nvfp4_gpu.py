@@ -5,8 +5,8 @@ power-of-two scale per row; the GEMMs run tcgen05 kind::mxf4nvf4.
 1. The library's packed weight codes, block scales and row scales, decoded
    on the host from the two formats' definitions, equal the oracle's NVFP4
    quantisation of the same bf16 weights bit for bit (the rule leaves one
-   right answer: both divisions are IEEE single precision, both roundings
-   to nearest even).
+   right answer: the division, reciprocal and product are IEEE single
+   precision, both roundings to nearest even).
 2. The same for the activation rows the library quantises on the fly (each
    expert input row z in dispatch order, each hidden row h), taken from the
    library's own bf16 z and H: the quantiser sees the same values on both

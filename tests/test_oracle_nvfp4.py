@@ -6,8 +6,10 @@ is NVIDIA's published one: E2M1 elements, an E4M3 scale per 16 elements, a
 second-level scale (taken per row here, a power of two).  These pins hold
 the oracle to the format's definition: every E2M1 value round-trips, ties
 go to the even mantissa, block scales are the E4M3 rounding of the block
-maximum over 6 s_r, row scales the smallest powers of two that keep every
-block scale in E4M3's range, and the error stays within half a grid step.
+maximum over 6 s_r, elements are scaled by the single-precision reciprocal
+of their decoded block scale, row scales are the smallest powers of two that
+keep every block scale in E4M3's range, and the error stays within half a
+grid step.
 """
 import os
 import subprocess
@@ -81,6 +83,19 @@ def test_block_scale_is_the_e4m3_rounding_of_amax_over_6_sr():
                                                6.0 * 2.0 ** -9])
 
 
+def test_elements_are_scaled_by_the_rounded_reciprocal_of_the_block_scale():
+    """code = E2M1(x * RN(1 / (b s_r))), not E2M1(x / (b s_r)): with b = 1.875
+    (block maximum 11.25) the elements 2.34375 = 1.25 * 1.875 and 4.6875 =
+    2.5 * 1.875 divide to the ties 1.25 and 2.5 exactly (which go to the even
+    1 and 2), but 1 / 1.875 = 8/15 rounds up in single precision, so the
+    products lie just above the ties and round to 1.5 and 3."""
+    from fractions import Fraction
+    assert Fraction(float(np.float32(1) / np.float32(1.875))) > Fraction(8, 15)
+    q, s, b = oracle.nvfp4_rows(_row(ANCHOR, [11.25, 2.34375, 4.6875, -2.34375] + [0.0] * 12))
+    assert s[0] == 1.0 and b[0, 1] == 1.875
+    np.testing.assert_array_equal(q[0, 16:20], np.array([6.0, 1.5, 3.0, -1.5]) * 1.875)
+
+
 def test_row_scale_is_the_smallest_power_of_two_in_range():
     rng = np.random.default_rng(0)
     w = rng.standard_normal((64, 96)) * np.exp(rng.uniform(-12, 8, size=(64, 1)))
@@ -140,11 +155,14 @@ MUTATIONS = {
     "block_scale_not_rounded": ("    const double b = e4m3_round((double)t);", "    const double b = (double)t;"),
     "uniform_grid": ("    const double q = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);",
                      "    const double q = 0.5;"),
+    "division_instead_of_reciprocal": ("      const float y = x[i] * rcp;",
+                                       "      const float y = x[i] / den;"),
     "no_saturation": ("  if (a >= 6.0) {\n    r = 6.0;\n  } else {",
                       "  if (a >= 60.0) {\n    r = 6.0;\n  } else {"),
 }
 PINS = [test_every_e2m1_value_round_trips, test_ties_round_to_the_even_mantissa,
         test_block_scale_is_the_e4m3_rounding_of_amax_over_6_sr,
+        test_elements_are_scaled_by_the_rounded_reciprocal_of_the_block_scale,
         test_row_scale_is_the_smallest_power_of_two_in_range,
         test_values_lie_on_the_grid_and_within_half_a_step, test_zero_blocks_and_bf16_inputs]
 

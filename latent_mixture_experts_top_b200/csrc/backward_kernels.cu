@@ -10,6 +10,7 @@
 // do_k = g_k du; the expert's hidden gradient; ds_{id_k} = g_k (dg_k -
 // sum_j g_j dg_j) through the renormalised gates; dz = sum over slots of the
 // expert input gradients; dx = W_r^T ds + W_down^T dz + the shared experts'.
+#include <algorithm>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -250,38 +251,93 @@ __global__ void bias_grad_kernel(const float *__restrict__ ds, const int32_t *__
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= N) return;
   float acc = 0.0f;
-  for (int p = offsets[e]; p < offsets[e + 1]; ++p) acc += ds[perm[p]];
+  for (int p = offsets[e]; p < offsets[e + 1]; ++p)
+    if (perm[p] >= 0) acc += ds[perm[p]];  // padding rows of a padded order hold -1
   db[e] = acc;
+}
+
+// Zeroes the padding rows [ends[e], offsets[e + 1]) of expert e in up to four
+// bf16 matrices (blockIdx.y selects one; null pointers are skipped).
+__global__ void zero_pad_rows_kernel(const int32_t *__restrict__ offsets,
+                                     const int32_t *__restrict__ ends, int N, PadRowsArgs a) {
+  const int e = blockIdx.x, which = blockIdx.y;
+  if (e >= N || !a.ptr[which]) return;
+  const int r0 = ends[e], r1 = offsets[e + 1], vpr = a.cols[which] / 8;
+  uint4 *base = reinterpret_cast<uint4 *>(a.ptr[which]);
+  for (int i = threadIdx.x; i < (r1 - r0) * vpr; i += blockDim.x) {
+    const int r = r0 + i / vpr, v = i % vpr;
+    base[static_cast<size_t>(r) * vpr + v] = make_uint4(0, 0, 0, 0);
+  }
 }
 
 // bf16 mode, gate/up pre-activations as the tensor-core GEMM writes them: in
 // each 256-column block b, columns [0,128) hold the gate of hidden units
 // 128b .. 128b+127 and [128,256) the matching up (squared ReLU: column c is
-// the up of unit c).  Writes h (plain [rows][n]) and dAB (same interleaved
-// layout as AB) from dh (fp32, plain); either output may be null.
-__global__ void act_backward_tiled_kernel(const __nv_bfloat16 *__restrict__ AB, int ldab,
-                                          const float *__restrict__ dh, int lddh,
-                                          __nv_bfloat16 *__restrict__ h, int ldh,
-                                          __nv_bfloat16 *__restrict__ dAB, int lddab, int rows,
-                                          int n, int relu2) {
-  const int c = blockIdx.y * blockDim.x + threadIdx.x;  // rows on x: up to 2^31 - 1
-  const int r = blockIdx.x;
-  if (r >= rows || c >= n) return;
-  const size_t base = static_cast<size_t>(r) * ldab, dbase = static_cast<size_t>(r) * lddab;
-  const float g = dh ? dh[static_cast<size_t>(r) * lddh + c] : 0.0f;
-  if (relu2) {
-    const float rb = fmaxf(__bfloat162float(AB[base + c]), 0.0f);
-    if (h) h[static_cast<size_t>(r) * ldh + c] = __float2bfloat16_rn(rb * rb);
-    if (dAB) dAB[dbase + c] = __float2bfloat16_rn(g * 2.0f * rb);
-  } else {
-    const size_t ia = 256 * (c >> 7) + (c & 127), ib = ia + 128;
-    const float av = __bfloat162float(AB[base + ia]), bv = __bfloat162float(AB[base + ib]);
-    const float sg = 1.0f / (1.0f + expf(-av));
-    const float sl = av * sg;
-    if (h) h[static_cast<size_t>(r) * ldh + c] = __float2bfloat16_rn(sl * bv);
-    if (dAB) {
-      dAB[dbase + ia] = __float2bfloat16_rn(g * bv * sg * (1.0f + av * (1.0f - sg)));
-      dAB[dbase + ib] = __float2bfloat16_rn(g * sl);
+// the up of unit c).  dh [rows][n] (fp32 or bf16) -> dAB in the same
+// interleaved layout: SwiGLU da = dh b silu'(a), db = dh silu(a); squared
+// ReLU db = dh 2 relu(b).  Each thread takes 8 consecutive hidden units of a
+// row (16-byte loads and stores; consecutive threads, consecutive units).
+__device__ __forceinline__ void unpack_bf16x8(const uint4 q, float *v) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ uint4 pack_bf16x8(const float *v) {
+  uint4 q;
+  q.x = pack_bf16x2(v[0], v[1]);
+  q.y = pack_bf16x2(v[2], v[3]);
+  q.z = pack_bf16x2(v[4], v[5]);
+  q.w = pack_bf16x2(v[6], v[7]);
+  return q;
+}
+template <typename TD>
+__device__ __forceinline__ void load_dh8(const TD *p, float *v);
+template <>
+__device__ __forceinline__ void load_dh8<float>(const float *p, float *v) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load_dh8<__nv_bfloat16>(const __nv_bfloat16 *p, float *v) {
+  unpack_bf16x8(*reinterpret_cast<const uint4 *>(p), v);
+}
+
+template <typename TD>
+__global__ void __launch_bounds__(256) act_backward_rows_kernel(
+    const __nv_bfloat16 *__restrict__ AB, int ldab, const TD *__restrict__ dh, int lddh,
+    __nv_bfloat16 *__restrict__ dAB, int lddab, int rows, int n, int relu2) {
+  const int groups = n / 8;
+  const long long total = static_cast<long long>(rows) * groups;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / groups;
+    const int c = static_cast<int>(i - r * groups) * 8;
+    float g[8];
+    load_dh8<TD>(dh + r * lddh + c, g);
+    const __nv_bfloat16 *ab = AB + r * ldab;
+    __nv_bfloat16 *dab = dAB + r * lddab;
+    if (relu2) {
+      float b[8], db[8];
+      unpack_bf16x8(*reinterpret_cast<const uint4 *>(ab + c), b);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) db[j] = g[j] * 2.0f * fmaxf(b[j], 0.0f);
+      *reinterpret_cast<uint4 *>(dab + c) = pack_bf16x8(db);
+    } else {
+      const int ia = 256 * (c >> 7) + (c & 127), ib = ia + 128;
+      float a[8], b[8], da[8], db[8];
+      unpack_bf16x8(*reinterpret_cast<const uint4 *>(ab + ia), a);
+      unpack_bf16x8(*reinterpret_cast<const uint4 *>(ab + ib), b);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float sg = 1.0f / (1.0f + __expf(-a[j]));
+        da[j] = g[j] * b[j] * sg * (1.0f + a[j] * (1.0f - sg));
+        db[j] = g[j] * a[j] * sg;
+      }
+      *reinterpret_cast<uint4 *>(dab + ia) = pack_bf16x8(da);
+      *reinterpret_cast<uint4 *>(dab + ib) = pack_bf16x8(db);
     }
   }
 }
@@ -313,112 +369,27 @@ __global__ void transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ src, int
   }
 }
 
-// Token-major transpose for the weight-gradient GEMMs: dst[c][kstart[e] + j]
-// = src[offsets[e] + j][c] for the j < rows_e rows of expert e, and 0 for
-// rows_e <= j < klen[e] (the padding each expert's K range runs over).
-// Dense form (kstart == null): one block of T rows, zero-padded to a
-// multiple of 64.  One CTA per 64 tokens x 64 columns, 16-byte global loads
-// and stores on both sides.  C, lds, ldd multiples of 8.
-__global__ void __launch_bounds__(256) transpose_tokens_kernel(
-    const __nv_bfloat16 *__restrict__ src, int lds, int C, const int32_t *__restrict__ offsets,
-    const int32_t *__restrict__ kstart, int N, int T_dense, __nv_bfloat16 *__restrict__ dst,
-    long long ldd) {
-  __shared__ uint32_t tile[64][33];  // 64 tokens x 64 bf16 (33-word rows)
-  const int k0 = blockIdx.x * 64, c0 = blockIdx.y * 64;
-  int row0, rows;
-  if (kstart) {
-    if (k0 >= kstart[N]) return;
-    int lo = 0, hi = N;  // expert e with kstart[e] <= k0 < kstart[e+1]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (kstart[mid] <= k0) lo = mid; else hi = mid;
-    }
-    row0 = offsets[lo] + (k0 - kstart[lo]);
-    rows = offsets[lo + 1] - row0;
-  } else {
-    row0 = k0;
-    rows = T_dense - k0;
-  }
-  for (int v = threadIdx.x; v < 512; v += 256) {  // 64 tokens x 8 vectors of 8 columns
-    const int rr = v >> 3, cv = (v & 7) * 8;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (rr < rows && c0 + cv < C)
-      val = *reinterpret_cast<const uint4 *>(src + static_cast<size_t>(row0 + rr) * lds + c0 + cv);
-    uint32_t *t = &tile[rr][cv >> 1];
-    t[0] = val.x; t[1] = val.y; t[2] = val.z; t[3] = val.w;
-  }
-  __syncthreads();
-  const unsigned short *t16 = reinterpret_cast<const unsigned short *>(&tile[0][0]);
-  for (int v = threadIdx.x; v < 512; v += 256) {  // 64 columns x 8 vectors of 8 tokens
-    const int cc = v >> 3, kv = (v & 7) * 8;
-    if (c0 + cc >= C) continue;
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t lo16 = t16[(kv + 2 * i) * 66 + cc];
-      const uint32_t hi16 = t16[(kv + 2 * i + 1) * 66 + cc];
-      w[i] = lo16 | (hi16 << 16);
-    }
-    *reinterpret_cast<uint4 *>(dst + static_cast<long long>(c0 + cc) * ldd + k0 + kv) =
-        make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
-// Zeros the padding columns of a token-major transposed operand: for every
-// row c < n_rows and expert e, columns [kstart[e] + rows_e, kstart[e] +
-// klen[e]) (rows_e = offsets[e+1] - offsets[e]).
-__global__ void zero_pad_cols_kernel(__nv_bfloat16 *__restrict__ dst, long long ldd, int n_rows,
-                                     const int32_t *__restrict__ offsets,
-                                     const int32_t *__restrict__ kstart,
-                                     const int32_t *__restrict__ klen) {
-  const int e = blockIdx.x;
-  const int rows = offsets[e + 1] - offsets[e];
-  const int pad = klen[e] - rows;
-  if (pad <= 0) return;
-  const long long k0 = kstart[e] + rows;
-  for (int i = threadIdx.x; i < n_rows * pad; i += blockDim.x) {
-    const int c = i / pad, k = i % pad;
-    dst[c * ldd + k0 + k] = __float2bfloat16_rn(0.0f);
-  }
-}
-
-// Per-expert K ranges of the token-major transposed operands: klen[e] =
-// rows of e rounded up to 64, kstart = exclusive scan of klen (kstart[N] =
-// total), shift[e] = kstart[e] - offsets[e].  One block, N <= 1024.
-__global__ void padded_offsets_kernel(const int32_t *__restrict__ offsets, int N,
-                                      int32_t *__restrict__ kstart, int32_t *__restrict__ klen,
-                                      int32_t *__restrict__ shift) {
-  __shared__ int buf[1024];
-  const int e = threadIdx.x;
-  const int len = e < N ? ((offsets[e + 1] - offsets[e] + 63) & ~63) : 0;
-  buf[e] = len;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = e >= off ? buf[e - off] : 0;
-    __syncthreads();
-    buf[e] += v;
-    __syncthreads();
-  }
-  if (e < N) {
-    const int start = buf[e] - len;
-    kstart[e] = start;
-    klen[e] = len;
-    shift[e] = start - offsets[e];
-  }
-  if (e == N - 1) kstart[N] = buf[e];
-}
-
 }  // namespace
 
-cudaError_t launch_act_backward_tiled(const __nv_bfloat16 *AB, int ldab, const float *dh,
-                                      int lddh, __nv_bfloat16 *h, int ldh, __nv_bfloat16 *dAB,
-                                      int lddab, int rows, int n, bool relu2, cudaStream_t s) {
+template <typename TD>
+cudaError_t launch_act_backward_rows(const __nv_bfloat16 *AB, int ldab, const TD *dh, int lddh,
+                                     __nv_bfloat16 *dAB, int lddab, int rows, int n, bool relu2,
+                                     cudaStream_t s) {
   if (rows <= 0 || n <= 0) return cudaSuccess;
-  dim3 grid(rows, (n + 255) / 256);
-  act_backward_tiled_kernel<<<grid, 256, 0, s>>>(AB, ldab, dh, lddh, h, ldh, dAB, lddab, rows, n,
-                                                 relu2 ? 1 : 0);
+  if (n % 8 || ldab % 8 || lddh % 8 || lddab % 8) return cudaErrorInvalidValue;
+  const long long total = static_cast<long long>(rows) * (n / 8);
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148LL * 16));
+  act_backward_rows_kernel<TD><<<blocks, 256, 0, s>>>(AB, ldab, dh, lddh, dAB, lddab, rows, n,
+                                                      relu2 ? 1 : 0);
   return cudaGetLastError();
 }
+template cudaError_t launch_act_backward_rows<float>(const __nv_bfloat16 *, int, const float *,
+                                                     int, __nv_bfloat16 *, int, int, int, bool,
+                                                     cudaStream_t);
+template cudaError_t launch_act_backward_rows<__nv_bfloat16>(const __nv_bfloat16 *, int,
+                                                             const __nv_bfloat16 *, int,
+                                                             __nv_bfloat16 *, int, int, int, bool,
+                                                             cudaStream_t);
 
 cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int lds, int R, int C,
                                   const int32_t *row_expert, const int32_t *shift,
@@ -428,21 +399,6 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int lds, int R, int 
   dim3 grid((C + 31) / 32, (R + 31) / 32, batch);
   transpose_bf16_kernel<<<grid, 256, 0, s>>>(src, lds, R, C, row_expert, shift, dst, ldd,
                                              src_batch, dst_batch);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_zero_pad_cols(__nv_bfloat16 *dst, long long ldd, int n_rows,
-                                 const int32_t *offsets, const int32_t *kstart,
-                                 const int32_t *klen, int N, cudaStream_t s) {
-  if (N <= 0 || n_rows <= 0) return cudaSuccess;
-  zero_pad_cols_kernel<<<N, 256, 0, s>>>(dst, ldd, n_rows, offsets, kstart, klen);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_padded_offsets(const int32_t *offsets, int N, int32_t *kstart, int32_t *klen,
-                                  int32_t *shift, cudaStream_t s) {
-  if (N <= 0 || N > 1024) return cudaErrorInvalidValue;
-  padded_offsets_kernel<<<1, 1024, 0, s>>>(offsets, N, kstart, klen, shift);
   return cudaGetLastError();
 }
 
@@ -492,16 +448,6 @@ cudaError_t launch_slot_grad(const float *du, int lddu, const TO *O, int l, cons
   return cudaGetLastError();
 }
 
-cudaError_t launch_transpose_tokens(const __nv_bfloat16 *src, int lds, int C,
-                                    const int32_t *offsets, const int32_t *kstart, int N,
-                                    int64_t k_cols, int T_dense, __nv_bfloat16 *dst, long long ldd,
-                                    cudaStream_t s) {
-  if (C <= 0 || k_cols <= 0) return cudaSuccess;
-  if (C % 8 || lds % 8 || ldd % 8) return cudaErrorInvalidValue;
-  dim3 grid(static_cast<unsigned>((k_cols + 63) / 64), (C + 63) / 64);
-  transpose_tokens_kernel<<<grid, 256, 0, s>>>(src, lds, C, offsets, kstart, N, T_dense, dst, ldd);
-  return cudaGetLastError();
-}
 template cudaError_t launch_slot_grad<float>(const float *, int, const float *, int,
                                              const int32_t *, const float *, int, int, float *,
                                              float *, cudaStream_t);
@@ -539,6 +485,15 @@ cudaError_t launch_bias_grad(const float *ds, const int32_t *offsets, const int3
                              float *db, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   bias_grad_kernel<<<(N + 127) / 128, 128, 0, s>>>(ds, offsets, perm, N, db);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_pad_rows(const int32_t *offsets, const int32_t *ends, int N,
+                                 const PadRowsArgs &a, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  for (int i = 0; i < 4; ++i)
+    if (a.ptr[i] && a.cols[i] % 8) return cudaErrorInvalidValue;
+  zero_pad_rows_kernel<<<dim3(N, 4), 256, 0, s>>>(offsets, ends, N, a);
   return cudaGetLastError();
 }
 

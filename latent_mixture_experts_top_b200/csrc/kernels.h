@@ -13,6 +13,15 @@ struct TileEntry {
   int32_t row0, row_end, expert, pad;
 };
 
+// Segment padding of the dispatch order: pad > 1 starts each expert's rows at
+// a multiple of pad (offsets are the padded starts, offsets[N] the padded
+// total, ends[e] the end of expert e's real rows); pad == 1: no padding.
+struct SegPad {
+  int pad;
+  int32_t *ends;
+};
+constexpr SegPad kNoPad = {1, nullptr};
+
 // ---- routing (route_kernels.cu)
 // ids/gates from fp32 logits [T][ld] (+ bias [N]); one warp per token.  If
 // counts is non-null the
@@ -45,7 +54,8 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
                             int32_t *pos, int32_t *row_expert, TileEntry *tiles,
                             int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s,
                             TileEntry *tiles2 = nullptr, int32_t *n_tiles2 = nullptr,
-                            int tile_m2 = 0, int max_tiles2 = 0, bool check_ids = false);
+                            int tile_m2 = 0, int max_tiles2 = 0, bool check_ids = false,
+                            SegPad seg = kNoPad);
 
 // Expert parallelism, receiving side.  recv_counts [W][NL]: rows that source
 // rank s sent for local expert e; the received rows lie source-major and,
@@ -77,7 +87,7 @@ cudaError_t launch_route_select(const float *logits, int ld, const float *bias, 
                                 int32_t *arrivals, int32_t *offsets, TileEntry *tiles,
                                 int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
                                 int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s,
-                                bool pdl = false);
+                                bool pdl = false, SegPad seg = kNoPad);
 cudaError_t launch_scatter_permute(const int32_t *ids, int T, int K, int N, const int32_t *counts,
                                    int chunk, const int32_t *offsets, int32_t *perm, int32_t *pos,
                                    int32_t *row_expert, const void *src, int row_bytes, void *dst,
@@ -154,10 +164,6 @@ struct TcParams {
   __nv_bfloat16 *out2; int ld_out2;  // TC_X_FUSED shared region, with raw
   float *out_f32;      // TC_OUT / TC_EXPERT_DOWN: fp32 output [rows][ld_out]
   __nv_bfloat16 *out_h; int ld_h;  // TC_EXPERT_GU with raw: the hidden h as well
-  // TC_EXPERT_DOWN computing dH = DO W_o[e]: instead of storing dH, the
-  // epilogue applies the activation backward with the pre-activations
-  // act_ab [rows][ld_ab] (gate/up layout of the GU GEMM) and writes act_dab.
-  const __nv_bfloat16 *act_ab; __nv_bfloat16 *act_dab; int ld_ab;
   // E4M3 operands (TC_EXPERT_GU / TC_EXPERT_DOWN with b_scale set): A is
   // E4M3 [rows][Kdim] with one scale per row in a_scale, B is the E4M3 weight
   // tiled in 256-row x 128-byte blocks (launch_quantize_e4m3_tiles) and
@@ -173,10 +179,12 @@ struct TcParams {
   // TMEM (see launch_quantize_nvfp4_tiles); the MMA is kind::mxf4nvf4 over
   // 256-element K-blocks.
   const uint8_t *a_sf, *b_sf;
-  // TC_WGRAD: A [M][*] and B [*][*] are plain row-major token-major matrices
-  // (K runs along their rows' contiguous axis); group g reduces over
-  // K-columns [k_start[g], k_start[g] + k_len[g]) (multiples of 64; dense:
-  // k_start == null and K = Kdim); n_tiles_n counts 256-row tiles of B.
+  // TC_WGRAD: dW = A^T B with A [tokens][M] and B [tokens][N] the token-major
+  // (row-major, tokens on rows) matrices themselves, read MN-major through
+  // {64, 64} boxes; group g reduces over token rows [k_start[g], k_start[g] +
+  // k_len[g]) (multiples of 64; k_len null: up to k_start[g + 1]; dense:
+  // k_start null and rows [0, Kdim), rows past the maps' end read as zero);
+  // n_tiles_n counts 256-column tiles of B.
   int wg_kind, groups;
   const int32_t *k_start, *k_len;
   int wg_d, wg_l, wg_m, wg_ns, wg_ms, wg_n, wg_npad, wg_lpad;  // layer sizes for the destinations
@@ -306,11 +314,24 @@ cudaError_t launch_scatter_ds(const float *ds, const int32_t *ids, int T, int K,
 cudaError_t launch_bias_grad(const float *ds, const int32_t *offsets, const int32_t *perm, int N,
                              float *db, cudaStream_t s);
 
-// bf16: gate/up pre-activations AB in the GEMM's 128-interleaved layout
-// (squared ReLU: plain up) -> h (plain) and dAB (interleaved); see the kernel.
-cudaError_t launch_act_backward_tiled(const __nv_bfloat16 *AB, int ldab, const float *dh,
-                                      int lddh, __nv_bfloat16 *h, int ldh, __nv_bfloat16 *dAB,
-                                      int lddab, int rows, int n, bool relu2, cudaStream_t s);
+// Zeroes the padding rows [ends[e], offsets[e + 1]) of every expert (a padded
+// dispatch order, see SegPad) in up to four bf16 row-major matrices ptr[i]
+// with cols[i] columns (a multiple of 8); null entries are skipped.
+struct PadRowsArgs {
+  void *ptr[4];
+  int cols[4];
+};
+cudaError_t launch_zero_pad_rows(const int32_t *offsets, const int32_t *ends, int N,
+                                 const PadRowsArgs &a, cudaStream_t s);
+
+// bf16: gate/up pre-activations AB [rows][ldab] in the GEMM's 128-interleaved
+// layout (squared ReLU: plain up) and the hidden gradient dh [rows][lddh]
+// (TD = float or bf16) -> dAB [rows][lddab] in the same layout; n hidden
+// units per row (n, ldab, lddh, lddab multiples of 8).
+template <typename TD>
+cudaError_t launch_act_backward_rows(const __nv_bfloat16 *AB, int ldab, const TD *dh, int lddh,
+                                     __nv_bfloat16 *dAB, int lddab, int rows, int n, bool relu2,
+                                     cudaStream_t s);
 // dst[c][col(r)] = src[r][c]; col(r) = r, or r + shift[row_expert[r]];
 // `batch` independent matrices, src / dst advanced by src_batch / dst_batch.
 cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int lds, int R, int C,
@@ -318,23 +339,6 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int lds, int R, int 
                                   __nv_bfloat16 *dst, long long ldd, cudaStream_t s,
                                   int batch = 1, long long src_batch = 0,
                                   long long dst_batch = 0);
-// Token-major transpose for the weight gradients: dst[c][kstart[e] + j] =
-// src[offsets[e] + j][c] (zeros up to klen[e]); dense (kstart null): T_dense
-// rows, zero-padded to a multiple of 64.  k_cols: the destination columns to
-// cover (grouped: the workspace width; dense: round64(T)).
-cudaError_t launch_transpose_tokens(const __nv_bfloat16 *src, int lds, int C,
-                                    const int32_t *offsets, const int32_t *kstart, int N,
-                                    int64_t k_cols, int T_dense, __nv_bfloat16 *dst, long long ldd,
-                                    cudaStream_t s);
-// Zeros dst[c][kstart[e] + rows_e .. kstart[e] + klen[e]) for c < n_rows.
-cudaError_t launch_zero_pad_cols(__nv_bfloat16 *dst, long long ldd, int n_rows,
-                                 const int32_t *offsets, const int32_t *kstart,
-                                 const int32_t *klen, int N, cudaStream_t s);
-// klen[e] = round64(rows of e), kstart = its exclusive scan (kstart[N] =
-// total), shift[e] = kstart[e] - offsets[e].  N <= 1024.
-cudaError_t launch_padded_offsets(const int32_t *offsets, int N, int32_t *kstart, int32_t *klen,
-                                  int32_t *shift, cudaStream_t s);
-
 // Failure-detection self-test (see lmoe_selftest_wait_timeout).
 cudaError_t launch_wait_selftest(int32_t *status, long long limit_ns, cudaStream_t s);
 

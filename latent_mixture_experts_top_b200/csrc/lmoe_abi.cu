@@ -44,6 +44,7 @@ struct Workspace {
   void *x_stage = nullptr, *y_stage = nullptr;
   int32_t *status = nullptr;
   int32_t *arrivals = nullptr;  // fused routing: the last-block counter (zero between launches)
+  int32_t *seg_end = nullptr;   // training: the end of each expert's rows in the padded order
   // E4M3 / NVFP4 routed experts: the expert GEMMs' A operands with row scales
   uint8_t *zq = nullptr, *hq = nullptr;  // [TK][l], [TK][m] (NVFP4: packed, half the bytes)
   float *zq_scale = nullptr, *hq_scale = nullptr;  // [TK]
@@ -59,7 +60,7 @@ struct BwdWorkspace {
   float *dU = nullptr;                  // [T][ky] dy . [W_up | S_o]
   float *ds = nullptr;                  // [TK] router-logit gradient per slot
   void *DO = nullptr;                   // [TK][l] expert-output gradient (permuted)
-  float *dH = nullptr;                  // [TK][m]
+  float *dH = nullptr;  // fp32 [TK][m]; bf16 mode: the hidden gradient, bf16 [Kp][m]
   void *dA = nullptr, *dB = nullptr;    // [TK][m]
   float *dZp = nullptr;                 // [TK][l]
   float *dz = nullptr;                  // [T][l]
@@ -71,10 +72,9 @@ struct BwdWorkspace {
   void *ABs = nullptr;     // [T][sh_rows]  shared gate/up pre-activations (W_x layout)
   void *dAB = nullptr;     // [TK][gu_rows]
   void *dXcat = nullptr;   // [T][nx_rows] = [dS (router) | dz | shared dAB], W_x columns
-  void *DOT = nullptr, *HT = nullptr, *dABT = nullptr, *zpT = nullptr;  // [*][Kp] token-major
-  void *dyT = nullptr, *ucatT = nullptr, *dXcatT = nullptr, *xT = nullptr;  // [*][Tp]
-  int32_t *kstart = nullptr, *klen = nullptr, *shift = nullptr;  // [N'+1]
-  int64_t Kp = 0, Tp = 0;
+  // Rows of the per-pair buffers in the backward's padded dispatch order
+  // (each expert's rows start at a multiple of 64; see backward_bf16).
+  int64_t Kp = 0;
 };
 
 }  // namespace
@@ -145,7 +145,10 @@ struct lmoe_layer {
   void *w_guT = nullptr;  // [N][l][gu_rows]
   void *w_xT = nullptr;   // [d][nx_rows]
   TensorMap64 tm_wyT, tm_woT, tm_wguT, tm_wxT, tm_DO, tm_dAB, tm_dXcat;
-  TensorMap64 tm_DOT, tm_HT, tm_dABT, tm_zpT, tm_dyT, tm_ucatT, tm_dXcatT, tm_xT;
+  // weight-gradient operands read MN-major ({64, 64} boxes of the token-major
+  // matrices in the padded order)
+  TensorMap64 tm_DOmn, tm_Hmn, tm_dABmn, tm_zpmn;
+  TensorMap64 tm_dH_out;  // the hidden gradient's store map (bf16 in the dH buffer)
 };
 
 namespace {
@@ -180,9 +183,8 @@ void free_all(lmoe_layer *h) {
                   h->ws.x_stage, h->ws.y_stage, h->ws.status, h->bw.a, h->bw.b, h->bw.dU,
                   h->bw.ds, h->bw.DO, h->bw.dH, h->bw.dA, h->bw.dB, h->bw.dZp, h->bw.dz,
                   h->bw.as, h->bw.bs, h->bw.das, h->bw.dbs, h->bw.dsfull, h->bw.AB,
-                  h->bw.ABs, h->bw.dAB, h->bw.dXcat, h->bw.DOT, h->bw.HT, h->bw.dABT,
-                  h->bw.zpT, h->bw.dyT, h->bw.ucatT, h->bw.dXcatT, h->bw.xT, h->bw.kstart,
-                  h->bw.klen, h->bw.shift, h->w_yT, h->w_oT, h->w_guT, h->w_xT, h->w_gu8,
+                  h->bw.ABs, h->bw.dAB, h->bw.dXcat, h->ws.seg_end,
+                  h->w_yT, h->w_oT, h->w_guT, h->w_xT, h->w_gu8,
                   h->w_o8, h->gu_scale, h->o_scale, h->gu_sf, h->o_sf, h->ws.zq_sf, h->ws.hq_sf,
                   h->ws.ep_tiles, h->ws.ep_tiles2,
                   h->ws.ep_n_tiles, h->ws.ep_n_tiles2, h->ws.arrivals, h->ws.zq, h->ws.hq,
@@ -313,6 +315,12 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   }
   const size_t T = h->Tmax, TK = static_cast<size_t>(h->Tmax) * h->K, es = h->esize;
   const size_t N = h->N, d = h->d, l = h->l, m = h->m;
+  // bf16 training handles: the per-pair buffers hold the backward's padded
+  // dispatch order (each expert's rows start at a multiple of 64)
+  const bool padded = cfg->training != 0 && h->bf16;
+  h->bw.Kp = padded ? static_cast<int64_t>((TK + 63) / 64 * 64 + 64 * N) : 0;
+  const size_t TKr = padded ? static_cast<size_t>(h->bw.Kp) : TK;
+  if (padded) h->h_rows = std::max(h->h_rows, static_cast<int64_t>(TKr));
   h->max_tiles = static_cast<int>(TK / kTileM + N + 1);
   h->max_tiles2 = static_cast<int>(TK / (2 * kTileM) + N + 1);
   h->n_pad = (h->N + kTileN - 1) / kTileN * kTileN;
@@ -329,13 +337,13 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   Workspace &w = h->ws;
   bool ok = dalloc(&w.logits, T * N * 4) && dalloc(&w.ids, TK * 4) && dalloc(&w.gates, TK * 4) &&
             dalloc(&w.chunk_counts, dispatch_count_elems(h->Tmax, h->route_chunk, h->N) * 4) &&
-            dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TK * 4) && dalloc(&w.pos, TK * 4) &&
-            dalloc(&w.row_expert, TK * 4) &&
+            dalloc(&w.offsets, (N + 1) * 4) && dalloc(&w.perm, TKr * 4) &&
+            dalloc(&w.pos, TK * 4) && dalloc(&w.row_expert, TKr * 4) &&
             dalloc(&w.tiles, static_cast<size_t>(h->max_tiles) * sizeof(TileEntry)) &&
             dalloc(&w.n_tiles, 16) &&
             dalloc(&w.tiles2, static_cast<size_t>(h->max_tiles2) * sizeof(TileEntry)) &&
-            dalloc(&w.n_tiles2, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TK * l * es) &&
-            dalloc(&w.H, static_cast<size_t>(h->h_rows) * m * es) && dalloc(&w.O, TK * l * es) &&
+            dalloc(&w.n_tiles2, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TKr * l * es) &&
+            dalloc(&w.H, static_cast<size_t>(h->h_rows) * m * es) && dalloc(&w.O, TKr * l * es) &&
             dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
             dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16) && dalloc(&w.arrivals, 16);
   if (ok) {  // weights
@@ -385,24 +393,16 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     BwdWorkspace &b = h->bw;
     const size_t nsms = static_cast<size_t>(h->ns) * h->ms;
     ok = dalloc(&b.a, TK * m * es) && dalloc(&b.b, TK * m * es) &&
-         dalloc(&b.dU, T * h->ky * 4) && dalloc(&b.ds, TK * 4) && dalloc(&b.DO, TK * l * es) &&
-         dalloc(&b.dH, TK * m * 4) && dalloc(&b.dA, TK * m * es) && dalloc(&b.dB, TK * m * es) &&
-         dalloc(&b.dZp, TK * l * 4) && dalloc(&b.dz, T * l * 4) && dalloc(&b.as, T * nsms * es) &&
+         dalloc(&b.dU, T * h->ky * 4) && dalloc(&b.ds, TK * 4) && dalloc(&b.DO, TKr * l * es) &&
+         dalloc(&b.dH, std::max(TK * m * 4, TKr * m * 2)) && dalloc(&b.dA, TK * m * es) && dalloc(&b.dB, TK * m * es) &&
+         dalloc(&b.dZp, TKr * l * 4) && dalloc(&b.dz, T * l * 4) && dalloc(&b.as, T * nsms * es) &&
          dalloc(&b.bs, T * nsms * es) && dalloc(&b.das, T * nsms * es) &&
          dalloc(&b.dbs, T * nsms * es) && dalloc(&b.dsfull, T * N * 4);
     if (ok && h->bf16) {
-      const size_t gu = h->gu_rows, nx = h->nx_rows, ky = h->ky;
-      b.Kp = static_cast<int64_t>((TK + 63) / 64 * 64 + 64 * N);
-      b.Tp = static_cast<int64_t>((T + 63) / 64 * 64);
-      const size_t Kp = b.Kp, Tp = b.Tp;
-      ok = dalloc(&b.AB, TK * gu * 2) && dalloc(&b.ABs, T * h->sh_rows * 2) &&
-           dalloc(&b.dAB, TK * gu * 2) && dalloc(&b.dXcat, T * nx * 2) &&
-           dalloc(&b.DOT, l * Kp * 2) && dalloc(&b.HT, m * Kp * 2) &&
-           dalloc(&b.dABT, gu * Kp * 2) && dalloc(&b.zpT, l * Kp * 2) &&
-           dalloc(&b.dyT, d * Tp * 2) && dalloc(&b.ucatT, ky * Tp * 2) &&
-           dalloc(&b.dXcatT, nx * Tp * 2) && dalloc(&b.xT, d * Tp * 2) &&
-           dalloc(&b.kstart, (N + 1) * 4) && dalloc(&b.klen, (N + 1) * 4) &&
-           dalloc(&b.shift, (N + 1) * 4) &&
+      const size_t gu = h->gu_rows, nx = h->nx_rows;
+      ok = dalloc(&b.AB, TKr * gu * 2) && dalloc(&b.ABs, T * h->sh_rows * 2) &&
+           dalloc(&b.dAB, TKr * gu * 2) && dalloc(&b.dXcat, T * nx * 2) &&
+           dalloc(&w.seg_end, N * 4) &&
            dalloc(&h->w_yT, btile_rows(1, h->ky, h->d) * 64 * 2) &&
            dalloc(&h->w_oT, btile_rows(h->N, h->m, h->l) * 64 * 2) &&
            dalloc(&h->w_guT, btile_rows(h->N, h->l, h->gu_rows) * 64 * 2) &&
@@ -424,13 +424,13 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
     return LMOE_ERR_CUDA;
   }
   if (h->bf16) {
-    rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TK), h->l, h->l, kTileM);
+    rc = make_map(&h->tm_zp, w.zp, static_cast<int64_t>(TKr), h->l, h->l, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_h, w.H, h->h_rows, h->m, h->m, kTileM);
     if (rc == LMOE_OK) rc = make_map(&h->tm_ucat, w.ucat, h->Tmax, h->ky, h->ky, kTileM);
     if (rc == LMOE_OK &&
         (make_tmap_bf16_out(h->tm_out_z.bytes, w.z, h->Tmax, h->l, h->l) != 0 ||
          make_tmap_bf16_out(h->tm_out_h.bytes, w.H, h->h_rows, h->m, h->m) != 0 ||
-         make_tmap_bf16_out(h->tm_out_o.bytes, w.O, static_cast<int64_t>(TK), h->l, h->l) != 0))
+         make_tmap_bf16_out(h->tm_out_o.bytes, w.O, static_cast<int64_t>(TKr), h->l, h->l) != 0))
       rc = LMOE_ERR_CUDA;
     // B operands: [tiled rows][64], one {64, 256} box per K-block tile
     if (rc == LMOE_OK)
@@ -469,11 +469,11 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
       rc = make_map(&h->tm_wy2, h->w_y, btile_rows(1, h->d, h->ky), 64, 64, kTileN / 2);
     if (rc == LMOE_OK && h->training) {
       BwdWorkspace &b = h->bw;
-      const int64_t Kp = b.Kp, Tp = b.Tp;
+      const int64_t rows = static_cast<int64_t>(TKr);
       const int gu = h->gu_rows, nx = h->nx_rows;
       // A operands of the K-major backward GEMMs ({64, 128} boxes)
-      rc = make_map(&h->tm_DO, b.DO, static_cast<int64_t>(TK), h->l, h->l, kTileM);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_dAB, b.dAB, static_cast<int64_t>(TK), gu, gu, kTileM);
+      rc = make_map(&h->tm_DO, b.DO, rows, h->l, h->l, kTileM);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_dAB, b.dAB, rows, gu, gu, kTileM);
       if (rc == LMOE_OK) rc = make_map(&h->tm_dXcat, b.dXcat, h->Tmax, nx, nx, kTileM);
       // transposed weights, K-block tiled ({64, 256} boxes)
       if (rc == LMOE_OK) rc = make_map(&h->tm_wyT, h->w_yT, btile_rows(1, h->ky, h->d), 64, 64, kTileN);
@@ -481,15 +481,17 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
       if (rc == LMOE_OK)
         rc = make_map(&h->tm_wguT, h->w_guT, btile_rows(h->N, h->l, gu), 64, 64, kTileN);
       if (rc == LMOE_OK) rc = make_map(&h->tm_wxT, h->w_xT, btile_rows(1, h->d, nx), 64, 64, kTileN);
-      // weight-gradient operands: token-major, A {64, 128}, B {64, 256}
-      if (rc == LMOE_OK) rc = make_map(&h->tm_DOT, b.DOT, h->l, Kp, Kp, kTileM);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_HT, b.HT, h->m, Kp, Kp, kTileN);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_dABT, b.dABT, gu, Kp, Kp, kTileM);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_zpT, b.zpT, h->l, Kp, Kp, kTileN);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_dyT, b.dyT, h->d, Tp, Tp, kTileM);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_ucatT, b.ucatT, h->ky, Tp, Tp, kTileN);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_dXcatT, b.dXcatT, nx, Tp, Tp, kTileM);
-      if (rc == LMOE_OK) rc = make_map(&h->tm_xT, b.xT, h->d, Tp, Tp, kTileN);
+      // expert weight-gradient operands, read MN-major: {64, 64} boxes of the
+      // token-major matrices (the dense ones' maps are made per call, with
+      // exactly T rows)
+      if (rc == LMOE_OK) rc = make_map(&h->tm_DOmn, b.DO, rows, h->l, h->l, 64);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_Hmn, w.H, rows, h->m, h->m, 64);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_dABmn, b.dAB, rows, gu, gu, 64);
+      if (rc == LMOE_OK) rc = make_map(&h->tm_zpmn, w.zp, rows, h->l, h->l, 64);
+      // bf16 mode keeps the hidden gradient dH in bf16 [rows][m] inside the
+      // (fp32-sized) dH buffer
+      if (rc == LMOE_OK && make_tmap_bf16_out(h->tm_dH_out.bytes, b.dH, rows, h->m, h->m) != 0)
+        rc = LMOE_ERR_CUDA;
     }
     if (rc == LMOE_OK &&
         (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
@@ -686,9 +688,13 @@ static int check_call(lmoe_handle h, int32_t T) {
 // permute_dst: also write the z rows in dispatch order there (full only).
 static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cudaStream_t s,
                              void *shared_raw = nullptr, bool marks = true,
-                             void *permute_dst = nullptr) {
+                             void *permute_dst = nullptr, SegPad seg = kNoPad) {
   Workspace &w = h->ws;
   cudaError_t e = cudaSuccess;
+  if (seg.pad > 1) {  // padded order: its padding rows keep perm = -1
+    e = cudaMemsetAsync(w.perm, 0xFF, static_cast<size_t>(h->bw.Kp) * 4, s);
+    if (e != cudaSuccess) return e;
+  }
   if (h->bf16) {
     TensorMap64 tm_x;
     if (make_map(&tm_x, x, T, h->d, h->d, kTileM) != LMOE_OK) return cudaErrorInvalidValue;
@@ -778,7 +784,7 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     e = launch_route_select(w.logits, h->N, h->b_router, T, h->N, h->K, w.ids, w.gates,
                             w.chunk_counts, kFusedChunk, w.arrivals, w.offsets, w.tiles,
                             w.n_tiles, kTileM, h->max_tiles, w.tiles2, w.n_tiles2, 2 * kTileM,
-                            h->max_tiles2, s, true);
+                            h->max_tiles2, s, true, seg);
     h->launches += 1;
     if (e != cudaSuccess) return e;
     if (full && marks) mark(h, 2, s);
@@ -803,7 +809,7 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
   if (full && marks) mark(h, 2, s);
   e = launch_dispatch(w.ids, T, h->K, h->N, w.chunk_counts, kDispatchChunk, true, w.offsets,
                       w.perm, w.pos, w.row_expert, w.tiles, w.n_tiles, kTileM, h->max_tiles, s,
-                      w.tiles2, w.n_tiles2, 2 * kTileM, h->max_tiles2);
+                      w.tiles2, w.n_tiles2, 2 * kTileM, h->max_tiles2, false, seg);
   h->launches += 2;
   if (e != cudaSuccess) return e;
   if (full && marks) mark(h, 3, s);
@@ -1226,10 +1232,9 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
   Workspace &w = h->ws;
   BwdWorkspace &b = h->bw;
   const int d = h->d, l = h->l, m = h->m, N = h->N, K = h->K, ky = h->ky;
-  const int nx = h->nx_rows, gu = h->gu_rows, TK = T * K;
+  const int nx = h->nx_rows, gu = h->gu_rows;
   const int n_pad = h->n_pad, l_pad = h->l_pad;
   const bool relu2 = h->relu2 != 0;
-  const int64_t Tp = (T + 63) / 64 * 64, Kp = b.Kp;
   bf *ucat = static_cast<bf *>(w.ucat), *dXcat = static_cast<bf *>(b.dXcat);
   int64_t &L = h->launches;
   auto gemm = [&](const TensorMap64 &ta, const TensorMap64 &tb, const TcParams &p, int tiles) {
@@ -1242,10 +1247,14 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
       make_map(&tm_dy, dy, T, d, d, kTileM) != LMOE_OK)
     return cudaErrorInvalidValue;
   const int m_tiles_T = (T + kTileM - 1) / kTileM;
-  // ---- forward activations
-  LMOE_TRY(run_route(h, x, T, true, s, b.ABs));
+  // ---- forward activations, in the padded dispatch order: each expert's rows
+  // start at a multiple of 64 (so that the weight gradients can read each
+  // expert's rows of the token-major matrices as whole 64-row K-blocks), the
+  // padding rows of zp are zeros
+  const SegPad seg = {64, w.seg_end};
+  LMOE_TRY(run_route(h, x, T, true, s, b.ABs, true, nullptr, seg));
   ++L;
-  LMOE_TRY(launch_permute_rows(w.z, w.perm, K, TK, l * 2, w.zp, s));
+  LMOE_TRY(launch_permute_rows(w.z, w.perm, K, static_cast<int>(b.Kp), l * 2, w.zp, s));
   {
     TcParams p = {};  // expert gate/up pre-activations AB
     p.mode = TC_EXPERT_GU; p.Kdim = l; p.n_tiles_n = (gu + kTileN - 1) / kTileN; p.raw = 1;
@@ -1273,25 +1282,34 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
     p.out_f32 = b.dU; p.ld_out = ky; p.status = w.status;
     LMOE_TRY(gemm(tm_dy, h->tm_wyT, p, m_tiles_T * p.n_tiles_n));
   }
-  // shared experts: hidden (for dS_o) into ucat's shared columns, pre-activation
-  // gradients into dXcat's shared columns
+  // shared experts: pre-activation gradients into dXcat's shared columns
   const int nsms = h->ns * h->ms;
   if (nsms > 0) {
     ++L;
-    LMOE_TRY(launch_act_backward_tiled(static_cast<bf *>(b.ABs), h->sh_rows, b.dU + l, ky,
-                                       nullptr, 0, dXcat + n_pad + l_pad, nx, T, nsms, relu2, s));
+    LMOE_TRY(launch_act_backward_rows<float>(static_cast<bf *>(b.ABs), h->sh_rows, b.dU + l, ky,
+                                             dXcat + n_pad + l_pad, nx, T, nsms, relu2, s));
   }
   // ---- gates, expert-output gradients, expert backward
   ++L;
   LMOE_TRY(launch_slot_grad<bf>(b.dU, ky, static_cast<bf *>(w.O), l, w.pos, w.gates, T, K, b.ds,
                                 static_cast<bf *>(b.DO), s));
   {
-    TcParams p = {};  // dH = DO W_o[e], then dAB = activation backward (in the epilogue)
+    // dH = DO W_o[e] (bf16, through the forward epilogue's TMA stores), then the
+    // activation backward dAB from dH and the recomputed AB, element-wise: as a
+    // kernel of its own it keeps far more loads in flight than the GEMM's
+    // eight epilogue warps could
+    TcParams p = {};
     p.mode = TC_EXPERT_DOWN; p.Kdim = l; p.n_tiles_n = (m + kTileN - 1) / kTileN;
     p.tiles = w.tiles; p.n_mtiles = w.n_tiles;
-    p.ld_out = m; p.relu2 = h->relu2; p.status = w.status;
-    p.act_ab = static_cast<const bf *>(b.AB); p.act_dab = static_cast<bf *>(b.dAB); p.ld_ab = gu;
-    LMOE_TRY(gemm(h->tm_DO, h->tm_woT, p, h->num_sms));
+    p.out = reinterpret_cast<bf *>(b.dH); p.ld_out = m; p.status = w.status; p.tma_out = 1;
+    ++L;
+    LMOE_TRY(launch_tc_gemm(h->tm_DO.bytes, h->tm_woT.bytes, p, h->num_sms, h->num_sms, s,
+                            nullptr, h->tm_dH_out.bytes));
+    ++L;
+    LMOE_TRY(launch_act_backward_rows<bf>(static_cast<const bf *>(b.AB), gu,
+                                          reinterpret_cast<const bf *>(b.dH), m,
+                                          static_cast<bf *>(b.dAB), gu, static_cast<int>(b.Kp), m,
+                                          relu2, s));
   }
   {
     TcParams p = {};  // dZp = dAB W_gu[e]  (fp32 [TK][l])
@@ -1317,7 +1335,8 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
     p.out = static_cast<bf *>(dx); p.ld_out = d; p.status = w.status;
     LMOE_TRY(gemm(h->tm_dXcat, h->tm_wxT, p, m_tiles_T * p.n_tiles_n));
   }
-  // ---- weight gradients: token-major transposes, then A^T B per group
+  // ---- weight gradients: A^T B straight from the token-major matrices
+  // (read MN-major), K running over tokens
   auto fill_sizes = [&](TcParams &p) {
     p.wg_d = d; p.wg_l = l; p.wg_m = m; p.wg_ns = h->ns; p.wg_ms = h->ms; p.wg_n = N;
     p.wg_npad = n_pad; p.wg_lpad = l_pad; p.relu2 = h->relu2; p.status = w.status;
@@ -1325,60 +1344,55 @@ static cudaError_t backward_bf16(lmoe_layer *h, const void *x, const void *dy, v
     p.g_upx = g->w_upx; p.g_out = g->w_out; p.g_sgate = g->s_gate; p.g_sup = g->s_up;
     p.g_sout = g->s_out;
   };
-  L += 4;
-  // (row stride b.Tp, the maps' width; this call reduces over Tp columns)
-  LMOE_TRY(launch_transpose_tokens(static_cast<const bf *>(dy), d, d, nullptr, nullptr, 0, Tp, T,
-                                   static_cast<bf *>(b.dyT), b.Tp, s));
-  LMOE_TRY(launch_transpose_tokens(ucat, ky, ky, nullptr, nullptr, 0, Tp, T,
-                                   static_cast<bf *>(b.ucatT), b.Tp, s));
-  LMOE_TRY(launch_transpose_tokens(dXcat, nx, nx, nullptr, nullptr, 0, Tp, T,
-                                   static_cast<bf *>(b.dXcatT), b.Tp, s));
-  LMOE_TRY(launch_transpose_tokens(static_cast<const bf *>(x), d, d, nullptr, nullptr, 0, Tp, T,
-                                   static_cast<bf *>(b.xT), b.Tp, s));
   {
+    // dense: the maps hold exactly T rows, so a ragged last K-block reads zeros
+    TensorMap64 tm_dy_mn, tm_ucat_mn, tm_dX_mn, tm_x_mn;
+    if (make_map(&tm_dy_mn, dy, T, d, d, 64) != LMOE_OK ||
+        make_map(&tm_ucat_mn, ucat, T, ky, ky, 64) != LMOE_OK ||
+        make_map(&tm_dX_mn, dXcat, T, nx, nx, 64) != LMOE_OK ||
+        make_map(&tm_x_mn, x, T, d, d, 64) != LMOE_OK)
+      return cudaErrorInvalidValue;
+    const int Tp = (T + 63) / 64 * 64;  // whole K-blocks; rows from T on read as zeros
     TcParams p = {};  // [dW_up | dS_o] = dy^T [u | h_s]
-    p.mode = TC_WGRAD; p.wg_kind = WG_Y; p.groups = 1; p.M = d; p.Kdim = static_cast<int>(Tp);
+    p.mode = TC_WGRAD; p.wg_kind = WG_Y; p.groups = 1; p.M = d; p.Kdim = Tp;
     p.n_tiles_n = (ky + kTileN - 1) / kTileN;
     fill_sizes(p);
-    LMOE_TRY(gemm(h->tm_dyT, h->tm_ucatT, p, (d + kTileM - 1) / kTileM * p.n_tiles_n));
-  }
-  {
-    TcParams p = {};  // [dW_r ; dW_down ; dS_g / dS_u] = dXcat^T x
-    p.mode = TC_WGRAD; p.wg_kind = WG_X; p.groups = 1; p.M = nx; p.Kdim = static_cast<int>(Tp);
-    p.n_tiles_n = (d + kTileN - 1) / kTileN;
-    fill_sizes(p);
-    LMOE_TRY(gemm(h->tm_dXcatT, h->tm_xT, p, (nx + kTileM - 1) / kTileM * p.n_tiles_n));
+    LMOE_TRY(gemm(tm_dy_mn, tm_ucat_mn, p, (d + kTileM - 1) / kTileM * p.n_tiles_n));
+    TcParams q = {};  // [dW_r ; dW_down ; dS_g / dS_u] = dXcat^T x
+    q.mode = TC_WGRAD; q.wg_kind = WG_X; q.groups = 1; q.M = nx; q.Kdim = Tp;
+    q.n_tiles_n = (d + kTileN - 1) / kTileN;
+    fill_sizes(q);
+    LMOE_TRY(gemm(tm_dX_mn, tm_x_mn, q, (nx + kTileM - 1) / kTileM * q.n_tiles_n));
   }
   if (g->b_router) {
     ++L;
     LMOE_TRY(launch_bias_grad(b.ds, w.offsets, w.perm, N, g->b_router, s));
   }
-  // grouped: each expert's rows at a 64-aligned K range of the transposes
-  L += 5;
-  LMOE_TRY(launch_padded_offsets(w.offsets, N, b.kstart, b.klen, b.shift, s));
-  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(b.DO), l, l, w.offsets, b.kstart, N, Kp, 0,
-                                   static_cast<bf *>(b.DOT), Kp, s));
-  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(w.H), m, m, w.offsets, b.kstart, N, Kp, 0,
-                                   static_cast<bf *>(b.HT), Kp, s));
-  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(b.dAB), gu, gu, w.offsets, b.kstart, N, Kp, 0,
-                                   static_cast<bf *>(b.dABT), Kp, s));
-  LMOE_TRY(launch_transpose_tokens(static_cast<bf *>(w.zp), l, l, w.offsets, b.kstart, N, Kp, 0,
-                                   static_cast<bf *>(b.zpT), Kp, s));
+  // grouped: expert e reduces over its padded rows [offsets[e], offsets[e + 1]),
+  // whose padding rows must be zero in both operands (zp's already are)
+  {
+    ++L;
+    PadRowsArgs pr = {};
+    pr.ptr[0] = b.DO; pr.cols[0] = l;
+    pr.ptr[1] = w.H; pr.cols[1] = m;
+    pr.ptr[2] = b.dAB; pr.cols[2] = gu;
+    LMOE_TRY(launch_zero_pad_rows(w.offsets, w.seg_end, N, pr, s));
+  }
   {
     TcParams p = {};  // dW_o[e] = DO_e^T H_e
     p.mode = TC_WGRAD; p.wg_kind = WG_O; p.groups = N; p.M = l; p.Kdim = 64;
-    p.k_start = b.kstart; p.k_len = b.klen;
+    p.k_start = w.offsets; p.k_len = nullptr;
     p.n_tiles_n = (m + kTileN - 1) / kTileN;
     fill_sizes(p);
-    LMOE_TRY(gemm(h->tm_DOT, h->tm_HT, p, N * ((l + kTileM - 1) / kTileM) * p.n_tiles_n));
+    LMOE_TRY(gemm(h->tm_DOmn, h->tm_Hmn, p, N * ((l + kTileM - 1) / kTileM) * p.n_tiles_n));
   }
   {
     TcParams p = {};  // [dW_g ; dW_u][e] = dAB_e^T zp_e
     p.mode = TC_WGRAD; p.wg_kind = WG_GU; p.groups = N; p.M = gu; p.Kdim = 64;
-    p.k_start = b.kstart; p.k_len = b.klen;
+    p.k_start = w.offsets; p.k_len = nullptr;
     p.n_tiles_n = (l + kTileN - 1) / kTileN;
     fill_sizes(p);
-    LMOE_TRY(gemm(h->tm_dABT, h->tm_zpT, p, N * ((gu + kTileM - 1) / kTileM) * p.n_tiles_n));
+    LMOE_TRY(gemm(h->tm_dABmn, h->tm_zpmn, p, N * ((gu + kTileM - 1) / kTileM) * p.n_tiles_n));
   }
 #undef LMOE_TRY
   return cudaSuccess;

@@ -227,6 +227,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   return desc;
 }
 
+// MN-major operand tile staged by TMA with 128-byte swizzle, {64, 64} boxes
+// of a token-major matrix: each box is 64 K-rows of 64 MN-elements (128
+// bytes), 8-row groups 1024 bytes apart (stride byte offset); the tile's
+// 64-element MN chunks are boxes 8 KB apart (leading byte offset).  `addr`
+// must be 1024-aligned; advancing by 2048 bytes selects the next K = 16 rows.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t addr) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);  // start address
+  desc |= static_cast<uint64_t>(8192u >> 4) << 16;        // leading byte offset: MN chunks
+  desc |= static_cast<uint64_t>(1024u >> 4) << 32;        // stride byte offset: 8 K-rows
+  desc |= static_cast<uint64_t>(1u) << 46;                // descriptor version (sm_100)
+  desc |= static_cast<uint64_t>(2u) << 61;                // 128-byte swizzle
+  return desc;
+}
+
 // 32 rows of 16 bytes, contiguous, no swizzle: the source of a 32x128b
 // tcgen05.cp.  8-row core matrices of 128 bytes follow one another (stride
 // byte offset 128); there is one core matrix along the row.
@@ -243,6 +258,10 @@ __device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t addr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with A and B MN-major (bits 15 and 16).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 15) | (1u << 16);
 }
 // kind::f8f6f4 instruction descriptor: E4M3 A and B (format 0 in bits [7,10)
 // and [10,13)), f32 accumulate, K-major A and B.

@@ -208,27 +208,30 @@ __device__ void write_tiles(TileEntry *tiles, int tstart, int max_tiles, int e, 
 }
 
 // Phase 2 body, run by one block of kScanThreads threads.
-__device__ void scan_and_tables(int32_t *__restrict__ counts, int n_chunks, int N,
-                                int32_t *__restrict__ offsets, TileEntry *__restrict__ tiles,
-                                int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
-                                TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2,
-                                int tile_m2, int max_tiles2) {
+// Offsets and tile tables from the expert totals of this thread's experts
+// e0 .. e0+3 (all threads of the block call it).  seg.pad > 1: each expert's
+// rows start at a multiple of seg.pad (offsets[e] is the padded start,
+// offsets[N] the padded total, seg.ends[e] = offsets[e] + the expert's count);
+// the tile tables cover the real rows only.
+__device__ void offsets_and_tables(const int (&tot)[kScanPerThread], int e0, int N, SegPad seg,
+                                   int32_t *__restrict__ offsets, TileEntry *__restrict__ tiles,
+                                   int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+                                   TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2,
+                                   int tile_m2, int max_tiles2) {
   __shared__ int warp_sums[32];
-  const int e0 = threadIdx.x * kScanPerThread;  // experts e0 .. e0+3
-  int tot[kScanPerThread], mt[kScanPerThread], mt2[kScanPerThread];
-  int my_tot = 0, my_mt = 0, my_mt2 = 0;
+  int span[kScanPerThread], mt[kScanPerThread], mt2[kScanPerThread];
+  int my_span = 0, my_mt = 0, my_mt2 = 0;
 #pragma unroll
   for (int i = 0; i < kScanPerThread; ++i) {
-    const int e = e0 + i;
-    tot[i] = e < N ? scan_expert_row(counts, e, n_chunks) : 0;
+    span[i] = seg.pad > 1 ? (tot[i] + seg.pad - 1) / seg.pad * seg.pad : tot[i];
     mt[i] = (tot[i] + tile_m - 1) / tile_m;
     mt2[i] = tiles2 ? (tot[i] + tile_m2 - 1) / tile_m2 : 0;
-    my_tot += tot[i];
+    my_span += span[i];
     my_mt += mt[i];
     my_mt2 += mt2[i];
   }
   int all = 0, all_tiles = 0, all_tiles2 = 0;
-  int off = block_exclusive_scan(my_tot, warp_sums, &all);
+  int off = block_exclusive_scan(my_span, warp_sums, &all);
   int tstart = block_exclusive_scan(my_mt, warp_sums, &all_tiles);
   int tstart2 = block_exclusive_scan(my_mt2, warp_sums, &all_tiles2);
 #pragma unroll
@@ -236,10 +239,11 @@ __device__ void scan_and_tables(int32_t *__restrict__ counts, int n_chunks, int 
     const int e = e0 + i;
     if (e < N) {
       offsets[e] = off;
+      if (seg.ends) seg.ends[e] = off + tot[i];
       write_tiles(tiles, tstart, max_tiles, e, off, tot[i], tile_m);
       if (tiles2) write_tiles(tiles2, tstart2, max_tiles2, e, off, tot[i], tile_m2);
     }
-    off += tot[i];
+    off += span[i];
     tstart += mt[i];
     tstart2 += mt2[i];
   }
@@ -250,12 +254,28 @@ __device__ void scan_and_tables(int32_t *__restrict__ counts, int n_chunks, int 
   }
 }
 
+__device__ void scan_and_tables(int32_t *__restrict__ counts, int n_chunks, int N, SegPad seg,
+                                int32_t *__restrict__ offsets, TileEntry *__restrict__ tiles,
+                                int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+                                TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2,
+                                int tile_m2, int max_tiles2) {
+  const int e0 = threadIdx.x * kScanPerThread;  // experts e0 .. e0+3
+  int tot[kScanPerThread];
+#pragma unroll
+  for (int i = 0; i < kScanPerThread; ++i) {
+    const int e = e0 + i;
+    tot[i] = e < N ? scan_expert_row(counts, e, n_chunks) : 0;
+  }
+  offsets_and_tables(tot, e0, N, seg, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
+                     n_tiles2, tile_m2, max_tiles2);
+}
+
 __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
-    int32_t *__restrict__ counts, int n_chunks, int N, int32_t *__restrict__ offsets,
+    int32_t *__restrict__ counts, int n_chunks, int N, SegPad seg, int32_t *__restrict__ offsets,
     TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
     TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2, int tile_m2,
     int max_tiles2) {
-  scan_and_tables(counts, n_chunks, N, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
+  scan_and_tables(counts, n_chunks, N, seg, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
                   n_tiles2, tile_m2, max_tiles2);
 }
 
@@ -268,13 +288,13 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
 // totals go through shared memory to the block-wide scans of offsets and
 // tile starts.  N <= 1024.
 __device__ void scan_and_tables_warps(int32_t *__restrict__ counts, int n_chunks, int N,
-                                      int32_t *__restrict__ offsets, TileEntry *__restrict__ tiles,
+                                      SegPad seg, int32_t *__restrict__ offsets,
+                                      TileEntry *__restrict__ tiles,
                                       int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
                                       TileEntry *__restrict__ tiles2,
                                       int32_t *__restrict__ n_tiles2, int tile_m2,
                                       int max_tiles2) {
   __shared__ int totals[1024];
-  __shared__ int warp_sums[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int ncp = (n_chunks + 3) & ~3;
   const int nv = ncp / 4;                       // int4 vectors per row
@@ -314,39 +334,14 @@ __device__ void scan_and_tables_warps(int32_t *__restrict__ counts, int n_chunks
   __syncthreads();
   // experts e0 .. e0+3 per thread, as in scan_and_tables
   const int e0 = threadIdx.x * kScanPerThread;
-  int tot[kScanPerThread], mt[kScanPerThread], mt2[kScanPerThread];
-  int my_tot = 0, my_mt = 0, my_mt2 = 0;
+  int tot[kScanPerThread];
 #pragma unroll
   for (int i = 0; i < kScanPerThread; ++i) {
     const int e = e0 + i;
     tot[i] = e < N ? totals[e] : 0;
-    mt[i] = (tot[i] + tile_m - 1) / tile_m;
-    mt2[i] = tiles2 ? (tot[i] + tile_m2 - 1) / tile_m2 : 0;
-    my_tot += tot[i];
-    my_mt += mt[i];
-    my_mt2 += mt2[i];
   }
-  int all = 0, all_tiles = 0, all_tiles2 = 0;
-  int off = block_exclusive_scan(my_tot, warp_sums, &all);
-  int tstart = block_exclusive_scan(my_mt, warp_sums, &all_tiles);
-  int tstart2 = block_exclusive_scan(my_mt2, warp_sums, &all_tiles2);
-#pragma unroll
-  for (int i = 0; i < kScanPerThread; ++i) {
-    const int e = e0 + i;
-    if (e < N) {
-      offsets[e] = off;
-      write_tiles(tiles, tstart, max_tiles, e, off, tot[i], tile_m);
-      if (tiles2) write_tiles(tiles2, tstart2, max_tiles2, e, off, tot[i], tile_m2);
-    }
-    off += tot[i];
-    tstart += mt[i];
-    tstart2 += mt2[i];
-  }
-  if (threadIdx.x == 0) {
-    offsets[N] = all;
-    *n_tiles = min(all_tiles, max_tiles);
-    if (tiles2) *n_tiles2 = min(all_tiles2, max_tiles2);
-  }
+  offsets_and_tables(tot, e0, N, seg, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
+                     n_tiles2, tile_m2, max_tiles2);
 }
 
 // Top-K', dispatch histogram and scan in one launch.  Block c takes the
@@ -364,7 +359,7 @@ __global__ void __launch_bounds__(1024) route_select_kernel(
     int n_chunks, int chunk, int32_t *__restrict__ arrivals, int32_t *__restrict__ offsets,
     TileEntry *__restrict__ tiles, int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
     TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2, int tile_m2,
-    int max_tiles2) {
+    int max_tiles2, SegPad seg) {
   __shared__ int hist[1024];
   __shared__ int is_last;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -384,8 +379,8 @@ __global__ void __launch_bounds__(1024) route_select_kernel(
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  scan_and_tables_warps(counts, n_chunks, N, offsets, tiles, n_tiles, tile_m, max_tiles, tiles2,
-                        n_tiles2, tile_m2, max_tiles2);
+  scan_and_tables_warps(counts, n_chunks, N, seg, offsets, tiles, n_tiles, tile_m, max_tiles,
+                        tiles2, n_tiles2, tile_m2, max_tiles2);
   if (threadIdx.x == 0) *arrivals = 0;
 }
 
@@ -607,9 +602,13 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4 *__restri
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
-  const int tok = perm[r] / K;
-  const uint4 *s = src + static_cast<size_t>(tok) * vecs_per_row;
+  const int flat = perm[r];
   uint4 *d = dst + static_cast<size_t>(r) * vecs_per_row;
+  if (flat < 0) {  // a padding row of a padded dispatch order: zeros
+    for (int v = lane; v < vecs_per_row; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const uint4 *s = src + static_cast<size_t>(flat / K) * vecs_per_row;
   for (int v = lane; v < vecs_per_row; v += 32) d[v] = s[v];
 }
 
@@ -761,8 +760,9 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
                             int32_t *pos, int32_t *row_expert, TileEntry *tiles,
                             int32_t *n_tiles, int tile_m, int max_tiles, cudaStream_t s,
                             TileEntry *tiles2, int32_t *n_tiles2, int tile_m2, int max_tiles2,
-                            bool check_ids) {
+                            bool check_ids, SegPad seg) {
   if (N > 1024 || chunk % 32 || chunk < 32 || chunk > 256) return cudaErrorInvalidValue;
+  if (seg.pad < 1 || (seg.pad > 1 && !seg.ends)) return cudaErrorInvalidValue;
   const int nc = dispatch_chunks(T, chunk);
   if (nc > 0 && !counts_ready) {
     dispatch_count_kernel<<<nc, 256, N * sizeof(int32_t), s>>>(ids, T, K, N, chunk_counts, nc,
@@ -771,9 +771,9 @@ cudaError_t launch_dispatch(const int32_t *ids, int T, int K, int N, int32_t *ch
     if (e != cudaSuccess) return e;
   }
   if (tiles2 && (!n_tiles2 || tile_m2 <= 0)) return cudaErrorInvalidValue;
-  dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_counts, nc, N, offsets, tiles, n_tiles,
-                                                   tile_m, max_tiles, tiles2, n_tiles2, tile_m2,
-                                                   max_tiles2);
+  dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_counts, nc, N, seg, offsets, tiles,
+                                                   n_tiles, tile_m, max_tiles, tiles2, n_tiles2,
+                                                   tile_m2, max_tiles2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || nc == 0) return e;
   const int warps = chunk / 32;
@@ -819,17 +819,18 @@ cudaError_t launch_route_select(const float *logits, int ld, const float *bias, 
                                 int32_t *arrivals, int32_t *offsets, TileEntry *tiles,
                                 int32_t *n_tiles, int tile_m, int max_tiles, TileEntry *tiles2,
                                 int32_t *n_tiles2, int tile_m2, int max_tiles2, cudaStream_t s,
-                                bool pdl) {
+                                bool pdl, SegPad seg) {
   if (T <= 0) return cudaSuccess;
   if (!fused_route_ok(N, K, chunk) || !tiles2 || !n_tiles2 || tile_m2 <= 0)
     return cudaErrorInvalidValue;
+  if (seg.pad < 1 || (seg.pad > 1 && !seg.ends)) return cudaErrorInvalidValue;
   const int nc = dispatch_chunks(T, chunk);
   const int vpl = (N + 31) / 32;
   cudaError_t e;
 #define LMOE_ROUTE(V)                                                                            \
   e = launch_ex(route_select_kernel<V>, dim3(nc), dim3(32 * chunk), 0, s, pdl, logits, ld, bias, T, N, \
                 K, ids, gates, counts, nc, chunk, arrivals, offsets, tiles, n_tiles, tile_m,     \
-                max_tiles, tiles2, n_tiles2, tile_m2, max_tiles2)
+                max_tiles, tiles2, n_tiles2, tile_m2, max_tiles2, seg)
   if (vpl <= 1) LMOE_ROUTE(1);
   else if (vpl <= 2) LMOE_ROUTE(2);
   else if (vpl <= 4) LMOE_ROUTE(4);

@@ -74,6 +74,8 @@ constexpr int NUM_EPI_WARPS = 8;              // two per TMEM lane quarter
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, TN);
 constexpr uint32_t IDESC8 = ptx::idesc_e4m3_f32(TM, TN);
 constexpr uint32_t IDESC4 = ptx::idesc_nvf4(TM, TN);
+constexpr uint32_t IDESC_MN = ptx::idesc_bf16_f32_mn(TM, TN);  // TC_WGRAD: MN-major A and B
+constexpr int MN_BOX_BYTES = 64 * 64 * 2;  // one {64, 64} bf16 box of an MN-major tile
 // operand formats of the single-CTA kernel
 constexpr int kBf16 = 0, kE4m3 = 1, kNvf4 = 2;
 // NVFP4 scale blocks of one stage: A 128 rows x 16 scales, B 256 rows x 16,
@@ -127,11 +129,10 @@ static_assert(smem_bytes<kNvf4>(true) <= 232448, "shared memory per CTA");
 struct Tile {
   int a_row, b_row, n_tile, row_hi;
   int mt;     // grouped modes: the M-tile's index in the tile table
-  int k0;     // first K column (A, and B when b_plain)
+  int k0;     // first K index (TC_WGRAD: the first token row of A and B)
   int nkb;    // K-blocks of this tile
   int group;  // TC_WGRAD group
   int expert; // grouped modes: the expert of the tile
-  bool b_plain;  // B is a plain row-major matrix (else K-block tiled)
 };
 
 __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tiles,
@@ -144,7 +145,6 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
   tl.mt = 0;
   tl.group = 0;
   tl.expert = 0;
-  tl.b_plain = false;
   if (p.mode == TC_WGRAD) {
     const int per = m_tiles * p.n_tiles_n;
     const int g = t / per, r = t % per;
@@ -154,10 +154,9 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
     tl.n_tile = n;
     tl.row_hi = p.M;
     tl.group = g;
-    tl.b_plain = true;
-    if (p.k_start) {
+    if (p.k_start) {  // group g's token rows (k_len null: up to the next group's start)
       tl.k0 = p.k_start[g];
-      tl.nkb = p.k_len[g] / kb_elems;
+      tl.nkb = (p.k_len ? p.k_len[g] : p.k_start[g + 1] - p.k_start[g]) / kb_elems;
     }
   } else if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
     const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
@@ -209,6 +208,56 @@ __device__ __forceinline__ void store_f32x32(float *dst, const float *v) {
   float4 *d = reinterpret_cast<float4 *>(dst);
 #pragma unroll
   for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// Row-coalesced stores through the warp's staging buffer (backward
+// epilogues).  Lane i holds 32 values of row i and that row's destination
+// (null: not stored); the values go through shared memory so that each store
+// instruction writes whole row segments (128 bytes of fp32 or 64 bytes of
+// bf16 per row) instead of 16 bytes of 32 different rows.  All 32 lanes call
+// these together; destinations are 16-byte aligned.
+__device__ __forceinline__ void store_rows_f32x32(uint8_t *stage, const float *v, float *dst) {
+  const int lane = threadIdx.x & 31;
+  float4 *st = reinterpret_cast<float4 *>(stage);  // [32][8], chunk k of row r at k ^ (r & 7)
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    st[lane * 8 + (k ^ (lane & 7))] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  __syncwarp();
+  const int ch = lane & 7;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int rr = 4 * j + (lane >> 3);
+    float *d = reinterpret_cast<float *>(
+        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(dst), rr));
+    const float4 val = st[rr * 8 + (ch ^ (rr & 7))];
+    if (d) reinterpret_cast<float4 *>(d)[ch] = val;
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ void store_rows_bf16x32(uint8_t *stage, const float *v,
+                                                   __nv_bfloat16 *dst) {
+  const int lane = threadIdx.x & 31;
+  uint4 *st = reinterpret_cast<uint4 *>(stage);  // [32][4], chunk k of row r at k ^ ((r >> 1) & 3)
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * k + 0], v[8 * k + 1]);
+    w.y = pack_bf16x2(v[8 * k + 2], v[8 * k + 3]);
+    w.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
+    w.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
+    st[lane * 4 + (k ^ ((lane >> 1) & 3))] = w;
+  }
+  __syncwarp();
+  const int ch = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int rr = 8 * j + (lane >> 2);
+    __nv_bfloat16 *d = reinterpret_cast<__nv_bfloat16 *>(
+        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(dst), rr));
+    const uint4 val = st[rr * 4 + (ch ^ ((rr >> 1) & 3))];
+    if (d) reinterpret_cast<uint4 *>(d)[ch] = val;
+  }
+  __syncwarp();
 }
 
 // Per-warp state of the TMA-store epilogue.  map == null: the warp stores
@@ -342,7 +391,8 @@ __device__ __forceinline__ float *wgrad_row_dst(const TcParams &p, int row, int 
 }
 
 __device__ __forceinline__ void epi_wgrad(uint32_t taddr, bool valid, const TcParams &p, int row,
-                                          int group, int col0, bool empty, int half) {
+                                          int group, int col0, bool empty, int half,
+                                          uint8_t *stage) {
   const int ky = p.wg_l + p.wg_ns * p.wg_ms;
   int ld = 0;
   float *rowp = nullptr;
@@ -362,20 +412,20 @@ __device__ __forceinline__ void epi_wgrad(uint32_t taddr, bool valid, const TcPa
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
     }
     const int col = col0 + c * 32;
-    if (!valid || col >= n_cols) continue;
-    float *dst;
-    if (p.wg_kind == WG_Y) {  // columns [0, l): dW_up; then each shared expert's dS_o
-      if (col < p.wg_l) {
-        dst = p.g_up + static_cast<size_t>(row) * p.wg_l + col;
-      } else {
-        const int cc = col - p.wg_l, j = cc / p.wg_ms;
-        dst = p.g_sout + (static_cast<size_t>(j) * p.wg_d + row) * p.wg_ms + (cc - j * p.wg_ms);
+    float *dst = nullptr;
+    if (valid && col < n_cols) {
+      if (p.wg_kind == WG_Y) {  // columns [0, l): dW_up; then each shared expert's dS_o
+        if (col < p.wg_l) {
+          dst = p.g_up + static_cast<size_t>(row) * p.wg_l + col;
+        } else {
+          const int cc = col - p.wg_l, j = cc / p.wg_ms;
+          dst = p.g_sout + (static_cast<size_t>(j) * p.wg_d + row) * p.wg_ms + (cc - j * p.wg_ms);
+        }
+      } else if (rowp) {
+        dst = rowp + col;
       }
-    } else {
-      if (!rowp) continue;
-      dst = rowp + col;
     }
-    store_f32x32(dst, v);
+    store_rows_f32x32(stage, v, dst);
   }
 }
 
@@ -401,7 +451,7 @@ __device__ __forceinline__ void epi_swiglu(uint32_t taddr, bool valid, __nv_bflo
 // accumulator) and the SwiGLU hidden (h_dst + hcol0) of one tile.
 __device__ __forceinline__ void epi_swiglu_raw(uint32_t taddr, bool valid,
                                                __nv_bfloat16 *raw_dst, __nv_bfloat16 *h_dst,
-                                               int half) {
+                                               int half, uint8_t *stage) {
 #pragma unroll 1
   for (int c = half * (TN / 128); c < (half + 1) * (TN / 128); ++c) {
     uint32_t g[32], u[32];
@@ -415,18 +465,16 @@ __device__ __forceinline__ void epi_swiglu_raw(uint32_t taddr, bool valid,
       uv[j] = __uint_as_float(u[j]);
       h[j] = silu_bf16out(gv[j]) * uv[j];
     }
-    if (valid) {
-      store_bf16x32(raw_dst + c * 32, gv);
-      store_bf16x32(raw_dst + TN / 2 + c * 32, uv);
-      store_bf16x32(h_dst + c * 32, h);
-    }
+    store_rows_bf16x32(stage, gv, valid ? raw_dst + c * 32 : nullptr);
+    store_rows_bf16x32(stage, uv, valid ? raw_dst + TN / 2 + c * 32 : nullptr);
+    store_rows_bf16x32(stage, h, valid ? h_dst + c * 32 : nullptr);
   }
 }
 
 // Squared ReLU: raw up pre-activation and h = relu(b)^2, masked at n_cols.
 __device__ __forceinline__ void epi_relu2_raw(uint32_t taddr, bool valid, __nv_bfloat16 *raw_dst,
                                               __nv_bfloat16 *h_dst, int col0, int n_cols,
-                                              int half) {
+                                              int half, uint8_t *stage) {
 #pragma unroll 1
   for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
     uint32_t r[32];
@@ -440,61 +488,27 @@ __device__ __forceinline__ void epi_relu2_raw(uint32_t taddr, bool valid, __nv_b
       h[j] = a * a;
     }
     const int col = col0 + c * 32;
-    if (valid && col < n_cols) {
-      store_bf16x32(raw_dst + col, bv);
-      store_bf16x32(h_dst + col, h);
-    }
+    const bool st = valid && col < n_cols;
+    store_rows_bf16x32(stage, bv, st ? raw_dst + col : nullptr);
+    store_rows_bf16x32(stage, h, st ? h_dst + col : nullptr);
   }
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16 *src, float *v) {
-  const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 w = s4[q];
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[8 * q + 2 * i] = __uint_as_float(ws[i] << 16);
-      v[8 * q + 2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
-    }
-  }
-}
-
-// dh (accumulator) of hidden units col0 .. col0+255 of row `row` -> the
-// pre-activation gradients, written in the GU GEMM's layout:
-// SwiGLU da = dh b silu'(a), db = dh silu(a); squared ReLU db = dh 2 relu(b).
-__device__ __forceinline__ void epi_act_backward(uint32_t taddr, bool valid, const TcParams &p,
-                                                 int row, int col0, int n_units, int half) {
+// fp32 outputs of the backward (dU, dZp): 256 accumulator columns -> the row
+// segment row_dst + col0 .., chunks past n_cols skipped, row-coalesced.
+__device__ __forceinline__ void epi_plain_f32_rows(uint32_t taddr, bool valid, float *row_dst,
+                                                   int col0, int n_cols, int half,
+                                                   uint8_t *stage) {
 #pragma unroll 1
   for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
     uint32_t r[32];
     ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
     ptx::tmem_ld_wait();
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
     const int col = col0 + c * 32;
-    if (!valid || col >= n_units) continue;
-    const size_t base = static_cast<size_t>(row) * p.ld_ab;
-    if (p.relu2) {
-      float bv[32], db[32];
-      load_bf16x32(p.act_ab + base + col, bv);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) db[j] = __uint_as_float(r[j]) * 2.0f * fmaxf(bv[j], 0.0f);
-      store_bf16x32(p.act_dab + base + col, db);
-    } else {
-      const size_t ia = base + 256 * (col >> 7) + (col & 127), ib = ia + 128;
-      float av[32], bv[32], da[32], db[32];
-      load_bf16x32(p.act_ab + ia, av);
-      load_bf16x32(p.act_ab + ib, bv);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float dh = __uint_as_float(r[j]);
-        const float sg = 1.0f / (1.0f + __expf(-av[j]));
-        da[j] = dh * bv[j] * sg * (1.0f + av[j] * (1.0f - sg));
-        db[j] = dh * av[j] * sg;
-      }
-      store_bf16x32(p.act_dab + ia, da);
-      store_bf16x32(p.act_dab + ib, db);
-    }
+    store_rows_f32x32(stage, v, valid && col < n_cols ? row_dst + col : nullptr);
   }
 }
 
@@ -651,13 +665,13 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
           if (p.relu2)
             epi_relu2_raw(taddr, valid, p.out2 + static_cast<size_t>(row) * p.ld_out2,
                           p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
-                          col0 - p.z_end, p.n_cols2, half);
+                          col0 - p.z_end, p.n_cols2, half, sink.buf);
           else
             epi_swiglu_raw(taddr, valid,
                            p.out2 + static_cast<size_t>(row) * p.ld_out2 + (col0 - p.z_end),
                            p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0 +
                                (col0 - p.z_end) / 2,
-                           half);
+                           half, sink.buf);
         } else if (p.relu2) {
           epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + p.out_col0,
                     col0 - p.z_end, p.n_cols2, half);
@@ -674,10 +688,11 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
           else epi_swiglu_scaled(taddr, valid, hrow, col0 / 2, sa, scl, half, &sink);
         } else if (kBwd && p.raw && p.relu2)
           epi_relu2_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out,
-                        p.out_h + static_cast<size_t>(row) * p.ld_h, col0, p.n_cols2, half);
+                        p.out_h + static_cast<size_t>(row) * p.ld_h, col0, p.n_cols2, half,
+                        sink.buf);
         else if (kBwd && p.raw)
           epi_swiglu_raw(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out + col0,
-                         p.out_h + static_cast<size_t>(row) * p.ld_h + col0 / 2, half);
+                         p.out_h + static_cast<size_t>(row) * p.ld_h + col0 / 2, half, sink.buf);
         else if (p.relu2)
           epi_relu2(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0, p.n_cols2,
                     half, &sink);
@@ -686,7 +701,8 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
                      &sink);
         break;
       case TC_WGRAD:
-        if constexpr (kBwd) epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half);
+        if constexpr (kBwd)
+          epi_wgrad(taddr, valid, p, row, tl.group, col0, tl.nkb == 0, half, sink.buf);
         break;
       default:  // TC_EXPERT_DOWN, TC_OUT
         if constexpr (kF8) {
@@ -694,11 +710,9 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
                            p.ld_out, sa,
                            p.b_scale + static_cast<size_t>(tl.expert) * p.b_scale_ld + col0,
                            half, &sink);
-        } else if (kBwd && p.act_dab)
-          epi_act_backward(taddr, valid, p, row, col0, p.ld_out, half);
-        else if (kBwd && p.out_f32)
-          epi_plain<true>(taddr, valid, p.out_f32 + static_cast<size_t>(row) * p.ld_out, col0,
-                          p.ld_out, half);
+        } else if (kBwd && p.out_f32)
+          epi_plain_f32_rows(taddr, valid, p.out_f32 + static_cast<size_t>(row) * p.ld_out, col0,
+                             p.ld_out, half, sink.buf);
         else
           epi_plain<false>(taddr, valid, p.out + static_cast<size_t>(row) * p.ld_out, col0,
                            p.ld_out, half, &sink);
@@ -796,6 +810,20 @@ __global__ void __launch_bounds__(Cfg<kQ>::NUM_THREADS, 1)
           const bool a32 = kF8 && tl.row_hi - tl.a_row <= 32;
           ptx::mbar_arrive_expect_tx(&ctl->full[s], (a32 ? A_BYTES / 4 : A_BYTES) + B_BYTES +
                                                         Cfg<kQ>::SF_BYTES);
+          if (kBwd && p.mode == TC_WGRAD) {
+            // MN-major operands straight from the token-major matrices: A as
+            // two {64, 64} boxes (M columns a_row.., token rows kx..), B as four
+            // (N columns b_row..); rows past a matrix's end read as zeros
+#pragma unroll
+            for (int c = 0; c < TM / 64; ++c)
+              ptx::tma_load_2d(smA + s * A_BYTES + c * MN_BOX_BYTES, &tmA, &ctl->full[s],
+                               tl.a_row + 64 * c, kx);
+#pragma unroll
+            for (int c = 0; c < TN / 64; ++c)
+              ptx::tma_load_2d(smB + s * B_BYTES + c * MN_BOX_BYTES, &tmB, &ctl->full[s],
+                               tl.b_row + 64 * c, kx);
+            continue;
+          }
           ptx::tma_load_2d(smA + s * A_BYTES, a32 ? &tmA32 : &tmA, &ctl->full[s], kx, tl.a_row);
           if constexpr (kQ == kNvf4) {
             // this stage's scale blocks: the A tile's (by M-tile) and the B
@@ -809,10 +837,7 @@ __global__ void __launch_bounds__(Cfg<kQ>::NUM_THREADS, 1)
                                          nkb_all + kb) * SFB_BYTES,
                            SFB_BYTES, &ctl->full[s]);
           }
-          if (tl.b_plain)
-            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], kx, tl.b_row);
-          else
-            ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
+          ptx::tma_load_2d(smB + s * B_BYTES, &tmB, &ctl->full[s], 0, tl.b_row + kb * TN);
         }
       }
       if (!ok) {  // let every copy still in flight land before the CTA exits
@@ -876,6 +901,9 @@ __global__ void __launch_bounds__(Cfg<kQ>::NUM_THREADS, 1)
             else if constexpr (kQ == kE4m3)
               ptx::mma_e4m3(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
                             ptx::smem_desc_sw128(b_addr + k * 32), IDESC8, (kb | k) != 0);
+            else if (kBwd && p.mode == TC_WGRAD)  // MN-major: K = 16 rows = 2048 bytes
+              ptx::mma_bf16(d_tmem, ptx::smem_desc_mn_sw128(a_addr + k * 2048),
+                            ptx::smem_desc_mn_sw128(b_addr + k * 2048), IDESC_MN, (kb | k) != 0);
             else
               ptx::mma_bf16(d_tmem, ptx::smem_desc_sw128(a_addr + k * 32),
                             ptx::smem_desc_sw128(b_addr + k * 32), IDESC, (kb | k) != 0);
@@ -1001,7 +1029,6 @@ __device__ __forceinline__ Tile decode_pair_tile(const TcParams &p, int t, int m
   tl.nkb = p.Kdim / TKB;
   tl.group = 0;
   tl.expert = 0;
-  tl.b_plain = false;
   int row0, b0;
   if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
     const int m = t % m_tiles2, n = p.n_tile_base + t / m_tiles2;  // consecutive pairs share B
@@ -1323,7 +1350,7 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(tc_gemm_kernel<true, kBf16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes<kBf16>(false)));
+                               static_cast<int>(smem_bytes<kBf16>(true)));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(tc_gemm_kernel<false, kE4m3>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1335,7 +1362,7 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
     if (e != cudaSuccess) return e;
     attr_done = dev;
   }
-  const bool bwd = p.mode == TC_WGRAD || p.raw || p.act_dab || p.out_f32 || p.out_h;
+  const bool bwd = p.mode == TC_WGRAD || p.raw || p.out_f32 || p.out_h;
   const bool fp8 = p.b_scale != nullptr;      // quantised operands (E4M3 or NVFP4)
   const bool fp4 = fp8 && p.b_sf != nullptr;  // NVFP4: block scales as well
   if (fp8 && (bwd || !p.a_scale || (p.mode != TC_EXPERT_GU && p.mode != TC_EXPERT_DOWN)))
@@ -1361,9 +1388,9 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   else if (fp8)
     e = launch_ex(tc_gemm_kernel<false, kE4m3>, dim3(grid), dim3(Cfg<kE4m3>::NUM_THREADS),
                   smem_bytes<kE4m3>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
-  else if (bwd)
+  else if (bwd)  // with the staging buffers (row-coalesced epilogue stores)
     e = launch_ex(tc_gemm_kernel<true, kBf16>, dim3(grid), dim3(Cfg<kBf16>::NUM_THREADS),
-                  smem_bytes<kBf16>(false), s, pdl, a, b, a32, o, p);
+                  smem_bytes<kBf16>(true), s, pdl, a, b, a32, o, p);
   else
     e = launch_ex(tc_gemm_kernel<false, kBf16>, dim3(grid), dim3(Cfg<kBf16>::NUM_THREADS),
                   smem_bytes<kBf16>(p.tma_out != 0), s, pdl, a, b, a32, o, p);
@@ -1392,7 +1419,7 @@ cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcP
     dev_pairs = n;
     attr_dev = dev;
   }
-  const bool bwd = p.mode == TC_WGRAD || p.raw || p.act_dab || p.out_f32 || p.out_h;
+  const bool bwd = p.mode == TC_WGRAD || p.raw || p.out_f32 || p.out_h;
   if (bwd || p.b_scale || (p.tma_out && !tmapOut)) return cudaErrorInvalidValue;
   if (p.Kdim % TKB || p.Kdim <= 0 || p.n_tiles_n <= 0) return cudaErrorInvalidValue;
   const int pairs = max_pairs < dev_pairs ? max_pairs : dev_pairs;

@@ -26,13 +26,18 @@ def _lmoe():
     return lmoe
 
 
-def _backward_case(cfg, T=None, max_tokens=None, seed=0, tol=None):
+def _backward_case(cfg, T=None, max_tokens=None, seed=0, tol=None, warm_seed=None):
     lm = _lmoe()
     T = cfg.T if T is None else T
     inp = synth.make_inputs(cfg, seed, "cuda", T=T)
     dy = synth.make_cotangent(cfg, seed, "cuda", T=T)
     layer = lm.LatentMoELayer(cfg, inp, max_tokens=max_tokens or cfg.T, training=True)
     x = inp["x"]
+    if warm_seed is not None:
+        # an earlier call on other tokens leaves its rows in the workspace
+        xw = synth.make_inputs(cfg, warm_seed, "cuda", T=max_tokens or cfg.T)["x"]
+        dyw = synth.make_cotangent(cfg, warm_seed, "cuda", T=max_tokens or cfg.T)
+        layer.backward(xw, dyw)
     dx, grads = layer.backward(x, dy)
     ids, gates, offsets, perm = layer.route(x)
     torch.cuda.synchronize()
@@ -84,6 +89,12 @@ def test_backward_bf16_mid_swiglu_bias():
 
 def test_backward_bf16_mid_relu2():
     _backward_case(MID_RELU2_BF16)
+
+
+def test_backward_bf16_after_a_larger_call():
+    """A call on fewer tokens after one on more: the expert row ranges move,
+    and rows the earlier call wrote must not leak into the weight gradients."""
+    _backward_case(MID_BF16, T=200, max_tokens=300, warm_seed=7)
 
 
 def test_backward_bf16_readme_acc_shape():

@@ -181,9 +181,13 @@ int lmoe_route(lmoe_handle h, const void *x_dev, int32_t T, int32_t *ids,
 int lmoe_forward(lmoe_handle h, const void *x_dev, void *y_dev, int32_t T, void *stream);
 
 /* End-to-end variant with HOST buffers: copies x_host to a handle-owned
- * device staging buffer, runs lmoe_forward, copies y back to y_host, and
- * synchronises `stream` before returning.  Pinned host memory gives full
- * copy bandwidth.  Errors: as lmoe_forward. */
+ * device staging buffer, runs the forward, copies y back to y_host, and
+ * synchronises `stream` before returning.  For T >= 4096 the tokens are
+ * split into up to 4 chunks of at least 2048: a chunk's copy in, forward and
+ * copy out overlap the other chunks' (two handle-owned copy streams; the
+ * forwards run on `stream` in order).  Each token's output is the one a
+ * single call computes.  Pinned host memory gives full copy bandwidth and
+ * the overlap.  Errors: as lmoe_forward. */
 int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T,
                       void *stream);
 

@@ -79,6 +79,10 @@ struct BwdWorkspace {
 
 }  // namespace
 
+// lmoe_forward_host's pipeline: at most this many chunks, of at least this
+// many tokens each
+constexpr int kHostChunks = 4, kHostChunkTokens = 2048;
+
 struct lmoe_layer {
   lmoe_config cfg;
   int d = 0, l = 0, m = 0, N = 0, K = 0, ns = 0, ms = 0, Tmax = 0;
@@ -129,6 +133,9 @@ struct lmoe_layer {
   // the router/down GEMM and joined before the output GEMM.
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  // lmoe_forward_host: copy streams and per-chunk events of its pipeline
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in[kHostChunks] = {}, ev_out[kHostChunks] = {};
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
   TensorMap64 tm_out_z, tm_out_h, tm_out_o;  // epilogue TMA stores: z, H, O
   // B operands of the CTA-pair GEMMs: the same tiled matrices, {64, 128} boxes
@@ -196,6 +203,16 @@ void free_all(lmoe_layer *h) {
   if (h->side) cudaStreamDestroy(h->side);
   h->ev_fork = h->ev_join = nullptr;
   h->side = nullptr;
+  for (int i = 0; i < kHostChunks; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+    h->ev_in[i] = h->ev_out[i] = nullptr;
+  }
+  if (h->ev_start) cudaEventDestroy(h->ev_start);
+  if (h->h2d) cudaStreamDestroy(h->h2d);
+  if (h->d2h) cudaStreamDestroy(h->d2h);
+  h->ev_start = nullptr;
+  h->h2d = h->d2h = nullptr;
 }
 
 int validate(const lmoe_config *c, lmoe_layer *h) {
@@ -503,6 +520,17 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
       delete h;
       return rc;
     }
+  }
+  bool st_ok = cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; st_ok && i < kHostChunks; ++i)
+    st_ok = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!st_ok) {
+    free_all(h);
+    delete h;
+    return LMOE_ERR_CUDA;
   }
   *out = h;
   return LMOE_OK;
@@ -1444,13 +1472,36 @@ int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T
   DeviceGuard g(h->device);
   if (!g.ok) return LMOE_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t bytes = static_cast<size_t>(T) * h->d * h->esize;
-  if (cudaMemcpyAsync(h->ws.x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  // A pipeline over token chunks: chunk c's copy in (h2d stream), its forward
+  // (the caller's stream) and its copy out (d2h stream) run while the other
+  // chunks copy or compute.  Every token's output is computed exactly as in
+  // one call (the layer is row-wise in the tokens), only the order of work
+  // changes.  Chunks of at least kHostChunkTokens tokens, at most kHostChunks.
+  const int n_chunks = std::max(1, std::min(kHostChunks, T / kHostChunkTokens));
+  const size_t row_bytes = static_cast<size_t>(h->d) * h->esize;
+  const uint8_t *xh = static_cast<const uint8_t *>(x_host);
+  uint8_t *yh = static_cast<uint8_t *>(y_host);
+  uint8_t *xd = static_cast<uint8_t *>(h->ws.x_stage), *yd = static_cast<uint8_t *>(h->ws.y_stage);
+  // the copies start after the work already queued on the caller's stream
+  if (cudaEventRecord(h->ev_start, s) != cudaSuccess ||
+      cudaStreamWaitEvent(h->h2d, h->ev_start, 0) != cudaSuccess)
     return LMOE_ERR_CUDA;
-  rc = forward_impl(h, h->ws.x_stage, h->ws.y_stage, T, s);
-  if (rc != LMOE_OK) return rc;
-  if (cudaMemcpyAsync(y_host, h->ws.y_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return LMOE_ERR_CUDA;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int t0 = static_cast<int>(static_cast<int64_t>(T) * c / n_chunks);
+    const int t1 = static_cast<int>(static_cast<int64_t>(T) * (c + 1) / n_chunks);
+    const size_t off = static_cast<size_t>(t0) * row_bytes, bytes = (t1 - t0) * row_bytes;
+    if (cudaMemcpyAsync(xd + off, xh + off, bytes, cudaMemcpyHostToDevice, h->h2d) != cudaSuccess ||
+        cudaEventRecord(h->ev_in[c], h->h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(s, h->ev_in[c], 0) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    rc = forward_impl(h, xd + off, yd + off, t1 - t0, s);
+    if (rc != LMOE_OK) return rc;
+    if (cudaEventRecord(h->ev_out[c], s) != cudaSuccess ||
+        cudaStreamWaitEvent(h->d2h, h->ev_out[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(yh + off, yd + off, bytes, cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(h->d2h) != cudaSuccess) return LMOE_ERR_CUDA;
   return cuda_err(cudaStreamSynchronize(s));
 }
 

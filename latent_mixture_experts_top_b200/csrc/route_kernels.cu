@@ -30,20 +30,33 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 
 // ---------------------------------------------------------------- top-K'
 // One warp per token.  Lane j holds experts e = 32 i + j (i < VPL) as 32-bit
-// order-preserving keys of their logits.  Each of the K' rounds takes the
-// warp maximum of the keys (one REDUX), then the smallest expert index holding
-// that maximum (a second REDUX) -- so equal logits go to the lower index --
-// and removes exactly that entry.  Gates: g_k = e^{s_k - s_0} /
-// sum_j e^{s_j - s_0}, which equals softmax(s) at the selected experts
-// renormalised to sum to one (the softmax denominator cancels).
-// select_token: one token's selection by the calling warp.  The chosen
-// expert of each slot is counted in hist[e] (shared memory) when hist is
-// given, else in gcount[e * gstride] (global) when gcount is given.
+// order-preserving keys of their logits.  The selection order is by key
+// descending, and equal keys go to the lower expert index.  Gates: g_k =
+// e^{s_k - s_0} / sum_j e^{s_j - s_0}, which equals softmax(s) at the selected
+// experts renormalised to sum to one (the softmax denominator cancels).
+//
+// Each of the K' rounds takes the warp maximum of the candidate keys (one
+// REDUX), then the smallest expert index holding that maximum (a second
+// REDUX), and removes exactly that candidate.  With wbuf (64 entries of this
+// warp's shared memory) and K' <= 32 the rounds run over a short candidate
+// list: tau, the K'-th largest of the 32 lane maxima, is at most the K'-th
+// largest key (those K' maxima are K' distinct keys), so every key of the
+// top-K' is >= tau; when at most 64 keys reach tau they are gathered, two per
+// lane, and the rounds take their maximum from two registers instead of VPL.
+// Otherwise the rounds run over all VPL keys of each lane.  Both give the
+// same selection.  The chosen expert of each slot is counted in hist[e]
+// (shared memory) when hist is given, else in gcount[e * gstride] (global)
+// when gcount is given.
+__device__ __forceinline__ bool key_before(uint32_t ka, uint32_t ea, uint32_t kb, uint32_t eb) {
+  return ka > kb || (ka == kb && ea < eb);
+}
+
 template <int VPL>
 __device__ __forceinline__ void select_token(const float *__restrict__ logits, int ld,
                                              const float *__restrict__ bias, int N, int K, int t,
                                              int32_t *__restrict__ ids, float *__restrict__ gates,
-                                             int *hist, int32_t *gcount, int gstride) {
+                                             int *hist, int32_t *gcount, int gstride,
+                                             uint2 *wbuf = nullptr) {
   const int lane = threadIdx.x & 31;
   const float *row = logits + static_cast<size_t>(t) * ld;
   uint32_t key[VPL];
@@ -54,34 +67,105 @@ __device__ __forceinline__ void select_token(const float *__restrict__ logits, i
   }
   int32_t *ids_row = ids + static_cast<size_t>(t) * K;
   float *g_row = gates + static_cast<size_t>(t) * K;
-  float s0 = 0.0f;
-  for (int k = 0; k < K; ++k) {
-    uint32_t m = key[0];
+  // the lane of slot k (k < 32) keeps its key and expert
+  uint32_t slot_key = 0u, slot_e = 0u;
+  bool short_list = false;
+  if (wbuf && K <= 32) {
+    uint32_t lm = key[0];
 #pragma unroll
-    for (int i = 1; i < VPL; ++i) m = max(m, key[i]);
-    const uint32_t wm = __reduce_max_sync(kFull, m);
-    uint32_t cand = 0xFFFFFFFFu;
+    for (int i = 1; i < VPL; ++i) lm = max(lm, key[i]);
+    // bitonic sort of the lane maxima, descending (lane 0 the largest)
+    uint32_t v = lm;
 #pragma unroll
-    for (int i = VPL - 1; i >= 0; --i)
-      if (key[i] == wm) cand = static_cast<uint32_t>(i * 32 + lane);
-    const uint32_t e = __reduce_min_sync(kFull, cand);
+    for (int k = 2; k <= 32; k <<= 1) {
 #pragma unroll
-    for (int i = 0; i < VPL; ++i)
-      if (static_cast<uint32_t>(i * 32 + lane) == e) key[i] = 0u;
-    const float v = key_float(wm);
-    if (k == 0) s0 = v;
-    if ((k & 31) == lane) {  // the same lane re-reads this slot below
-      ids_row[k] = static_cast<int32_t>(e);
-      g_row[k] = v;
-      if (hist) atomicAdd(hist + e, 1);
-      else if (gcount) atomicAdd(gcount + static_cast<size_t>(e) * gstride, 1);
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const uint32_t o = __shfl_xor_sync(kFull, v, j);
+        v = (((lane & k) == 0) == ((lane & j) == 0)) ? max(v, o) : min(v, o);
+      }
+    }
+    const uint32_t tau = __shfl_sync(kFull, v, K - 1);  // > 0: K <= N keys are real
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) c += key[i] >= tau ? 1 : 0;
+    const int total = static_cast<int>(__reduce_add_sync(kFull, static_cast<uint32_t>(c)));
+    if (total <= 64) {
+      short_list = true;
+      int pos = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, pos, off);
+        if (lane >= off) pos += y;
+      }
+      pos -= c;  // exclusive prefix: this lane's first entry
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (key[i] >= tau) wbuf[pos++] = make_uint2(key[i], static_cast<uint32_t>(i * 32 + lane));
+      __syncwarp();
+      // two candidates per lane, a before b; empty entries: key 0
+      uint2 a = lane < total ? wbuf[lane] : make_uint2(0u, 0xFFFFFFFFu);
+      uint2 b = lane + 32 < total ? wbuf[lane + 32] : make_uint2(0u, 0xFFFFFFFFu);
+      __syncwarp();  // wbuf may be refilled by the warp's next token
+      if (key_before(b.x, b.y, a.x, a.y)) {
+        const uint2 tmp = a;
+        a = b;
+        b = tmp;
+      }
+      for (int k = 0; k < K; ++k) {
+        const uint32_t wm = __reduce_max_sync(kFull, a.x);
+        const uint32_t e = __reduce_min_sync(kFull, a.x == wm ? a.y : 0xFFFFFFFFu);
+        if (a.y == e) {  // the one lane that held it
+          a = b;
+          b = make_uint2(0u, 0xFFFFFFFFu);
+        }
+        if (lane == k) {
+          slot_key = wm;
+          slot_e = e;
+        }
+      }
     }
   }
-  float sum = 0.0f;
-  for (int k = lane; k < K; k += 32) sum += expf(g_row[k] - s0);
+  if (!short_list) {
+    for (int k = 0; k < K; ++k) {
+      uint32_t m = key[0];
+#pragma unroll
+      for (int i = 1; i < VPL; ++i) m = max(m, key[i]);
+      const uint32_t wm = __reduce_max_sync(kFull, m);
+      uint32_t cand = 0xFFFFFFFFu;
+#pragma unroll
+      for (int i = VPL - 1; i >= 0; --i)
+        if (key[i] == wm) cand = static_cast<uint32_t>(i * 32 + lane);
+      const uint32_t e = __reduce_min_sync(kFull, cand);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (static_cast<uint32_t>(i * 32 + lane) == e) key[i] = 0u;
+      if ((k & 31) == lane) {  // slots past 32 go straight to memory
+        if (k < 32) {
+          slot_key = wm;
+          slot_e = e;
+        } else {
+          ids_row[k] = static_cast<int32_t>(e);
+          g_row[k] = key_float(wm);
+          if (hist) atomicAdd(hist + e, 1);
+          else if (gcount) atomicAdd(gcount + static_cast<size_t>(e) * gstride, 1);
+        }
+      }
+    }
+  }
+  const float s0 = key_float(__shfl_sync(kFull, slot_key, 0));
+  const bool mine = lane < K;
+  const float ex = mine ? expf(key_float(slot_key) - s0) : 0.0f;
+  float sum = ex;
+  for (int k = lane + 32; k < K; k += 32) sum += expf(g_row[k] - s0);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
-  for (int k = lane; k < K; k += 32) g_row[k] = expf(g_row[k] - s0) / sum;
+  if (mine) {
+    ids_row[lane] = static_cast<int32_t>(slot_e);
+    g_row[lane] = ex / sum;
+    if (hist) atomicAdd(hist + slot_e, 1);
+    else if (gcount) atomicAdd(gcount + static_cast<size_t>(slot_e) * gstride, 1);
+  }
+  for (int k = lane + 32; k < K; k += 32) g_row[k] = expf(g_row[k] - s0) / sum;
 }
 
 // topk_kernel: one warp per token.  If `counts` is given ([N][n_chunks],
@@ -280,30 +364,108 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
 }
 
 // ---------------------------------------------------------------- fused routing
-// Phase 2 with one warp per expert row (any number of warps): lane j takes a
-// contiguous run of the row's chunk counts, the warp scans the runs' sums, and
-// each count becomes the exclusive prefix within its row, as in
-// scan_and_tables.  A row costs two short passes over one run per lane
-// instead of one thread walking the whole row in dependent groups.  Expert
-// totals go through shared memory to the block-wide scans of offsets and
-// tile starts.  N <= 1024.
-__device__ void scan_and_tables_warps(int32_t *__restrict__ counts, int n_chunks, int N,
-                                      SegPad seg, int32_t *__restrict__ offsets,
-                                      TileEntry *__restrict__ tiles,
-                                      int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
-                                      TileEntry *__restrict__ tiles2,
-                                      int32_t *__restrict__ n_tiles2, int tile_m2,
-                                      int max_tiles2) {
-  __shared__ int totals[1024];
+// Phase 2 for the fused routing launch: each row of the count matrix becomes
+// the exclusive prefix of its chunk counts, as in scan_and_tables, and the
+// row's total goes to totals[e].  The rows are independent, so the loads of
+// several rows are issued before any row is scanned: the scan costs a few
+// dependent memory round trips instead of two per row.
+//
+// Short rows (at most 8 vectors, 32 chunks): one row per thread, the whole
+// row in registers, scanned serially.
+__device__ __forceinline__ int scan_row_thread(int4 *row, int nv, int n_chunks) {
+  int4 q[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) q[v] = v < nv ? __ldcg(row + v) : make_int4(0, 0, 0, 0);
+  int run = 0;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    if (v >= nv) break;
+    const int c = 4 * v;
+    int4 o;
+    o.x = run; run += c + 0 < n_chunks ? q[v].x : 0;
+    o.y = run; run += c + 1 < n_chunks ? q[v].y : 0;
+    o.z = run; run += c + 2 < n_chunks ? q[v].z : 0;
+    o.w = run; run += c + 3 < n_chunks ? q[v].w : 0;
+    row[v] = o;
+  }
+  return run;
+}
+
+// Longer rows: one warp per row, R rows per warp at a time.  Lane j holds the
+// PER consecutive vectors j*PER .. j*PER+PER-1 of each of its rows (entries
+// past n_chunks are row padding and count as zero); the warp scans the lanes'
+// sums, and each lane writes its run's prefixes.
+template <int PER, int R>
+__device__ __forceinline__ void scan_rows_warp(int32_t *__restrict__ counts, int ncp,
+                                               int n_chunks, int N, int *totals) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const int ncp = (n_chunks + 3) & ~3;
-  const int nv = ncp / 4;                       // int4 vectors per row
-  const int per = (nv + 31) / 32;               // vectors per lane (contiguous)
+  const int nv = ncp / 4;
+  for (int e0 = warp * R; e0 < N; e0 += nwarps * R) {
+    int4 q[R][PER];
+    int sum[R], incl[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const bool on = e0 + r < N;
+      const int4 *row = reinterpret_cast<const int4 *>(counts + static_cast<size_t>(on ? e0 + r : 0) * ncp);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int v = lane * PER + i;
+        q[r][i] = on && v < nv ? __ldcg(row + v) : make_int4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      int s = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int c = 4 * (lane * PER + i);
+        s += (c + 0 < n_chunks ? q[r][i].x : 0) + (c + 1 < n_chunks ? q[r][i].y : 0) +
+             (c + 2 < n_chunks ? q[r][i].z : 0) + (c + 3 < n_chunks ? q[r][i].w : 0);
+      }
+      sum[r] = s;
+      incl[r] = s;
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int y = __shfl_up_sync(kFull, incl[r], off);
+        if (lane >= off) incl[r] += y;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e = e0 + r;
+      if (e >= N) break;  // the same for every lane
+      int4 *row = reinterpret_cast<int4 *>(counts + static_cast<size_t>(e) * ncp);
+      int run = incl[r] - sum[r];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int v = lane * PER + i;
+        if (v >= nv) break;
+        const int c = 4 * v;
+        int4 o;
+        o.x = run; run += c + 0 < n_chunks ? q[r][i].x : 0;
+        o.y = run; run += c + 1 < n_chunks ? q[r][i].y : 0;
+        o.z = run; run += c + 2 < n_chunks ? q[r][i].z : 0;
+        o.w = run; run += c + 3 < n_chunks ? q[r][i].w : 0;
+        row[v] = o;
+      }
+      if (lane == 31) totals[e] = incl[r];
+    }
+  }
+}
+
+// Rows of any length: one warp per row, each lane a contiguous run of vectors
+// read twice (once for its sum, once for the prefixes).
+__device__ void scan_rows_warp_any(int32_t *__restrict__ counts, int ncp, int n_chunks, int N,
+                                   int *totals) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int nv = ncp / 4;
+  const int per = (nv + 31) / 32;
   for (int e = warp; e < N; e += nwarps) {
     int4 *row = reinterpret_cast<int4 *>(counts + static_cast<size_t>(e) * ncp);
     const int v0 = lane * per, v1 = min(nv, v0 + per);
-    // pass 1: the lane's sum (its run of chunk counts; entries past n_chunks
-    // are row padding and count as zero)
     int sum = 0;
     for (int v = v0; v < v1; ++v) {
       const int4 q = __ldcg(row + v);
@@ -317,7 +479,6 @@ __device__ void scan_and_tables_warps(int32_t *__restrict__ counts, int n_chunks
       const int y = __shfl_up_sync(kFull, incl, off);
       if (lane >= off) incl += y;
     }
-    // pass 2: each count becomes the number of pairs in the chunks before it
     int run = incl - sum;
     for (int v = v0; v < v1; ++v) {
       const int4 q = __ldcg(row + v);
@@ -330,6 +491,33 @@ __device__ void scan_and_tables_warps(int32_t *__restrict__ counts, int n_chunks
       row[v] = o;
     }
     if (lane == 31) totals[e] = incl;
+  }
+}
+
+// Phase 2 of the fused launch (any number of warps, N <= 1024): the row scans
+// above by row length, then the block-wide scans of offsets and tile starts.
+__device__ void scan_and_tables_warps(int32_t *__restrict__ counts, int n_chunks, int N,
+                                      SegPad seg, int32_t *__restrict__ offsets,
+                                      TileEntry *__restrict__ tiles,
+                                      int32_t *__restrict__ n_tiles, int tile_m, int max_tiles,
+                                      TileEntry *__restrict__ tiles2,
+                                      int32_t *__restrict__ n_tiles2, int tile_m2,
+                                      int max_tiles2) {
+  __shared__ int totals[1024];
+  const int ncp = (n_chunks + 3) & ~3;
+  const int nv = ncp / 4;  // int4 vectors per row
+  if (nv <= 8) {
+    for (int e = threadIdx.x; e < N; e += blockDim.x)
+      totals[e] = scan_row_thread(reinterpret_cast<int4 *>(counts + static_cast<size_t>(e) * ncp),
+                                  nv, n_chunks);
+  } else if (nv <= 32) {
+    scan_rows_warp<1, 4>(counts, ncp, n_chunks, N, totals);
+  } else if (nv <= 64) {
+    scan_rows_warp<2, 4>(counts, ncp, n_chunks, N, totals);
+  } else if (nv <= 128) {
+    scan_rows_warp<4, 2>(counts, ncp, n_chunks, N, totals);
+  } else {
+    scan_rows_warp_any(counts, ncp, n_chunks, N, totals);
   }
   __syncthreads();
   // experts e0 .. e0+3 per thread, as in scan_and_tables
@@ -361,6 +549,7 @@ __global__ void __launch_bounds__(1024) route_select_kernel(
     TileEntry *__restrict__ tiles2, int32_t *__restrict__ n_tiles2, int tile_m2,
     int max_tiles2, SegPad seg) {
   __shared__ int hist[1024];
+  __shared__ uint2 cand[32][64];  // each warp's top-K' candidate list
   __shared__ int is_last;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
@@ -368,7 +557,7 @@ __global__ void __launch_bounds__(1024) route_select_kernel(
   __syncthreads();
   const int t0 = blockIdx.x * chunk, t1 = min(T, t0 + chunk);
   for (int t = t0 + warp; t < t1; t += nwarps)  // one pass: nwarps == chunk
-    select_token<VPL>(logits, ld, bias, N, K, t, ids, gates, hist, nullptr, 0);
+    select_token<VPL>(logits, ld, bias, N, K, t, ids, gates, hist, nullptr, 0, cand[warp]);
   __syncthreads();
   const int ncp = (n_chunks + 3) & ~3;
   for (int e = threadIdx.x; e < N; e += blockDim.x)

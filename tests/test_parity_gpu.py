@@ -239,6 +239,38 @@ def test_hot_expert_and_starved_experts():
     layer.close()
 
 
+@pytest.mark.parametrize("pattern", ["four_levels", "thirty_equal"])
+def test_exact_ties_route_to_lower_index(pattern):
+    """Exactly equal router scores (zero router weights, a bias with repeated
+    values): the selection takes the lower expert index among equal scores and
+    the gates are equal.  "four_levels" (bias e % 4: 64 experts share the top
+    score) leaves too many candidates for the short list; "thirty_equal"
+    (thirty experts on distinct lanes share the top score) fills it with ties."""
+    from dataclasses import replace
+    cfg = configs.README_ACC
+    N, K, T = cfg.n_routed, cfg.k_active, 256
+    inp = dict(_inputs(cfg))
+    inp["w_router"] = torch.zeros_like(inp["w_router"])
+    bias = torch.zeros(N, device="cuda")
+    if pattern == "four_levels":
+        bias += (torch.arange(N, device="cuda") % 4).float()
+        top = [e for e in range(N) if e % 4 == 3]
+    else:
+        chosen = sorted(5 + 7 * k for k in range(30))
+        bias[chosen] = 1.0
+        top = chosen
+    inp["b_router"] = bias
+    layer = _lmoe().LatentMoELayer(replace(cfg, router_bias_std=1.0), inp, max_tokens=T)
+    ids, gates, offsets, perm = layer.route(inp["x"][:T].contiguous())
+    torch.cuda.synchronize()
+    want = np.array(top[:K], dtype=np.int32)
+    assert (ids.cpu().numpy() == want[None, :]).all()
+    g = gates.cpu().numpy()
+    assert (g == g[0, 0]).all() and abs(float(g[0, 0]) - 1.0 / K) < 1e-7
+    pu.check_dispatch(ids.cpu().numpy(), offsets.cpu().numpy(), perm.cpu().numpy(), N)
+    layer.close()
+
+
 @pytest.mark.parametrize("cfg", [configs.TINY_F32, configs.README_ACC], ids=["f32", "bf16"])
 def test_deterministic(cfg):
     inp = _inputs(cfg)

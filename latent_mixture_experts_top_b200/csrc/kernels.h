@@ -201,7 +201,21 @@ struct TcParams {
   // on the same stream.
   int pdl;
   int32_t *status;
+  // Split reduction (dense pair launches only: TC_OUT, and TC_X_FUSED over the
+  // router and z columns): k_split > 1 cuts the K-blocks into k_split slices of
+  // consecutive K-blocks, each tile-slice a work item of its own, so that a
+  // launch with few output tiles still fills the GPU.  Each item writes its
+  // fp32 partial to part [k_split][M][n_tiles_n * 256]; launch_splitk_reduce
+  // then sums the slices in slice order and applies the mode's output step.
+  int k_split;         // at most kMaxKSplit
+  float *part;
 };
+constexpr int kMaxKSplit = 16;
+
+// The output step of a split launch: out = sum over slices of p.part, in
+// slice order (fp32), then by mode: TC_OUT bf16 y; TC_X_FUSED fp32 router
+// logits and bf16 z.  pdl: launched right after the split GEMM on s.
+cudaError_t launch_splitk_reduce(const TcParams &p, cudaStream_t s, bool pdl);
 
 // B operands of the tcgen05 GEMMs are stored K-block tiled: for each group
 // (expert, or the whole matrix), N-tile n of 256 rows and K-block kb of 64

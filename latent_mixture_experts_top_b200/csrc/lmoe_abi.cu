@@ -45,6 +45,7 @@ struct Workspace {
   int32_t *status = nullptr;
   int32_t *arrivals = nullptr;  // fused routing: the last-block counter (zero between launches)
   int32_t *seg_end = nullptr;   // training: the end of each expert's rows in the padded order
+  float *part = nullptr;        // bf16: fp32 partials of split dense GEMMs (kPartFloats)
   // E4M3 / NVFP4 routed experts: the expert GEMMs' A operands with row scales
   uint8_t *zq = nullptr, *hq = nullptr;  // [TK][l], [TK][m] (NVFP4: packed, half the bytes)
   float *zq_scale = nullptr, *hq_scale = nullptr;  // [TK]
@@ -82,6 +83,12 @@ struct BwdWorkspace {
 // lmoe_forward_host's pipeline: at most this many chunks, of at least this
 // many tokens each
 constexpr int kHostChunks = 4, kHostChunkTokens = 2048;
+// Split reductions of the dense pair GEMMs (the x-GEMM's router and z columns,
+// the output GEMM) when their output tiles fill fewer than half of the CTA
+// pairs (few tokens): at most kMaxSplit slices of at least kMinSplitKb
+// K-blocks each, the partials of one launch within kPartFloats.
+constexpr int kMaxSplit = kMaxKSplit, kMinSplitKb = 4;
+constexpr size_t kPartFloats = static_cast<size_t>(96) * 256 * 256;  // 24 MiB
 
 struct lmoe_layer {
   lmoe_config cfg;
@@ -195,7 +202,7 @@ void free_all(lmoe_layer *h) {
                   h->w_o8, h->gu_scale, h->o_scale, h->gu_sf, h->o_sf, h->ws.zq_sf, h->ws.hq_sf,
                   h->ws.ep_tiles, h->ws.ep_tiles2,
                   h->ws.ep_n_tiles, h->ws.ep_n_tiles2, h->ws.arrivals, h->ws.zq, h->ws.hq,
-                  h->ws.zq_scale, h->ws.hq_scale};
+                  h->ws.zq_scale, h->ws.hq_scale, h->ws.part};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
@@ -363,6 +370,7 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
             dalloc(&w.H, static_cast<size_t>(h->h_rows) * m * es) && dalloc(&w.O, TKr * l * es) &&
             dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
             dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16) && dalloc(&w.arrivals, 16);
+  if (ok && h->bf16) ok = dalloc(&w.part, kPartFloats * 4);
   if (ok) {  // weights
     if (h->bf16) {
       // K-block-tiled B operands (see launch_repack_btiles)
@@ -702,6 +710,23 @@ static void mark(lmoe_layer *h, int i, cudaStream_t s) {
   }
 }
 
+// Slices for a dense launch of `tiles` output tiles over nkb K-blocks, M rows
+// and `cols` output columns on `slots` CTAs (or CTA pairs): 1 (no split) once
+// the tiles fill half of the slots; otherwise enough slices to fill them,
+// each non-empty.  A split launch runs on single CTAs when its tokens fit one
+// 128-row M-tile (a pair's 256-row MMA would be mostly empty rows).  Calls
+// of kHostChunkTokens tokens or more never split, so that lmoe_forward_host's
+// chunks take the same path (and give the same bits) as one call over all
+// their tokens.
+static int split_for(int tiles, int nkb, int M, int cols, int slots) {
+  if (M >= kHostChunkTokens || tiles <= 0 || 2 * tiles > slots) return 1;
+  int ks = std::min(std::min(slots / tiles, kMaxSplit), nkb / kMinSplitKb);
+  while (ks > 1 && static_cast<size_t>(ks) * M * cols > kPartFloats) --ks;
+  if (ks < 2) return 1;
+  const int per = (nkb + ks - 1) / ks;
+  return (nkb + per - 1) / per;
+}
+
 static int check_call(lmoe_handle h, int32_t T) {
   if (!h) return LMOE_ERR_NULL_ARG;
   if (!h->loaded) return LMOE_ERR_NOT_LOADED;
@@ -749,8 +774,21 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     p.tma_out = 1;  // z through TMA stores (the logits are stored directly)
     const int m_tiles = (T + kTileM - 1) / kTileM;
     const int m_tiles2 = (T + 2 * kTileM - 1) / (2 * kTileM);
-    e = launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, p, m_tiles2 * p.n_tiles_n, s,
-                            h->tm_out_z.bytes);
+    // few tokens: split the reduction (partials, then launch_splitk_reduce)
+    const bool one_mtile = m_tiles == 1;
+    const int xs = split_for((one_mtile ? m_tiles : m_tiles2) * p.n_tiles_n, h->d / 64, T,
+                             p.n_tiles_n * kTileN, one_mtile ? h->num_sms : h->num_sms / 2);
+    if (xs > 1) {
+      p.k_split = xs;
+      p.part = w.part;
+    }
+    if (xs > 1 && one_mtile) {
+      p.tma_out = 0;
+      e = launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, p, h->num_sms, p.n_tiles_n * xs, s);
+    } else {
+      e = launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, p, m_tiles2 * p.n_tiles_n * xs, s,
+                              h->tm_out_z.bytes);
+    }
     h->launches += 1;
     const int shared_tiles_n = (h->nx_rows - h->n_pad - h->l_pad) / kTileN;
     if (e == cudaSuccess && full && shared_tiles_n > 0) {
@@ -758,6 +796,8 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       // the side stream: it overlaps the routing kernels; the output GEMM joins
       // it.  The backward's raw variant runs on the single-CTA kernel.
       TcParams q = p;
+      q.k_split = 0;
+      q.part = nullptr;
       q.n_tile_base = (h->n_pad + h->l_pad) / kTileN;
       q.n_tiles_n = shared_tiles_n;
       // direct stores: the smaller shared-memory footprint lets the routing
@@ -780,6 +820,10 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
                                                       std::max(1, h->num_sms / 3)),
                                              h->side);
       if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
+      h->launches += 1;
+    }
+    if (e == cudaSuccess && xs > 1) {
+      e = launch_splitk_reduce(p, s, false);
       h->launches += 1;
     }
   } else {
@@ -997,8 +1041,24 @@ static cudaError_t run_combine_out_bf16(lmoe_layer *h, const void *O, void *y, i
   TensorMap64 tm_y;
   q.tma_out = make_tmap_bf16_out(tm_y.bytes, y, T, h->d, h->d) == 0 ? 1 : 0;
   const int tiles2 = (T + 2 * kTileM - 1) / (2 * kTileM) * q.n_tiles_n;
-  e = launch_tc_gemm_pair(h->tm_ucat.bytes, h->tm_wy2.bytes, q, tiles2, s, tm_y.bytes);
+  // few tokens: split the reduction (partials, then launch_splitk_reduce)
+  const bool one_mtile = T <= kTileM;
+  const int ys = split_for(one_mtile ? q.n_tiles_n : tiles2, h->ky / 64, T,
+                           q.n_tiles_n * kTileN, one_mtile ? h->num_sms : h->num_sms / 2);
+  if (ys > 1) {
+    q.k_split = ys;
+    q.part = w.part;
+    q.tma_out = 0;
+  }
+  if (ys > 1 && one_mtile)
+    e = launch_tc_gemm(h->tm_ucat.bytes, h->tm_wy.bytes, q, h->num_sms, q.n_tiles_n * ys, s);
+  else
+    e = launch_tc_gemm_pair(h->tm_ucat.bytes, h->tm_wy2.bytes, q, tiles2 * ys, s, tm_y.bytes);
   h->launches += 1;
+  if (e == cudaSuccess && ys > 1) {
+    e = launch_splitk_reduce(q, s, true);
+    h->launches += 1;
+  }
   return e;
 }
 

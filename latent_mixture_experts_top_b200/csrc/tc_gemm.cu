@@ -159,9 +159,18 @@ __device__ __forceinline__ Tile decode_tile(const TcParams &p, int t, int m_tile
       tl.nkb = (p.k_len ? p.k_len[g] : p.k_start[g + 1] - p.k_start[g]) / kb_elems;
     }
   } else if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
-    const int m = t % m_tiles, n = p.n_tile_base + t / m_tiles;  // consecutive CTAs share B
+    // consecutive CTAs share B; with k_split, item r of an M-tile is slice
+    // r % k_split of N-tile r / k_split (its K-blocks from k0 on; the slice
+    // index in group)
+    const int ks = p.k_split > 1 ? p.k_split : 1;
+    const int m = t % m_tiles, r = t / m_tiles;
+    const int split = r % ks, n = p.n_tile_base + r / ks;
+    const int per = (nkb_all + ks - 1) / ks;
     tl.a_row = m * TM;
-    tl.b_row = n * nkb_all * TN;  // first K-block tile of B's N-tile n
+    tl.b_row = (n * nkb_all + split * per) * TN;  // first K-block tile of the slice
+    tl.k0 = split * per * kb_elems;
+    tl.nkb = min(per, nkb_all - split * per);
+    tl.group = split;
     tl.n_tile = n;
     tl.row_hi = p.M;
   } else {
@@ -652,6 +661,25 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, const Tile &tl,
   constexpr int kHalfStep = Cfg<kQ>::EPI_WARPS / 4;
   // kF8: the A row's scale (rows past the tile's end are not stored)
   const float sa = (kF8 && valid) ? p.a_scale[row] : 0.0f;
+  if (!kBwd && !kF8 && p.k_split > 1) {
+    // one slice of a split reduction: the fp32 partial of this tile's rows
+    const int ld = p.n_tiles_n * TN;
+    float *dst = p.part + (static_cast<size_t>(tl.group) * p.M + row) * ld +
+                 (col0 - p.n_tile_base * TN);
+    for (int half = half0; half < 2; half += kHalfStep) {
+#pragma unroll 1
+      for (int c = half * (TN / 64); c < (half + 1) * (TN / 64); ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(taddr + c * 32, r);
+        ptx::tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (valid) store_f32x32(dst + c * 32, v);
+      }
+    }
+    return;
+  }
   for (int half = half0; half < 2; half += kHalfStep) {
     switch (p.mode) {
       case TC_X_FUSED:
@@ -785,7 +813,8 @@ __global__ void __launch_bounds__(Cfg<kQ>::NUM_THREADS, 1)
   // everything above touched only shared memory, TMEM and the parameters
   griddep_wait();
   const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n
-                            : m_tiles * p.n_tiles_n * (p.mode == TC_WGRAD ? p.groups : 1);
+                            : m_tiles * p.n_tiles_n *
+                                  (p.mode == TC_WGRAD ? p.groups : p.k_split > 1 ? p.k_split : 1);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1031,9 +1060,18 @@ __device__ __forceinline__ Tile decode_pair_tile(const TcParams &p, int t, int m
   tl.expert = 0;
   int row0, b0;
   if (p.mode == TC_X_FUSED || p.mode == TC_OUT) {
-    const int m = t % m_tiles2, n = p.n_tile_base + t / m_tiles2;  // consecutive pairs share B
+    // consecutive pairs share B; with k_split, item r of an M-tile is slice
+    // r % k_split of N-tile r / k_split (K-blocks [k0, k0 + nkb) of that slice,
+    // its index in group)
+    const int m = t % m_tiles2, r = t / m_tiles2;
+    const int ks = p.k_split > 1 ? p.k_split : 1;
+    const int split = r % ks, n = p.n_tile_base + r / ks;
+    const int nkb_all = tl.nkb, per = (nkb_all + ks - 1) / ks;
     row0 = m * 2 * TM;
-    b0 = n * tl.nkb * TN;
+    b0 = (n * nkb_all + split * per) * TN;
+    tl.k0 = split * per * TKB;
+    tl.nkb = min(per, nkb_all - split * per);
+    tl.group = split;
     tl.n_tile = n;
     tl.row_hi = p.M;
   } else {
@@ -1110,7 +1148,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kBf16>::NUM_THRE
   const uint32_t tmem_base = ctl->tmem_base;
   // everything above touched only shared memory, TMEM and the parameters
   griddep_wait();
-  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n : m_tiles2 * p.n_tiles_n;
+  const int total = grouped ? (*p.n_mtiles) * p.n_tiles_n
+                            : m_tiles2 * p.n_tiles_n * (p.k_split > 1 ? p.k_split : 1);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1133,7 +1172,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kBf16>::NUM_THRE
           }
           if (leader) ptx::mbar_arrive_expect_tx(&ctl->full[s], tx);
           const uint32_t bar = full0 + s * 8;
-          if (load_a) ptx::tma_load_2d_pair(smA + s * A_BYTES, &tmA, bar, kb * TKB, tl.a_row);
+          if (load_a) ptx::tma_load_2d_pair(smA + s * A_BYTES, &tmA, bar, tl.k0 + kb * TKB, tl.a_row);
           ptx::tma_load_2d_pair(smB + s * P_B_BYTES, &tmB, bar, 0, tl.b_row + kb * TN);
         }
       }
@@ -1150,10 +1189,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kBf16>::NUM_THRE
       const uint32_t empty_peer = ptx::map_to_rank(empty_me, peer);
       const uint32_t accf_me = ptx::smem_u32(&ctl->acc_full[0]);
       const uint32_t accf_peer = ptx::map_to_rank(accf_me, peer);
-      const int nkb = p.Kdim / TKB;
       int it = 0, tl_count = 0;
       bool ok = true;
       for (int t = cid; t < total && ok; t += ncl, ++tl_count) {
+        bool unused_rows;
+        const int nkb = decode_pair_tile(p, t, m_tiles2, rank, &unused_rows).nkb;
         const int acc = tl_count & 1;
         const uint32_t acc_ph = (tl_count >> 1) & 1;
         if (!ptx::mbar_wait(&ctl->acc_empty[acc], acc_ph ^ 1, abort_flag)) {
@@ -1250,6 +1290,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kBf16>::NUM_THRE
   }
 }
 
+// Output step of a split reduction: each thread sums one 4-column group of
+// one row over the slices, in slice order, and stores it by mode (TC_OUT: y in
+// bf16; TC_X_FUSED: router logits in fp32, z in bf16).
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const TcParams p) {
+  griddep_wait();
+  const int ld = p.n_tiles_n * TN, groups = ld / 4;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<int64_t>(p.M) * groups) return;
+  const int row = static_cast<int>(i / groups), c = static_cast<int>(i % groups) * 4;
+  const size_t slice = static_cast<size_t>(p.M) * ld;
+  const float *src = p.part + static_cast<size_t>(row) * ld + c;
+  // every slice's load in flight at once, then the sum in slice order
+  float4 b[kMaxKSplit];
+#pragma unroll
+  for (int k = 0; k < kMaxKSplit; ++k)
+    if (k < p.k_split) b[k] = __ldcg(reinterpret_cast<const float4 *>(src + k * slice));
+  float4 a = b[0];
+#pragma unroll
+  for (int k = 1; k < kMaxKSplit; ++k) {
+    if (k < p.k_split) {
+      a.x += b[k].x;
+      a.y += b[k].y;
+      a.z += b[k].z;
+      a.w += b[k].w;
+    }
+  }
+  const float v[4] = {a.x, a.y, a.z, a.w};
+  const int col = p.n_tile_base * TN + c;  // column of the launch's output space
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int cj = col + j;
+    if (p.mode == TC_OUT) {
+      if (cj < p.ld_out) p.out[static_cast<size_t>(row) * p.ld_out + cj] = __float2bfloat16_rn(v[j]);
+    } else if (cj < p.r_end) {
+      if (cj < p.n_routed) p.logits[static_cast<size_t>(row) * p.ld_logits + cj] = v[j];
+    } else if (cj < p.z_end && cj - p.r_end < p.l) {
+      p.z[static_cast<size_t>(row) * p.ld_z + (cj - p.r_end)] = __float2bfloat16_rn(v[j]);
+    }
+  }
+}
+
 // Failure-detection self-test: one warp waits, with the same bounded wait as
 // the GEMM roles, on an mbarrier that nothing ever completes; the wait runs
 // out after limit_ns and the status word records it.  No fault, no hang.
@@ -1285,6 +1366,25 @@ EncodeTiledFn encode_fn() {
 }
 
 }  // namespace
+
+// A split reduction is valid for the dense output modes (TC_OUT; TC_X_FUSED
+// over the router and z columns only) with a partial buffer, every slice
+// holding at least one K-block.
+static bool split_ok(const TcParams &p, int kb_elems) {
+  const int nkb = p.Kdim / kb_elems, per = (nkb + p.k_split - 1) / p.k_split;
+  const bool x_cols =
+      p.mode == TC_X_FUSED && !p.raw && (p.n_tile_base + p.n_tiles_n) * TN <= p.z_end;
+  return p.part && p.k_split <= kMaxKSplit && (p.mode == TC_OUT || x_cols) &&
+         (p.k_split - 1) * per < nkb;
+}
+
+cudaError_t launch_splitk_reduce(const TcParams &p, cudaStream_t s, bool pdl) {
+  if (p.k_split < 2 || !p.part || p.M <= 0) return cudaErrorInvalidValue;
+  const int64_t items = static_cast<int64_t>(p.M) * (p.n_tiles_n * TN / 4);
+  const int blocks = static_cast<int>((items + 255) / 256);
+  cudaError_t e = launch_ex(splitk_reduce_kernel, dim3(blocks), dim3(256), 0, s, pdl, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 int make_tmap_bf16(void *tmap_out, const void *base, int64_t rows, int64_t cols,
                    int64_t row_stride_elems, int box_rows) {
@@ -1368,6 +1468,7 @@ cudaError_t launch_tc_gemm(const void *tmapA, const void *tmapB, const TcParams 
   if (fp8 && (bwd || !p.a_scale || (p.mode != TC_EXPERT_GU && p.mode != TC_EXPERT_DOWN)))
     return cudaErrorInvalidValue;
   if (fp4 != (p.a_sf != nullptr)) return cudaErrorInvalidValue;
+  if (p.k_split > 1 && (fp8 || bwd || !split_ok(p, TKB))) return cudaErrorInvalidValue;
   if (p.tma_out && (bwd || p.mode == TC_WGRAD || !tmapOut)) return cudaErrorInvalidValue;
   // NVFP4: whole 16-element scale blocks and 16-byte rows (a ragged last
   // K-block is read as zero codes); else whole K-blocks
@@ -1422,6 +1523,7 @@ cudaError_t launch_tc_gemm_pair(const void *tmapA, const void *tmapB2, const TcP
   const bool bwd = p.mode == TC_WGRAD || p.raw || p.out_f32 || p.out_h;
   if (bwd || p.b_scale || (p.tma_out && !tmapOut)) return cudaErrorInvalidValue;
   if (p.Kdim % TKB || p.Kdim <= 0 || p.n_tiles_n <= 0) return cudaErrorInvalidValue;
+  if (p.k_split > 1 && !split_ok(p, TKB)) return cudaErrorInvalidValue;
   const int pairs = max_pairs < dev_pairs ? max_pairs : dev_pairs;
   if (pairs <= 0) return cudaSuccess;
   CUtensorMap a, b, o;

@@ -176,8 +176,14 @@ int lmoe_route(lmoe_handle h, const void *x_dev, int32_t T, int32_t *ids,
 /* The layer forward: y_dev [T][d] = layer(x_dev [T][d]), element type
  * cfg.dtype.  x and y must not overlap and must start on 16-byte boundaries
  * (the kernels move them with 16-byte vectors and TMA).  Graph-capturable:
- * no host sync, no allocation.  T == 0 is a no-op.  Errors: NULL_ARG,
- * NOT_LOADED, TOO_MANY_TOKENS, MISALIGNED, CUDA. */
+ * no host sync, no allocation.  T == 0 is a no-op.  The output is
+ * deterministic for a given T.  A call of fewer than 2048 tokens whose dense
+ * GEMMs (router and down-projection, output projection) have too few output
+ * tiles to fill the GPU splits their reductions into slices summed in a fixed
+ * order, so its y may differ from a larger call's y for the same tokens by
+ * fp32 summation order (the routing is unaffected unless two scores tie to
+ * within that rounding).  Errors: NULL_ARG, NOT_LOADED, TOO_MANY_TOKENS,
+ * MISALIGNED, CUDA. */
 int lmoe_forward(lmoe_handle h, const void *x_dev, void *y_dev, int32_t T, void *stream);
 
 /* End-to-end variant with HOST buffers: copies x_host to a handle-owned
@@ -186,7 +192,9 @@ int lmoe_forward(lmoe_handle h, const void *x_dev, void *y_dev, int32_t T, void 
  * split into up to 4 chunks of at least 2048: a chunk's copy in, forward and
  * copy out overlap the other chunks' (two handle-owned copy streams; the
  * forwards run on `stream` in order).  Each token's output is the one a
- * single call computes.  Pinned host memory gives full copy bandwidth and
+ * single lmoe_forward call over all T tokens computes, bit for bit (chunks
+ * are never small enough to split their reductions).  Pinned host memory
+ * gives full copy bandwidth and
  * the overlap.  Errors: as lmoe_forward. */
 int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T,
                       void *stream);

@@ -88,6 +88,10 @@ constexpr int kHostChunks = 4, kHostChunkTokens = 2048;
 // pairs (few tokens): at most kMaxSplit slices of at least kMinSplitKb
 // K-blocks each, the partials of one launch within kPartFloats.
 constexpr int kMaxSplit = kMaxKSplit, kMinSplitKb = 4;
+// The shared experts' gate/up GEMM overlaps the routing on a side stream when
+// it takes at most this many K-block waves on its capped CTA pairs (README
+// acc: 8 waves x 32 K-blocks; the prefill layer's 42 x 64 runs first instead).
+constexpr int kSideKbWaves = 1024;
 constexpr size_t kPartFloats = static_cast<size_t>(96) * 256 * 256;  // 24 MiB
 
 struct lmoe_layer {
@@ -810,16 +814,25 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
         q.out2 = static_cast<__nv_bfloat16 *>(shared_raw);
         q.ld_out2 = h->sh_rows;
       }
-      e = cudaEventRecord(h->ev_fork, s);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
-      if (e == cudaSuccess)
-        e = shared_raw ? launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, q, h->num_sms,
-                                        m_tiles * shared_tiles_n, h->side)
-                       : launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, q,
-                                             std::min(m_tiles2 * shared_tiles_n,
-                                                      std::max(1, h->num_sms / 3)),
-                                             h->side);
-      if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
+      // A long shared GEMM (more than kSideKbWaves K-block waves on its capped
+      // pairs) would outlast the routing and hold SMs into the persistent
+      // gate/up GEMM, whose CTAs there would start late: it then runs first,
+      // on the main stream and every SM.
+      const int cap = std::max(1, h->num_sms / 3), shared_tiles = m_tiles2 * shared_tiles_n;
+      const bool side = shared_raw || (shared_tiles + cap - 1) / cap * (h->d / 64) <= kSideKbWaves;
+      if (side) {
+        e = cudaEventRecord(h->ev_fork, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
+        if (e == cudaSuccess)
+          e = shared_raw ? launch_tc_gemm(tm_x.bytes, h->tm_wx.bytes, q, h->num_sms,
+                                          m_tiles * shared_tiles_n, h->side)
+                         : launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, q,
+                                               std::min(shared_tiles, cap), h->side);
+        if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
+      } else {
+        e = launch_tc_gemm_pair(tm_x.bytes, h->tm_wx2.bytes, q, shared_tiles, s);
+        if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, s);
+      }
       h->launches += 1;
     }
     if (e == cudaSuccess && xs > 1) {

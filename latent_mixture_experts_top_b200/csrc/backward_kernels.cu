@@ -432,9 +432,6 @@ cudaError_t launch_act_backward(const TI *a, const TI *b, int ldab, const float 
 template cudaError_t launch_act_backward<float, float>(const float *, const float *, int,
                                                        const float *, int, float *, int, float *,
                                                        float *, int, int, int, bool, cudaStream_t);
-template cudaError_t launch_act_backward<__nv_bfloat16, __nv_bfloat16>(
-    const __nv_bfloat16 *, const __nv_bfloat16 *, int, const float *, int, __nv_bfloat16 *, int,
-    __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, bool, cudaStream_t);
 
 template <typename TO>
 cudaError_t launch_slot_grad(const float *du, int lddu, const TO *O, int l, const int32_t *pos,

@@ -25,10 +25,6 @@ template <typename T>
 __device__ __forceinline__ float ld(const T *p, size_t i);
 template <>
 __device__ __forceinline__ float ld<float>(const float *p, size_t i) { return p[i]; }
-template <>
-__device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
-  return __bfloat162float(p[i]);
-}
 template <typename T>
 __device__ __forceinline__ void st(T *p, size_t i, float v);
 template <>

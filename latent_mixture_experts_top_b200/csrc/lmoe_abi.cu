@@ -796,9 +796,10 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     h->launches += 1;
     const int shared_tiles_n = (h->nx_rows - h->n_pad - h->l_pad) / kTileN;
     if (e == cudaSuccess && full && shared_tiles_n > 0) {
-      // Shared experts' gate/up (the shared column range of the same matrix) on
-      // the side stream: it overlaps the routing kernels; the output GEMM joins
-      // it.  The backward's raw variant runs on the single-CTA kernel.
+      // Shared experts' gate/up (the shared column range of the same matrix),
+      // normally on the side stream, where it overlaps the routing kernels (a
+      // long one runs first instead, below); the output GEMM joins it.  The
+      // backward's raw variant runs on the single-CTA kernel.
       TcParams q = p;
       q.k_split = 0;
       q.part = nullptr;

@@ -90,8 +90,13 @@ constexpr int kHostChunks = 4, kHostChunkTokens = 2048;
 constexpr int kMaxSplit = kMaxKSplit, kMinSplitKb = 4;
 // The shared experts' gate/up GEMM overlaps the routing on a side stream when
 // it takes at most this many K-block waves on its capped CTA pairs (README
-// acc: 8 waves x 32 K-blocks; the prefill layer's 42 x 64 runs first instead).
+// acc: 6 waves x 32 K-blocks; the prefill layer's 35 x 64 runs first instead).
 constexpr int kSideKbWaves = 1024;
+// Calls of at least this many tokens permute z with a positions-only scatter
+// and a destination-major row copy instead of the scatter's own copy: beside
+// the side-stream shared GEMM (README acc) the two launches end sooner; at
+// decode the extra launch costs more than it saves.
+constexpr int kRowCopyTokens = 1024;
 constexpr size_t kPartFloats = static_cast<size_t>(96) * 256 * 256;  // 24 MiB
 
 struct lmoe_layer {
@@ -807,8 +812,8 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       q.n_tiles_n = shared_tiles_n;
       // direct stores: the smaller shared-memory footprint lets the routing
       // kernels run beside this launch's CTAs.  The paired launch is capped at
-      // a third of the SMs (each CTA pair loops over its tiles), so that the
-      // routing kernels and the first expert tiles find free SMs.
+      // num_sms * 2 / 5 CTA pairs (59 pairs, 118 of 148 SMs; each pair loops
+      // over its tiles), so that the routing kernels find free SMs.
       q.tma_out = 0;
       if (shared_raw) {
         q.raw = 1;
@@ -819,7 +824,7 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
       // pairs) would outlast the routing and hold SMs into the persistent
       // gate/up GEMM, whose CTAs there would start late: it then runs first,
       // on the main stream and every SM.
-      const int cap = std::max(1, h->num_sms / 3), shared_tiles = m_tiles2 * shared_tiles_n;
+      const int cap = std::max(1, h->num_sms * 2 / 5), shared_tiles = m_tiles2 * shared_tiles_n;
       const bool side = shared_raw || (shared_tiles + cap - 1) / cap * (h->d / 64) <= kSideKbWaves;
       if (side) {
         e = cudaEventRecord(h->ev_fork, s);
@@ -874,15 +879,23 @@ static cudaError_t run_route(lmoe_layer *h, const void *x, int T, bool full, cud
     h->launches += 1;
     if (e != cudaSuccess) return e;
     if (full && marks) mark(h, 2, s);
+    // From kRowCopyTokens tokens on, the scatter writes positions only and a
+    // destination-major copy (one warp per permuted row) fills permute_dst;
+    // below, the scatter also copies the rows (one launch less).
+    const bool row_copy = permute_dst && T >= kRowCopyTokens;
+    const bool fused_copy = permute_dst && !row_copy;
     e = launch_scatter_permute(w.ids, T, h->K, h->N, w.chunk_counts, kFusedChunk, w.offsets,
-                               w.perm, w.pos, w.row_expert, permute_dst ? w.z : nullptr, rb,
-                               permute_dst, h->route_shares, s, true);
+                               w.perm, w.pos, w.row_expert, fused_copy ? w.z : nullptr, rb,
+                               fused_copy ? permute_dst : nullptr, h->route_shares, s, true);
     h->launches += 1;
     if (e != cudaSuccess) return e;
-    if (full && marks) {
-      mark(h, 3, s);  // the permutation ran inside the scatter: stage 3 is empty
-      mark(h, 4, s);
+    if (full && marks) mark(h, 3, s);
+    if (row_copy) {
+      e = launch_permute_rows(w.z, w.perm, h->K, T * h->K, rb, permute_dst, s);
+      h->launches += 1;
+      if (e != cudaSuccess) return e;
     }
+    if (full && marks) mark(h, 4, s);  // empty stage when the scatter copied the rows
     return e;
   }
   // top-K' also builds the dispatch histogram (into the zeroed count matrix)

@@ -195,6 +195,32 @@ def test_ragged_token_counts(cfg, T):
     layer.close()
 
 
+@pytest.mark.parametrize("T", [1023, 1024, 1025])
+def test_permuted_rows_on_both_copy_paths(T):
+    """Below 1024 tokens the scatter itself copies z into dispatch order; from 1024 on, a
+    positions-only scatter and a row-copy launch do.  Either way the permuted rows are
+    zp[r] = z[perm[r] // K'] bit for bit, and y matches the oracle."""
+    cfg = configs.README_ACC
+    inp = _inputs(cfg)
+    x = inp["x"][:T].contiguous()
+    layer, y, ids, gates, offsets, perm = _run(cfg, inp, x=x, max_tokens=cfg.T)
+    K, l = cfg.k_active, cfg.l
+    z = layer.debug_tensor(1, torch.bfloat16, (T, l)).view(torch.int16)
+    zp = layer.debug_tensor(2, torch.bfloat16, (T * K, l)).view(torch.int16)
+    src = perm.long() // K
+    assert torch.equal(zp, z[src])
+    L = pu.oracle_layer(inp, K)
+    x_np = synth.to_numpy(x)
+    s_ref = oracle.router_logits(L, x_np)
+    ids_g = ids.cpu().numpy()
+    _, flipped = pu.check_routing(ids_g, gates.cpu().numpy(), s_ref, K)
+    pu.check_dispatch(ids_g, offsets.cpu().numpy(), perm.cpu().numpy(), cfg.n_routed)
+    tok = pu.sample_tokens(T, 48)
+    y_ref = pu.reference_y(L, x_np, tok, ids_g, flipped)
+    assert pu.rel_err(pu.y_to_numpy(y)[tok], y_ref) <= pu.TOL_BF16
+    layer.close()
+
+
 @pytest.mark.parametrize("cfg", [configs.TINY_F32, configs.README_ACC], ids=["f32", "bf16"])
 def test_zero_tokens(cfg):
     lm = _lmoe()

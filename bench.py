@@ -15,8 +15,10 @@ tokens (the layer forward has no exchange step on one GPU): weak scaling.
 The JSON line also carries: the roofline of the dominant kernel (per-stage
 CUDA events recorded inside the library during a second timed pass, so that
 the first pass -- the `value` -- times plain forwards), the whole
-layer's roofline, an end-to-end number through lmoe_forward_host (host
-buffers, copies inside the timed region), the fp64 oracle timed on a bounded
+layer's roofline, an end-to-end number through lmoe_forward_host_batches
+(a stream of batches in host buffers, every batch's copies inside the timed
+region; the single-call lmoe_forward_host rate beside it), the fp64 oracle
+timed on a bounded
 sample on the host cores, the launch count, and SM clocks sampled during the
 timed region.  --impl reference times the oracle alone on the same workload.
 """
@@ -479,20 +481,32 @@ def run_ours(args):
                   "frac": 1e3 * t_roof / ms_per_step,
                   "achieved_tflops": F / (ms_per_step / 1e3) / 1e12}
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: a stream of
+    # e2e_steps batches (two pinned host buffer pairs, alternating), each
+    # batch copied in, computed and copied out inside the timed region
     e2e_steps = args.e2e_steps or max(3, min(K, 50))
-    x_h = x.cpu().pin_memory()
-    y_h = torch.empty_like(x_h).pin_memory()
-    lmoe.lmoe_forward_host(layer.handle, x_h, y_h, cfg.T)
+    x_hs = [x.cpu().pin_memory() for _ in range(2)]
+    y_hs = [torch.empty_like(x_hs[0]).pin_memory() for _ in range(2)]
+    xs = [x_hs[i % 2] for i in range(e2e_steps)]
+    ys = [y_hs[i % 2] for i in range(e2e_steps)]
+    lmoe.lmoe_forward_host_batches(layer.handle, xs[:2], ys[:2], cfg.T)
     barrier()
     t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        lmoe.lmoe_forward_host(layer.handle, x_h, y_h, cfg.T)
+    lmoe.lmoe_forward_host_batches(layer.handle, xs, ys, cfg.T)
     e2e_s = allmax(time.perf_counter() - t0)
+    # one batch per call (copies overlap only within the call)
+    barrier()
+    t1 = time.perf_counter()
+    for _ in range(3):
+        lmoe.lmoe_forward_host(layer.handle, x_hs[0], y_hs[0], cfg.T)
+    single_s = allmax(time.perf_counter() - t1)
     io_bytes = cfg.T * cfg.d * x.element_size()
     e2e = {"value": cfg.T * world * e2e_steps / e2e_s, "unit": UNIT,
            "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
-           "steps": e2e_steps, "api": "lmoe_forward_host (pinned host buffers)"}
+           "steps": e2e_steps,
+           "api": "lmoe_forward_host_batches (pinned host buffers, one call over the steps)",
+           "single_call": {"value": cfg.T * world * 3 / single_s, "unit": UNIT,
+                           "api": "lmoe_forward_host, one call per step", "steps": 3}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -199,6 +199,22 @@ int lmoe_forward(lmoe_handle h, const void *x_dev, void *y_dev, int32_t T, void 
 int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T,
                       void *stream);
 
+/* A sequence of host batches, for serving: n_batches independent forwards
+ * of T tokens each, batch b from x_hosts[b] ([T][d], host memory) into
+ * y_hosts[b] (caller-owned, [T][d]).  Batch b's copy in runs while batch
+ * b - 1 computes and its copy out while batch b + 1 computes, through two
+ * handle-owned device staging sets (allocated by lmoe_create; each holds
+ * max_tokens * d elements of x and as many of y) and the two copy streams
+ * of lmoe_forward_host; the forwards run on `stream` in batch order.  Each y is
+ * the one lmoe_forward computes for that batch, bit for bit.  Returns after
+ * `stream` and the copies have finished; pinned host memory gives the
+ * overlap.  No counterpart in the pages (host I/O around the layer).
+ * Errors: NULL_ARG (a NULL array or entry with n_batches, T > 0),
+ * INVALID_CONFIG (n_batches < 0), UNSUPPORTED (expert-parallel handle), and
+ * those of lmoe_forward. */
+int lmoe_forward_host_batches(lmoe_handle h, int32_t n_batches, const void *const *x_hosts,
+                              void *const *y_hosts, int32_t T, void *stream);
+
 /* Derived sizes: l = d / alpha, N', K'.  Any output pointer may be NULL. */
 int lmoe_get_dims(lmoe_handle h, int32_t *l, int32_t *n_routed, int32_t *k_active);
 

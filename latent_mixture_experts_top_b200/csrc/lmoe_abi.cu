@@ -42,6 +42,7 @@ struct Workspace {
   int32_t *n_tiles2 = nullptr;
   void *z = nullptr, *zp = nullptr, *H = nullptr, *O = nullptr, *ucat = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
+  void *x_stage2 = nullptr, *y_stage2 = nullptr;  // lmoe_forward_host_batches' second set
   int32_t *status = nullptr;
   int32_t *arrivals = nullptr;  // fused routing: the last-block counter (zero between launches)
   int32_t *seg_end = nullptr;   // training: the end of each expert's rows in the padded order
@@ -152,6 +153,8 @@ struct lmoe_layer {
   // lmoe_forward_host: copy streams and per-chunk events of its pipeline
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t ev_start = nullptr, ev_in[kHostChunks] = {}, ev_out[kHostChunks] = {};
+  // lmoe_forward_host_batches, per staging set: forward done, copy out done
+  cudaEvent_t ev_done[2] = {}, ev_yfree[2] = {};
   TensorMap64 tm_wx, tm_wgu, tm_wo, tm_wy, tm_zp, tm_h, tm_ucat;
   TensorMap64 tm_out_z, tm_out_h, tm_out_o;  // epilogue TMA stores: z, H, O
   // B operands of the CTA-pair GEMMs: the same tiled matrices, {64, 128} boxes
@@ -203,7 +206,7 @@ void free_all(lmoe_layer *h) {
                   h->w_out, h->s_gate, h->s_up, h->w_y, h->ws.logits, h->ws.ids, h->ws.gates,
                   h->ws.chunk_counts, h->ws.offsets, h->ws.perm, h->ws.pos, h->ws.row_expert,
                   h->ws.tiles, h->ws.n_tiles, h->ws.tiles2, h->ws.n_tiles2, h->ws.z, h->ws.zp, h->ws.H, h->ws.O, h->ws.ucat,
-                  h->ws.x_stage, h->ws.y_stage, h->ws.status, h->bw.a, h->bw.b, h->bw.dU,
+                  h->ws.x_stage, h->ws.y_stage, h->ws.x_stage2, h->ws.y_stage2, h->ws.status, h->bw.a, h->bw.b, h->bw.dU,
                   h->bw.ds, h->bw.DO, h->bw.dH, h->bw.dA, h->bw.dB, h->bw.dZp, h->bw.dz,
                   h->bw.as, h->bw.bs, h->bw.das, h->bw.dbs, h->bw.dsfull, h->bw.AB,
                   h->bw.ABs, h->bw.dAB, h->bw.dXcat, h->ws.seg_end,
@@ -223,6 +226,11 @@ void free_all(lmoe_layer *h) {
     if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
     if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
     h->ev_in[i] = h->ev_out[i] = nullptr;
+  }
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_done[i]) cudaEventDestroy(h->ev_done[i]);
+    if (h->ev_yfree[i]) cudaEventDestroy(h->ev_yfree[i]);
+    h->ev_done[i] = h->ev_yfree[i] = nullptr;
   }
   if (h->ev_start) cudaEventDestroy(h->ev_start);
   if (h->h2d) cudaStreamDestroy(h->h2d);
@@ -378,7 +386,8 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
             dalloc(&w.n_tiles2, 16) && dalloc(&w.z, T * l * es) && dalloc(&w.zp, TKr * l * es) &&
             dalloc(&w.H, static_cast<size_t>(h->h_rows) * m * es) && dalloc(&w.O, TKr * l * es) &&
             dalloc(&w.ucat, T * h->ky * es) && dalloc(&w.x_stage, T * d * es) &&
-            dalloc(&w.y_stage, T * d * es) && dalloc(&w.status, 16) && dalloc(&w.arrivals, 16);
+            dalloc(&w.y_stage, T * d * es) && dalloc(&w.x_stage2, T * d * es) &&
+            dalloc(&w.y_stage2, T * d * es) && dalloc(&w.status, 16) && dalloc(&w.arrivals, 16);
   if (ok && h->bf16) ok = dalloc(&w.part, kPartFloats * 4);
   if (ok) {  // weights
     if (h->bf16) {
@@ -544,6 +553,9 @@ int lmoe_create(const lmoe_config *cfg, lmoe_handle *out) {
   for (int i = 0; st_ok && i < kHostChunks; ++i)
     st_ok = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
             cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; st_ok && i < 2; ++i)
+    st_ok = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&h->ev_yfree[i], cudaEventDisableTiming) == cudaSuccess;
   if (!st_ok) {
     free_all(h);
     delete h;
@@ -1586,6 +1598,51 @@ int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T
     if (cudaEventRecord(h->ev_out[c], s) != cudaSuccess ||
         cudaStreamWaitEvent(h->d2h, h->ev_out[c], 0) != cudaSuccess ||
         cudaMemcpyAsync(yh + off, yd + off, bytes, cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(h->d2h) != cudaSuccess) return LMOE_ERR_CUDA;
+  return cuda_err(cudaStreamSynchronize(s));
+}
+
+int lmoe_forward_host_batches(lmoe_handle h, int32_t n_batches, const void *const *x_hosts,
+                              void *const *y_hosts, int32_t T, void *stream) {
+  int rc = check_call(h, T);
+  if (rc != LMOE_OK) return rc;
+  if (h->ep_world > 1) return LMOE_ERR_UNSUPPORTED;
+  if (n_batches < 0) return LMOE_ERR_INVALID_CONFIG;
+  if (n_batches == 0 || T == 0) return LMOE_OK;
+  if (!x_hosts || !y_hosts) return LMOE_ERR_NULL_ARG;
+  for (int b = 0; b < n_batches; ++b)
+    if (!x_hosts[b] || !y_hosts[b]) return LMOE_ERR_NULL_ARG;
+  DeviceGuard g(h->device);
+  if (!g.ok) return LMOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Batch b uses staging set b % 2: its copy in (h2d stream) overlaps batch
+  // b - 1's forward (the caller's stream), and its copy out (d2h stream) the
+  // forward of batch b + 1.  A set is refilled only after batch b - 2's
+  // forward has read x from it (ev_done) and its copy out has read y
+  // (ev_yfree).
+  const size_t bytes = static_cast<size_t>(T) * h->d * h->esize;
+  void *xd[2] = {h->ws.x_stage, h->ws.x_stage2}, *yd[2] = {h->ws.y_stage, h->ws.y_stage2};
+  // the copies start after the work already queued on the caller's stream
+  if (cudaEventRecord(h->ev_start, s) != cudaSuccess ||
+      cudaStreamWaitEvent(h->h2d, h->ev_start, 0) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  for (int b = 0; b < n_batches; ++b) {
+    const int k = b & 1;
+    if (b >= 2 && cudaStreamWaitEvent(h->h2d, h->ev_done[k], 0) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    if (cudaMemcpyAsync(xd[k], x_hosts[b], bytes, cudaMemcpyHostToDevice, h->h2d) != cudaSuccess ||
+        cudaEventRecord(h->ev_in[k], h->h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(s, h->ev_in[k], 0) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    if (b >= 2 && cudaStreamWaitEvent(s, h->ev_yfree[k], 0) != cudaSuccess) return LMOE_ERR_CUDA;
+    rc = forward_impl(h, xd[k], yd[k], T, s);
+    if (rc != LMOE_OK) return rc;
+    if (cudaEventRecord(h->ev_done[k], s) != cudaSuccess ||
+        cudaStreamWaitEvent(h->d2h, h->ev_done[k], 0) != cudaSuccess ||
+        cudaMemcpyAsync(y_hosts[b], yd[k], bytes, cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess ||
+        cudaEventRecord(h->ev_yfree[k], h->d2h) != cudaSuccess)
       return LMOE_ERR_CUDA;
   }
   if (cudaStreamSynchronize(h->d2h) != cudaSuccess) return LMOE_ERR_CUDA;

@@ -30,8 +30,8 @@ STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_CONFIG", -2: "LMOE_ERR_NULL_ARG",
           -6: "LMOE_ERR_DEVICE_TIMEOUT", -7: "LMOE_ERR_UNSUPPORTED",
           -8: "LMOE_ERR_OUT_OF_MEMORY", -9: "LMOE_ERR_MISALIGNED"}
 EXPORTED = ("lmoe_create", "lmoe_load_weights", "lmoe_route", "lmoe_forward",
-            "lmoe_forward_host", "lmoe_get_dims", "lmoe_device_status", "lmoe_debug_buffer",
-            "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc",
+            "lmoe_forward_host", "lmoe_forward_host_batches", "lmoe_get_dims",
+            "lmoe_device_status", "lmoe_debug_buffer", "lmoe_profile", "lmoe_stage_times", "lmoe_dispatch_noalloc",
             "lmoe_selftest_wait_timeout", "lmoe_backward", "lmoe_ep_dispatch", "lmoe_ep_experts",
             "lmoe_ep_combine", "lmoe_strerror", "lmoe_destroy")
 LMOE_NUM_STAGES = 8
@@ -66,6 +66,8 @@ _lib.lmoe_load_weights.argtypes = [P, C.POINTER(lmoe_weights), P]
 _lib.lmoe_route.argtypes = [P, P, I32, P, P, P, P, P]
 _lib.lmoe_forward.argtypes = [P, P, P, I32, P]
 _lib.lmoe_forward_host.argtypes = [P, P, P, I32, P]
+_lib.lmoe_forward_host_batches.argtypes = [P, I32, C.POINTER(C.c_void_p),
+                                            C.POINTER(C.c_void_p), I32, P]
 _lib.lmoe_get_dims.argtypes = [P, C.POINTER(I32), C.POINTER(I32), C.POINTER(I32)]
 _lib.lmoe_device_status.argtypes = [P, P]
 _lib.lmoe_debug_buffer.argtypes = [P, I32, C.POINTER(C.c_void_p), C.POINTER(C.c_int64)]
@@ -162,6 +164,17 @@ def lmoe_forward(handle: int, x, y, T: int, stream=None) -> None:
 def lmoe_forward_host(handle: int, x_host, y_host, T: int, stream=None) -> None:
     _check(_lib.lmoe_forward_host(handle, _ptr(x_host), _ptr(y_host), T, _stream(stream)),
            "lmoe_forward_host")
+
+
+def lmoe_forward_host_batches(handle: int, x_hosts, y_hosts, T: int, stream=None) -> None:
+    """x_hosts, y_hosts: equal-length sequences of host tensors ([T][d] each)."""
+    if len(x_hosts) != len(y_hosts):
+        raise ValueError("x_hosts and y_hosts differ in length")
+    n = len(x_hosts)
+    xs = (C.c_void_p * max(n, 1))(*[_ptr(t) for t in x_hosts])
+    ys = (C.c_void_p * max(n, 1))(*[_ptr(t) for t in y_hosts])
+    _check(_lib.lmoe_forward_host_batches(handle, n, xs, ys, T, _stream(stream)),
+           "lmoe_forward_host_batches")
 
 
 def lmoe_get_dims(handle: int):

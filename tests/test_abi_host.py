@@ -100,6 +100,7 @@ def test_null_arguments(lib):
     assert lib.lmoe_ep_dispatch(None, None, 0, None, None, None) == -2
     assert lib.lmoe_ep_experts(None, None, None, 0, None, None) == -2
     assert lib.lmoe_ep_combine(None, None, None, 0, None) == -2
+    assert lib.lmoe_forward_host_batches(None, 0, None, None, 0, None) == -2
 
 
 def test_strerror_names_every_code(lib):

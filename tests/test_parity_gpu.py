@@ -323,6 +323,32 @@ def test_forward_host_matches_device_path():
     layer.close()
 
 
+@pytest.mark.parametrize("n", [1, 2, 5])
+def test_forward_host_batches_match_device_path(n):
+    """Each batch of a stream (two staging sets, copies overlapping the neighbours'
+    forwards) gives lmoe_forward's y for that batch, bit for bit; batches differ."""
+    cfg = configs.README_ACC
+    inp = _inputs(cfg)
+    lm = _lmoe()
+    layer = lm.LatentMoELayer(cfg, inp)
+    T = 1536
+    xs_dev = [inp["x"][(i * 512) % (cfg.T - T):][:T].contiguous() for i in range(n)]
+    xs_dev = [x * (1.0 + 0.25 * i) for i, x in enumerate(xs_dev)]
+    y_ref = [layer.forward(x).cpu() for x in xs_dev]
+    x_h = [x.cpu().pin_memory() for x in xs_dev]
+    y_h = [torch.full_like(x, float("nan")).pin_memory() for x in x_h]
+    lm.lmoe_forward_host_batches(layer.handle, x_h, y_h, T)
+    for i in range(n):
+        assert torch.equal(y_h[i], y_ref[i]), i
+    assert lm.lmoe_device_status(layer.handle) == 0
+    # no batches, no tokens, and NULL entries
+    lm.lmoe_forward_host_batches(layer.handle, [], [], T)
+    lm.lmoe_forward_host_batches(layer.handle, x_h, y_h, 0)
+    with pytest.raises(RuntimeError):
+        lm.lmoe_forward_host_batches(layer.handle, [x_h[0], None], [y_h[0], y_h[0]], T)
+    layer.close()
+
+
 def test_call_errors_on_device_handle():
     cfg = configs.TINY_F32
     lm = _lmoe()

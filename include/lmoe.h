@@ -208,7 +208,9 @@ int lmoe_forward_host(lmoe_handle h, const void *x_host, void *y_host, int32_t T
  * of lmoe_forward_host; the forwards run on `stream` in batch order.  Each y is
  * the one lmoe_forward computes for that batch, bit for bit.  Returns after
  * `stream` and the copies have finished; pinned host memory gives the
- * overlap.  No counterpart in the pages (host I/O around the layer).
+ * overlap.  The arrays may repeat a buffer (the copies of one stream run in
+ * batch order), but no y buffer may overlap an x buffer.  No counterpart in
+ * the pages (host I/O around the layer).
  * Errors: NULL_ARG (a NULL array or entry with n_batches, T > 0),
  * INVALID_CONFIG (n_batches < 0), UNSUPPORTED (expert-parallel handle), and
  * those of lmoe_forward. */

@@ -323,16 +323,17 @@ def test_forward_host_matches_device_path():
     layer.close()
 
 
-@pytest.mark.parametrize("n", [1, 2, 5])
-def test_forward_host_batches_match_device_path(n):
+@pytest.mark.parametrize("cfg,n,T", [(configs.README_ACC, 1, 1536), (configs.README_ACC, 2, 1536),
+                                     (configs.README_ACC, 5, 1536), (configs.TINY_F32, 3, 40)],
+                         ids=["bf16-1", "bf16-2", "bf16-5", "f32-3"])
+def test_forward_host_batches_match_device_path(cfg, n, T):
     """Each batch of a stream (two staging sets, copies overlapping the neighbours'
     forwards) gives lmoe_forward's y for that batch, bit for bit; batches differ."""
-    cfg = configs.README_ACC
     inp = _inputs(cfg)
     lm = _lmoe()
     layer = lm.LatentMoELayer(cfg, inp)
-    T = 1536
-    xs_dev = [inp["x"][(i * 512) % (cfg.T - T):][:T].contiguous() for i in range(n)]
+    step = max(1, (cfg.T - T) // 5)
+    xs_dev = [inp["x"][(i * step) % (cfg.T - T + 1):][:T].contiguous() for i in range(n)]
     xs_dev = [x * (1.0 + 0.25 * i) for i, x in enumerate(xs_dev)]
     y_ref = [layer.forward(x).cpu() for x in xs_dev]
     x_h = [x.cpu().pin_memory() for x in xs_dev]
